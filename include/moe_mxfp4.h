@@ -1,0 +1,240 @@
+/*
+ * moe_mxfp4.h — C ABI of the packed-MXFP4 W4A16 top-4 MoE expert FFN for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (model card "LFM2.5-24B-A2B — Packed MXFP4 Inference"):
+ *   - table "Model and quantization": expert weights are E2M1 FP4 values,
+ *     two per byte, with one E8M0 scale per 32 values; activations are BF16;
+ *     the packed GEMVs accumulate in FP32 and produce BF16 outputs; each MoE
+ *     layer routes every token to 4 of its experts.
+ *   - section "GPU routing inside resident-layer graphs": router projection,
+ *     expert bias where configured, dynamic top-k selection and routing
+ *     coefficients, recomputed on the GPU each call, with no copy of the
+ *     selected ids to the host.
+ *   - section "What was optimized" > "Grouped top-4 expert execution": one
+ *     grouped packed GEMV for gate, one for up, activation and
+ *     multiplication, one grouped packed GEMV for down, and a fused
+ *     routing-weighted combination that keeps the sequential BF16
+ *     multiply/add rounding of a one-expert-at-a-time runner.
+ *   - section "Direct reads from GPU-resident weights": experts are read in
+ *     place through a persistent device table of expert addresses; no
+ *     staging copy, no BF16 copy of the weights.
+ * The SwiGLU expert is three matrices, gate and up (I x H) and down (H x I)
+ * ("LFM2.5-24B-A2B on Your Own Hardware", section "Where do the 2.45B active
+ * parameters actually go?").
+ *
+ * Exact arithmetic of one (token t, slot j) with expert e = ids[t][j]:
+ *   g = BF16(sum_h Wg[e][i][h] x[t][h])       (FP32 accumulation)
+ *   u = BF16(sum_h Wu[e][i][h] x[t][h])
+ *   h[i] = BF16( BF16(silu(g)) * u )
+ *   o[n] = BF16(sum_i Wd[e][n][i] h[i])
+ * and the combine, in slot order j = 0..k-1, starting from y = +0:
+ *   y = BF16( y + BF16( o_j * BF16(w_j) ) )
+ *   optionally followed by y = BF16(residual + y).
+ *
+ * Conventions for every call:
+ *   - BF16 tensors are passed as uint16_t bit patterns.
+ *   - All tensors are row-major and contiguous.  Pointers documented as
+ *     "device" must point to memory of the current CUDA device (cudaMalloc'd,
+ *     e.g. by PyTorch); the library checks this and returns
+ *     MOE_ERR_NOT_DEVICE otherwise.  Device pointers must be 16-byte aligned
+ *     (MOE_ERR_ALIGN otherwise).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *     moe_route / moe_forward only enqueue kernels: they never allocate,
+ *     never synchronise and never copy weights, so they may be captured in a
+ *     CUDA graph.
+ *   - The library never takes ownership of caller memory: weights, workspace
+ *     and I/O buffers must stay valid until moe_destroy (weights, workspace)
+ *     or until the enqueued work completes (inputs/outputs).
+ *   - Every call returns a moe_status_t; nothing is thrown across the ABI.
+ *     A call that returns an error has enqueued nothing.
+ *
+ * Packed weight layout (the model card calls the checkpoint layout "custom"
+ * and does not describe it; this is the layout of this library):
+ *   codes  uint8 [E][3][rows][K/2]: matrix 0 = gate (rows I, K H),
+ *          1 = up (rows I, K H), 2 = down (rows H, K I).  Element 2i of a
+ *          row is the low nibble of byte i, element 2i+1 the high nibble.
+ *          E2M1 code c: sign = bit 3, magnitude {0,.5,1,1.5,2,3,4,6}[c&7].
+ *   scales uint8 [E][3][rows][K/32]: E8M0, value 2^(s-127), s = 255 is NaN;
+ *          one per 32 consecutive K elements.
+ */
+#ifndef MOE_MXFP4_H
+#define MOE_MXFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct moe_ctx *moe_handle_t;
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_ARG = -1,           /* bad shape, null pointer, T out of range  */
+    MOE_ERR_NOT_LOADED = -2,    /* weights or workspace not set yet         */
+    MOE_ERR_NOT_DEVICE = -3,    /* pointer is not memory of this device     */
+    MOE_ERR_ALIGN = -4,         /* pointer not 16-byte aligned              */
+    MOE_ERR_WORKSPACE = -5,     /* workspace too small for this T           */
+    MOE_ERR_CUDA = -6,          /* a CUDA runtime call failed               */
+    MOE_ERR_DEVICE_STATUS = -7, /* a kernel flagged bad input (ids)         */
+    MOE_ERR_UNSUPPORTED = -8    /* current device is not sm_100             */
+} moe_status_t;
+
+/* Bits of the device status word read by moe_get_status. */
+#define MOE_DEVICE_BAD_EXPERT_ID 0x1u /* an id outside [0, E): slot zeroed */
+
+/* Flags of moe_route_ex. */
+#define MOE_ROUTE_RMSNORM 0x1u /* x is a residual stream r: route
+                                  xn = BF16(r / sqrt(mean(r^2) + 1e-6))
+                                  and write xn to x_norm */
+
+/* Flags of moe_forward_ex. */
+#define MOE_FWD_KEEP_INTERMEDIATES 0x1u /* also store h [T][k][I] and
+                                           o [T][k][H] in the workspace
+                                           (moe_get_intermediates)         */
+#define MOE_FWD_FORCE_DECODE 0x2u  /* per-(token,slot) GEMV path            */
+#define MOE_FWD_FORCE_GROUPED 0x4u /* (token,expert)-sorted grouped path    */
+#define MOE_FWD_PHASE_GATEUP 0x8u  /* run only the gate/up/SwiGLU kernel(s);
+                                      h stays in the workspace              */
+#define MOE_FWD_PHASE_DOWN 0x10u   /* run only the down + combine kernel(s)
+                                      on the h of the preceding
+                                      MOE_FWD_PHASE_GATEUP call (same T,
+                                      ids, same handle and workspace); the
+                                      two calls together equal one forward  */
+
+/* Create a layer of E experts with hidden size H, intermediate size I and
+ * top_k experts per token.  Requires H % 32 == 0, I % 32 == 0, H >= 32,
+ * I >= 32, 1 <= top_k <= min(E, 8), E <= 1024.  Host-only: allocates the
+ * handle, touches no GPU.  *out receives the handle (NULL on error).
+ * Errors: MOE_ERR_ARG. */
+MOE_API int moe_create(int E, int H, int I, int top_k, moe_handle_t *out);
+
+/* Release the handle and the small device block it allocated at load time
+ * (expert table, status word).  Caller memory is never freed.  NULL is a
+ * no-op.  Synchronises the device if a device block exists. */
+MOE_API int moe_destroy(moe_handle_t h);
+
+/* Bind contiguously stored packed weights (layout above): codes device
+ * uint8 [E][3][I*H/2], scales device uint8 [E][3][I*H/32].  Both 16-byte
+ * aligned.  Nothing is copied: the library builds the device expert table
+ * from these base addresses and reads the weights in place.  Allocates the
+ * handle's device block (expert table + status word) on first use and
+ * synchronises the device once.  Errors: ARG, NOT_DEVICE, ALIGN, CUDA,
+ * UNSUPPORTED. */
+MOE_API int moe_load_packed(moe_handle_t h, const uint8_t *codes_u8,
+                    const uint8_t *scales_e8m0);
+
+/* Bind experts stored anywhere: codes_ptrs / scales_ptrs are HOST arrays of
+ * 3*E DEVICE pointers, entry 3*e+m pointing at matrix m (0 gate, 1 up,
+ * 2 down) of expert e in the per-matrix layout above ([rows][K/2] and
+ * [rows][K/32]).  Every pointer 16-byte aligned.  Same ownership and
+ * errors as moe_load_packed. */
+MOE_API int moe_load_expert_table(moe_handle_t h, const uint8_t *const *codes_ptrs,
+                          const uint8_t *const *scales_ptrs);
+
+/* Bytes of device workspace needed for up to max_tokens tokens per call.
+ * Errors: ARG. */
+MOE_API int moe_workspace_bytes(moe_handle_t h, int max_tokens, size_t *bytes);
+
+/* Give the handle a device workspace (owned by the caller, 256-byte
+ * aligned, at least moe_workspace_bytes(max_tokens) bytes).  Zeroes it
+ * (synchronously).  Several handles may share one workspace if their calls
+ * are ordered on one stream.  Errors: ARG, NOT_DEVICE, ALIGN, WORKSPACE,
+ * CUDA. */
+MOE_API int moe_set_workspace(moe_handle_t h, void *workspace, size_t bytes,
+                      int max_tokens);
+
+/* Routing for T tokens (1 <= T <= max_tokens of the workspace):
+ *   logits[t][e] = sum_h x[t][h] * router_w[e][h]   (FP32 accumulation)
+ *                  (+ router_bias[e] if router_bias != NULL)
+ *   topk_ids[t][0..k-1] = experts of the k largest logits, descending,
+ *                          equal logits -> lower expert id first
+ *   topk_w[t][j] = softmax over the k selected logits (FP32).
+ * x: device BF16 [T][H]; router_w: device BF16 [E][H]; router_bias: device
+ * FP32 [E] or NULL; topk_ids: device int32 [T][k]; topk_w: device FP32
+ * [T][k].  Errors: ARG, NOT_LOADED (no workspace), NOT_DEVICE, ALIGN,
+ * WORKSPACE, CUDA. */
+MOE_API int moe_route(moe_handle_t h, const uint16_t *x, int T,
+              const uint16_t *router_w, const float *router_bias,
+              int32_t *topk_ids, float *topk_w, void *stream);
+
+/* moe_route plus options.  flags: MOE_ROUTE_RMSNORM (then x_norm, device
+ * BF16 [T][H], receives the normalised input that is routed; otherwise
+ * x_norm must be NULL).  logits: device FP32 [T][E] that receives the
+ * (biased) logits, or NULL. */
+MOE_API int moe_route_ex(moe_handle_t h, const uint16_t *x, int T,
+                 const uint16_t *router_w, const float *router_bias,
+                 unsigned flags, uint16_t *x_norm, float *logits,
+                 int32_t *topk_ids, float *topk_w, void *stream);
+
+/* Expert FFN + combine for T tokens with given routing (e.g. from
+ * moe_route):  y[t] = sequential BF16 combine of the k expert outputs.
+ * x: device BF16 [T][H]; topk_ids: device int32 [T][k]; topk_w: device FP32
+ * [T][k]; y: device BF16 [T][H] (must not alias x).  An id outside [0, E)
+ * makes that slot contribute 0 and sets MOE_DEVICE_BAD_EXPERT_ID in the
+ * device status word.  T = 1..4 runs the per-(token, slot) GEMV path;
+ * larger T the (token, expert)-sorted grouped path.  Errors: ARG,
+ * NOT_LOADED, NOT_DEVICE, ALIGN, WORKSPACE, CUDA. */
+MOE_API int moe_forward(moe_handle_t h, const uint16_t *x, int T,
+                const int32_t *topk_ids, const float *topk_w, uint16_t *y,
+                void *stream);
+
+/* moe_forward plus options.  residual: device BF16 [T][H] or NULL; if given,
+ * y = BF16(residual + combine) (residual may alias y).  flags: the
+ * MOE_FWD_* bits above. */
+MOE_API int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T,
+                   const int32_t *topk_ids, const float *topk_w,
+                   const uint16_t *residual, uint16_t *y, unsigned flags,
+                   void *stream);
+
+/* Device pointers to the intermediates kept by the last moe_forward_ex with
+ * MOE_FWD_KEEP_INTERMEDIATES: h BF16 [T][k][I] (SwiGLU outputs) and o BF16
+ * [T][k][H] (expert outputs before the combine).  They live in the
+ * workspace until the next forward.  Errors: NOT_LOADED. */
+MOE_API int moe_get_intermediates(moe_handle_t h, const uint16_t **h_out,
+                          const uint16_t **o_out);
+
+/* Synchronise the device, return the device status word (MOE_DEVICE_* bits)
+ * of this handle in *device_status and clear it.  Errors: NOT_LOADED, CUDA.
+ */
+MOE_API int moe_get_status(moe_handle_t h, unsigned *device_status);
+
+/* Packed bytes of one expert: 3*I*H/2 code bytes + 3*I*H/32 scale bytes
+ * (5,013,504 for H=2048, I=1536).  Errors: ARG. */
+MOE_API int moe_bytes_per_expert(moe_handle_t h, size_t *bytes);
+
+/* Performance switches (both on by default; results do not depend on them):
+ * use_pdl: launch each kernel with programmatic stream serialization so it
+ * can start while the previous kernel of the stream drains; prefetch_down:
+ * the gate/up kernel asks L2 to fetch the selected experts' down matrices
+ * while it streams gate/up.  Errors: ARG. */
+MOE_API int moe_set_tuning(moe_handle_t h, int use_pdl, int prefetch_down);
+
+/* Human-readable name of a status code (static string, never NULL). */
+MOE_API const char *moe_status_string(int status);
+
+/* MOE_OK if the current device is sm_100 (B200), else MOE_ERR_UNSUPPORTED
+ * or MOE_ERR_CUDA. */
+MOE_API int moe_device_check(void);
+
+/* Test hook: dequantise n packed elements (n % 32 == 0) with the same
+ * in-register decode the GEMV kernels use; out[j] = E2M1(code j) *
+ * 2^(scales[j/32]-127) in FP32.  codes device uint8 [n/2], scales device
+ * uint8 [n/32], out device FP32 [n].  Errors: ARG, NOT_DEVICE, ALIGN, CUDA.
+ */
+MOE_API int moe_debug_dequant(const uint8_t *codes, const uint8_t *scales, int64_t n,
+                      float *out, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_MXFP4_H */

@@ -1,0 +1,321 @@
+"""Packed-MXFP4 W4A16 top-4 MoE expert FFN for NVIDIA B200 (sm_100a).
+
+Python binding of the C-ABI library ``libmoe_mxfp4.so`` (declared in
+``include/moe_mxfp4.h``). The functions below carry the C names and only
+marshal arguments: torch tensors give device pointers, the current torch
+stream gives the CUDA stream, every step of the computation runs in the
+library's kernels. There is no CPU fallback: if the library is missing or the
+device is not sm_100, the calls raise.
+
+``MoELayer`` and ``MoEStack`` bundle the calls with their buffers: a single
+layer (route + experts + combine) and a stack of layers (weightless RMSNorm,
+route, experts, combine with residual add, per layer) captured in one CUDA
+graph per decode step.
+"""
+from __future__ import annotations
+
+import ctypes as C
+
+import torch
+
+from ._lib import MoEError, check, library_path, load
+
+__all__ = [
+    "MoEError", "MoELayer", "MoEStack", "library_path", "load",
+    "moe_create", "moe_destroy", "moe_load_packed", "moe_load_expert_table",
+    "moe_workspace_bytes", "moe_set_workspace", "moe_route", "moe_route_ex",
+    "moe_forward", "moe_forward_ex", "moe_get_intermediates", "moe_get_status",
+    "moe_bytes_per_expert", "moe_set_tuning", "moe_device_check", "moe_debug_dequant",
+    "ROUTE_RMSNORM", "FWD_KEEP_INTERMEDIATES", "FWD_FORCE_DECODE", "FWD_FORCE_GROUPED",
+    "FWD_PHASE_GATEUP", "FWD_PHASE_DOWN",
+    "DEVICE_BAD_EXPERT_ID",
+]
+
+ROUTE_RMSNORM = 0x1
+FWD_KEEP_INTERMEDIATES = 0x1
+FWD_FORCE_DECODE = 0x2
+FWD_FORCE_GROUPED = 0x4
+FWD_PHASE_GATEUP = 0x8
+FWD_PHASE_DOWN = 0x10
+DEVICE_BAD_EXPERT_ID = 0x1
+
+
+def _p(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _s(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+def _need(t, dtype, name, ndim=None):
+    if t is None:
+        return
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise MoEError(name, -1)
+    if ndim is not None and t.dim() != ndim:
+        raise MoEError(name, -1)
+
+
+# ------------------------------------------------------------ C-ABI names
+
+def moe_create(E: int, H: int, I: int, top_k: int) -> int:
+    h = C.c_void_p()
+    check("moe_create", load().moe_create(E, H, I, top_k, C.byref(h)))
+    return h.value
+
+
+def moe_destroy(h: int) -> None:
+    check("moe_destroy", load().moe_destroy(C.c_void_p(h)))
+
+
+def moe_load_packed(h: int, codes: torch.Tensor, scales: torch.Tensor) -> None:
+    _need(codes, torch.uint8, "moe_load_packed")
+    _need(scales, torch.uint8, "moe_load_packed")
+    check("moe_load_packed", load().moe_load_packed(C.c_void_p(h), _p(codes), _p(scales)))
+
+
+def moe_load_expert_table(h: int, codes_ptrs, scales_ptrs) -> None:
+    """codes_ptrs / scales_ptrs: sequences of 3*E device addresses (ints)."""
+    n = len(codes_ptrs)
+    ca = (C.c_void_p * n)(*codes_ptrs)
+    sa = (C.c_void_p * n)(*scales_ptrs)
+    check("moe_load_expert_table", load().moe_load_expert_table(C.c_void_p(h), ca, sa))
+
+
+def moe_workspace_bytes(h: int, max_tokens: int) -> int:
+    n = C.c_size_t()
+    check("moe_workspace_bytes", load().moe_workspace_bytes(C.c_void_p(h), max_tokens, C.byref(n)))
+    return n.value
+
+
+def moe_set_workspace(h: int, ws: torch.Tensor, max_tokens: int) -> None:
+    _need(ws, torch.uint8, "moe_set_workspace")
+    check("moe_set_workspace",
+          load().moe_set_workspace(C.c_void_p(h), _p(ws), ws.numel(), max_tokens))
+
+
+def moe_route(h, x, router_w, router_bias, topk_ids, topk_w, stream=None) -> None:
+    moe_route_ex(h, x, router_w, router_bias, 0, None, None, topk_ids, topk_w, stream)
+
+
+def moe_route_ex(h, x, router_w, router_bias, flags, x_norm, logits, topk_ids, topk_w,
+                 stream=None) -> None:
+    _need(x, torch.bfloat16, "moe_route", 2)
+    _need(router_w, torch.bfloat16, "moe_route", 2)
+    _need(router_bias, torch.float32, "moe_route")
+    _need(x_norm, torch.bfloat16, "moe_route")
+    _need(logits, torch.float32, "moe_route")
+    _need(topk_ids, torch.int32, "moe_route")
+    _need(topk_w, torch.float32, "moe_route")
+    check("moe_route", load().moe_route_ex(
+        C.c_void_p(h), _p(x), x.shape[0], _p(router_w), _p(router_bias), flags, _p(x_norm),
+        _p(logits), _p(topk_ids), _p(topk_w), _s(stream)))
+
+
+def moe_forward(h, x, topk_ids, topk_w, y, stream=None) -> None:
+    moe_forward_ex(h, x, topk_ids, topk_w, None, y, 0, stream)
+
+
+def moe_forward_ex(h, x, topk_ids, topk_w, residual, y, flags, stream=None) -> None:
+    _need(x, torch.bfloat16, "moe_forward", 2)
+    _need(topk_ids, torch.int32, "moe_forward")
+    _need(topk_w, torch.float32, "moe_forward")
+    _need(residual, torch.bfloat16, "moe_forward")
+    _need(y, torch.bfloat16, "moe_forward")
+    check("moe_forward", load().moe_forward_ex(
+        C.c_void_p(h), _p(x), x.shape[0], _p(topk_ids), _p(topk_w), _p(residual), _p(y),
+        flags, _s(stream)))
+
+
+def moe_get_intermediates(h: int):
+    """Device addresses (h_ptr, o_ptr) of the intermediates of the last forward
+    run with FWD_KEEP_INTERMEDIATES."""
+    hp, op = C.c_void_p(), C.c_void_p()
+    check("moe_get_intermediates",
+          load().moe_get_intermediates(C.c_void_p(h), C.byref(hp), C.byref(op)))
+    return hp.value, op.value
+
+
+def moe_get_status(h: int) -> int:
+    v = C.c_uint()
+    check("moe_get_status", load().moe_get_status(C.c_void_p(h), C.byref(v)))
+    return v.value
+
+
+def moe_bytes_per_expert(h: int) -> int:
+    n = C.c_size_t()
+    check("moe_bytes_per_expert", load().moe_bytes_per_expert(C.c_void_p(h), C.byref(n)))
+    return n.value
+
+
+def moe_set_tuning(h: int, use_pdl: bool, prefetch_down: bool) -> None:
+    check("moe_set_tuning", load().moe_set_tuning(C.c_void_p(h), int(use_pdl), int(prefetch_down)))
+
+
+def moe_device_check() -> None:
+    check("moe_device_check", load().moe_device_check())
+
+
+def moe_debug_dequant(codes, scales, n, out, stream=None) -> None:
+    _need(codes, torch.uint8, "moe_debug_dequant")
+    _need(scales, torch.uint8, "moe_debug_dequant")
+    _need(out, torch.float32, "moe_debug_dequant")
+    check("moe_debug_dequant", load().moe_debug_dequant(_p(codes), _p(scales), n, _p(out), _s(stream)))
+
+
+# ------------------------------------------------------------- bundles
+
+class MoELayer:
+    """One MoE layer bound to packed weights already on the device.
+
+    codes uint8 [E, 3*I*H/2] and scales uint8 [E, 3*I*H/32] (layout of
+    include/moe_mxfp4.h) are read in place; the layer keeps references to
+    them. ``router_w`` BF16 [E, H], ``router_b`` FP32 [E] or None.
+    """
+
+    def __init__(self, E, H, I, top_k, codes, scales, router_w=None, router_b=None,
+                 max_tokens=4, workspace=None):
+        moe_device_check()
+        self.E, self.H, self.I, self.k = E, H, I, top_k
+        self.codes, self.scales = codes, scales
+        self.router_w, self.router_b = router_w, router_b
+        self.max_tokens = max_tokens
+        self.handle = moe_create(E, H, I, top_k)
+        try:
+            moe_load_packed(self.handle, codes, scales)
+            need = moe_workspace_bytes(self.handle, max_tokens)
+            if workspace is None:
+                workspace = torch.empty(need, dtype=torch.uint8, device=codes.device)
+            self.workspace = workspace
+            moe_set_workspace(self.handle, workspace, max_tokens)
+        except Exception:
+            moe_destroy(self.handle)
+            self.handle = None
+            raise
+
+    def close(self):
+        if getattr(self, "handle", None):
+            moe_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def route(self, x, ids=None, w=None, logits=None, x_norm=None, rmsnorm=False, stream=None):
+        T = x.shape[0]
+        dev = x.device
+        ids = ids if ids is not None else torch.empty(T, self.k, dtype=torch.int32, device=dev)
+        w = w if w is not None else torch.empty(T, self.k, dtype=torch.float32, device=dev)
+        flags = ROUTE_RMSNORM if rmsnorm else 0
+        if rmsnorm and x_norm is None:
+            x_norm = torch.empty_like(x)
+        moe_route_ex(self.handle, x, self.router_w, self.router_b, flags,
+                     x_norm if rmsnorm else None, logits, ids, w, stream)
+        return (ids, w, x_norm) if rmsnorm else (ids, w)
+
+    def forward(self, x, ids, w, y=None, residual=None, flags=0, stream=None):
+        y = y if y is not None else torch.empty_like(x)
+        moe_forward_ex(self.handle, x, ids, w, residual, y, flags, stream)
+        return y
+
+    def __call__(self, x, stream=None):
+        ids, w = self.route(x, stream=stream)
+        return self.forward(x, ids, w, stream=stream)
+
+    def intermediates(self, T):
+        """Views (h [T,k,I], o [T,k,H], BF16) into the workspace of the last
+        forward run with FWD_KEEP_INTERMEDIATES."""
+        hp, op = moe_get_intermediates(self.handle)
+        base = self.workspace.data_ptr()
+        hv = self.workspace[hp - base: hp - base + T * self.k * self.I * 2]
+        ov = self.workspace[op - base: op - base + T * self.k * self.H * 2]
+        return (hv.view(torch.bfloat16).view(T, self.k, self.I),
+                ov.view(torch.bfloat16).view(T, self.k, self.H))
+
+    def status(self) -> int:
+        return moe_get_status(self.handle)
+
+
+class MoEStack:
+    """A stack of MoE layers run as one decode step on a residual stream r:
+    per layer xn = RMSNorm(r) (weightless, eps 1e-6), route(xn), experts,
+    r = BF16(r + combine).  ``step()`` replays one CUDA graph of all layers.
+    Layers share one workspace (they run in order on one stream)."""
+
+    def __init__(self, layers_weights, E, H, I, top_k, T=1, device="cuda"):
+        moe_device_check()
+        self.E, self.H, self.I, self.k, self.T = E, H, I, top_k, T
+        self.layers = []
+        ws = None
+        for (codes, scales, router_w, router_b) in layers_weights:
+            L = MoELayer(E, H, I, top_k, codes, scales, router_w, router_b, max_tokens=T,
+                         workspace=ws)
+            ws = L.workspace
+            self.layers.append(L)
+        dev = torch.device(device)
+        n = len(self.layers)
+        self.r = torch.zeros(T, H, dtype=torch.bfloat16, device=dev)
+        self.xn = torch.zeros(T, H, dtype=torch.bfloat16, device=dev)
+        self.ids = torch.zeros(n, T, top_k, dtype=torch.int32, device=dev)
+        self.w = torch.zeros(n, T, top_k, dtype=torch.float32, device=dev)
+        self.graph = None
+        self.stream = torch.cuda.Stream(device=dev)
+
+    def set_tuning(self, use_pdl=True, prefetch_down=True):
+        for L in self.layers:
+            moe_set_tuning(L.handle, use_pdl, prefetch_down)
+
+    def enqueue(self, stream=None):
+        """Enqueue one decode step (all layers) on `stream`."""
+        for l, L in enumerate(self.layers):
+            moe_route_ex(L.handle, self.r, L.router_w, L.router_b, ROUTE_RMSNORM, self.xn, None,
+                         self.ids[l], self.w[l], stream)
+            moe_forward_ex(L.handle, self.xn, self.ids[l], self.w[l], self.r, self.r, 0, stream)
+
+    def capture(self):
+        """Capture one decode step into a CUDA graph (warm-up run first)."""
+        s = self.stream
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            saved = self.r.clone()
+            self.enqueue(s)
+            self.r.copy_(saved)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            self.enqueue(s)
+        self.graph = g
+        return g
+
+    def step(self):
+        """One decode step: replay the captured graph (captures on first use)."""
+        if self.graph is None:
+            self.capture()
+        self.graph.replay()
+
+    def decode_host(self, x_host, y_host):
+        """Decode the tokens of x_host one step each (T rows per step) from
+        host memory: per step, copy its input into the residual stream,
+        replay the captured step, copy the residual stream back into y_host.
+        Returns after the last copy has landed.  Pinned buffers make the
+        copies asynchronous."""
+        if self.graph is None:
+            self.capture()
+        T = self.T
+        for i in range(x_host.shape[0] // T):
+            self.r.copy_(x_host[i * T:(i + 1) * T], non_blocking=True)
+            self.graph.replay()
+            y_host[i * T:(i + 1) * T].copy_(self.r, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+        return y_host
+
+    def close(self):
+        self.graph = None
+        for L in self.layers:
+            L.close()

@@ -1,0 +1,414 @@
+// api.cu — host implementation of the C ABI declared in include/moe_mxfp4.h.
+//
+// The handle holds shapes, the device expert table (the persistent device
+// pointer table of the model card's section "Direct reads from GPU-resident
+// weights"), a device status word and the caller's workspace.  route/forward
+// validate their arguments on the host and then only enqueue kernels: no
+// allocation, no synchronisation, no weight copy, so a whole layer (or a whole
+// stack of layers) can be captured in one CUDA graph (model card sections
+// "Grouped top-4 expert execution" and "Shared capture stream").
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+
+#include "../../include/moe_mxfp4.h"
+#include "kernels.cuh"
+
+struct moe_ctx {
+    int E = 0, H = 0, I = 0, k = 0;
+    int device = -1;
+    int num_sms = 0;
+    void *dblock = nullptr;               // device: ExpertPtrs[E], then status word
+    moe::ExpertPtrs *d_table = nullptr;
+    unsigned *d_status = nullptr;
+    bool loaded = false;
+    uint8_t *ws = nullptr;
+    size_t ws_bytes = 0;
+    int max_tokens = 0;
+    bool kept = false;                    // last forward kept intermediates
+    bool use_pdl = true;
+    bool prefetch_down = true;
+};
+
+namespace {
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct WsLayout {
+    size_t counters, logits, h, o, total;
+};
+
+WsLayout ws_layout(const moe_ctx *c, int maxT) {
+    WsLayout L;
+    size_t off = 0;
+    auto take = [&](size_t n) {
+        size_t o = off;
+        off = align_up(off + n, 256);
+        return o;
+    };
+    L.counters = take((size_t)maxT * sizeof(unsigned));
+    L.logits = take((size_t)maxT * c->E * sizeof(float));
+    L.h = take((size_t)maxT * c->k * c->I * 2);
+    L.o = take((size_t)maxT * c->k * c->H * 2);
+    L.total = off;
+    return L;
+}
+
+int check_device_ptr(const moe_ctx *c, const void *p, size_t align) {
+    if (!p) return MOE_ERR_ARG;
+    if (((uintptr_t)p) & (align - 1)) return MOE_ERR_ALIGN;
+    cudaPointerAttributes a;
+    cudaError_t e = cudaPointerGetAttributes(&a, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_NOT_DEVICE;
+    }
+    if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return MOE_ERR_NOT_DEVICE;
+    if (c && a.device != c->device) return MOE_ERR_NOT_DEVICE;
+    return MOE_OK;
+}
+
+int current_device_ok(int *dev, int *sms) {
+    int d = -1;
+    if (cudaGetDevice(&d) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    int major = 0, n = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, d) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    if (major != 10) return MOE_ERR_UNSUPPORTED;
+    if (dev) *dev = d;
+    if (sms) *sms = n;
+    return MOE_OK;
+}
+
+int ensure_device_block(moe_ctx *c) {
+    if (c->dblock) return MOE_OK;
+    int rc = current_device_ok(&c->device, &c->num_sms);
+    if (rc != MOE_OK) return rc;
+    size_t tbytes = align_up(sizeof(moe::ExpertPtrs) * (size_t)c->E, 256);
+    void *p = nullptr;
+    if (cudaMalloc(&p, tbytes + 256) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    if (cudaMemset(p, 0, tbytes + 256) != cudaSuccess) {
+        cudaGetLastError();
+        cudaFree(p);
+        return MOE_ERR_CUDA;
+    }
+    c->dblock = p;
+    c->d_table = reinterpret_cast<moe::ExpertPtrs *>(p);
+    c->d_status = reinterpret_cast<unsigned *>(static_cast<uint8_t *>(p) + tbytes);
+    return MOE_OK;
+}
+
+int upload_table(moe_ctx *c, const moe::ExpertPtrs *host_table) {
+    cudaError_t e = cudaMemcpy(c->d_table, host_table, sizeof(moe::ExpertPtrs) * (size_t)c->E,
+                               cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    c->loaded = true;
+    return MOE_OK;
+}
+
+int cuda_rc(cudaError_t e) {
+    if (e == cudaSuccess) return MOE_OK;
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_create(int E, int H, int I, int top_k, moe_handle_t *out) {
+    if (!out) return MOE_ERR_ARG;
+    *out = nullptr;
+    if (E < 1 || E > 1024 || H < 32 || I < 32 || H % 32 || I % 32) return MOE_ERR_ARG;
+    if (top_k < 1 || top_k > moe::kMaxTopK || top_k > E) return MOE_ERR_ARG;
+    if (H > 16384 || I > 16384) return MOE_ERR_ARG;
+    moe_ctx *c = new (std::nothrow) moe_ctx;
+    if (!c) return MOE_ERR_ARG;
+    c->E = E;
+    c->H = H;
+    c->I = I;
+    c->k = top_k;
+    *out = c;
+    return MOE_OK;
+}
+
+int moe_destroy(moe_handle_t h) {
+    if (!h) return MOE_OK;
+    int rc = MOE_OK;
+    if (h->dblock) {
+        cudaDeviceSynchronize();
+        rc = cuda_rc(cudaFree(h->dblock));
+    }
+    delete h;
+    return rc;
+}
+
+int moe_load_packed(moe_handle_t h, const uint8_t *codes_u8, const uint8_t *scales_e8m0) {
+    if (!h || !codes_u8 || !scales_e8m0) return MOE_ERR_ARG;
+    int rc = ensure_device_block(h);
+    if (rc != MOE_OK) return rc;
+    if ((rc = check_device_ptr(h, codes_u8, 16)) != MOE_OK) return rc;
+    if ((rc = check_device_ptr(h, scales_e8m0, 16)) != MOE_OK) return rc;
+    const size_t mc = (size_t)h->I * h->H / 2, ms = (size_t)h->I * h->H / 32;
+    if (ms % 16) return MOE_ERR_ALIGN;  // every matrix must start 16-byte aligned
+    moe::ExpertPtrs *t = new (std::nothrow) moe::ExpertPtrs[h->E];
+    if (!t) return MOE_ERR_ARG;
+    for (int e = 0; e < h->E; ++e)
+        for (int m = 0; m < 3; ++m) {
+            t[e].codes[m] = codes_u8 + ((size_t)e * 3 + m) * mc;
+            t[e].scales[m] = scales_e8m0 + ((size_t)e * 3 + m) * ms;
+        }
+    rc = upload_table(h, t);
+    delete[] t;
+    return rc;
+}
+
+int moe_load_expert_table(moe_handle_t h, const uint8_t *const *codes_ptrs,
+                          const uint8_t *const *scales_ptrs) {
+    if (!h || !codes_ptrs || !scales_ptrs) return MOE_ERR_ARG;
+    int rc = ensure_device_block(h);
+    if (rc != MOE_OK) return rc;
+    moe::ExpertPtrs *t = new (std::nothrow) moe::ExpertPtrs[h->E];
+    if (!t) return MOE_ERR_ARG;
+    for (int e = 0; e < h->E && rc == MOE_OK; ++e)
+        for (int m = 0; m < 3 && rc == MOE_OK; ++m) {
+            const uint8_t *cp = codes_ptrs[3 * e + m], *sp = scales_ptrs[3 * e + m];
+            if ((rc = check_device_ptr(h, cp, 16)) != MOE_OK) break;
+            if ((rc = check_device_ptr(h, sp, 16)) != MOE_OK) break;
+            t[e].codes[m] = cp;
+            t[e].scales[m] = sp;
+        }
+    if (rc == MOE_OK) rc = upload_table(h, t);
+    delete[] t;
+    return rc;
+}
+
+int moe_workspace_bytes(moe_handle_t h, int max_tokens, size_t *bytes) {
+    if (!h || !bytes || max_tokens < 1) return MOE_ERR_ARG;
+    *bytes = ws_layout(h, max_tokens).total;
+    return MOE_OK;
+}
+
+int moe_set_workspace(moe_handle_t h, void *workspace, size_t bytes, int max_tokens) {
+    if (!h || !workspace || max_tokens < 1) return MOE_ERR_ARG;
+    int rc = ensure_device_block(h);
+    if (rc != MOE_OK) return rc;
+    if ((rc = check_device_ptr(h, workspace, 256)) != MOE_OK) return rc;
+    if (bytes < ws_layout(h, max_tokens).total) return MOE_ERR_WORKSPACE;
+    if ((rc = cuda_rc(cudaMemset(workspace, 0, bytes))) != MOE_OK) return rc;
+    h->ws = static_cast<uint8_t *>(workspace);
+    h->ws_bytes = bytes;
+    h->max_tokens = max_tokens;
+    h->kept = false;
+    return MOE_OK;
+}
+
+int moe_route_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *router_w,
+                 const float *router_bias, unsigned flags, uint16_t *x_norm, float *logits,
+                 int32_t *topk_ids, float *topk_w, void *stream) {
+    if (!h || T < 1) return MOE_ERR_ARG;
+    if (flags & ~MOE_ROUTE_RMSNORM) return MOE_ERR_ARG;
+    const bool norm = flags & MOE_ROUTE_RMSNORM;
+    if (norm != (x_norm != nullptr)) return MOE_ERR_ARG;
+    if (!h->ws) return MOE_ERR_NOT_LOADED;
+    if (T > h->max_tokens) return MOE_ERR_WORKSPACE;
+    int rc;
+    if ((rc = check_device_ptr(h, x, 16)) != MOE_OK) return rc;
+    if ((rc = check_device_ptr(h, router_w, 16)) != MOE_OK) return rc;
+    if (router_bias && (rc = check_device_ptr(h, router_bias, 4)) != MOE_OK) return rc;
+    if (norm && (rc = check_device_ptr(h, x_norm, 16)) != MOE_OK) return rc;
+    if (logits && (rc = check_device_ptr(h, logits, 4)) != MOE_OK) return rc;
+    if ((rc = check_device_ptr(h, topk_ids, 4)) != MOE_OK) return rc;
+    if ((rc = check_device_ptr(h, topk_w, 4)) != MOE_OK) return rc;
+    const WsLayout L = ws_layout(h, h->max_tokens);
+    moe::RouteParams p;
+    p.x = x;
+    p.wr = router_w;
+    p.bias = router_bias;
+    p.x_norm = x_norm;
+    p.logits_ws = reinterpret_cast<float *>(h->ws + L.logits);
+    p.logits_out = logits;
+    p.ids = topk_ids;
+    p.w = topk_w;
+    p.counters = reinterpret_cast<unsigned *>(h->ws + L.counters);
+    p.T = T;
+    p.E = h->E;
+    p.H = h->H;
+    p.k = h->k;
+    p.rmsnorm = norm ? 1 : 0;
+    p.eps = 1e-6f;
+    return cuda_rc(moe::launch_route(p, static_cast<cudaStream_t>(stream), h->use_pdl));
+}
+
+int moe_route(moe_handle_t h, const uint16_t *x, int T, const uint16_t *router_w,
+              const float *router_bias, int32_t *topk_ids, float *topk_w, void *stream) {
+    return moe_route_ex(h, x, T, router_w, router_bias, 0u, nullptr, nullptr, topk_ids, topk_w,
+                        stream);
+}
+
+int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk_ids,
+                   const float *topk_w, const uint16_t *residual, uint16_t *y, unsigned flags,
+                   void *stream) {
+    if (!h || T < 1) return MOE_ERR_ARG;
+    const unsigned known = MOE_FWD_KEEP_INTERMEDIATES | MOE_FWD_FORCE_DECODE |
+                           MOE_FWD_FORCE_GROUPED | MOE_FWD_PHASE_GATEUP | MOE_FWD_PHASE_DOWN;
+    if (flags & ~known) return MOE_ERR_ARG;
+    if ((flags & MOE_FWD_FORCE_DECODE) && (flags & MOE_FWD_FORCE_GROUPED)) return MOE_ERR_ARG;
+    if ((flags & MOE_FWD_PHASE_GATEUP) && (flags & MOE_FWD_PHASE_DOWN)) return MOE_ERR_ARG;
+    const bool run_gu = !(flags & MOE_FWD_PHASE_DOWN);
+    const bool run_dn = !(flags & MOE_FWD_PHASE_GATEUP);
+    if (!h->loaded || !h->ws) return MOE_ERR_NOT_LOADED;
+    if (T > h->max_tokens) return MOE_ERR_WORKSPACE;
+    int rc;
+    if ((rc = check_device_ptr(h, x, 16)) != MOE_OK) return rc;
+    if ((rc = check_device_ptr(h, topk_ids, 4)) != MOE_OK) return rc;
+    if ((rc = check_device_ptr(h, topk_w, 4)) != MOE_OK) return rc;
+    if ((rc = check_device_ptr(h, y, 16)) != MOE_OK) return rc;
+    if (residual && (rc = check_device_ptr(h, residual, 16)) != MOE_OK) return rc;
+    if (y == x) return MOE_ERR_ARG;
+    if (!moe::decode_shape_supported(h->H, h->I)) return MOE_ERR_ARG;
+
+    const WsLayout L = ws_layout(h, h->max_tokens);
+    const bool keep = flags & MOE_FWD_KEEP_INTERMEDIATES;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint16_t *hbuf = reinterpret_cast<uint16_t *>(h->ws + L.h);
+    uint16_t *obuf = reinterpret_cast<uint16_t *>(h->ws + L.o);
+
+    // per-(token, slot) GEMV path, in chunks of up to kDecodeMaxT tokens (fewer
+    // when the staged activations of a chunk would not fit in shared memory)
+    int chunk = moe::kDecodeMaxT;
+    while (chunk > 1 && (moe::gateup_decode_smem(chunk, h->H) > moe::kMaxDecodeSmem ||
+                         moe::down_decode_smem(chunk, h->k, h->I,
+                                               (chunk * h->H + h->num_sms - 1) / h->num_sms) >
+                             moe::kMaxDecodeSmem))
+        --chunk;
+    if (moe::down_decode_smem(1, h->k, h->I, (h->H + h->num_sms - 1) / h->num_sms) >
+        moe::kMaxDecodeSmem)
+        return MOE_ERR_ARG;
+    for (int t0 = 0; t0 < T; t0 += chunk) {
+        const int Tc = (T - t0 < chunk) ? T - t0 : chunk;
+        moe::GateUpParams g;
+        g.table = h->d_table;
+        g.x = x + (size_t)t0 * h->H;
+        g.ids = topk_ids + (size_t)t0 * h->k;
+        g.h = hbuf + (size_t)t0 * h->k * h->I;
+        g.status = h->d_status;
+        g.T = Tc;
+        g.k = h->k;
+        g.E = h->E;
+        g.H = h->H;
+        g.I = h->I;
+        g.prefetch_down = h->prefetch_down ? 1 : 0;
+        if (run_gu &&
+            (rc = cuda_rc(moe::launch_gateup_decode(g, h->num_sms, s, h->use_pdl))) != MOE_OK)
+            return rc;
+
+        moe::DownParams d;
+        d.table = h->d_table;
+        d.h = g.h;
+        d.ids = g.ids;
+        d.w = topk_w + (size_t)t0 * h->k;
+        d.residual = residual ? residual + (size_t)t0 * h->H : nullptr;
+        d.y = y + (size_t)t0 * h->H;
+        d.o_keep = keep ? obuf + (size_t)t0 * h->k * h->H : nullptr;
+        d.status = h->d_status;
+        d.T = Tc;
+        d.k = h->k;
+        d.E = h->E;
+        d.H = h->H;
+        d.I = h->I;
+        const int rows = Tc * h->H;
+        d.rows_per_cta = (rows + h->num_sms - 1) / h->num_sms;
+        const int grid = (rows + d.rows_per_cta - 1) / d.rows_per_cta;
+        if (run_dn && (rc = cuda_rc(moe::launch_down_decode(d, grid, s, h->use_pdl))) != MOE_OK)
+            return rc;
+    }
+    h->kept = keep;
+    return MOE_OK;
+}
+
+int moe_forward(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk_ids,
+                const float *topk_w, uint16_t *y, void *stream) {
+    return moe_forward_ex(h, x, T, topk_ids, topk_w, nullptr, y, 0u, stream);
+}
+
+int moe_get_intermediates(moe_handle_t h, const uint16_t **h_out, const uint16_t **o_out) {
+    if (!h || !h_out || !o_out) return MOE_ERR_ARG;
+    if (!h->ws || !h->kept) return MOE_ERR_NOT_LOADED;
+    const WsLayout L = ws_layout(h, h->max_tokens);
+    *h_out = reinterpret_cast<const uint16_t *>(h->ws + L.h);
+    *o_out = reinterpret_cast<const uint16_t *>(h->ws + L.o);
+    return MOE_OK;
+}
+
+int moe_get_status(moe_handle_t h, unsigned *device_status) {
+    if (!h || !device_status) return MOE_ERR_ARG;
+    if (!h->dblock) return MOE_ERR_NOT_LOADED;
+    int rc;
+    if ((rc = cuda_rc(cudaDeviceSynchronize())) != MOE_OK) return rc;
+    unsigned v = 0;
+    if ((rc = cuda_rc(cudaMemcpy(&v, h->d_status, sizeof v, cudaMemcpyDeviceToHost))) != MOE_OK)
+        return rc;
+    if ((rc = cuda_rc(cudaMemset(h->d_status, 0, sizeof v))) != MOE_OK) return rc;
+    *device_status = v;
+    return MOE_OK;
+}
+
+int moe_bytes_per_expert(moe_handle_t h, size_t *bytes) {
+    if (!h || !bytes) return MOE_ERR_ARG;
+    *bytes = (size_t)3 * h->I * h->H / 2 + (size_t)3 * h->I * h->H / 32;
+    return MOE_OK;
+}
+
+int moe_set_tuning(moe_handle_t h, int use_pdl, int prefetch_down) {
+    if (!h) return MOE_ERR_ARG;
+    h->use_pdl = use_pdl != 0;
+    h->prefetch_down = prefetch_down != 0;
+    return MOE_OK;
+}
+
+const char *moe_status_string(int status) {
+    switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_ARG: return "MOE_ERR_ARG: invalid argument";
+    case MOE_ERR_NOT_LOADED: return "MOE_ERR_NOT_LOADED: weights or workspace not set";
+    case MOE_ERR_NOT_DEVICE: return "MOE_ERR_NOT_DEVICE: pointer is not memory of the current device";
+    case MOE_ERR_ALIGN: return "MOE_ERR_ALIGN: pointer not aligned";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace too small";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: CUDA runtime error";
+    case MOE_ERR_DEVICE_STATUS: return "MOE_ERR_DEVICE_STATUS: a kernel flagged invalid input";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: device is not sm_100";
+    default: return "unknown moe status";
+    }
+}
+
+int moe_device_check(void) { return current_device_ok(nullptr, nullptr); }
+
+int moe_debug_dequant(const uint8_t *codes, const uint8_t *scales, int64_t n, float *out,
+                      void *stream) {
+    if (n < 0 || n % 32) return MOE_ERR_ARG;
+    int rc = current_device_ok(nullptr, nullptr);
+    if (rc != MOE_OK) return rc;
+    if (n == 0) return MOE_OK;
+    if ((rc = check_device_ptr(nullptr, codes, 16)) != MOE_OK) return rc;
+    if ((rc = check_device_ptr(nullptr, scales, 1)) != MOE_OK) return rc;
+    if ((rc = check_device_ptr(nullptr, out, 16)) != MOE_OK) return rc;
+    return cuda_rc(moe::launch_debug_dequant(codes, scales, n, out, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

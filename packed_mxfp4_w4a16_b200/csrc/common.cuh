@@ -1,0 +1,200 @@
+// common.cuh — device helpers shared by the sm_100a kernels of this library.
+//
+// Number formats (model card "LFM2.5-24B-A2B — Packed MXFP4 Inference", table
+// "Model and quantization"): weights are E2M1 FP4 codes, two per byte, each 32
+// consecutive K elements share one E8M0 exponent; activations and outputs are
+// BF16; dot products accumulate in FP32.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Addresses of one expert's three packed matrices (0 gate, 1 up, 2 down):
+// codes [rows][K/2] and E8M0 scales [rows][K/32] of each.
+struct ExpertPtrs {
+    const uint8_t *codes[3];
+    const uint8_t *scales[3];
+};
+
+// ----------------------------------------------------------------- BF16 --
+
+__device__ __forceinline__ float bf16_to_f32(uint32_t b) {
+    return __uint_as_float(b << 16);
+}
+
+// Round an FP32 value to BF16 (nearest, ties to even; NaN stays NaN).
+__device__ __forceinline__ uint16_t f32_to_bf16(float f) {
+    uint16_t r;
+    asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(f));
+    return r;
+}
+
+// Round to BF16 and back: the value of a BF16 rounding point.
+__device__ __forceinline__ float round_bf16(float f) {
+    return bf16_to_f32(f32_to_bf16(f));
+}
+
+// ------------------------------------------------------------ loads ------
+
+// 16-byte streaming load of read-only data: no L1 allocation, 256-byte L2
+// fetch granularity (the rows are streamed once per call).
+__device__ __forceinline__ uint4 ld_stream16(const void *p) {
+    uint4 r;
+    asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t ld_stream_u8(const uint8_t *p) {
+    uint16_t r;
+    asm("ld.global.nc.L1::no_allocate.u8 %0, [%1];" : "=h"(r) : "l"(p));
+    return r;
+}
+
+// Hint: bring [p, p + bytes) into L2 (bytes a multiple of 16, p 16-aligned).
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes)
+                 : "memory");
+}
+
+// -------------------------------------------------------- E8M0 / E2M1 ----
+
+// 2^(e-127) in FP32: e = 0 gives the subnormal 2^-127, e = 255 gives NaN.
+__device__ __forceinline__ float e8m0_to_f32(uint32_t e) {
+    uint32_t bits = e << 23;
+    bits = (e == 0u) ? 0x00400000u : bits;
+    bits = (e == 255u) ? 0x7FC00000u : bits;
+    return __uint_as_float(bits);
+}
+
+// The 16-entry E2M1 table applied in registers by the sm_100a conversion
+// instruction: each byte of w (two codes, low nibble = lower element) becomes
+// an f16x2 word, exactly (every E2M1 value is an FP16 value).
+__device__ __forceinline__ void e2m1x8_to_f16x8(uint32_t w, uint32_t (&out)[4]) {
+    asm("{\n\t"
+        ".reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t"
+        "}"
+        : "=r"(out[0]), "=r"(out[1]), "=r"(out[2]), "=r"(out[3])
+        : "r"(w));
+}
+
+__device__ __forceinline__ float f16_bits_to_f32(uint32_t h) {
+    float f;
+    asm("{ .reg .f16 t; mov.b16 t, %1; cvt.f32.f16 %0, t; }" : "=f"(f) : "h"((uint16_t)h));
+    return f;
+}
+
+// Dot product of 8 packed E2M1 codes (one 32-bit word, element order: byte 0
+// low nibble first) with 8 FP16 activations (four f16x2 words), accumulated
+// in FP32 (each product is exact, one rounding per add).  a0 receives the
+// even elements, a1 the odd ones.
+__device__ __forceinline__ void dot8_e2m1_f16(uint32_t w, uint32_t x01, uint32_t x23,
+                                              uint32_t x45, uint32_t x67, float &a0,
+                                              float &a1) {
+    asm("{\n\t"
+        ".reg .b8 b0, b1, b2, b3;\n\t"
+        ".reg .b32 p0, p1, p2, p3;\n\t"
+        ".reg .f16 w0, w1, w2, w3, w4, w5, w6, w7;\n\t"
+        ".reg .f16 x0, x1, x2, x3, x4, x5, x6, x7;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 p0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 p1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 p2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 p3, b3;\n\t"
+        "mov.b32 {w0, w1}, p0;\n\t"
+        "mov.b32 {w2, w3}, p1;\n\t"
+        "mov.b32 {w4, w5}, p2;\n\t"
+        "mov.b32 {w6, w7}, p3;\n\t"
+        "mov.b32 {x0, x1}, %3;\n\t"
+        "mov.b32 {x2, x3}, %4;\n\t"
+        "mov.b32 {x4, x5}, %5;\n\t"
+        "mov.b32 {x6, x7}, %6;\n\t"
+        "fma.rn.f32.f16 %0, w0, x0, %0;\n\t"
+        "fma.rn.f32.f16 %1, w1, x1, %1;\n\t"
+        "fma.rn.f32.f16 %0, w2, x2, %0;\n\t"
+        "fma.rn.f32.f16 %1, w3, x3, %1;\n\t"
+        "fma.rn.f32.f16 %0, w4, x4, %0;\n\t"
+        "fma.rn.f32.f16 %1, w5, x5, %1;\n\t"
+        "fma.rn.f32.f16 %0, w6, x6, %0;\n\t"
+        "fma.rn.f32.f16 %1, w7, x7, %1;\n\t"
+        "}"
+        : "+f"(a0), "+f"(a1)
+        : "r"(w), "r"(x01), "r"(x23), "r"(x45), "r"(x67));
+}
+
+// One 32-element group (16 code bytes) against its 32 FP16 activations
+// (16 f16x2 words): the unscaled partial sum of the group.
+__device__ __forceinline__ float dot32_e2m1_f16(const uint4 &c, const uint32_t *x) {
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    dot8_e2m1_f16(c.x, x[0], x[1], x[2], x[3], a0, a1);
+    dot8_e2m1_f16(c.y, x[4], x[5], x[6], x[7], a2, a3);
+    dot8_e2m1_f16(c.z, x[8], x[9], x[10], x[11], a0, a1);
+    dot8_e2m1_f16(c.w, x[12], x[13], x[14], x[15], a2, a3);
+    return (a0 + a1) + (a2 + a3);
+}
+
+// ------------------------------------------------ FP16 staging of BF16 ----
+// The GEMVs multiply FP16 weights (exact E2M1 values) with activations held
+// in FP16.  A BF16 vector v is staged as v * 2^-c with c chosen from max|v|
+// so that the largest element lands in [2^14, 2^15): every element within
+// 2^29 of the maximum converts exactly (BF16 has 8 significant bits, FP16
+// 11), smaller ones lose bits far below FP32 accumulation noise.  The dot
+// product is multiplied back by 2^c in FP32.
+
+__device__ __forceinline__ int f16_stage_exponent(float amax) {
+    if (!(amax > 0.f) || !(amax <= 3.0e38f))
+        return 0;  // zero, NaN or inf: stage unscaled
+    int e = (int)((__float_as_uint(amax) >> 23) & 0xFFu);
+    if (e == 0)
+        e = 1;  // subnormal maximum
+    return (e - 127) - 14;
+}
+
+__device__ __forceinline__ uint16_t f32_to_f16_bits(float f) {
+    uint16_t r;
+    asm("cvt.rn.f16.f32 %0, %1;" : "=h"(r) : "f"(f));
+    return r;
+}
+
+// ------------------------------------------------------------- warps -----
+
+template <int TL>
+__device__ __forceinline__ float team_sum(float v) {
+#pragma unroll
+    for (int o = TL / 2; o > 0; o >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// ------------------------------------------- programmatic launch ---------
+
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+}  // namespace moe

@@ -1,0 +1,67 @@
+// kernels.cuh — launch parameters and entry points of the sm_100a kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kDecodeMaxT = 4;      // tokens handled by the per-(token,slot) GEMV path
+constexpr int kMaxTopK = 8;
+constexpr int kGemvThreads = 512;   // 16 warps, one CTA per SM
+constexpr int kRouteThreads = 256;  // 8 warps, one expert row per warp
+constexpr unsigned kBadExpertId = 0x1u;
+constexpr size_t kMaxDecodeSmem = 200 * 1024;  // dynamic shared memory cap of the GEMVs
+
+struct RouteParams {
+    const uint16_t *x;      // [T][H] BF16 (residual stream when rmsnorm)
+    const uint16_t *wr;     // [E][H] BF16
+    const float *bias;      // [E] or null
+    uint16_t *x_norm;       // [T][H] or null
+    float *logits_ws;       // [T][E] workspace
+    float *logits_out;      // [T][E] or null
+    int32_t *ids;           // [T][k]
+    float *w;               // [T][k]
+    unsigned *counters;     // [T], zero between calls
+    int T, E, H, k;
+    int rmsnorm;
+    float eps;
+};
+
+struct GateUpParams {
+    const ExpertPtrs *table;  // [E]
+    const uint16_t *x;        // [T][H]
+    const int32_t *ids;       // [T][k]
+    uint16_t *h;              // [T][k][I]
+    unsigned *status;
+    int T, k, E, H, I;
+    int prefetch_down;        // L2-prefetch the selected down matrices
+};
+
+struct DownParams {
+    const ExpertPtrs *table;
+    const uint16_t *h;         // [T][k][I]
+    const int32_t *ids;        // [T][k]
+    const float *w;            // [T][k]
+    const uint16_t *residual;  // [T][H] or null
+    uint16_t *y;               // [T][H]
+    uint16_t *o_keep;          // [T][k][H] or null
+    unsigned *status;
+    int T, k, E, H, I;
+    int rows_per_cta;
+};
+
+// Host-side launchers (decode.cu).  `pdl` sets programmatic stream
+// serialization so the kernel may start while the previous one drains.
+cudaError_t launch_route(const RouteParams &p, cudaStream_t s, bool pdl);
+cudaError_t launch_gateup_decode(const GateUpParams &p, int grid, cudaStream_t s, bool pdl);
+cudaError_t launch_down_decode(const DownParams &p, int grid, cudaStream_t s, bool pdl);
+cudaError_t launch_debug_dequant(const uint8_t *codes, const uint8_t *scales, int64_t n,
+                                 float *out, cudaStream_t s);
+size_t gateup_decode_smem(int T, int H);
+size_t down_decode_smem(int T, int k, int I, int rows_per_cta);
+bool decode_shape_supported(int H, int I);
+
+}  // namespace moe

@@ -1,0 +1,74 @@
+"""Helpers shared by the GPU parity tests: move seeded inputs to the device,
+bring results back as BF16 bits, and the comparison rules."""
+import numpy as np
+import torch
+
+import oracle
+
+TOL = 1e-2  # max|gpu - oracle| <= TOL * rms(oracle), per output vector
+
+
+def dev_bf16(u16: np.ndarray) -> torch.Tensor:
+    a = np.ascontiguousarray(u16, dtype=np.uint16)
+    return torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def host_bf16(t: torch.Tensor) -> np.ndarray:
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def dev_u8(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint8)).cuda()
+
+
+def dev_layer(L):
+    """workloads.LayerInputs -> device tensors (codes, scales, router_w, router_b)."""
+    rb = None if L.router_b is None else torch.from_numpy(L.router_b).cuda()
+    return dev_u8(L.codes), dev_u8(L.scales), dev_bf16(L.router_w), rb
+
+
+def f64(u16):
+    return oracle.bf16_to_f64_array(u16)
+
+
+def assert_close_rms(gpu_u16, ref_u16, tol=TOL, what=""):
+    """Per vector (last axis): max|gpu - ref| <= tol * rms(ref).  Returns the
+    number of elements that differ at all (BF16 rounding flips)."""
+    g = f64(gpu_u16).reshape(-1, np.shape(ref_u16)[-1])
+    r = f64(ref_u16).reshape(g.shape)
+    assert np.all(np.isfinite(g)) and np.all(np.isfinite(r)), what
+    rms = np.sqrt(np.mean(r * r, axis=1))
+    err = np.max(np.abs(g - r), axis=1)
+    bad = err > tol * rms
+    assert not np.any(bad), (f"{what}: max err {err[bad].max():.3e} vs rms "
+                             f"{rms[bad].min():.3e} in {bad.sum()} vectors")
+    return int(np.count_nonzero(g != r))
+
+
+def near_tie_tokens(logits: np.ndarray, k: int, rel=1e-4):
+    """Tokens whose oracle logits leave a gap < rel*max|logit| between any two
+    of the k+1 largest (the selection or the slot order could flip under a
+    different summation order)."""
+    flags = []
+    for row in np.atleast_2d(logits):
+        s = np.sort(row)[::-1][: k + 1]
+        gaps = s[:-1] - s[1:]
+        flags.append(bool(np.min(gaps) < rel * np.max(np.abs(row))))
+    return np.array(flags)
+
+
+def check_routing(gpu_ids, gpu_w, gpu_logits, ref_ids, ref_w, ref_logits, k):
+    """Ids bit-exact to the oracle except on flagged near-ties, where they must
+    equal the oracle's selector applied to the GPU's own logits.  Weights
+    within 1e-5 relative.  Returns the number of near-tie tokens."""
+    ties = near_tie_tokens(ref_logits, k)
+    np.testing.assert_allclose(gpu_logits, ref_logits, rtol=1e-4, atol=1e-4)
+    for t in range(gpu_ids.shape[0]):
+        if ties[t]:
+            ids2, w2 = oracle.select_topk(gpu_logits[t].astype(np.float64), k)
+            np.testing.assert_array_equal(gpu_ids[t], ids2[0])
+            np.testing.assert_allclose(gpu_w[t], w2[0], rtol=1e-5, atol=1e-6)
+        else:
+            np.testing.assert_array_equal(gpu_ids[t], ref_ids[t])
+            np.testing.assert_allclose(gpu_w[t], ref_w[t], rtol=1e-5, atol=1e-6)
+    return int(ties.sum())

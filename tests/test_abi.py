@@ -1,0 +1,105 @@
+"""The C-ABI library loads and exports every symbol include/*.h declares, and
+host-side validation works without a GPU."""
+import ctypes as C
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+from conftest import ROOT
+
+HEADERS = glob.glob(os.path.join(ROOT, "include", "*.h"))
+
+
+def declared_functions():
+    names = set()
+    for h in HEADERS:
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(moe_\w+)\s*\(", src, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from packed_mxfp4_w4a16_b200 import _lib
+    return _lib.load()
+
+
+def test_header_declares_the_four_calls():
+    names = declared_functions()
+    for n in ("moe_create", "moe_load_packed", "moe_route", "moe_forward"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from packed_mxfp4_w4a16_b200 import _lib
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.library_path()],
+                         capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    declared = declared_functions()
+    assert declared, "no declarations parsed"
+    missing = declared - exported
+    assert not missing, f"declared but not exported: {sorted(missing)}"
+    # the binding declares exactly the header's functions
+    bound = {name for name, _, _ in _lib.SIGNATURES}
+    assert bound == declared
+    # nothing but the C ABI leaks out of the library
+    extra = {s for s in exported if s.startswith("moe_")} - declared
+    assert not extra
+
+
+def test_create_validates_shapes(lib):
+    h = C.c_void_p()
+    ok = [(64, 2048, 1536, 4), (16, 512, 384, 4), (1, 32, 32, 1), (8, 64, 96, 8)]
+    for E, H, I, k in ok:
+        assert lib.moe_create(E, H, I, k, C.byref(h)) == 0 and h.value
+        assert lib.moe_destroy(h) == 0
+    bad = [(0, 2048, 1536, 4), (64, 2047, 1536, 4), (64, 2048, 1530, 4), (64, 2048, 1536, 0),
+           (64, 2048, 1536, 9), (3, 64, 64, 4), (2000, 64, 64, 4), (64, 16, 64, 1)]
+    for E, H, I, k in bad:
+        h = C.c_void_p(123)
+        assert lib.moe_create(E, H, I, k, C.byref(h)) == -1
+        assert h.value is None
+    assert lib.moe_create(64, 2048, 1536, 4, None) == -1
+    assert lib.moe_destroy(None) == 0
+
+
+def test_bytes_per_expert_closed_form(lib):
+    h = C.c_void_p()
+    assert lib.moe_create(64, 2048, 1536, 4, C.byref(h)) == 0
+    n = C.c_size_t()
+    assert lib.moe_bytes_per_expert(h, C.byref(n)) == 0
+    # 3*2048*1536 weights at 0.5 + 1/32 byte each
+    assert n.value == 5013504
+    ws = C.c_size_t()
+    assert lib.moe_workspace_bytes(h, 1, C.byref(ws)) == 0 and ws.value > 0
+    ws4 = C.c_size_t()
+    assert lib.moe_workspace_bytes(h, 4, C.byref(ws4)) == 0 and ws4.value > ws.value
+    assert lib.moe_workspace_bytes(h, 0, C.byref(ws)) == -1
+    lib.moe_destroy(h)
+
+
+def test_calls_fail_cleanly_without_weights_or_device(lib):
+    h = C.c_void_p()
+    assert lib.moe_create(16, 512, 384, 4, C.byref(h)) == 0
+    # no workspace / weights: forward and route refuse before touching CUDA
+    assert lib.moe_forward(h, None, 1, None, None, None, None) in (-1, -2)
+    assert lib.moe_route(h, None, 1, None, None, None, None, None) in (-1, -2)
+    assert lib.moe_forward(h, None, 0, None, None, None, None) == -1
+    st = C.c_uint()
+    assert lib.moe_get_status(h, C.byref(st)) == -2
+    hp, op = C.c_void_p(), C.c_void_p()
+    assert lib.moe_get_intermediates(h, C.byref(hp), C.byref(op)) == -2
+    assert lib.moe_set_tuning(h, 1, 0) == 0
+    lib.moe_destroy(h)
+
+
+def test_status_strings(lib):
+    for code in range(-8, 1):
+        s = lib.moe_status_string(code).decode()
+        assert s.startswith("MOE_")
+    assert lib.moe_status_string(-99).decode() == "unknown moe status"

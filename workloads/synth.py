@@ -85,8 +85,15 @@ WORKLOADS = {
 
 
 def rng_for(seed: int, *stream: int) -> np.random.Generator:
-    """Independent, reproducible generator for (seed, stream...)."""
-    return np.random.default_rng([seed, *stream])
+    """Independent, reproducible generator for (seed, stream...) (SFC64 bit
+    generator seeded through a SeedSequence)."""
+    return np.random.Generator(np.random.SFC64(np.random.SeedSequence([seed, *stream])))
+
+
+def uniform_bytes(n: int, rng: np.random.Generator) -> np.ndarray:
+    """n independent bytes uniform over 0..255."""
+    words = rng.integers(0, 2 ** 64 - 1, size=(n + 7) // 8, dtype=np.uint64, endpoint=True)
+    return words.view(np.uint8)[:n]
 
 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -114,8 +121,7 @@ def make_expert_weights(shape: LayerShape, rng: np.random.Generator):
     Returns (codes uint8 [E, 3*I*H/2], scales uint8 [E, 3*I*H/32]).
     """
     n_codes = shape.E * shape.codes_per_expert
-    codes = np.frombuffer(rng.bytes(n_codes), dtype=np.uint8).reshape(
-        shape.E, shape.codes_per_expert)
+    codes = uniform_bytes(n_codes, rng).reshape(shape.E, shape.codes_per_expert)
     scales = rng.integers(E8M0_LO, E8M0_HI + 1,
                           size=(shape.E, shape.scales_per_expert),
                           dtype=np.uint8)
