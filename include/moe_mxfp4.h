@@ -111,8 +111,8 @@ typedef enum moe_status {
                                       two calls together equal one forward  */
 
 /* Create a layer of E experts with hidden size H, intermediate size I and
- * top_k experts per token.  Requires H % 32 == 0, I % 32 == 0, H >= 32,
- * I >= 32, 1 <= top_k <= min(E, 8), E <= 1024.  Host-only: allocates the
+ * top_k experts per token.  Requires H % 32 == 0, I % 32 == 0,
+ * 32 <= H <= 4096, 32 <= I <= 4096, 1 <= top_k <= min(E, 8), E <= 1024.  Host-only: allocates the
  * handle, touches no GPU.  *out receives the handle (NULL on error).
  * Errors: MOE_ERR_ARG. */
 MOE_API int moe_create(int E, int H, int I, int top_k, moe_handle_t *out);

@@ -136,7 +136,7 @@ int moe_create(int E, int H, int I, int top_k, moe_handle_t *out) {
     *out = nullptr;
     if (E < 1 || E > 1024 || H < 32 || I < 32 || H % 32 || I % 32) return MOE_ERR_ARG;
     if (top_k < 1 || top_k > moe::kMaxTopK || top_k > E) return MOE_ERR_ARG;
-    if (H > 16384 || I > 16384) return MOE_ERR_ARG;
+    if (H > 4096 || I > 4096) return MOE_ERR_ARG;
     moe_ctx *c = new (std::nothrow) moe_ctx;
     if (!c) return MOE_ERR_ARG;
     c->E = E;
@@ -314,6 +314,12 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
         g.H = h->H;
         g.I = h->I;
         g.prefetch_down = h->prefetch_down ? 1 : 0;
+        {
+            const size_t mc = (size_t)h->H * h->I / 2, ms = (size_t)h->H * h->I / 32;
+            const size_t n = (size_t)h->num_sms;
+            g.pf_codes = (uint32_t)(((mc + n - 1) / n + 15) / 16 * 16);
+            g.pf_scales = (uint32_t)(((ms + n - 1) / n + 15) / 16 * 16);
+        }
         if (run_gu &&
             (rc = cuda_rc(moe::launch_gateup_decode(g, h->num_sms, s, h->use_pdl))) != MOE_OK)
             return rc;

@@ -153,14 +153,33 @@ __device__ __forceinline__ int f16_stage_exponent(float amax) {
     if (!(amax > 0.f) || !(amax <= 3.0e38f))
         return 0;  // zero, NaN or inf: stage unscaled
     int e = (int)((__float_as_uint(amax) >> 23) & 0xFFu);
-    if (e == 0)
-        e = 1;  // subnormal maximum
-    return (e - 127) - 14;
+    // c = (biased exponent of max) - 127 - 14, clamped so that 2^-c stays a
+    // normal FP32 value (vectors whose max is below 2^-113 are staged with
+    // less headroom; they are far below any activation scale in practice)
+    int c = e - 141;
+    return c < -127 ? -127 : c;
+}
+
+// 2^-c for c in [-127, 113], exact, as an FP32 normal number.
+__device__ __forceinline__ float pow2_neg(int c) {
+    return __uint_as_float((uint32_t)(127 - c) << 23);
+}
+
+// 2^c for c in [-127, 113], exact (2^-127 is the subnormal 0x00400000).
+__device__ __forceinline__ float pow2(int c) {
+    return c >= -126 ? __uint_as_float((uint32_t)(c + 127) << 23) : __uint_as_float(0x00400000u);
 }
 
 __device__ __forceinline__ uint16_t f32_to_f16_bits(float f) {
     uint16_t r;
     asm("cvt.rn.f16.f32 %0, %1;" : "=h"(r) : "f"(f));
+    return r;
+}
+
+// Two FP32 values -> one f16x2 word (lo in the low half), round to nearest.
+__device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
 

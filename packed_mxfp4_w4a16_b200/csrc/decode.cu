@@ -34,65 +34,81 @@
 namespace moe {
 
 constexpr int kGemvWarps = kGemvThreads / 32;
+constexpr int kDownWarps = kDownThreads / 32;
 
 // ------------------------------------------------------------------ route --
+// grid (E, ceil(T / 8)); warp w of CTA (e, b) computes logit[t = 8b + w][e].
+// The router row is fetched before the programmatic-launch wait (it is a
+// constant input), so its DRAM latency overlaps the previous kernel's tail.
+
+constexpr int kRouteWarps = kRouteThreads / 32;
+constexpr int kRouteMaxChunks = 16;  // H <= 16 * 32 * 8 = 4096 for the register path
 
 __global__ void __launch_bounds__(kRouteThreads)
 route_kernel(const RouteParams p) {
-    extern __shared__ float xs[];  // [H] the routed vector in FP32
-    __shared__ float s_red[kRouteThreads / 32];
     __shared__ int s_last;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int t = blockIdx.y, H = p.H, E = p.E, k = p.k;
-    const uint16_t *xt = p.x + (size_t)t * H;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int e = blockIdx.x, H = p.H, E = p.E, k = p.k;
+    const int t = blockIdx.y * kRouteWarps + warp;
+    const int nch = H >> 3;  // 16-byte chunks of 8 BF16
+    const bool active = t < p.T;
+
+    uint4 wv[kRouteMaxChunks];
+    const uint16_t *row = p.wr + (size_t)e * H;
+#pragma unroll
+    for (int m = 0; m < kRouteMaxChunks; ++m) {
+        const int c = lane + 32 * m;
+        wv[m] = (active && c < nch) ? *reinterpret_cast<const uint4 *>(row + (size_t)c * 8)
+                                    : make_uint4(0u, 0u, 0u, 0u);
+    }
 
     pdl_wait();
     pdl_launch_dependents();
 
-    if (p.rmsnorm) {
-        // weightless RMSNorm: xn = BF16(r / sqrt(mean(r^2) + eps))
+    if (active) {
+        const uint16_t *xt = p.x + (size_t)t * H;
+        uint4 xv[kRouteMaxChunks];
         float ss = 0.f;
-        for (int i = tid; i < H; i += kRouteThreads) {
-            float v = bf16_to_f32(xt[i]);
-            ss = fmaf(v, v, ss);
+#pragma unroll
+        for (int m = 0; m < kRouteMaxChunks; ++m) {
+            const int c = lane + 32 * m;
+            xv[m] = c < nch ? *reinterpret_cast<const uint4 *>(xt + (size_t)c * 8)
+                            : make_uint4(0u, 0u, 0u, 0u);
+            if (p.rmsnorm) {
+                const uint32_t w4[4] = {xv[m].x, xv[m].y, xv[m].z, xv[m].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float a = bf16_to_f32(w4[q] & 0xFFFFu), b = bf16_to_f32(w4[q] >> 16);
+                    ss = fmaf(a, a, ss);
+                    ss = fmaf(b, b, ss);
+                }
+            }
         }
-        ss = warp_sum(ss);
-        if (lane == 0) s_red[warp] = ss;
-        __syncthreads();
-        if (warp == 0) {
-            float v = lane < kRouteThreads / 32 ? s_red[lane] : 0.f;
-            v = warp_sum(v);
-            if (lane == 0) s_red[0] = 1.0f / sqrtf(v / (float)H + p.eps);
-        }
-        __syncthreads();
-        const float inv = s_red[0];
-        for (int i = tid; i < H; i += kRouteThreads) {
-            uint16_t b = f32_to_bf16(bf16_to_f32(xt[i]) * inv);
-            xs[i] = bf16_to_f32(b);
-            if (blockIdx.x == 0) p.x_norm[(size_t)t * H + i] = b;
-        }
-    } else {
-        for (int i = tid; i < H; i += kRouteThreads) xs[i] = bf16_to_f32(xt[i]);
-    }
-    __syncthreads();
-
-    // one expert row per warp: logits = x . Wr[e] in FP32 (+ bias)
-    const int nchunk = H >> 3;  // 8 BF16 per 16-byte chunk
-    for (int e = blockIdx.x * (kRouteThreads / 32) + warp; e < E;
-         e += gridDim.x * (kRouteThreads / 32)) {
-        const uint16_t *row = p.wr + (size_t)e * H;
+        float inv = 1.f;
+        if (p.rmsnorm) inv = 1.0f / sqrtf(warp_sum(ss) / (float)H + p.eps);
         float acc = 0.f;
-        for (int c = lane; c < nchunk; c += 32) {
-            uint4 v = *reinterpret_cast<const uint4 *>(row + (size_t)c * 8);
-            const float *xv = xs + c * 8;
-            acc = fmaf(bf16_to_f32(v.x & 0xFFFFu), xv[0], acc);
-            acc = fmaf(bf16_to_f32(v.x >> 16), xv[1], acc);
-            acc = fmaf(bf16_to_f32(v.y & 0xFFFFu), xv[2], acc);
-            acc = fmaf(bf16_to_f32(v.y >> 16), xv[3], acc);
-            acc = fmaf(bf16_to_f32(v.z & 0xFFFFu), xv[4], acc);
-            acc = fmaf(bf16_to_f32(v.z >> 16), xv[5], acc);
-            acc = fmaf(bf16_to_f32(v.w & 0xFFFFu), xv[6], acc);
-            acc = fmaf(bf16_to_f32(v.w >> 16), xv[7], acc);
+#pragma unroll
+        for (int m = 0; m < kRouteMaxChunks; ++m) {
+            const int c = lane + 32 * m;
+            if (c < nch) {
+                uint32_t x4[4] = {xv[m].x, xv[m].y, xv[m].z, xv[m].w};
+                const uint32_t r4[4] = {wv[m].x, wv[m].y, wv[m].z, wv[m].w};
+                if (p.rmsnorm) {
+                    // weightless RMSNorm: xn = BF16(r / sqrt(mean(r^2) + eps))
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        x4[q] = (uint32_t)f32_to_bf16(bf16_to_f32(x4[q] & 0xFFFFu) * inv) |
+                                ((uint32_t)f32_to_bf16(bf16_to_f32(x4[q] >> 16) * inv) << 16);
+                    if (e == 0)
+                        *reinterpret_cast<uint4 *>(p.x_norm + (size_t)t * H + (size_t)c * 8) =
+                            make_uint4(x4[0], x4[1], x4[2], x4[3]);
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    acc = fmaf(bf16_to_f32(x4[q] & 0xFFFFu), bf16_to_f32(r4[q] & 0xFFFFu), acc);
+                    acc = fmaf(bf16_to_f32(x4[q] >> 16), bf16_to_f32(r4[q] >> 16), acc);
+                }
+            }
         }
         acc = warp_sum(acc);
         if (lane == 0) {
@@ -101,46 +117,58 @@ route_kernel(const RouteParams p) {
         }
     }
 
-    // the last CTA of this token selects (no waiting: an arrival counter)
+    // the last CTA of this token block selects; an arrival counter, no waiting
     __syncthreads();
-    if (tid == 0) {
+    if (threadIdx.x == 0) {
         __threadfence();
-        unsigned prev = atomicAdd(p.counters + t, 1u);
-        s_last = (prev == gridDim.x - 1);
+        const unsigned prev = atomicAdd(p.counters + blockIdx.y, 1u);
+        s_last = (prev == (unsigned)E - 1u);
     }
     __syncthreads();
-    if (!s_last || warp != 0) return;
+    if (!s_last || !active) return;
     __threadfence();
 
+    // top-k of logits[t][0..E): ids descending, equal logits -> lower id.
+    // Each round: warp-wide max of an order-preserving key of the logit, then
+    // the minimum id among the lanes holding that key (two redux operations).
     const float *lg = p.logits_ws + (size_t)t * E;
+    constexpr int kMaxPerLane = 32;  // E <= 1024
+    const int per = (E + 31) >> 5;
+    uint32_t key[kMaxPerLane];
+#pragma unroll
+    for (int m = 0; m < kMaxPerLane; ++m) {
+        const int ee = lane + 32 * m;
+        uint32_t kk = 0u;  // below every logit: never chosen
+        if (m < per && ee < E) {
+            const float v = __ldcg(lg + ee);
+            const uint32_t b = __float_as_uint(v);
+            kk = (v != v) ? 0u : ((b & 0x80000000u) ? ~b : (b | 0x80000000u));
+        }
+        key[m] = kk;
+    }
     int chosen[kMaxTopK];
     float chosen_v[kMaxTopK];
     for (int j = 0; j < k; ++j) {
-        float bv = -INFINITY;
+        uint32_t bk = 0u;
         int bi = 0x7FFFFFFF;
-        for (int e = lane; e < E; e += 32) {
-            bool taken = false;
-            for (int q = 0; q < j; ++q) taken |= (chosen[q] == e);
-            float v = __ldcg(lg + e);
-            if (!taken && (v > bv || (v == bv && e < bi))) {
-                bv = v;
-                bi = e;
-            }
-        }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (ov > bv || (ov == bv && oi < bi)) {
-                bv = ov;
-                bi = oi;
+        for (int m = 0; m < kMaxPerLane; ++m)
+            if (key[m] > bk) {  // ascending m: ties keep the lower id
+                bk = key[m];
+                bi = lane + 32 * m;
             }
+        const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
+        const int wi = (int)__reduce_min_sync(0xffffffffu, bk == wk ? (uint32_t)bi : 0x7FFFFFFFu);
+        chosen[j] = wi;
+        chosen_v[j] = __uint_as_float((wk & 0x80000000u) ? (wk & 0x7FFFFFFFu) : ~wk);
+        if ((wi & 31) == lane && wi < E) {
+#pragma unroll
+            for (int m = 0; m < kMaxPerLane; ++m)
+                if (m == (wi >> 5)) key[m] = 0u;
         }
-        chosen[j] = bi;
-        chosen_v[j] = bv;
     }
     if (lane == 0) {
-        // coefficients: softmax over the k selected logits (slot 0 is the max)
+        // coefficients: softmax over the k selected logits (slot 0 holds the max)
         float z = 0.f, ex[kMaxTopK];
         for (int j = 0; j < k; ++j) {
             ex[j] = expf(chosen_v[j] - chosen_v[0]);
@@ -150,264 +178,311 @@ route_kernel(const RouteParams p) {
             p.ids[(size_t)t * k + j] = chosen[j];
             p.w[(size_t)t * k + j] = ex[j] / z;
         }
-        p.counters[t] = 0u;
     }
     if (p.logits_out)
-        for (int e = lane; e < E; e += 32) p.logits_out[(size_t)t * E + e] = __ldcg(lg + e);
+        for (int ee = lane; ee < E; ee += 32) p.logits_out[(size_t)t * E + ee] = __ldcg(lg + ee);
+    if (warp == 0 && lane == 0) p.counters[blockIdx.y] = 0u;
 }
 
-// --------------------------------------------------------------- staging --
+// ------------------------------------------------------------- team tools --
+// A "team" of TL lanes (TL a power of two, aligned in the warp) owns one packed
+// row at a time; lane lt of the team holds the KCH consecutive 16-byte chunks
+// [lt*KCH, lt*KCH + KCH) of the row (one E8M0 group each) and the matching
+// FP16-staged activations in registers.  Teams are independent: their
+// shuffles use the team's own lane mask.
 
-// Stage BF16 vector v[0..n) as FP16 words in shared memory (scaled by 2^-c,
-// c from the vector's max |v|); returns c.  Called by one warp.
-__device__ __forceinline__ int stage_f16_warp(const uint16_t *v, int n, uint32_t *dst,
-                                              int lane) {
-    float m = 0.f;
-    const uint32_t *v2 = reinterpret_cast<const uint32_t *>(v);
-    for (int i = lane; i < (n >> 1); i += 32) {
-        uint32_t pr = v2[i];
-        m = fmaxf(m, fmaxf(fabsf(bf16_to_f32(pr & 0xFFFFu)), fabsf(bf16_to_f32(pr >> 16))));
+template <int TL>
+__device__ __forceinline__ unsigned team_mask(int lane) {
+    return TL == 32 ? 0xffffffffu : (((1u << TL) - 1u) << (lane & ~(TL - 1)));
+}
+
+template <int TL>
+__device__ __forceinline__ float team_max(float v, unsigned mask) {
+#pragma unroll
+    for (int o = TL / 2; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(mask, v, o));
+    return v;
+}
+
+template <int TL>
+__device__ __forceinline__ float team_add(float v, unsigned mask) {
+#pragma unroll
+    for (int o = TL / 2; o > 0; o >>= 1) v += __shfl_xor_sync(mask, v, o);
+    return v;
+}
+
+// Load this lane's part of BF16 vector v (K elements), stage it as FP16 words
+// scaled by 2^-c where c comes from the team-wide max |v|; returns c.
+template <int TL, int KCH>
+__device__ __forceinline__ int stage_x(const uint16_t *v, int lt, int C, unsigned mask,
+                                       uint32_t (&xw)[KCH][16]) {
+    uint4 raw[KCH][4];
+    float m[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < KCH; ++u) {
+        const int c = lt * KCH + u;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            raw[u][q] = c < C ? *reinterpret_cast<const uint4 *>(v + (size_t)c * 32 + q * 8)
+                              : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t w4[4] = {raw[u][q].x, raw[u][q].y, raw[u][q].z, raw[u][q].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                m[i] = fmaxf(m[i], fmaxf(fabsf(bf16_to_f32(w4[i] & 0xFFFFu)),
+                                         fabsf(bf16_to_f32(w4[i] >> 16))));
+        }
     }
-    m = warp_max(m);
-    const int c = f16_stage_exponent(m);
-    for (int i = lane; i < (n >> 1); i += 32) {
-        uint32_t pr = v2[i];
-        float a = scalbnf(bf16_to_f32(pr & 0xFFFFu), -c);
-        float b = scalbnf(bf16_to_f32(pr >> 16), -c);
-        dst[i] = (uint32_t)f32_to_f16_bits(a) | ((uint32_t)f32_to_f16_bits(b) << 16);
-    }
+    const int c = f16_stage_exponent(team_max<TL>(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), mask));
+    const float sf = pow2_neg(c);
+#pragma unroll
+    for (int u = 0; u < KCH; ++u)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t w4[4] = {raw[u][q].x, raw[u][q].y, raw[u][q].z, raw[u][q].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                xw[u][q * 4 + i] = f32x2_to_f16x2(bf16_to_f32(w4[i] & 0xFFFFu) * sf,
+                                                  bf16_to_f32(w4[i] >> 16) * sf);
+        }
     return c;
 }
 
-// Sum over the KCH chunks of one lane of a packed row against staged FP16
-// activations (xw = the row's activation words).  Each chunk is one E8M0 group.
-template <int TL, int KCH>
-__device__ __forceinline__ float row_partial(const uint4 (&cw)[KCH], const uint32_t (&sc)[KCH],
-                                             const uint32_t *xw, int lt, int C) {
+template <int KCH>
+__device__ __forceinline__ void load_chunks(const uint8_t *codes, const uint8_t *scales, bool ok,
+                                            int lt, int C, uint4 (&cw)[KCH], uint32_t (&sc)[KCH]) {
+#pragma unroll
+    for (int u = 0; u < KCH; ++u) {
+        const int c = lt * KCH + u;
+        if (ok && c < C) {
+            cw[u] = ld_stream16(codes + (size_t)c * 16);
+            sc[u] = ld_stream_u8(scales + c);
+        } else {
+            cw[u] = make_uint4(0u, 0u, 0u, 0u);
+            sc[u] = 127u;
+        }
+    }
+}
+
+template <int KCH>
+__device__ __forceinline__ float chunks_dot(const uint4 (&cw)[KCH], const uint32_t (&sc)[KCH],
+                                            const uint32_t (&xw)[KCH][16]) {
     float acc = 0.f;
 #pragma unroll
-    for (int m = 0; m < KCH; ++m) {
-        const int c = lt + m * TL;
-        if (c < C) {
-            const uint4 *xv = reinterpret_cast<const uint4 *>(xw + c * 16);
-            uint32_t x[16];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint4 v = xv[q];
-                x[4 * q + 0] = v.x;
-                x[4 * q + 1] = v.y;
-                x[4 * q + 2] = v.z;
-                x[4 * q + 3] = v.w;
-            }
-            acc = fmaf(dot32_e2m1_f16(cw[m], x), e8m0_to_f32(sc[m]), acc);
-        }
+    for (int u = 0; u < KCH; ++u) {
+        float a0 = 0.f, a1 = 0.f;
+        dot8_e2m1_f16(cw[u].x, xw[u][0], xw[u][1], xw[u][2], xw[u][3], a0, a1);
+        dot8_e2m1_f16(cw[u].y, xw[u][4], xw[u][5], xw[u][6], xw[u][7], a0, a1);
+        dot8_e2m1_f16(cw[u].z, xw[u][8], xw[u][9], xw[u][10], xw[u][11], a0, a1);
+        dot8_e2m1_f16(cw[u].w, xw[u][12], xw[u][13], xw[u][14], xw[u][15], a0, a1);
+        acc = fmaf(a0 + a1, e8m0_to_f32(sc[u]), acc);
     }
     return acc;
 }
 
-template <int TL, int KCH>
-__device__ __forceinline__ void load_row(const uint8_t *codes, const uint8_t *scales, bool ok,
-                                         int lt, int C, uint4 (&cw)[KCH], uint32_t (&sc)[KCH]) {
-#pragma unroll
-    for (int m = 0; m < KCH; ++m) {
-        const int c = lt + m * TL;
-        if (ok && c < C) {
-            cw[m] = ld_stream16(codes + (size_t)c * 16);
-            sc[m] = ld_stream_u8(scales + c);
-        } else {
-            cw[m] = make_uint4(0u, 0u, 0u, 0u);
-            sc[m] = 127u;
-        }
-    }
-}
-
 // ----------------------------------------------------------- gate / up ----
 
-// L2 prefetch of this CTA's share of the selected experts' down matrices, so
+// L2 prefetch of this CTA's slice of the selected experts' down matrices, so
 // that the down GEMV that follows reads them from L2 while the DRAM keeps
-// streaming.  Experts repeated across (token, slot) pairs are fetched once.
-__device__ void prefetch_down_share(const GateUpParams &p) {
+// streaming.  One lane per (token, slot) pair; an expert chosen by several
+// pairs is fetched by the lowest such lane only.  Slices are 16-byte multiples
+// computed on the host (codes: pf_codes bytes, scales: pf_scales bytes).
+__device__ __forceinline__ void prefetch_down_slice(const GateUpParams &p, int lane) {
     const int P = p.T * p.k;
-    const size_t mc = (size_t)p.H * p.I / 2, ms = (size_t)p.H * p.I / 32;
-    for (int which = 0; which < 2; ++which) {
-        const size_t per = which ? ms : mc;
-        const size_t total = per * (size_t)P;
-        const size_t b0 = (total * blockIdx.x / gridDim.x) & ~(size_t)15;
-        const size_t b1 = (blockIdx.x + 1 == gridDim.x) ? total
-                                                         : ((total * (blockIdx.x + 1) / gridDim.x) & ~(size_t)15);
-        for (size_t b = b0; b < b1;) {
-            const int q = (int)(b / per);
-            const size_t off = b - (size_t)q * per;
-            const size_t len = min(b1 - b, per - off);
-            const int e = p.ids[q];
-            bool dup = false;
-            for (int q2 = 0; q2 < q; ++q2) dup |= (p.ids[q2] == e);
-            if (!dup && e >= 0 && e < p.E) {
-                const uint8_t *base = (which ? p.table[e].scales[2] : p.table[e].codes[2]) + off;
-                for (size_t o = 0; o < len; o += 32768) {
-                    const uint32_t n = (uint32_t)min((size_t)32768, len - o);
-                    if (n >= 16) prefetch_l2_bulk(base + o, n & ~15u);
-                }
+    const int Pr = (P + 31) & ~31;  // every lane iterates the same number of times
+    for (int q = lane; q < Pr; q += 32) {
+        const int e = q < P ? p.ids[q] : -1;
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        const bool leader = (__ffs(same) - 1) == lane;
+        if (q < P && leader && e >= 0 && e < p.E) {
+            const size_t mc = (size_t)p.H * p.I / 2, ms = (size_t)p.H * p.I / 32;
+            const size_t oc = (size_t)blockIdx.x * p.pf_codes;
+            const size_t os = (size_t)blockIdx.x * p.pf_scales;
+            if (oc < mc) {
+                const size_t n = min((size_t)p.pf_codes, mc - oc);
+                prefetch_l2_bulk(p.table[e].codes[2] + oc, (uint32_t)n);
             }
-            b += len;
+            if (os < ms) {
+                const size_t n = min((size_t)p.pf_scales, ms - os);
+                prefetch_l2_bulk(p.table[e].scales[2] + os, (uint32_t)n);
+            }
         }
     }
 }
 
+// Items are (pair q = t*k + j, row i), q-major; each team owns a contiguous
+// range of items and processes two rows per step (gate and up of each).
 template <int TL, int KCH>
 __global__ void __launch_bounds__(kGemvThreads, 1)
 gateup_decode_kernel(const GateUpParams p) {
-    extern __shared__ __align__(16) uint32_t sx[];  // [T][H/2] FP16 words
-    __shared__ int s_c[kDecodeMaxT];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int H = p.H, I = p.I, k = p.k, T = p.T;
-    const int C = H >> 5, hw = H >> 1;
+    constexpr int TPW = 32 / TL;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lt = lane & (TL - 1);
+    const unsigned mask = team_mask<TL>(lane);
+    const int H = p.H, I = p.I, k = p.k;
+    const int C = H >> 5;
+    const size_t rc = (size_t)H >> 1, rs = (size_t)H >> 5;  // bytes per row: codes, scales
 
     pdl_wait();  // x and ids come from earlier kernels
     pdl_launch_dependents();
+    if (p.prefetch_down && warp == kGemvWarps - 1) prefetch_down_slice(p, lane);
 
-    if (p.prefetch_down && tid == 0) prefetch_down_share(p);
+    const long long N = (long long)p.T * k * I;
+    const long long nteams = (long long)gridDim.x * kGemvWarps * TPW;
+    const long long team = ((long long)blockIdx.x * kGemvWarps + warp) * TPW + (lane / TL);
+    long long it = N * team / nteams;
+    const long long end = N * (team + 1) / nteams;
 
-    for (int t = warp; t < T; t += kGemvWarps) {
-        int c = stage_f16_warp(p.x + (size_t)t * H, H, sx + (size_t)t * hw, lane);
-        if (lane == 0) s_c[t] = c;
-    }
-    __syncthreads();
+    uint32_t xw[KCH][16];
+    int cur_tok = -1, cur_q = -1;
+    float xs = 1.f;
+    bool bad = false;
+    const uint8_t *gc = nullptr, *gs = nullptr, *uc = nullptr, *us = nullptr;
 
-    // items (pair q = t*k + j, row i), q-major; each warp owns a contiguous
-    // range, its 32/TL teams take items round-robin, two at a time.
-    constexpr int TPW = 32 / TL;
-    const int lt = lane % TL, tw = lane / TL;
-    const long long N = (long long)T * k * I;
-    const long long gw = (long long)blockIdx.x * kGemvWarps + warp;
-    const long long GW = (long long)gridDim.x * kGemvWarps;
-    const long long wb = N * gw / GW, we = N * (gw + 1) / GW;
-
-    for (long long base = wb; base < we; base += 2 * TPW) {
-        long long item[2] = {base + tw, base + TPW + tw};
+    while (it < end) {
+        const int q = (int)(it / I);
+        const int row = (int)(it - (long long)q * I);
+        // a second row of the same pair in this step if there is one
+        const bool two = (it + 1 < end) && (row + 1 < I);
+        if (q != cur_q) {
+            const int e = p.ids[q];
+            bad = (e < 0 || e >= p.E);
+            if (!bad) {
+                const ExpertPtrs *ep = p.table + e;
+                gc = ep->codes[0];
+                gs = ep->scales[0];
+                uc = ep->codes[1];
+                us = ep->scales[1];
+            }
+            cur_q = q;
+        }
         uint4 cg[2][KCH], cu[2][KCH];
         uint32_t sg[2][KCH], su[2][KCH];
-        int q[2], row[2], tok[2];
-        bool valid[2], bad[2];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-            valid[u] = item[u] < we;
-            q[u] = valid[u] ? (int)(item[u] / I) : 0;
-            row[u] = valid[u] ? (int)(item[u] - (long long)q[u] * I) : 0;
-            tok[u] = q[u] / k;
-            int e = valid[u] ? p.ids[q[u]] : 0;
-            bad[u] = valid[u] && (e < 0 || e >= p.E);
-            const bool ok = valid[u] && !bad[u];
-            const uint8_t *gc = nullptr, *gs = nullptr, *uc = nullptr, *us = nullptr;
-            if (ok) {
-                const ExpertPtrs *ep = p.table + e;
-                gc = ep->codes[0] + (size_t)row[u] * (H >> 1);
-                gs = ep->scales[0] + (size_t)row[u] * (H >> 5);
-                uc = ep->codes[1] + (size_t)row[u] * (H >> 1);
-                us = ep->scales[1] + (size_t)row[u] * (H >> 5);
-            }
-            load_row<TL, KCH>(gc, gs, ok, lt, C, cg[u], sg[u]);
-            load_row<TL, KCH>(uc, us, ok, lt, C, cu[u], su[u]);
+            const bool ok = !bad && (u == 0 || two);
+            const size_t r = (size_t)(row + u);
+            load_chunks<KCH>(gc + r * rc, gs + r * rs, ok, lt, C, cg[u], sg[u]);
+            load_chunks<KCH>(uc + r * rc, us + r * rs, ok, lt, C, cu[u], su[u]);
         }
+        const int tok = q / k;
+        if (tok != cur_tok) {
+            xs = pow2(stage_x<TL, KCH>(p.x + (size_t)tok * H, lt, C, mask, xw));
+            cur_tok = tok;
+        }
+        float v[4];
+        v[0] = chunks_dot<KCH>(cg[0], sg[0], xw);
+        v[1] = chunks_dot<KCH>(cu[0], su[0], xw);
+        v[2] = chunks_dot<KCH>(cg[1], sg[1], xw);
+        v[3] = chunks_dot<KCH>(cu[1], su[1], xw);
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const uint32_t *xw = sx + (size_t)tok[u] * hw;
-            float ag = row_partial<TL, KCH>(cg[u], sg[u], xw, lt, C);
-            float au = row_partial<TL, KCH>(cu[u], su[u], xw, lt, C);
-            ag = team_sum<TL>(ag);
-            au = team_sum<TL>(au);
-            if (lt == 0 && valid[u]) {
-                uint16_t out = 0;
-                if (!bad[u]) {
-                    const int c = s_c[tok[u]];
-                    const float g = round_bf16(scalbnf(ag, c));
-                    const float uu = round_bf16(scalbnf(au, c));
-                    const float s = round_bf16(g / (1.0f + expf(-g)));
-                    out = f32_to_bf16(s * uu);
-                } else {
-                    atomicOr(p.status, kBadExpertId);
-                }
-                p.h[(size_t)q[u] * I + row[u]] = out;
+        for (int i = 0; i < 4; ++i) v[i] = team_add<TL>(v[i], mask);
+        if (lt < 2 && (lt == 0 || two)) {
+            const float ag = lt == 0 ? v[0] : v[2];
+            const float au = lt == 0 ? v[1] : v[3];
+            uint16_t out = 0;
+            if (!bad) {
+                const float g = round_bf16(ag * xs);
+                const float uu = round_bf16(au * xs);
+                const float s = round_bf16(g / (1.0f + expf(-g)));
+                out = f32_to_bf16(s * uu);
+            } else if (lt == 0) {
+                atomicOr(p.status, kBadExpertId);
             }
+            p.h[(size_t)q * I + row + lt] = out;
         }
+        it += two ? 2 : 1;
     }
 }
 
 // ---------------------------------------------------------------- down -----
+// CTA = a range of output rows (t, n) for every slot j; the warps of slot
+// group j stream the down rows of expert ids[t][j]; the combine runs in
+// shared memory after one barrier.  The first rows' weights are requested
+// before the programmatic-launch wait (the routing is final by then: the
+// gate/up kernel released this grid only after its own wait).
 
 template <int TL, int KCH>
-__global__ void __launch_bounds__(kGemvThreads, 1)
+__global__ void __launch_bounds__(kDownThreads, 1)
 down_decode_kernel(const DownParams p) {
-    extern __shared__ __align__(16) uint32_t sd[];
-    __shared__ int s_c[kDecodeMaxT * kMaxTopK];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    extern __shared__ __align__(16) float so[];  // [k][R]
+    constexpr int TPW = 32 / TL;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lt = lane & (TL - 1);
+    const unsigned mask = team_mask<TL>(lane);
     const int H = p.H, I = p.I, k = p.k, T = p.T;
-    const int P = T * k, C = I >> 5, iw = I >> 1;
+    const int C = I >> 5;
+    const size_t rc = (size_t)I >> 1, rs = (size_t)I >> 5;
     const int R = p.rows_per_cta;
-    uint32_t *sh = sd;                                    // [P][I/2] FP16 words
-    float *so = reinterpret_cast<float *>(sd + (size_t)P * iw);  // [k][R]
+    const int r0 = blockIdx.x * R;
+    const int r1 = min(r0 + R, T * H);
+
+    const int groups = kDownWarps / k;  // warps per slot
+    const int j = warp % k, gi = warp / k;
+    const int tps = groups * TPW;       // teams per slot
+    const int ti = gi * TPW + lane / TL;
+    const bool worker = gi < groups;
+
+    // rows of this team: r0 + ti, r0 + ti + tps, ...; two per step
+    int rr = r0 + ti;
+    uint4 cw[2][KCH];
+    uint32_t sc[2][KCH];
+    bool bad[2] = {false, false};
+    auto fetch = [&](int rbase) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int r = rbase + u * tps;
+            const bool valid = worker && r < r1;
+            const int t = valid ? r / H : 0;
+            const int n = r - t * H;
+            const int e = valid ? p.ids[t * k + j] : 0;
+            bad[u] = valid && (e < 0 || e >= p.E);
+            const bool ok = valid && !bad[u];
+            const uint8_t *dc = nullptr, *ds = nullptr;
+            if (ok) {
+                dc = p.table[e].codes[2] + (size_t)n * rc;
+                ds = p.table[e].scales[2] + (size_t)n * rs;
+            }
+            load_chunks<KCH>(dc, ds, ok, lt, C, cw[u], sc[u]);
+        }
+    };
+    fetch(rr);
 
     pdl_wait();  // h comes from the gate/up kernel
     pdl_launch_dependents();
 
-    for (int q = warp; q < P; q += kGemvWarps) {
-        int c = stage_f16_warp(p.h + (size_t)q * I, I, sh + (size_t)q * iw, lane);
-        if (lane == 0) s_c[q] = c;
-    }
-    __syncthreads();
-
-    const int r0 = blockIdx.x * R;
-    const int r1 = min(r0 + R, T * H);
-    constexpr int TPW = 32 / TL;
-    const int groups = kGemvWarps / k;  // warps per slot
-    const int j = warp % k, gi = warp / k;
-    const int lt = lane % TL, tw = lane / TL;
-    const int tps = groups * TPW;       // teams per slot
-    const int ti = gi * TPW + tw;
-
-    if (gi < groups && r0 < r1) {
-        for (int base = r0; base < r1; base += 2 * tps) {
-            int rr[2] = {base + ti, base + tps + ti};
-            uint4 cw[2][KCH];
-            uint32_t sc[2][KCH];
-            int qq[2];
-            bool valid[2], bad[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                valid[u] = rr[u] < r1;
-                const int t = valid[u] ? rr[u] / H : 0;
-                const int n = rr[u] - t * H;
-                qq[u] = t * k + j;
-                const int e = valid[u] ? p.ids[qq[u]] : 0;
-                bad[u] = valid[u] && (e < 0 || e >= p.E);
-                const bool ok = valid[u] && !bad[u];
-                const uint8_t *dc = nullptr, *ds = nullptr;
-                if (ok) {
-                    const ExpertPtrs *ep = p.table + e;
-                    dc = ep->codes[2] + (size_t)n * (I >> 1);
-                    ds = ep->scales[2] + (size_t)n * (I >> 5);
-                }
-                load_row<TL, KCH>(dc, ds, ok, lt, C, cw[u], sc[u]);
-            }
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                float a = row_partial<TL, KCH>(cw[u], sc[u], sh + (size_t)qq[u] * iw, lt, C);
-                a = team_sum<TL>(a);
-                if (lt == 0 && valid[u]) {
-                    float o = 0.f;
-                    if (!bad[u])
-                        o = round_bf16(scalbnf(a, s_c[qq[u]]));
-                    else
-                        atomicOr(p.status, kBadExpertId);
-                    so[j * R + (rr[u] - r0)] = o;
-                }
+    uint32_t xw[KCH][16];
+    int cur_tok = -1;
+    float xs = 1.f;
+    while (worker && rr < r1) {
+        const int t = rr / H;
+        if (t != cur_tok) {
+            xs = pow2(stage_x<TL, KCH>(p.h + ((size_t)t * k + j) * I, lt, C, mask, xw));
+            cur_tok = t;
+        }
+        // both rows of a step belong to token t unless the second crosses into
+        // the next token; then it is recomputed in the next step
+        const int rb = rr + tps;
+        const bool second = rb < r1 && rb / H == t;
+        float a0 = chunks_dot<KCH>(cw[0], sc[0], xw);
+        float a1 = chunks_dot<KCH>(cw[1], sc[1], xw);
+        a0 = team_add<TL>(a0, mask);
+        a1 = team_add<TL>(a1, mask);
+        const bool b0 = bad[0], b1 = bad[1];
+        const int rnext = second ? rr + 2 * tps : rr + tps;
+        if (rnext < r1) fetch(rnext);
+        if (lt == 0) {
+            so[j * R + (rr - r0)] = b0 ? 0.f : round_bf16(a0 * xs);
+            if (b0) atomicOr(p.status, kBadExpertId);
+            if (second) {
+                so[j * R + (rb - r0)] = b1 ? 0.f : round_bf16(a1 * xs);
+                if (b1) atomicOr(p.status, kBadExpertId);
             }
         }
+        rr = rnext;
     }
     __syncthreads();
 
     // sequential BF16 combine in slot order, optional residual add
-    for (int r = r0 + tid; r < r1; r += kGemvThreads) {
+    for (int r = r0 + threadIdx.x; r < r1; r += kDownThreads) {
         const int t = r / H, n = r - t * H;
         float y = 0.f;
         for (int jj = 0; jj < k; ++jj) {
@@ -475,24 +550,17 @@ void pick_team(int C, int &TL, int &KCH) {
     KCH = (C + 31) / 32;
 }
 
-constexpr size_t kMaxSmem = kMaxDecodeSmem;
 
 template <int TL, int KCH>
 cudaError_t launch_gu(const GateUpParams &p, int grid, cudaStream_t s, bool pdl) {
-    auto kern = gateup_decode_kernel<TL, KCH>;
-    size_t smem = gateup_decode_smem(p.T, p.H);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxSmem);
-    if (e != cudaSuccess) return e;
-    return launch_ex(kern, dim3(grid), dim3(kGemvThreads), smem, s, pdl, p);
+    return launch_ex(gateup_decode_kernel<TL, KCH>, dim3(grid), dim3(kGemvThreads), 0, s, pdl, p);
 }
 
 template <int TL, int KCH>
 cudaError_t launch_dn(const DownParams &p, int grid, cudaStream_t s, bool pdl) {
-    auto kern = down_decode_kernel<TL, KCH>;
-    size_t smem = down_decode_smem(p.T, p.k, p.I, p.rows_per_cta);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxSmem);
-    if (e != cudaSuccess) return e;
-    return launch_ex(kern, dim3(grid), dim3(kGemvThreads), smem, s, pdl, p);
+    const size_t smem = down_decode_smem(p.T, p.k, p.I, p.rows_per_cta);
+    if (smem > 48 * 1024) return cudaErrorInvalidValue;
+    return launch_ex(down_decode_kernel<TL, KCH>, dim3(grid), dim3(kDownThreads), smem, s, pdl, p);
 }
 
 #define MOE_TEAM_DISPATCH(FN, C, ...)                                   \
@@ -530,20 +598,15 @@ bool decode_shape_supported(int H, int I) {
     return kch <= 4;
 }
 
-size_t gateup_decode_smem(int T, int H) { return (size_t)T * H * 2; }
+size_t gateup_decode_smem(int, int) { return 0; }
 
-size_t down_decode_smem(int T, int k, int I, int rows_per_cta) {
-    return (size_t)T * k * I * 2 + (size_t)k * rows_per_cta * 4;
+size_t down_decode_smem(int, int k, int, int rows_per_cta) {
+    return (size_t)k * rows_per_cta * 4;
 }
 
 cudaError_t launch_route(const RouteParams &p, cudaStream_t s, bool pdl) {
-    const int wpb = kRouteThreads / 32;
-    const int nblk = (p.E + wpb - 1) / wpb;
-    size_t smem = (size_t)p.H * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kMaxSmem);
-    if (e != cudaSuccess) return e;
-    return launch_ex(route_kernel, dim3(nblk, p.T), dim3(kRouteThreads), smem, s, pdl, p);
+    const int tblocks = (p.T + kRouteWarps - 1) / kRouteWarps;
+    return launch_ex(route_kernel, dim3(p.E, tblocks), dim3(kRouteThreads), 0, s, pdl, p);
 }
 
 cudaError_t launch_gateup_decode(const GateUpParams &p, int grid, cudaStream_t s, bool pdl) {

@@ -10,7 +10,8 @@ namespace moe {
 
 constexpr int kDecodeMaxT = 4;      // tokens handled by the per-(token,slot) GEMV path
 constexpr int kMaxTopK = 8;
-constexpr int kGemvThreads = 512;   // 16 warps, one CTA per SM
+constexpr int kGemvThreads = 512;   // gate/up GEMV: 16 warps, one CTA per SM
+constexpr int kDownThreads = 384;   // down GEMV + combine: 12 warps, one CTA per SM
 constexpr int kRouteThreads = 256;  // 8 warps, one expert row per warp
 constexpr unsigned kBadExpertId = 0x1u;
 constexpr size_t kMaxDecodeSmem = 200 * 1024;  // dynamic shared memory cap of the GEMVs
@@ -38,6 +39,7 @@ struct GateUpParams {
     unsigned *status;
     int T, k, E, H, I;
     int prefetch_down;        // L2-prefetch the selected down matrices
+    uint32_t pf_codes, pf_scales;  // per-CTA prefetch slice (bytes, multiple of 16)
 };
 
 struct DownParams {

@@ -31,18 +31,36 @@ def f64(u16):
     return oracle.bf16_to_f64_array(u16)
 
 
-def assert_close_rms(gpu_u16, ref_u16, tol=TOL, what=""):
-    """Per vector (last axis): max|gpu - ref| <= tol * rms(ref).  Returns the
-    number of elements that differ at all (BF16 rounding flips)."""
-    g = f64(gpu_u16).reshape(-1, np.shape(ref_u16)[-1])
-    r = f64(ref_u16).reshape(g.shape)
+def ulp_distance(a_u16, b_u16):
+    """Number of BF16 values between a and b (0 = equal, 1 = adjacent)."""
+    def ordinal(u):
+        u = np.asarray(u, dtype=np.int64)
+        return np.where(u & 0x8000, -(u & 0x7FFF), u)
+    return np.abs(ordinal(a_u16) - ordinal(b_u16))
+
+
+def assert_close_rms(gpu_u16, ref_u16, tol=TOL, what="", max_ulps=1, max_flip_frac=0.01):
+    """Per vector (last axis): every element within tol * rms(ref) of the
+    oracle, except rounding flips: elements where the GPU (FP32 accumulation)
+    and the oracle (FP64) land on BF16 values at most `max_ulps` apart because
+    the exact value sits near a BF16 rounding midpoint.  One BF16 ulp exceeds
+    1e-2 * rms for any element above ~1.28 * rms, so such flips are allowed,
+    counted, and must stay rare (<= max_flip_frac of the elements).
+    Returns (flips, elements that differ at all)."""
+    gpu_u16 = np.asarray(gpu_u16).reshape(-1, np.shape(ref_u16)[-1])
+    ref_u16 = np.asarray(ref_u16).reshape(gpu_u16.shape)
+    g, r = f64(gpu_u16), f64(ref_u16)
     assert np.all(np.isfinite(g)) and np.all(np.isfinite(r)), what
-    rms = np.sqrt(np.mean(r * r, axis=1))
-    err = np.max(np.abs(g - r), axis=1)
-    bad = err > tol * rms
-    assert not np.any(bad), (f"{what}: max err {err[bad].max():.3e} vs rms "
-                             f"{rms[bad].min():.3e} in {bad.sum()} vectors")
-    return int(np.count_nonzero(g != r))
+    rms = np.sqrt(np.mean(r * r, axis=1, keepdims=True))
+    err = np.abs(g - r)
+    within = err <= tol * rms
+    ulps = ulp_distance(gpu_u16, ref_u16)
+    flip = (~within) & (ulps <= max_ulps)
+    bad = (~within) & ~flip
+    assert not np.any(bad), (f"{what}: {bad.sum()} elements beyond tolerance, worst "
+                             f"{(err / rms)[bad].max():.3e} x rms, {ulps[bad].max()} ulps")
+    assert flip.mean() <= max_flip_frac, f"{what}: flip fraction {flip.mean():.4f}"
+    return int(flip.sum()), int(np.count_nonzero(g != r))
 
 
 def near_tie_tokens(logits: np.ndarray, k: int, rel=1e-4):

@@ -92,7 +92,7 @@ def _forward_checks(L, x, layer, ids, w, T, shape):
                                        shape.I, want_o=True, want_h=True)
     assert_close_rms(h_g, h_r, what="h")
     assert_close_rms(o_g, o_r, what="o")
-    assert_close_rms(y_g, y_r, what="y")
+    assert_close_rms(y_g, y_r, what="y", max_ulps=2)
     # the combine is bit-exact given the kernel's own expert outputs
     for t in range(T):
         np.testing.assert_array_equal(y_g[t], oracle.combine(o_g[t], w_h[t]))
@@ -130,7 +130,7 @@ def test_layer_end_to_end(shape, T):
         if ties == 0:
             _, _, y_r = oracle.moe_layer(x, L.router_w, L.router_b, L.codes, L.scales, shape.E,
                                          shape.H, shape.I, shape.top_k)
-            assert_close_rms(host_bf16(y), y_r, what="layer y")
+            assert_close_rms(host_bf16(y), y_r, what="layer y", max_ulps=2)
         layer.close()
 
 
@@ -171,7 +171,7 @@ def test_invalid_ids_zero_the_slot_and_flag():
     assert layer.status() == 0  # cleared by the read
     y_r = oracle.moe_forward(x, ids_h, w_h.astype(np.float64), L.codes, L.scales, shape.E,
                              shape.H, shape.I)
-    assert_close_rms(host_bf16(y), y_r, what="y with invalid ids")
+    assert_close_rms(host_bf16(y), y_r, what="y with invalid ids", max_ulps=2)
     layer.close()
 
 
@@ -200,7 +200,7 @@ def test_residual_fused_add():
                       y=rd, residual=rd)  # in place
     y_r = oracle.moe_forward(x, ids_h, w_h.astype(np.float64), L.codes, L.scales, shape.E,
                              shape.H, shape.I, residual=r)
-    assert_close_rms(host_bf16(y), y_r, what="residual y")
+    assert_close_rms(host_bf16(y), y_r, what="residual y", max_ulps=2)
     layer.close()
 
 

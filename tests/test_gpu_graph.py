@@ -94,7 +94,7 @@ def test_stack_per_layer_parity_and_graph(shape, n_layers, bias):
         w_g = st.w[l].cpu().numpy().astype(np.float64)
         r_out_ref = oracle.moe_forward(xn_g, ids_g, w_g, L.codes, L.scales, shape.E, shape.H,
                                        shape.I, residual=r_in)
-        assert_close_rms(host_bf16(st.r), r_out_ref, what=f"layer {l} residual out")
+        assert_close_rms(host_bf16(st.r), r_out_ref, what=f"layer {l} residual out", max_ulps=2)
     r_eager = host_bf16(st.r).copy()
 
     # the captured step replays to the same bits
