@@ -218,6 +218,43 @@ MOE_API int moe_bytes_per_expert(moe_handle_t h, size_t *bytes);
  * while it streams gate/up.  Errors: ARG. */
 MOE_API int moe_set_tuning(moe_handle_t h, int use_pdl, int prefetch_down);
 
+/* ---------------------------------------------------------------------
+ * Forward without any device allocation.  No counterpart in the paper: this
+ * entry point exists for callers that may not call cudaMalloc -- code that
+ * runs inside another framework's memory pool or allocator callback, hosts
+ * whose device memory is budgeted and accounted elsewhere, or paths that
+ * must not allocate while other streams are being captured.  It computes
+ * exactly what moe_create + moe_load_packed + moe_set_workspace +
+ * moe_forward_ex(residual) compute, with the same kernels, but without a
+ * handle: its scratch (expert table, status word, SwiGLU activations h)
+ * lives in one file-scope device array of MOE_NOALLOC_SCRATCH_BYTES bytes
+ * that every GPU loading this library holds until the process exits.
+ *
+ * Limits (beyond them the call returns MOE_ERR_WORKSPACE and enqueues
+ * nothing): E <= MOE_NOALLOC_MAX_EXPERTS and T * top_k * I * 2 <=
+ * MOE_NOALLOC_MAX_H_BYTES.  Shapes as for moe_create.
+ * Arguments: codes_u8 / scales_e8m0 as for moe_load_packed (device,
+ * contiguous [E][3][...], 16-byte aligned, read in place); x, topk_ids,
+ * topk_w, residual (or NULL; may alias y), y as for moe_forward_ex.  These
+ * pointers are not checked to be device memory (that check would itself be
+ * a runtime call per pointer); they must be.
+ * The first call on a device (with that device current) looks up the
+ * scratch's device address with cudaGetSymbolAddress; make that first call
+ * before any stream capture.  Every call rewrites the shared scratch (the
+ * expert table by a cudaMemcpyAsync from the host stack, the status word by
+ * a cudaMemsetAsync) on `stream`: calls that overlap on the GPU (different
+ * streams, or different threads without ordering) race on it.
+ * Errors: ARG, ALIGN, WORKSPACE, UNSUPPORTED, CUDA. */
+#define MOE_NOALLOC_MAX_EXPERTS 256
+#define MOE_NOALLOC_MAX_H_BYTES (512u * 1024u)
+#define MOE_NOALLOC_SCRATCH_BYTES (12288u + 256u + MOE_NOALLOC_MAX_H_BYTES)
+MOE_API int moe_forward_noalloc(int E, int H, int I, int top_k,
+                                const uint8_t *codes_u8,
+                                const uint8_t *scales_e8m0, const uint16_t *x,
+                                int T, const int32_t *topk_ids,
+                                const float *topk_w, const uint16_t *residual,
+                                uint16_t *y, void *stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 MOE_API const char *moe_status_string(int status);
 

@@ -26,6 +26,7 @@ __all__ = [
     "moe_workspace_bytes", "moe_set_workspace", "moe_route", "moe_route_ex",
     "moe_forward", "moe_forward_ex", "moe_get_intermediates", "moe_get_status",
     "moe_bytes_per_expert", "moe_set_tuning", "moe_device_check", "moe_debug_dequant",
+    "moe_forward_noalloc",
     "ROUTE_RMSNORM", "FWD_KEEP_INTERMEDIATES", "FWD_FORCE_DECODE", "FWD_FORCE_GROUPED",
     "FWD_PHASE_GATEUP", "FWD_PHASE_DOWN",
     "DEVICE_BAD_EXPERT_ID",
@@ -163,6 +164,23 @@ def moe_debug_dequant(codes, scales, n, out, stream=None) -> None:
     _need(scales, torch.uint8, "moe_debug_dequant")
     _need(out, torch.float32, "moe_debug_dequant")
     check("moe_debug_dequant", load().moe_debug_dequant(_p(codes), _p(scales), n, _p(out), _s(stream)))
+
+
+def moe_forward_noalloc(E, H, I, top_k, codes, scales, x, topk_ids, topk_w, residual, y,
+                        stream=None) -> None:
+    """Expert FFN + combine for callers that may not allocate device memory:
+    no handle, no workspace; scratch lives in a fixed device array inside the
+    library (see include/moe_mxfp4.h for its limits and its sharing rules)."""
+    _need(codes, torch.uint8, "moe_forward_noalloc")
+    _need(scales, torch.uint8, "moe_forward_noalloc")
+    _need(x, torch.bfloat16, "moe_forward_noalloc", 2)
+    _need(topk_ids, torch.int32, "moe_forward_noalloc")
+    _need(topk_w, torch.float32, "moe_forward_noalloc")
+    _need(residual, torch.bfloat16, "moe_forward_noalloc")
+    _need(y, torch.bfloat16, "moe_forward_noalloc")
+    check("moe_forward_noalloc", load().moe_forward_noalloc(
+        E, H, I, top_k, _p(codes), _p(scales), _p(x), x.shape[0], _p(topk_ids), _p(topk_w),
+        _p(residual), _p(y), _s(stream)))
 
 
 # ------------------------------------------------------------- bundles

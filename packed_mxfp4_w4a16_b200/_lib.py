@@ -39,6 +39,7 @@ SIGNATURES = [
     ("moe_status_string", C.c_char_p, [_i]),
     ("moe_device_check", _i, []),
     ("moe_debug_dequant", _i, [_vp, _vp, _i64, _vp, _vp]),
+    ("moe_forward_noalloc", _i, [_i, _i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp]),
 ]
 
 
