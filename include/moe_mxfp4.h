@@ -90,6 +90,8 @@ typedef enum moe_status {
 
 /* Bits of the device status word read by moe_get_status. */
 #define MOE_DEVICE_BAD_EXPERT_ID 0x1u /* an id outside [0, E): slot zeroed */
+#define MOE_DEVICE_TIMEOUT 0x2u       /* a bounded in-kernel wait gave up;
+                                         outputs of that call are invalid */
 
 /* Flags of moe_route_ex. */
 #define MOE_ROUTE_RMSNORM 0x1u /* x is a residual stream r: route
@@ -194,6 +196,25 @@ MOE_API int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T,
                    const int32_t *topk_ids, const float *topk_w,
                    const uint16_t *residual, uint16_t *y, unsigned flags,
                    void *stream);
+
+/* One whole layer: routing + expert FFN + combine, with the routing computed
+ * inside the expert kernels (no separate top-k launch, no id round trip):
+ *   - route_flags MOE_ROUTE_RMSNORM: x is a residual stream r; the layer
+ *     routes and runs the experts on xn = BF16(r / sqrt(mean(r^2) + 1e-6)),
+ *     written to x_norm (device BF16 [T][H], distinct from x and y).
+ *   - logits (device FP32 [T][E] or NULL) receives the (biased) logits;
+ *     topk_ids / topk_w (device [T][k] or NULL) receive the routing.
+ *   - residual (or NULL; may alias y and x) is added as in moe_forward_ex;
+ *     fwd_flags may hold MOE_FWD_KEEP_INTERMEDIATES.
+ * Results equal moe_route_ex followed by moe_forward_ex.  For T > 4 the
+ * call runs exactly that sequence and then topk_ids / topk_w are required.
+ * Errors: as moe_route_ex and moe_forward_ex. */
+MOE_API int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T,
+                         const uint16_t *router_w, const float *router_bias,
+                         unsigned route_flags, uint16_t *x_norm, float *logits,
+                         int32_t *topk_ids, float *topk_w,
+                         const uint16_t *residual, uint16_t *y,
+                         unsigned fwd_flags, void *stream);
 
 /* Device pointers to the intermediates kept by the last moe_forward_ex with
  * MOE_FWD_KEEP_INTERMEDIATES: h BF16 [T][k][I] (SwiGLU outputs) and o BF16

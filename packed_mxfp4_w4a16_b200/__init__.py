@@ -24,7 +24,7 @@ __all__ = [
     "MoEError", "MoELayer", "MoEStack", "library_path", "load",
     "moe_create", "moe_destroy", "moe_load_packed", "moe_load_expert_table",
     "moe_workspace_bytes", "moe_set_workspace", "moe_route", "moe_route_ex",
-    "moe_forward", "moe_forward_ex", "moe_get_intermediates", "moe_get_status",
+    "moe_forward", "moe_forward_ex", "moe_layer_ex", "moe_get_intermediates", "moe_get_status",
     "moe_bytes_per_expert", "moe_set_tuning", "moe_device_check", "moe_debug_dequant",
     "moe_forward_noalloc",
     "ROUTE_RMSNORM", "FWD_KEEP_INTERMEDIATES", "FWD_FORCE_DECODE", "FWD_FORCE_GROUPED",
@@ -39,6 +39,7 @@ FWD_FORCE_GROUPED = 0x4
 FWD_PHASE_GATEUP = 0x8
 FWD_PHASE_DOWN = 0x10
 DEVICE_BAD_EXPERT_ID = 0x1
+DEVICE_TIMEOUT = 0x2
 
 
 def _p(t):
@@ -128,6 +129,23 @@ def moe_forward_ex(h, x, topk_ids, topk_w, residual, y, flags, stream=None) -> N
     check("moe_forward", load().moe_forward_ex(
         C.c_void_p(h), _p(x), x.shape[0], _p(topk_ids), _p(topk_w), _p(residual), _p(y),
         flags, _s(stream)))
+
+
+def moe_layer_ex(h, x, router_w, router_bias, route_flags, x_norm, logits, topk_ids, topk_w,
+                 residual, y, fwd_flags, stream=None) -> None:
+    _need(x, torch.bfloat16, "moe_layer_ex", 2)
+    _need(router_w, torch.bfloat16, "moe_layer_ex", 2)
+    _need(router_bias, torch.float32, "moe_layer_ex")
+    _need(x_norm, torch.bfloat16, "moe_layer_ex")
+    _need(logits, torch.float32, "moe_layer_ex")
+    _need(topk_ids, torch.int32, "moe_layer_ex")
+    _need(topk_w, torch.float32, "moe_layer_ex")
+    _need(residual, torch.bfloat16, "moe_layer_ex")
+    _need(y, torch.bfloat16, "moe_layer_ex")
+    check("moe_layer_ex", load().moe_layer_ex(
+        C.c_void_p(h), _p(x), x.shape[0], _p(router_w), _p(router_bias), route_flags,
+        _p(x_norm), _p(logits), _p(topk_ids), _p(topk_w), _p(residual), _p(y), fwd_flags,
+        _s(stream)))
 
 
 def moe_get_intermediates(h: int):
@@ -291,9 +309,8 @@ class MoEStack:
     def enqueue(self, stream=None):
         """Enqueue one decode step (all layers) on `stream`."""
         for l, L in enumerate(self.layers):
-            moe_route_ex(L.handle, self.r, L.router_w, L.router_b, ROUTE_RMSNORM, self.xn, None,
-                         self.ids[l], self.w[l], stream)
-            moe_forward_ex(L.handle, self.xn, self.ids[l], self.w[l], self.r, self.r, 0, stream)
+            moe_layer_ex(L.handle, self.r, L.router_w, L.router_b, ROUTE_RMSNORM, self.xn, None,
+                         self.ids[l], self.w[l], self.r, self.r, 0, stream)
 
     def capture(self):
         """Capture one decode step into a CUDA graph (warm-up run first)."""

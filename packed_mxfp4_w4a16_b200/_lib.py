@@ -32,6 +32,7 @@ SIGNATURES = [
     ("moe_route_ex", _i, [_vp, _vp, _i, _vp, _vp, _u, _vp, _vp, _vp, _vp, _vp]),
     ("moe_forward", _i, [_vp, _vp, _i, _vp, _vp, _vp, _vp]),
     ("moe_forward_ex", _i, [_vp, _vp, _i, _vp, _vp, _vp, _vp, _u, _vp]),
+    ("moe_layer_ex", _i, [_vp, _vp, _i, _vp, _vp, _u, _vp, _vp, _vp, _vp, _vp, _vp, _u, _vp]),
     ("moe_get_intermediates", _i, [_vp, C.POINTER(_vp), C.POINTER(_vp)]),
     ("moe_get_status", _i, [_vp, C.POINTER(_u)]),
     ("moe_bytes_per_expert", _i, [_vp, C.POINTER(_sz)]),

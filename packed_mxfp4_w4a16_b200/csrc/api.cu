@@ -31,6 +31,8 @@ struct moe_ctx {
     bool kept = false;                    // last forward kept intermediates
     bool use_pdl = true;
     bool prefetch_down = true;
+    const uint8_t *codes_base = nullptr;   // set by moe_load_packed (contiguous layout)
+    const uint8_t *scales_base = nullptr;
 };
 
 namespace {
@@ -38,7 +40,7 @@ namespace {
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct WsLayout {
-    size_t counters, logits, h, o, total;
+    size_t counters, logits, h, o, x16, x16_exp, total;
 };
 
 WsLayout ws_layout(const moe_ctx *c, int maxT) {
@@ -53,6 +55,8 @@ WsLayout ws_layout(const moe_ctx *c, int maxT) {
     L.logits = take((size_t)maxT * c->E * sizeof(float));
     L.h = take((size_t)maxT * c->k * c->I * 2);
     L.o = take((size_t)maxT * c->k * c->H * 2);
+    L.x16 = take((size_t)maxT * c->H * 2);
+    L.x16_exp = take((size_t)maxT * sizeof(int));
     L.total = off;
     return L;
 }
@@ -175,6 +179,10 @@ int moe_load_packed(moe_handle_t h, const uint8_t *codes_u8, const uint8_t *scal
         }
     rc = upload_table(h, t);
     delete[] t;
+    if (rc == MOE_OK) {
+        h->codes_base = codes_u8;
+        h->scales_base = scales_e8m0;
+    }
     return rc;
 }
 
@@ -195,6 +203,7 @@ int moe_load_expert_table(moe_handle_t h, const uint8_t *const *codes_ptrs,
         }
     if (rc == MOE_OK) rc = upload_table(h, t);
     delete[] t;
+    if (rc == MOE_OK) h->codes_base = h->scales_base = nullptr;
     return rc;
 }
 
@@ -252,6 +261,8 @@ int moe_route_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
     p.k = h->k;
     p.rmsnorm = norm ? 1 : 0;
     p.eps = 1e-6f;
+    p.x16 = nullptr;
+    p.x16_exp = nullptr;
     return cuda_rc(moe::launch_route(p, static_cast<cudaStream_t>(stream), h->use_pdl));
 }
 
@@ -292,20 +303,30 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
     // per-(token, slot) GEMV path, in chunks of up to kDecodeMaxT tokens (fewer
     // when the staged activations of a chunk would not fit in shared memory)
     int chunk = moe::kDecodeMaxT;
-    while (chunk > 1 && (moe::gateup_decode_smem(chunk, h->H) > moe::kMaxDecodeSmem ||
+    while (chunk > 1 && (moe::gateup_decode_smem(chunk, h->H) > moe::kDownSmemMax ||
                          moe::down_decode_smem(chunk, h->k, h->I,
                                                (chunk * h->H + h->num_sms - 1) / h->num_sms) >
-                             moe::kMaxDecodeSmem))
+                             moe::kDownSmemMax))
         --chunk;
     if (moe::down_decode_smem(1, h->k, h->I, (h->H + h->num_sms - 1) / h->num_sms) >
-        moe::kMaxDecodeSmem)
+        moe::kDownSmemMax)
         return MOE_ERR_ARG;
     for (int t0 = 0; t0 < T; t0 += chunk) {
         const int Tc = (T - t0 < chunk) ? T - t0 : chunk;
         moe::GateUpParams g;
         g.table = h->d_table;
+        g.codes_base = h->codes_base;
+        g.scales_base = h->scales_base;
+        g.codes_stride = (size_t)h->I * h->H / 2;
+        g.scales_stride = (size_t)h->I * h->H / 32;
         g.x = x + (size_t)t0 * h->H;
+        g.x16 = nullptr;
+        g.x16_exp = nullptr;
         g.ids = topk_ids + (size_t)t0 * h->k;
+        g.logits = nullptr;
+        g.ids_out = nullptr;
+        g.w_out = nullptr;
+        g.nslots = moe::gateup_tma_slots(h->H);
         g.h = hbuf + (size_t)t0 * h->k * h->I;
         g.status = h->d_status;
         g.T = Tc;
@@ -326,9 +347,14 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
 
         moe::DownParams d;
         d.table = h->d_table;
+        d.codes_base = h->codes_base;
+        d.scales_base = h->scales_base;
+        d.codes_stride = (size_t)h->I * h->H / 2;
+        d.scales_stride = (size_t)h->I * h->H / 32;
         d.h = g.h;
         d.ids = g.ids;
         d.w = topk_w + (size_t)t0 * h->k;
+        d.logits = nullptr;
         d.residual = residual ? residual + (size_t)t0 * h->H : nullptr;
         d.y = y + (size_t)t0 * h->H;
         d.o_keep = keep ? obuf + (size_t)t0 * h->k * h->H : nullptr;
@@ -351,6 +377,123 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
 int moe_forward(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk_ids,
                 const float *topk_w, uint16_t *y, void *stream) {
     return moe_forward_ex(h, x, T, topk_ids, topk_w, nullptr, y, 0u, stream);
+}
+
+int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *router_w,
+                 const float *router_bias, unsigned route_flags, uint16_t *x_norm,
+                 float *logits, int32_t *topk_ids, float *topk_w, const uint16_t *residual,
+                 uint16_t *y, unsigned fwd_flags, void *stream) {
+    if (!h || T < 1) return MOE_ERR_ARG;
+    if (route_flags & ~MOE_ROUTE_RMSNORM) return MOE_ERR_ARG;
+    if (fwd_flags & ~MOE_FWD_KEEP_INTERMEDIATES) return MOE_ERR_ARG;
+    const bool norm = route_flags & MOE_ROUTE_RMSNORM;
+    if (norm != (x_norm != nullptr)) return MOE_ERR_ARG;
+    if (!h->loaded || !h->ws) return MOE_ERR_NOT_LOADED;
+    if (T > h->max_tokens) return MOE_ERR_WORKSPACE;
+    int rc;
+    if ((rc = check_device_ptr(h, x, 16)) != MOE_OK) return rc;
+    if ((rc = check_device_ptr(h, router_w, 16)) != MOE_OK) return rc;
+    if (router_bias && (rc = check_device_ptr(h, router_bias, 4)) != MOE_OK) return rc;
+    if (norm && (rc = check_device_ptr(h, x_norm, 16)) != MOE_OK) return rc;
+    if (logits && (rc = check_device_ptr(h, logits, 4)) != MOE_OK) return rc;
+    if (topk_ids && (rc = check_device_ptr(h, topk_ids, 4)) != MOE_OK) return rc;
+    if (topk_w && (rc = check_device_ptr(h, topk_w, 4)) != MOE_OK) return rc;
+    if (residual && (rc = check_device_ptr(h, residual, 16)) != MOE_OK) return rc;
+    if ((rc = check_device_ptr(h, y, 16)) != MOE_OK) return rc;
+    if (norm && (x_norm == x || x_norm == y)) return MOE_ERR_ARG;
+    if (!moe::decode_shape_supported(h->H, h->I)) return MOE_ERR_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const WsLayout L = ws_layout(h, h->max_tokens);
+    float *lg = reinterpret_cast<float *>(h->ws + L.logits);
+
+    if (T > moe::kDecodeMaxT) {
+        // many tokens: explicit routing, then the forward on the given ids
+        int32_t *ids = topk_ids;
+        float *w = topk_w;
+        if (!ids || !w) return MOE_ERR_ARG;
+        if ((rc = moe_route_ex(h, x, T, router_w, router_bias, route_flags, x_norm, logits, ids,
+                               w, stream)) != MOE_OK)
+            return rc;
+        return moe_forward_ex(h, norm ? x_norm : x, T, ids, w, residual, y, fwd_flags, stream);
+    }
+
+    moe::RouteParams rp;
+    rp.x = x;
+    rp.wr = router_w;
+    rp.bias = router_bias;
+    rp.x_norm = x_norm;
+    rp.logits_ws = lg;
+    rp.logits_out = logits;
+    rp.ids = nullptr;
+    rp.w = nullptr;
+    rp.counters = nullptr;
+    rp.T = T;
+    rp.E = h->E;
+    rp.H = h->H;
+    rp.k = h->k;
+    rp.rmsnorm = norm ? 1 : 0;
+    rp.eps = 1e-6f;
+    rp.x16 = reinterpret_cast<uint32_t *>(h->ws + L.x16);
+    rp.x16_exp = reinterpret_cast<int *>(h->ws + L.x16_exp);
+    if ((rc = cuda_rc(moe::launch_route_logits(rp, s, h->use_pdl))) != MOE_OK) return rc;
+
+    const bool keep = fwd_flags & MOE_FWD_KEEP_INTERMEDIATES;
+    moe::GateUpParams g;
+    g.table = h->d_table;
+    g.codes_base = h->codes_base;
+    g.scales_base = h->scales_base;
+    g.codes_stride = (size_t)h->I * h->H / 2;
+    g.scales_stride = (size_t)h->I * h->H / 32;
+    g.x = norm ? x_norm : x;
+    g.x16 = rp.x16;
+    g.x16_exp = rp.x16_exp;
+    g.ids = nullptr;
+    g.logits = lg;
+    g.ids_out = topk_ids;
+    g.w_out = topk_w;
+    g.h = reinterpret_cast<uint16_t *>(h->ws + L.h);
+    g.status = h->d_status;
+    g.T = T;
+    g.k = h->k;
+    g.E = h->E;
+    g.H = h->H;
+    g.I = h->I;
+    g.prefetch_down = h->prefetch_down ? 1 : 0;
+    {
+        const size_t mc = (size_t)h->H * h->I / 2, ms = (size_t)h->H * h->I / 32;
+        const size_t n = (size_t)h->num_sms;
+        g.pf_codes = (uint32_t)(((mc + n - 1) / n + 15) / 16 * 16);
+        g.pf_scales = (uint32_t)(((ms + n - 1) / n + 15) / 16 * 16);
+    }
+    g.nslots = moe::gateup_tma_slots(h->H);
+    if ((rc = cuda_rc(moe::launch_gateup_decode(g, h->num_sms, s, h->use_pdl))) != MOE_OK)
+        return rc;
+
+    moe::DownParams d;
+    d.table = h->d_table;
+    d.codes_base = h->codes_base;
+    d.scales_base = h->scales_base;
+    d.codes_stride = (size_t)h->I * h->H / 2;
+    d.scales_stride = (size_t)h->I * h->H / 32;
+    d.h = g.h;
+    d.ids = nullptr;
+    d.w = nullptr;
+    d.logits = lg;
+    d.residual = residual;
+    d.y = y;
+    d.o_keep = keep ? reinterpret_cast<uint16_t *>(h->ws + L.o) : nullptr;
+    d.status = h->d_status;
+    d.T = T;
+    d.k = h->k;
+    d.E = h->E;
+    d.H = h->H;
+    d.I = h->I;
+    const int rows = T * h->H;
+    d.rows_per_cta = (rows + h->num_sms - 1) / h->num_sms;
+    const int grid = (rows + d.rows_per_cta - 1) / d.rows_per_cta;
+    if ((rc = cuda_rc(moe::launch_down_decode(d, grid, s, h->use_pdl))) != MOE_OK) return rc;
+    h->kept = keep;
+    return MOE_OK;
 }
 
 int moe_get_intermediates(moe_handle_t h, const uint16_t **h_out, const uint16_t **o_out) {

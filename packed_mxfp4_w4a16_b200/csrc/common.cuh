@@ -183,6 +183,69 @@ __device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
     return r;
 }
 
+// ------------------------------------------------- mbarrier / bulk copy ----
+// Shared-memory barriers that count completed bytes of asynchronous bulk
+// copies (TMA engine, non-tensor form: 16-byte aligned addresses, sizes in
+// multiples of 16 bytes).  Every wait is bounded: after kMaxSpin unsuccessful
+// polls it gives up and the caller records an error in the status word.
+
+constexpr unsigned kTimeoutStatus = 0x2u;  // a bounded wait gave up
+constexpr int kMaxSpin = 1 << 20;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// producer: announce `bytes` of incoming copies and arrive (count 1)
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; "
+        "selp.u32 %0, 1, 0, p; }"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for phase `parity` of `bar` to complete; false if it did not within
+// kMaxSpin polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity) {
+#pragma unroll 1
+    for (int i = 0; i < kMaxSpin; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+// global -> shared bulk copy completing `bytes` on `bar`
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, unsigned bytes,
+                                         uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // ------------------------------------------------------------- warps -----
 
 template <int TL>
@@ -205,6 +268,78 @@ __device__ __forceinline__ float warp_sum(float v) {
     for (int o = 16; o > 0; o >>= 1)
         v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
+}
+
+// ---------------------------------------------------------------- top-k --
+// Top-k of one token's logits (E values in global memory, read through L2):
+// descending, equal logits -> lower expert id, NaN never chosen; coefficients
+// = softmax over the k chosen logits.  Called by one full warp; every lane
+// returns the same ids[0..k) and w[0..k).  Each round takes the warp-wide max
+// of an order-preserving key, then the lowest id among lanes holding it.
+__device__ __forceinline__ uint32_t logit_key(float v) {
+    const uint32_t b = __float_as_uint(v);
+    return (v != v) ? 0u : ((b & 0x80000000u) ? ~b : (b | 0x80000000u));
+}
+
+// Top-k of one token's E logits by one warp (strictly greater wins, the lower
+// expert id on equal logits), then the softmax of the k chosen logits.  Lane j
+// (j < k) returns the j-th selection in (id, w); other lanes return id = -1.
+// Round j takes the warp-wide max key and the lowest id holding it, then
+// clears that key; k rounds, one redux pair each.
+template <int PER>  // logits per lane: E <= 32 * PER
+__device__ __forceinline__ void warp_topk(const float *lg, int E, int k, int lane, int &id,
+                                          float &w) {
+    uint32_t key[PER];
+#pragma unroll
+    for (int m = 0; m < PER; ++m) {
+        const int e = lane + 32 * m;
+        key[m] = e < E ? logit_key(__ldcg(lg + e)) : 0u;
+    }
+    id = -1;
+    float mylv = 0.f, top = 0.f;
+#pragma unroll 1
+    for (int j = 0; j < k; ++j) {
+        uint32_t bk = 0u;
+        int bi = 0x7FFFFFFF;
+#pragma unroll
+        for (int m = 0; m < PER; ++m)
+            if (key[m] > bk) {
+                bk = key[m];
+                bi = lane + 32 * m;
+            }
+        const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
+        const int wi = (int)__reduce_min_sync(0xffffffffu, bk == wk ? (uint32_t)bi : 0x7FFFFFFFu);
+        const float lv = __uint_as_float((wk & 0x80000000u) ? (wk & 0x7FFFFFFFu) : ~wk);
+        if (j == 0) top = lv;
+        if (lane == j) {
+            id = wi;
+            mylv = lv;
+        }
+#pragma unroll
+        for (int m = 0; m < PER; ++m)
+            if (wi == lane + 32 * m) key[m] = 0u;
+    }
+    // softmax over the chosen logits: lane j < k holds exp(l_j - l_0)
+    const float mine = lane < k ? expf(mylv - top) : 0.f;
+    float z = mine;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    w = mine / z;
+}
+
+// Larger expert counts: out of line, to keep the hot kernels' code small.
+static __device__ __noinline__ void warp_topk_wide(const float *lg, int E, int k, int lane,
+                                                   int &id, float &w) {
+    warp_topk<32>(lg, E, k, lane, id, w);
+}
+
+// Dispatch on E (up to 1024 experts).
+__device__ __forceinline__ void warp_topk_any(const float *lg, int E, int k, int lane, int &id,
+                                              float &w) {
+    if (E <= 64)
+        warp_topk<2>(lg, E, k, lane, id, w);
+    else
+        warp_topk_wide(lg, E, k, lane, id, w);
 }
 
 // ------------------------------------------- programmatic launch ---------

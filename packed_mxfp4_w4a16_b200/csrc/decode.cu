@@ -37,59 +37,85 @@ constexpr int kGemvWarps = kGemvThreads / 32;
 constexpr int kDownWarps = kDownThreads / 32;
 
 // ------------------------------------------------------------------ route --
-// grid (E, ceil(T / 8)); warp w of CTA (e, b) computes logit[t = 8b + w][e].
-// The router row is fetched before the programmatic-launch wait (it is a
-// constant input), so its DRAM latency overlaps the previous kernel's tail.
+// route_logits_kernel: grid (E, ceil(T / kRouteTokensPerCta)); CTA (e, b)
+// computes logit[t][e] for its tokens with all 256 threads on one dot product
+// (each thread owns 16-byte chunks c = tid, tid + 256 of the row).  The
+// router row is a constant input, fetched before the programmatic-launch
+// wait.  With rmsnorm the CTA first reduces sum(r^2) of the token, rounds
+// xn = BF16(r / sqrt(mean(r^2) + eps)) element-wise (CTA e = 0 also stores
+// xn) and routes xn.  Top-k is done by the consumers of the logits.
 
-constexpr int kRouteWarps = kRouteThreads / 32;
-constexpr int kRouteMaxChunks = 16;  // H <= 16 * 32 * 8 = 4096 for the register path
+constexpr int kRouteTokensPerCta = 8;
+constexpr int kRouteMaxCpt = 2;  // 16-byte chunks per thread: H <= 2 * 256 * 8 = 4096
+
+// Sum (or max) over the CTA with one barrier: warp partials to `red`
+// (a buffer used only once per call site), every thread adds them up.
+__device__ __forceinline__ float block_sum_route(float v, float *red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    v = warp_sum(v);
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < kRouteThreads / 32; ++i) s += red[i];
+    return s;
+}
+
+__device__ __forceinline__ float block_max_route(float v, float *red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    v = warp_max(v);
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < kRouteThreads / 32; ++i) s = fmaxf(s, red[i]);
+    return s;
+}
 
 __global__ void __launch_bounds__(kRouteThreads)
-route_kernel(const RouteParams p) {
-    __shared__ int s_last;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int e = blockIdx.x, H = p.H, E = p.E, k = p.k;
-    const int t = blockIdx.y * kRouteWarps + warp;
-    const int nch = H >> 3;  // 16-byte chunks of 8 BF16
-    const bool active = t < p.T;
-
-    uint4 wv[kRouteMaxChunks];
+route_logits_kernel(const RouteParams p) {
+    __shared__ float red[3][kRouteThreads / 32];
+    const int tid = threadIdx.x;
+    const int e = blockIdx.x, H = p.H, E = p.E;
+    const int nch = H >> 3;
     const uint16_t *row = p.wr + (size_t)e * H;
+    uint4 wv[kRouteMaxCpt];
 #pragma unroll
-    for (int m = 0; m < kRouteMaxChunks; ++m) {
-        const int c = lane + 32 * m;
-        wv[m] = (active && c < nch) ? *reinterpret_cast<const uint4 *>(row + (size_t)c * 8)
-                                    : make_uint4(0u, 0u, 0u, 0u);
+    for (int m = 0; m < kRouteMaxCpt; ++m) {
+        const int c = tid + kRouteThreads * m;
+        wv[m] = c < nch ? *reinterpret_cast<const uint4 *>(row + (size_t)c * 8)
+                        : make_uint4(0u, 0u, 0u, 0u);
     }
-
     pdl_wait();
     pdl_launch_dependents();
 
-    if (active) {
+    const int t0 = blockIdx.y * kRouteTokensPerCta;
+    const int t1 = min(p.T, t0 + kRouteTokensPerCta);
+    #pragma unroll 1
+    for (int t = t0; t < t1; ++t) {
+        if (t > t0) __syncthreads();  // red[] is reused for the next token
         const uint16_t *xt = p.x + (size_t)t * H;
-        uint4 xv[kRouteMaxChunks];
+        uint4 xv[kRouteMaxCpt];
         float ss = 0.f;
 #pragma unroll
-        for (int m = 0; m < kRouteMaxChunks; ++m) {
-            const int c = lane + 32 * m;
+        for (int m = 0; m < kRouteMaxCpt; ++m) {
+            const int c = tid + kRouteThreads * m;
             xv[m] = c < nch ? *reinterpret_cast<const uint4 *>(xt + (size_t)c * 8)
                             : make_uint4(0u, 0u, 0u, 0u);
-            if (p.rmsnorm) {
-                const uint32_t w4[4] = {xv[m].x, xv[m].y, xv[m].z, xv[m].w};
+            const uint32_t w4[4] = {xv[m].x, xv[m].y, xv[m].z, xv[m].w};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float a = bf16_to_f32(w4[q] & 0xFFFFu), b = bf16_to_f32(w4[q] >> 16);
-                    ss = fmaf(a, a, ss);
-                    ss = fmaf(b, b, ss);
-                }
+            for (int q = 0; q < 4; ++q) {
+                const float a = bf16_to_f32(w4[q] & 0xFFFFu), b = bf16_to_f32(w4[q] >> 16);
+                ss = fmaf(a, a, ss);
+                ss = fmaf(b, b, ss);
             }
         }
         float inv = 1.f;
-        if (p.rmsnorm) inv = 1.0f / sqrtf(warp_sum(ss) / (float)H + p.eps);
-        float acc = 0.f;
+        if (p.rmsnorm) inv = 1.0f / sqrtf(block_sum_route(ss, red[0]) / (float)H + p.eps);
+        float acc = 0.f, amax = 0.f;
 #pragma unroll
-        for (int m = 0; m < kRouteMaxChunks; ++m) {
-            const int c = lane + 32 * m;
+        for (int m = 0; m < kRouteMaxCpt; ++m) {
+            const int c = tid + kRouteThreads * m;
             if (c < nch) {
                 uint32_t x4[4] = {xv[m].x, xv[m].y, xv[m].z, xv[m].w};
                 const uint32_t r4[4] = {wv[m].x, wv[m].y, wv[m].z, wv[m].w};
@@ -103,91 +129,101 @@ route_kernel(const RouteParams p) {
                         *reinterpret_cast<uint4 *>(p.x_norm + (size_t)t * H + (size_t)c * 8) =
                             make_uint4(x4[0], x4[1], x4[2], x4[3]);
                 }
+                xv[m] = make_uint4(x4[0], x4[1], x4[2], x4[3]);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    acc = fmaf(bf16_to_f32(x4[q] & 0xFFFFu), bf16_to_f32(r4[q] & 0xFFFFu), acc);
-                    acc = fmaf(bf16_to_f32(x4[q] >> 16), bf16_to_f32(r4[q] >> 16), acc);
+                    const float a = bf16_to_f32(x4[q] & 0xFFFFu), b = bf16_to_f32(x4[q] >> 16);
+                    acc = fmaf(a, bf16_to_f32(r4[q] & 0xFFFFu), acc);
+                    acc = fmaf(b, bf16_to_f32(r4[q] >> 16), acc);
+                    amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
                 }
             }
         }
-        acc = warp_sum(acc);
-        if (lane == 0) {
-            if (p.bias) acc += p.bias[e];
-            p.logits_ws[(size_t)t * E + e] = acc;
+        const float logit = block_sum_route(acc, red[1]);
+        if (tid == 0) {
+            const float v = p.bias ? logit + p.bias[e] : logit;
+            p.logits_ws[(size_t)t * E + e] = v;
+            if (p.logits_out) p.logits_out[(size_t)t * E + e] = v;
         }
-    }
-
-    // the last CTA of this token block selects; an arrival counter, no waiting
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        const unsigned prev = atomicAdd(p.counters + blockIdx.y, 1u);
-        s_last = (prev == (unsigned)E - 1u);
-    }
-    __syncthreads();
-    if (!s_last || !active) return;
-    __threadfence();
-
-    // top-k of logits[t][0..E): ids descending, equal logits -> lower id.
-    // Each round: warp-wide max of an order-preserving key of the logit, then
-    // the minimum id among the lanes holding that key (two redux operations).
-    const float *lg = p.logits_ws + (size_t)t * E;
-    constexpr int kMaxPerLane = 32;  // E <= 1024
-    const int per = (E + 31) >> 5;
-    uint32_t key[kMaxPerLane];
+        if (e == 0 && p.x16) {
+            // the expert GEMVs' FP16 staging of the routed vector, done once here
+            const int c16 = f16_stage_exponent(block_max_route(amax, red[2]));
+            const float sf = pow2_neg(c16);
 #pragma unroll
-    for (int m = 0; m < kMaxPerLane; ++m) {
-        const int ee = lane + 32 * m;
-        uint32_t kk = 0u;  // below every logit: never chosen
-        if (m < per && ee < E) {
-            const float v = __ldcg(lg + ee);
-            const uint32_t b = __float_as_uint(v);
-            kk = (v != v) ? 0u : ((b & 0x80000000u) ? ~b : (b | 0x80000000u));
-        }
-        key[m] = kk;
-    }
-    int chosen[kMaxTopK];
-    float chosen_v[kMaxTopK];
-    for (int j = 0; j < k; ++j) {
-        uint32_t bk = 0u;
-        int bi = 0x7FFFFFFF;
-#pragma unroll
-        for (int m = 0; m < kMaxPerLane; ++m)
-            if (key[m] > bk) {  // ascending m: ties keep the lower id
-                bk = key[m];
-                bi = lane + 32 * m;
+            for (int m = 0; m < kRouteMaxCpt; ++m) {
+                const int c = tid + kRouteThreads * m;
+                if (c < nch) {
+                    const uint32_t x4[4] = {xv[m].x, xv[m].y, xv[m].z, xv[m].w};
+                    uint4 o;
+                    o.x = f32x2_to_f16x2(bf16_to_f32(x4[0] & 0xFFFFu) * sf, bf16_to_f32(x4[0] >> 16) * sf);
+                    o.y = f32x2_to_f16x2(bf16_to_f32(x4[1] & 0xFFFFu) * sf, bf16_to_f32(x4[1] >> 16) * sf);
+                    o.z = f32x2_to_f16x2(bf16_to_f32(x4[2] & 0xFFFFu) * sf, bf16_to_f32(x4[2] >> 16) * sf);
+                    o.w = f32x2_to_f16x2(bf16_to_f32(x4[3] & 0xFFFFu) * sf, bf16_to_f32(x4[3] >> 16) * sf);
+                    *reinterpret_cast<uint4 *>(p.x16 + (size_t)t * (H >> 1) + (size_t)c * 4) = o;
+                }
             }
-        const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
-        const int wi = (int)__reduce_min_sync(0xffffffffu, bk == wk ? (uint32_t)bi : 0x7FFFFFFFu);
-        chosen[j] = wi;
-        chosen_v[j] = __uint_as_float((wk & 0x80000000u) ? (wk & 0x7FFFFFFFu) : ~wk);
-        if ((wi & 31) == lane && wi < E) {
-#pragma unroll
-            for (int m = 0; m < kMaxPerLane; ++m)
-                if (m == (wi >> 5)) key[m] = 0u;
+            if (tid == 0) p.x16_exp[t] = c16;
         }
     }
-    if (lane == 0) {
-        // coefficients: softmax over the k selected logits (slot 0 holds the max)
-        float z = 0.f, ex[kMaxTopK];
-        for (int j = 0; j < k; ++j) {
-            ex[j] = expf(chosen_v[j] - chosen_v[0]);
-            z += ex[j];
-        }
-        for (int j = 0; j < k; ++j) {
-            p.ids[(size_t)t * k + j] = chosen[j];
-            p.w[(size_t)t * k + j] = ex[j] / z;
+}
+
+// topk_kernel: grid ceil(T / 8), 256 threads; warp w selects for token
+// 8 * blockIdx.x + w and writes ids / w (standalone routing call).
+__global__ void __launch_bounds__(kRouteThreads)
+topk_kernel(const RouteParams p) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (kRouteThreads / 32) + (threadIdx.x >> 5);
+    if (t >= p.T) return;
+    int id;
+    float w;
+    warp_topk_any(p.logits_ws + (size_t)t * p.E, p.E, p.k, lane, id, w);
+    if (lane < p.k) {
+        p.ids[(size_t)t * p.k + lane] = id;
+        p.w[(size_t)t * p.k + lane] = w;
+    }
+}
+
+// One token's top-k by the calling warp into shared memory (ids) and,
+// optionally, global memory (ids_out, w_out).  Out of line.
+__device__ __noinline__ void topk_token_to_smem(const float *lg, int E, int k, int *s_ids,
+                                                int32_t *ids_out, float *w_out) {
+    const int lane = threadIdx.x & 31;
+    int id;
+    float w;
+    warp_topk_any(lg, E, k, lane, id, w);
+    if (lane < k) {
+        s_ids[lane] = id;
+        if (ids_out) ids_out[lane] = id;
+        if (w_out) w_out[lane] = w;
+    }
+}
+
+// Routing inside the expert kernels: warp t of the CTA selects for token t
+// (T <= kDecodeMaxT) into shared memory; CTA 0 also publishes ids / w.
+// Out of line (runs once per call).
+__device__ __noinline__ void route_into_smem(const float *logits, int T, int E, int k,
+                                                int *s_ids, float *s_w, int32_t *ids_out,
+                                                float *w_out) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (warp < T) {
+        int id;
+        float w;
+        warp_topk_any(logits + (size_t)warp * E, E, k, lane, id, w);
+        if (lane < k) {
+            s_ids[warp * k + lane] = id;
+            if (s_w) s_w[warp * k + lane] = w;
+            if (blockIdx.x == 0 && ids_out) ids_out[warp * k + lane] = id;
+            if (blockIdx.x == 0 && w_out) w_out[warp * k + lane] = w;
         }
     }
-    if (p.logits_out)
-        for (int ee = lane; ee < E; ee += 32) p.logits_out[(size_t)t * E + ee] = __ldcg(lg + ee);
-    if (warp == 0 && lane == 0) p.counters[blockIdx.y] = 0u;
 }
 
 // ------------------------------------------------------------- team tools --
 // A "team" of TL lanes (TL a power of two, aligned in the warp) owns one packed
-// row at a time; lane lt of the team holds the KCH consecutive 16-byte chunks
-// [lt*KCH, lt*KCH + KCH) of the row (one E8M0 group each) and the matching
+// row at a time; lane lt of the team holds the KCH 16-byte chunks
+// c = lt + TL*u (u < KCH) of the row (one E8M0 group each) and the matching
 // FP16-staged activations in registers.  Teams are independent: their
 // shuffles use the team's own lane mask.
 
@@ -219,7 +255,7 @@ __device__ __forceinline__ int stage_x(const uint16_t *v, int lt, int C, unsigne
     float m[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int u = 0; u < KCH; ++u) {
-        const int c = lt * KCH + u;
+        const int c = lt + TL * u;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             raw[u][q] = c < C ? *reinterpret_cast<const uint4 *>(v + (size_t)c * 32 + q * 8)
@@ -246,12 +282,12 @@ __device__ __forceinline__ int stage_x(const uint16_t *v, int lt, int C, unsigne
     return c;
 }
 
-template <int KCH>
+template <int TL, int KCH>
 __device__ __forceinline__ void load_chunks(const uint8_t *codes, const uint8_t *scales, bool ok,
                                             int lt, int C, uint4 (&cw)[KCH], uint32_t (&sc)[KCH]) {
 #pragma unroll
     for (int u = 0; u < KCH; ++u) {
-        const int c = lt * KCH + u;
+        const int c = lt + TL * u;
         if (ok && c < C) {
             cw[u] = ld_stream16(codes + (size_t)c * 16);
             sc[u] = ld_stream_u8(scales + c);
@@ -285,24 +321,30 @@ __device__ __forceinline__ float chunks_dot(const uint4 (&cw)[KCH], const uint32
 // streaming.  One lane per (token, slot) pair; an expert chosen by several
 // pairs is fetched by the lowest such lane only.  Slices are 16-byte multiples
 // computed on the host (codes: pf_codes bytes, scales: pf_scales bytes).
-__device__ __forceinline__ void prefetch_down_slice(const GateUpParams &p, int lane) {
+__device__ __forceinline__ void prefetch_down_slice(const GateUpParams &p, const int *s_ids,
+                                                    int lane) {
     const int P = p.T * p.k;
     const int Pr = (P + 31) & ~31;  // every lane iterates the same number of times
+    #pragma unroll 1
     for (int q = lane; q < Pr; q += 32) {
-        const int e = q < P ? p.ids[q] : -1;
+        const int e = q < P ? s_ids[q] : -1;
         const unsigned same = __match_any_sync(0xffffffffu, e);
         const bool leader = (__ffs(same) - 1) == lane;
         if (q < P && leader && e >= 0 && e < p.E) {
             const size_t mc = (size_t)p.H * p.I / 2, ms = (size_t)p.H * p.I / 32;
             const size_t oc = (size_t)blockIdx.x * p.pf_codes;
             const size_t os = (size_t)blockIdx.x * p.pf_scales;
+            const uint8_t *dc = p.codes_base ? p.codes_base + (size_t)(3 * e + 2) * p.codes_stride
+                                             : p.table[e].codes[2];
+            const uint8_t *ds = p.codes_base ? p.scales_base + (size_t)(3 * e + 2) * p.scales_stride
+                                             : p.table[e].scales[2];
             if (oc < mc) {
                 const size_t n = min((size_t)p.pf_codes, mc - oc);
-                prefetch_l2_bulk(p.table[e].codes[2] + oc, (uint32_t)n);
+                prefetch_l2_bulk(dc + oc, (uint32_t)n);
             }
             if (os < ms) {
                 const size_t n = min((size_t)p.pf_scales, ms - os);
-                prefetch_l2_bulk(p.table[e].scales[2] + os, (uint32_t)n);
+                prefetch_l2_bulk(ds + os, (uint32_t)n);
             }
         }
     }
@@ -321,9 +363,16 @@ gateup_decode_kernel(const GateUpParams p) {
     const int C = H >> 5;
     const size_t rc = (size_t)H >> 1, rs = (size_t)H >> 5;  // bytes per row: codes, scales
 
-    pdl_wait();  // x and ids come from earlier kernels
+    __shared__ int s_ids[kDecodeMaxT * kMaxTopK];
+    pdl_wait();  // x and the routing come from earlier kernels
     pdl_launch_dependents();
-    if (p.prefetch_down && warp == kGemvWarps - 1) prefetch_down_slice(p, lane);
+    if (p.ids) {
+        for (int q = threadIdx.x; q < p.T * k; q += kGemvThreads) s_ids[q] = p.ids[q];
+    } else {
+        route_into_smem(p.logits, p.T, p.E, k, s_ids, nullptr, p.ids_out, p.w_out);
+    }
+    __syncthreads();
+    if (p.prefetch_down && warp == kGemvWarps - 1) prefetch_down_slice(p, s_ids, lane);
 
     const long long N = (long long)p.T * k * I;
     const long long nteams = (long long)gridDim.x * kGemvWarps * TPW;
@@ -337,13 +386,14 @@ gateup_decode_kernel(const GateUpParams p) {
     bool bad = false;
     const uint8_t *gc = nullptr, *gs = nullptr, *uc = nullptr, *us = nullptr;
 
+    #pragma unroll 1
     while (it < end) {
         const int q = (int)(it / I);
         const int row = (int)(it - (long long)q * I);
         // a second row of the same pair in this step if there is one
         const bool two = (it + 1 < end) && (row + 1 < I);
         if (q != cur_q) {
-            const int e = p.ids[q];
+            const int e = s_ids[q];
             bad = (e < 0 || e >= p.E);
             if (!bad) {
                 const ExpertPtrs *ep = p.table + e;
@@ -360,8 +410,8 @@ gateup_decode_kernel(const GateUpParams p) {
         for (int u = 0; u < 2; ++u) {
             const bool ok = !bad && (u == 0 || two);
             const size_t r = (size_t)(row + u);
-            load_chunks<KCH>(gc + r * rc, gs + r * rs, ok, lt, C, cg[u], sg[u]);
-            load_chunks<KCH>(uc + r * rc, us + r * rs, ok, lt, C, cu[u], su[u]);
+            load_chunks<TL, KCH>(gc + r * rc, gs + r * rs, ok, lt, C, cg[u], sg[u]);
+            load_chunks<TL, KCH>(uc + r * rc, us + r * rs, ok, lt, C, cu[u], su[u]);
         }
         const int tok = q / k;
         if (tok != cur_tok) {
@@ -393,17 +443,353 @@ gateup_decode_kernel(const GateUpParams p) {
     }
 }
 
+// ------------------------------------------------- gate / up, bulk copies --
+// The CTA owns items [cb, ce) (rows of the selected experts' gate and up
+// matrices, (pair, row) order).  A producer warp selects the experts (from
+// the router logits, or takes the given ids), then streams the CTA's rows into
+// a ring of shared-memory slots with bulk copies that complete on per-slot
+// mbarriers; slot s holds kTmaSlotRows consecutive items (gate codes,
+// up codes, gate scales, up scales).  For T = 1 the whole CTA range (~40
+// rows, ~90 KB) is requested at once, so the DRAM sees the layer's entire
+// gate/up stream immediately.  The consumer warps each take one row per
+// slot, decode it from shared memory against register-staged activations,
+// and release the slot.  Every wait is bounded; a timeout sets a status bit
+// and the kernel drains its outstanding copies before returning.
+
+constexpr int kTmaConsumers = 23;
+constexpr int kTmaThreads = (kTmaConsumers + 1) * 32;
+constexpr int kTmaSlotRows = kTmaConsumers;
+constexpr int kTmaMaxSlots = 16;
+constexpr size_t kTmaSmemBudget = 200 * 1024;
+
+__host__ __device__ __forceinline__ size_t tma_slot_bytes(int H) {
+    return (size_t)kTmaSlotRows * 2 * ((size_t)H / 2 + (size_t)H / 32);
+}
+
+template <int KCH>
+__global__ void __launch_bounds__(kTmaThreads, 1)
+gateup_tma_kernel(const GateUpParams p) {
+    extern __shared__ __align__(128) uint8_t ring[];
+    __shared__ __align__(8) uint64_t full[kTmaMaxSlots];
+    __shared__ __align__(8) uint64_t empty[kTmaMaxSlots];
+    __shared__ int s_ids[kDecodeMaxT * kMaxTopK];
+    __shared__ ExpertPtrs s_tab[kDecodeMaxT * kMaxTopK];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int H = p.H, I = p.I, k = p.k, T = p.T, E = p.E;
+    const int C = H >> 5;
+    const size_t rc = (size_t)H >> 1, rs = (size_t)H >> 5;
+    const size_t slot_bytes = tma_slot_bytes(H);
+    const size_t up_off = (size_t)kTmaSlotRows * rc;
+    const size_t gs_off = 2 * up_off, us_off = gs_off + (size_t)kTmaSlotRows * rs;
+    const int nslots = p.nslots;
+    // this CTA's items [cb, ce): 32-bit math (T * k * I <= 4 * 8 * 4096), the
+    // quotient computed in floating point and corrected
+    const int N = T * k * I;
+    const int G = (int)gridDim.x;
+    auto split = [&](int c) {
+        int v = (int)(((double)N * c) / G);
+        while ((long long)v * G > (long long)N * c) --v;
+        while ((long long)(v + 1) * G <= (long long)N * c) ++v;
+        return v;
+    };
+    const int cb = split((int)blockIdx.x), ce = split((int)blockIdx.x + 1);
+    const int nsteps = (ce - cb + kTmaSlotRows - 1) / kTmaSlotRows;
+    const int nbar = min(nslots, nsteps);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < nbar; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kTmaConsumers);
+        }
+        mbar_fence_init();
+    }
+    __syncthreads();
+    pdl_wait();  // x and the routing come from earlier kernels
+    pdl_launch_dependents();
+
+    if (warp == kTmaConsumers) {
+        // ---- producer warp ----
+        const int P = T * k;
+        if (p.ids) {
+            #pragma unroll 1
+            for (int q = lane; q < P; q += 32) s_ids[q] = p.ids[q];
+        } else {
+            #pragma unroll 1
+            for (int t = 0; t < T; ++t)
+                topk_token_to_smem(p.logits + (size_t)t * E, E, k, s_ids + t * k,
+                                   blockIdx.x == 0 ? p.ids_out + (p.ids_out ? t * k : 0) : nullptr,
+                                   blockIdx.x == 0 ? p.w_out + (p.w_out ? t * k : 0) : nullptr);
+        }
+        __syncwarp();
+        #pragma unroll 1
+        for (int q = lane; q < P; q += 32) {
+            const int e = s_ids[q];
+            if (e >= 0 && e < E) {
+                if (p.codes_base) {
+                    ExpertPtrs ep;
+#pragma unroll
+                    for (int m = 0; m < 3; ++m) {
+                        ep.codes[m] = p.codes_base + (size_t)(3 * e + m) * p.codes_stride;
+                        ep.scales[m] = p.scales_base + (size_t)(3 * e + m) * p.scales_stride;
+                    }
+                    s_tab[q] = ep;
+                } else {
+                    s_tab[q] = p.table[e];
+                }
+            }
+        }
+        __syncwarp();
+        // Initial fill of the ring: one lane per (slot, pair segment, matrix)
+        // copy, all in one round; lane 8 s + 0 also announces slot s's bytes.
+        // Later slots reuse ring buffers and are issued by lane 0 in order.
+        const int nfill = min(nsteps, nslots);
+        #pragma unroll 1
+        for (int task = lane; task < 8 * nfill; task += 32) {
+            const int s = task >> 3, sub = task & 7, seg = sub >> 2, m = sub & 3;
+            const int r0 = cb + s * kTmaSlotRows;
+            const int r1 = min(ce, r0 + kTmaSlotRows);
+            const int qa = r0 / I, qb = (r1 - 1) / I;  // at most two pairs per slot
+            uint8_t *base = ring + (size_t)s * slot_bytes;
+            if (sub == 0) {
+                unsigned bytes = 0;
+                #pragma unroll 1
+                for (int q = qa; q <= qb; ++q) {
+                    const int e = s_ids[q];
+                    const int n = min(r1, (q + 1) * I) - max(r0, q * I);
+                    if (e >= 0 && e < E) bytes += (unsigned)(2 * n) * (unsigned)(rc + rs);
+                }
+                mbar_arrive_expect_tx(&full[s], bytes);
+            }
+            const int q = qa + seg;
+            if (q <= qb) {
+                const int e = s_ids[q];
+                const int a = max(r0, q * I);
+                const int n = min(r1, (q + 1) * I) - a;
+                if (e >= 0 && e < E) {
+                    const size_t idx = (size_t)(a - r0), i0 = (size_t)(a - q * I);
+                    const ExpertPtrs &ep = s_tab[q];
+                    const size_t dst = m == 0   ? idx * rc
+                                       : m == 1 ? up_off + idx * rc
+                                       : m == 2 ? gs_off + idx * rs
+                                                : us_off + idx * rs;
+                    const uint8_t *src = m == 0   ? ep.codes[0] + i0 * rc
+                                         : m == 1 ? ep.codes[1] + i0 * rc
+                                         : m == 2 ? ep.scales[0] + i0 * rs
+                                                  : ep.scales[1] + i0 * rs;
+                    const unsigned nb = (unsigned)(m < 2 ? n * rc : n * rs);
+                    bulk_g2s(base + dst, src, nb, &full[s]);
+                }
+            }
+        }
+        bool ok = true;
+        #pragma unroll 1
+        for (int s = nfill; s < nsteps && ok && lane == 0; ++s) {
+            const int b = s % nslots;
+            if (!mbar_wait(&empty[b], (unsigned)((s / nslots) - 1) & 1u)) {
+                atomicOr(p.status, kTimeoutStatus);
+                ok = false;
+                break;
+            }
+            uint8_t *base = ring + (size_t)b * slot_bytes;
+            const int r0 = cb + s * kTmaSlotRows;
+            const int r1 = min(ce, r0 + kTmaSlotRows);
+            const int qa = r0 / I, qb = (r1 - 1) / I;
+            unsigned bytes = 0;
+            #pragma unroll 1
+            for (int q = qa; q <= qb; ++q) {
+                const int e = s_ids[q];
+                const int n = min(r1, (q + 1) * I) - max(r0, q * I);
+                if (e >= 0 && e < E) bytes += (unsigned)(2 * n) * (unsigned)(rc + rs);
+            }
+            mbar_arrive_expect_tx(&full[b], bytes);
+            #pragma unroll 1
+            for (int q = qa; q <= qb; ++q) {
+                const int e = s_ids[q];
+                const int a = max(r0, q * I);
+                const int n = min(r1, (q + 1) * I) - a;
+                if (e >= 0 && e < E) {
+                    const size_t idx = (size_t)(a - r0), i0 = (size_t)(a - q * I);
+                    const ExpertPtrs &ep = s_tab[q];
+                    bulk_g2s(base + idx * rc, ep.codes[0] + i0 * rc, (unsigned)(n * rc), &full[b]);
+                    bulk_g2s(base + up_off + idx * rc, ep.codes[1] + i0 * rc, (unsigned)(n * rc),
+                             &full[b]);
+                    bulk_g2s(base + gs_off + idx * rs, ep.scales[0] + i0 * rs, (unsigned)(n * rs),
+                             &full[b]);
+                    bulk_g2s(base + us_off + idx * rs, ep.scales[1] + i0 * rs, (unsigned)(n * rs),
+                             &full[b]);
+                }
+            }
+        }
+        __syncwarp();
+        if (p.prefetch_down) prefetch_down_slice(p, s_ids, lane);
+        // no copy may still be in flight into this CTA's shared memory at exit
+        for (int s = max(0, nsteps - nbar) + lane; s < nsteps; s += 32)
+            mbar_wait(&full[s % nslots], (unsigned)(s / nslots) & 1u);
+        return;
+    }
+
+    // ---- consumer warps: one row per slot each ----
+    uint32_t xw[KCH][16];
+    int cur_tok = -1;
+    float xs = 1.f;
+    bool failed = false;
+    // FP16 activations of token `tok` into registers: loaded as staged by the
+    // router when available, else staged here.  Plain (L1-allocating) loads:
+    // every warp of the CTA reads the same vector, so one L2 read per SM
+    // serves all of them.
+    auto get_x = [&](int tok) {
+        if (p.x16) {
+            const uint32_t *xv = p.x16 + (size_t)tok * (H >> 1);
+#pragma unroll
+            for (int u = 0; u < KCH; ++u) {
+                const int c = lane + 32 * u;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 v = c < C ? reinterpret_cast<const uint4 *>(xv + (size_t)c * 16)[q]
+                                          : make_uint4(0u, 0u, 0u, 0u);
+                    xw[u][4 * q] = v.x;
+                    xw[u][4 * q + 1] = v.y;
+                    xw[u][4 * q + 2] = v.z;
+                    xw[u][4 * q + 3] = v.w;
+                }
+            }
+            xs = pow2(p.x16_exp[tok]);
+        } else {
+            xs = pow2(stage_x<32, KCH>(p.x + (size_t)tok * H, lane, C, 0xffffffffu, xw));
+        }
+        cur_tok = tok;
+    };
+    #pragma unroll 1
+    for (int s = 0; s < nsteps; ++s) {
+        const int b = s % nslots;
+        const int row = cb + s * kTmaSlotRows + warp;
+        if (row < ce && !failed) {
+            // activations first: staging overlaps the slot's copies in flight
+            const int tok = (row / I) / k;
+            if (tok != cur_tok) get_x(tok);
+            if (!mbar_wait(&full[b], (unsigned)(s / nslots) & 1u)) {
+                failed = true;
+                if (lane == 0) atomicOr(p.status, kTimeoutStatus);
+            } else {
+                const int q = row / I;
+                const int i = row - q * I;
+                const int e = s_ids[q];
+                const bool bad = e < 0 || e >= E;
+                const uint8_t *base = ring + (size_t)b * slot_bytes;
+                uint4 cg[KCH], cu[KCH];
+                uint32_t sg[KCH], su[KCH];
+#pragma unroll
+                for (int u = 0; u < KCH; ++u) {
+                    const int c = lane + 32 * u;
+                    if (c < C && !bad) {
+                        cg[u] = *reinterpret_cast<const uint4 *>(base + (size_t)warp * rc + (size_t)c * 16);
+                        cu[u] = *reinterpret_cast<const uint4 *>(base + up_off + (size_t)warp * rc +
+                                                                (size_t)c * 16);
+                        sg[u] = base[gs_off + (size_t)warp * rs + c];
+                        su[u] = base[us_off + (size_t)warp * rs + c];
+                    } else {
+                        cg[u] = cu[u] = make_uint4(0u, 0u, 0u, 0u);
+                        sg[u] = su[u] = 127u;
+                    }
+                }
+                float ag = chunks_dot<KCH>(cg, sg, xw);
+                float au = chunks_dot<KCH>(cu, su, xw);
+                ag = warp_sum(ag);
+                au = warp_sum(au);
+                if (lane == 0) {
+                    uint16_t out = 0;
+                    if (!bad) {
+                        const float g = round_bf16(ag * xs);
+                        const float uu = round_bf16(au * xs);
+                        const float sl = round_bf16(g / (1.0f + expf(-g)));
+                        out = f32_to_bf16(sl * uu);
+                    } else {
+                        atomicOr(p.status, kBadExpertId);
+                    }
+                    p.h[(size_t)q * I + i] = out;
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[b]);
+    }
+}
+
 // ---------------------------------------------------------------- down -----
-// CTA = a range of output rows (t, n) for every slot j; the warps of slot
-// group j stream the down rows of expert ids[t][j]; the combine runs in
-// shared memory after one barrier.  The first rows' weights are requested
-// before the programmatic-launch wait (the routing is final by then: the
-// gate/up kernel released this grid only after its own wait).
+// CTA = a range of output rows (t, n) for every slot j.  Before the
+// programmatic-launch wait (the routing is final by then: the gate/up grid
+// released this one only after its own wait) the CTA selects the experts and
+// requests its first down rows.  After the wait it stages the k*T SwiGLU
+// vectors h once into shared memory as FP16, then teams of TL lanes (slot
+// group j = warp % k) stream their rows against them.  Expert outputs meet in
+// shared memory for the sequential BF16 combine.
+
+// Stage the P BF16 vectors h[q][0..I) into shared memory as FP16 words, each
+// scaled by 2^-c_q (c_q from the vector's max |h|); s_xs[q] = 2^c_q.  One pass
+// over h: every 16-byte piece is read once (raw into sh) while its max |h|
+// goes to s_max[q] (warp max, then a shared atomic max on the non-negative
+// float bits); after one barrier each thread converts its own pieces in place.
+// s_max[0..P) must be zero on entry.  Out of line: it runs once per call and
+// keeps the kernel's code small.
+__device__ __noinline__ void stage_h_block(const uint16_t *h, int P, int I, uint32_t *sh,
+                                           float *s_xs, unsigned *s_max) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int n4 = I >> 3;  // 16-byte pieces per vector
+    const int total = P * n4;
+    const uint4 *hv = reinterpret_cast<const uint4 *>(h);
+    uint4 *sv = reinterpret_cast<uint4 *>(sh);
+    // every lane of a warp runs the same trip count (warp-wide votes inside)
+#pragma unroll 1
+    for (int base = warp * 32; base < total; base += kDownThreads) {
+        const int i = base + lane;
+        const bool valid = i < total;
+        float m = 0.f;
+        int q = -1;
+        if (valid) {
+            const uint4 v = hv[i];
+            sv[i] = v;
+            q = i / n4;
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+                m = fmaxf(m, fmaxf(fabsf(bf16_to_f32(w4[r] & 0xFFFFu)),
+                                   fabsf(bf16_to_f32(w4[r] >> 16))));
+        }
+        if (__all_sync(0xffffffffu, q == __shfl_sync(0xffffffffu, q, 0))) {
+            m = warp_max(m);
+            if (lane == 0 && q >= 0) atomicMax(s_max + q, __float_as_uint(m));
+        } else if (valid) {
+            atomicMax(s_max + q, __float_as_uint(m));
+        }
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int i = threadIdx.x; i < total; i += kDownThreads) {
+        const float sf = pow2_neg(f16_stage_exponent(__uint_as_float(s_max[i / n4])));
+        const uint4 v = sv[i];
+        uint4 o;
+        o.x = f32x2_to_f16x2(bf16_to_f32(v.x & 0xFFFFu) * sf, bf16_to_f32(v.x >> 16) * sf);
+        o.y = f32x2_to_f16x2(bf16_to_f32(v.y & 0xFFFFu) * sf, bf16_to_f32(v.y >> 16) * sf);
+        o.z = f32x2_to_f16x2(bf16_to_f32(v.z & 0xFFFFu) * sf, bf16_to_f32(v.z >> 16) * sf);
+        o.w = f32x2_to_f16x2(bf16_to_f32(v.w & 0xFFFFu) * sf, bf16_to_f32(v.w >> 16) * sf);
+        sv[i] = o;
+    }
+    if (threadIdx.x < P) s_xs[threadIdx.x] = pow2(f16_stage_exponent(__uint_as_float(s_max[threadIdx.x])));
+    __syncthreads();
+}
+
+__device__ __forceinline__ const uint8_t *down_codes(const DownParams &p, int e) {
+    return p.codes_base ? p.codes_base + (size_t)(3 * e + 2) * p.codes_stride : p.table[e].codes[2];
+}
+__device__ __forceinline__ const uint8_t *down_scales(const DownParams &p, int e) {
+    return p.codes_base ? p.scales_base + (size_t)(3 * e + 2) * p.scales_stride
+                        : p.table[e].scales[2];
+}
 
 template <int TL, int KCH>
 __global__ void __launch_bounds__(kDownThreads, 1)
 down_decode_kernel(const DownParams p) {
-    extern __shared__ __align__(16) float so[];  // [k][R]
+    extern __shared__ __align__(16) uint8_t sm[];
     constexpr int TPW = 32 / TL;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int lt = lane & (TL - 1);
@@ -414,12 +800,31 @@ down_decode_kernel(const DownParams p) {
     const int R = p.rows_per_cta;
     const int r0 = blockIdx.x * R;
     const int r1 = min(r0 + R, T * H);
+    const int P = T * k;
+    uint32_t *sh = reinterpret_cast<uint32_t *>(sm);                       // [P][I/2] FP16 words
+    float *so = reinterpret_cast<float *>(sm + (size_t)P * I * 2);         // [k][R]
+    __shared__ int s_ids[kDecodeMaxT * kMaxTopK];
+    __shared__ float s_w[kDecodeMaxT * kMaxTopK];
+    __shared__ float s_xs[kDecodeMaxT * kMaxTopK];
+    __shared__ unsigned s_hmax[kDecodeMaxT * kMaxTopK];
 
     const int groups = kDownWarps / k;  // warps per slot
     const int j = warp % k, gi = warp / k;
     const int tps = groups * TPW;       // teams per slot
     const int ti = gi * TPW + lane / TL;
     const bool worker = gi < groups;
+
+    // routing for this call's tokens
+    if (threadIdx.x < P) s_hmax[threadIdx.x] = 0u;
+    if (p.ids) {
+        for (int q = threadIdx.x; q < P; q += kDownThreads) {
+            s_ids[q] = __ldcg(p.ids + q);
+            s_w[q] = __ldcg(p.w + q);
+        }
+    } else {
+        route_into_smem(p.logits, T, p.E, k, s_ids, s_w, nullptr, nullptr);
+    }
+    __syncthreads();
 
     // rows of this team: r0 + ti, r0 + ti + tps, ...; two per step
     int rr = r0 + ti;
@@ -433,15 +838,15 @@ down_decode_kernel(const DownParams p) {
             const bool valid = worker && r < r1;
             const int t = valid ? r / H : 0;
             const int n = r - t * H;
-            const int e = valid ? p.ids[t * k + j] : 0;
+            const int e = valid ? s_ids[t * k + j] : 0;
             bad[u] = valid && (e < 0 || e >= p.E);
             const bool ok = valid && !bad[u];
             const uint8_t *dc = nullptr, *ds = nullptr;
             if (ok) {
-                dc = p.table[e].codes[2] + (size_t)n * rc;
-                ds = p.table[e].scales[2] + (size_t)n * rs;
+                dc = down_codes(p, e) + (size_t)n * rc;
+                ds = down_scales(p, e) + (size_t)n * rs;
             }
-            load_chunks<KCH>(dc, ds, ok, lt, C, cw[u], sc[u]);
+            load_chunks<TL, KCH>(dc, ds, ok, lt, C, cw[u], sc[u]);
         }
     };
     fetch(rr);
@@ -449,21 +854,37 @@ down_decode_kernel(const DownParams p) {
     pdl_wait();  // h comes from the gate/up kernel
     pdl_launch_dependents();
 
-    uint32_t xw[KCH][16];
-    int cur_tok = -1;
-    float xs = 1.f;
+    // stage every h[t][j] once into shared memory as FP16
+    stage_h_block(p.h, P, I, sh, s_xs, s_hmax);
+
+    #pragma unroll 1
     while (worker && rr < r1) {
         const int t = rr / H;
-        if (t != cur_tok) {
-            xs = pow2(stage_x<TL, KCH>(p.h + ((size_t)t * k + j) * I, lt, C, mask, xw));
-            cur_tok = t;
-        }
+        const uint32_t *xv = sh + (size_t)(t * k + j) * (I >> 1);
+        const float xs = s_xs[t * k + j];
         // both rows of a step belong to token t unless the second crosses into
         // the next token; then it is recomputed in the next step
         const int rb = rr + tps;
         const bool second = rb < r1 && rb / H == t;
-        float a0 = chunks_dot<KCH>(cw[0], sc[0], xw);
-        float a1 = chunks_dot<KCH>(cw[1], sc[1], xw);
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int u = 0; u < KCH; ++u) {
+            const int c = lt + TL * u;
+            if (c < C) {
+                const uint4 *xq = reinterpret_cast<const uint4 *>(xv + (size_t)c * 16);
+                uint32_t x[16];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 v = xq[q];
+                    x[4 * q] = v.x;
+                    x[4 * q + 1] = v.y;
+                    x[4 * q + 2] = v.z;
+                    x[4 * q + 3] = v.w;
+                }
+                a0 = fmaf(dot32_e2m1_f16(cw[0][u], x), e8m0_to_f32(sc[0][u]), a0);
+                a1 = fmaf(dot32_e2m1_f16(cw[1][u], x), e8m0_to_f32(sc[1][u]), a1);
+            }
+        }
         a0 = team_add<TL>(a0, mask);
         a1 = team_add<TL>(a1, mask);
         const bool b0 = bad[0], b1 = bad[1];
@@ -482,12 +903,13 @@ down_decode_kernel(const DownParams p) {
     __syncthreads();
 
     // sequential BF16 combine in slot order, optional residual add
+    #pragma unroll 1
     for (int r = r0 + threadIdx.x; r < r1; r += kDownThreads) {
         const int t = r / H, n = r - t * H;
         float y = 0.f;
         for (int jj = 0; jj < k; ++jj) {
             const float o = so[jj * R + (r - r0)];
-            const float wb = round_bf16(p.w[(size_t)t * k + jj]);
+            const float wb = round_bf16(s_w[t * k + jj]);
             y = round_bf16(y + round_bf16(o * wb));
             if (p.o_keep) p.o_keep[((size_t)t * k + jj) * H + n] = f32_to_bf16(o);
         }
@@ -558,8 +980,16 @@ cudaError_t launch_gu(const GateUpParams &p, int grid, cudaStream_t s, bool pdl)
 
 template <int TL, int KCH>
 cudaError_t launch_dn(const DownParams &p, int grid, cudaStream_t s, bool pdl) {
+    static bool attr_set = false;
     const size_t smem = down_decode_smem(p.T, p.k, p.I, p.rows_per_cta);
-    if (smem > 48 * 1024) return cudaErrorInvalidValue;
+    if (smem > kDownSmemMax) return cudaErrorInvalidValue;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(down_decode_kernel<TL, KCH>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kDownSmemMax);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
     return launch_ex(down_decode_kernel<TL, KCH>, dim3(grid), dim3(kDownThreads), smem, s, pdl, p);
 }
 
@@ -590,6 +1020,29 @@ cudaError_t launch_dn(const DownParams &p, int grid, cudaStream_t s, bool pdl) {
 
 }  // namespace
 
+bool gateup_tma_supported(int H) { return H % 512 == 0 && H <= 4096; }
+
+int gateup_tma_slots(int H) {
+    const size_t sb = tma_slot_bytes(H);
+    size_t n = kTmaSmemBudget / sb;
+    if (n > (size_t)kTmaMaxSlots) n = kTmaMaxSlots;
+    return (int)n;
+}
+
+template <int KCH>
+cudaError_t launch_gu_tma(const GateUpParams &p, int grid, cudaStream_t s, bool pdl) {
+    static bool attr_set = false;
+    const size_t smem = (size_t)p.nslots * tma_slot_bytes(p.H);
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(gateup_tma_kernel<KCH>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kTmaSmemBudget);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    return launch_ex(gateup_tma_kernel<KCH>, dim3(grid), dim3(kTmaThreads), smem, s, pdl, p);
+}
+
 bool decode_shape_supported(int H, int I) {
     int tl, kch;
     pick_team(H / 32, tl, kch);
@@ -600,16 +1053,36 @@ bool decode_shape_supported(int H, int I) {
 
 size_t gateup_decode_smem(int, int) { return 0; }
 
-size_t down_decode_smem(int, int k, int, int rows_per_cta) {
-    return (size_t)k * rows_per_cta * 4;
+size_t down_decode_smem(int T, int k, int I, int rows_per_cta) {
+    return (size_t)T * k * I * 2 + (size_t)k * rows_per_cta * 4;
+}
+
+cudaError_t launch_route_logits(const RouteParams &p, cudaStream_t s, bool pdl) {
+    const int tblocks = (p.T + kRouteTokensPerCta - 1) / kRouteTokensPerCta;
+    return launch_ex(route_logits_kernel, dim3(p.E, tblocks), dim3(kRouteThreads), 0, s, pdl, p);
+}
+
+cudaError_t launch_topk(const RouteParams &p, cudaStream_t s, bool pdl) {
+    const int blocks = (p.T + kRouteThreads / 32 - 1) / (kRouteThreads / 32);
+    return launch_ex(topk_kernel, dim3(blocks), dim3(kRouteThreads), 0, s, pdl, p);
 }
 
 cudaError_t launch_route(const RouteParams &p, cudaStream_t s, bool pdl) {
-    const int tblocks = (p.T + kRouteWarps - 1) / kRouteWarps;
-    return launch_ex(route_kernel, dim3(p.E, tblocks), dim3(kRouteThreads), 0, s, pdl, p);
+    cudaError_t e = launch_route_logits(p, s, pdl);
+    if (e != cudaSuccess) return e;
+    return launch_topk(p, s, pdl);
 }
 
 cudaError_t launch_gateup_decode(const GateUpParams &p, int grid, cudaStream_t s, bool pdl) {
+    if (p.nslots >= 2 && gateup_tma_supported(p.H)) {
+        switch ((p.H / 32 + 31) / 32) {
+        case 1: return launch_gu_tma<1>(p, grid, s, pdl);
+        case 2: return launch_gu_tma<2>(p, grid, s, pdl);
+        case 3: return launch_gu_tma<3>(p, grid, s, pdl);
+        case 4: return launch_gu_tma<4>(p, grid, s, pdl);
+        default: return cudaErrorInvalidValue;
+        }
+    }
     MOE_TEAM_DISPATCH(launch_gu, p.H / 32, p, grid, s, pdl);
 }
 

@@ -11,7 +11,7 @@ namespace moe {
 constexpr int kDecodeMaxT = 4;      // tokens handled by the per-(token,slot) GEMV path
 constexpr int kMaxTopK = 8;
 constexpr int kGemvThreads = 512;   // gate/up GEMV: 16 warps, one CTA per SM
-constexpr int kDownThreads = 384;   // down GEMV + combine: 12 warps, one CTA per SM
+constexpr int kDownThreads = 768;   // down GEMV + combine: 24 warps, one CTA per SM
 constexpr int kRouteThreads = 256;  // 8 warps, one expert row per warp
 constexpr unsigned kBadExpertId = 0x1u;
 constexpr size_t kMaxDecodeSmem = 200 * 1024;  // dynamic shared memory cap of the GEMVs
@@ -26,6 +26,8 @@ struct RouteParams {
     int32_t *ids;           // [T][k]
     float *w;               // [T][k]
     unsigned *counters;     // [T], zero between calls
+    uint32_t *x16;          // [T][H/2] FP16-staged routed vector (f16x2 words) or null
+    int *x16_exp;           // [T] its staging exponent c (values are x * 2^-c)
     int T, E, H, k;
     int rmsnorm;
     float eps;
@@ -33,20 +35,33 @@ struct RouteParams {
 
 struct GateUpParams {
     const ExpertPtrs *table;  // [E]
+    // contiguous layout fast path (weights bound with one base address):
+    // matrix m of expert e at base + (3 e + m) * stride; null: use the table
+    const uint8_t *codes_base, *scales_base;
+    size_t codes_stride, scales_stride;
     const uint16_t *x;        // [T][H]
-    const int32_t *ids;       // [T][k]
+    const uint32_t *x16;      // [T][H/2] pre-staged FP16 x (from the router) or null
+    const int *x16_exp;       // [T] staging exponents of x16
+    const int32_t *ids;       // [T][k] given routing, or null: route from logits
+    const float *logits;      // [T][E] when ids is null
+    int32_t *ids_out;         // [T][k] or null: written by CTA 0 when routing
+    float *w_out;             // [T][k] or null: from logits
     uint16_t *h;              // [T][k][I]
     unsigned *status;
     int T, k, E, H, I;
     int prefetch_down;        // L2-prefetch the selected down matrices
     uint32_t pf_codes, pf_scales;  // per-CTA prefetch slice (bytes, multiple of 16)
+    int nslots;               // shared-memory ring slots of the bulk-copy kernel
 };
 
 struct DownParams {
     const ExpertPtrs *table;
+    const uint8_t *codes_base, *scales_base;  // contiguous layout fast path (or null)
+    size_t codes_stride, scales_stride;
     const uint16_t *h;         // [T][k][I]
-    const int32_t *ids;        // [T][k]
-    const float *w;            // [T][k]
+    const int32_t *ids;        // [T][k] given routing, or null: route from logits
+    const float *w;            // [T][k] given routing weights (ids != null)
+    const float *logits;       // [T][E] when ids is null
     const uint16_t *residual;  // [T][H] or null
     uint16_t *y;               // [T][H]
     uint16_t *o_keep;          // [T][k][H] or null
@@ -58,12 +73,17 @@ struct DownParams {
 // Host-side launchers (decode.cu).  `pdl` sets programmatic stream
 // serialization so the kernel may start while the previous one drains.
 cudaError_t launch_route(const RouteParams &p, cudaStream_t s, bool pdl);
+cudaError_t launch_route_logits(const RouteParams &p, cudaStream_t s, bool pdl);
+cudaError_t launch_topk(const RouteParams &p, cudaStream_t s, bool pdl);
+bool gateup_tma_supported(int H);
+int gateup_tma_slots(int H);
 cudaError_t launch_gateup_decode(const GateUpParams &p, int grid, cudaStream_t s, bool pdl);
 cudaError_t launch_down_decode(const DownParams &p, int grid, cudaStream_t s, bool pdl);
 cudaError_t launch_debug_dequant(const uint8_t *codes, const uint8_t *scales, int64_t n,
                                  float *out, cudaStream_t s);
 size_t gateup_decode_smem(int T, int H);
 size_t down_decode_smem(int T, int k, int I, int rows_per_cta);
+constexpr size_t kDownSmemMax = 200 * 1024;
 bool decode_shape_supported(int H, int I);
 
 }  // namespace moe

@@ -105,13 +105,30 @@ extern "C" int moe_forward_noalloc(int E, int H, int I, int top_k, const uint8_t
         return MOE_ERR_CUDA;
     }
 
-    // same per-(token, slot) GEMV path as moe_forward, in token chunks
-    for (int t0 = 0; t0 < T; t0 += moe::kDecodeMaxT) {
-        const int Tc = (T - t0 < moe::kDecodeMaxT) ? T - t0 : moe::kDecodeMaxT;
+    // same per-(token, slot) GEMV path as moe_forward, in token chunks sized so
+    // that the down kernel's staged activations fit in shared memory
+    int chunk = moe::kDecodeMaxT;
+    while (chunk > 1 && moe::down_decode_smem(chunk, top_k, I, (chunk * H + sms - 1) / sms) >
+                            moe::kDownSmemMax)
+        --chunk;
+    if (moe::down_decode_smem(1, top_k, I, (H + sms - 1) / sms) > moe::kDownSmemMax)
+        return MOE_ERR_ARG;
+    for (int t0 = 0; t0 < T; t0 += chunk) {
+        const int Tc = (T - t0 < chunk) ? T - t0 : chunk;
         moe::GateUpParams g;
         g.table = d_table;
+        g.codes_base = codes_u8;
+        g.scales_base = scales_e8m0;
+        g.codes_stride = mc;
+        g.scales_stride = ms;
         g.x = x + (size_t)t0 * H;
+        g.x16 = nullptr;
+        g.x16_exp = nullptr;
         g.ids = topk_ids + (size_t)t0 * top_k;
+        g.logits = nullptr;
+        g.ids_out = nullptr;
+        g.w_out = nullptr;
+        g.nslots = moe::gateup_tma_slots(H);
         g.h = d_h + (size_t)t0 * top_k * I;
         g.status = d_status;
         g.T = Tc;
@@ -128,9 +145,14 @@ extern "C" int moe_forward_noalloc(int E, int H, int I, int top_k, const uint8_t
         }
         moe::DownParams d;
         d.table = d_table;
+        d.codes_base = codes_u8;
+        d.scales_base = scales_e8m0;
+        d.codes_stride = mc;
+        d.scales_stride = ms;
         d.h = g.h;
         d.ids = g.ids;
         d.w = topk_w + (size_t)t0 * top_k;
+        d.logits = nullptr;
         d.residual = residual ? residual + (size_t)t0 * H : nullptr;
         d.y = y + (size_t)t0 * H;
         d.o_keep = nullptr;
