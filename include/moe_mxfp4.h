@@ -198,7 +198,8 @@ MOE_API int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T,
                    void *stream);
 
 /* One whole layer: routing + expert FFN + combine, with the routing computed
- * inside the expert kernels (no separate top-k launch, no id round trip):
+ * inside the expert kernels (no separate top-k launch, no id round trip; see
+ * moe_set_fusion):
  *   - route_flags MOE_ROUTE_RMSNORM: x is a residual stream r; the layer
  *     routes and runs the experts on xn = BF16(r / sqrt(mean(r^2) + 1e-6)),
  *     written to x_norm (device BF16 [T][H], distinct from x and y).
@@ -238,6 +239,18 @@ MOE_API int moe_bytes_per_expert(moe_handle_t h, size_t *bytes);
  * the gate/up kernel asks L2 to fetch the selected experts' down matrices
  * while it streams gate/up.  Errors: ARG. */
 MOE_API int moe_set_tuning(moe_handle_t h, int use_pdl, int prefetch_down);
+
+/* Launch structure of moe_layer_ex for T <= 4 (off by default; results are
+ * bit-identical either way): fused_router != 0 computes the RMSNorm, the
+ * router logits and the top-k inside the gate/up launch (one CTA per SM;
+ * the CTA of index e publishes expert e's logit to the others through the
+ * workspace) and hands the routing to the down launch
+ * through the workspace; 0 runs a separate router launch first.  Shapes the
+ * fused launch cannot hold (E > 256, H not a multiple of 512 or above 4096)
+ * use the separate launch regardless.  The workspace carries call counters
+ * for this: one workspace must not serve two calls at the same time.
+ * Errors: ARG. */
+MOE_API int moe_set_fusion(moe_handle_t h, int fused_router);
 
 /* ---------------------------------------------------------------------
  * Forward without any device allocation.  No counterpart in the paper: this

@@ -173,6 +173,10 @@ def moe_set_tuning(h: int, use_pdl: bool, prefetch_down: bool) -> None:
     check("moe_set_tuning", load().moe_set_tuning(C.c_void_p(h), int(use_pdl), int(prefetch_down)))
 
 
+def moe_set_fusion(h: int, fused_router: bool) -> None:
+    check("moe_set_fusion", load().moe_set_fusion(C.c_void_p(h), int(fused_router)))
+
+
 def moe_device_check() -> None:
     check("moe_device_check", load().moe_device_check())
 

@@ -37,6 +37,7 @@ SIGNATURES = [
     ("moe_get_status", _i, [_vp, C.POINTER(_u)]),
     ("moe_bytes_per_expert", _i, [_vp, C.POINTER(_sz)]),
     ("moe_set_tuning", _i, [_vp, _i, _i]),
+    ("moe_set_fusion", _i, [_vp, _i]),
     ("moe_status_string", C.c_char_p, [_i]),
     ("moe_device_check", _i, []),
     ("moe_debug_dequant", _i, [_vp, _vp, _i64, _vp, _vp]),

@@ -31,6 +31,7 @@ struct moe_ctx {
     bool kept = false;                    // last forward kept intermediates
     bool use_pdl = true;
     bool prefetch_down = true;
+    bool fused_router = false;            // moe_layer_ex: router inside the gate/up launch
     const uint8_t *codes_base = nullptr;   // set by moe_load_packed (contiguous layout)
     const uint8_t *scales_base = nullptr;
 };
@@ -40,7 +41,10 @@ namespace {
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct WsLayout {
-    size_t counters, logits, h, o, x16, x16_exp, total;
+    size_t counters, logits, h, o, x16, x16_exp;
+    size_t hand_seq, hand_ack, hand_ent;  // fused-layer routing handoff
+    size_t logit_ent;                     // fused-layer tagged logits
+    size_t total;
 };
 
 WsLayout ws_layout(const moe_ctx *c, int maxT) {
@@ -57,6 +61,10 @@ WsLayout ws_layout(const moe_ctx *c, int maxT) {
     L.o = take((size_t)maxT * c->k * c->H * 2);
     L.x16 = take((size_t)maxT * c->H * 2);
     L.x16_exp = take((size_t)maxT * sizeof(int));
+    L.hand_seq = take((size_t)moe::kHandMaxCtas * sizeof(unsigned));
+    L.hand_ack = take((size_t)moe::kHandMaxCtas * sizeof(unsigned));
+    L.hand_ent = take((size_t)moe::kHandMaxCtas * moe::kHandStride * 2 * sizeof(uint2));
+    L.logit_ent = take((size_t)moe::kDecodeMaxT * moe::kFusedMaxE * sizeof(uint2));
     L.total = off;
     return L;
 }
@@ -313,7 +321,7 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
         return MOE_ERR_ARG;
     for (int t0 = 0; t0 < T; t0 += chunk) {
         const int Tc = (T - t0 < chunk) ? T - t0 : chunk;
-        moe::GateUpParams g;
+        moe::GateUpParams g = {};
         g.table = h->d_table;
         g.codes_base = h->codes_base;
         g.scales_base = h->scales_base;
@@ -345,7 +353,7 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
             (rc = cuda_rc(moe::launch_gateup_decode(g, h->num_sms, s, h->use_pdl))) != MOE_OK)
             return rc;
 
-        moe::DownParams d;
+        moe::DownParams d = {};
         d.table = h->d_table;
         d.codes_base = h->codes_base;
         d.scales_base = h->scales_base;
@@ -417,6 +425,86 @@ int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
         return moe_forward_ex(h, norm ? x_norm : x, T, ids, w, residual, y, fwd_flags, stream);
     }
 
+    const bool keep = fwd_flags & MOE_FWD_KEEP_INTERMEDIATES;
+    const int G = h->num_sms;
+    size_t fsmem = 0;
+    int fslots = 0;
+    unsigned fregion = 0;
+    const int frows = (T * h->H + G - 1) / G;
+    if (h->fused_router && moe::layer_gateup_plan(T, h->E, h->H, G, &fsmem, &fslots, &fregion) &&
+        moe::down_decode_smem(T, h->k, h->I, frows) <= moe::kDownSmemMax) {
+        // router + gate/up in one launch, then the down kernel on the same grid
+        // size (the routing handoff is per CTA index)
+        moe::RouteHandoff hand;
+        hand.seq = reinterpret_cast<unsigned *>(h->ws + L.hand_seq);
+        hand.ack = reinterpret_cast<unsigned *>(h->ws + L.hand_ack);
+        hand.ent = reinterpret_cast<uint2 *>(h->ws + L.hand_ent);
+        moe::GateUpParams g = {};
+        g.table = h->d_table;
+        g.codes_base = h->codes_base;
+        g.scales_base = h->scales_base;
+        g.codes_stride = (size_t)h->I * h->H / 2;
+        g.scales_stride = (size_t)h->I * h->H / 32;
+        g.x = norm ? x_norm : x;
+        g.x16 = nullptr;
+        g.x16_exp = nullptr;
+        g.ids = nullptr;
+        g.logits = nullptr;
+        g.ids_out = topk_ids;
+        g.w_out = topk_w;
+        g.h = reinterpret_cast<uint16_t *>(h->ws + L.h);
+        g.status = h->d_status;
+        g.T = T;
+        g.k = h->k;
+        g.E = h->E;
+        g.H = h->H;
+        g.I = h->I;
+        g.prefetch_down = h->prefetch_down ? 1 : 0;
+        {
+            const size_t mc = (size_t)h->H * h->I / 2, ms = (size_t)h->H * h->I / 32;
+            g.pf_codes = (uint32_t)(((mc + G - 1) / G + 15) / 16 * 16);
+            g.pf_scales = (uint32_t)(((ms + G - 1) / G + 15) / 16 * 16);
+        }
+        g.nslots = fslots;
+        moe::FusedRouteParams fr;
+        fr.xr = x;
+        fr.wr = router_w;
+        fr.bias = router_bias;
+        fr.x_norm = norm ? x_norm : nullptr;
+        fr.logits_out = logits;
+        fr.logit_ent = reinterpret_cast<uint2 *>(h->ws + L.logit_ent);
+        fr.hand = hand;
+        fr.rmsnorm = norm ? 1 : 0;
+        fr.eps = 1e-6f;
+        fr.region_bytes = fregion;
+        if ((rc = cuda_rc(moe::launch_layer_gateup(g, fr, G, fsmem, s, h->use_pdl))) != MOE_OK)
+            return rc;
+        moe::DownParams d = {};
+        d.table = h->d_table;
+        d.codes_base = h->codes_base;
+        d.scales_base = h->scales_base;
+        d.codes_stride = g.codes_stride;
+        d.scales_stride = g.scales_stride;
+        d.h = g.h;
+        d.ids = nullptr;
+        d.w = nullptr;
+        d.logits = nullptr;
+        d.hand = hand;
+        d.residual = residual;
+        d.y = y;
+        d.o_keep = keep ? reinterpret_cast<uint16_t *>(h->ws + L.o) : nullptr;
+        d.status = h->d_status;
+        d.T = T;
+        d.k = h->k;
+        d.E = h->E;
+        d.H = h->H;
+        d.I = h->I;
+        d.rows_per_cta = frows;
+        if ((rc = cuda_rc(moe::launch_down_decode(d, G, s, h->use_pdl))) != MOE_OK) return rc;
+        h->kept = keep;
+        return MOE_OK;
+    }
+
     moe::RouteParams rp;
     rp.x = x;
     rp.wr = router_w;
@@ -437,8 +525,7 @@ int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
     rp.x16_exp = reinterpret_cast<int *>(h->ws + L.x16_exp);
     if ((rc = cuda_rc(moe::launch_route_logits(rp, s, h->use_pdl))) != MOE_OK) return rc;
 
-    const bool keep = fwd_flags & MOE_FWD_KEEP_INTERMEDIATES;
-    moe::GateUpParams g;
+    moe::GateUpParams g = {};
     g.table = h->d_table;
     g.codes_base = h->codes_base;
     g.scales_base = h->scales_base;
@@ -469,7 +556,7 @@ int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
     if ((rc = cuda_rc(moe::launch_gateup_decode(g, h->num_sms, s, h->use_pdl))) != MOE_OK)
         return rc;
 
-    moe::DownParams d;
+    moe::DownParams d = {};
     d.table = h->d_table;
     d.codes_base = h->codes_base;
     d.scales_base = h->scales_base;
@@ -528,6 +615,12 @@ int moe_set_tuning(moe_handle_t h, int use_pdl, int prefetch_down) {
     if (!h) return MOE_ERR_ARG;
     h->use_pdl = use_pdl != 0;
     h->prefetch_down = prefetch_down != 0;
+    return MOE_OK;
+}
+
+int moe_set_fusion(moe_handle_t h, int fused_router) {
+    if (!h) return MOE_ERR_ARG;
+    h->fused_router = fused_router != 0;
     return MOE_OK;
 }
 

@@ -286,14 +286,15 @@ __device__ __forceinline__ uint32_t logit_key(float v) {
 // (j < k) returns the j-th selection in (id, w); other lanes return id = -1.
 // Round j takes the warp-wide max key and the lowest id holding it, then
 // clears that key; k rounds, one redux pair each.
-template <int PER>  // logits per lane: E <= 32 * PER
+// SMEM: the logits are in shared memory (else global memory, read through L2).
+template <int PER, bool SMEM = false>  // logits per lane: E <= 32 * PER
 __device__ __forceinline__ void warp_topk(const float *lg, int E, int k, int lane, int &id,
                                           float &w) {
     uint32_t key[PER];
 #pragma unroll
     for (int m = 0; m < PER; ++m) {
         const int e = lane + 32 * m;
-        key[m] = e < E ? logit_key(__ldcg(lg + e)) : 0u;
+        key[m] = e < E ? logit_key(SMEM ? lg[e] : __ldcg(lg + e)) : 0u;
     }
     id = -1;
     float mylv = 0.f, top = 0.f;
@@ -328,18 +329,53 @@ __device__ __forceinline__ void warp_topk(const float *lg, int E, int k, int lan
 }
 
 // Larger expert counts: out of line, to keep the hot kernels' code small.
-static __device__ __noinline__ void warp_topk_wide(const float *lg, int E, int k, int lane,
-                                                   int &id, float &w) {
-    warp_topk<32>(lg, E, k, lane, id, w);
+// Returns {id, w bits} (by value: no local-memory outputs).
+template <bool SMEM>
+static __device__ __noinline__ uint2 warp_topk_wide(const float *lg, int E, int k, int lane) {
+    int id;
+    float w;
+    warp_topk<32, SMEM>(lg, E, k, lane, id, w);
+    return make_uint2((unsigned)id, __float_as_uint(w));
 }
 
 // Dispatch on E (up to 1024 experts).
+template <bool SMEM = false>
 __device__ __forceinline__ void warp_topk_any(const float *lg, int E, int k, int lane, int &id,
                                               float &w) {
     if (E <= 64)
-        warp_topk<2>(lg, E, k, lane, id, w);
-    else
-        warp_topk_wide(lg, E, k, lane, id, w);
+        warp_topk<2, SMEM>(lg, E, k, lane, id, w);
+    else {
+        const uint2 r = warp_topk_wide<SMEM>(lg, E, k, lane);
+        id = (int)r.x;
+        w = __uint_as_float(r.y);
+    }
+}
+
+// ------------------------------------------------------- gpu-scope words --
+// Relaxed gpu-scope accesses (through L2, coherent across SMs).
+
+__device__ __forceinline__ unsigned ld_relaxed_gpu(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_relaxed_gpu(unsigned *p, unsigned v) {
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// {a, b} as one 64-bit scalar access (a in the low word): naturally aligned,
+// it is single-copy atomic, so a reader sees both halves of one write.
+__device__ __forceinline__ void st_relaxed_gpu_v2(uint2 *p, unsigned a, unsigned b) {
+    asm volatile("{ .reg .b64 t; mov.b64 t, {%1, %2}; st.relaxed.gpu.global.b64 [%0], t; }" ::"l"(p),
+                 "r"(a), "r"(b)
+                 : "memory");
+}
+__device__ __forceinline__ uint2 ld_relaxed_gpu_v2(const uint2 *p) {
+    uint2 v;
+    asm volatile("{ .reg .b64 t; ld.relaxed.gpu.global.b64 t, [%2]; mov.b64 {%0, %1}, t; }"
+                 : "=r"(v.x), "=r"(v.y)
+                 : "l"(p)
+                 : "memory");
+    return v;
 }
 
 // ------------------------------------------- programmatic launch ---------

@@ -29,12 +29,10 @@
 #include <math.h>
 #include <stdint.h>
 
-#include "kernels.cuh"
+#include "gemv.cuh"
 
 namespace moe {
 
-constexpr int kGemvWarps = kGemvThreads / 32;
-constexpr int kDownWarps = kDownThreads / 32;
 
 // ------------------------------------------------------------------ route --
 // route_logits_kernel: grid (E, ceil(T / kRouteTokensPerCta)); CTA (e, b)
@@ -185,171 +183,6 @@ topk_kernel(const RouteParams p) {
     }
 }
 
-// One token's top-k by the calling warp into shared memory (ids) and,
-// optionally, global memory (ids_out, w_out).  Out of line.
-__device__ __noinline__ void topk_token_to_smem(const float *lg, int E, int k, int *s_ids,
-                                                int32_t *ids_out, float *w_out) {
-    const int lane = threadIdx.x & 31;
-    int id;
-    float w;
-    warp_topk_any(lg, E, k, lane, id, w);
-    if (lane < k) {
-        s_ids[lane] = id;
-        if (ids_out) ids_out[lane] = id;
-        if (w_out) w_out[lane] = w;
-    }
-}
-
-// Routing inside the expert kernels: warp t of the CTA selects for token t
-// (T <= kDecodeMaxT) into shared memory; CTA 0 also publishes ids / w.
-// Out of line (runs once per call).
-__device__ __noinline__ void route_into_smem(const float *logits, int T, int E, int k,
-                                                int *s_ids, float *s_w, int32_t *ids_out,
-                                                float *w_out) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (warp < T) {
-        int id;
-        float w;
-        warp_topk_any(logits + (size_t)warp * E, E, k, lane, id, w);
-        if (lane < k) {
-            s_ids[warp * k + lane] = id;
-            if (s_w) s_w[warp * k + lane] = w;
-            if (blockIdx.x == 0 && ids_out) ids_out[warp * k + lane] = id;
-            if (blockIdx.x == 0 && w_out) w_out[warp * k + lane] = w;
-        }
-    }
-}
-
-// ------------------------------------------------------------- team tools --
-// A "team" of TL lanes (TL a power of two, aligned in the warp) owns one packed
-// row at a time; lane lt of the team holds the KCH 16-byte chunks
-// c = lt + TL*u (u < KCH) of the row (one E8M0 group each) and the matching
-// FP16-staged activations in registers.  Teams are independent: their
-// shuffles use the team's own lane mask.
-
-template <int TL>
-__device__ __forceinline__ unsigned team_mask(int lane) {
-    return TL == 32 ? 0xffffffffu : (((1u << TL) - 1u) << (lane & ~(TL - 1)));
-}
-
-template <int TL>
-__device__ __forceinline__ float team_max(float v, unsigned mask) {
-#pragma unroll
-    for (int o = TL / 2; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(mask, v, o));
-    return v;
-}
-
-template <int TL>
-__device__ __forceinline__ float team_add(float v, unsigned mask) {
-#pragma unroll
-    for (int o = TL / 2; o > 0; o >>= 1) v += __shfl_xor_sync(mask, v, o);
-    return v;
-}
-
-// Load this lane's part of BF16 vector v (K elements), stage it as FP16 words
-// scaled by 2^-c where c comes from the team-wide max |v|; returns c.
-template <int TL, int KCH>
-__device__ __forceinline__ int stage_x(const uint16_t *v, int lt, int C, unsigned mask,
-                                       uint32_t (&xw)[KCH][16]) {
-    uint4 raw[KCH][4];
-    float m[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int u = 0; u < KCH; ++u) {
-        const int c = lt + TL * u;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            raw[u][q] = c < C ? *reinterpret_cast<const uint4 *>(v + (size_t)c * 32 + q * 8)
-                              : make_uint4(0u, 0u, 0u, 0u);
-            const uint32_t w4[4] = {raw[u][q].x, raw[u][q].y, raw[u][q].z, raw[u][q].w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                m[i] = fmaxf(m[i], fmaxf(fabsf(bf16_to_f32(w4[i] & 0xFFFFu)),
-                                         fabsf(bf16_to_f32(w4[i] >> 16))));
-        }
-    }
-    const int c = f16_stage_exponent(team_max<TL>(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), mask));
-    const float sf = pow2_neg(c);
-#pragma unroll
-    for (int u = 0; u < KCH; ++u)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint32_t w4[4] = {raw[u][q].x, raw[u][q].y, raw[u][q].z, raw[u][q].w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                xw[u][q * 4 + i] = f32x2_to_f16x2(bf16_to_f32(w4[i] & 0xFFFFu) * sf,
-                                                  bf16_to_f32(w4[i] >> 16) * sf);
-        }
-    return c;
-}
-
-template <int TL, int KCH>
-__device__ __forceinline__ void load_chunks(const uint8_t *codes, const uint8_t *scales, bool ok,
-                                            int lt, int C, uint4 (&cw)[KCH], uint32_t (&sc)[KCH]) {
-#pragma unroll
-    for (int u = 0; u < KCH; ++u) {
-        const int c = lt + TL * u;
-        if (ok && c < C) {
-            cw[u] = ld_stream16(codes + (size_t)c * 16);
-            sc[u] = ld_stream_u8(scales + c);
-        } else {
-            cw[u] = make_uint4(0u, 0u, 0u, 0u);
-            sc[u] = 127u;
-        }
-    }
-}
-
-template <int KCH>
-__device__ __forceinline__ float chunks_dot(const uint4 (&cw)[KCH], const uint32_t (&sc)[KCH],
-                                            const uint32_t (&xw)[KCH][16]) {
-    float acc = 0.f;
-#pragma unroll
-    for (int u = 0; u < KCH; ++u) {
-        float a0 = 0.f, a1 = 0.f;
-        dot8_e2m1_f16(cw[u].x, xw[u][0], xw[u][1], xw[u][2], xw[u][3], a0, a1);
-        dot8_e2m1_f16(cw[u].y, xw[u][4], xw[u][5], xw[u][6], xw[u][7], a0, a1);
-        dot8_e2m1_f16(cw[u].z, xw[u][8], xw[u][9], xw[u][10], xw[u][11], a0, a1);
-        dot8_e2m1_f16(cw[u].w, xw[u][12], xw[u][13], xw[u][14], xw[u][15], a0, a1);
-        acc = fmaf(a0 + a1, e8m0_to_f32(sc[u]), acc);
-    }
-    return acc;
-}
-
-// ----------------------------------------------------------- gate / up ----
-
-// L2 prefetch of this CTA's slice of the selected experts' down matrices, so
-// that the down GEMV that follows reads them from L2 while the DRAM keeps
-// streaming.  One lane per (token, slot) pair; an expert chosen by several
-// pairs is fetched by the lowest such lane only.  Slices are 16-byte multiples
-// computed on the host (codes: pf_codes bytes, scales: pf_scales bytes).
-__device__ __forceinline__ void prefetch_down_slice(const GateUpParams &p, const int *s_ids,
-                                                    int lane) {
-    const int P = p.T * p.k;
-    const int Pr = (P + 31) & ~31;  // every lane iterates the same number of times
-    #pragma unroll 1
-    for (int q = lane; q < Pr; q += 32) {
-        const int e = q < P ? s_ids[q] : -1;
-        const unsigned same = __match_any_sync(0xffffffffu, e);
-        const bool leader = (__ffs(same) - 1) == lane;
-        if (q < P && leader && e >= 0 && e < p.E) {
-            const size_t mc = (size_t)p.H * p.I / 2, ms = (size_t)p.H * p.I / 32;
-            const size_t oc = (size_t)blockIdx.x * p.pf_codes;
-            const size_t os = (size_t)blockIdx.x * p.pf_scales;
-            const uint8_t *dc = p.codes_base ? p.codes_base + (size_t)(3 * e + 2) * p.codes_stride
-                                             : p.table[e].codes[2];
-            const uint8_t *ds = p.codes_base ? p.scales_base + (size_t)(3 * e + 2) * p.scales_stride
-                                             : p.table[e].scales[2];
-            if (oc < mc) {
-                const size_t n = min((size_t)p.pf_codes, mc - oc);
-                prefetch_l2_bulk(dc + oc, (uint32_t)n);
-            }
-            if (os < ms) {
-                const size_t n = min((size_t)p.pf_scales, ms - os);
-                prefetch_l2_bulk(ds + os, (uint32_t)n);
-            }
-        }
-    }
-}
-
 // Items are (pair q = t*k + j, row i), q-major; each team owns a contiguous
 // range of items and processes two rows per step (gate and up of each).
 template <int TL, int KCH>
@@ -444,27 +277,10 @@ gateup_decode_kernel(const GateUpParams p) {
 }
 
 // ------------------------------------------------- gate / up, bulk copies --
-// The CTA owns items [cb, ce) (rows of the selected experts' gate and up
-// matrices, (pair, row) order).  A producer warp selects the experts (from
-// the router logits, or takes the given ids), then streams the CTA's rows into
-// a ring of shared-memory slots with bulk copies that complete on per-slot
-// mbarriers; slot s holds kTmaSlotRows consecutive items (gate codes,
-// up codes, gate scales, up scales).  For T = 1 the whole CTA range (~40
+// Rows of the selected experts stream into a shared-memory ring with bulk
+// copies (ring_produce / ring_consume).  For T = 1 the whole CTA range (~40
 // rows, ~90 KB) is requested at once, so the DRAM sees the layer's entire
-// gate/up stream immediately.  The consumer warps each take one row per
-// slot, decode it from shared memory against register-staged activations,
-// and release the slot.  Every wait is bounded; a timeout sets a status bit
-// and the kernel drains its outstanding copies before returning.
-
-constexpr int kTmaConsumers = 23;
-constexpr int kTmaThreads = (kTmaConsumers + 1) * 32;
-constexpr int kTmaSlotRows = kTmaConsumers;
-constexpr int kTmaMaxSlots = 16;
-constexpr size_t kTmaSmemBudget = 200 * 1024;
-
-__host__ __device__ __forceinline__ size_t tma_slot_bytes(int H) {
-    return (size_t)kTmaSlotRows * 2 * ((size_t)H / 2 + (size_t)H / 32);
-}
+// gate/up stream immediately.
 
 template <int KCH>
 __global__ void __launch_bounds__(kTmaThreads, 1)
@@ -475,40 +291,16 @@ gateup_tma_kernel(const GateUpParams p) {
     __shared__ int s_ids[kDecodeMaxT * kMaxTopK];
     __shared__ ExpertPtrs s_tab[kDecodeMaxT * kMaxTopK];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int H = p.H, I = p.I, k = p.k, T = p.T, E = p.E;
+    const int H = p.H, k = p.k, T = p.T, E = p.E;
     const int C = H >> 5;
-    const size_t rc = (size_t)H >> 1, rs = (size_t)H >> 5;
-    const size_t slot_bytes = tma_slot_bytes(H);
-    const size_t up_off = (size_t)kTmaSlotRows * rc;
-    const size_t gs_off = 2 * up_off, us_off = gs_off + (size_t)kTmaSlotRows * rs;
-    const int nslots = p.nslots;
-    // this CTA's items [cb, ce): 32-bit math (T * k * I <= 4 * 8 * 4096), the
-    // quotient computed in floating point and corrected
-    const int N = T * k * I;
-    const int G = (int)gridDim.x;
-    auto split = [&](int c) {
-        int v = (int)(((double)N * c) / G);
-        while ((long long)v * G > (long long)N * c) --v;
-        while ((long long)(v + 1) * G <= (long long)N * c) ++v;
-        return v;
-    };
-    const int cb = split((int)blockIdx.x), ce = split((int)blockIdx.x + 1);
-    const int nsteps = (ce - cb + kTmaSlotRows - 1) / kTmaSlotRows;
-    const int nbar = min(nslots, nsteps);
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < nbar; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kTmaConsumers);
-        }
-        mbar_fence_init();
-    }
+    const RingGeom g = ring_geom(p);
+    if (threadIdx.x == 0) ring_init(g, full, empty);
     __syncthreads();
     pdl_wait();  // x and the routing come from earlier kernels
     pdl_launch_dependents();
 
     if (warp == kTmaConsumers) {
-        // ---- producer warp ----
+        // ---- producer warp: the call's routing, then the ring ----
         const int P = T * k;
         if (p.ids) {
             #pragma unroll 1
@@ -521,123 +313,17 @@ gateup_tma_kernel(const GateUpParams p) {
                                    blockIdx.x == 0 ? p.w_out + (p.w_out ? t * k : 0) : nullptr);
         }
         __syncwarp();
-        #pragma unroll 1
-        for (int q = lane; q < P; q += 32) {
-            const int e = s_ids[q];
-            if (e >= 0 && e < E) {
-                if (p.codes_base) {
-                    ExpertPtrs ep;
-#pragma unroll
-                    for (int m = 0; m < 3; ++m) {
-                        ep.codes[m] = p.codes_base + (size_t)(3 * e + m) * p.codes_stride;
-                        ep.scales[m] = p.scales_base + (size_t)(3 * e + m) * p.scales_stride;
-                    }
-                    s_tab[q] = ep;
-                } else {
-                    s_tab[q] = p.table[e];
-                }
-            }
-        }
-        __syncwarp();
-        // Initial fill of the ring: one lane per (slot, pair segment, matrix)
-        // copy, all in one round; lane 8 s + 0 also announces slot s's bytes.
-        // Later slots reuse ring buffers and are issued by lane 0 in order.
-        const int nfill = min(nsteps, nslots);
-        #pragma unroll 1
-        for (int task = lane; task < 8 * nfill; task += 32) {
-            const int s = task >> 3, sub = task & 7, seg = sub >> 2, m = sub & 3;
-            const int r0 = cb + s * kTmaSlotRows;
-            const int r1 = min(ce, r0 + kTmaSlotRows);
-            const int qa = r0 / I, qb = (r1 - 1) / I;  // at most two pairs per slot
-            uint8_t *base = ring + (size_t)s * slot_bytes;
-            if (sub == 0) {
-                unsigned bytes = 0;
-                #pragma unroll 1
-                for (int q = qa; q <= qb; ++q) {
-                    const int e = s_ids[q];
-                    const int n = min(r1, (q + 1) * I) - max(r0, q * I);
-                    if (e >= 0 && e < E) bytes += (unsigned)(2 * n) * (unsigned)(rc + rs);
-                }
-                mbar_arrive_expect_tx(&full[s], bytes);
-            }
-            const int q = qa + seg;
-            if (q <= qb) {
-                const int e = s_ids[q];
-                const int a = max(r0, q * I);
-                const int n = min(r1, (q + 1) * I) - a;
-                if (e >= 0 && e < E) {
-                    const size_t idx = (size_t)(a - r0), i0 = (size_t)(a - q * I);
-                    const ExpertPtrs &ep = s_tab[q];
-                    const size_t dst = m == 0   ? idx * rc
-                                       : m == 1 ? up_off + idx * rc
-                                       : m == 2 ? gs_off + idx * rs
-                                                : us_off + idx * rs;
-                    const uint8_t *src = m == 0   ? ep.codes[0] + i0 * rc
-                                         : m == 1 ? ep.codes[1] + i0 * rc
-                                         : m == 2 ? ep.scales[0] + i0 * rs
-                                                  : ep.scales[1] + i0 * rs;
-                    const unsigned nb = (unsigned)(m < 2 ? n * rc : n * rs);
-                    bulk_g2s(base + dst, src, nb, &full[s]);
-                }
-            }
-        }
-        bool ok = true;
-        #pragma unroll 1
-        for (int s = nfill; s < nsteps && ok && lane == 0; ++s) {
-            const int b = s % nslots;
-            if (!mbar_wait(&empty[b], (unsigned)((s / nslots) - 1) & 1u)) {
-                atomicOr(p.status, kTimeoutStatus);
-                ok = false;
-                break;
-            }
-            uint8_t *base = ring + (size_t)b * slot_bytes;
-            const int r0 = cb + s * kTmaSlotRows;
-            const int r1 = min(ce, r0 + kTmaSlotRows);
-            const int qa = r0 / I, qb = (r1 - 1) / I;
-            unsigned bytes = 0;
-            #pragma unroll 1
-            for (int q = qa; q <= qb; ++q) {
-                const int e = s_ids[q];
-                const int n = min(r1, (q + 1) * I) - max(r0, q * I);
-                if (e >= 0 && e < E) bytes += (unsigned)(2 * n) * (unsigned)(rc + rs);
-            }
-            mbar_arrive_expect_tx(&full[b], bytes);
-            #pragma unroll 1
-            for (int q = qa; q <= qb; ++q) {
-                const int e = s_ids[q];
-                const int a = max(r0, q * I);
-                const int n = min(r1, (q + 1) * I) - a;
-                if (e >= 0 && e < E) {
-                    const size_t idx = (size_t)(a - r0), i0 = (size_t)(a - q * I);
-                    const ExpertPtrs &ep = s_tab[q];
-                    bulk_g2s(base + idx * rc, ep.codes[0] + i0 * rc, (unsigned)(n * rc), &full[b]);
-                    bulk_g2s(base + up_off + idx * rc, ep.codes[1] + i0 * rc, (unsigned)(n * rc),
-                             &full[b]);
-                    bulk_g2s(base + gs_off + idx * rs, ep.scales[0] + i0 * rs, (unsigned)(n * rs),
-                             &full[b]);
-                    bulk_g2s(base + us_off + idx * rs, ep.scales[1] + i0 * rs, (unsigned)(n * rs),
-                             &full[b]);
-                }
-            }
-        }
-        __syncwarp();
-        if (p.prefetch_down) prefetch_down_slice(p, s_ids, lane);
-        // no copy may still be in flight into this CTA's shared memory at exit
-        for (int s = max(0, nsteps - nbar) + lane; s < nsteps; s += 32)
-            mbar_wait(&full[s % nslots], (unsigned)(s / nslots) & 1u);
+        ring_produce(p, g, ring, full, empty, s_ids, s_tab, lane, [] {});
         return;
     }
 
-    // ---- consumer warps: one row per slot each ----
-    uint32_t xw[KCH][16];
-    int cur_tok = -1;
-    float xs = 1.f;
-    bool failed = false;
+    // ---- consumer warps ----
     // FP16 activations of token `tok` into registers: loaded as staged by the
     // router when available, else staged here.  Plain (L1-allocating) loads:
     // every warp of the CTA reads the same vector, so one L2 read per SM
     // serves all of them.
-    auto get_x = [&](int tok) {
+    ring_consume<KCH>(p, g, ring, full, empty, s_ids, warp, lane,
+                      [&](int tok, uint32_t (&xw)[KCH][16]) -> float {
         if (p.x16) {
             const uint32_t *xv = p.x16 + (size_t)tok * (H >> 1);
 #pragma unroll
@@ -653,66 +339,10 @@ gateup_tma_kernel(const GateUpParams p) {
                     xw[u][4 * q + 3] = v.w;
                 }
             }
-            xs = pow2(p.x16_exp[tok]);
-        } else {
-            xs = pow2(stage_x<32, KCH>(p.x + (size_t)tok * H, lane, C, 0xffffffffu, xw));
+            return pow2(p.x16_exp[tok]);
         }
-        cur_tok = tok;
-    };
-    #pragma unroll 1
-    for (int s = 0; s < nsteps; ++s) {
-        const int b = s % nslots;
-        const int row = cb + s * kTmaSlotRows + warp;
-        if (row < ce && !failed) {
-            // activations first: staging overlaps the slot's copies in flight
-            const int tok = (row / I) / k;
-            if (tok != cur_tok) get_x(tok);
-            if (!mbar_wait(&full[b], (unsigned)(s / nslots) & 1u)) {
-                failed = true;
-                if (lane == 0) atomicOr(p.status, kTimeoutStatus);
-            } else {
-                const int q = row / I;
-                const int i = row - q * I;
-                const int e = s_ids[q];
-                const bool bad = e < 0 || e >= E;
-                const uint8_t *base = ring + (size_t)b * slot_bytes;
-                uint4 cg[KCH], cu[KCH];
-                uint32_t sg[KCH], su[KCH];
-#pragma unroll
-                for (int u = 0; u < KCH; ++u) {
-                    const int c = lane + 32 * u;
-                    if (c < C && !bad) {
-                        cg[u] = *reinterpret_cast<const uint4 *>(base + (size_t)warp * rc + (size_t)c * 16);
-                        cu[u] = *reinterpret_cast<const uint4 *>(base + up_off + (size_t)warp * rc +
-                                                                (size_t)c * 16);
-                        sg[u] = base[gs_off + (size_t)warp * rs + c];
-                        su[u] = base[us_off + (size_t)warp * rs + c];
-                    } else {
-                        cg[u] = cu[u] = make_uint4(0u, 0u, 0u, 0u);
-                        sg[u] = su[u] = 127u;
-                    }
-                }
-                float ag = chunks_dot<KCH>(cg, sg, xw);
-                float au = chunks_dot<KCH>(cu, su, xw);
-                ag = warp_sum(ag);
-                au = warp_sum(au);
-                if (lane == 0) {
-                    uint16_t out = 0;
-                    if (!bad) {
-                        const float g = round_bf16(ag * xs);
-                        const float uu = round_bf16(au * xs);
-                        const float sl = round_bf16(g / (1.0f + expf(-g)));
-                        out = f32_to_bf16(sl * uu);
-                    } else {
-                        atomicOr(p.status, kBadExpertId);
-                    }
-                    p.h[(size_t)q * I + i] = out;
-                }
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[b]);
-    }
+        return pow2(stage_x<32, KCH>(p.x + (size_t)tok * H, lane, C, 0xffffffffu, xw));
+    });
 }
 
 // ---------------------------------------------------------------- down -----
@@ -778,6 +408,37 @@ __device__ __noinline__ void stage_h_block(const uint16_t *h, int P, int I, uint
     __syncthreads();
 }
 
+// Routing handed over by CTA blockIdx.x of the fused router + gate/up kernel
+// of the same call (RouteHandoff), by one warp: lane q < P polls (bounded) its
+// two tagged entries until both carry the expected tag; lane 0 acknowledges.
+// A timeout flags the status, marks the slots invalid (id -1: zero output)
+// and resynchronises the acknowledgement.  Out of line.
+static __device__ __noinline__ void take_handoff(const RouteHandoff h, int P, int *s_ids,
+                                                 float *s_w, unsigned *status) {
+    const int lane = threadIdx.x & 31;
+    const int slot = (int)blockIdx.x;
+    const unsigned want = ld_relaxed_gpu(h.ack + slot) + 1u;
+    bool ok = true;
+    if (lane < P) {
+        const uint2 *e = h.ent + ((size_t)slot * kHandStride + lane) * 2;
+        uint2 a = make_uint2(0u, 0u), b = make_uint2(0u, 0u);
+        ok = false;
+        #pragma unroll 1
+        for (int i = 0; i < kMaxSpin && !ok; ++i) {
+            a = ld_relaxed_gpu_v2(e);
+            b = ld_relaxed_gpu_v2(e + 1);
+            ok = a.x == want && b.x == want;
+        }
+        s_ids[lane] = ok ? (int)a.y : -1;
+        s_w[lane] = ok ? __uint_as_float(b.y) : 0.f;
+    }
+    const bool all_ok = __all_sync(0xffffffffu, ok);
+    if (lane == 0) {
+        if (!all_ok) atomicOr(status, kTimeoutStatus);
+        st_relaxed_gpu(h.ack + slot, all_ok ? want : ld_relaxed_gpu(h.seq + slot));
+    }
+}
+
 __device__ __forceinline__ const uint8_t *down_codes(const DownParams &p, int e) {
     return p.codes_base ? p.codes_base + (size_t)(3 * e + 2) * p.codes_stride : p.table[e].codes[2];
 }
@@ -786,7 +447,57 @@ __device__ __forceinline__ const uint8_t *down_scales(const DownParams &p, int e
                         : p.table[e].scales[2];
 }
 
-template <int TL, int KCH>
+// Shared-memory offset of the down rows (after the staged h and the expert
+// outputs), 16-byte aligned for the bulk copies.
+__host__ __device__ __forceinline__ size_t down_rows_offset(int T, int k, int I, int R) {
+    return ((size_t)T * k * I * 2 + (size_t)k * R * 4 + 15) & ~(size_t)15;
+}
+
+// By one thread: the CTA's down rows [r0, r1) of every slot into shared memory
+// (one bulk copy per slot, token segment and codes / scales), completing on
+// *bar; rows of an invalid expert id are not fetched.  Out of line.
+static __device__ __noinline__ void issue_down_rows(const ExpertPtrs *table,
+                                                    const uint8_t *codes_base,
+                                                    const uint8_t *scales_base, size_t cstride,
+                                                    size_t sstride, int E, int H, int I, int k,
+                                                    const int *s_ids, int r0, int r1, int R,
+                                                    uint8_t *rows_c, uint8_t *rows_s,
+                                                    uint64_t *bar) {
+    const size_t rc = (size_t)I >> 1, rs = (size_t)I >> 5;
+    unsigned bytes = 0;
+    #pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+        if (pass == 1) mbar_arrive_expect_tx(bar, bytes);
+        #pragma unroll 1
+        for (int a = r0; a < r1;) {
+            const int t = a / H;
+            const int b = min(r1, (t + 1) * H);
+            const size_t n0 = (size_t)(a - t * H), cnt = (size_t)(b - a);
+            #pragma unroll 1
+            for (int j = 0; j < k; ++j) {
+                const int e = s_ids[t * k + j];
+                if (e < 0 || e >= E) continue;
+                if (pass == 0) {
+                    bytes += (unsigned)(cnt * (rc + rs));
+                } else {
+                    const size_t li = (size_t)j * R + (size_t)(a - r0);
+                    const uint8_t *dc = codes_base ? codes_base + (size_t)(3 * e + 2) * cstride
+                                                   : table[e].codes[2];
+                    const uint8_t *ds = codes_base ? scales_base + (size_t)(3 * e + 2) * sstride
+                                                   : table[e].scales[2];
+                    bulk_g2s(rows_c + li * rc, dc + n0 * rc, (unsigned)(cnt * rc), bar);
+                    bulk_g2s(rows_s + li * rs, ds + n0 * rs, (unsigned)(cnt * rs), bar);
+                }
+            }
+            a = b;
+        }
+    }
+}
+
+// SR: every down row of the CTA is copied into shared memory with bulk copies
+// before the programmatic-launch wait (rows: [k][R] codes, then [k][R] scales);
+// otherwise each team streams its rows from global memory two at a time.
+template <int TL, int KCH, bool SR>
 __global__ void __launch_bounds__(kDownThreads, 1)
 down_decode_kernel(const DownParams p) {
     extern __shared__ __align__(16) uint8_t sm[];
@@ -803,6 +514,9 @@ down_decode_kernel(const DownParams p) {
     const int P = T * k;
     uint32_t *sh = reinterpret_cast<uint32_t *>(sm);                       // [P][I/2] FP16 words
     float *so = reinterpret_cast<float *>(sm + (size_t)P * I * 2);         // [k][R]
+    uint8_t *rows_c = sm + down_rows_offset(T, k, I, R);                   // SR: [k][R][I/2]
+    uint8_t *rows_s = rows_c + (size_t)k * R * rc;                          // SR: [k][R][I/32]
+    __shared__ __align__(8) uint64_t s_rbar;
     __shared__ int s_ids[kDecodeMaxT * kMaxTopK];
     __shared__ float s_w[kDecodeMaxT * kMaxTopK];
     __shared__ float s_xs[kDecodeMaxT * kMaxTopK];
@@ -816,13 +530,19 @@ down_decode_kernel(const DownParams p) {
 
     // routing for this call's tokens
     if (threadIdx.x < P) s_hmax[threadIdx.x] = 0u;
+    if (SR && threadIdx.x == 0) {
+        mbar_init(&s_rbar, 1);
+        mbar_fence_init();
+    }
     if (p.ids) {
         for (int q = threadIdx.x; q < P; q += kDownThreads) {
             s_ids[q] = __ldcg(p.ids + q);
             s_w[q] = __ldcg(p.w + q);
         }
-    } else {
+    } else if (p.logits) {
         route_into_smem(p.logits, T, p.E, k, s_ids, s_w, nullptr, nullptr);
+    } else if (warp == 0) {
+        take_handoff(p.hand, P, s_ids, s_w, p.status);
     }
     __syncthreads();
 
@@ -841,24 +561,52 @@ down_decode_kernel(const DownParams p) {
             const int e = valid ? s_ids[t * k + j] : 0;
             bad[u] = valid && (e < 0 || e >= p.E);
             const bool ok = valid && !bad[u];
-            const uint8_t *dc = nullptr, *ds = nullptr;
-            if (ok) {
-                dc = down_codes(p, e) + (size_t)n * rc;
-                ds = down_scales(p, e) + (size_t)n * rs;
+            if (SR) {
+                const size_t li = (size_t)j * R + (size_t)(r - r0);
+                const uint8_t *dc = rows_c + li * rc, *ds = rows_s + li * rs;
+#pragma unroll
+                for (int v = 0; v < KCH; ++v) {
+                    const int c = lt + TL * v;
+                    if (ok && c < C) {
+                        cw[u][v] = *reinterpret_cast<const uint4 *>(dc + (size_t)c * 16);
+                        sc[u][v] = ds[c];
+                    } else {
+                        cw[u][v] = make_uint4(0u, 0u, 0u, 0u);
+                        sc[u][v] = 127u;
+                    }
+                }
+            } else {
+                const uint8_t *dc = nullptr, *ds = nullptr;
+                if (ok) {
+                    dc = down_codes(p, e) + (size_t)n * rc;
+                    ds = down_scales(p, e) + (size_t)n * rs;
+                }
+                load_chunks<TL, KCH>(dc, ds, ok, lt, C, cw[u], sc[u]);
             }
-            load_chunks<TL, KCH>(dc, ds, ok, lt, C, cw[u], sc[u]);
         }
     };
-    fetch(rr);
+    if (SR) {
+        if (threadIdx.x == 0)
+            issue_down_rows(p.table, p.codes_base, p.scales_base, p.codes_stride, p.scales_stride,
+                            p.E, H, I, k, s_ids, r0, r1, R, rows_c, rows_s, &s_rbar);
+    } else {
+        fetch(rr);
+    }
 
     pdl_wait();  // h comes from the gate/up kernel
     pdl_launch_dependents();
 
     // stage every h[t][j] once into shared memory as FP16
     stage_h_block(p.h, P, I, sh, s_xs, s_hmax);
+    bool rows_ok = true;
+    if (SR) {
+        rows_ok = __syncthreads_and(mbar_wait(&s_rbar, 0u)) != 0;  // uniform over the CTA
+        if (!rows_ok && threadIdx.x == 0) atomicOr(p.status, kTimeoutStatus);
+        if (rows_ok) fetch(rr);
+    }
 
     #pragma unroll 1
-    while (worker && rr < r1) {
+    while (worker && rows_ok && rr < r1) {
         const int t = rr / H;
         const uint32_t *xv = sh + (size_t)(t * k + j) * (I >> 1);
         const float xs = s_xs[t * k + j];
@@ -916,6 +664,8 @@ down_decode_kernel(const DownParams p) {
         if (p.residual) y = round_bf16(bf16_to_f32(p.residual[r]) + y);
         p.y[r] = f32_to_bf16(y);
     }
+    // no row copy may outlive the CTA (complete unless its wait timed out)
+    if (SR && !rows_ok && threadIdx.x == 0) mbar_wait(&s_rbar, 0u);
 }
 
 // --------------------------------------------------------------- debug -----
@@ -943,22 +693,6 @@ __global__ void debug_dequant_kernel(const uint8_t *codes, const uint8_t *scales
 
 namespace {
 
-template <typename... KArgs, typename... Args>
-cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                      cudaStream_t s, bool pdl, Args &&...args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
-}
-
 // (TL, KCH) for K/32 = C chunks per row: a team of TL lanes, KCH chunks per lane.
 void pick_team(int C, int &TL, int &KCH) {
     const int tls[4] = {32, 16, 8, 4};
@@ -978,19 +712,31 @@ cudaError_t launch_gu(const GateUpParams &p, int grid, cudaStream_t s, bool pdl)
     return launch_ex(gateup_decode_kernel<TL, KCH>, dim3(grid), dim3(kGemvThreads), 0, s, pdl, p);
 }
 
-template <int TL, int KCH>
-cudaError_t launch_dn(const DownParams &p, int grid, cudaStream_t s, bool pdl) {
+template <int TL, int KCH, bool SR>
+cudaError_t launch_dn_v(const DownParams &p, int grid, size_t smem, cudaStream_t s, bool pdl) {
     static bool attr_set = false;
-    const size_t smem = down_decode_smem(p.T, p.k, p.I, p.rows_per_cta);
-    if (smem > kDownSmemMax) return cudaErrorInvalidValue;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(down_decode_kernel<TL, KCH>,
+        cudaError_t e = cudaFuncSetAttribute(down_decode_kernel<TL, KCH, SR>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kDownSmemMax);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    return launch_ex(down_decode_kernel<TL, KCH>, dim3(grid), dim3(kDownThreads), smem, s, pdl, p);
+    return launch_ex(down_decode_kernel<TL, KCH, SR>, dim3(grid), dim3(kDownThreads), smem, s, pdl,
+                     p);
+}
+
+// The shared-memory-rows variant when its copies are 16-byte shaped (I a
+// multiple of 512) and the rows fit; else rows stream from global memory.
+template <int TL, int KCH>
+cudaError_t launch_dn(const DownParams &p, int grid, cudaStream_t s, bool pdl) {
+    const size_t smem = down_decode_smem(p.T, p.k, p.I, p.rows_per_cta);
+    if (smem > kDownSmemMax) return cudaErrorInvalidValue;
+    const size_t smem_sr = down_rows_offset(p.T, p.k, p.I, p.rows_per_cta) +
+                           (size_t)p.k * p.rows_per_cta * ((size_t)p.I / 2 + (size_t)p.I / 32);
+    if (p.I % 512 == 0 && smem_sr <= kDownSmemMax)
+        return launch_dn_v<TL, KCH, true>(p, grid, smem_sr, s, pdl);
+    return launch_dn_v<TL, KCH, false>(p, grid, smem, s, pdl);
 }
 
 #define MOE_TEAM_DISPATCH(FN, C, ...)                                   \

@@ -54,6 +54,37 @@ struct GateUpParams {
     int nslots;               // shared-memory ring slots of the bulk-copy kernel
 };
 
+// Routing handed from the fused router + gate/up kernel to the down kernel of
+// the same call, one copy per CTA index i (both grids have the same size).
+// Every entry is an 8-byte word {tag, value} written and read as one access,
+// so a reader that sees the expected tag also sees the value: gate/up CTA i
+// writes its ids / w with tag seq[i] + 1 and then stores seq[i] + 1; down CTA
+// i polls (bounded) until its entries carry ack[i] + 1, then stores that in
+// ack[i].  Between calls seq[i] == ack[i].  The down kernel can thus route
+// before its programmatic-launch wait without relying on that wait.
+constexpr int kHandMaxCtas = 256;
+constexpr int kHandStride = kDecodeMaxT * kMaxTopK;
+struct RouteHandoff {
+    unsigned *seq;   // [kHandMaxCtas] publications made by gate/up CTA i
+    unsigned *ack;   // [kHandMaxCtas] publications taken by down CTA i
+    uint2 *ent;      // [kHandMaxCtas][kHandStride][2]: {tag, id}, {tag, w bits}
+};
+
+// Router half of the fused router + gate/up launch.
+constexpr int kFusedMaxE = 256;  // experts of the fused router (E/2 per CTA)
+struct FusedRouteParams {
+    const uint16_t *xr;      // [T][H] layer input (the residual stream when rmsnorm)
+    const uint16_t *wr;      // [E][H] BF16 router
+    const float *bias;       // [E] or null
+    uint16_t *x_norm;        // [T][H] written when rmsnorm (CTA 0)
+    float *logits_out;       // [T][E] or null
+    uint2 *logit_ent;        // [T][E] {tag, logit bits}: CTA e % G publishes expert e
+    RouteHandoff hand;
+    int rmsnorm;
+    float eps;
+    unsigned region_bytes;   // dynamic shared memory before the routed-vector buffer
+};
+
 struct DownParams {
     const ExpertPtrs *table;
     const uint8_t *codes_base, *scales_base;  // contiguous layout fast path (or null)
@@ -68,6 +99,7 @@ struct DownParams {
     unsigned *status;
     int T, k, E, H, I;
     int rows_per_cta;
+    RouteHandoff hand;         // used when ids and logits are both null
 };
 
 // Host-side launchers (decode.cu).  `pdl` sets programmatic stream
@@ -79,6 +111,12 @@ bool gateup_tma_supported(int H);
 int gateup_tma_slots(int H);
 cudaError_t launch_gateup_decode(const GateUpParams &p, int grid, cudaStream_t s, bool pdl);
 cudaError_t launch_down_decode(const DownParams &p, int grid, cudaStream_t s, bool pdl);
+// Fused router + gate/up (layer.cu): one CTA per SM, grid = SM count.  layer_gateup_plan returns the dynamic shared memory and
+// ring slots for (T, E, H), or false when the shape needs the unfused path.
+bool layer_gateup_plan(int T, int E, int H, int grid, size_t *smem, int *nslots,
+                       unsigned *region_bytes);
+cudaError_t launch_layer_gateup(const GateUpParams &p, const FusedRouteParams &r, int grid,
+                                size_t smem, cudaStream_t s, bool pdl);
 cudaError_t launch_debug_dequant(const uint8_t *codes, const uint8_t *scales, int64_t n,
                                  float *out, cudaStream_t s);
 size_t gateup_decode_smem(int T, int H);

@@ -115,7 +115,7 @@ extern "C" int moe_forward_noalloc(int E, int H, int I, int top_k, const uint8_t
         return MOE_ERR_ARG;
     for (int t0 = 0; t0 < T; t0 += chunk) {
         const int Tc = (T - t0 < chunk) ? T - t0 : chunk;
-        moe::GateUpParams g;
+        moe::GateUpParams g = {};
         g.table = d_table;
         g.codes_base = codes_u8;
         g.scales_base = scales_e8m0;
@@ -143,7 +143,7 @@ extern "C" int moe_forward_noalloc(int E, int H, int I, int top_k, const uint8_t
             cudaGetLastError();
             return MOE_ERR_CUDA;
         }
-        moe::DownParams d;
+        moe::DownParams d = {};
         d.table = d_table;
         d.codes_base = codes_u8;
         d.scales_base = scales_e8m0;

@@ -160,8 +160,10 @@ def test_tokens_beyond_decode_chunk():
     layer.close()
 
 
-def test_invalid_ids_zero_the_slot_and_flag():
-    shape = synth.TINY
+@pytest.mark.parametrize("shape", [synth.TINY, synth.L24B])
+def test_invalid_ids_zero_the_slot_and_flag(shape):
+    """TINY streams down rows from global memory, L24B copies them into shared
+    memory first (rows of an invalid id are not fetched there)."""
     L, x, layer = make(shape, 4, 2)
     ids_h = np.array([[3, 99, 5, -1], [0, 1, 2, 3]], dtype=np.int32)
     w_h = np.array([[0.4, 0.3, 0.2, 0.1], [0.25] * 4], dtype=np.float32)
