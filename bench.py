@@ -52,6 +52,9 @@ def parse_args():
     ap.add_argument("--no-pdl", action="store_true")
     ap.add_argument("--no-prefetch", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=N_LAYERS,
+                    help="layers in the stack (fewer: a smaller case for profiling; "
+                         "the bench workload is the full stack)")
     return ap.parse_args()
 
 
@@ -100,7 +103,7 @@ def csrc_digest():
 def stored_traffic():
     """DRAM bytes per gate/up launch from the committed ncu summary, if it was
     taken from the current kernel sources; else None."""
-    p = os.path.join(ROOT, "profiles", "gateup_decode_traffic.json")
+    p = os.path.join(ROOT, "profiles", "gateup_tma_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
@@ -235,13 +238,13 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ ours
 
-def build_stack(torch, moe, seed):
+def build_stack(torch, moe, seed, n_layers):
     def gen(l):
         return synth.make_layer(SHAPE, seed=seed, layer=l)
 
     weights = []
     with ThreadPoolExecutor(4) as ex:
-        for L in ex.map(gen, range(N_LAYERS)):
+        for L in ex.map(gen, range(n_layers)):
             codes = torch.from_numpy(L.codes).cuda()
             scales = torch.from_numpy(L.scales).cuda()
             rw = torch.from_numpy(L.router_w.view(np.int16)).cuda().view(torch.bfloat16)
@@ -266,7 +269,8 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    st = build_stack(torch, moe, seed=args.seed + rank)
+    n_layers = args.layers
+    st = build_stack(torch, moe, seed=args.seed + rank, n_layers=n_layers)
     st.set_tuning(use_pdl=not args.no_pdl, prefetch_down=not args.no_prefetch)
     x0 = torch.from_numpy(synth.make_tokens(1, SHAPE.H, seed=args.seed + rank, stream=3)
                           .view(np.int16)).cuda().view(torch.bfloat16)
@@ -304,7 +308,7 @@ def run_ours(args):
     # bytes per token from the routing of the last replay (distinct experts)
     ids = st.ids.cpu().numpy()
     step_bytes = sum(bytes_per_layer(SHAPE, len(set(ids[l].ravel().tolist())), 1)
-                     for l in range(N_LAYERS))
+                     for l in range(n_layers))
     gbs = step_bytes * TOKENS_PER_STEP * args.steps / (t_ms / 1e3) / 1e9
     peak, peak_kind = load_peaks()
 
@@ -322,7 +326,9 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": t_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "e2m1xbf16->f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "layers": N_LAYERS, "T": 1, "E": SHAPE.E,
+        "config": {"workload": WORKLOAD if n_layers == N_LAYERS else
+                   WORKLOAD.replace(f"{N_LAYERS} MoE layers", f"{n_layers} MoE layers"),
+                   "layers": n_layers, "T": 1, "E": SHAPE.E,
                    "H": SHAPE.H, "I": SHAPE.I, "top_k": SHAPE.top_k,
                    "tokens_per_step": TOKENS_PER_STEP, "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (12.19 GB resident, 0.77 GB streamed per token "
@@ -331,13 +337,13 @@ def run_ours(args):
         "hbm_gbs": gbs, "hbm_frac": gbs / peak, "hbm_peak_gbs": peak,
         "hbm_peak_kind": peak_kind, "bytes_per_token": step_bytes,
         "us_per_token": t_ms * 1e3 / (TOKENS_PER_STEP * args.steps),
-        "roofline": {"bound": "hbm", "kernel": "gateup_decode_kernel",
+        "roofline": {"bound": "hbm", "kernel": "gateup_tma_kernel",
                      "achieved": gu_gbs, "peak": peak, "unit": "GB/s",
                      "frac": gu_gbs / peak, "traffic": stored_traffic(),
                      "bytes_per_launch": gu_bytes, "peak_kind": peak_kind},
         "kernels": kern,
         "e2e": e2e,
-        "gpu_launches": 3 * N_LAYERS * TOKENS_PER_STEP * args.steps,
+        "gpu_launches": 3 * n_layers * TOKENS_PER_STEP * args.steps,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
