@@ -240,17 +240,27 @@ MOE_API int moe_bytes_per_expert(moe_handle_t h, size_t *bytes);
  * while it streams gate/up.  Errors: ARG. */
 MOE_API int moe_set_tuning(moe_handle_t h, int use_pdl, int prefetch_down);
 
-/* Launch structure of moe_layer_ex for T <= 4 (off by default; results are
- * bit-identical either way): fused_router != 0 computes the RMSNorm, the
- * router logits and the top-k inside the gate/up launch (one CTA per SM;
- * the CTA of index e publishes expert e's logit to the others through the
- * workspace) and hands the routing to the down launch
- * through the workspace; 0 runs a separate router launch first.  Shapes the
- * fused launch cannot hold (E > 256, H not a multiple of 512 or above 4096)
- * use the separate launch regardless.  The workspace carries call counters
- * for this: one workspace must not serve two calls at the same time.
- * Errors: ARG. */
-MOE_API int moe_set_fusion(moe_handle_t h, int fused_router);
+/* Launch structure of moe_layer_ex for T <= 4; results are bit-identical
+ * in every mode:
+ *   MOE_FUSION_NONE (default): a router launch, the gate/up launch, the down
+ *     launch;
+ *   MOE_FUSION_ROUTER: the RMSNorm, the router logits and the top-k run
+ *     inside the gate/up launch (one CTA per SM; the CTA of index e
+ *     publishes expert e's logit to the others through the workspace), and
+ *     the routing reaches the down launch through the workspace;
+ *   MOE_FUSION_LAYER: the whole layer in one launch (the down phase waits,
+ *     bounded, for every CTA's gate/up through per-CTA words in the
+ *     workspace).
+ * A mode falls back to the next simpler one for shapes it cannot hold in
+ * shared memory (LAYER: H <= 2048, I a multiple of 512 and small T; ROUTER:
+ * E <= 256, H a multiple of 512 up to 4096) and LAYER also when
+ * MOE_FWD_KEEP_INTERMEDIATES is asked.  The workspace carries per-call
+ * counters for the fused modes: one workspace must not serve two calls at
+ * the same time.  Errors: ARG (unknown mode). */
+#define MOE_FUSION_NONE 0
+#define MOE_FUSION_ROUTER 1
+#define MOE_FUSION_LAYER 2
+MOE_API int moe_set_fusion(moe_handle_t h, int mode);
 
 /* ---------------------------------------------------------------------
  * Forward without any device allocation.  No counterpart in the paper: this

@@ -29,6 +29,7 @@ __all__ = [
     "moe_forward_noalloc",
     "ROUTE_RMSNORM", "FWD_KEEP_INTERMEDIATES", "FWD_FORCE_DECODE", "FWD_FORCE_GROUPED",
     "FWD_PHASE_GATEUP", "FWD_PHASE_DOWN",
+    "FUSION_NONE", "FUSION_ROUTER", "FUSION_LAYER", "moe_set_fusion",
     "DEVICE_BAD_EXPERT_ID",
 ]
 
@@ -38,6 +39,7 @@ FWD_FORCE_DECODE = 0x2
 FWD_FORCE_GROUPED = 0x4
 FWD_PHASE_GATEUP = 0x8
 FWD_PHASE_DOWN = 0x10
+FUSION_NONE, FUSION_ROUTER, FUSION_LAYER = 0, 1, 2
 DEVICE_BAD_EXPERT_ID = 0x1
 DEVICE_TIMEOUT = 0x2
 
@@ -173,8 +175,8 @@ def moe_set_tuning(h: int, use_pdl: bool, prefetch_down: bool) -> None:
     check("moe_set_tuning", load().moe_set_tuning(C.c_void_p(h), int(use_pdl), int(prefetch_down)))
 
 
-def moe_set_fusion(h: int, fused_router: bool) -> None:
-    check("moe_set_fusion", load().moe_set_fusion(C.c_void_p(h), int(fused_router)))
+def moe_set_fusion(h: int, mode: int) -> None:
+    check("moe_set_fusion", load().moe_set_fusion(C.c_void_p(h), int(mode)))
 
 
 def moe_device_check() -> None:
@@ -309,6 +311,11 @@ class MoEStack:
     def set_tuning(self, use_pdl=True, prefetch_down=True):
         for L in self.layers:
             moe_set_tuning(L.handle, use_pdl, prefetch_down)
+
+    def set_fusion(self, mode):
+        """Launch structure of every layer (FUSION_NONE / _ROUTER / _LAYER)."""
+        for L in self.layers:
+            moe_set_fusion(L.handle, mode)
 
     def enqueue(self, stream=None):
         """Enqueue one decode step (all layers) on `stream`."""

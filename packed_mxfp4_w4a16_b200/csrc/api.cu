@@ -31,7 +31,7 @@ struct moe_ctx {
     bool kept = false;                    // last forward kept intermediates
     bool use_pdl = true;
     bool prefetch_down = true;
-    bool fused_router = false;            // moe_layer_ex: router inside the gate/up launch
+    int fusion = 0;                       // moe_layer_ex launch structure (moe_set_fusion)
     const uint8_t *codes_base = nullptr;   // set by moe_load_packed (contiguous layout)
     const uint8_t *scales_base = nullptr;
 };
@@ -44,6 +44,8 @@ struct WsLayout {
     size_t counters, logits, h, o, x16, x16_exp;
     size_t hand_seq, hand_ack, hand_ent;  // fused-layer routing handoff
     size_t logit_ent;                     // fused-layer tagged logits
+    size_t h_tag;                         // one-launch layer: tagged h
+    size_t perm, offs, h16, h_exp;        // grouped path: sorted pairs, staged h
     size_t total;
 };
 
@@ -65,6 +67,11 @@ WsLayout ws_layout(const moe_ctx *c, int maxT) {
     L.hand_ack = take((size_t)moe::kHandMaxCtas * sizeof(unsigned));
     L.hand_ent = take((size_t)moe::kHandMaxCtas * moe::kHandStride * 2 * sizeof(uint2));
     L.logit_ent = take((size_t)moe::kDecodeMaxT * moe::kFusedMaxE * sizeof(uint2));
+    L.h_tag = take((size_t)maxT * c->k * c->I * sizeof(uint2));
+    L.perm = take((size_t)maxT * c->k * sizeof(int));
+    L.offs = take((size_t)(c->E + 1) * sizeof(int));
+    L.h16 = take((size_t)maxT * c->k * c->I * 2);
+    L.h_exp = take((size_t)maxT * c->k * sizeof(int));
     L.total = off;
     return L;
 }
@@ -308,6 +315,48 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
     uint16_t *hbuf = reinterpret_cast<uint16_t *>(h->ws + L.h);
     uint16_t *obuf = reinterpret_cast<uint16_t *>(h->ws + L.o);
 
+    // (token, expert)-sorted grouped path on the tensor cores: batches beyond
+    // the decode sizes, or when asked (the phase flags time the decode path)
+    const bool phase = flags & (MOE_FWD_PHASE_GATEUP | MOE_FWD_PHASE_DOWN);
+    const bool grouped = !phase && !(flags & MOE_FWD_FORCE_DECODE) &&
+                         (T > moe::kDecodeMaxT || (flags & MOE_FWD_FORCE_GROUPED)) &&
+                         moe::grouped_supported(h->E, h->H, h->I);
+    if ((flags & MOE_FWD_FORCE_GROUPED) && !grouped) return MOE_ERR_ARG;
+    if (grouped) {
+        for (int t0 = 0; t0 < T; t0 += moe::kGroupedMaxT) {
+            const int Tc = (T - t0 < moe::kGroupedMaxT) ? T - t0 : moe::kGroupedMaxT;
+            moe::GroupedParams gp = {};
+            gp.table = h->d_table;
+            gp.codes_base = h->codes_base;
+            gp.scales_base = h->scales_base;
+            gp.codes_stride = (size_t)h->I * h->H / 2;
+            gp.scales_stride = (size_t)h->I * h->H / 32;
+            gp.x = x + (size_t)t0 * h->H;
+            gp.ids = topk_ids + (size_t)t0 * h->k;
+            gp.w = topk_w + (size_t)t0 * h->k;
+            gp.residual = residual ? residual + (size_t)t0 * h->H : nullptr;
+            gp.y = y + (size_t)t0 * h->H;
+            gp.o_keep = nullptr;  // o itself lands in the workspace buffer kept below
+            gp.perm = reinterpret_cast<int *>(h->ws + L.perm);
+            gp.offs = reinterpret_cast<int *>(h->ws + L.offs);
+            gp.x16 = reinterpret_cast<uint32_t *>(h->ws + L.x16);
+            gp.x_exp = reinterpret_cast<int *>(h->ws + L.x16_exp);
+            gp.h = hbuf + (size_t)t0 * h->k * h->I;
+            gp.h16 = reinterpret_cast<uint32_t *>(h->ws + L.h16);
+            gp.h_exp = reinterpret_cast<int *>(h->ws + L.h_exp);
+            gp.o = obuf + (size_t)t0 * h->k * h->H;
+            gp.status = h->d_status;
+            gp.T = Tc;
+            gp.k = h->k;
+            gp.E = h->E;
+            gp.H = h->H;
+            gp.I = h->I;
+            if ((rc = cuda_rc(moe::launch_grouped(gp, s, h->use_pdl))) != MOE_OK) return rc;
+        }
+        h->kept = keep;
+        return MOE_OK;
+    }
+
     // per-(token, slot) GEMV path, in chunks of up to kDecodeMaxT tokens (fewer
     // when the staged activations of a chunk would not fit in shared memory)
     int chunk = moe::kDecodeMaxT;
@@ -431,8 +480,14 @@ int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
     int fslots = 0;
     unsigned fregion = 0;
     const int frows = (T * h->H + G - 1) / G;
-    if (h->fused_router && moe::layer_gateup_plan(T, h->E, h->H, G, &fsmem, &fslots, &fregion) &&
-        moe::down_decode_smem(T, h->k, h->I, frows) <= moe::kDownSmemMax) {
+    unsigned fdown = 0;
+    int lrows = 0;
+    const bool whole = h->fusion >= MOE_FUSION_LAYER && !keep &&
+                       moe::layer_plan(T, h->E, h->H, h->I, h->k, G, &fsmem, &fslots, &fregion,
+                                       &fdown, &lrows);
+    if (whole || (h->fusion >= MOE_FUSION_ROUTER &&
+                  moe::layer_gateup_plan(T, h->E, h->H, G, &fsmem, &fslots, &fregion) &&
+                  moe::down_decode_smem(T, h->k, h->I, frows) <= moe::kDownSmemMax)) {
         // router + gate/up in one launch, then the down kernel on the same grid
         // size (the routing handoff is per CTA index)
         moe::RouteHandoff hand;
@@ -459,7 +514,8 @@ int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
         g.E = h->E;
         g.H = h->H;
         g.I = h->I;
-        g.prefetch_down = h->prefetch_down ? 1 : 0;
+        // the one-launch layer copies its down rows into shared memory itself
+        g.prefetch_down = (h->prefetch_down && !whole) ? 1 : 0;
         {
             const size_t mc = (size_t)h->H * h->I / 2, ms = (size_t)h->H * h->I / 32;
             g.pf_codes = (uint32_t)(((mc + G - 1) / G + 15) / 16 * 16);
@@ -477,6 +533,19 @@ int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
         fr.rmsnorm = norm ? 1 : 0;
         fr.eps = 1e-6f;
         fr.region_bytes = fregion;
+        if (whole) {
+            // router + gate/up + down + combine in one launch
+            moe::LayerDownParams dp = {};
+            dp.residual = residual;
+            dp.y = y;
+            dp.h_tag = reinterpret_cast<uint2 *>(h->ws + L.h_tag);
+            dp.rows_per_cta = lrows;
+            dp.down_off = fdown;
+            if ((rc = cuda_rc(moe::launch_layer(g, fr, dp, G, fsmem, s, h->use_pdl))) != MOE_OK)
+                return rc;
+            h->kept = false;
+            return MOE_OK;
+        }
         if ((rc = cuda_rc(moe::launch_layer_gateup(g, fr, G, fsmem, s, h->use_pdl))) != MOE_OK)
             return rc;
         moe::DownParams d = {};
@@ -618,9 +687,9 @@ int moe_set_tuning(moe_handle_t h, int use_pdl, int prefetch_down) {
     return MOE_OK;
 }
 
-int moe_set_fusion(moe_handle_t h, int fused_router) {
-    if (!h) return MOE_ERR_ARG;
-    h->fused_router = fused_router != 0;
+int moe_set_fusion(moe_handle_t h, int mode) {
+    if (!h || mode < MOE_FUSION_NONE || mode > MOE_FUSION_LAYER) return MOE_ERR_ARG;
+    h->fusion = mode;
     return MOE_OK;
 }
 

@@ -369,6 +369,15 @@ __device__ __forceinline__ void st_relaxed_gpu_v2(uint2 *p, unsigned a, unsigned
                  "r"(a), "r"(b)
                  : "memory");
 }
+// Two such 64-bit words (each single-copy atomic on its own).
+__device__ __forceinline__ void ld_relaxed_gpu_2x64(const uint2 *p, uint2 &a, uint2 &b) {
+    asm volatile(
+        "{ .reg .b64 t0, t1; ld.relaxed.gpu.global.v2.b64 {t0, t1}, [%4];"
+        " mov.b64 {%0, %1}, t0; mov.b64 {%2, %3}, t1; }"
+        : "=r"(a.x), "=r"(a.y), "=r"(b.x), "=r"(b.y)
+        : "l"(p)
+        : "memory");
+}
 __device__ __forceinline__ uint2 ld_relaxed_gpu_v2(const uint2 *p) {
     uint2 v;
     asm volatile("{ .reg .b64 t; ld.relaxed.gpu.global.b64 t, [%2]; mov.b64 {%0, %1}, t; }"

@@ -29,7 +29,7 @@
 #include <math.h>
 #include <stdint.h>
 
-#include "gemv.cuh"
+#include "down.cuh"
 
 namespace moe {
 
@@ -342,7 +342,7 @@ gateup_tma_kernel(const GateUpParams p) {
             return pow2(p.x16_exp[tok]);
         }
         return pow2(stage_x<32, KCH>(p.x + (size_t)tok * H, lane, C, 0xffffffffu, xw));
-    });
+    }, [&](size_t idx, uint16_t v) { p.h[idx] = v; });
 }
 
 // ---------------------------------------------------------------- down -----
@@ -353,60 +353,6 @@ gateup_tma_kernel(const GateUpParams p) {
 // vectors h once into shared memory as FP16, then teams of TL lanes (slot
 // group j = warp % k) stream their rows against them.  Expert outputs meet in
 // shared memory for the sequential BF16 combine.
-
-// Stage the P BF16 vectors h[q][0..I) into shared memory as FP16 words, each
-// scaled by 2^-c_q (c_q from the vector's max |h|); s_xs[q] = 2^c_q.  One pass
-// over h: every 16-byte piece is read once (raw into sh) while its max |h|
-// goes to s_max[q] (warp max, then a shared atomic max on the non-negative
-// float bits); after one barrier each thread converts its own pieces in place.
-// s_max[0..P) must be zero on entry.  Out of line: it runs once per call and
-// keeps the kernel's code small.
-__device__ __noinline__ void stage_h_block(const uint16_t *h, int P, int I, uint32_t *sh,
-                                           float *s_xs, unsigned *s_max) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int n4 = I >> 3;  // 16-byte pieces per vector
-    const int total = P * n4;
-    const uint4 *hv = reinterpret_cast<const uint4 *>(h);
-    uint4 *sv = reinterpret_cast<uint4 *>(sh);
-    // every lane of a warp runs the same trip count (warp-wide votes inside)
-#pragma unroll 1
-    for (int base = warp * 32; base < total; base += kDownThreads) {
-        const int i = base + lane;
-        const bool valid = i < total;
-        float m = 0.f;
-        int q = -1;
-        if (valid) {
-            const uint4 v = hv[i];
-            sv[i] = v;
-            q = i / n4;
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int r = 0; r < 4; ++r)
-                m = fmaxf(m, fmaxf(fabsf(bf16_to_f32(w4[r] & 0xFFFFu)),
-                                   fabsf(bf16_to_f32(w4[r] >> 16))));
-        }
-        if (__all_sync(0xffffffffu, q == __shfl_sync(0xffffffffu, q, 0))) {
-            m = warp_max(m);
-            if (lane == 0 && q >= 0) atomicMax(s_max + q, __float_as_uint(m));
-        } else if (valid) {
-            atomicMax(s_max + q, __float_as_uint(m));
-        }
-    }
-    __syncthreads();
-#pragma unroll 1
-    for (int i = threadIdx.x; i < total; i += kDownThreads) {
-        const float sf = pow2_neg(f16_stage_exponent(__uint_as_float(s_max[i / n4])));
-        const uint4 v = sv[i];
-        uint4 o;
-        o.x = f32x2_to_f16x2(bf16_to_f32(v.x & 0xFFFFu) * sf, bf16_to_f32(v.x >> 16) * sf);
-        o.y = f32x2_to_f16x2(bf16_to_f32(v.y & 0xFFFFu) * sf, bf16_to_f32(v.y >> 16) * sf);
-        o.z = f32x2_to_f16x2(bf16_to_f32(v.z & 0xFFFFu) * sf, bf16_to_f32(v.z >> 16) * sf);
-        o.w = f32x2_to_f16x2(bf16_to_f32(v.w & 0xFFFFu) * sf, bf16_to_f32(v.w >> 16) * sf);
-        sv[i] = o;
-    }
-    if (threadIdx.x < P) s_xs[threadIdx.x] = pow2(f16_stage_exponent(__uint_as_float(s_max[threadIdx.x])));
-    __syncthreads();
-}
 
 // Routing handed over by CTA blockIdx.x of the fused router + gate/up kernel
 // of the same call (RouteHandoff), by one warp: lane q < P polls (bounded) its
@@ -439,61 +385,6 @@ static __device__ __noinline__ void take_handoff(const RouteHandoff h, int P, in
     }
 }
 
-__device__ __forceinline__ const uint8_t *down_codes(const DownParams &p, int e) {
-    return p.codes_base ? p.codes_base + (size_t)(3 * e + 2) * p.codes_stride : p.table[e].codes[2];
-}
-__device__ __forceinline__ const uint8_t *down_scales(const DownParams &p, int e) {
-    return p.codes_base ? p.scales_base + (size_t)(3 * e + 2) * p.scales_stride
-                        : p.table[e].scales[2];
-}
-
-// Shared-memory offset of the down rows (after the staged h and the expert
-// outputs), 16-byte aligned for the bulk copies.
-__host__ __device__ __forceinline__ size_t down_rows_offset(int T, int k, int I, int R) {
-    return ((size_t)T * k * I * 2 + (size_t)k * R * 4 + 15) & ~(size_t)15;
-}
-
-// By one thread: the CTA's down rows [r0, r1) of every slot into shared memory
-// (one bulk copy per slot, token segment and codes / scales), completing on
-// *bar; rows of an invalid expert id are not fetched.  Out of line.
-static __device__ __noinline__ void issue_down_rows(const ExpertPtrs *table,
-                                                    const uint8_t *codes_base,
-                                                    const uint8_t *scales_base, size_t cstride,
-                                                    size_t sstride, int E, int H, int I, int k,
-                                                    const int *s_ids, int r0, int r1, int R,
-                                                    uint8_t *rows_c, uint8_t *rows_s,
-                                                    uint64_t *bar) {
-    const size_t rc = (size_t)I >> 1, rs = (size_t)I >> 5;
-    unsigned bytes = 0;
-    #pragma unroll 1
-    for (int pass = 0; pass < 2; ++pass) {
-        if (pass == 1) mbar_arrive_expect_tx(bar, bytes);
-        #pragma unroll 1
-        for (int a = r0; a < r1;) {
-            const int t = a / H;
-            const int b = min(r1, (t + 1) * H);
-            const size_t n0 = (size_t)(a - t * H), cnt = (size_t)(b - a);
-            #pragma unroll 1
-            for (int j = 0; j < k; ++j) {
-                const int e = s_ids[t * k + j];
-                if (e < 0 || e >= E) continue;
-                if (pass == 0) {
-                    bytes += (unsigned)(cnt * (rc + rs));
-                } else {
-                    const size_t li = (size_t)j * R + (size_t)(a - r0);
-                    const uint8_t *dc = codes_base ? codes_base + (size_t)(3 * e + 2) * cstride
-                                                   : table[e].codes[2];
-                    const uint8_t *ds = codes_base ? scales_base + (size_t)(3 * e + 2) * sstride
-                                                   : table[e].scales[2];
-                    bulk_g2s(rows_c + li * rc, dc + n0 * rc, (unsigned)(cnt * rc), bar);
-                    bulk_g2s(rows_s + li * rs, ds + n0 * rs, (unsigned)(cnt * rs), bar);
-                }
-            }
-            a = b;
-        }
-    }
-}
-
 // SR: every down row of the CTA is copied into shared memory with bulk copies
 // before the programmatic-launch wait (rows: [k][R] codes, then [k][R] scales);
 // otherwise each team streams its rows from global memory two at a time.
@@ -501,13 +392,8 @@ template <int TL, int KCH, bool SR>
 __global__ void __launch_bounds__(kDownThreads, 1)
 down_decode_kernel(const DownParams p) {
     extern __shared__ __align__(16) uint8_t sm[];
-    constexpr int TPW = 32 / TL;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int lt = lane & (TL - 1);
-    const unsigned mask = team_mask<TL>(lane);
+    const int warp = threadIdx.x >> 5;
     const int H = p.H, I = p.I, k = p.k, T = p.T;
-    const int C = I >> 5;
-    const size_t rc = (size_t)I >> 1, rs = (size_t)I >> 5;
     const int R = p.rows_per_cta;
     const int r0 = blockIdx.x * R;
     const int r1 = min(r0 + R, T * H);
@@ -515,18 +401,12 @@ down_decode_kernel(const DownParams p) {
     uint32_t *sh = reinterpret_cast<uint32_t *>(sm);                       // [P][I/2] FP16 words
     float *so = reinterpret_cast<float *>(sm + (size_t)P * I * 2);         // [k][R]
     uint8_t *rows_c = sm + down_rows_offset(T, k, I, R);                   // SR: [k][R][I/2]
-    uint8_t *rows_s = rows_c + (size_t)k * R * rc;                          // SR: [k][R][I/32]
+    uint8_t *rows_s = rows_c + (size_t)k * R * ((size_t)I >> 1);           // SR: [k][R][I/32]
     __shared__ __align__(8) uint64_t s_rbar;
     __shared__ int s_ids[kDecodeMaxT * kMaxTopK];
     __shared__ float s_w[kDecodeMaxT * kMaxTopK];
     __shared__ float s_xs[kDecodeMaxT * kMaxTopK];
     __shared__ unsigned s_hmax[kDecodeMaxT * kMaxTopK];
-
-    const int groups = kDownWarps / k;  // warps per slot
-    const int j = warp % k, gi = warp / k;
-    const int tps = groups * TPW;       // teams per slot
-    const int ti = gi * TPW + lane / TL;
-    const bool worker = gi < groups;
 
     // routing for this call's tokens
     if (threadIdx.x < P) s_hmax[threadIdx.x] = 0u;
@@ -546,51 +426,13 @@ down_decode_kernel(const DownParams p) {
     }
     __syncthreads();
 
-    // rows of this team: r0 + ti, r0 + ti + tps, ...; two per step
-    int rr = r0 + ti;
-    uint4 cw[2][KCH];
-    uint32_t sc[2][KCH];
-    bool bad[2] = {false, false};
-    auto fetch = [&](int rbase) {
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int r = rbase + u * tps;
-            const bool valid = worker && r < r1;
-            const int t = valid ? r / H : 0;
-            const int n = r - t * H;
-            const int e = valid ? s_ids[t * k + j] : 0;
-            bad[u] = valid && (e < 0 || e >= p.E);
-            const bool ok = valid && !bad[u];
-            if (SR) {
-                const size_t li = (size_t)j * R + (size_t)(r - r0);
-                const uint8_t *dc = rows_c + li * rc, *ds = rows_s + li * rs;
-#pragma unroll
-                for (int v = 0; v < KCH; ++v) {
-                    const int c = lt + TL * v;
-                    if (ok && c < C) {
-                        cw[u][v] = *reinterpret_cast<const uint4 *>(dc + (size_t)c * 16);
-                        sc[u][v] = ds[c];
-                    } else {
-                        cw[u][v] = make_uint4(0u, 0u, 0u, 0u);
-                        sc[u][v] = 127u;
-                    }
-                }
-            } else {
-                const uint8_t *dc = nullptr, *ds = nullptr;
-                if (ok) {
-                    dc = down_codes(p, e) + (size_t)n * rc;
-                    ds = down_scales(p, e) + (size_t)n * rs;
-                }
-                load_chunks<TL, KCH>(dc, ds, ok, lt, C, cw[u], sc[u]);
-            }
-        }
-    };
+    const DownSrc src = {p.table, p.codes_base, p.scales_base, p.codes_stride, p.scales_stride};
+    DownRows<TL, KCH, SR> rows(H, I, k, p.E, R, r0, r1, src, s_ids, rows_c, rows_s);
     if (SR) {
         if (threadIdx.x == 0)
-            issue_down_rows(p.table, p.codes_base, p.scales_base, p.codes_stride, p.scales_stride,
-                            p.E, H, I, k, s_ids, r0, r1, R, rows_c, rows_s, &s_rbar);
+            issue_down_rows(src, p.E, H, I, k, s_ids, r0, r1, R, rows_c, rows_s, &s_rbar);
     } else {
-        fetch(rr);
+        rows.fetch(rows.rr);
     }
 
     pdl_wait();  // h comes from the gate/up kernel
@@ -602,68 +444,13 @@ down_decode_kernel(const DownParams p) {
     if (SR) {
         rows_ok = __syncthreads_and(mbar_wait(&s_rbar, 0u)) != 0;  // uniform over the CTA
         if (!rows_ok && threadIdx.x == 0) atomicOr(p.status, kTimeoutStatus);
-        if (rows_ok) fetch(rr);
+        if (rows_ok) rows.fetch(rows.rr);
     }
-
-    #pragma unroll 1
-    while (worker && rows_ok && rr < r1) {
-        const int t = rr / H;
-        const uint32_t *xv = sh + (size_t)(t * k + j) * (I >> 1);
-        const float xs = s_xs[t * k + j];
-        // both rows of a step belong to token t unless the second crosses into
-        // the next token; then it is recomputed in the next step
-        const int rb = rr + tps;
-        const bool second = rb < r1 && rb / H == t;
-        float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-        for (int u = 0; u < KCH; ++u) {
-            const int c = lt + TL * u;
-            if (c < C) {
-                const uint4 *xq = reinterpret_cast<const uint4 *>(xv + (size_t)c * 16);
-                uint32_t x[16];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint4 v = xq[q];
-                    x[4 * q] = v.x;
-                    x[4 * q + 1] = v.y;
-                    x[4 * q + 2] = v.z;
-                    x[4 * q + 3] = v.w;
-                }
-                a0 = fmaf(dot32_e2m1_f16(cw[0][u], x), e8m0_to_f32(sc[0][u]), a0);
-                a1 = fmaf(dot32_e2m1_f16(cw[1][u], x), e8m0_to_f32(sc[1][u]), a1);
-            }
-        }
-        a0 = team_add<TL>(a0, mask);
-        a1 = team_add<TL>(a1, mask);
-        const bool b0 = bad[0], b1 = bad[1];
-        const int rnext = second ? rr + 2 * tps : rr + tps;
-        if (rnext < r1) fetch(rnext);
-        if (lt == 0) {
-            so[j * R + (rr - r0)] = b0 ? 0.f : round_bf16(a0 * xs);
-            if (b0) atomicOr(p.status, kBadExpertId);
-            if (second) {
-                so[j * R + (rb - r0)] = b1 ? 0.f : round_bf16(a1 * xs);
-                if (b1) atomicOr(p.status, kBadExpertId);
-            }
-        }
-        rr = rnext;
-    }
+    if (rows_ok) rows.run(sh, s_xs, so, p.status);
     __syncthreads();
 
     // sequential BF16 combine in slot order, optional residual add
-    #pragma unroll 1
-    for (int r = r0 + threadIdx.x; r < r1; r += kDownThreads) {
-        const int t = r / H, n = r - t * H;
-        float y = 0.f;
-        for (int jj = 0; jj < k; ++jj) {
-            const float o = so[jj * R + (r - r0)];
-            const float wb = round_bf16(s_w[t * k + jj]);
-            y = round_bf16(y + round_bf16(o * wb));
-            if (p.o_keep) p.o_keep[((size_t)t * k + jj) * H + n] = f32_to_bf16(o);
-        }
-        if (p.residual) y = round_bf16(bf16_to_f32(p.residual[r]) + y);
-        p.y[r] = f32_to_bf16(y);
-    }
+    down_combine(r0, r1, H, k, R, so, s_w, p.residual, p.y, p.o_keep);
     // no row copy may outlive the CTA (complete unless its wait timed out)
     if (SR && !rows_ok && threadIdx.x == 0) mbar_wait(&s_rbar, 0u);
 }
@@ -693,20 +480,6 @@ __global__ void debug_dequant_kernel(const uint8_t *codes, const uint8_t *scales
 
 namespace {
 
-// (TL, KCH) for K/32 = C chunks per row: a team of TL lanes, KCH chunks per lane.
-void pick_team(int C, int &TL, int &KCH) {
-    const int tls[4] = {32, 16, 8, 4};
-    for (int i = 0; i < 4; ++i)
-        if (C % tls[i] == 0 && C / tls[i] <= 4) {
-            TL = tls[i];
-            KCH = C / tls[i];
-            return;
-        }
-    TL = 32;
-    KCH = (C + 31) / 32;
-}
-
-
 template <int TL, int KCH>
 cudaError_t launch_gu(const GateUpParams &p, int grid, cudaStream_t s, bool pdl) {
     return launch_ex(gateup_decode_kernel<TL, KCH>, dim3(grid), dim3(kGemvThreads), 0, s, pdl, p);
@@ -732,8 +505,7 @@ template <int TL, int KCH>
 cudaError_t launch_dn(const DownParams &p, int grid, cudaStream_t s, bool pdl) {
     const size_t smem = down_decode_smem(p.T, p.k, p.I, p.rows_per_cta);
     if (smem > kDownSmemMax) return cudaErrorInvalidValue;
-    const size_t smem_sr = down_rows_offset(p.T, p.k, p.I, p.rows_per_cta) +
-                           (size_t)p.k * p.rows_per_cta * ((size_t)p.I / 2 + (size_t)p.I / 32);
+    const size_t smem_sr = down_rows_smem(p.T, p.k, p.I, p.rows_per_cta);
     if (p.I % 512 == 0 && smem_sr <= kDownSmemMax)
         return launch_dn_v<TL, KCH, true>(p, grid, smem_sr, s, pdl);
     return launch_dn_v<TL, KCH, false>(p, grid, smem, s, pdl);

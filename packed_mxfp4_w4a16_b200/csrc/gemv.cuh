@@ -370,12 +370,13 @@ __device__ __forceinline__ void ring_produce(const GateUpParams &p, const RingGe
 }
 
 // Consumer warps: one row per slot each.  get_x(tok, xw) fills the warp's
-// FP16-staged activations of token tok and returns their scale 2^c.
-template <int KCH, class GetX>
+// FP16-staged activations of token tok and returns their scale 2^c;
+// emit_h(index, bf16) stores h[q][i] (index q I + i).
+template <int KCH, class GetX, class EmitH>
 __device__ __forceinline__ void ring_consume(const GateUpParams &p, const RingGeom &g,
                                              const uint8_t *ring, uint64_t *full,
                                              uint64_t *empty, const int *s_ids, int warp,
-                                             int lane, GetX &&get_x) {
+                                             int lane, GetX &&get_x, EmitH &&emit_h) {
     const int E = p.E, I = p.I, k = p.k;
     const int C = p.H >> 5;
     const int cb = g.cb, ce = g.ce, nsteps = g.nsteps, nslots = g.nslots;
@@ -435,7 +436,7 @@ __device__ __forceinline__ void ring_consume(const GateUpParams &p, const RingGe
                     } else {
                         atomicOr(p.status, kBadExpertId);
                     }
-                    p.h[(size_t)q * I + i] = out;
+                    emit_h((size_t)q * I + i, out);
                 }
             }
         }
@@ -443,6 +444,20 @@ __device__ __forceinline__ void ring_consume(const GateUpParams &p, const RingGe
         if (lane == 0) mbar_arrive(&empty[b]);
     }
 }
+
+// (TL, KCH) for K/32 = C chunks per row: a team of TL lanes, KCH chunks per lane.
+inline void pick_team(int C, int &TL, int &KCH) {
+    const int tls[4] = {32, 16, 8, 4};
+    for (int i = 0; i < 4; ++i)
+        if (C % tls[i] == 0 && C / tls[i] <= 4) {
+            TL = tls[i];
+            KCH = C / tls[i];
+            return;
+        }
+    TL = 32;
+    KCH = (C + 31) / 32;
+}
+
 
 // Launch with cudaLaunchKernelEx; `pdl` sets programmatic stream serialization
 // so the kernel may start while the previous one drains.

@@ -1,0 +1,433 @@
+// grouped.cu — the (token, expert)-sorted grouped path of the packed-MXFP4
+// W4A16 MoE expert FFN, for batches of tokens (prefill chunks, many decode
+// streams).
+//
+// Sources: model card "LFM2.5-24B-A2B — Packed MXFP4 Inference", "Grouped
+// top-4 expert execution" (grouped gate / up / down products, activation and
+// multiplication, fused combine keeping sequential BF16 multiply/add
+// rounding) and table "Model and quantization" (E2M1 + E8M0 per 32, BF16
+// activations, FP32 accumulation); the MLX page on quantized MoE ("Gather
+// quantized matmul", sorting the (token, expert) pairs so that each expert's
+// tokens form one contiguous group before the quantized product).
+//
+// Launch sequence (one stream, programmatic serialization):
+//   grouped_prep_kernel      CTA 0: stable counting sort of the T k (token,
+//                            slot) pairs by expert -> perm, offs.  CTAs 1..T:
+//                            FP16 staging of each token's activations.
+//   grouped_mma_kernel<2>    per (expert, 32 gate/up rows): h = SwiGLU of the
+//                            expert's tokens, on the tensor cores.
+//   grouped_stage_h_kernel   per pair: FP16 staging of h.
+//   grouped_mma_kernel<1>    per (expert, 32 down rows): o = BF16(W_down h).
+//   grouped_combine_kernel   per token: sequential BF16 combine (+ residual).
+//
+// Tensor-core tile.  A CTA holds 32 packed rows of one expert matrix (codes
+// and E8M0 scales, copied to shared memory with 16-byte asynchronous copies
+// into a row-padded layout) and runs 8 warps: 2 row tiles of 16 x 4 quarters
+// of the K groups.  mma.m16n8k16 (FP16 x FP16 -> FP32) takes A = the E2M1
+// codes converted to FP16 in registers (exact) and B = the FP16-staged
+// activations of 8 tokens.  Within each 32-element group the K order is
+// permuted identically for A and B so that each thread's A operand is one
+// aligned 4-byte word of the row (8 codes) and its B operand one 16-byte piece
+// of the activation row; the group's partial product (two MMAs, fresh
+// accumulator) is then scaled by the group's E8M0 exponent in FP32 and added
+// to the running FP32 sum, which is exactly per-group scaling.  The K quarters
+// are added in a fixed order at the end.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "gemv.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kGpThreads = 256;   // 8 warps
+constexpr int kGpRows = 32;       // matrix rows per CTA (2 row tiles of 16)
+constexpr int kGpChunk = 32;      // tokens per pass (4 column tiles of 8)
+constexpr int kGpMaxE = 1024;
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// d = A B + c for one m16n8k16 tile, FP16 operands, FP32 accumulators.
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                        uint32_t a3, uint32_t b0, uint32_t b1, const float (&c)[4]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%10, %11, %12, %13};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(c[2]),
+          "f"(c[3]));
+}
+
+__device__ __forceinline__ const uint8_t *mat_codes(const GroupedParams &p, int e, int m) {
+    return p.codes_base ? p.codes_base + (size_t)(3 * e + m) * p.codes_stride : p.table[e].codes[m];
+}
+__device__ __forceinline__ const uint8_t *mat_scales(const GroupedParams &p, int e, int m) {
+    return p.codes_base ? p.scales_base + (size_t)(3 * e + m) * p.scales_stride
+                        : p.table[e].scales[m];
+}
+
+// FP16 staging of the BF16 vector v[0..n) (as the decode path stages it): the
+// CTA's max |v| picks c, out = v 2^-c as f16x2 words; returns c.  All threads.
+__device__ __forceinline__ int stage_vector_f16(const uint16_t *v, int n, uint32_t *out,
+                                                float *red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int npc = n >> 3;  // 8-element pieces
+    float m = 0.f;
+    for (int c = threadIdx.x; c < npc; c += kGpThreads) {
+        const uint4 x = reinterpret_cast<const uint4 *>(v)[c];
+        const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            m = fmaxf(m, fmaxf(fabsf(bf16_to_f32(w4[q] & 0xFFFFu)), fabsf(bf16_to_f32(w4[q] >> 16))));
+    }
+    m = warp_max(m);
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < kGpThreads / 32; ++i) amax = fmaxf(amax, red[i]);
+    const int e = f16_stage_exponent(amax);
+    const float sf = pow2_neg(e);
+    for (int c = threadIdx.x; c < npc; c += kGpThreads) {
+        const uint4 x = reinterpret_cast<const uint4 *>(v)[c];
+        uint4 o;
+        o.x = f32x2_to_f16x2(bf16_to_f32(x.x & 0xFFFFu) * sf, bf16_to_f32(x.x >> 16) * sf);
+        o.y = f32x2_to_f16x2(bf16_to_f32(x.y & 0xFFFFu) * sf, bf16_to_f32(x.y >> 16) * sf);
+        o.z = f32x2_to_f16x2(bf16_to_f32(x.z & 0xFFFFu) * sf, bf16_to_f32(x.z >> 16) * sf);
+        o.w = f32x2_to_f16x2(bf16_to_f32(x.w & 0xFFFFu) * sf, bf16_to_f32(x.w >> 16) * sf);
+        reinterpret_cast<uint4 *>(out)[c] = o;
+    }
+    return e;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ prep --
+// CTA 0: stable counting sort of the pairs q = t k + j by expert (ties in pair
+// order); invalid ids are left out of every segment and flag the status.
+// CTAs 1..T: FP16 staging of token t = blockIdx.x - 1.
+__global__ void __launch_bounds__(kGpThreads) grouped_prep_kernel(const GroupedParams p) {
+    __shared__ int s_cnt[kGpMaxE];
+    __shared__ float s_red[kGpThreads / 32];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (blockIdx.x > 0) {
+        const int t = blockIdx.x - 1;
+        const int c = stage_vector_f16(p.x + (size_t)t * p.H, p.H, p.x16 + (size_t)t * (p.H >> 1),
+                                       s_red);
+        if (threadIdx.x == 0) p.x_exp[t] = c;
+        return;
+    }
+    const int E = p.E, P = p.T * p.k;
+    for (int e = threadIdx.x; e < E; e += kGpThreads) s_cnt[e] = 0;
+    __syncthreads();
+    bool bad = false;
+    for (int q = threadIdx.x; q < P; q += kGpThreads) {
+        const int e = p.ids[q];
+        if (e >= 0 && e < E)
+            atomicAdd(&s_cnt[e], 1);
+        else
+            bad = true;
+    }
+    if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(p.status, kBadExpertId);
+    if (warp == 0) {
+        // exclusive scan: lane L sums a block of ceil(E/32) counts, the warp
+        // scans the block sums, each lane then writes its block's starts
+        const int per = (E + 31) / 32;
+        const int b0 = min(E, lane * per), b1 = min(E, b0 + per);
+        int sum = 0;
+        for (int e = b0; e < b1; ++e) sum += s_cnt[e];
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - sum;
+        for (int e = b0; e < b1; ++e) {
+            const int c = s_cnt[e];
+            s_cnt[e] = run;  // becomes the next free slot of expert e
+            p.offs[e] = run;
+            run += c;
+        }
+        if (lane == 31) p.offs[E] = incl;
+        __syncwarp();
+        // placement in pair order, 32 pairs per round: the rank of a pair among
+        // the round's pairs of the same expert comes from a match vote
+        for (int base = 0; base < P; base += 32) {
+            const int q = base + lane;
+            const int e = q < P ? p.ids[q] : -1;
+            const bool valid = e >= 0 && e < E;
+            const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : E + lane);
+            const int rank = __popc(peers & ((1u << lane) - 1u));
+            const int pos = valid ? s_cnt[e] + rank : 0;
+            __syncwarp();
+            if (valid && rank == 0) s_cnt[e] += __popc(peers);
+            if (valid) p.perm[pos] = q;
+            __syncwarp();
+        }
+    }
+}
+
+// -------------------------------------------------- tensor-core products --
+// NMAT = 2: gate and up rows [i0, i0 + 32) of expert blockIdx.y against the
+// staged activations of its tokens -> h (SwiGLU, BF16) of its pairs.
+// NMAT = 1: down rows [n0, n0 + 32) against the staged h of its pairs ->
+// o (BF16) of its pairs.
+template <int NMAT>
+__global__ void __launch_bounds__(kGpThreads) grouped_mma_kernel(const GroupedParams p) {
+    extern __shared__ __align__(16) uint8_t sm[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int e = blockIdx.y;
+    pdl_wait();
+    pdl_launch_dependents();
+    const int seg0 = p.offs[e], n_e = p.offs[e + 1] - seg0;
+    if (n_e <= 0) return;  // uniform: no token chose this expert
+
+    const int K = NMAT == 2 ? p.H : p.I;     // reduction length
+    const int M = NMAT == 2 ? p.I : p.H;     // rows of the matrix
+    const int row0 = blockIdx.x * kGpRows;
+    const int ng = K >> 5;                   // 32-element groups
+    const size_t rc = (size_t)K >> 1, rs = (size_t)K >> 5;
+    const size_t rcp = rc + 16, rsp = rs + 16;  // padded row pitches (bank spread)
+    uint8_t *s_codes = sm;                                    // [NMAT][32][rcp]
+    uint8_t *s_scales = sm + (size_t)NMAT * kGpRows * rcp;    // [NMAT][32][rsp]
+    float *s_red = reinterpret_cast<float *>(s_scales + (size_t)NMAT * kGpRows * rsp);
+    // s_red: [3 quarters][2 row tiles][32 lanes][NMAT * 16] partial sums
+
+    // ---- the 32 rows of each matrix into shared memory ----
+    const int rows = min(kGpRows, M - row0);
+#pragma unroll
+    for (int m = 0; m < NMAT; ++m) {
+        const int mat = NMAT == 2 ? m : 2;
+        const uint8_t *gc = mat_codes(p, e, mat) + (size_t)row0 * rc;
+        const uint8_t *gs = mat_scales(p, e, mat) + (size_t)row0 * rs;
+        const int c16 = (int)(rc >> 4);
+        for (int i = threadIdx.x; i < rows * c16; i += kGpThreads) {
+            const int r = i / c16, c = i - r * c16;
+            cp_async16(s_codes + ((size_t)m * kGpRows + r) * rcp + (size_t)c * 16,
+                       gc + (size_t)r * rc + (size_t)c * 16);
+        }
+        const int c4 = (int)(rs >> 2);
+        for (int i = threadIdx.x; i < rows * c4; i += kGpThreads) {
+            const int r = i / c4, c = i - r * c4;
+            cp_async4(s_scales + ((size_t)m * kGpRows + r) * rsp + (size_t)c * 4,
+                      gs + (size_t)r * rs + (size_t)c * 4);
+        }
+    }
+    cp_async_wait_all();
+    __syncthreads();
+
+    const int g = lane >> 2, q = lane & 3;
+    const int rt = warp & 1, kq = warp >> 1;  // row tile, K quarter
+    const int gq = (ng + 3) >> 2;
+    const int gb = min(ng, kq * gq), ge = min(ng, gb + gq);
+    const int r_lo = rt * 16 + g, r_hi = r_lo + 8;  // this thread's two A rows
+    const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+
+    #pragma unroll 1
+    for (int tc = 0; tc < n_e; tc += kGpChunk) {
+        // B rows (activation vectors) of this thread's column in each of the 4
+        // column tiles: column g of tile nt is token tc + 8 nt + g of the group
+        const uint32_t *brow[4];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            const int idx = tc + nt * 8 + g;
+            brow[nt] = nullptr;
+            if (idx < n_e) {
+                const int pr = p.perm[seg0 + idx];
+                brow[nt] = NMAT == 2 ? p.x16 + (size_t)(pr / p.k) * (K >> 1)
+                                     : p.h16 + (size_t)pr * (K >> 1);
+            }
+        }
+        const int ntv = min(4, (n_e - tc + 7) >> 3);  // column tiles in use (uniform)
+        float acc[NMAT][4][4];
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[m][nt][i] = 0.f;
+
+        #pragma unroll 1
+        for (int G = gb; G < ge; ++G) {
+            uint32_t fa[NMAT][2][4];  // [mat][row lo / hi][f16x2 of codes 8q..8q+7]
+            float sc[NMAT][2];
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m) {
+                const uint8_t *cb = s_codes + (size_t)m * kGpRows * rcp + (size_t)G * 16 + 4 * q;
+                const uint8_t *sb = s_scales + (size_t)m * kGpRows * rsp + G;
+                e2m1x8_to_f16x8(*reinterpret_cast<const uint32_t *>(cb + (size_t)r_lo * rcp), fa[m][0]);
+                e2m1x8_to_f16x8(*reinterpret_cast<const uint32_t *>(cb + (size_t)r_hi * rcp), fa[m][1]);
+                sc[m][0] = e8m0_to_f32(sb[(size_t)r_lo * rsp]);
+                sc[m][1] = e8m0_to_f32(sb[(size_t)r_hi * rsp]);
+            }
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                if (nt < ntv) {
+                    const uint4 b = brow[nt] ? __ldg(reinterpret_cast<const uint4 *>(
+                                                   brow[nt] + (size_t)G * 16 + 4 * q))
+                                             : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                    for (int m = 0; m < NMAT; ++m) {
+                        float d[4];
+                        // group G: slots 2q, 2q+1 / 2q+8, 2q+9 of the first MMA carry
+                        // elements 8q + {0,1} / {2,3}; of the second 8q + {4,5} / {6,7}
+                        mma_f16(d, fa[m][0][0], fa[m][1][0], fa[m][0][1], fa[m][1][1], b.x, b.y,
+                                zero);
+                        mma_f16(d, fa[m][0][2], fa[m][1][2], fa[m][0][3], fa[m][1][3], b.z, b.w,
+                                d);
+                        acc[m][nt][0] = fmaf(d[0], sc[m][0], acc[m][nt][0]);
+                        acc[m][nt][1] = fmaf(d[1], sc[m][0], acc[m][nt][1]);
+                        acc[m][nt][2] = fmaf(d[2], sc[m][1], acc[m][nt][2]);
+                        acc[m][nt][3] = fmaf(d[3], sc[m][1], acc[m][nt][3]);
+                    }
+                }
+            }
+        }
+        // ---- the 4 K quarters, added in order 0, 1, 2, 3 ----
+        if (kq > 0) {
+            float *dst = s_red + ((size_t)((kq - 1) * 2 + rt) * 32 + lane) * (NMAT * 16);
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) dst[(m * 4 + nt) * 4 + i] = acc[m][nt][i];
+        }
+        __syncthreads();
+        if (kq == 0) {
+#pragma unroll
+            for (int qq = 1; qq < 4; ++qq) {
+                const float *src = s_red + ((size_t)((qq - 1) * 2 + rt) * 32 + lane) * (NMAT * 16);
+#pragma unroll
+                for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+                    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) acc[m][nt][i] += src[(m * 4 + nt) * 4 + i];
+            }
+            // ---- epilogue: rows r_lo / r_hi, columns 2q, 2q + 1 of each tile ----
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int idx = tc + nt * 8 + 2 * q + cc;
+                    if (nt >= ntv || idx >= n_e) continue;
+                    const int pr = p.perm[seg0 + idx];
+#pragma unroll
+                    for (int hr = 0; hr < 2; ++hr) {
+                        const int r = row0 + (hr ? r_hi : r_lo);
+                        if (r >= M) continue;
+                        if (NMAT == 2) {
+                            const float xs = pow2(p.x_exp[pr / p.k]);
+                            const float gv = round_bf16(acc[0][nt][hr * 2 + cc] * xs);
+                            const float uv = round_bf16(acc[NMAT - 1][nt][hr * 2 + cc] * xs);
+                            const float sl = round_bf16(gv / (1.0f + expf(-gv)));
+                            p.h[(size_t)pr * M + r] = f32_to_bf16(sl * uv);
+                        } else {
+                            const float hs = pow2(p.h_exp[pr]);
+                            p.o[(size_t)pr * M + r] = f32_to_bf16(acc[0][nt][hr * 2 + cc] * hs);
+                        }
+                    }
+                }
+        }
+        __syncthreads();  // s_red is reused by the next chunk
+    }
+}
+
+// ------------------------------------------------------------- stage h --
+__global__ void __launch_bounds__(kGpThreads) grouped_stage_h_kernel(const GroupedParams p) {
+    __shared__ float s_red[kGpThreads / 32];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int pr = blockIdx.x;
+    const int e = p.ids[pr];
+    if (e < 0 || e >= p.E) return;  // uniform: the pair has no h
+    const int c = stage_vector_f16(p.h + (size_t)pr * p.I, p.I, p.h16 + (size_t)pr * (p.I >> 1),
+                                   s_red);
+    if (threadIdx.x == 0) p.h_exp[pr] = c;
+}
+
+// ------------------------------------------------------------- combine --
+// y[t] = sequential BF16 combine of the k expert outputs in slot order (a pair
+// with an invalid id contributes 0), then the optional residual add.
+__global__ void __launch_bounds__(kGpThreads) grouped_combine_kernel(const GroupedParams p) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int t = blockIdx.x, k = p.k, H = p.H;
+    for (int n = threadIdx.x; n < H; n += kGpThreads) {
+        float y = 0.f;
+        for (int j = 0; j < k; ++j) {
+            const int pr = t * k + j;
+            const int e = p.ids[pr];
+            const float o = (e >= 0 && e < p.E) ? bf16_to_f32(p.o[(size_t)pr * H + n]) : 0.f;
+            const float wb = round_bf16(p.w[pr]);
+            y = round_bf16(y + round_bf16(o * wb));
+            if (p.o_keep) p.o_keep[(size_t)pr * H + n] = f32_to_bf16(o);
+        }
+        if (p.residual) y = round_bf16(bf16_to_f32(p.residual[(size_t)t * H + n]) + y);
+        p.y[(size_t)t * H + n] = f32_to_bf16(y);
+    }
+}
+
+// ------------------------------------------------------------------ host --
+
+bool grouped_supported(int E, int H, int I) {
+    return E <= kGpMaxE && H % 128 == 0 && I % 128 == 0 && H <= 4096 && I <= 4096;
+}
+
+namespace {
+
+size_t mma_smem(int nmat, int K) {
+    const size_t rcp = (size_t)K / 2 + 16, rsp = (size_t)K / 32 + 16;
+    return (size_t)nmat * kGpRows * (rcp + rsp) + (size_t)3 * 2 * 32 * nmat * 16 * sizeof(float);
+}
+
+template <int NMAT>
+cudaError_t launch_mma(const GroupedParams &p, cudaStream_t s, bool pdl) {
+    const int K = NMAT == 2 ? p.H : p.I, M = NMAT == 2 ? p.I : p.H;
+    const size_t smem = mma_smem(NMAT, K);
+    static size_t attr_smem = 0;  // largest dynamic shared memory enabled so far
+    if (smem > attr_smem) {
+        cudaError_t e = cudaFuncSetAttribute(grouped_mma_kernel<NMAT>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_smem = smem;
+    }
+    return launch_ex(grouped_mma_kernel<NMAT>, dim3((M + kGpRows - 1) / kGpRows, p.E),
+                     dim3(kGpThreads), smem, s, pdl, p);
+}
+
+}  // namespace
+
+cudaError_t launch_grouped(const GroupedParams &p, cudaStream_t s, bool pdl) {
+    if (p.T < 1 || p.T > kGroupedMaxT || !grouped_supported(p.E, p.H, p.I))
+        return cudaErrorInvalidValue;
+    cudaError_t e;
+    if ((e = launch_ex(grouped_prep_kernel, dim3(p.T + 1), dim3(kGpThreads), 0, s, pdl, p)) !=
+        cudaSuccess)
+        return e;
+    if ((e = launch_mma<2>(p, s, pdl)) != cudaSuccess) return e;
+    if ((e = launch_ex(grouped_stage_h_kernel, dim3(p.T * p.k), dim3(kGpThreads), 0, s, pdl, p)) !=
+        cudaSuccess)
+        return e;
+    if ((e = launch_mma<1>(p, s, pdl)) != cudaSuccess) return e;
+    return launch_ex(grouped_combine_kernel, dim3(p.T), dim3(kGpThreads), 0, s, pdl, p);
+}
+
+}  // namespace moe

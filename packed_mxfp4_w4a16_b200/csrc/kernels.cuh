@@ -85,6 +85,15 @@ struct FusedRouteParams {
     unsigned region_bytes;   // dynamic shared memory before the routed-vector buffer
 };
 
+// Down half of the one-launch layer (router + gate/up + down in one grid).
+struct LayerDownParams {
+    const uint16_t *residual;  // [T][H] or null
+    uint16_t *y;               // [T][H]
+    uint2 *h_tag;              // [T][k][I] {tag, BF16 h}: h exchanged between the CTAs
+    int rows_per_cta;          // R: output rows of each CTA
+    unsigned down_off;         // dynamic shared memory offset of the down region
+};
+
 struct DownParams {
     const ExpertPtrs *table;
     const uint8_t *codes_base, *scales_base;  // contiguous layout fast path (or null)
@@ -102,6 +111,33 @@ struct DownParams {
     RouteHandoff hand;         // used when ids and logits are both null
 };
 
+// The (token, expert)-sorted grouped path (grouped.cu), for batches of tokens.
+constexpr int kGroupedMaxT = 256;  // tokens per grouped launch sequence (more: chunks)
+struct GroupedParams {
+    const ExpertPtrs *table;
+    const uint8_t *codes_base, *scales_base;  // contiguous layout fast path (or null)
+    size_t codes_stride, scales_stride;
+    const uint16_t *x;         // [T][H] BF16
+    const int32_t *ids;        // [T][k]
+    const float *w;            // [T][k]
+    const uint16_t *residual;  // [T][H] or null
+    uint16_t *y;               // [T][H]
+    uint16_t *o_keep;          // [T][k][H] or null
+    // workspace
+    int *perm;                 // [T k] pair indices t k + j, sorted by (expert, pair)
+    int *offs;                 // [E + 1] start of each expert's segment in perm
+    uint32_t *x16;             // [T][H/2] FP16-staged x (f16x2 words)
+    int *x_exp;                // [T] staging exponents of x16
+    uint16_t *h;               // [T k][I] BF16 SwiGLU outputs
+    uint32_t *h16;             // [T k][I/2] FP16-staged h
+    int *h_exp;                // [T k] staging exponents of h16
+    uint16_t *o;               // [T k][H] BF16 expert outputs
+    unsigned *status;
+    int T, k, E, H, I;
+};
+bool grouped_supported(int E, int H, int I);
+cudaError_t launch_grouped(const GroupedParams &p, cudaStream_t s, bool pdl);
+
 // Host-side launchers (decode.cu).  `pdl` sets programmatic stream
 // serialization so the kernel may start while the previous one drains.
 cudaError_t launch_route(const RouteParams &p, cudaStream_t s, bool pdl);
@@ -117,6 +153,15 @@ bool layer_gateup_plan(int T, int E, int H, int grid, size_t *smem, int *nslots,
                        unsigned *region_bytes);
 cudaError_t launch_layer_gateup(const GateUpParams &p, const FusedRouteParams &r, int grid,
                                 size_t smem, cudaStream_t s, bool pdl);
+// The whole layer in one launch (T small enough for the gate/up ring, the
+// routed vector and the CTA's down rows to share one SM's shared memory, and
+// I a multiple of 512): layer_plan returns its dynamic shared memory, ring
+// slots and the offsets, or false.
+bool layer_plan(int T, int E, int H, int I, int k, int grid, size_t *smem, int *nslots,
+                unsigned *region_bytes, unsigned *down_off, int *rows_per_cta);
+cudaError_t launch_layer(const GateUpParams &p, const FusedRouteParams &r,
+                         const LayerDownParams &d, int grid, size_t smem, cudaStream_t s,
+                         bool pdl);
 cudaError_t launch_debug_dequant(const uint8_t *codes, const uint8_t *scales, int64_t n,
                                  float *out, cudaStream_t s);
 size_t gateup_decode_smem(int T, int H);

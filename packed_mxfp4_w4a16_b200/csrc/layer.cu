@@ -24,6 +24,14 @@
 // tag = seq[b] + 1 is unique to the call.  The routing goes to the down kernel
 // of the same call through the per-CTA handoff, with the same tag.
 //
+// With a down team shape (TLD > 0) the same grid also runs the down GEMV and
+// the combine: the producer issues bulk copies of the CTA's down rows into
+// shared memory right after routing; the consumers write each h value with
+// this call's tag as one 8-byte word; every CTA then stages all of h, each
+// piece re-read (bounded) until it carries the tag, and reduces its rows as
+// the standalone down kernel does.  No kernel boundary and no grid-wide wait
+// remain inside the layer: each CTA waits only for the h values it reads.
+//
 // Every reduction follows the standalone router kernel's order (its thread
 // tid owns the 16-byte pieces tid and tid + 256 of a row; warp sums; the 8
 // warp partials added in order), so x_norm, the logits and the routing are
@@ -32,7 +40,7 @@
 #include <math.h>
 #include <stdint.h>
 
-#include "gemv.cuh"
+#include "down.cuh"
 
 namespace moe {
 
@@ -100,9 +108,13 @@ static __device__ __noinline__ void fused_topk(const float *s_logits, int T, int
 
 }  // namespace
 
-template <int KCH>
+// TLD == 0: router + gate/up (a down kernel follows); TLD > 0: the whole
+// layer, down teams of TLD lanes holding KCHD chunks each.
+template <int KCH, int TLD, int KCHD>
 __global__ void __launch_bounds__(kTmaThreads, 1)
-layer_gateup_kernel(const GateUpParams p, const FusedRouteParams r) {
+layer_kernel(const GateUpParams p, const FusedRouteParams r, const LayerDownParams dp) {
+    static_assert(kTmaThreads == kDownThreads, "one CTA shape for both phases");
+    constexpr bool kWhole = TLD > 0;
     extern __shared__ __align__(128) uint8_t ring[];
     __shared__ __align__(8) uint64_t full[kTmaMaxSlots];
     __shared__ __align__(8) uint64_t empty[kTmaMaxSlots];
@@ -113,6 +125,9 @@ layer_gateup_kernel(const GateUpParams p, const FusedRouteParams r) {
     __shared__ float s_red[kRouteWarps][kDecodeMaxT][2];
     __shared__ int s_xexp[kDecodeMaxT];
     __shared__ unsigned s_tag;
+    __shared__ __align__(8) uint64_t s_dbar;               // kWhole: the CTA's down rows
+    __shared__ float s_xs[kDecodeMaxT * kMaxTopK];          // kWhole: h staging scales
+    __shared__ unsigned s_hmax[kDecodeMaxT * kMaxTopK];     // kWhole: h staging maxima
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int H = p.H, k = p.k, T = p.T, E = p.E;
     const int C = H >> 5;
@@ -133,8 +148,13 @@ layer_gateup_kernel(const GateUpParams p, const FusedRouteParams r) {
             if (c < nch) wv[u] = row[c];
         }
     }
+    if (kWhole && threadIdx.x < T * k) s_hmax[threadIdx.x] = 0u;
     if (threadIdx.x == 0) {
         ring_init(g, full, empty);
+        if (kWhole) {
+            mbar_init(&s_dbar, 1);
+            mbar_fence_init();
+        }
         // seq[b]: written by the CTA of the same index two launches back,
         // complete before this grid could start
         s_tag = ld_relaxed_gpu(r.hand.seq + blockIdx.x) + 1u;
@@ -263,9 +283,21 @@ layer_gateup_kernel(const GateUpParams p, const FusedRouteParams r) {
         __syncthreads();  // s_red is reused by the next expert
     }
 
+    // down region (kWhole): staged h, expert outputs, the CTA's down rows
+    const int I = p.I;
+    const int R = dp.rows_per_cta;
+    const int dr0 = (int)blockIdx.x * R, dr1 = min(dr0 + R, T * H);
+    uint8_t *dreg = ring + dp.down_off;
+    uint32_t *sh = reinterpret_cast<uint32_t *>(dreg);
+    float *so = reinterpret_cast<float *>(dreg + (size_t)T * k * I * 2);
+    uint8_t *rows_c = dreg + down_rows_offset(T, k, I, R);
+    uint8_t *rows_s = rows_c + (size_t)k * R * ((size_t)I >> 1);
+    const DownSrc src = {p.table, p.codes_base, p.scales_base, p.codes_stride, p.scales_stride};
+
     if (warp == kTmaConsumers) {
         // ---- producer warp: all logits, routing, the ring, and (with the
-        // first copies in flight) the routing for the caller and the down kernel ----
+        // first copies in flight) the routing for the caller, the down rows
+        // (kWhole) or the handoff to the down kernel ----
         if (!gather_logits(r.logit_ent, T * E, tag, s_logits) && lane == 0)
             atomicOr(p.status, kTimeoutStatus);
         __syncwarp();
@@ -273,42 +305,74 @@ layer_gateup_kernel(const GateUpParams p, const FusedRouteParams r) {
         __syncwarp();
         ring_produce(p, g, ring, full, empty, s_ids, s_tab, lane, [&] {
             const int P = T * k;
-            uint2 *ent = r.hand.ent + (size_t)blockIdx.x * kHandStride * 2;
-            if (lane < P) {
-                st_relaxed_gpu_v2(ent + 2 * lane, tag, (unsigned)s_ids[lane]);
-                st_relaxed_gpu_v2(ent + 2 * lane + 1, tag, __float_as_uint(s_w[lane]));
-                if (blockIdx.x == 0) {
-                    if (p.ids_out) p.ids_out[lane] = s_ids[lane];
-                    if (p.w_out) p.w_out[lane] = s_w[lane];
+            if (kWhole) {
+                if (lane == 0)
+                    issue_down_rows(src, E, H, I, k, s_ids, dr0, dr1, R, rows_c, rows_s, &s_dbar);
+            } else {
+                uint2 *ent = r.hand.ent + (size_t)blockIdx.x * kHandStride * 2;
+                if (lane < P) {
+                    st_relaxed_gpu_v2(ent + 2 * lane, tag, (unsigned)s_ids[lane]);
+                    st_relaxed_gpu_v2(ent + 2 * lane + 1, tag, __float_as_uint(s_w[lane]));
                 }
             }
-            if (lane == 0) st_relaxed_gpu(r.hand.seq + blockIdx.x, tag);
-        });
-        return;
-    }
-
-    // ---- consumer warps: activations from the routed vector in shared memory ----
-    ring_consume<KCH>(p, g, ring, full, empty, s_ids, warp, lane,
-                      [&](int tok, uint32_t (&xw)[KCH][16]) -> float {
-        const int c16 = s_xexp[tok];
-        const float sf = pow2_neg(c16);
-        const uint16_t *v = sx + (size_t)tok * H;
-#pragma unroll
-        for (int u = 0; u < KCH; ++u) {
-            const int c = lane + 32 * u;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint4 raw = c < C ? reinterpret_cast<const uint4 *>(v + (size_t)c * 32)[q]
-                                        : make_uint4(0u, 0u, 0u, 0u);
-                const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    xw[u][q * 4 + i] = f32x2_to_f16x2(bf16_to_f32(w4[i] & 0xFFFFu) * sf,
-                                                      bf16_to_f32(w4[i] >> 16) * sf);
+            if (blockIdx.x == 0 && lane < P) {
+                if (p.ids_out) p.ids_out[lane] = s_ids[lane];
+                if (p.w_out) p.w_out[lane] = s_w[lane];
             }
+            if (lane == 0) {
+                st_relaxed_gpu(r.hand.seq + blockIdx.x, tag);
+                // the down phase runs here: keep the handoff acknowledgement
+                // in step for later two-launch calls on this workspace
+                if (kWhole) st_relaxed_gpu(r.hand.ack + blockIdx.x, tag);
+            }
+        });
+        if (!kWhole) return;
+    } else {
+        // ---- consumer warps: activations from the routed vector in shared memory ----
+        ring_consume<KCH>(p, g, ring, full, empty, s_ids, warp, lane,
+                          [&](int tok, uint32_t (&xw)[KCH][16]) -> float {
+            const int c16 = s_xexp[tok];
+            const float sf = pow2_neg(c16);
+            const uint16_t *v = sx + (size_t)tok * H;
+#pragma unroll
+            for (int u = 0; u < KCH; ++u) {
+                const int c = lane + 32 * u;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 raw = c < C ? reinterpret_cast<const uint4 *>(v + (size_t)c * 32)[q]
+                                            : make_uint4(0u, 0u, 0u, 0u);
+                    const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        xw[u][q * 4 + i] = f32x2_to_f16x2(bf16_to_f32(w4[i] & 0xFFFFu) * sf,
+                                                          bf16_to_f32(w4[i] >> 16) * sf);
+                }
+            }
+            return pow2(c16);
+        }, [&](size_t idx, uint16_t v) {
+            if (kWhole)
+                st_relaxed_gpu_v2(dp.h_tag + idx, tag, v);
+            else
+                p.h[idx] = v;
+        });
+        if (!kWhole) return;
+    }
+    if constexpr (kWhole) {
+        // ---- down phase: stage every h (tagged) -> the CTA's rows ----
+        const int P = T * k;
+        bool ok = stage_h_tagged(dp.h_tag, P, I, tag, sh, s_xs, s_hmax);
+        if (!ok && threadIdx.x == 0) atomicOr(p.status, kTimeoutStatus);
+        ok = __syncthreads_and(ok && mbar_wait(&s_dbar, 0u)) != 0;  // uniform over the CTA
+        DownRows<TLD, KCHD, true> rows(H, I, k, E, R, dr0, dr1, src, s_ids, rows_c, rows_s);
+        if (ok) {
+            rows.fetch(rows.rr);
+            rows.run(sh, s_xs, so, p.status);
         }
-        return pow2(c16);
-    });
+        __syncthreads();
+        if (ok) down_combine(dr0, dr1, H, k, R, so, s_w, dp.residual, dp.y, nullptr);
+        // no row copy may outlive the CTA (complete unless its wait timed out)
+        if (!ok && threadIdx.x == 0) mbar_wait(&s_dbar, 0u);
+    }
 }
 
 // ------------------------------------------------------------------ host --
@@ -332,14 +396,38 @@ bool layer_gateup_plan(int T, int E, int H, int grid, size_t *smem, int *nslots,
     return true;
 }
 
+bool layer_plan(int T, int E, int H, int I, int k, int grid, size_t *smem, int *nslots,
+                unsigned *region_bytes, unsigned *down_off, int *rows_per_cta) {
+    if (T < 1 || T > kDecodeMaxT || E < 1 || E > kFusedMaxE || k < 1 || k > kMaxTopK) return false;
+    if (grid < 1 || grid > kHandMaxCtas) return false;
+    if (!gateup_tma_supported(H) || H > 2048 || I % 512 != 0 || I > 4096) return false;
+    if (kDownWarps < k) return false;
+    const int R = (T * H + grid - 1) / grid;
+    const size_t sx = (size_t)T * H * 2;
+    const size_t down = down_rows_smem(T, k, I, R);
+    const size_t slot = tma_slot_bytes(H);
+    if (sx + down + 2 * slot > kFusedSmemBudget) return false;
+    size_t n = (kFusedSmemBudget - sx - down - 128) / slot;
+    if (n > (size_t)kTmaMaxSlots) n = kTmaMaxSlots;
+    const size_t region = (n * slot + 127) & ~(size_t)127;
+    const size_t doff = region + sx;  // 16-byte aligned: sx is a multiple of 1024
+    if (doff + down > kFusedSmemBudget) return false;
+    *smem = doff + down;
+    *nslots = (int)n;
+    *region_bytes = (unsigned)region;
+    *down_off = (unsigned)doff;
+    *rows_per_cta = R;
+    return true;
+}
+
 namespace {
 
-template <int KCH>
-cudaError_t launch_fused(const GateUpParams &p, const FusedRouteParams &r, int grid, size_t smem,
-                         cudaStream_t s, bool pdl) {
+template <int KCH, int TLD, int KCHD>
+cudaError_t launch_lk(const GateUpParams &p, const FusedRouteParams &r, const LayerDownParams &d,
+                      int grid, size_t smem, cudaStream_t s, bool pdl) {
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(layer_gateup_kernel<KCH>,
+        cudaError_t e = cudaFuncSetAttribute(layer_kernel<KCH, TLD, KCHD>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kFusedSmemBudget);
         if (e != cudaSuccess) return e;
@@ -352,26 +440,53 @@ cudaError_t launch_fused(const GateUpParams &p, const FusedRouteParams &r, int g
     cfg.stream = s;
     // One CTA per SM and grid = SM count: every CTA becomes resident as the
     // previous kernel's CTAs leave (nothing else runs on the stream), which the
-    // logit polling relies on; the polls are bounded all the same.  No
-    // cooperative attribute: it would hold every CTA back until the whole GPU
-    // is free and lose the overlap with the previous kernel.
+    // logit polling and the done words rely on; the waits are bounded all the
+    // same.  No cooperative attribute: it would hold every CTA back until the
+    // whole GPU is free and lose the overlap with the previous kernel.
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, layer_gateup_kernel<KCH>, p, r);
+    return cudaLaunchKernelEx(&cfg, layer_kernel<KCH, TLD, KCHD>, p, r, d);
+}
+
+template <int KCH>
+cudaError_t launch_whole(const GateUpParams &p, const FusedRouteParams &r, const LayerDownParams &d,
+                         int grid, size_t smem, cudaStream_t s, bool pdl) {
+    int tl, kch;
+    pick_team(p.I / 32, tl, kch);
+    switch (tl * 10 + kch) {
+    case 161: return launch_lk<KCH, 16, 1>(p, r, d, grid, smem, s, pdl);
+    case 321: return launch_lk<KCH, 32, 1>(p, r, d, grid, smem, s, pdl);
+    case 163: return launch_lk<KCH, 16, 3>(p, r, d, grid, smem, s, pdl);
+    case 322: return launch_lk<KCH, 32, 2>(p, r, d, grid, smem, s, pdl);
+    case 323: return launch_lk<KCH, 32, 3>(p, r, d, grid, smem, s, pdl);
+    case 324: return launch_lk<KCH, 32, 4>(p, r, d, grid, smem, s, pdl);
+    default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace
 
 cudaError_t launch_layer_gateup(const GateUpParams &p, const FusedRouteParams &r, int grid,
                                 size_t smem, cudaStream_t s, bool pdl) {
+    const LayerDownParams none = {};
     switch ((p.H / 32 + 31) / 32) {
-    case 1: return launch_fused<1>(p, r, grid, smem, s, pdl);
-    case 2: return launch_fused<2>(p, r, grid, smem, s, pdl);
-    case 3: return launch_fused<3>(p, r, grid, smem, s, pdl);
-    case 4: return launch_fused<4>(p, r, grid, smem, s, pdl);
+    case 1: return launch_lk<1, 0, 0>(p, r, none, grid, smem, s, pdl);
+    case 2: return launch_lk<2, 0, 0>(p, r, none, grid, smem, s, pdl);
+    case 3: return launch_lk<3, 0, 0>(p, r, none, grid, smem, s, pdl);
+    case 4: return launch_lk<4, 0, 0>(p, r, none, grid, smem, s, pdl);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_layer(const GateUpParams &p, const FusedRouteParams &r,
+                         const LayerDownParams &d, int grid, size_t smem, cudaStream_t s,
+                         bool pdl) {
+    switch ((p.H / 32 + 31) / 32) {
+    case 1: return launch_whole<1>(p, r, d, grid, smem, s, pdl);
+    case 2: return launch_whole<2>(p, r, d, grid, smem, s, pdl);
     default: return cudaErrorInvalidValue;
     }
 }

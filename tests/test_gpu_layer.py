@@ -1,7 +1,8 @@
-"""moe_layer_ex: the one-launch router + gate/up path (CTA pairs exchanging
-router halves through distributed shared memory, routing handed to the down
-launch through the workspace) against the separate router launch and against
-moe_route_ex + moe_forward_ex, bit for bit, and against the oracle."""
+"""moe_layer_ex in its three launch structures -- the whole layer in one
+launch, the router inside the gate/up launch (logits exchanged between CTAs and
+the routing handed to the down launch through tagged workspace words), and
+separate launches -- against each other and against moe_route_ex +
+moe_forward_ex, bit for bit, and against the oracle."""
 import numpy as np
 import pytest
 import torch
@@ -47,6 +48,8 @@ def _host(b):
     (synth.L24B, 1, False, True), (synth.L24B, 2, False, True), (synth.L24B, 4, True, False),
     (synth.L8B, 3, True, True), (synth.TINY, 1, False, False), (synth.TINY, 4, True, True)])
 def test_fused_layer_bitwise_equals_unfused_and_split(shape, T, bias, rmsnorm):
+    """Every launch structure gives the same bits (the one-launch layer falls
+    back to two launches where its shared memory plan does not fit)."""
     L = synth.make_layer(shape, seed=51, bias=bias)
     codes, scales, rw, rb = dev_layer(L)
     layer = moe.MoELayer(shape.E, shape.H, shape.I, shape.top_k, codes, scales, rw, rb,
@@ -57,17 +60,20 @@ def test_fused_layer_bitwise_equals_unfused_and_split(shape, T, bias, rmsnorm):
         x = dev_bf16(synth.make_tokens(T, shape.H, seed=51, stream=call))
         res = dev_bf16(synth.make_tokens(T, shape.H, seed=52, stream=call)) if call % 2 else None
         outs = {}
-        for mode in ("fused", "unfused", "split"):
+        modes = {"layer": moe.FUSION_LAYER, "fused": moe.FUSION_ROUTER,
+                 "unfused": moe.FUSION_NONE, "split": None}
+        for mode, fusion in modes.items():
             b = _bufs(T, shape)
-            moe.moe_set_fusion(layer.handle, mode == "fused")
-            (_split if mode == "split" else _layer_ex)(layer, x, b, rmsnorm, res)
+            if fusion is not None:
+                moe.moe_set_fusion(layer.handle, fusion)
+            (_split if fusion is None else _layer_ex)(layer, x, b, rmsnorm, res)
             torch.cuda.synchronize()
             outs[mode] = _host(b)
-        assert layer.status() == 0
-        for mode in ("unfused", "split"):
+            assert layer.status() == 0, mode
+        for mode in ("fused", "unfused", "split"):
             for key in ("xn", "logits", "ids", "w", "y"):
-                np.testing.assert_array_equal(outs["fused"][key], outs[mode][key],
-                                              err_msg=f"{key}: fused vs {mode}, call {call}")
+                np.testing.assert_array_equal(outs["layer"][key], outs[mode][key],
+                                              err_msg=f"{key}: one launch vs {mode}, call {call}")
         # and the result is the oracle's layer (routing checked with near-tie care)
         xr = host_bf16(x)
         xn_r = oracle.rmsnorm(xr) if rmsnorm else xr
@@ -85,20 +91,27 @@ def test_fused_layer_bitwise_equals_unfused_and_split(shape, T, bias, rmsnorm):
     layer.close()
 
 
-def test_fused_layer_in_graph_with_shared_workspace():
+@pytest.mark.parametrize("fusion", [1, 2])
+def test_fused_layer_in_graph_with_shared_workspace(fusion):
     """A captured stack of fused layers sharing one workspace replays to the
-    eager bits, replay after replay (the handoff sequence keeps advancing)."""
+    eager bits, replay after replay (the per-call tags keep advancing)."""
     shape = synth.L24B
     layers = [synth.make_layer(shape, seed=61, layer=l) for l in range(3)]
     st = moe.MoEStack([dev_layer(L) for L in layers], shape.E, shape.H, shape.I, shape.top_k)
     r0 = dev_bf16(synth.make_tokens(1, shape.H, seed=61, stream=1))
-    st.r.copy_(r0)
-    st.enqueue()
-    torch.cuda.synchronize()
-    r1 = host_bf16(st.r).copy()
-    st.enqueue()
-    torch.cuda.synchronize()
-    r2 = host_bf16(st.r).copy()
+    want = {}
+    for mode in (moe.FUSION_NONE, fusion):  # the fused stack matches the unfused one
+        st.set_fusion(mode)
+        st.r.copy_(r0)
+        st.enqueue()
+        torch.cuda.synchronize()
+        r1 = host_bf16(st.r).copy()
+        st.enqueue()
+        torch.cuda.synchronize()
+        want[mode] = (r1, host_bf16(st.r).copy())
+    np.testing.assert_array_equal(want[fusion][0], want[moe.FUSION_NONE][0])
+    np.testing.assert_array_equal(want[fusion][1], want[moe.FUSION_NONE][1])
+    r1, r2 = want[fusion]
     st.r.copy_(r0)
     st.capture()
     for want in (r1, r2):
