@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--no-pdl", action="store_true")
     ap.add_argument("--no-prefetch", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-batched", action="store_true",
+                    help="skip the grouped-path measurements at batch sizes beyond decode")
     ap.add_argument("--layers", type=int, default=N_LAYERS,
                     help="layers in the stack (fewer: a smaller case for profiling; "
                          "the bench workload is the full stack)")
@@ -61,6 +63,23 @@ def parse_args():
 def dist_env():
     return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
             int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def max_over_ranks(value, world, device):
+    """The largest of every rank's value (the job ends when its slowest rank
+    does); the value itself on a single rank."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank, world, t_ms):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * world / (t_ms / 1e3)
 
 
 def load_peaks():
@@ -298,12 +317,8 @@ def run_ours(args):
         torch.cuda.synchronize()
         barrier()
     t_ms = e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([t_ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_ms = float(tt.item())
-    tokens = TOKENS_PER_STEP * args.steps * world
-    tok_s = tokens / (t_ms / 1e3)
+    t_ms = max_over_ranks(t_ms, world, "cuda")
+    tok_s = job_throughput(TOKENS_PER_STEP * args.steps, world, t_ms)
 
     # bytes per token from the routing of the last replay (distinct experts)
     ids = st.ids.cpu().numpy()
@@ -320,6 +335,9 @@ def run_ours(args):
 
     # ---- end to end through the public API with host buffers ----
     e2e = run_e2e(torch, st, args)
+
+    # ---- the grouped path at batch sizes beyond decode (one layer) ----
+    batched = batched_cases(torch, moe, st, args.seed) if not args.skip_batched else None
 
     out = {
         "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world,
@@ -343,6 +361,7 @@ def run_ours(args):
                      "bytes_per_launch": gu_bytes, "peak_kind": peak_kind},
         "kernels": kern,
         "e2e": e2e,
+        "batched": batched,
         "gpu_launches": 3 * n_layers * TOKENS_PER_STEP * args.steps,
         "clocks": clk.summary(),
     }
@@ -399,6 +418,55 @@ def kernel_breakdown(torch, moe, st, reps):
     return {"route_us": route, "gateup_us": gu, "down_us": dn,
             "share": {"route": route / total, "gateup": gu / total, "down": dn / total},
             "launches_timed_per_kind": cnt}
+
+
+BATCHED_CASES = ((32, "uniform"), (32, "zipf"), (64, "uniform"), (256, "uniform"),
+                 (256, "zipf"))
+
+
+def batched_cases(torch, moe, st, seed, reps=20):
+    """The grouped (token, expert)-sorted path on one 24B layer of the stack at
+    batch sizes beyond decode: synthetic routing (k distinct experts per token,
+    uniform or Zipf(1.1) popularity), moe_forward timed in a CUDA graph of
+    `reps` calls.  Bytes: the touched experts' packed weights + activations."""
+    L = st.layers[0]
+    out = []
+    expert = 3 * SHAPE.I * SHAPE.H // 2 + 3 * SHAPE.I * SHAPE.H // 32
+    tmax = max(t for t, _ in BATCHED_CASES)
+    lay = moe.MoELayer(SHAPE.E, SHAPE.H, SHAPE.I, SHAPE.top_k, L.codes, L.scales, L.router_w,
+                       L.router_b, max_tokens=tmax)
+    s = torch.cuda.Stream()
+    for T, dist in BATCHED_CASES:
+        x = torch.from_numpy(synth.make_tokens(T, SHAPE.H, seed=seed, stream=T)
+                             .view(np.int16)).cuda().view(torch.bfloat16)
+        ids_h, w_h = synth.make_routing(T, SHAPE.E, SHAPE.top_k, dist,
+                                        synth.rng_for(seed, 91, T))
+        ids, w = torch.from_numpy(ids_h).cuda(), torch.from_numpy(w_h).cuda()
+        y = torch.empty_like(x)
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            lay.forward(x, ids, w, y=y, stream=s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(reps):
+                lay.forward(x, ids, w, y=y, stream=s)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / reps
+        touched = len(set(ids_h.ravel().tolist()))
+        nbytes = touched * expert + T * SHAPE.H * 2 * 2
+        out.append({"T": T, "routing": dist, "experts_touched": touched,
+                    "us_per_call": us, "tokens_per_s": T / (us * 1e-6),
+                    "hbm_gbs": nbytes / (us * 1e-6) / 1e9})
+        del g
+    lay.close()
+    return out
 
 
 def run_e2e(torch, st, args):

@@ -14,18 +14,20 @@
 //   grouped_prep_kernel      CTA 0: stable counting sort of the T k (token,
 //                            slot) pairs by expert -> perm, offs.  CTAs 1..T:
 //                            FP16 staging of each token's activations.
-//   grouped_mma_kernel<2>    per (expert, 32 gate/up rows): h = SwiGLU of the
+//   grouped_mma_kernel<2>    per (expert, 16 gate/up rows): h = SwiGLU of the
 //                            expert's tokens, on the tensor cores.
 //   grouped_stage_h_kernel   per pair: FP16 staging of h.
-//   grouped_mma_kernel<1>    per (expert, 32 down rows): o = BF16(W_down h).
+//   grouped_mma_kernel<1>    per (expert, 16 down rows): o = BF16(W_down h).
 //   grouped_combine_kernel   per token: sequential BF16 combine (+ residual).
 //
-// Tensor-core tile.  A CTA holds 32 packed rows of one expert matrix (codes
+// Tensor-core tile.  A CTA holds 16 packed rows of one expert matrix (codes
 // and E8M0 scales, copied to shared memory with 16-byte asynchronous copies
-// into a row-padded layout) and runs 8 warps: 2 row tiles of 16 x 4 quarters
-// of the K groups.  mma.m16n8k16 (FP16 x FP16 -> FP32) takes A = the E2M1
+// into a row-padded layout) and runs 4 warps, one per quarter of the K
+// groups; small tiles keep several CTAs per SM, so one CTA's copies overlap
+// another's products.  mma.m16n8k16 (FP16 x FP16 -> FP32) takes A = the E2M1
 // codes converted to FP16 in registers (exact) and B = the FP16-staged
-// activations of 8 tokens.  Within each 32-element group the K order is
+// activations of 8 tokens (staged to shared memory per chunk of 8, row-padded
+// so that the fragment loads are conflict-free).  Within each 32-element group the K order is
 // permuted identically for A and B so that each thread's A operand is one
 // aligned 4-byte word of the row (8 codes) and its B operand one 16-byte piece
 // of the activation row; the group's partial product (two MMAs, fresh
@@ -42,9 +44,9 @@ namespace moe {
 
 namespace {
 
-constexpr int kGpThreads = 256;   // 8 warps
-constexpr int kGpRows = 32;       // matrix rows per CTA (2 row tiles of 16)
-constexpr int kGpChunk = 32;      // tokens per pass (4 column tiles of 8)
+constexpr int kGpThreads = 256;   // prep / staging / combine CTAs
+constexpr int kMmaThreads = 128;  // product CTAs: 4 warps, one per quarter of K
+constexpr int kGpRows = 16;       // matrix rows per product CTA (one row tile)
 constexpr int kGpMaxE = 1024;
 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
@@ -183,12 +185,12 @@ __global__ void __launch_bounds__(kGpThreads) grouped_prep_kernel(const GroupedP
 }
 
 // -------------------------------------------------- tensor-core products --
-// NMAT = 2: gate and up rows [i0, i0 + 32) of expert blockIdx.y against the
+// NMAT = 2: gate and up rows [i0, i0 + 16) of expert blockIdx.y against the
 // staged activations of its tokens -> h (SwiGLU, BF16) of its pairs.
-// NMAT = 1: down rows [n0, n0 + 32) against the staged h of its pairs ->
+// NMAT = 1: down rows [n0, n0 + 16) against the staged h of its pairs ->
 // o (BF16) of its pairs.
 template <int NMAT>
-__global__ void __launch_bounds__(kGpThreads) grouped_mma_kernel(const GroupedParams p) {
+__global__ void __launch_bounds__(kMmaThreads) grouped_mma_kernel(const GroupedParams p) {
     extern __shared__ __align__(16) uint8_t sm[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int e = blockIdx.y;
@@ -203,12 +205,14 @@ __global__ void __launch_bounds__(kGpThreads) grouped_mma_kernel(const GroupedPa
     const int ng = K >> 5;                   // 32-element groups
     const size_t rc = (size_t)K >> 1, rs = (size_t)K >> 5;
     const size_t rcp = rc + 16, rsp = rs + 16;  // padded row pitches (bank spread)
-    uint8_t *s_codes = sm;                                    // [NMAT][32][rcp]
-    uint8_t *s_scales = sm + (size_t)NMAT * kGpRows * rcp;    // [NMAT][32][rsp]
+    const size_t bp = (size_t)K * 2 + 64;       // padded pitch of a staged B row
+    uint8_t *s_codes = sm;                                    // [NMAT][16][rcp]
+    uint8_t *s_scales = sm + (size_t)NMAT * kGpRows * rcp;    // [NMAT][16][rsp]
     float *s_red = reinterpret_cast<float *>(s_scales + (size_t)NMAT * kGpRows * rsp);
-    // s_red: [3 quarters][2 row tiles][32 lanes][NMAT * 16] partial sums
+    // s_red: [3 quarters][32 lanes][NMAT * 4] partial sums
+    uint8_t *s_b = reinterpret_cast<uint8_t *>(s_red + 3 * 32 * NMAT * 4);  // [8][bp] FP16 rows
 
-    // ---- the 32 rows of each matrix into shared memory ----
+    // ---- the 16 rows of each matrix into shared memory ----
     const int rows = min(kGpRows, M - row0);
 #pragma unroll
     for (int m = 0; m < NMAT; ++m) {
@@ -216,136 +220,127 @@ __global__ void __launch_bounds__(kGpThreads) grouped_mma_kernel(const GroupedPa
         const uint8_t *gc = mat_codes(p, e, mat) + (size_t)row0 * rc;
         const uint8_t *gs = mat_scales(p, e, mat) + (size_t)row0 * rs;
         const int c16 = (int)(rc >> 4);
-        for (int i = threadIdx.x; i < rows * c16; i += kGpThreads) {
+        for (int i = threadIdx.x; i < rows * c16; i += kMmaThreads) {
             const int r = i / c16, c = i - r * c16;
             cp_async16(s_codes + ((size_t)m * kGpRows + r) * rcp + (size_t)c * 16,
                        gc + (size_t)r * rc + (size_t)c * 16);
         }
         const int c4 = (int)(rs >> 2);
-        for (int i = threadIdx.x; i < rows * c4; i += kGpThreads) {
+        for (int i = threadIdx.x; i < rows * c4; i += kMmaThreads) {
             const int r = i / c4, c = i - r * c4;
             cp_async4(s_scales + ((size_t)m * kGpRows + r) * rsp + (size_t)c * 4,
                       gs + (size_t)r * rs + (size_t)c * 4);
         }
     }
+    // B: the staged FP16 vectors of 8 tokens (x of the pair's token for
+    // gate / up, h of the pair for down), absent ones as zero rows
+    const int cb16 = (int)((size_t)K * 2 >> 4);
+    auto stage_b = [&](int tc) {
+        for (int i = threadIdx.x; i < 8 * cb16; i += kMmaThreads) {
+            const int tk = i / cb16, c = i - tk * cb16;
+            uint8_t *dst = s_b + (size_t)tk * bp + (size_t)c * 16;
+            const int idx = tc + tk;
+            if (idx < n_e) {
+                const int pr = p.perm[seg0 + idx];
+                const uint32_t *src = NMAT == 2 ? p.x16 + (size_t)(pr / p.k) * (K >> 1)
+                                                : p.h16 + (size_t)pr * (K >> 1);
+                cp_async16(dst, reinterpret_cast<const uint8_t *>(src) + (size_t)c * 16);
+            } else {
+                *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+    };
+    stage_b(0);
     cp_async_wait_all();
     __syncthreads();
 
     const int g = lane >> 2, q = lane & 3;
-    const int rt = warp & 1, kq = warp >> 1;  // row tile, K quarter
+    const int kq = warp;  // K quarter
     const int gq = (ng + 3) >> 2;
     const int gb = min(ng, kq * gq), ge = min(ng, gb + gq);
-    const int r_lo = rt * 16 + g, r_hi = r_lo + 8;  // this thread's two A rows
+    const int r_lo = g, r_hi = g + 8;  // this thread's two A rows
     const float zero[4] = {0.f, 0.f, 0.f, 0.f};
 
     #pragma unroll 1
-    for (int tc = 0; tc < n_e; tc += kGpChunk) {
-        // B rows (activation vectors) of this thread's column in each of the 4
-        // column tiles: column g of tile nt is token tc + 8 nt + g of the group
-        const uint32_t *brow[4];
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-            const int idx = tc + nt * 8 + g;
-            brow[nt] = nullptr;
-            if (idx < n_e) {
-                const int pr = p.perm[seg0 + idx];
-                brow[nt] = NMAT == 2 ? p.x16 + (size_t)(pr / p.k) * (K >> 1)
-                                     : p.h16 + (size_t)pr * (K >> 1);
-            }
+    for (int tc = 0; tc < n_e; tc += 8) {
+        if (tc > 0) {
+            stage_b(tc);
+            cp_async_wait_all();
+            __syncthreads();
         }
-        const int ntv = min(4, (n_e - tc + 7) >> 3);  // column tiles in use (uniform)
-        float acc[NMAT][4][4];
+        float acc[NMAT][4];
 #pragma unroll
         for (int m = 0; m < NMAT; ++m)
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) acc[m][nt][i] = 0.f;
+            for (int i = 0; i < 4; ++i) acc[m][i] = 0.f;
+        // column g of the tile is token tc + g of the group
+        const uint8_t *bcol = s_b + (size_t)g * bp + 16 * q;
 
-        #pragma unroll 1
+        #pragma unroll 2
         for (int G = gb; G < ge; ++G) {
-            uint32_t fa[NMAT][2][4];  // [mat][row lo / hi][f16x2 of codes 8q..8q+7]
-            float sc[NMAT][2];
+            const uint4 b = *reinterpret_cast<const uint4 *>(bcol + (size_t)G * 64);
 #pragma unroll
             for (int m = 0; m < NMAT; ++m) {
                 const uint8_t *cb = s_codes + (size_t)m * kGpRows * rcp + (size_t)G * 16 + 4 * q;
                 const uint8_t *sb = s_scales + (size_t)m * kGpRows * rsp + G;
-                e2m1x8_to_f16x8(*reinterpret_cast<const uint32_t *>(cb + (size_t)r_lo * rcp), fa[m][0]);
-                e2m1x8_to_f16x8(*reinterpret_cast<const uint32_t *>(cb + (size_t)r_hi * rcp), fa[m][1]);
-                sc[m][0] = e8m0_to_f32(sb[(size_t)r_lo * rsp]);
-                sc[m][1] = e8m0_to_f32(sb[(size_t)r_hi * rsp]);
-            }
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                if (nt < ntv) {
-                    const uint4 b = brow[nt] ? __ldg(reinterpret_cast<const uint4 *>(
-                                                   brow[nt] + (size_t)G * 16 + 4 * q))
-                                             : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-                    for (int m = 0; m < NMAT; ++m) {
-                        float d[4];
-                        // group G: slots 2q, 2q+1 / 2q+8, 2q+9 of the first MMA carry
-                        // elements 8q + {0,1} / {2,3}; of the second 8q + {4,5} / {6,7}
-                        mma_f16(d, fa[m][0][0], fa[m][1][0], fa[m][0][1], fa[m][1][1], b.x, b.y,
-                                zero);
-                        mma_f16(d, fa[m][0][2], fa[m][1][2], fa[m][0][3], fa[m][1][3], b.z, b.w,
-                                d);
-                        acc[m][nt][0] = fmaf(d[0], sc[m][0], acc[m][nt][0]);
-                        acc[m][nt][1] = fmaf(d[1], sc[m][0], acc[m][nt][1]);
-                        acc[m][nt][2] = fmaf(d[2], sc[m][1], acc[m][nt][2]);
-                        acc[m][nt][3] = fmaf(d[3], sc[m][1], acc[m][nt][3]);
-                    }
-                }
+                uint32_t fa[2][4];  // [row lo / hi][f16x2 of codes 8q..8q+7]
+                e2m1x8_to_f16x8(*reinterpret_cast<const uint32_t *>(cb + (size_t)r_lo * rcp), fa[0]);
+                e2m1x8_to_f16x8(*reinterpret_cast<const uint32_t *>(cb + (size_t)r_hi * rcp), fa[1]);
+                const float s_lo = e8m0_to_f32(sb[(size_t)r_lo * rsp]);
+                const float s_hi = e8m0_to_f32(sb[(size_t)r_hi * rsp]);
+                float dd[4];
+                // group G: slots 2q, 2q+1 / 2q+8, 2q+9 of the first MMA carry
+                // elements 8q + {0,1} / {2,3}; of the second 8q + {4,5} / {6,7}
+                mma_f16(dd, fa[0][0], fa[1][0], fa[0][1], fa[1][1], b.x, b.y, zero);
+                mma_f16(dd, fa[0][2], fa[1][2], fa[0][3], fa[1][3], b.z, b.w, dd);
+                acc[m][0] = fmaf(dd[0], s_lo, acc[m][0]);
+                acc[m][1] = fmaf(dd[1], s_lo, acc[m][1]);
+                acc[m][2] = fmaf(dd[2], s_hi, acc[m][2]);
+                acc[m][3] = fmaf(dd[3], s_hi, acc[m][3]);
             }
         }
         // ---- the 4 K quarters, added in order 0, 1, 2, 3 ----
         if (kq > 0) {
-            float *dst = s_red + ((size_t)((kq - 1) * 2 + rt) * 32 + lane) * (NMAT * 16);
+            float *dst = s_red + ((size_t)(kq - 1) * 32 + lane) * (NMAT * 4);
 #pragma unroll
             for (int m = 0; m < NMAT; ++m)
 #pragma unroll
-                for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) dst[(m * 4 + nt) * 4 + i] = acc[m][nt][i];
+                for (int i = 0; i < 4; ++i) dst[m * 4 + i] = acc[m][i];
         }
         __syncthreads();
         if (kq == 0) {
 #pragma unroll
             for (int qq = 1; qq < 4; ++qq) {
-                const float *src = s_red + ((size_t)((qq - 1) * 2 + rt) * 32 + lane) * (NMAT * 16);
+                const float *src = s_red + ((size_t)(qq - 1) * 32 + lane) * (NMAT * 4);
 #pragma unroll
                 for (int m = 0; m < NMAT; ++m)
 #pragma unroll
-                    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) acc[m][nt][i] += src[(m * 4 + nt) * 4 + i];
+                    for (int i = 0; i < 4; ++i) acc[m][i] += src[m * 4 + i];
             }
-            // ---- epilogue: rows r_lo / r_hi, columns 2q, 2q + 1 of each tile ----
+            // ---- epilogue: rows r_lo / r_hi, columns (tokens) 2q, 2q + 1 ----
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
+            for (int cc = 0; cc < 2; ++cc) {
+                const int idx = tc + 2 * q + cc;
+                if (idx >= n_e) continue;
+                const int pr = p.perm[seg0 + idx];
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int idx = tc + nt * 8 + 2 * q + cc;
-                    if (nt >= ntv || idx >= n_e) continue;
-                    const int pr = p.perm[seg0 + idx];
-#pragma unroll
-                    for (int hr = 0; hr < 2; ++hr) {
-                        const int r = row0 + (hr ? r_hi : r_lo);
-                        if (r >= M) continue;
-                        if (NMAT == 2) {
-                            const float xs = pow2(p.x_exp[pr / p.k]);
-                            const float gv = round_bf16(acc[0][nt][hr * 2 + cc] * xs);
-                            const float uv = round_bf16(acc[NMAT - 1][nt][hr * 2 + cc] * xs);
-                            const float sl = round_bf16(gv / (1.0f + expf(-gv)));
-                            p.h[(size_t)pr * M + r] = f32_to_bf16(sl * uv);
-                        } else {
-                            const float hs = pow2(p.h_exp[pr]);
-                            p.o[(size_t)pr * M + r] = f32_to_bf16(acc[0][nt][hr * 2 + cc] * hs);
-                        }
+                for (int hr = 0; hr < 2; ++hr) {
+                    const int r = row0 + (hr ? r_hi : r_lo);
+                    if (r >= M) continue;
+                    if (NMAT == 2) {
+                        const float xs = pow2(p.x_exp[pr / p.k]);
+                        const float gv = round_bf16(acc[0][hr * 2 + cc] * xs);
+                        const float uv = round_bf16(acc[NMAT - 1][hr * 2 + cc] * xs);
+                        const float sl = round_bf16(gv / (1.0f + expf(-gv)));
+                        p.h[(size_t)pr * M + r] = f32_to_bf16(sl * uv);
+                    } else {
+                        const float hs = pow2(p.h_exp[pr]);
+                        p.o[(size_t)pr * M + r] = f32_to_bf16(acc[0][hr * 2 + cc] * hs);
                     }
                 }
+            }
         }
-        __syncthreads();  // s_red is reused by the next chunk
+        __syncthreads();  // s_red and s_b are reused by the next chunk
     }
 }
 
@@ -394,7 +389,8 @@ namespace {
 
 size_t mma_smem(int nmat, int K) {
     const size_t rcp = (size_t)K / 2 + 16, rsp = (size_t)K / 32 + 16;
-    return (size_t)nmat * kGpRows * (rcp + rsp) + (size_t)3 * 2 * 32 * nmat * 16 * sizeof(float);
+    return (size_t)nmat * kGpRows * (rcp + rsp) + (size_t)3 * 32 * nmat * 4 * sizeof(float) +
+           (size_t)8 * ((size_t)K * 2 + 64);
 }
 
 template <int NMAT>
@@ -410,7 +406,7 @@ cudaError_t launch_mma(const GroupedParams &p, cudaStream_t s, bool pdl) {
         attr_smem = smem;
     }
     return launch_ex(grouped_mma_kernel<NMAT>, dim3((M + kGpRows - 1) / kGpRows, p.E),
-                     dim3(kGpThreads), smem, s, pdl, p);
+                     dim3(kMmaThreads), smem, s, pdl, p);
 }
 
 }  // namespace
