@@ -6,9 +6,10 @@
 // top-4 expert execution" (grouped gate / up / down products, activation and
 // multiplication, fused combine keeping sequential BF16 multiply/add
 // rounding) and table "Model and quantization" (E2M1 + E8M0 per 32, BF16
-// activations, FP32 accumulation); the MLX page on quantized MoE ("Gather
-// quantized matmul", sorting the (token, expert) pairs so that each expert's
-// tokens form one contiguous group before the quantized product).
+// activations, FP32 accumulation); page "LFM2.5-8B-A1B — Core AI (.aimodel)",
+// section "Provenance" (its batched SwitchGLU serves the 64-token prefill by
+// sorting the (token, expert) pairs, so that each expert's tokens form one
+// contiguous group before the quantized product).
 //
 // Launch sequence (one stream, programmatic serialization):
 //   grouped_prep_kernel      CTA 0: stable counting sort of the T k (token,
