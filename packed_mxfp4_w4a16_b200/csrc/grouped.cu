@@ -22,19 +22,17 @@
 //   grouped_combine_kernel   per token: sequential BF16 combine (+ residual).
 //
 // Tensor-core tile.  A CTA holds 16 packed rows of one expert matrix (codes
-// and E8M0 scales, copied to shared memory with 16-byte asynchronous copies
-// into a row-padded layout) and runs 4 warps, one per quarter of the K
-// groups; small tiles keep several CTAs per SM, so one CTA's copies overlap
-// another's products.  mma.m16n8k16 (FP16 x FP16 -> FP32) takes A = the E2M1
-// codes converted to FP16 in registers (exact) and B = the FP16-staged
-// activations of 8 tokens (staged to shared memory per chunk of 8, row-padded
-// so that the fragment loads are conflict-free).  Within each 32-element group the K order is
-// permuted identically for A and B so that each thread's A operand is one
-// aligned 4-byte word of the row (8 codes) and its B operand one 16-byte piece
-// of the activation row; the group's partial product (two MMAs, fresh
-// accumulator) is then scaled by the group's E8M0 exponent in FP32 and added
-// to the running FP32 sum, which is exactly per-group scaling.  The K quarters
-// are added in a fixed order at the end.
+// and E8M0 scales; gate and up together) in shared memory and passes the
+// expert's tokens through in chunks of 8 FP16-staged activation rows, all in
+// row-padded layouts (conflict-free fragment loads).
+// mma.m16n8k16 (FP16 x FP16 -> FP32) takes A = the E2M1 codes converted to
+// FP16 in registers (exact) and B = the activations.  Within each 32-element
+// group the K order is permuted identically for A and B so that each thread's
+// A operand is one aligned 4-byte word of the row (8 codes) and its B operand
+// one 16-byte piece of the activation row; the group's partial product (two
+// MMAs, fresh accumulator) is then scaled by the group's E8M0 exponent in
+// FP32 and added to the running FP32 sum, which is exactly per-group scaling.
+// The K quarters (one per warp of a row tile) are added in a fixed order.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -46,8 +44,7 @@ namespace moe {
 namespace {
 
 constexpr int kGpThreads = 256;   // prep / staging / combine CTAs
-constexpr int kMmaThreads = 128;  // product CTAs: 4 warps, one per quarter of K
-constexpr int kGpRows = 16;       // matrix rows per product CTA (one row tile)
+constexpr int kGpRows = 16;       // rows of one MMA row tile
 constexpr int kGpMaxE = 1024;
 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
@@ -57,9 +54,6 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
 __device__ __forceinline__ void cp_async4(void *dst, const void *src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src)
                  : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
 // d = A B + c for one m16n8k16 tile, FP16 operands, FP32 accumulators.
@@ -186,12 +180,28 @@ __global__ void __launch_bounds__(kGpThreads) grouped_prep_kernel(const GroupedP
 }
 
 // -------------------------------------------------- tensor-core products --
-// NMAT = 2: gate and up rows [i0, i0 + 16) of expert blockIdx.y against the
-// staged activations of its tokens -> h (SwiGLU, BF16) of its pairs.
-// NMAT = 1: down rows [n0, n0 + 16) against the staged h of its pairs ->
-// o (BF16) of its pairs.
-template <int NMAT>
-__global__ void __launch_bounds__(kMmaThreads) grouped_mma_kernel(const GroupedParams p) {
+// NMAT = 2: gate and up rows of expert blockIdx.y against the FP16-staged x
+// of its tokens -> h (SwiGLU, BF16) of its pairs.  NMAT = 1: down rows
+// against the staged h of its pairs -> o (BF16) of its pairs.
+//
+// One CTA per (RT row tiles of 16 rows, expert): the tiles' packed rows
+// (codes and E8M0 scales of NMAT matrices) stay in shared memory while the
+// expert's tokens pass through in chunks of 8 (the B tile).  Warp w works on
+// row tile w / 4 and the (w % 4)-th quarter of the K groups; the quarters are
+// added in a fixed order through shared memory and the quarter-0 warp of each
+// tile writes its results.  Several CTAs per SM hide one another's copy and
+// barrier latency.
+
+constexpr int kRowTiles = 1;  // row tiles per CTA
+
+template <int N>
+__device__ __forceinline__ void cp_async_commit_wait() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+template <int NMAT, int RT>
+__global__ void __launch_bounds__(128 * RT) grouped_mma_kernel(const GroupedParams p) {
+    constexpr int kWarps = 4 * RT;
     extern __shared__ __align__(16) uint8_t sm[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int e = blockIdx.y;
@@ -200,73 +210,70 @@ __global__ void __launch_bounds__(kMmaThreads) grouped_mma_kernel(const GroupedP
     const int seg0 = p.offs[e], n_e = p.offs[e + 1] - seg0;
     if (n_e <= 0) return;  // uniform: no token chose this expert
 
-    const int K = NMAT == 2 ? p.H : p.I;     // reduction length
-    const int M = NMAT == 2 ? p.I : p.H;     // rows of the matrix
-    const int row0 = blockIdx.x * kGpRows;
-    const int ng = K >> 5;                   // 32-element groups
-    const size_t rc = (size_t)K >> 1, rs = (size_t)K >> 5;
-    const size_t rcp = rc + 16, rsp = rs + 16;  // padded row pitches (bank spread)
-    const size_t bp = (size_t)K * 2 + 64;       // padded pitch of a staged B row
-    uint8_t *s_codes = sm;                                    // [NMAT][16][rcp]
-    uint8_t *s_scales = sm + (size_t)NMAT * kGpRows * rcp;    // [NMAT][16][rsp]
-    float *s_red = reinterpret_cast<float *>(s_scales + (size_t)NMAT * kGpRows * rsp);
-    // s_red: [3 quarters][32 lanes][NMAT * 4] partial sums
-    uint8_t *s_b = reinterpret_cast<uint8_t *>(s_red + 3 * 32 * NMAT * 4);  // [8][bp] FP16 rows
+    const int K = NMAT == 2 ? p.H : p.I;  // reduction length
+    const int M = NMAT == 2 ? p.I : p.H;  // rows of the matrix (a multiple of 16 RT)
+    const int row0 = blockIdx.x * (kGpRows * RT);
+    const int ng = K >> 5;                // 32-element groups
+    const uint32_t rc = (uint32_t)K >> 1, rs = (uint32_t)K >> 5;
+    const uint32_t rcp = rc + 16, rsp = rs + 16;  // padded row pitches (bank spread)
+    const uint32_t bp = (uint32_t)K * 2 + 64;     // padded pitch of a staged B row
+    constexpr int R = kGpRows * RT;               // rows held by the CTA
+    uint8_t *s_codes = sm;                                      // [NMAT][R][rcp]
+    uint8_t *s_scales = sm + NMAT * R * rcp;                    // [NMAT][R][rsp]
+    float *s_red = reinterpret_cast<float *>(s_scales + NMAT * R * rsp);
+    // s_red: [RT][3 quarters][32 lanes][NMAT * 4] partial sums
+    uint8_t *s_b = reinterpret_cast<uint8_t *>(s_red + RT * 3 * 32 * NMAT * 4);  // [8][bp]
 
-    // ---- the 16 rows of each matrix into shared memory ----
-    const int rows = min(kGpRows, M - row0);
+    // ---- the CTA's rows of each matrix into shared memory ----
 #pragma unroll
     for (int m = 0; m < NMAT; ++m) {
         const int mat = NMAT == 2 ? m : 2;
         const uint8_t *gc = mat_codes(p, e, mat) + (size_t)row0 * rc;
         const uint8_t *gs = mat_scales(p, e, mat) + (size_t)row0 * rs;
-        const int c16 = (int)(rc >> 4);
-        for (int i = threadIdx.x; i < rows * c16; i += kMmaThreads) {
-            const int r = i / c16, c = i - r * c16;
-            cp_async16(s_codes + ((size_t)m * kGpRows + r) * rcp + (size_t)c * 16,
-                       gc + (size_t)r * rc + (size_t)c * 16);
-        }
-        const int c4 = (int)(rs >> 2);
-        for (int i = threadIdx.x; i < rows * c4; i += kMmaThreads) {
-            const int r = i / c4, c = i - r * c4;
-            cp_async4(s_scales + ((size_t)m * kGpRows + r) * rsp + (size_t)c * 4,
-                      gs + (size_t)r * rs + (size_t)c * 4);
+        const int c16 = (int)(rc >> 4), c4 = (int)(rs >> 2);
+        for (int r = warp; r < R; r += kWarps) {
+            uint8_t *dc = s_codes + (m * R + r) * rcp;
+            uint8_t *ds = s_scales + (m * R + r) * rsp;
+            for (int c = lane; c < c16; c += 32) cp_async16(dc + c * 16, gc + r * rc + c * 16);
+            for (int c = lane; c < c4; c += 32) cp_async4(ds + c * 4, gs + r * rs + c * 4);
         }
     }
-    // B: the staged FP16 vectors of 8 tokens (x of the pair's token for
-    // gate / up, h of the pair for down), absent ones as zero rows
-    const int cb16 = (int)((size_t)K * 2 >> 4);
+    // B: the staged FP16 vectors of up to 8 tokens (x of the pair's token for
+    // gate / up, h of the pair for down); the columns of absent tokens hold
+    // whatever the buffer held and only feed results that are not written
+    const int cb16 = K >> 3;
     auto stage_b = [&](int tc) {
-        for (int i = threadIdx.x; i < 8 * cb16; i += kMmaThreads) {
-            const int tk = i / cb16, c = i - tk * cb16;
-            uint8_t *dst = s_b + (size_t)tk * bp + (size_t)c * 16;
+        for (int tk = warp; tk < 8; tk += kWarps) {
             const int idx = tc + tk;
-            if (idx < n_e) {
-                const int pr = p.perm[seg0 + idx];
-                const uint32_t *src = NMAT == 2 ? p.x16 + (size_t)(pr / p.k) * (K >> 1)
-                                                : p.h16 + (size_t)pr * (K >> 1);
-                cp_async16(dst, reinterpret_cast<const uint8_t *>(src) + (size_t)c * 16);
-            } else {
-                *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
-            }
+            if (idx >= n_e) break;
+            const int pr = p.perm[seg0 + idx];
+            const uint8_t *src = reinterpret_cast<const uint8_t *>(
+                NMAT == 2 ? p.x16 + (size_t)(pr / p.k) * (K >> 1) : p.h16 + (size_t)pr * (K >> 1));
+            uint8_t *dst = s_b + tk * bp;
+            for (int c = lane; c < cb16; c += 32) cp_async16(dst + c * 16, src + c * 16);
         }
     };
     stage_b(0);
-    cp_async_wait_all();
+    cp_async_commit_wait<0>();
     __syncthreads();
 
     const int g = lane >> 2, q = lane & 3;
-    const int kq = warp;  // K quarter
+    const int rt = warp >> 2, kq = warp & 3;  // row tile, K quarter
     const int gq = (ng + 3) >> 2;
     const int gb = min(ng, kq * gq), ge = min(ng, gb + gq);
-    const int r_lo = g, r_hi = g + 8;  // this thread's two A rows
     const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+    // this thread's A words (rows g / g + 8 of its tile) and scales
+    const uint8_t *a_lo = s_codes + (rt * kGpRows + g) * rcp + 4 * q;
+    const uint8_t *s_lo = s_scales + (rt * kGpRows + g) * rsp;
+    const uint32_t a_hi = 8 * rcp, sc_hi = 8 * rsp;
+    const uint32_t a_m = R * rcp, sc_m = R * rsp;
+    const uint8_t *bcol = s_b + g * bp + 16 * q;  // column g = token tc + g of the group
 
     #pragma unroll 1
     for (int tc = 0; tc < n_e; tc += 8) {
         if (tc > 0) {
             stage_b(tc);
-            cp_async_wait_all();
+            cp_async_commit_wait<0>();
             __syncthreads();
         }
         float acc[NMAT][4];
@@ -274,35 +281,34 @@ __global__ void __launch_bounds__(kMmaThreads) grouped_mma_kernel(const GroupedP
         for (int m = 0; m < NMAT; ++m)
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[m][i] = 0.f;
-        // column g of the tile is token tc + g of the group
-        const uint8_t *bcol = s_b + (size_t)g * bp + 16 * q;
 
-        #pragma unroll 2
+        #pragma unroll 4
         for (int G = gb; G < ge; ++G) {
-            const uint4 b = *reinterpret_cast<const uint4 *>(bcol + (size_t)G * 64);
+            const uint4 b = *reinterpret_cast<const uint4 *>(bcol + G * 64);
 #pragma unroll
             for (int m = 0; m < NMAT; ++m) {
-                const uint8_t *cb = s_codes + (size_t)m * kGpRows * rcp + (size_t)G * 16 + 4 * q;
-                const uint8_t *sb = s_scales + (size_t)m * kGpRows * rsp + G;
-                uint32_t fa[2][4];  // [row lo / hi][f16x2 of codes 8q..8q+7]
-                e2m1x8_to_f16x8(*reinterpret_cast<const uint32_t *>(cb + (size_t)r_lo * rcp), fa[0]);
-                e2m1x8_to_f16x8(*reinterpret_cast<const uint32_t *>(cb + (size_t)r_hi * rcp), fa[1]);
-                const float s_lo = e8m0_to_f32(sb[(size_t)r_lo * rsp]);
-                const float s_hi = e8m0_to_f32(sb[(size_t)r_hi * rsp]);
+                const uint8_t *cb = a_lo + m * a_m + G * 16;
+                const uint8_t *sb = s_lo + m * sc_m + G;
+                uint32_t fa[2][4];  // [row g / g + 8][f16x2 of codes 8q..8q+7]
+                e2m1x8_to_f16x8(*reinterpret_cast<const uint32_t *>(cb), fa[0]);
+                e2m1x8_to_f16x8(*reinterpret_cast<const uint32_t *>(cb + a_hi), fa[1]);
+                const float sl = e8m0_to_f32(sb[0]);
+                const float sh = e8m0_to_f32(sb[sc_hi]);
                 float dd[4];
                 // group G: slots 2q, 2q+1 / 2q+8, 2q+9 of the first MMA carry
                 // elements 8q + {0,1} / {2,3}; of the second 8q + {4,5} / {6,7}
                 mma_f16(dd, fa[0][0], fa[1][0], fa[0][1], fa[1][1], b.x, b.y, zero);
                 mma_f16(dd, fa[0][2], fa[1][2], fa[0][3], fa[1][3], b.z, b.w, dd);
-                acc[m][0] = fmaf(dd[0], s_lo, acc[m][0]);
-                acc[m][1] = fmaf(dd[1], s_lo, acc[m][1]);
-                acc[m][2] = fmaf(dd[2], s_hi, acc[m][2]);
-                acc[m][3] = fmaf(dd[3], s_hi, acc[m][3]);
+                acc[m][0] = fmaf(dd[0], sl, acc[m][0]);
+                acc[m][1] = fmaf(dd[1], sl, acc[m][1]);
+                acc[m][2] = fmaf(dd[2], sh, acc[m][2]);
+                acc[m][3] = fmaf(dd[3], sh, acc[m][3]);
             }
         }
-        // ---- the 4 K quarters, added in order 0, 1, 2, 3 ----
+        // ---- the 4 K quarters of each row tile, added in order 0, 1, 2, 3 ----
+        float *red = s_red + rt * (3 * 32 * NMAT * 4);
         if (kq > 0) {
-            float *dst = s_red + ((size_t)(kq - 1) * 32 + lane) * (NMAT * 4);
+            float *dst = red + ((kq - 1) * 32 + lane) * (NMAT * 4);
 #pragma unroll
             for (int m = 0; m < NMAT; ++m)
 #pragma unroll
@@ -312,13 +318,13 @@ __global__ void __launch_bounds__(kMmaThreads) grouped_mma_kernel(const GroupedP
         if (kq == 0) {
 #pragma unroll
             for (int qq = 1; qq < 4; ++qq) {
-                const float *src = s_red + ((size_t)(qq - 1) * 32 + lane) * (NMAT * 4);
+                const float *src = red + ((qq - 1) * 32 + lane) * (NMAT * 4);
 #pragma unroll
                 for (int m = 0; m < NMAT; ++m)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) acc[m][i] += src[m * 4 + i];
             }
-            // ---- epilogue: rows r_lo / r_hi, columns (tokens) 2q, 2q + 1 ----
+            // ---- epilogue: rows g / g + 8 of the tile, columns (tokens) 2q, 2q + 1 ----
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
                 const int idx = tc + 2 * q + cc;
@@ -326,8 +332,7 @@ __global__ void __launch_bounds__(kMmaThreads) grouped_mma_kernel(const GroupedP
                 const int pr = p.perm[seg0 + idx];
 #pragma unroll
                 for (int hr = 0; hr < 2; ++hr) {
-                    const int r = row0 + (hr ? r_hi : r_lo);
-                    if (r >= M) continue;
+                    const int r = row0 + rt * kGpRows + g + 8 * hr;
                     if (NMAT == 2) {
                         const float xs = pow2(p.x_exp[pr / p.k]);
                         const float gv = round_bf16(acc[0][hr * 2 + cc] * xs);
@@ -341,7 +346,7 @@ __global__ void __launch_bounds__(kMmaThreads) grouped_mma_kernel(const GroupedP
                 }
             }
         }
-        __syncthreads();  // s_red and s_b are reused by the next chunk
+        if (tc + 8 < n_e) __syncthreads();  // s_red and s_b are reused by the next chunk
     }
 }
 
@@ -382,15 +387,14 @@ __global__ void __launch_bounds__(kGpThreads) grouped_combine_kernel(const Group
 
 // ------------------------------------------------------------------ host --
 
-bool grouped_supported(int E, int H, int I) {
-    return E <= kGpMaxE && H % 128 == 0 && I % 128 == 0 && H <= 4096 && I <= 4096;
-}
-
 namespace {
 
+constexpr size_t kMmaSmemBudget = 220 * 1024;
+
 size_t mma_smem(int nmat, int K) {
+    const size_t R = (size_t)kGpRows * kRowTiles;
     const size_t rcp = (size_t)K / 2 + 16, rsp = (size_t)K / 32 + 16;
-    return (size_t)nmat * kGpRows * (rcp + rsp) + (size_t)3 * 32 * nmat * 4 * sizeof(float) +
+    return (size_t)nmat * R * (rcp + rsp) + (size_t)kRowTiles * 3 * 32 * nmat * 4 * sizeof(float) +
            (size_t)8 * ((size_t)K * 2 + 64);
 }
 
@@ -400,17 +404,23 @@ cudaError_t launch_mma(const GroupedParams &p, cudaStream_t s, bool pdl) {
     const size_t smem = mma_smem(NMAT, K);
     static size_t attr_smem = 0;  // largest dynamic shared memory enabled so far
     if (smem > attr_smem) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_mma_kernel<NMAT>,
+        cudaError_t e = cudaFuncSetAttribute(grouped_mma_kernel<NMAT, kRowTiles>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
         attr_smem = smem;
     }
-    return launch_ex(grouped_mma_kernel<NMAT>, dim3((M + kGpRows - 1) / kGpRows, p.E),
-                     dim3(kMmaThreads), smem, s, pdl, p);
+    return launch_ex(grouped_mma_kernel<NMAT, kRowTiles>, dim3(M / (kGpRows * kRowTiles), p.E),
+                     dim3(128 * kRowTiles), smem, s, pdl, p);
 }
 
 }  // namespace
+
+bool grouped_supported(int E, int H, int I) {
+    // the pipeline stages of both products must fit the shared memory budget
+    return E <= kGpMaxE && H % 128 == 0 && I % 128 == 0 && H <= 4096 && I <= 4096 &&
+           mma_smem(2, H) <= kMmaSmemBudget && mma_smem(1, I) <= kMmaSmemBudget;
+}
 
 cudaError_t launch_grouped(const GroupedParams &p, cudaStream_t s, bool pdl) {
     if (p.T < 1 || p.T > kGroupedMaxT || !grouped_supported(p.E, p.H, p.I))
