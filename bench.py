@@ -110,10 +110,15 @@ def gateup_bytes(shape, pairs, prefetch_down):
     return pairs * (gu + (dn if prefetch_down else 0))
 
 
+# the translation unit of the decode kernels (gateup_tma_kernel among them)
+# and every header it includes: a change to any of them may change the kernel
+DECODE_TU = ("decode.cu", "down.cuh", "gemv.cuh", "kernels.cuh", "common.cuh")
+
+
 def csrc_digest():
     h = hashlib.sha256()
     d = os.path.join(ROOT, "packed_mxfp4_w4a16_b200", "csrc")
-    for name in sorted(os.listdir(d)):
+    for name in DECODE_TU:
         with open(os.path.join(d, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -380,44 +385,56 @@ def run_ours(args):
 
 
 def kernel_breakdown(torch, moe, st, reps):
-    """Replays a copy of one decode token with an external timing event
-    between every kernel and returns the average duration of each kind."""
+    """Average launch duration of each decode kernel kind, measured live: for
+    each kind a CUDA graph holds that kind's launch of every layer, back to
+    back on the stack's stream (programmatic serialization between them, as
+    in the decode graph), timed with CUDA events around whole replays.  The
+    routing of the last decoded token stays in place, so every launch does
+    the work of a real token.  The down-only graph reads its matrices from
+    HBM (no gate/up launch before it stages them into L2)."""
     n = len(st.layers)
-    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
-          for _ in range(n)]
     s = st.stream
     saved = st.r.clone()
-    g = torch.cuda.CUDAGraph()
-    s.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.graph(g, stream=s):
-        for l, L in enumerate(st.layers):
-            ev[l][0].record(s)
-            moe.moe_route_ex(L.handle, st.r, L.router_w, L.router_b, moe.ROUTE_RMSNORM, st.xn,
-                             None, st.ids[l], st.w[l], s)
-            ev[l][1].record(s)
-            moe.moe_forward_ex(L.handle, st.xn, st.ids[l], st.w[l], st.r, st.r,
-                               moe.FWD_PHASE_GATEUP, s)
-            ev[l][2].record(s)
-            moe.moe_forward_ex(L.handle, st.xn, st.ids[l], st.w[l], st.r, st.r,
-                               moe.FWD_PHASE_DOWN, s)
-            ev[l][3].record(s)
-    tot = [0.0, 0.0, 0.0]
-    for i in range(reps + 2):
-        g.replay()
+
+    def route(l, L):
+        moe.moe_route_ex(L.handle, st.r, L.router_w, L.router_b, moe.ROUTE_RMSNORM, st.xn, None,
+                         st.ids[l], st.w[l], s)
+
+    def gateup(l, L):
+        moe.moe_forward_ex(L.handle, st.xn, st.ids[l], st.w[l], st.r, st.r,
+                           moe.FWD_PHASE_GATEUP, s)
+
+    def down(l, L):
+        moe.moe_forward_ex(L.handle, st.xn, st.ids[l], st.w[l], st.r, st.r,
+                           moe.FWD_PHASE_DOWN, s)
+
+    per = {}
+    for name, fn in (("route", route), ("gateup", gateup), ("down", down)):
+        g = torch.cuda.CUDAGraph()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.graph(g, stream=s):
+            for l, L in enumerate(st.layers):
+                fn(l, L)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(s):  # replays and events on the stack's stream
+            for _ in range(3):
+                g.replay()
+            torch.cuda.synchronize()
+            e0.record(s)
+            for _ in range(reps):
+                g.replay()
+            e1.record(s)
         torch.cuda.synchronize()
-        if i < 2:
-            continue
-        for l in range(n):
-            for q in range(3):
-                tot[q] += ev[l][q].elapsed_time(ev[l][q + 1])
+        per[name] = e0.elapsed_time(e1) * 1e3 / (reps * n)
+        del g
     st.r.copy_(saved)
-    del g
-    cnt = reps * n
-    route, gu, dn = (t / cnt * 1e3 for t in tot)
-    total = route + gu + dn
-    return {"route_us": route, "gateup_us": gu, "down_us": dn,
-            "share": {"route": route / total, "gateup": gu / total, "down": dn / total},
-            "launches_timed_per_kind": cnt}
+    total = sum(per.values())
+    return {"route_us": per["route"], "gateup_us": per["gateup"], "down_us": per["down"],
+            "share": {k: v / total for k, v in per.items()},
+            "launches_timed_per_kind": reps * n,
+            "method": "per kind: a graph of that kind's launch for every layer, back to back "
+                      "with programmatic serialization, CUDA events around the replays"}
 
 
 BATCHED_CASES = ((32, "uniform"), (32, "zipf"), (64, "uniform"), (256, "uniform"),

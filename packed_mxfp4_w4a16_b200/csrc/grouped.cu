@@ -192,7 +192,7 @@ __global__ void __launch_bounds__(kGpThreads) grouped_prep_kernel(const GroupedP
 // tile writes its results.  Several CTAs per SM hide one another's copy and
 // barrier latency.
 
-constexpr int kRowTiles = 1;  // row tiles per CTA
+constexpr int kRowTiles = 2;  // row tiles per CTA
 
 template <int N>
 __device__ __forceinline__ void cp_async_commit_wait() {
@@ -370,18 +370,51 @@ __global__ void __launch_bounds__(kGpThreads) grouped_combine_kernel(const Group
     pdl_wait();
     pdl_launch_dependents();
     const int t = blockIdx.x, k = p.k, H = p.H;
-    for (int n = threadIdx.x; n < H; n += kGpThreads) {
-        float y = 0.f;
-        for (int j = 0; j < k; ++j) {
-            const int pr = t * k + j;
-            const int e = p.ids[pr];
-            const float o = (e >= 0 && e < p.E) ? bf16_to_f32(p.o[(size_t)pr * H + n]) : 0.f;
-            const float wb = round_bf16(p.w[pr]);
-            y = round_bf16(y + round_bf16(o * wb));
-            if (p.o_keep) p.o_keep[(size_t)pr * H + n] = f32_to_bf16(o);
+    // the token's slots: expert ids (validity) and BF16-rounded weights, read
+    // once, before the expert output rows (k <= kMaxTopK)
+    bool ok[kMaxTopK];
+    float wb[kMaxTopK];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+        const int e = j < k ? p.ids[t * k + j] : -1;
+        ok[j] = e >= 0 && e < p.E;
+        wb[j] = j < k ? round_bf16(p.w[t * k + j]) : 0.f;
+    }
+    // 8 consecutive elements per thread (H is a multiple of 128)
+    for (int c = threadIdx.x; c < (H >> 3); c += kGpThreads) {
+        uint4 ov[kMaxTopK];
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j)
+            ov[j] = (j < k && ok[j])
+                        ? reinterpret_cast<const uint4 *>(p.o + (size_t)(t * k + j) * H)[c]
+                        : make_uint4(0u, 0u, 0u, 0u);
+        uint4 rv = make_uint4(0u, 0u, 0u, 0u);
+        if (p.residual) rv = reinterpret_cast<const uint4 *>(p.residual + (size_t)t * H)[c];
+        const uint32_t *rw = &rv.x;
+        uint32_t out[4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float y = 0.f;
+#pragma unroll
+            for (int j = 0; j < kMaxTopK; ++j) {
+                if (j >= k) break;
+                const uint32_t word = (&ov[j].x)[i >> 1];
+                const float o = bf16_to_f32((i & 1) ? word >> 16 : word & 0xFFFFu);
+                y = round_bf16(y + round_bf16(o * wb[j]));
+            }
+            if (p.residual) {
+                const uint32_t word = rw[i >> 1];
+                y = round_bf16(bf16_to_f32((i & 1) ? word >> 16 : word & 0xFFFFu) + y);
+            }
+            const uint32_t b = f32_to_bf16(y);
+            out[i >> 1] = (i & 1) ? (out[i >> 1] | (b << 16)) : b;
         }
-        if (p.residual) y = round_bf16(bf16_to_f32(p.residual[(size_t)t * H + n]) + y);
-        p.y[(size_t)t * H + n] = f32_to_bf16(y);
+        reinterpret_cast<uint4 *>(p.y + (size_t)t * H)[c] = make_uint4(out[0], out[1], out[2], out[3]);
+        if (p.o_keep) {
+#pragma unroll
+            for (int j = 0; j < kMaxTopK; ++j)
+                if (j < k) reinterpret_cast<uint4 *>(p.o_keep + (size_t)(t * k + j) * H)[c] = ov[j];
+        }
     }
 }
 
