@@ -97,6 +97,13 @@ typedef enum moe_status {
 #define MOE_ROUTE_RMSNORM 0x1u /* x is a residual stream r: route
                                   xn = BF16(r / sqrt(mean(r^2) + 1e-6))
                                   and write xn to x_norm */
+#define MOE_ROUTE_SIGMOID 0x2u /* sigmoid scoring: s_e = sigmoid(l_e) of
+                                  the unbiased logit; the k experts with
+                                  the largest s_e + bias_e are selected
+                                  (bias only steers selection); their
+                                  coefficients are s_j / sum of the k
+                                  selected s.  Without it: top-k of the
+                                  (biased) logits, softmax over them.  */
 
 /* Flags of moe_forward_ex. */
 #define MOE_FWD_KEEP_INTERMEDIATES 0x1u /* also store h [T][k][I] and
@@ -170,8 +177,10 @@ MOE_API int moe_route(moe_handle_t h, const uint16_t *x, int T,
 
 /* moe_route plus options.  flags: MOE_ROUTE_RMSNORM (then x_norm, device
  * BF16 [T][H], receives the normalised input that is routed; otherwise
- * x_norm must be NULL).  logits: device FP32 [T][E] that receives the
- * (biased) logits, or NULL. */
+ * x_norm must be NULL) and MOE_ROUTE_SIGMOID (the scoring above).  logits:
+ * device FP32 [T][E] that receives the logits, or NULL: biased with the
+ * softmax scoring, unbiased with MOE_ROUTE_SIGMOID (the bias enters only the
+ * selection key). */
 MOE_API int moe_route_ex(moe_handle_t h, const uint16_t *x, int T,
                  const uint16_t *router_w, const float *router_bias,
                  unsigned flags, uint16_t *x_norm, float *logits,
@@ -203,12 +212,15 @@ MOE_API int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T,
  *   - route_flags MOE_ROUTE_RMSNORM: x is a residual stream r; the layer
  *     routes and runs the experts on xn = BF16(r / sqrt(mean(r^2) + 1e-6)),
  *     written to x_norm (device BF16 [T][H], distinct from x and y).
- *   - logits (device FP32 [T][E] or NULL) receives the (biased) logits;
- *     topk_ids / topk_w (device [T][k] or NULL) receive the routing.
+ *   - route_flags MOE_ROUTE_SIGMOID: sigmoid scoring as in moe_route_ex.
+ *   - logits (device FP32 [T][E] or NULL) receives the logits as in
+ *     moe_route_ex; topk_ids / topk_w (device [T][k] or NULL) receive the
+ *     routing.
  *   - residual (or NULL; may alias y and x) is added as in moe_forward_ex;
  *     fwd_flags may hold MOE_FWD_KEEP_INTERMEDIATES.
- * Results equal moe_route_ex followed by moe_forward_ex.  For T > 4 the
- * call runs exactly that sequence and then topk_ids / topk_w are required.
+ * Results equal moe_route_ex followed by moe_forward_ex.  For T > 4, and
+ * with MOE_ROUTE_SIGMOID, the call runs exactly that sequence and then
+ * topk_ids / topk_w are required.
  * Errors: as moe_route_ex and moe_forward_ex. */
 MOE_API int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T,
                          const uint16_t *router_w, const float *router_bias,

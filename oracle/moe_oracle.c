@@ -19,8 +19,9 @@
  *         execution" (gate GEMV, up GEMV, activation and multiplication,
  *         down GEMV, routing-weighted combination that keeps the serial
  *         runner's sequential BF16 multiply/add rounding); section "GPU
- *         routing inside resident-layer graphs" (router projection, expert
- *         bias where configured, dynamic top-k, routing coefficients).
+ *         routing inside resident-layer graphs" (router projection, sigmoid
+ *         scores, expert bias where configured, dynamic top-k, routing
+ *         coefficients).
  *   [BW]  "LFM2.5-24B-A2B on Your Own Hardware: The RAM, KV Cache and
  *         Bandwidth Budget": section "Where do the 2.45B active parameters
  *         actually go?" (SwiGLU expert = gate, up, down; H=2048, I=1536).
@@ -34,6 +35,11 @@
  *   - Router: logits = x . Wr^T (+ bias[e] if given), not rounded; top-k by
  *     logit, descending, ties to the lower expert id; coefficients =
  *     softmax over the k selected logits.
+ *   - Sigmoid router (the page's own listing of the routing steps, in its
+ *     order): logits l = x . Wr^T (no bias), scores s = 1 / (1 + e^-l), the
+ *     expert bias added to the scores for the selection only, top-k of
+ *     s + bias (ties to the lower id), coefficients = the selected s
+ *     divided by their sum.
  *   - FFN rounding points: g, u -> BF16; s = BF16(silu(g)); h = BF16(s*u);
  *     o = BF16(Wd . h).
  *   - Combine: wb = BF16(w_j); p_j = BF16(o_j * wb_j); y starts at +0 and
@@ -162,6 +168,43 @@ void oracle_select_topk(const double *logits, int E, int k, int32_t *ids,
         w[j] /= z;
 }
 
+/* Sigmoid scoring of one token's unbiased logits: scores s_e = 1/(1+e^-l_e);
+ * selection key s_e + bias[e] (bias may be NULL); top-k of the keys by
+ * repeated arg-max with a strict '>' scanning ids upward (ties to the lower
+ * id); coefficients w_j = s_j / (s_0 + ... + s_{k-1}) of the selected.
+ * [MC] "GPU routing inside resident-layer graphs": sigmoid scores, expert
+ * bias where configured, dynamic top-k selection, routing coefficients. */
+void oracle_select_topk_sigmoid(const double *logits, const float *bias, int E,
+                                int k, int32_t *ids, double *w)
+{
+    double *s = (double *)malloc(sizeof(double) * (size_t)E);
+    double *key = (double *)malloc(sizeof(double) * (size_t)E);
+    char *taken = (char *)calloc((size_t)E, 1);
+    for (int e = 0; e < E; ++e) {
+        s[e] = 1.0 / (1.0 + exp(-logits[e]));
+        key[e] = s[e] + (bias ? (double)bias[e] : 0.0);
+    }
+    for (int j = 0; j < k; ++j) {
+        int best = -1;
+        for (int e = 0; e < E; ++e) {
+            if (taken[e])
+                continue;
+            if (best < 0 || key[e] > key[best])
+                best = e;
+        }
+        taken[best] = 1;
+        ids[j] = best;
+    }
+    double z = 0.0;
+    for (int j = 0; j < k; ++j)
+        z += s[ids[j]];
+    for (int j = 0; j < k; ++j)
+        w[j] = s[ids[j]] / z;
+    free(taken);
+    free(key);
+    free(s);
+}
+
 /* Router projection for T tokens: logits[t][e] = sum_h x[t][h] * Wr[e][h]
  * (+ bias[e] when bias != NULL), then top-k + softmax.
  * [MC] "GPU routing inside resident-layer graphs": router projection, expert
@@ -184,6 +227,29 @@ void oracle_route(const uint16_t *x, int T, int H, const uint16_t *Wr, int E,
                 logits_out[(size_t)t * E + e] = s;
         }
         oracle_select_topk(lg, E, k, ids + (size_t)t * k, w + (size_t)t * k);
+    }
+    free(lg);
+}
+
+/* As oracle_route with sigmoid scoring: the logits stay unbiased (they are
+ * what logits_out receives) and the bias enters the selection key only. */
+void oracle_route_sigmoid(const uint16_t *x, int T, int H, const uint16_t *Wr,
+                          int E, const float *bias, int k, int32_t *ids,
+                          double *w, double *logits_out)
+{
+    double *lg = (double *)malloc(sizeof(double) * (size_t)E);
+    for (int t = 0; t < T; ++t) {
+        for (int e = 0; e < E; ++e) {
+            double s = 0.0;
+            for (int h = 0; h < H; ++h)
+                s += oracle_bf16_to_double(x[(size_t)t * H + h]) *
+                     oracle_bf16_to_double(Wr[(size_t)e * H + h]);
+            lg[e] = s;
+            if (logits_out)
+                logits_out[(size_t)t * E + e] = s;
+        }
+        oracle_select_topk_sigmoid(lg, bias, E, k, ids + (size_t)t * k,
+                                   w + (size_t)t * k);
     }
     free(lg);
 }

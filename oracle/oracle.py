@@ -41,6 +41,8 @@ def _declare(L):
     L.oracle_dequant_f32.argtypes = [vp, vp, i64, vp]
     L.oracle_select_topk.argtypes = [vp, i32, i32, vp, vp]
     L.oracle_route.argtypes = [vp, i32, i32, vp, i32, vp, i32, vp, vp, vp]
+    L.oracle_select_topk_sigmoid.argtypes = [vp, vp, i32, i32, vp, vp]
+    L.oracle_route_sigmoid.argtypes = [vp, i32, i32, vp, i32, vp, i32, vp, vp, vp]
     L.oracle_expert.argtypes = [vp, vp, vp, i32, i32, vp, vp]
     L.oracle_combine.argtypes = [vp, vp, i32, i32, vp, vp]
     L.oracle_moe_forward.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp, vp,
@@ -51,8 +53,9 @@ def _declare(L):
     L.oracle_stack_step.argtypes = [vp, i32, i32, i32, i32, i32, i32, vp, vp,
                                     vp, vp, dbl, vp]
     for name in ("oracle_dequant", "oracle_dequant_f32", "oracle_select_topk",
-                 "oracle_route", "oracle_expert", "oracle_combine",
-                 "oracle_moe_forward", "oracle_moe_layer", "oracle_rmsnorm",
+                 "oracle_select_topk_sigmoid", "oracle_route", "oracle_route_sigmoid",
+                 "oracle_expert", "oracle_combine", "oracle_moe_forward", "oracle_moe_layer",
+                 "oracle_rmsnorm",
                  "oracle_stack_step"):
         getattr(L, name).restype = None
 
@@ -137,9 +140,24 @@ def select_topk(logits: np.ndarray, k: int):
     return ids, w
 
 
-def route(x, router_w, bias, k):
+def select_topk_sigmoid(logits: np.ndarray, bias, k: int):
+    """Sigmoid scoring of each row of unbiased logits [T, E]: top-k of
+    sigmoid(l) + bias, coefficients = the selected sigmoid scores over their
+    sum -> (ids [T,k], w [T,k])."""
+    logits = _c(np.atleast_2d(logits), np.float64)
+    T, E = logits.shape
+    b = _c(bias, np.float32) if bias is not None else None
+    ids = np.empty((T, k), dtype=np.int32)
+    w = np.empty((T, k), dtype=np.float64)
+    for t in range(T):
+        lib().oracle_select_topk_sigmoid(_p(logits[t]), _p(b), E, k, _p(ids[t]), _p(w[t]))
+    return ids, w
+
+
+def route(x, router_w, bias, k, sigmoid=False):
     """x bf16 [T,H], router_w bf16 [E,H], bias f32 [E] or None ->
-    (ids int32 [T,k], w f64 [T,k], logits f64 [T,E])."""
+    (ids int32 [T,k], w f64 [T,k], logits f64 [T,E]).  sigmoid: sigmoid
+    scoring (logits unbiased, bias in the selection key only)."""
     x, router_w = _c(x, np.uint16), _c(router_w, np.uint16)
     T, H = x.shape
     E = router_w.shape[0]
@@ -147,7 +165,8 @@ def route(x, router_w, bias, k):
     ids = np.empty((T, k), dtype=np.int32)
     w = np.empty((T, k), dtype=np.float64)
     lg = np.empty((T, E), dtype=np.float64)
-    lib().oracle_route(_p(x), T, H, _p(router_w), E, _p(b), k, _p(ids), _p(w), _p(lg))
+    fn = lib().oracle_route_sigmoid if sigmoid else lib().oracle_route
+    fn(_p(x), T, H, _p(router_w), E, _p(b), k, _p(ids), _p(w), _p(lg))
     return ids, w, lg
 
 

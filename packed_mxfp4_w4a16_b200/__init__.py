@@ -27,13 +27,14 @@ __all__ = [
     "moe_forward", "moe_forward_ex", "moe_layer_ex", "moe_get_intermediates", "moe_get_status",
     "moe_bytes_per_expert", "moe_set_tuning", "moe_device_check", "moe_debug_dequant",
     "moe_forward_noalloc",
-    "ROUTE_RMSNORM", "FWD_KEEP_INTERMEDIATES", "FWD_FORCE_DECODE", "FWD_FORCE_GROUPED",
+    "ROUTE_RMSNORM", "ROUTE_SIGMOID", "FWD_KEEP_INTERMEDIATES", "FWD_FORCE_DECODE", "FWD_FORCE_GROUPED",
     "FWD_PHASE_GATEUP", "FWD_PHASE_DOWN",
     "FUSION_NONE", "FUSION_ROUTER", "FUSION_LAYER", "moe_set_fusion",
     "DEVICE_BAD_EXPERT_ID",
 ]
 
 ROUTE_RMSNORM = 0x1
+ROUTE_SIGMOID = 0x2
 FWD_KEEP_INTERMEDIATES = 0x1
 FWD_FORCE_DECODE = 0x2
 FWD_FORCE_GROUPED = 0x4
@@ -248,12 +249,13 @@ class MoELayer:
         except Exception:
             pass
 
-    def route(self, x, ids=None, w=None, logits=None, x_norm=None, rmsnorm=False, stream=None):
+    def route(self, x, ids=None, w=None, logits=None, x_norm=None, rmsnorm=False, sigmoid=False,
+              stream=None):
         T = x.shape[0]
         dev = x.device
         ids = ids if ids is not None else torch.empty(T, self.k, dtype=torch.int32, device=dev)
         w = w if w is not None else torch.empty(T, self.k, dtype=torch.float32, device=dev)
-        flags = ROUTE_RMSNORM if rmsnorm else 0
+        flags = (ROUTE_RMSNORM if rmsnorm else 0) | (ROUTE_SIGMOID if sigmoid else 0)
         if rmsnorm and x_norm is None:
             x_norm = torch.empty_like(x)
         moe_route_ex(self.handle, x, self.router_w, self.router_b, flags,

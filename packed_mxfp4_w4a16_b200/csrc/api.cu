@@ -246,7 +246,7 @@ int moe_route_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
                  const float *router_bias, unsigned flags, uint16_t *x_norm, float *logits,
                  int32_t *topk_ids, float *topk_w, void *stream) {
     if (!h || T < 1) return MOE_ERR_ARG;
-    if (flags & ~MOE_ROUTE_RMSNORM) return MOE_ERR_ARG;
+    if (flags & ~(MOE_ROUTE_RMSNORM | MOE_ROUTE_SIGMOID)) return MOE_ERR_ARG;
     const bool norm = flags & MOE_ROUTE_RMSNORM;
     if (norm != (x_norm != nullptr)) return MOE_ERR_ARG;
     if (!h->ws) return MOE_ERR_NOT_LOADED;
@@ -275,6 +275,7 @@ int moe_route_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
     p.H = h->H;
     p.k = h->k;
     p.rmsnorm = norm ? 1 : 0;
+    p.sigmoid = (flags & MOE_ROUTE_SIGMOID) ? 1 : 0;
     p.eps = 1e-6f;
     p.x16 = nullptr;
     p.x16_exp = nullptr;
@@ -441,7 +442,7 @@ int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
                  float *logits, int32_t *topk_ids, float *topk_w, const uint16_t *residual,
                  uint16_t *y, unsigned fwd_flags, void *stream) {
     if (!h || T < 1) return MOE_ERR_ARG;
-    if (route_flags & ~MOE_ROUTE_RMSNORM) return MOE_ERR_ARG;
+    if (route_flags & ~(MOE_ROUTE_RMSNORM | MOE_ROUTE_SIGMOID)) return MOE_ERR_ARG;
     if (fwd_flags & ~MOE_FWD_KEEP_INTERMEDIATES) return MOE_ERR_ARG;
     const bool norm = route_flags & MOE_ROUTE_RMSNORM;
     if (norm != (x_norm != nullptr)) return MOE_ERR_ARG;
@@ -463,8 +464,10 @@ int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
     const WsLayout L = ws_layout(h, h->max_tokens);
     float *lg = reinterpret_cast<float *>(h->ws + L.logits);
 
-    if (T > moe::kDecodeMaxT) {
-        // many tokens: explicit routing, then the forward on the given ids
+    if (T > moe::kDecodeMaxT || (route_flags & MOE_ROUTE_SIGMOID)) {
+        // many tokens, or sigmoid scoring (the fused launch structures select
+        // by softmax scoring only): explicit routing, then the forward on the
+        // given ids
         int32_t *ids = topk_ids;
         float *w = topk_w;
         if (!ids || !w) return MOE_ERR_ARG;
@@ -575,6 +578,7 @@ int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
     }
 
     moe::RouteParams rp;
+    rp.sigmoid = 0;
     rp.x = x;
     rp.wr = router_w;
     rp.bias = router_bias;

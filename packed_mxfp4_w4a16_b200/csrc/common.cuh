@@ -86,6 +86,42 @@ __device__ __forceinline__ void e2m1x8_to_f16x8(uint32_t w, uint32_t (&out)[4]) 
         : "r"(w));
 }
 
+// d = A B + c for one m16n8k16 tile, FP16 operands, FP32 accumulators.
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                        uint32_t a3, uint32_t b0, uint32_t b1, const float (&c)[4]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%10, %11, %12, %13};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(c[2]),
+          "f"(c[3]));
+}
+
+// One 32-element scale group of 16 packed rows against 8 FP16 columns on the
+// tensor cores, scaled per row by the group's E8M0 exponent and added to acc.
+// The group's K order is permuted identically for A and B: thread (g, q) of
+// the warp supplies codes 8q..8q+7 of rows g and g+8 (one 4-byte word each,
+// w_lo / w_hi) and elements 8q..8q+7 of column g (b).  Slots 2q, 2q+1 / 2q+8,
+// 2q+9 of the first MMA then carry elements 8q + {0,1} / {2,3}, of the second
+// 8q + {4,5} / {6,7}.  The group's partial product (fresh accumulator) times
+// the row's 2^(e-127) is added in FP32: exactly per-group scaling.
+// acc: rows g / g + 8 x columns 2q, 2q + 1 (acc[0], acc[1] / acc[2], acc[3]).
+__device__ __forceinline__ void mma_group_e2m1(float (&acc)[4], uint32_t w_lo, uint32_t w_hi,
+                                               uint32_t s_lo, uint32_t s_hi, const uint4 &b) {
+    uint32_t fa[2][4];
+    e2m1x8_to_f16x8(w_lo, fa[0]);
+    e2m1x8_to_f16x8(w_hi, fa[1]);
+    const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+    float dd[4];
+    mma_f16(dd, fa[0][0], fa[1][0], fa[0][1], fa[1][1], b.x, b.y, zero);
+    mma_f16(dd, fa[0][2], fa[1][2], fa[0][3], fa[1][3], b.z, b.w, dd);
+    const float sl = e8m0_to_f32(s_lo), sh = e8m0_to_f32(s_hi);
+    acc[0] = fmaf(dd[0], sl, acc[0]);
+    acc[1] = fmaf(dd[1], sl, acc[1]);
+    acc[2] = fmaf(dd[2], sh, acc[2]);
+    acc[3] = fmaf(dd[3], sh, acc[3]);
+}
+
 __device__ __forceinline__ float f16_bits_to_f32(uint32_t h) {
     float f;
     asm("{ .reg .f16 t; mov.b16 t, %1; cvt.f32.f16 %0, t; }" : "=f"(f) : "h"((uint16_t)h));
@@ -236,14 +272,40 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, unsigned parity) {
     return false;
 }
 
-// global -> shared bulk copy completing `bytes` on `bar`
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, unsigned bytes,
-                                         uint64_t *bar) {
+// L2 eviction priorities for cache-hinted accesses.  The packed expert rows
+// are read once per token and stream through L2 far faster than it holds
+// them (hundreds of MB per token against 126 MB): marked evict-first, they
+// leave the small state that every layer reuses (router weights, activations,
+// routing, kernel code) in L2.  The router weights are marked evict-last.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// Global -> shared bulk copy completing `bytes` on `bar`, with an L2
+// eviction policy for the source lines.
+__device__ __forceinline__ void bulk_g2s_hint(void *dst, const void *src, unsigned bytes,
+                                              uint64_t *bar, uint64_t pol) {
     asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-            "r"(smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
+        "[%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
         : "memory");
+}
+
+// 16-byte global load with an L2 eviction policy.
+__device__ __forceinline__ uint4 ld_hint16(const void *p, uint64_t pol) {
+    uint4 r;
+    asm volatile("ld.global.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p), "l"(pol));
+    return r;
 }
 
 // ------------------------------------------------------------- warps -----
@@ -282,19 +344,29 @@ __device__ __forceinline__ uint32_t logit_key(float v) {
 }
 
 // Top-k of one token's E logits by one warp (strictly greater wins, the lower
-// expert id on equal logits), then the softmax of the k chosen logits.  Lane j
-// (j < k) returns the j-th selection in (id, w); other lanes return id = -1.
-// Round j takes the warp-wide max key and the lowest id holding it, then
-// clears that key; k rounds, one redux pair each.
+// expert id on equal keys), then the coefficients.  Lane j (j < k) returns
+// the j-th selection in (id, w); other lanes return id = -1.  Round j takes
+// the warp-wide max key and the lowest id holding it, then clears that key;
+// k rounds, one redux pair each.
+// SIG false: key = the logit, w = softmax over the k chosen logits.
+// SIG true: s_e = sigmoid(l_e) in FP32, key = s_e + bias[e] (bias may be
+// null), w = s_j / sum of the k chosen s.
 // SMEM: the logits are in shared memory (else global memory, read through L2).
-template <int PER, bool SMEM = false>  // logits per lane: E <= 32 * PER
+template <int PER, bool SMEM = false, bool SIG = false>  // logits per lane: E <= 32 * PER
 __device__ __forceinline__ void warp_topk(const float *lg, int E, int k, int lane, int &id,
-                                          float &w) {
+                                          float &w, const float *bias = nullptr) {
     uint32_t key[PER];
+    float sv[PER];
 #pragma unroll
     for (int m = 0; m < PER; ++m) {
         const int e = lane + 32 * m;
-        key[m] = e < E ? logit_key(SMEM ? lg[e] : __ldcg(lg + e)) : 0u;
+        const float l = e < E ? (SMEM ? lg[e] : __ldcg(lg + e)) : 0.f;
+        if (SIG) {
+            sv[m] = 1.0f / (1.0f + expf(-l));
+            key[m] = e < E ? logit_key(sv[m] + (bias ? __ldg(bias + e) : 0.f)) : 0u;
+        } else {
+            key[m] = e < E ? logit_key(l) : 0u;
+        }
     }
     id = -1;
     float mylv = 0.f, top = 0.f;
@@ -310,7 +382,15 @@ __device__ __forceinline__ void warp_topk(const float *lg, int E, int k, int lan
             }
         const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
         const int wi = (int)__reduce_min_sync(0xffffffffu, bk == wk ? (uint32_t)bi : 0x7FFFFFFFu);
-        const float lv = __uint_as_float((wk & 0x80000000u) ? (wk & 0x7FFFFFFFu) : ~wk);
+        float lv = __uint_as_float((wk & 0x80000000u) ? (wk & 0x7FFFFFFFu) : ~wk);
+        if (SIG) {
+            // the chosen expert's unbiased score, from the lane that holds it
+            float mine_s = 0.f;
+#pragma unroll
+            for (int m = 0; m < PER; ++m)
+                if ((wi >> 5) == m) mine_s = sv[m];
+            lv = __shfl_sync(0xffffffffu, mine_s, wi & 31);
+        }
         if (j == 0) top = lv;
         if (lane == j) {
             id = wi;
@@ -320,8 +400,8 @@ __device__ __forceinline__ void warp_topk(const float *lg, int E, int k, int lan
         for (int m = 0; m < PER; ++m)
             if (wi == lane + 32 * m) key[m] = 0u;
     }
-    // softmax over the chosen logits: lane j < k holds exp(l_j - l_0)
-    const float mine = lane < k ? expf(mylv - top) : 0.f;
+    // SIG: lane j < k holds s_j; else exp(l_j - l_0) (softmax)
+    const float mine = lane < k ? (SIG ? mylv : expf(mylv - top)) : 0.f;
     float z = mine;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
@@ -330,22 +410,23 @@ __device__ __forceinline__ void warp_topk(const float *lg, int E, int k, int lan
 
 // Larger expert counts: out of line, to keep the hot kernels' code small.
 // Returns {id, w bits} (by value: no local-memory outputs).
-template <bool SMEM>
-static __device__ __noinline__ uint2 warp_topk_wide(const float *lg, int E, int k, int lane) {
+template <bool SMEM, bool SIG = false>
+static __device__ __noinline__ uint2 warp_topk_wide(const float *lg, int E, int k, int lane,
+                                                    const float *bias) {
     int id;
     float w;
-    warp_topk<32, SMEM>(lg, E, k, lane, id, w);
+    warp_topk<32, SMEM, SIG>(lg, E, k, lane, id, w, bias);
     return make_uint2((unsigned)id, __float_as_uint(w));
 }
 
 // Dispatch on E (up to 1024 experts).
-template <bool SMEM = false>
+template <bool SMEM = false, bool SIG = false>
 __device__ __forceinline__ void warp_topk_any(const float *lg, int E, int k, int lane, int &id,
-                                              float &w) {
+                                              float &w, const float *bias = nullptr) {
     if (E <= 64)
-        warp_topk<2, SMEM>(lg, E, k, lane, id, w);
+        warp_topk<2, SMEM, SIG>(lg, E, k, lane, id, w, bias);
     else {
-        const uint2 r = warp_topk_wide<SMEM>(lg, E, k, lane);
+        const uint2 r = warp_topk_wide<SMEM, SIG>(lg, E, k, lane, bias);
         id = (int)r.x;
         w = __uint_as_float(r.y);
     }

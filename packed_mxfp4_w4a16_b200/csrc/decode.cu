@@ -77,12 +77,12 @@ route_logits_kernel(const RouteParams p) {
     const int e = blockIdx.x, H = p.H, E = p.E;
     const int nch = H >> 3;
     const uint16_t *row = p.wr + (size_t)e * H;
+    const uint64_t pol = l2_evict_last_policy();  // reused by every token
     uint4 wv[kRouteMaxCpt];
 #pragma unroll
     for (int m = 0; m < kRouteMaxCpt; ++m) {
         const int c = tid + kRouteThreads * m;
-        wv[m] = c < nch ? *reinterpret_cast<const uint4 *>(row + (size_t)c * 8)
-                        : make_uint4(0u, 0u, 0u, 0u);
+        wv[m] = c < nch ? ld_hint16(row + (size_t)c * 8, pol) : make_uint4(0u, 0u, 0u, 0u);
     }
     pdl_wait();
     pdl_launch_dependents();
@@ -139,7 +139,9 @@ route_logits_kernel(const RouteParams p) {
         }
         const float logit = block_sum_route(acc, red[1]);
         if (tid == 0) {
-            const float v = p.bias ? logit + p.bias[e] : logit;
+            // sigmoid scoring keeps the logit unbiased (the bias enters the
+            // selection key in the top-k)
+            const float v = (p.bias && !p.sigmoid) ? logit + p.bias[e] : logit;
             p.logits_ws[(size_t)t * E + e] = v;
             if (p.logits_out) p.logits_out[(size_t)t * E + e] = v;
         }
@@ -176,7 +178,10 @@ topk_kernel(const RouteParams p) {
     if (t >= p.T) return;
     int id;
     float w;
-    warp_topk_any(p.logits_ws + (size_t)t * p.E, p.E, p.k, lane, id, w);
+    if (p.sigmoid)
+        warp_topk_any<false, true>(p.logits_ws + (size_t)t * p.E, p.E, p.k, lane, id, w, p.bias);
+    else
+        warp_topk_any(p.logits_ws + (size_t)t * p.E, p.E, p.k, lane, id, w);
     if (lane < p.k) {
         p.ids[(size_t)t * p.k + lane] = id;
         p.w[(size_t)t * p.k + lane] = w;

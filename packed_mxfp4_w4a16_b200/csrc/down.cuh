@@ -51,6 +51,7 @@ static __device__ __noinline__ void issue_down_rows(const DownSrc src, int E, in
                                                     uint8_t *rows_c, uint8_t *rows_s,
                                                     uint64_t *bar) {
     const size_t rc = (size_t)I >> 1, rs = (size_t)I >> 5;
+    const uint64_t pol = l2_evict_first_policy();  // the rows are read once
     unsigned bytes = 0;
     #pragma unroll 1
     for (int pass = 0; pass < 2; ++pass) {
@@ -68,10 +69,10 @@ static __device__ __noinline__ void issue_down_rows(const DownSrc src, int E, in
                     bytes += (unsigned)(cnt * (rc + rs));
                 } else {
                     const size_t li = (size_t)j * R + (size_t)(a - r0);
-                    bulk_g2s(rows_c + li * rc, dsrc_codes(src, e) + n0 * rc, (unsigned)(cnt * rc),
-                             bar);
-                    bulk_g2s(rows_s + li * rs, dsrc_scales(src, e) + n0 * rs, (unsigned)(cnt * rs),
-                             bar);
+                    bulk_g2s_hint(rows_c + li * rc, dsrc_codes(src, e) + n0 * rc,
+                                  (unsigned)(cnt * rc), bar, pol);
+                    bulk_g2s_hint(rows_s + li * rs, dsrc_scales(src, e) + n0 * rs,
+                                  (unsigned)(cnt * rs), bar, pol);
                 }
             }
             a = b;

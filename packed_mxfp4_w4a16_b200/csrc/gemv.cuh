@@ -261,6 +261,7 @@ __device__ __forceinline__ void ring_produce(const GateUpParams &p, const RingGe
     const int cb = g.cb, ce = g.ce, nsteps = g.nsteps, nbar = g.nbar, nslots = g.nslots;
     const size_t rc = g.rc, rs = g.rs, slot_bytes = g.slot_bytes;
     const size_t up_off = g.up_off, gs_off = g.gs_off, us_off = g.us_off;
+    const uint64_t pol = l2_evict_first_policy();  // the rows are read once
     #pragma unroll 1
     for (int q = lane; q < P; q += 32) {
         const int e = s_ids[q];
@@ -317,7 +318,7 @@ __device__ __forceinline__ void ring_produce(const GateUpParams &p, const RingGe
                                      : m == 2 ? ep.scales[0] + i0 * rs
                                               : ep.scales[1] + i0 * rs;
                 const unsigned nb = (unsigned)(m < 2 ? n * rc : n * rs);
-                bulk_g2s(base + dst, src, nb, &full[s]);
+                bulk_g2s_hint(base + dst, src, nb, &full[s], pol);
             }
         }
     }
@@ -352,13 +353,14 @@ __device__ __forceinline__ void ring_produce(const GateUpParams &p, const RingGe
             if (e >= 0 && e < E) {
                 const size_t idx = (size_t)(a - r0), i0 = (size_t)(a - q * I);
                 const ExpertPtrs &ep = s_tab[q];
-                bulk_g2s(base + idx * rc, ep.codes[0] + i0 * rc, (unsigned)(n * rc), &full[b]);
-                bulk_g2s(base + up_off + idx * rc, ep.codes[1] + i0 * rc, (unsigned)(n * rc),
-                         &full[b]);
-                bulk_g2s(base + gs_off + idx * rs, ep.scales[0] + i0 * rs, (unsigned)(n * rs),
-                         &full[b]);
-                bulk_g2s(base + us_off + idx * rs, ep.scales[1] + i0 * rs, (unsigned)(n * rs),
-                         &full[b]);
+                bulk_g2s_hint(base + idx * rc, ep.codes[0] + i0 * rc, (unsigned)(n * rc),
+                              &full[b], pol);
+                bulk_g2s_hint(base + up_off + idx * rc, ep.codes[1] + i0 * rc,
+                              (unsigned)(n * rc), &full[b], pol);
+                bulk_g2s_hint(base + gs_off + idx * rs, ep.scales[0] + i0 * rs,
+                              (unsigned)(n * rs), &full[b], pol);
+                bulk_g2s_hint(base + us_off + idx * rs, ep.scales[1] + i0 * rs,
+                              (unsigned)(n * rs), &full[b], pol);
             }
         }
     }

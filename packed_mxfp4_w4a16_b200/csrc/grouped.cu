@@ -56,17 +56,6 @@ __device__ __forceinline__ void cp_async4(void *dst, const void *src) {
                  : "memory");
 }
 
-// d = A B + c for one m16n8k16 tile, FP16 operands, FP32 accumulators.
-__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                        uint32_t a3, uint32_t b0, uint32_t b1, const float (&c)[4]) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-        "{%8, %9}, {%10, %11, %12, %13};"
-        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]), "f"(c[2]),
-          "f"(c[3]));
-}
-
 __device__ __forceinline__ const uint8_t *mat_codes(const GroupedParams &p, int e, int m) {
     return p.codes_base ? p.codes_base + (size_t)(3 * e + m) * p.codes_stride : p.table[e].codes[m];
 }
@@ -261,7 +250,6 @@ __global__ void __launch_bounds__(128 * RT) grouped_mma_kernel(const GroupedPara
     const int rt = warp >> 2, kq = warp & 3;  // row tile, K quarter
     const int gq = (ng + 3) >> 2;
     const int gb = min(ng, kq * gq), ge = min(ng, gb + gq);
-    const float zero[4] = {0.f, 0.f, 0.f, 0.f};
     // this thread's A words (rows g / g + 8 of its tile) and scales
     const uint8_t *a_lo = s_codes + (rt * kGpRows + g) * rcp + 4 * q;
     const uint8_t *s_lo = s_scales + (rt * kGpRows + g) * rsp;
@@ -289,20 +277,8 @@ __global__ void __launch_bounds__(128 * RT) grouped_mma_kernel(const GroupedPara
             for (int m = 0; m < NMAT; ++m) {
                 const uint8_t *cb = a_lo + m * a_m + G * 16;
                 const uint8_t *sb = s_lo + m * sc_m + G;
-                uint32_t fa[2][4];  // [row g / g + 8][f16x2 of codes 8q..8q+7]
-                e2m1x8_to_f16x8(*reinterpret_cast<const uint32_t *>(cb), fa[0]);
-                e2m1x8_to_f16x8(*reinterpret_cast<const uint32_t *>(cb + a_hi), fa[1]);
-                const float sl = e8m0_to_f32(sb[0]);
-                const float sh = e8m0_to_f32(sb[sc_hi]);
-                float dd[4];
-                // group G: slots 2q, 2q+1 / 2q+8, 2q+9 of the first MMA carry
-                // elements 8q + {0,1} / {2,3}; of the second 8q + {4,5} / {6,7}
-                mma_f16(dd, fa[0][0], fa[1][0], fa[0][1], fa[1][1], b.x, b.y, zero);
-                mma_f16(dd, fa[0][2], fa[1][2], fa[0][3], fa[1][3], b.z, b.w, dd);
-                acc[m][0] = fmaf(dd[0], sl, acc[m][0]);
-                acc[m][1] = fmaf(dd[1], sl, acc[m][1]);
-                acc[m][2] = fmaf(dd[2], sh, acc[m][2]);
-                acc[m][3] = fmaf(dd[3], sh, acc[m][3]);
+                mma_group_e2m1(acc[m], *reinterpret_cast<const uint32_t *>(cb),
+                               *reinterpret_cast<const uint32_t *>(cb + a_hi), sb[0], sb[sc_hi], b);
             }
         }
         // ---- the 4 K quarters of each row tile, added in order 0, 1, 2, 3 ----

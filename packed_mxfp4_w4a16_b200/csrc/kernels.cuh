@@ -30,6 +30,7 @@ struct RouteParams {
     int *x16_exp;           // [T] its staging exponent c (values are x * 2^-c)
     int T, E, H, k;
     int rmsnorm;
+    int sigmoid;            // sigmoid scoring (bias steers selection only)
     float eps;
 };
 

@@ -142,10 +142,11 @@ layer_kernel(const GateUpParams p, const FusedRouteParams r, const LayerDownPara
     uint4 wv[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
     if (rthread && (int)blockIdx.x < E) {
         const uint4 *row = reinterpret_cast<const uint4 *>(r.wr + (size_t)blockIdx.x * H);
+        const uint64_t pol = l2_evict_last_policy();  // reused by every token
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             const int c = threadIdx.x + kRouteThreads * u;
-            if (c < nch) wv[u] = row[c];
+            if (c < nch) wv[u] = ld_hint16(row + c, pol);
         }
     }
     if (kWhole && threadIdx.x < T * k) s_hmax[threadIdx.x] = 0u;
@@ -250,10 +251,11 @@ layer_kernel(const GateUpParams p, const FusedRouteParams r, const LayerDownPara
         if (rthread) {
             if (e != (int)blockIdx.x) {
                 const uint4 *row = reinterpret_cast<const uint4 *>(r.wr + (size_t)e * H);
+                const uint64_t pol = l2_evict_last_policy();
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
                     const int c = threadIdx.x + kRouteThreads * u;
-                    wv[u] = c < nch ? row[c] : make_uint4(0u, 0u, 0u, 0u);
+                    wv[u] = c < nch ? ld_hint16(row + c, pol) : make_uint4(0u, 0u, 0u, 0u);
                 }
             }
             #pragma unroll 1

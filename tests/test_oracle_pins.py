@@ -266,6 +266,65 @@ def test_route_bias_is_added_to_logits():
     assert np.all(ids2[:, 0] == 17) and np.all(w2[:, 0] > 0.999)
 
 
+def test_sigmoid_route_hand_worked_example():
+    """Logits whose sigmoids are exact small fractions: sigmoid(0) = 1/2,
+    sigmoid(ln 3) = 3/4, sigmoid(ln 1/3) = 1/4, sigmoid(ln 9) = 9/10.
+    Without bias the top-2 are experts 3 (0.9) and 1 (0.75), coefficients
+    0.9/1.65 and 0.75/1.65.  A bias of +0.7 on expert 2 (key 0.95) and -0.5
+    on expert 3 (key 0.4) selects experts 2 and 1 instead, and the
+    coefficients still come from the unbiased scores: 0.25/1.0, 0.75/1.0."""
+    lg = np.array([[0.0, np.log(3.0), np.log(1.0 / 3.0), np.log(9.0)]])
+    ids, w = oracle.select_topk_sigmoid(lg, None, 2)
+    assert ids.tolist() == [[3, 1]]
+    np.testing.assert_allclose(w[0], [0.9 / 1.65, 0.75 / 1.65], rtol=1e-14)
+    bias = np.array([0.0, 0.0, 0.7, -0.5], dtype=np.float32)
+    ids, w = oracle.select_topk_sigmoid(lg, bias, 2)
+    assert ids.tolist() == [[2, 1]]
+    np.testing.assert_allclose(w[0], [0.25, 0.75], rtol=1e-14)
+    # k = E: every expert, coefficients 0.5, 0.75, 0.25, 0.9 over 2.4
+    ids, w = oracle.select_topk_sigmoid(lg, None, 4)
+    assert ids.tolist() == [[3, 1, 0, 2]]
+    np.testing.assert_allclose(w[0], np.array([0.9, 0.75, 0.5, 0.25]) / 2.4, rtol=1e-14)
+
+
+def test_sigmoid_route_without_bias_selects_as_softmax_route():
+    """The sigmoid is increasing: without bias both scorings select the same
+    experts in the same order (their coefficients differ)."""
+    rng = np.random.default_rng(13)
+    lg = rng.standard_normal((50, 64)) * 3.0
+    ids_s, w_s = oracle.select_topk_sigmoid(lg, None, 4)
+    ids_m, _ = oracle.select_topk(lg, 4)
+    np.testing.assert_array_equal(ids_s, ids_m)
+    np.testing.assert_allclose(w_s.sum(axis=1), 1.0, rtol=1e-14)
+    assert np.all(np.diff(w_s, axis=1) <= 0)
+
+
+def test_sigmoid_route_ties_and_logits_unbiased():
+    lg = np.array([[0.5, 2.0, 1.0, 2.0, 1.0, 2.0, -1.0, 0.0]])
+    ids, w = oracle.select_topk_sigmoid(lg, None, 4)
+    assert ids.tolist() == [[1, 3, 5, 2]]
+    assert w[0, 0] == w[0, 1] == w[0, 2]
+    rng = np.random.default_rng(14)
+    E, H, k = 32, 128, 4
+    x = synth.f32_to_bf16_bits(rng.standard_normal((3, H), dtype=np.float32))
+    Wr = synth.f32_to_bf16_bits(rng.standard_normal((E, H), dtype=np.float32) * 0.02)
+    b = rng.standard_normal(E).astype(np.float32)
+    ids, w, lg = oracle.route(x, Wr, b, k, sigmoid=True)
+    _, _, lg0 = oracle.route(x, Wr, None, k)
+    np.testing.assert_array_equal(lg, lg0)  # the bias does not enter the logits
+    ids2, w2 = oracle.select_topk_sigmoid(lg0, b, k)
+    np.testing.assert_array_equal(ids, ids2)
+    np.testing.assert_array_equal(w, w2)
+    # a large bias on one expert forces it into slot 0 whatever its score
+    b2 = np.zeros(E, dtype=np.float32)
+    b2[17] = 10.0
+    ids3, w3, _ = oracle.route(x, Wr, b2, k, sigmoid=True)
+    assert np.all(ids3[:, 0] == 17)
+    s = 1.0 / (1.0 + np.exp(-lg0))
+    np.testing.assert_allclose(w3[:, 0], s[:, 17] / np.take_along_axis(s, ids3, 1).sum(1),
+                               rtol=1e-13)
+
+
 # ----------------------------------------------------------------- combine
 
 def test_combine_hand_derived_examples(golden):
