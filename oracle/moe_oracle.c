@@ -22,6 +22,10 @@
  *         routing inside resident-layer graphs" (router projection, sigmoid
  *         scores, expert bias where configured, dynamic top-k, routing
  *         coefficients).
+ *   [NV]  "primitive-ai/LFM2.5-24B-A2B-NVFP4A16" (model card of an NVFP4
+ *         weight-only build): sections "What's quantized to what" (routed
+ *         experts in NVFP4, compute in 16-bit; format nvfp4-pack-quantized;
+ *         w1 and w3 of each expert share one global scale).
  *   [BW]  "LFM2.5-24B-A2B on Your Own Hardware: The RAM, KV Cache and
  *         Bandwidth Budget": section "Where do the 2.45B active parameters
  *         actually go?" (SwiGLU expert = gate, up, down; H=2048, I=1536).
@@ -46,6 +50,12 @@
  *     y = BF16(y + p_j) for j = 0..k-1 in slot order.
  *   - Stack: xn = BF16(r / sqrt(mean(r^2) + 1e-6)) (weightless RMSNorm
  *     before each layer), r' = BF16(r + y).
+ *   - NVFP4 ([NV] names the format only): E2M1 codes packed as above; one
+ *     FP8 E4M3 scale per 16 consecutive K elements (scales [E][3][rows][K/16]:
+ *     sign, 4 exponent bits with bias 7, 3 mantissa bits, exponent 0
+ *     subnormal, S.1111.111 NaN, no infinity); one FP32 multiplier per
+ *     expert shared by gate and up and one for down (gscales [E][2]);
+ *     w = e2m1(c) * e4m3(s) * g.
  */
 #include <math.h>
 #include <stddef.h>
@@ -117,6 +127,38 @@ static double weight_at(const uint8_t *row_codes, const uint8_t *row_scales,
     uint8_t byte = row_codes[j >> 1];
     unsigned nib = (j & 1) ? (unsigned)(byte >> 4) : (unsigned)(byte & 0x0F);
     return oracle_e2m1_value(nib) * oracle_e8m0_value(row_scales[j >> 5]);
+}
+
+/* [NV] FP8 E4M3 block scale, one per 16 weight values. */
+double oracle_e4m3_value(unsigned b)
+{
+    unsigned sign = (b >> 7) & 1u, ex = (b >> 3) & 15u, man = b & 7u;
+    double m;
+    if (ex == 15u && man == 7u)
+        return NAN;
+    if (ex == 0u)
+        m = ldexp((double)man / 8.0, -6);          /* subnormal */
+    else
+        m = ldexp(1.0 + (double)man / 8.0, (int)ex - 7);
+    return sign ? -m : m;
+}
+
+/* NVFP4 weight element j of a packed row: the E2M1 code times the E4M3
+ * scale of its 16-element block times the tensor's global multiplier. */
+static double weight_at_nv(const uint8_t *row_codes, const uint8_t *row_scales,
+                           double gscale, int64_t j)
+{
+    uint8_t byte = row_codes[j >> 1];
+    unsigned nib = (j & 1) ? (unsigned)(byte >> 4) : (unsigned)(byte & 0x0F);
+    return oracle_e2m1_value(nib) * oracle_e4m3_value(row_scales[j >> 4]) * gscale;
+}
+
+/* NVFP4 dequantisation of n consecutive elements (n a multiple of 16). */
+void oracle_dequant_nvfp4(const uint8_t *codes, const uint8_t *scales,
+                          double gscale, int64_t n, double *out)
+{
+    for (int64_t j = 0; j < n; ++j)
+        out[j] = weight_at_nv(codes, scales, gscale, j);
 }
 
 /* Dequantise n consecutive elements (n a multiple of 32). */
@@ -258,31 +300,41 @@ void oracle_route_sigmoid(const uint16_t *x, int T, int H, const uint16_t *Wr,
 
 static double silu(double g) { return g / (1.0 + exp(-g)); }
 
-/* One SwiGLU expert on one BF16 activation vector.
+/* One SwiGLU expert on one BF16 activation vector, for either weight format.
  * [MC] "Grouped top-4 expert execution": gate projection, up projection,
  * activation and multiplication, down projection; "Model and quantization":
  * accumulation wider than BF16, BF16 outputs.  [BW]: the expert is the three
  * matrices gate, up (I x H) and down (H x I).
- *   codes_e / scales_e: this expert's [3][rows][K/2] / [3][rows][K/32].
+ *   nv = 0 (MXFP4): codes_e / scales_e: this expert's [3][rows][K/2] /
+ *     [3][rows][K/32], gs ignored.
+ *   nv = 1 (NVFP4): scales_e [3][rows][K/16] E4M3, gs[0] multiplies gate and
+ *     up, gs[1] down.
  *   h_out (nullable): the BF16 SwiGLU output [I].  o_out: BF16 [H]. */
-void oracle_expert(const uint16_t *x, const uint8_t *codes_e,
-                   const uint8_t *scales_e, int H, int I, uint16_t *h_out,
-                   uint16_t *o_out)
+static void expert_any(const uint16_t *x, const uint8_t *codes_e,
+                       const uint8_t *scales_e, const float *gs, int nv,
+                       int H, int I, uint16_t *h_out, uint16_t *o_out)
 {
-    const size_t mc = (size_t)I * H / 2, ms = (size_t)I * H / 32;
+    const int sdiv = nv ? 16 : 32;  /* K elements per scale */
+    const size_t mc = (size_t)I * H / 2, ms = (size_t)I * H / (size_t)sdiv;
     const uint8_t *gate_c = codes_e, *up_c = codes_e + mc, *down_c = codes_e + 2 * mc;
     const uint8_t *gate_s = scales_e, *up_s = scales_e + ms, *down_s = scales_e + 2 * ms;
+    const double g_gu = nv ? (double)gs[0] : 1.0, g_dn = nv ? (double)gs[1] : 1.0;
     uint16_t *hb = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)I);
 
 #pragma omp parallel for schedule(static)
     for (int i = 0; i < I; ++i) {
-        const uint8_t *gc = gate_c + (size_t)i * (H / 2), *gs = gate_s + (size_t)i * (H / 32);
-        const uint8_t *uc = up_c + (size_t)i * (H / 2), *us = up_s + (size_t)i * (H / 32);
+        const uint8_t *gc = gate_c + (size_t)i * (H / 2), *gsc = gate_s + (size_t)i * (H / sdiv);
+        const uint8_t *uc = up_c + (size_t)i * (H / 2), *usc = up_s + (size_t)i * (H / sdiv);
         double g = 0.0, u = 0.0;
         for (int j = 0; j < H; ++j) {
             double xv = oracle_bf16_to_double(x[j]);
-            g += weight_at(gc, gs, j) * xv;
-            u += weight_at(uc, us, j) * xv;
+            if (nv) {
+                g += weight_at_nv(gc, gsc, g_gu, j) * xv;
+                u += weight_at_nv(uc, usc, g_gu, j) * xv;
+            } else {
+                g += weight_at(gc, gsc, j) * xv;
+                u += weight_at(uc, usc, j) * xv;
+            }
         }
         double gb = oracle_bf16_to_double(oracle_bf16_from_double(g));
         double ub = oracle_bf16_to_double(oracle_bf16_from_double(u));
@@ -292,15 +344,33 @@ void oracle_expert(const uint16_t *x, const uint8_t *codes_e,
 
 #pragma omp parallel for schedule(static)
     for (int n = 0; n < H; ++n) {
-        const uint8_t *dc = down_c + (size_t)n * (I / 2), *ds = down_s + (size_t)n * (I / 32);
+        const uint8_t *dc = down_c + (size_t)n * (I / 2), *ds = down_s + (size_t)n * (I / sdiv);
         double o = 0.0;
-        for (int j = 0; j < I; ++j)
-            o += weight_at(dc, ds, j) * oracle_bf16_to_double(hb[j]);
+        for (int j = 0; j < I; ++j) {
+            double wv = nv ? weight_at_nv(dc, ds, g_dn, j) : weight_at(dc, ds, j);
+            o += wv * oracle_bf16_to_double(hb[j]);
+        }
         o_out[n] = oracle_bf16_from_double(o);
     }
     if (h_out)
         memcpy(h_out, hb, sizeof(uint16_t) * (size_t)I);
     free(hb);
+}
+
+/* One MXFP4 expert (expert_any with nv = 0). */
+void oracle_expert(const uint16_t *x, const uint8_t *codes_e,
+                   const uint8_t *scales_e, int H, int I, uint16_t *h_out,
+                   uint16_t *o_out)
+{
+    expert_any(x, codes_e, scales_e, NULL, 0, H, I, h_out, o_out);
+}
+
+/* One NVFP4 expert: gs = {gate/up multiplier, down multiplier}. */
+void oracle_expert_nvfp4(const uint16_t *x, const uint8_t *codes_e,
+                         const uint8_t *scales_e, const float *gs, int H, int I,
+                         uint16_t *h_out, uint16_t *o_out)
+{
+    expert_any(x, codes_e, scales_e, gs, 1, H, I, h_out, o_out);
 }
 
 /* ------------------------------------------------------------- combine -- */
@@ -330,18 +400,20 @@ void oracle_combine(const uint16_t *o, const double *w, int k, int H,
 
 /* ---------------------------------------------------------- MoE layer -- */
 
-/* Experts + combine for T tokens with given routing.
+/* Experts + combine for T tokens with given routing, either weight format.
  *   x [T][H], ids [T][k], w [T][k] (double), codes [E][3*I*H/2],
- *   scales [E][3*I*H/32], residual [T][H] or NULL, y [T][H],
- *   o_out (nullable) [T][k][H], h_out (nullable) [T][k][I].
+ *   scales [E][3*I*H/32] (MXFP4) or [E][3*I*H/16] (NVFP4, with gscales
+ *   [E][2]), residual [T][H] or NULL, y [T][H], o_out (nullable)
+ *   [T][k][H], h_out (nullable) [T][k][I].
  * An id outside [0, E) gives a zero expert output for that slot. */
-void oracle_moe_forward(const uint16_t *x, int T, int E, int H, int I, int k,
-                        const int32_t *ids, const double *w,
-                        const uint8_t *codes, const uint8_t *scales,
-                        const uint16_t *residual, uint16_t *y,
-                        uint16_t *o_out, uint16_t *h_out)
+static void moe_forward_any(const uint16_t *x, int T, int E, int H, int I, int k,
+                            const int32_t *ids, const double *w,
+                            const uint8_t *codes, const uint8_t *scales,
+                            const float *gscales, int nv,
+                            const uint16_t *residual, uint16_t *y,
+                            uint16_t *o_out, uint16_t *h_out)
 {
-    const size_t ce = (size_t)3 * I * H / 2, se = (size_t)3 * I * H / 32;
+    const size_t ce = (size_t)3 * I * H / 2, se = (size_t)3 * I * H / (nv ? 16 : 32);
     uint16_t *o = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)k * H);
     for (int t = 0; t < T; ++t) {
         for (int j = 0; j < k; ++j) {
@@ -353,8 +425,9 @@ void oracle_moe_forward(const uint16_t *x, int T, int E, int H, int I, int k,
                     memset(hj, 0, sizeof(uint16_t) * (size_t)I);
                 continue;
             }
-            oracle_expert(x + (size_t)t * H, codes + (size_t)e * ce,
-                          scales + (size_t)e * se, H, I, hj, o + (size_t)j * H);
+            expert_any(x + (size_t)t * H, codes + (size_t)e * ce, scales + (size_t)e * se,
+                       nv ? gscales + (size_t)e * 2 : NULL, nv, H, I, hj,
+                       o + (size_t)j * H);
         }
         if (o_out)
             memcpy(o_out + (size_t)t * k * H, o, sizeof(uint16_t) * (size_t)k * H);
@@ -363,6 +436,26 @@ void oracle_moe_forward(const uint16_t *x, int T, int E, int H, int I, int k,
                        y + (size_t)t * H);
     }
     free(o);
+}
+
+void oracle_moe_forward(const uint16_t *x, int T, int E, int H, int I, int k,
+                        const int32_t *ids, const double *w,
+                        const uint8_t *codes, const uint8_t *scales,
+                        const uint16_t *residual, uint16_t *y,
+                        uint16_t *o_out, uint16_t *h_out)
+{
+    moe_forward_any(x, T, E, H, I, k, ids, w, codes, scales, NULL, 0, residual, y,
+                    o_out, h_out);
+}
+
+void oracle_moe_forward_nvfp4(const uint16_t *x, int T, int E, int H, int I, int k,
+                              const int32_t *ids, const double *w,
+                              const uint8_t *codes, const uint8_t *scales,
+                              const float *gscales, const uint16_t *residual,
+                              uint16_t *y, uint16_t *o_out, uint16_t *h_out)
+{
+    moe_forward_any(x, T, E, H, I, k, ids, w, codes, scales, gscales, 1, residual, y,
+                    o_out, h_out);
 }
 
 /* Full layer: route, experts, combine. */

@@ -37,6 +37,12 @@ def _declare(L):
     L.oracle_e2m1_value.restype = dbl
     L.oracle_e8m0_value.argtypes = [C.c_uint]
     L.oracle_e8m0_value.restype = dbl
+    L.oracle_e4m3_value.argtypes = [C.c_uint]
+    L.oracle_e4m3_value.restype = dbl
+    L.oracle_dequant_nvfp4.argtypes = [vp, vp, dbl, i64, vp]
+    L.oracle_expert_nvfp4.argtypes = [vp, vp, vp, vp, i32, i32, vp, vp]
+    L.oracle_moe_forward_nvfp4.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp, vp,
+                                           vp, vp, vp, vp, vp, vp]
     L.oracle_dequant.argtypes = [vp, vp, i64, vp]
     L.oracle_dequant_f32.argtypes = [vp, vp, i64, vp]
     L.oracle_select_topk.argtypes = [vp, i32, i32, vp, vp]
@@ -55,6 +61,7 @@ def _declare(L):
     for name in ("oracle_dequant", "oracle_dequant_f32", "oracle_select_topk",
                  "oracle_select_topk_sigmoid", "oracle_route", "oracle_route_sigmoid",
                  "oracle_expert", "oracle_combine", "oracle_moe_forward", "oracle_moe_layer",
+                 "oracle_dequant_nvfp4", "oracle_expert_nvfp4", "oracle_moe_forward_nvfp4",
                  "oracle_rmsnorm",
                  "oracle_stack_step"):
         getattr(L, name).restype = None
@@ -98,6 +105,11 @@ def e8m0_value(e: int) -> float:
     return lib().oracle_e8m0_value(int(e))
 
 
+def e4m3_value(b: int) -> float:
+    """FP8 E4M3 byte -> value (NVFP4 block scales)."""
+    return lib().oracle_e4m3_value(int(b))
+
+
 def bf16_from_f64_array(v: np.ndarray) -> np.ndarray:
     f = lib().oracle_bf16_from_double
     flat = np.asarray(v, dtype=np.float64).ravel()
@@ -124,6 +136,15 @@ def dequant_f32(codes: np.ndarray, scales: np.ndarray, n: int) -> np.ndarray:
     assert n % 32 == 0 and codes.size >= n // 2 and scales.size >= n // 32
     out = np.empty(n, dtype=np.float32)
     lib().oracle_dequant_f32(_p(codes), _p(scales), n, _p(out))
+    return out
+
+
+def dequant_nvfp4(codes: np.ndarray, scales: np.ndarray, gscale: float, n: int) -> np.ndarray:
+    """NVFP4: E2M1 codes x E4M3 scale per 16 x global multiplier."""
+    codes, scales = _c(codes, np.uint8), _c(scales, np.uint8)
+    assert n % 16 == 0 and codes.size >= n // 2 and scales.size >= n // 16
+    out = np.empty(n, dtype=np.float64)
+    lib().oracle_dequant_nvfp4(_p(codes), _p(scales), float(gscale), n, _p(out))
     return out
 
 
@@ -182,6 +203,18 @@ def expert(x, codes_e, scales_e, H, I):
     return h, o
 
 
+def expert_nvfp4(x, codes_e, scales_e, gs, H, I):
+    """One NVFP4 expert on one token -> (h bf16 [I], o bf16 [H]); gs =
+    (gate/up multiplier, down multiplier)."""
+    x = _c(x, np.uint16).ravel()
+    codes_e, scales_e = _c(codes_e, np.uint8), _c(scales_e, np.uint8)
+    gs = _c(gs, np.float32).ravel()
+    h = np.empty(I, dtype=np.uint16)
+    o = np.empty(H, dtype=np.uint16)
+    lib().oracle_expert_nvfp4(_p(x), _p(codes_e), _p(scales_e), _p(gs), H, I, _p(h), _p(o))
+    return h, o
+
+
 def combine(o, w, residual=None):
     """o bf16 [k,H], w [k] -> y bf16 [H] (sequential BF16 combine)."""
     o = _c(o, np.uint16)
@@ -191,6 +224,31 @@ def combine(o, w, residual=None):
     y = np.empty(H, dtype=np.uint16)
     lib().oracle_combine(_p(o), _p(w), k, H, _p(r), _p(y))
     return y
+
+
+def moe_forward_nvfp4(x, ids, w, codes, scales, gscales, E, H, I, residual=None,
+                      want_o=False, want_h=False):
+    """moe_forward for NVFP4 experts: scales [E, 3*I*H/16] E4M3 bytes,
+    gscales [E, 2] float32 (gate/up, down)."""
+    x = _c(x, np.uint16)
+    T = x.shape[0]
+    ids = _c(ids, np.int32)
+    k = ids.shape[1]
+    w = _c(w, np.float64)
+    codes, scales = _c(codes, np.uint8), _c(scales, np.uint8)
+    gscales = _c(gscales, np.float32)
+    r = _c(residual, np.uint16) if residual is not None else None
+    y = np.empty((T, H), dtype=np.uint16)
+    o = np.empty((T, k, H), dtype=np.uint16) if want_o else None
+    h = np.empty((T, k, I), dtype=np.uint16) if want_h else None
+    lib().oracle_moe_forward_nvfp4(_p(x), T, E, H, I, k, _p(ids), _p(w), _p(codes),
+                                   _p(scales), _p(gscales), _p(r), _p(y), _p(o), _p(h))
+    out = [y]
+    if want_o:
+        out.append(o)
+    if want_h:
+        out.append(h)
+    return out[0] if len(out) == 1 else tuple(out)
 
 
 def moe_forward(x, ids, w, codes, scales, E, H, I, residual=None,

@@ -438,3 +438,105 @@ def test_closed_forms(golden):
     # the oracle consumes exactly one expert's bytes per selected slot
     codes, scales = synth.make_expert_weights(synth.LayerShape(E=1, H=64, I=32), np.random.default_rng(0))
     assert codes.size == 3 * 64 * 32 // 2 and scales.size == 3 * 64 * 32 // 32
+
+
+# --------------------------------------------------------------- NVFP4
+
+def e4m3_torch(b):
+    """FP8 E4M3 bytes decoded by torch's own float8_e4m3fn dtype."""
+    t = torch.from_numpy(np.asarray(b, dtype=np.uint8).copy()).view(torch.float8_e4m3fn)
+    return t.to(torch.float64).numpy()
+
+
+def unpack_dense_nvfp4(codes_m, scales_m, g, rows, K):
+    """Independent unpacker: packed [rows][K/2] + E4M3 [rows][K/16] (decoded
+    by torch) times the global multiplier g -> f64."""
+    b = np.asarray(codes_m, dtype=np.uint8).reshape(rows, K // 2)
+    nib = np.empty((rows, K), dtype=np.int64)
+    nib[:, 0::2] = b & 0x0F
+    nib[:, 1::2] = b >> 4
+    table = np.array([e2m1_bitfield(c) for c in range(16)])
+    sc = np.repeat(e4m3_torch(scales_m).reshape(rows, K // 16), 16, axis=1)
+    return table[nib] * sc * float(np.float32(g))
+
+
+def test_e4m3_matches_torch_float8_all_bytes():
+    b = np.arange(256, dtype=np.uint8)
+    want = e4m3_torch(b)
+    got = np.array([oracle.e4m3_value(int(v)) for v in b])
+    nan = np.isnan(want)
+    assert nan.sum() == 2 and np.array_equal(np.isnan(got), nan)  # 0x7F, 0xFF
+    np.testing.assert_array_equal(got[~nan], want[~nan])
+    assert np.signbit(got[0x80]) and got[0x80] == 0.0
+    # closed forms: 1.0, the largest finite 448, the smallest subnormal 2^-9
+    assert (got[0x38], got[0x7E], got[0x01]) == (1.0, 448.0, 2.0 ** -9)
+
+
+def test_dequant_nvfp4_block_indexing():
+    """Code 2 (value 1.0) everywhere, a different E4M3 scale per 16-element
+    block: element j is scale[j // 16] times the multiplier."""
+    n = 64
+    codes = np.full(n // 2, 0x22, dtype=np.uint8)
+    scales = np.array([0x38, 0x40, 0x30, 0xB8], dtype=np.uint8)  # 1, 2, 0.5, -1
+    out = oracle.dequant_nvfp4(codes, scales, 0.75, n)
+    np.testing.assert_array_equal(out, np.repeat([0.75, 1.5, 0.375, -0.75], 16))
+
+
+def _rand_expert_nvfp4(H, I, seed):
+    rng = synth.rng_for(seed, 99)
+    shape = synth.LayerShape(E=1, H=H, I=I)
+    codes, scales, gs = synth.make_expert_weights_nvfp4(shape, rng)
+    x = synth.f32_to_bf16_bits(rng.standard_normal(H, dtype=np.float32))
+    return codes[0], scales[0], gs[0], x
+
+
+@pytest.mark.parametrize("H,I,seed", [(64, 32, 0), (128, 96, 1), (512, 384, 2)])
+def test_expert_nvfp4_matches_dense_bruteforce(H, I, seed):
+    codes, scales, gs, x = _rand_expert_nvfp4(H, I, seed)
+    h, o = oracle.expert_nvfp4(x, codes, scales, gs, H, I)
+    mc, ms = I * H // 2, I * H // 16
+    Wg = unpack_dense_nvfp4(codes[:mc], scales[:ms], gs[0], I, H)
+    Wu = unpack_dense_nvfp4(codes[mc:2 * mc], scales[ms:2 * ms], gs[0], I, H)
+    Wd = unpack_dense_nvfp4(codes[2 * mc:], scales[2 * ms:], gs[1], H, I)
+    xf = bf16_f64(x)
+    g = bf16_f64(bf16_via_f32(Wg @ xf))
+    u = bf16_f64(bf16_via_f32(Wu @ xf))
+    s = bf16_f64(bf16_via_f32(g / (1.0 + np.exp(-g))))
+    hb = bf16_via_f32(s * u)
+    ob = bf16_via_f32(Wd @ bf16_f64(hb))
+    dh, do = ulp_diff(h, hb), ulp_diff(o, ob)
+    assert dh.max() <= 1 and (dh > 0).sum() <= max(1, I // 500)
+    assert do.max() <= 1 and (do > 0).sum() <= max(1, H // 500)
+    # the gate/up multiplier is shared, the down one separate: swapping them
+    # changes the answer
+    h2, o2 = oracle.expert_nvfp4(x, codes, scales, gs[::-1].copy(), H, I)
+    assert (ulp_diff(o, o2) > 1).mean() > 0.3
+
+
+def test_expert_nvfp4_down_multiplier_doubling_doubles_output():
+    H, I = 128, 64
+    codes, scales, gs, x = _rand_expert_nvfp4(H, I, 4)
+    _, o = oracle.expert_nvfp4(x, codes, scales, gs, H, I)
+    gs2 = gs.copy()
+    gs2[1] *= 2
+    _, o2 = oracle.expert_nvfp4(x, codes, scales, gs2, H, I)
+    np.testing.assert_array_equal(bf16_f64(o2), 2.0 * bf16_f64(o))
+
+
+def test_nvfp4_reduces_to_mxfp4_when_scales_coincide():
+    """Block scales equal to the power of two of an E8M0 group scale (both
+    16-blocks of the group) and unit multipliers give the MXFP4 layer."""
+    shape = synth.LayerShape(E=4, H=128, I=96)
+    L = synth.make_layer(shape, seed=5)
+    # E8M0 118..124 = 2^-9 .. 2^-3: E4M3 0x01, 0x02, 0x04 (subnormal), then
+    # 0x08, 0x10, 0x18, 0x20
+    e4m3_of = {118: 0x01, 119: 0x02, 120: 0x04, 121: 0x08, 122: 0x10, 123: 0x18, 124: 0x20}
+    nv_scales = np.vectorize(e4m3_of.get)(np.repeat(L.scales, 2, axis=1)).astype(np.uint8)
+    gs = np.ones((shape.E, 2), dtype=np.float32)
+    x = synth.make_tokens(3, shape.H, seed=5)
+    ids = np.array([[0, 1, 2, 3], [3, 1, 0, 2], [2, 2, 1, 0]], dtype=np.int32)
+    w = np.array([[0.4, 0.3, 0.2, 0.1]] * 3)
+    y_mx = oracle.moe_forward(x, ids, w, L.codes, L.scales, shape.E, shape.H, shape.I)
+    y_nv = oracle.moe_forward_nvfp4(x, ids, w, L.codes, nv_scales, gs, shape.E, shape.H,
+                                    shape.I)
+    np.testing.assert_array_equal(y_nv, y_mx)

@@ -128,6 +128,25 @@ def make_expert_weights(shape: LayerShape, rng: np.random.Generator):
     return codes, scales
 
 
+def make_expert_weights_nvfp4(shape: LayerShape, rng: np.random.Generator):
+    """NVFP4 experts of one layer: packed E2M1 codes (uniform bytes), one FP8
+    E4M3 block scale per 16 K elements (positive normal values 2^-6 .. 1.875,
+    uniform over exponent fields 1..7 and the 8 mantissas), and per expert two
+    FP32 multipliers uniform in [0.01, 0.02] (gate/up shared, down).
+
+    Returns (codes uint8 [E, 3*I*H/2], scales uint8 [E, 3*I*H/16],
+    gscales float32 [E, 2]).
+    """
+    n_codes = shape.E * shape.codes_per_expert
+    codes = uniform_bytes(n_codes, rng).reshape(shape.E, shape.codes_per_expert)
+    n_sc = 3 * shape.I * shape.H // 16
+    ex = rng.integers(1, 8, size=(shape.E, n_sc), dtype=np.uint8)
+    man = rng.integers(0, 8, size=(shape.E, n_sc), dtype=np.uint8)
+    scales = ((ex << 3) | man).astype(np.uint8)
+    gscales = rng.uniform(0.01, 0.02, size=(shape.E, 2)).astype(np.float32)
+    return codes, scales, gscales
+
+
 def make_activations(T: int, H: int, rng: np.random.Generator) -> np.ndarray:
     """x ~ N(0, 1) in BF16 bits, [T, H]."""
     return f32_to_bf16_bits(rng.standard_normal((T, H), dtype=np.float32))
@@ -186,6 +205,7 @@ class LayerInputs:
     scales: np.ndarray     # uint8 [E, 3*I*H/32]
     router_w: np.ndarray   # uint16 (bf16) [E, H]
     router_b: np.ndarray | None  # float32 [E] or None
+    gscales: np.ndarray | None = None  # NVFP4: float32 [E, 2]; scales are E4M3 [E, 3*I*H/16]
 
 
 def make_layer(shape: LayerShape, seed: int, layer: int = 0,
@@ -195,6 +215,15 @@ def make_layer(shape: LayerShape, seed: int, layer: int = 0,
     router_w = make_router(shape, rng)
     router_b = make_router_bias(shape, rng) if bias else None
     return LayerInputs(shape, codes, scales, router_w, router_b)
+
+
+def make_layer_nvfp4(shape: LayerShape, seed: int, layer: int = 0,
+                     bias: bool = False) -> LayerInputs:
+    rng = rng_for(seed, 5, layer)
+    codes, scales, gscales = make_expert_weights_nvfp4(shape, rng)
+    router_w = make_router(shape, rng)
+    router_b = make_router_bias(shape, rng) if bias else None
+    return LayerInputs(shape, codes, scales, router_w, router_b, gscales)
 
 
 def make_tokens(T: int, H: int, seed: int, stream: int = 0) -> np.ndarray:
