@@ -149,6 +149,22 @@ MOE_API int moe_load_packed(moe_handle_t h, const uint8_t *codes_u8,
 MOE_API int moe_load_expert_table(moe_handle_t h, const uint8_t *const *codes_ptrs,
                           const uint8_t *const *scales_ptrs);
 
+/* Bind contiguously stored NVFP4 experts (page "primitive-ai/LFM2.5-24B-
+ * A2B-NVFP4A16", section "What's quantized to what": NVFP4 routed experts,
+ * 16-bit compute, w1 and w3 of an expert sharing one global scale).
+ * codes: device uint8 [E][3][I*H/2], E2M1 packed as for MXFP4; scales_e4m3:
+ * device uint8 [E][3][I*H/16], one FP8 E4M3 scale per 16 consecutive K
+ * elements; global_scales: device FP32 [E][2], per expert the multiplier of
+ * gate and up, then that of down.  Weight = e2m1(code) * e4m3(scale) *
+ * multiplier.  codes / scales 16-byte aligned, global_scales 4-byte aligned;
+ * read in place, caller-owned.  Requires H a multiple of 512 up to 4096 (the
+ * bulk-copy gate/up kernel).  NVFP4 layers run the per-(token, slot) path
+ * for every T (no grouped path, no fused launch structures; FORCE_GROUPED
+ * returns ARG).  moe_load_packed / moe_load_expert_table switch the handle
+ * back to MXFP4.  Errors: as moe_load_packed. */
+MOE_API int moe_load_packed_nvfp4(moe_handle_t h, const uint8_t *codes_u8,
+                                  const uint8_t *scales_e4m3, const float *global_scales);
+
 /* Bytes of device workspace needed for up to max_tokens tokens per call.
  * Errors: ARG. */
 MOE_API int moe_workspace_bytes(moe_handle_t h, int max_tokens, size_t *bytes);

@@ -22,7 +22,8 @@ from ._lib import MoEError, check, library_path, load
 
 __all__ = [
     "MoEError", "MoELayer", "MoEStack", "library_path", "load",
-    "moe_create", "moe_destroy", "moe_load_packed", "moe_load_expert_table",
+    "moe_create", "moe_destroy", "moe_load_packed", "moe_load_packed_nvfp4",
+    "moe_load_expert_table",
     "moe_workspace_bytes", "moe_set_workspace", "moe_route", "moe_route_ex",
     "moe_forward", "moe_forward_ex", "moe_layer_ex", "moe_get_intermediates", "moe_get_status",
     "moe_bytes_per_expert", "moe_set_tuning", "moe_device_check", "moe_debug_dequant",
@@ -79,6 +80,17 @@ def moe_load_packed(h: int, codes: torch.Tensor, scales: torch.Tensor) -> None:
     _need(codes, torch.uint8, "moe_load_packed")
     _need(scales, torch.uint8, "moe_load_packed")
     check("moe_load_packed", load().moe_load_packed(C.c_void_p(h), _p(codes), _p(scales)))
+
+
+def moe_load_packed_nvfp4(h: int, codes: torch.Tensor, scales: torch.Tensor,
+                          gscales: torch.Tensor) -> None:
+    """NVFP4 experts: codes uint8 [E, 3*I*H/2], E4M3 scales uint8
+    [E, 3*I*H/16], multipliers float32 [E, 2] (gate/up, down)."""
+    _need(codes, torch.uint8, "moe_load_packed_nvfp4")
+    _need(scales, torch.uint8, "moe_load_packed_nvfp4")
+    _need(gscales, torch.float32, "moe_load_packed_nvfp4")
+    check("moe_load_packed_nvfp4",
+          load().moe_load_packed_nvfp4(C.c_void_p(h), _p(codes), _p(scales), _p(gscales)))
 
 
 def moe_load_expert_table(h: int, codes_ptrs, scales_ptrs) -> None:
@@ -215,19 +227,24 @@ class MoELayer:
 
     codes uint8 [E, 3*I*H/2] and scales uint8 [E, 3*I*H/32] (layout of
     include/moe_mxfp4.h) are read in place; the layer keeps references to
-    them. ``router_w`` BF16 [E, H], ``router_b`` FP32 [E] or None.
+    them. ``router_w`` BF16 [E, H], ``router_b`` FP32 [E] or None.  With
+    ``gscales`` (float32 [E, 2]) the experts are NVFP4: scales are then E4M3
+    bytes [E, 3*I*H/16].
     """
 
     def __init__(self, E, H, I, top_k, codes, scales, router_w=None, router_b=None,
-                 max_tokens=4, workspace=None):
+                 max_tokens=4, workspace=None, gscales=None):
         moe_device_check()
         self.E, self.H, self.I, self.k = E, H, I, top_k
-        self.codes, self.scales = codes, scales
+        self.codes, self.scales, self.gscales = codes, scales, gscales
         self.router_w, self.router_b = router_w, router_b
         self.max_tokens = max_tokens
         self.handle = moe_create(E, H, I, top_k)
         try:
-            moe_load_packed(self.handle, codes, scales)
+            if gscales is None:
+                moe_load_packed(self.handle, codes, scales)
+            else:
+                moe_load_packed_nvfp4(self.handle, codes, scales, gscales)
             need = moe_workspace_bytes(self.handle, max_tokens)
             if workspace is None:
                 workspace = torch.empty(need, dtype=torch.uint8, device=codes.device)

@@ -34,6 +34,8 @@ struct moe_ctx {
     int fusion = 0;                       // moe_layer_ex launch structure (moe_set_fusion)
     const uint8_t *codes_base = nullptr;   // set by moe_load_packed (contiguous layout)
     const uint8_t *scales_base = nullptr;
+    int nv = 0;                           // NVFP4 weights (moe_load_packed_nvfp4)
+    const float *gscale = nullptr;        // NVFP4: [E][2] multipliers (gate/up, down)
 };
 
 namespace {
@@ -197,6 +199,38 @@ int moe_load_packed(moe_handle_t h, const uint8_t *codes_u8, const uint8_t *scal
     if (rc == MOE_OK) {
         h->codes_base = codes_u8;
         h->scales_base = scales_e8m0;
+        h->nv = 0;
+        h->gscale = nullptr;
+    }
+    return rc;
+}
+
+int moe_load_packed_nvfp4(moe_handle_t h, const uint8_t *codes_u8, const uint8_t *scales_e4m3,
+                          const float *global_scales) {
+    if (!h || !codes_u8 || !scales_e4m3 || !global_scales) return MOE_ERR_ARG;
+    // the NVFP4 gate/up rows run on the bulk-copy kernel only
+    if (!moe::gateup_tma_supported(h->H)) return MOE_ERR_ARG;
+    int rc = ensure_device_block(h);
+    if (rc != MOE_OK) return rc;
+    if ((rc = check_device_ptr(h, codes_u8, 16)) != MOE_OK) return rc;
+    if ((rc = check_device_ptr(h, scales_e4m3, 16)) != MOE_OK) return rc;
+    if ((rc = check_device_ptr(h, global_scales, 4)) != MOE_OK) return rc;
+    const size_t mc = (size_t)h->I * h->H / 2, ms = (size_t)h->I * h->H / 16;
+    if (ms % 16) return MOE_ERR_ALIGN;  // every matrix must start 16-byte aligned
+    moe::ExpertPtrs *t = new (std::nothrow) moe::ExpertPtrs[h->E];
+    if (!t) return MOE_ERR_ARG;
+    for (int e = 0; e < h->E; ++e)
+        for (int m = 0; m < 3; ++m) {
+            t[e].codes[m] = codes_u8 + ((size_t)e * 3 + m) * mc;
+            t[e].scales[m] = scales_e4m3 + ((size_t)e * 3 + m) * ms;
+        }
+    rc = upload_table(h, t);
+    delete[] t;
+    if (rc == MOE_OK) {
+        h->codes_base = codes_u8;
+        h->scales_base = scales_e4m3;
+        h->nv = 1;
+        h->gscale = global_scales;
     }
     return rc;
 }
@@ -218,7 +252,11 @@ int moe_load_expert_table(moe_handle_t h, const uint8_t *const *codes_ptrs,
         }
     if (rc == MOE_OK) rc = upload_table(h, t);
     delete[] t;
-    if (rc == MOE_OK) h->codes_base = h->scales_base = nullptr;
+    if (rc == MOE_OK) {
+        h->codes_base = h->scales_base = nullptr;
+        h->nv = 0;
+        h->gscale = nullptr;
+    }
     return rc;
 }
 
@@ -321,7 +359,7 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
     const bool phase = flags & (MOE_FWD_PHASE_GATEUP | MOE_FWD_PHASE_DOWN);
     const bool grouped = !phase && !(flags & MOE_FWD_FORCE_DECODE) &&
                          (T > moe::kDecodeMaxT || (flags & MOE_FWD_FORCE_GROUPED)) &&
-                         moe::grouped_supported(h->E, h->H, h->I);
+                         !h->nv && moe::grouped_supported(h->E, h->H, h->I);
     if ((flags & MOE_FWD_FORCE_GROUPED) && !grouped) return MOE_ERR_ARG;
     if (grouped) {
         for (int t0 = 0; t0 < T; t0 += moe::kGroupedMaxT) {
@@ -376,7 +414,7 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
         g.codes_base = h->codes_base;
         g.scales_base = h->scales_base;
         g.codes_stride = (size_t)h->I * h->H / 2;
-        g.scales_stride = (size_t)h->I * h->H / 32;
+        g.scales_stride = (size_t)h->I * h->H / (h->nv ? 16 : 32);
         g.x = x + (size_t)t0 * h->H;
         g.x16 = nullptr;
         g.x16_exp = nullptr;
@@ -384,7 +422,9 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
         g.logits = nullptr;
         g.ids_out = nullptr;
         g.w_out = nullptr;
-        g.nslots = moe::gateup_tma_slots(h->H);
+        g.nslots = moe::gateup_tma_slots(h->H, h->nv);
+        g.nv = h->nv;
+        g.gscale = h->gscale;
         g.h = hbuf + (size_t)t0 * h->k * h->I;
         g.status = h->d_status;
         g.T = Tc;
@@ -408,7 +448,7 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
         d.codes_base = h->codes_base;
         d.scales_base = h->scales_base;
         d.codes_stride = (size_t)h->I * h->H / 2;
-        d.scales_stride = (size_t)h->I * h->H / 32;
+        d.scales_stride = (size_t)h->I * h->H / (h->nv ? 16 : 32);
         d.h = g.h;
         d.ids = g.ids;
         d.w = topk_w + (size_t)t0 * h->k;
@@ -424,6 +464,8 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
         d.I = h->I;
         const int rows = Tc * h->H;
         d.rows_per_cta = (rows + h->num_sms - 1) / h->num_sms;
+        d.nv = h->nv;
+        d.gscale = h->gscale;
         const int grid = (rows + d.rows_per_cta - 1) / d.rows_per_cta;
         if (run_dn && (rc = cuda_rc(moe::launch_down_decode(d, grid, s, h->use_pdl))) != MOE_OK)
             return rc;
@@ -485,10 +527,11 @@ int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
     const int frows = (T * h->H + G - 1) / G;
     unsigned fdown = 0;
     int lrows = 0;
-    const bool whole = h->fusion >= MOE_FUSION_LAYER && !keep &&
+    // the fused launch structures run MXFP4 weights only
+    const bool whole = !h->nv && h->fusion >= MOE_FUSION_LAYER && !keep &&
                        moe::layer_plan(T, h->E, h->H, h->I, h->k, G, &fsmem, &fslots, &fregion,
                                        &fdown, &lrows);
-    if (whole || (h->fusion >= MOE_FUSION_ROUTER &&
+    if (whole || (!h->nv && h->fusion >= MOE_FUSION_ROUTER &&
                   moe::layer_gateup_plan(T, h->E, h->H, G, &fsmem, &fslots, &fregion) &&
                   moe::down_decode_smem(T, h->k, h->I, frows) <= moe::kDownSmemMax)) {
         // router + gate/up in one launch, then the down kernel on the same grid
@@ -502,7 +545,7 @@ int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
         g.codes_base = h->codes_base;
         g.scales_base = h->scales_base;
         g.codes_stride = (size_t)h->I * h->H / 2;
-        g.scales_stride = (size_t)h->I * h->H / 32;
+        g.scales_stride = (size_t)h->I * h->H / (h->nv ? 16 : 32);
         g.x = norm ? x_norm : x;
         g.x16 = nullptr;
         g.x16_exp = nullptr;
@@ -603,7 +646,7 @@ int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
     g.codes_base = h->codes_base;
     g.scales_base = h->scales_base;
     g.codes_stride = (size_t)h->I * h->H / 2;
-    g.scales_stride = (size_t)h->I * h->H / 32;
+    g.scales_stride = (size_t)h->I * h->H / (h->nv ? 16 : 32);
     g.x = norm ? x_norm : x;
     g.x16 = rp.x16;
     g.x16_exp = rp.x16_exp;
@@ -625,7 +668,9 @@ int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
         g.pf_codes = (uint32_t)(((mc + n - 1) / n + 15) / 16 * 16);
         g.pf_scales = (uint32_t)(((ms + n - 1) / n + 15) / 16 * 16);
     }
-    g.nslots = moe::gateup_tma_slots(h->H);
+    g.nslots = moe::gateup_tma_slots(h->H, h->nv);
+    g.nv = h->nv;
+    g.gscale = h->gscale;
     if ((rc = cuda_rc(moe::launch_gateup_decode(g, h->num_sms, s, h->use_pdl))) != MOE_OK)
         return rc;
 
@@ -634,7 +679,7 @@ int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
     d.codes_base = h->codes_base;
     d.scales_base = h->scales_base;
     d.codes_stride = (size_t)h->I * h->H / 2;
-    d.scales_stride = (size_t)h->I * h->H / 32;
+    d.scales_stride = (size_t)h->I * h->H / (h->nv ? 16 : 32);
     d.h = g.h;
     d.ids = nullptr;
     d.w = nullptr;
@@ -650,6 +695,8 @@ int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
     d.I = h->I;
     const int rows = T * h->H;
     d.rows_per_cta = (rows + h->num_sms - 1) / h->num_sms;
+    d.nv = h->nv;
+    d.gscale = h->gscale;
     const int grid = (rows + d.rows_per_cta - 1) / d.rows_per_cta;
     if ((rc = cuda_rc(moe::launch_down_decode(d, grid, s, h->use_pdl))) != MOE_OK) return rc;
     h->kept = keep;
@@ -680,7 +727,8 @@ int moe_get_status(moe_handle_t h, unsigned *device_status) {
 
 int moe_bytes_per_expert(moe_handle_t h, size_t *bytes) {
     if (!h || !bytes) return MOE_ERR_ARG;
-    *bytes = (size_t)3 * h->I * h->H / 2 + (size_t)3 * h->I * h->H / 32;
+    *bytes = h->nv ? (size_t)3 * h->I * h->H / 2 + (size_t)3 * h->I * h->H / 16 + 2 * sizeof(float)
+                   : (size_t)3 * h->I * h->H / 2 + (size_t)3 * h->I * h->H / 32;
     return MOE_OK;
 }
 

@@ -177,6 +177,38 @@ __device__ __forceinline__ float dot32_e2m1_f16(const uint4 &c, const uint32_t *
     return (a0 + a1) + (a2 + a3);
 }
 
+// NVFP4 ("primitive-ai/LFM2.5-24B-A2B-NVFP4A16", "What's quantized to
+// what"): a 32-element chunk carries two 16-element blocks, each with its own
+// FP8 E4M3 scale.  The two unscaled half sums of the chunk (codes 0..15 in
+// c.x, c.y; 16..31 in c.z, c.w).
+__device__ __forceinline__ void dot32_e2m1_f16_halves(const uint4 &c, const uint32_t *x,
+                                                      float &lo, float &hi) {
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    dot8_e2m1_f16(c.x, x[0], x[1], x[2], x[3], a0, a1);
+    dot8_e2m1_f16(c.y, x[4], x[5], x[6], x[7], a2, a3);
+    lo = (a0 + a1) + (a2 + a3);
+    a0 = a1 = a2 = a3 = 0.f;
+    dot8_e2m1_f16(c.z, x[8], x[9], x[10], x[11], a0, a1);
+    dot8_e2m1_f16(c.w, x[12], x[13], x[14], x[15], a2, a3);
+    hi = (a0 + a1) + (a2 + a3);
+}
+
+// Two FP8 E4M3 scales (the low and high byte of s) as FP32, exactly: the
+// sm_100a conversion instruction to f16x2 (every E4M3 value, subnormals and
+// NaN included, is an FP16 value), then FP16 -> FP32.
+__device__ __forceinline__ void e4m3x2_to_f32(uint32_t s, float &lo, float &hi) {
+    uint32_t h2;
+    asm("{\n\t"
+        ".reg .b16 t;\n\t"
+        "cvt.u16.u32 t, %1;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, t;\n\t"
+        "}"
+        : "=r"(h2)
+        : "r"(s));
+    lo = f16_bits_to_f32(h2 & 0xFFFFu);
+    hi = f16_bits_to_f32(h2 >> 16);
+}
+
 // ------------------------------------------------ FP16 staging of BF16 ----
 // The GEMVs multiply FP16 weights (exact E2M1 values) with activations held
 // in FP16.  A BF16 vector v is staged as v * 2^-c with c chosen from max|v|

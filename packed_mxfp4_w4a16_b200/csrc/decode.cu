@@ -287,7 +287,7 @@ gateup_decode_kernel(const GateUpParams p) {
 // rows, ~90 KB) is requested at once, so the DRAM sees the layer's entire
 // gate/up stream immediately.
 
-template <int KCH>
+template <int KCH, bool NV>
 __global__ void __launch_bounds__(kTmaThreads, 1)
 gateup_tma_kernel(const GateUpParams p) {
     extern __shared__ __align__(128) uint8_t ring[];
@@ -327,7 +327,7 @@ gateup_tma_kernel(const GateUpParams p) {
     // router when available, else staged here.  Plain (L1-allocating) loads:
     // every warp of the CTA reads the same vector, so one L2 read per SM
     // serves all of them.
-    ring_consume<KCH>(p, g, ring, full, empty, s_ids, warp, lane,
+    ring_consume<KCH, NV>(p, g, ring, full, empty, s_ids, warp, lane,
                       [&](int tok, uint32_t (&xw)[KCH][16]) -> float {
         if (p.x16) {
             const uint32_t *xv = p.x16 + (size_t)tok * (H >> 1);
@@ -393,7 +393,7 @@ static __device__ __noinline__ void take_handoff(const RouteHandoff h, int P, in
 // SR: every down row of the CTA is copied into shared memory with bulk copies
 // before the programmatic-launch wait (rows: [k][R] codes, then [k][R] scales);
 // otherwise each team streams its rows from global memory two at a time.
-template <int TL, int KCH, bool SR>
+template <int TL, int KCH, bool SR, bool NV>
 __global__ void __launch_bounds__(kDownThreads, 1)
 down_decode_kernel(const DownParams p) {
     extern __shared__ __align__(16) uint8_t sm[];
@@ -406,11 +406,12 @@ down_decode_kernel(const DownParams p) {
     uint32_t *sh = reinterpret_cast<uint32_t *>(sm);                       // [P][I/2] FP16 words
     float *so = reinterpret_cast<float *>(sm + (size_t)P * I * 2);         // [k][R]
     uint8_t *rows_c = sm + down_rows_offset(T, k, I, R);                   // SR: [k][R][I/2]
-    uint8_t *rows_s = rows_c + (size_t)k * R * ((size_t)I >> 1);           // SR: [k][R][I/32]
+    uint8_t *rows_s = rows_c + (size_t)k * R * ((size_t)I >> 1);           // SR: [k][R][I/32 or /16]
     __shared__ __align__(8) uint64_t s_rbar;
     __shared__ int s_ids[kDecodeMaxT * kMaxTopK];
     __shared__ float s_w[kDecodeMaxT * kMaxTopK];
     __shared__ float s_xs[kDecodeMaxT * kMaxTopK];
+    __shared__ float s_gs[kDecodeMaxT * kMaxTopK];  // NV: each pair's down multiplier
     __shared__ unsigned s_hmax[kDecodeMaxT * kMaxTopK];
 
     // routing for this call's tokens
@@ -432,10 +433,15 @@ down_decode_kernel(const DownParams p) {
     __syncthreads();
 
     const DownSrc src = {p.table, p.codes_base, p.scales_base, p.codes_stride, p.scales_stride};
-    DownRows<TL, KCH, SR> rows(H, I, k, p.E, R, r0, r1, src, s_ids, rows_c, rows_s);
+    if (NV && threadIdx.x < P) {  // read before the barriers inside stage_h_block
+        const int e = s_ids[threadIdx.x];
+        s_gs[threadIdx.x] = (e >= 0 && e < p.E) ? __ldg(p.gscale + 2 * e + 1) : 0.f;
+    }
+    DownRows<TL, KCH, SR, NV> rows(H, I, k, p.E, R, r0, r1, src, s_ids, rows_c, rows_s);
     if (SR) {
         if (threadIdx.x == 0)
-            issue_down_rows(src, p.E, H, I, k, s_ids, r0, r1, R, rows_c, rows_s, &s_rbar);
+            issue_down_rows(src, p.E, H, I, k, s_ids, r0, r1, R, rows_c, rows_s, &s_rbar,
+                            NV ? 1 : 0);
     } else {
         rows.fetch(rows.rr);
     }
@@ -451,7 +457,7 @@ down_decode_kernel(const DownParams p) {
         if (!rows_ok && threadIdx.x == 0) atomicOr(p.status, kTimeoutStatus);
         if (rows_ok) rows.fetch(rows.rr);
     }
-    if (rows_ok) rows.run(sh, s_xs, so, p.status);
+    if (rows_ok) rows.run(sh, s_xs, so, p.status, s_gs);
     __syncthreads();
 
     // sequential BF16 combine in slot order, optional residual add
@@ -490,30 +496,38 @@ cudaError_t launch_gu(const GateUpParams &p, int grid, cudaStream_t s, bool pdl)
     return launch_ex(gateup_decode_kernel<TL, KCH>, dim3(grid), dim3(kGemvThreads), 0, s, pdl, p);
 }
 
-template <int TL, int KCH, bool SR>
+template <int TL, int KCH, bool SR, bool NV>
 cudaError_t launch_dn_v(const DownParams &p, int grid, size_t smem, cudaStream_t s, bool pdl) {
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(down_decode_kernel<TL, KCH, SR>,
+        cudaError_t e = cudaFuncSetAttribute(down_decode_kernel<TL, KCH, SR, NV>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kDownSmemMax);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    return launch_ex(down_decode_kernel<TL, KCH, SR>, dim3(grid), dim3(kDownThreads), smem, s, pdl,
-                     p);
+    return launch_ex(down_decode_kernel<TL, KCH, SR, NV>, dim3(grid), dim3(kDownThreads), smem, s,
+                     pdl, p);
 }
 
 // The shared-memory-rows variant when its copies are 16-byte shaped (I a
 // multiple of 512) and the rows fit; else rows stream from global memory.
-template <int TL, int KCH>
+template <int TL, int KCH, bool NV>
 cudaError_t launch_dn(const DownParams &p, int grid, cudaStream_t s, bool pdl) {
     const size_t smem = down_decode_smem(p.T, p.k, p.I, p.rows_per_cta);
     if (smem > kDownSmemMax) return cudaErrorInvalidValue;
-    const size_t smem_sr = down_rows_smem(p.T, p.k, p.I, p.rows_per_cta);
+    const size_t smem_sr = down_rows_smem(p.T, p.k, p.I, p.rows_per_cta, NV ? 1 : 0);
     if (p.I % 512 == 0 && smem_sr <= kDownSmemMax)
-        return launch_dn_v<TL, KCH, true>(p, grid, smem_sr, s, pdl);
-    return launch_dn_v<TL, KCH, false>(p, grid, smem, s, pdl);
+        return launch_dn_v<TL, KCH, true, NV>(p, grid, smem_sr, s, pdl);
+    return launch_dn_v<TL, KCH, false, NV>(p, grid, smem, s, pdl);
+}
+template <int TL, int KCH>
+cudaError_t launch_dn_mx(const DownParams &p, int grid, cudaStream_t s, bool pdl) {
+    return launch_dn<TL, KCH, false>(p, grid, s, pdl);
+}
+template <int TL, int KCH>
+cudaError_t launch_dn_nv(const DownParams &p, int grid, cudaStream_t s, bool pdl) {
+    return launch_dn<TL, KCH, true>(p, grid, s, pdl);
 }
 
 #define MOE_TEAM_DISPATCH(FN, C, ...)                                   \
@@ -545,25 +559,26 @@ cudaError_t launch_dn(const DownParams &p, int grid, cudaStream_t s, bool pdl) {
 
 bool gateup_tma_supported(int H) { return H % 512 == 0 && H <= 4096; }
 
-int gateup_tma_slots(int H) {
-    const size_t sb = tma_slot_bytes(H);
+int gateup_tma_slots(int H, int nv) {
+    const size_t sb = tma_slot_bytes(H, nv);
     size_t n = kTmaSmemBudget / sb;
     if (n > (size_t)kTmaMaxSlots) n = kTmaMaxSlots;
     return (int)n;
 }
 
-template <int KCH>
+template <int KCH, bool NV>
 cudaError_t launch_gu_tma(const GateUpParams &p, int grid, cudaStream_t s, bool pdl) {
     static bool attr_set = false;
-    const size_t smem = (size_t)p.nslots * tma_slot_bytes(p.H);
+    const size_t smem = (size_t)p.nslots * tma_slot_bytes(p.H, NV ? 1 : 0);
+    if (smem > kTmaSmemBudget) return cudaErrorInvalidValue;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gateup_tma_kernel<KCH>,
+        cudaError_t e = cudaFuncSetAttribute(gateup_tma_kernel<KCH, NV>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kTmaSmemBudget);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    return launch_ex(gateup_tma_kernel<KCH>, dim3(grid), dim3(kTmaThreads), smem, s, pdl, p);
+    return launch_ex(gateup_tma_kernel<KCH, NV>, dim3(grid), dim3(kTmaThreads), smem, s, pdl, p);
 }
 
 bool decode_shape_supported(int H, int I) {
@@ -598,19 +613,28 @@ cudaError_t launch_route(const RouteParams &p, cudaStream_t s, bool pdl) {
 
 cudaError_t launch_gateup_decode(const GateUpParams &p, int grid, cudaStream_t s, bool pdl) {
     if (p.nslots >= 2 && gateup_tma_supported(p.H)) {
-        switch ((p.H / 32 + 31) / 32) {
-        case 1: return launch_gu_tma<1>(p, grid, s, pdl);
-        case 2: return launch_gu_tma<2>(p, grid, s, pdl);
-        case 3: return launch_gu_tma<3>(p, grid, s, pdl);
-        case 4: return launch_gu_tma<4>(p, grid, s, pdl);
+        switch ((p.H / 32 + 31) / 32 + (p.nv ? 4 : 0)) {
+        case 1: return launch_gu_tma<1, false>(p, grid, s, pdl);
+        case 2: return launch_gu_tma<2, false>(p, grid, s, pdl);
+        case 3: return launch_gu_tma<3, false>(p, grid, s, pdl);
+        case 4: return launch_gu_tma<4, false>(p, grid, s, pdl);
+        case 5: return launch_gu_tma<1, true>(p, grid, s, pdl);
+        case 6: return launch_gu_tma<2, true>(p, grid, s, pdl);
+        case 7: return launch_gu_tma<3, true>(p, grid, s, pdl);
+        case 8: return launch_gu_tma<4, true>(p, grid, s, pdl);
         default: return cudaErrorInvalidValue;
         }
     }
+    if (p.nv) return cudaErrorInvalidValue;  // NVFP4 runs on the bulk-copy kernel only
     MOE_TEAM_DISPATCH(launch_gu, p.H / 32, p, grid, s, pdl);
 }
 
 cudaError_t launch_down_decode(const DownParams &p, int grid, cudaStream_t s, bool pdl) {
-    MOE_TEAM_DISPATCH(launch_dn, p.I / 32, p, grid, s, pdl);
+    if (p.nv) {
+        MOE_TEAM_DISPATCH(launch_dn_nv, p.I / 32, p, grid, s, pdl);
+    } else {
+        MOE_TEAM_DISPATCH(launch_dn_mx, p.I / 32, p, grid, s, pdl);
+    }
 }
 
 cudaError_t launch_debug_dequant(const uint8_t *codes, const uint8_t *scales, int64_t n,

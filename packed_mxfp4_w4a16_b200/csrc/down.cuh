@@ -38,9 +38,10 @@ __device__ __forceinline__ int h_piece(int c, int q) { return (c << 2) | (q ^ ((
 __host__ __device__ __forceinline__ size_t down_rows_offset(int T, int k, int I, int R) {
     return ((size_t)T * k * I * 2 + (size_t)k * R * 4 + 15) & ~(size_t)15;
 }
-// Dynamic shared memory of the down phase with rows in shared memory.
-__host__ __device__ __forceinline__ size_t down_rows_smem(int T, int k, int I, int R) {
-    return down_rows_offset(T, k, I, R) + (size_t)k * R * ((size_t)I / 2 + (size_t)I / 32);
+// Dynamic shared memory of the down phase with rows in shared memory (nv:
+// NVFP4 rows, an E4M3 scale per 16 elements).
+__host__ __device__ __forceinline__ size_t down_rows_smem(int T, int k, int I, int R, int nv = 0) {
+    return down_rows_offset(T, k, I, R) + (size_t)k * R * ((size_t)I / 2 + (size_t)I / (nv ? 16 : 32));
 }
 
 // By one thread: the CTA's down rows [r0, r1) of every slot into shared memory
@@ -49,8 +50,8 @@ __host__ __device__ __forceinline__ size_t down_rows_smem(int T, int k, int I, i
 static __device__ __noinline__ void issue_down_rows(const DownSrc src, int E, int H, int I, int k,
                                                     const int *s_ids, int r0, int r1, int R,
                                                     uint8_t *rows_c, uint8_t *rows_s,
-                                                    uint64_t *bar) {
-    const size_t rc = (size_t)I >> 1, rs = (size_t)I >> 5;
+                                                    uint64_t *bar, int nv = 0) {
+    const size_t rc = (size_t)I >> 1, rs = (size_t)I >> (nv ? 4 : 5);
     const uint64_t pol = l2_evict_first_policy();  // the rows are read once
     unsigned bytes = 0;
     #pragma unroll 1
@@ -209,7 +210,7 @@ static __device__ __noinline__ bool stage_h_tagged(const uint2 *h_tag, int P, in
 // reduced.  Rows come from shared memory (SR: copied there by issue_down_rows)
 // or are streamed from global memory.  The expert output BF16(o) of row r and
 // slot j goes to so[j R + (r - r0)].
-template <int TL, int KCH, bool SR>
+template <int TL, int KCH, bool SR, bool NV = false>
 struct DownRows {
     int H, I, k, E, C, R, r0, r1, tps, j, lt, rr;
     unsigned mask;
@@ -231,7 +232,7 @@ struct DownRows {
         const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
         C = I >> 5;
         rc = (size_t)I >> 1;
-        rs = (size_t)I >> 5;
+        rs = (size_t)I >> (NV ? 4 : 5);
         lt = lane & (TL - 1);
         mask = team_mask<TL>(lane);
         const int groups = kDownWarps / k;  // warps per slot
@@ -261,10 +262,10 @@ struct DownRows {
                     const int c = lt + TL * v;
                     if (ok && c < C) {
                         cw[u][v] = *reinterpret_cast<const uint4 *>(dc + (size_t)c * 16);
-                        sc[u][v] = ds[c];
+                        sc[u][v] = NV ? *reinterpret_cast<const uint16_t *>(ds + 2 * c) : ds[c];
                     } else {
                         cw[u][v] = make_uint4(0u, 0u, 0u, 0u);
-                        sc[u][v] = 127u;
+                        sc[u][v] = NV ? 0x3838u : 127u;
                     }
                 }
             } else {
@@ -273,19 +274,21 @@ struct DownRows {
                     dc = dsrc_codes(src, e) + (size_t)n * rc;
                     ds = dsrc_scales(src, e) + (size_t)n * rs;
                 }
-                load_chunks<TL, KCH>(dc, ds, ok, lt, C, cw[u], sc[u]);
+                load_chunks<TL, KCH, NV>(dc, ds, ok, lt, C, cw[u], sc[u]);
             }
         }
     }
 
     // The loop, from the rows fetched by fetch(rr); h staged in sh / s_xs.
+    // NV: s_gs[q] is pair q's down multiplier (folded into the exact
+    // power-of-two staging scale).
     __device__ __forceinline__ void run(const uint32_t *sh, const float *s_xs, float *so,
-                                        unsigned *status) {
+                                        unsigned *status, const float *s_gs = nullptr) {
         #pragma unroll 1
         while (worker && rr < r1) {
             const int t = rr / H;
             const uint32_t *xv = sh + (size_t)(t * k + j) * (I >> 1);
-            const float xs = s_xs[t * k + j];
+            const float xs = NV ? s_xs[t * k + j] * s_gs[t * k + j] : s_xs[t * k + j];
             // both rows of a step belong to token t unless the second crosses
             // into the next token; then it is recomputed in the next step
             const int rb = rr + tps;
@@ -305,8 +308,18 @@ struct DownRows {
                         x[4 * q + 2] = v.z;
                         x[4 * q + 3] = v.w;
                     }
-                    a0 = fmaf(dot32_e2m1_f16(cw[0][u], x), e8m0_to_f32(sc[0][u]), a0);
-                    a1 = fmaf(dot32_e2m1_f16(cw[1][u], x), e8m0_to_f32(sc[1][u]), a1);
+                    if (NV) {
+                        float lo, hi, slo, shi;
+                        dot32_e2m1_f16_halves(cw[0][u], x, lo, hi);
+                        e4m3x2_to_f32(sc[0][u], slo, shi);
+                        a0 = fmaf(hi, shi, fmaf(lo, slo, a0));
+                        dot32_e2m1_f16_halves(cw[1][u], x, lo, hi);
+                        e4m3x2_to_f32(sc[1][u], slo, shi);
+                        a1 = fmaf(hi, shi, fmaf(lo, slo, a1));
+                    } else {
+                        a0 = fmaf(dot32_e2m1_f16(cw[0][u], x), e8m0_to_f32(sc[0][u]), a0);
+                        a1 = fmaf(dot32_e2m1_f16(cw[1][u], x), e8m0_to_f32(sc[1][u]), a1);
+                    }
                 }
             }
             a0 = team_add<TL>(a0, mask);

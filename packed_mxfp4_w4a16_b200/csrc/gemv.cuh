@@ -114,7 +114,9 @@ __device__ __forceinline__ int stage_x(const uint16_t *v, int lt, int C, unsigne
     return c;
 }
 
-template <int TL, int KCH>
+// NV: two E4M3 scale bytes per chunk (else one E8M0 byte); an absent chunk
+// gets codes 0 and a unit scale.
+template <int TL, int KCH, bool NV = false>
 __device__ __forceinline__ void load_chunks(const uint8_t *codes, const uint8_t *scales, bool ok,
                                             int lt, int C, uint4 (&cw)[KCH], uint32_t (&sc)[KCH]) {
 #pragma unroll
@@ -122,12 +124,29 @@ __device__ __forceinline__ void load_chunks(const uint8_t *codes, const uint8_t 
         const int c = lt + TL * u;
         if (ok && c < C) {
             cw[u] = ld_stream16(codes + (size_t)c * 16);
-            sc[u] = ld_stream_u8(scales + c);
+            sc[u] = NV ? (ld_stream_u8(scales + 2 * c) | (ld_stream_u8(scales + 2 * c + 1) << 8))
+                       : ld_stream_u8(scales + c);
         } else {
             cw[u] = make_uint4(0u, 0u, 0u, 0u);
-            sc[u] = 127u;
+            sc[u] = NV ? 0x3838u : 127u;
         }
     }
+}
+
+// NVFP4: each chunk's two 16-element half sums times their E4M3 scales.
+template <int KCH>
+__device__ __forceinline__ float chunks_dot_nv(const uint4 (&cw)[KCH], const uint32_t (&sc)[KCH],
+                                               const uint32_t (&xw)[KCH][16]) {
+    float acc = 0.f;
+#pragma unroll
+    for (int u = 0; u < KCH; ++u) {
+        float lo, hi, slo, shi;
+        dot32_e2m1_f16_halves(cw[u], xw[u], lo, hi);
+        e4m3x2_to_f32(sc[u], slo, shi);
+        acc = fmaf(lo, slo, acc);
+        acc = fmaf(hi, shi, acc);
+    }
+    return acc;
 }
 
 template <int KCH>
@@ -190,8 +209,9 @@ constexpr int kTmaSlotRows = kTmaConsumers;
 constexpr int kTmaMaxSlots = 16;
 constexpr size_t kTmaSmemBudget = 200 * 1024;
 
-__host__ __device__ __forceinline__ size_t tma_slot_bytes(int H) {
-    return (size_t)kTmaSlotRows * 2 * ((size_t)H / 2 + (size_t)H / 32);
+// nv: NVFP4 rows (an E4M3 scale per 16 elements instead of an E8M0 per 32).
+__host__ __device__ __forceinline__ size_t tma_slot_bytes(int H, int nv = 0) {
+    return (size_t)kTmaSlotRows * 2 * ((size_t)H / 2 + (size_t)H / (nv ? 16 : 32));
 }
 
 // ------------------------------------------------- gate / up ring phases --
@@ -229,8 +249,8 @@ __device__ __forceinline__ RingGeom ring_geom(const GateUpParams &p) {
     g.nsteps = (g.ce - g.cb + kTmaSlotRows - 1) / kTmaSlotRows;
     g.nbar = min(g.nslots, g.nsteps);
     g.rc = (size_t)p.H >> 1;
-    g.rs = (size_t)p.H >> 5;
-    g.slot_bytes = tma_slot_bytes(p.H);
+    g.rs = (size_t)p.H >> (p.nv ? 4 : 5);
+    g.slot_bytes = tma_slot_bytes(p.H, p.nv);
     g.up_off = (size_t)kTmaSlotRows * g.rc;
     g.gs_off = 2 * g.up_off;
     g.us_off = g.gs_off + (size_t)kTmaSlotRows * g.rs;
@@ -374,7 +394,7 @@ __device__ __forceinline__ void ring_produce(const GateUpParams &p, const RingGe
 // Consumer warps: one row per slot each.  get_x(tok, xw) fills the warp's
 // FP16-staged activations of token tok and returns their scale 2^c;
 // emit_h(index, bf16) stores h[q][i] (index q I + i).
-template <int KCH, class GetX, class EmitH>
+template <int KCH, bool NV = false, class GetX, class EmitH>
 __device__ __forceinline__ void ring_consume(const GateUpParams &p, const RingGeom &g,
                                              const uint8_t *ring, uint64_t *full,
                                              uint64_t *empty, const int *s_ids, int warp,
@@ -417,22 +437,30 @@ __device__ __forceinline__ void ring_consume(const GateUpParams &p, const RingGe
                         cg[u] = *reinterpret_cast<const uint4 *>(base + (size_t)warp * rc + (size_t)c * 16);
                         cu[u] = *reinterpret_cast<const uint4 *>(base + up_off + (size_t)warp * rc +
                                                                 (size_t)c * 16);
-                        sg[u] = base[gs_off + (size_t)warp * rs + c];
-                        su[u] = base[us_off + (size_t)warp * rs + c];
+                        if (NV) {
+                            sg[u] = *reinterpret_cast<const uint16_t *>(base + gs_off + (size_t)warp * rs + 2 * c);
+                            su[u] = *reinterpret_cast<const uint16_t *>(base + us_off + (size_t)warp * rs + 2 * c);
+                        } else {
+                            sg[u] = base[gs_off + (size_t)warp * rs + c];
+                            su[u] = base[us_off + (size_t)warp * rs + c];
+                        }
                     } else {
                         cg[u] = cu[u] = make_uint4(0u, 0u, 0u, 0u);
-                        sg[u] = su[u] = 127u;
+                        sg[u] = su[u] = NV ? 0x3838u : 127u;
                     }
                 }
-                float ag = chunks_dot<KCH>(cg, sg, xw);
-                float au = chunks_dot<KCH>(cu, su, xw);
+                float ag = NV ? chunks_dot_nv<KCH>(cg, sg, xw) : chunks_dot<KCH>(cg, sg, xw);
+                float au = NV ? chunks_dot_nv<KCH>(cu, su, xw) : chunks_dot<KCH>(cu, su, xw);
                 ag = warp_sum(ag);
                 au = warp_sum(au);
                 if (lane == 0) {
                     uint16_t out = 0;
                     if (!bad) {
-                        const float g = round_bf16(ag * xs);
-                        const float uu = round_bf16(au * xs);
+                        // NVFP4: the expert's gate/up multiplier, folded into
+                        // the exact power-of-two staging scale
+                        const float sx = NV ? xs * __ldg(p.gscale + 2 * e) : xs;
+                        const float g = round_bf16(ag * sx);
+                        const float uu = round_bf16(au * sx);
                         const float sl = round_bf16(g / (1.0f + expf(-g)));
                         out = f32_to_bf16(sl * uu);
                     } else {

@@ -53,6 +53,8 @@ struct GateUpParams {
     int prefetch_down;        // L2-prefetch the selected down matrices
     uint32_t pf_codes, pf_scales;  // per-CTA prefetch slice (bytes, multiple of 16)
     int nslots;               // shared-memory ring slots of the bulk-copy kernel
+    int nv;                   // NVFP4 weights: E4M3 scale per 16 (else E8M0 per 32)
+    const float *gscale;      // NVFP4: [E][2] FP32 multipliers (gate/up, down)
 };
 
 // Routing handed from the fused router + gate/up kernel to the down kernel of
@@ -110,6 +112,8 @@ struct DownParams {
     int T, k, E, H, I;
     int rows_per_cta;
     RouteHandoff hand;         // used when ids and logits are both null
+    int nv;                    // NVFP4 weights (see GateUpParams)
+    const float *gscale;       // NVFP4: [E][2] FP32 multipliers
 };
 
 // The (token, expert)-sorted grouped path (grouped.cu), for batches of tokens.
@@ -145,7 +149,7 @@ cudaError_t launch_route(const RouteParams &p, cudaStream_t s, bool pdl);
 cudaError_t launch_route_logits(const RouteParams &p, cudaStream_t s, bool pdl);
 cudaError_t launch_topk(const RouteParams &p, cudaStream_t s, bool pdl);
 bool gateup_tma_supported(int H);
-int gateup_tma_slots(int H);
+int gateup_tma_slots(int H, int nv = 0);
 cudaError_t launch_gateup_decode(const GateUpParams &p, int grid, cudaStream_t s, bool pdl);
 cudaError_t launch_down_decode(const DownParams &p, int grid, cudaStream_t s, bool pdl);
 // Fused router + gate/up (layer.cu): one CTA per SM, grid = SM count.  layer_gateup_plan returns the dynamic shared memory and

@@ -1,0 +1,137 @@
+"""NVFP4 experts (E2M1 codes, an FP8 E4M3 scale per 16 elements, an FP32
+multiplier per expert for gate/up and one for down) on the per-(token, slot)
+path against the oracle: SwiGLU vectors h, expert outputs o and combined y
+at the tolerance of the MXFP4 decode path; the combine bit-exact given the
+kernel's own o; every T (the path chunks beyond 4 tokens); invalid ids; the
+whole layer; argument errors."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import packed_mxfp4_w4a16_b200 as moe
+from gpu_util import assert_close_rms, dev_bf16, dev_u8, host_bf16
+from workloads import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _layer(shape, seed, max_tokens=4, bias=False):
+    L = synth.make_layer_nvfp4(shape, seed=seed, bias=bias)
+    rb = None if L.router_b is None else torch.from_numpy(L.router_b).cuda()
+    layer = moe.MoELayer(shape.E, shape.H, shape.I, shape.top_k, dev_u8(L.codes),
+                         dev_u8(L.scales), dev_bf16(L.router_w), rb, max_tokens=max_tokens,
+                         gscales=torch.from_numpy(L.gscales).cuda())
+    return L, layer
+
+
+def _check(L, layer, x, ids, w, shape, residual=None):
+    T = x.shape[0]
+    y = layer.forward(dev_bf16(x), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(),
+                      flags=moe.FWD_KEEP_INTERMEDIATES,
+                      residual=None if residual is None else dev_bf16(residual))
+    torch.cuda.synchronize()
+    h_g, o_g = layer.intermediates(T)
+    h_g, o_g, y_g = host_bf16(h_g), host_bf16(o_g), host_bf16(y)
+    w64 = w.astype(np.float64)
+    y_r, o_r, h_r = oracle.moe_forward_nvfp4(x, ids, w64, L.codes, L.scales, L.gscales, shape.E,
+                                             shape.H, shape.I, residual=residual, want_o=True,
+                                             want_h=True)
+    valid = (ids >= 0) & (ids < shape.E)
+    assert_close_rms(h_g[valid], h_r[valid], what="nvfp4 h")
+    assert_close_rms(o_g[valid], o_r[valid], what="nvfp4 o")
+    assert_close_rms(y_g, y_r, what="nvfp4 y", max_ulps=2)
+    for t in range(T):
+        o_t = np.where(valid[t][:, None], o_g[t], 0).astype(np.uint16)
+        want = oracle.combine(o_t, w64[t], None if residual is None else residual[t])
+        np.testing.assert_array_equal(y_g[t], want)
+    return y_g
+
+
+@pytest.mark.parametrize("shape,T", [(synth.TINY, 1), (synth.TINY, 4), (synth.L24B, 1),
+                                     (synth.L24B, 3), (synth.L8B, 4)])
+def test_nvfp4_forward_matches_oracle(shape, T):
+    L, layer = _layer(shape, 41)
+    x = synth.make_tokens(T, shape.H, seed=41, stream=T)
+    ids, w = synth.make_routing(T, shape.E, shape.top_k, "uniform", synth.rng_for(41, 13, T))
+    r = synth.make_tokens(T, shape.H, seed=42, stream=T) if T > 1 else None
+    _check(L, layer, x, ids, w, shape, residual=r)
+    assert layer.status() == 0
+    layer.close()
+
+
+def test_nvfp4_many_tokens_run_in_decode_chunks():
+    """Beyond 4 tokens NVFP4 stays on the per-(token, slot) path, in chunks."""
+    shape = synth.TINY
+    T = 11
+    L, layer = _layer(shape, 43, max_tokens=T)
+    x = synth.make_tokens(T, shape.H, seed=43)
+    ids, w = synth.make_routing(T, shape.E, shape.top_k, "zipf", synth.rng_for(43, 13, T))
+    _check(L, layer, x, ids, w, shape)
+    with pytest.raises(moe.MoEError):
+        layer.forward(dev_bf16(x), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(),
+                      flags=moe.FWD_FORCE_GROUPED)
+    layer.close()
+
+
+def test_nvfp4_invalid_ids_zero_the_slot_and_flag():
+    shape = synth.TINY
+    L, layer = _layer(shape, 44)
+    x = synth.make_tokens(3, shape.H, seed=44)
+    ids, w = synth.make_routing(3, shape.E, shape.top_k, "uniform", synth.rng_for(44, 13, 3))
+    ids[1, 2] = 77
+    ids[2, 0] = -5
+    _check(L, layer, x, ids, w, shape)
+    assert layer.status() & moe.DEVICE_BAD_EXPERT_ID
+    layer.close()
+
+
+def test_nvfp4_layer_is_route_then_forward():
+    """moe_layer_ex on NVFP4 experts (every fusion setting runs the separate
+    launches) gives the bits of moe_route_ex + moe_forward_ex."""
+    shape = synth.L24B
+    L, layer = _layer(shape, 45, bias=True)
+    T = 2
+    xr = dev_bf16(synth.make_tokens(T, shape.H, seed=45))
+    res = dev_bf16(synth.make_tokens(T, shape.H, seed=46))
+    outs = []
+    for mode in ("layer", moe.FUSION_NONE, moe.FUSION_ROUTER, moe.FUSION_LAYER):
+        xn = torch.zeros(T, shape.H, dtype=torch.bfloat16, device="cuda")
+        ids = torch.zeros(T, shape.top_k, dtype=torch.int32, device="cuda")
+        w = torch.zeros(T, shape.top_k, dtype=torch.float32, device="cuda")
+        y = torch.zeros(T, shape.H, dtype=torch.bfloat16, device="cuda")
+        if mode == "layer":
+            moe.moe_route_ex(layer.handle, xr, layer.router_w, layer.router_b,
+                             moe.ROUTE_RMSNORM, xn, None, ids, w)
+            moe.moe_forward_ex(layer.handle, xn, ids, w, res, y, 0)
+        else:
+            moe.moe_set_fusion(layer.handle, mode)
+            moe.moe_layer_ex(layer.handle, xr, layer.router_w, layer.router_b,
+                             moe.ROUTE_RMSNORM, xn, None, ids, w, res, y, 0)
+        torch.cuda.synchronize()
+        assert layer.status() == 0
+        outs.append([host_bf16(xn).copy(), ids.cpu().numpy(), w.cpu().numpy(),
+                     host_bf16(y).copy()])
+    for o in outs[1:]:
+        for a, b in zip(outs[0], o):
+            np.testing.assert_array_equal(a, b)
+    xn_h, ids_h, w_h, y_h = outs[0]
+    y_r = oracle.moe_forward_nvfp4(xn_h, ids_h, w_h.astype(np.float64), L.codes, L.scales,
+                                   L.gscales, shape.E, shape.H, shape.I,
+                                   residual=host_bf16(res))
+    assert_close_rms(y_h, y_r, what="nvfp4 layer y", max_ulps=2)
+    layer.close()
+
+
+def test_nvfp4_argument_errors():
+    """H must suit the bulk-copy gate/up kernel (a multiple of 512); the
+    multipliers are required."""
+    shape = synth.LayerShape(E=4, H=256, I=128, top_k=2)
+    L = synth.make_layer_nvfp4(shape, seed=47)
+    h = moe.moe_create(shape.E, shape.H, shape.I, shape.top_k)
+    try:
+        with pytest.raises(moe.MoEError):
+            moe.moe_load_packed_nvfp4(h, dev_u8(L.codes), dev_u8(L.scales),
+                                      torch.from_numpy(L.gscales).cuda())
+    finally:
+        moe.moe_destroy(h)
