@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--no-pdl", action="store_true")
     ap.add_argument("--no-prefetch", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-nvfp4", action="store_true",
+                    help="skip the decode measurement of the stack with NVFP4 experts")
     ap.add_argument("--skip-batched", action="store_true",
                     help="skip the grouped-path measurements at batch sizes beyond decode")
     ap.add_argument("--layers", type=int, default=N_LAYERS,
@@ -276,6 +278,54 @@ def build_stack(torch, moe, seed, n_layers):
     return moe.MoEStack(weights, SHAPE.E, SHAPE.H, SHAPE.I, SHAPE.top_k, T=1)
 
 
+def nvfp4_stack(torch, moe, st, args, max_steps=8):
+    """The same 38-layer decode with NVFP4 experts: each layer reuses the
+    MXFP4 layer's codes and router, with E4M3 block scales (a scale per 16,
+    positive normal values, exponent fields 1..7) and FP32 multipliers in
+    [0.01, 0.02] drawn on the device from a seeded generator.  Timed like
+    the main line (graph replays of 64 tokens per step, CUDA events)."""
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(args.seed + 7)
+    n_sc = 3 * SHAPE.I * SHAPE.H // 16
+    weights = []
+    for L in st.layers:
+        ex = torch.randint(1, 8, (SHAPE.E, n_sc), dtype=torch.uint8, device="cuda", generator=gen)
+        man = torch.randint(0, 8, (SHAPE.E, n_sc), dtype=torch.uint8, device="cuda", generator=gen)
+        sc = (ex << 3) | man
+        gs = torch.rand((SHAPE.E, 2), device="cuda", generator=gen) * 0.01 + 0.01
+        weights.append((L.codes, sc, L.router_w, L.router_b, gs))
+    nv = moe.MoEStack(weights, SHAPE.E, SHAPE.H, SHAPE.I, SHAPE.top_k, T=1)
+    nv.set_tuning(use_pdl=not args.no_pdl, prefetch_down=not args.no_prefetch)
+    nv.r.copy_(st.r)
+    nv.capture()
+    steps = max(1, min(max_steps, args.steps))
+    for _ in range(2 * TOKENS_PER_STEP):
+        nv.graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stream = torch.cuda.current_stream()
+    e0.record(stream)
+    for _ in range(steps * TOKENS_PER_STEP):
+        nv.graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_ms = e0.elapsed_time(e1)
+    for L in nv.layers:
+        assert L.status() == 0
+    ids = nv.ids.cpu().numpy()
+    per_expert = 3 * SHAPE.I * SHAPE.H // 2 + 3 * SHAPE.I * SHAPE.H // 16 + 8
+    tok_bytes = sum(len(set(ids[l].ravel().tolist())) * per_expert + SHAPE.E * SHAPE.H * 2
+                    + 2 * SHAPE.H * 2 for l in range(len(nv.layers)))
+    n_tok = steps * TOKENS_PER_STEP
+    out = {"workload": f"stack24b with NVFP4 experts ({len(nv.layers)} layers, E4M3 scale per "
+                       "16, FP32 multipliers), batch-1 decode",
+           "tokens_per_s": n_tok / (t_ms / 1e3), "us_per_token": t_ms * 1e3 / n_tok,
+           "bytes_per_token": tok_bytes, "hbm_gbs": tok_bytes * n_tok / (t_ms / 1e3) / 1e9,
+           "steps": steps}
+    nv.close()
+    return out
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -344,6 +394,9 @@ def run_ours(args):
     # ---- the grouped path at batch sizes beyond decode (one layer) ----
     batched = batched_cases(torch, moe, st, args.seed) if not args.skip_batched else None
 
+    # ---- the same stack with NVFP4 experts ----
+    nvfp4 = nvfp4_stack(torch, moe, st, args) if not args.skip_nvfp4 else None
+
     out = {
         "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
@@ -367,6 +420,7 @@ def run_ours(args):
         "kernels": kern,
         "e2e": e2e,
         "batched": batched,
+        "nvfp4": nvfp4,
         "gpu_launches": 3 * n_layers * TOKENS_PER_STEP * args.steps,
         "clocks": clk.summary(),
     }

@@ -306,16 +306,20 @@ class MoEStack:
     """A stack of MoE layers run as one decode step on a residual stream r:
     per layer xn = RMSNorm(r) (weightless, eps 1e-6), route(xn), experts,
     r = BF16(r + combine).  ``step()`` replays one CUDA graph of all layers.
-    Layers share one workspace (they run in order on one stream)."""
+    Layers share one workspace (they run in order on one stream).
+    ``layers_weights``: per layer (codes, scales, router_w, router_b), or
+    with a fifth item, the NVFP4 multipliers [E, 2] (see MoELayer)."""
 
     def __init__(self, layers_weights, E, H, I, top_k, T=1, device="cuda"):
         moe_device_check()
         self.E, self.H, self.I, self.k, self.T = E, H, I, top_k, T
         self.layers = []
         ws = None
-        for (codes, scales, router_w, router_b) in layers_weights:
+        for lw in layers_weights:
+            codes, scales, router_w, router_b = lw[:4]
+            gscales = lw[4] if len(lw) > 4 else None
             L = MoELayer(E, H, I, top_k, codes, scales, router_w, router_b, max_tokens=T,
-                         workspace=ws)
+                         workspace=ws, gscales=gscales)
             ws = L.workspace
             self.layers.append(L)
         dev = torch.device(device)

@@ -60,7 +60,9 @@ def _check(L, layer, x, ids, w, shape, flags=0, residual=None):
 @pytest.mark.parametrize("shape,T,dist", [
     (synth.L24B, 5, "uniform"), (synth.L24B, 32, "uniform"), (synth.L24B, 32, "zipf"),
     (synth.L24B, 64, "zipf"), (synth.L8B, 17, "zipf"), (synth.TINY, 8, "uniform"),
-    (synth.TINY, 33, "zipf")])
+    (synth.TINY, 33, "zipf"),
+    # groups of 12 tokens on average: two 8-token chunks per CTA
+    (synth.L24B, 200, "uniform"), (synth.TINY, 60, "uniform")])
 def test_grouped_matches_oracle(shape, T, dist):
     L, layer, x, ids, w = _setup(shape, 71, T, dist)
     _check(L, layer, x, ids, w, shape)
