@@ -118,6 +118,11 @@ typedef enum moe_status {
                                       MOE_FWD_PHASE_GATEUP call (same T,
                                       ids, same handle and workspace); the
                                       two calls together equal one forward  */
+#define MOE_FWD_FORCE_TCGEN05 0x20u /* grouped path with its products on
+                                      tcgen05 (TMEM accumulators, TMA tensor
+                                      loads of the packed codes); needs the
+                                      contiguous weights of moe_load_packed
+                                      and H, I multiples of 128, else ARG  */
 
 /* Create a layer of E experts with hidden size H, intermediate size I and
  * top_k experts per token.  Requires H % 32 == 0, I % 32 == 0,
@@ -208,7 +213,10 @@ MOE_API int moe_route_ex(moe_handle_t h, const uint16_t *x, int T,
  * [T][k]; y: device BF16 [T][H] (must not alias x).  An id outside [0, E)
  * makes that slot contribute 0 and sets MOE_DEVICE_BAD_EXPERT_ID in the
  * device status word.  T = 1..4 runs the per-(token, slot) GEMV path;
- * larger T the (token, expert)-sorted grouped path.  Errors: ARG,
+ * larger T the (token, expert)-sorted grouped path, in chunks of up to 2048
+ * tokens: its products run on mma.sync tiles, or with MOE_FWD_FORCE_TCGEN05
+ * on tcgen05 (BF16 weight tiles dequantised once per CTA, FP32 accumulators
+ * in tensor memory, packed codes brought in by TMA tensor loads).  Errors: ARG,
  * NOT_LOADED, NOT_DEVICE, ALIGN, WORKSPACE, CUDA. */
 MOE_API int moe_forward(moe_handle_t h, const uint16_t *x, int T,
                 const int32_t *topk_ids, const float *topk_w, uint16_t *y,

@@ -331,8 +331,14 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
                    void *stream) {
     if (!h || T < 1) return MOE_ERR_ARG;
     const unsigned known = MOE_FWD_KEEP_INTERMEDIATES | MOE_FWD_FORCE_DECODE |
-                           MOE_FWD_FORCE_GROUPED | MOE_FWD_PHASE_GATEUP | MOE_FWD_PHASE_DOWN;
+                           MOE_FWD_FORCE_GROUPED | MOE_FWD_PHASE_GATEUP | MOE_FWD_PHASE_DOWN |
+                           MOE_FWD_FORCE_TCGEN05;
     if (flags & ~known) return MOE_ERR_ARG;
+    if (flags & MOE_FWD_FORCE_TCGEN05) {
+        if (flags & MOE_FWD_FORCE_DECODE) return MOE_ERR_ARG;
+        if (h->nv || !h->codes_base || !moe::grouped_tc_supported(h->H, h->I)) return MOE_ERR_ARG;
+        flags |= MOE_FWD_FORCE_GROUPED;
+    }
     if ((flags & MOE_FWD_FORCE_DECODE) && (flags & MOE_FWD_FORCE_GROUPED)) return MOE_ERR_ARG;
     if ((flags & MOE_FWD_PHASE_GATEUP) && (flags & MOE_FWD_PHASE_DOWN)) return MOE_ERR_ARG;
     const bool run_gu = !(flags & MOE_FWD_PHASE_DOWN);
@@ -390,6 +396,7 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
             gp.E = h->E;
             gp.H = h->H;
             gp.I = h->I;
+            gp.tcgen05 = (flags & MOE_FWD_FORCE_TCGEN05) ? 1 : 0;
             if ((rc = cuda_rc(moe::launch_grouped(gp, s, h->use_pdl))) != MOE_OK) return rc;
         }
         h->kept = keep;

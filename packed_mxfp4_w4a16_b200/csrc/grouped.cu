@@ -438,12 +438,21 @@ cudaError_t launch_grouped(const GroupedParams &p, cudaStream_t s, bool pdl) {
     if ((e = launch_ex(grouped_prep_kernel, dim3(p.T + 1), dim3(kGpThreads), 0, s, pdl, p)) !=
         cudaSuccess)
         return e;
-    if ((e = launch_mma<2>(p, s, pdl)) != cudaSuccess) return e;
-    if ((e = launch_ex(grouped_stage_h_kernel, dim3(p.T * p.k), dim3(kGpThreads), 0, s, pdl, p)) !=
-        cudaSuccess)
-        return e;
-    if ((e = launch_mma<1>(p, s, pdl)) != cudaSuccess) return e;
+    if (p.tcgen05) {
+        // the products on tcgen05 (BF16 tiles, TMEM accumulators; they read
+        // x and h in BF16, so h needs no FP16 staging)
+        if (!p.codes_base || !grouped_tc_supported(p.H, p.I)) return cudaErrorInvalidValue;
+        if ((e = launch_grouped_tc_gateup(p, s, pdl)) != cudaSuccess) return e;
+        if ((e = launch_grouped_tc_down(p, s, pdl)) != cudaSuccess) return e;
+    } else {
+        if ((e = launch_mma<2>(p, s, pdl)) != cudaSuccess) return e;
+        if ((e = launch_ex(grouped_stage_h_kernel, dim3(p.T * p.k), dim3(kGpThreads), 0, s, pdl,
+                           p)) != cudaSuccess)
+            return e;
+        if ((e = launch_mma<1>(p, s, pdl)) != cudaSuccess) return e;
+    }
     return launch_ex(grouped_combine_kernel, dim3(p.T), dim3(kGpThreads), 0, s, pdl, p);
 }
+
 
 }  // namespace moe

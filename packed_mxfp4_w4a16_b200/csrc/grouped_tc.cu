@@ -1,0 +1,489 @@
+// grouped_tc.cu — the grouped expert products on the 5th-generation tensor
+// cores (tcgen05.mma with TMEM accumulators), for batches whose experts see
+// many tokens each (large prefill chunks).
+//
+// Sources: model card "LFM2.5-24B-A2B — Packed MXFP4 Inference", "Grouped
+// top-4 expert execution" (grouped gate / up / down products, activation and
+// multiplication) and table "Model and quantization" (E2M1 + E8M0 per 32,
+// BF16 activations, FP32 accumulation); page "LFM2.5-8B-A1B — Core AI
+// (.aimodel)", section "Provenance" (the batched path sorts the (token,
+// expert) pairs so that each expert's tokens form one group).
+//
+// One CTA per (128 rows of a matrix, expert), 16 warps.  The CTA walks K in
+// tiles of 64.  The packed codes of each tile (128 rows x 32 bytes per
+// matrix) arrive by one TMA tensor load into a ring of shared-memory slots,
+// several tiles ahead (mbarrier completion); per tile, the threads (four per
+// row, a quarter of the tile's K each) dequantise the 128 x 64 packed weights
+// of each matrix into BF16 (value = E2M1 code x 2^(e-127), exact in BF16: the
+// E8M0 scale is folded into A, so the tensor core accumulates the whole K
+// range in FP32 without a per-group step) and copy the BF16 activation rows
+// of up to 64 tokens of the expert (B, in a ring of its own, two tiles
+// ahead), both into shared memory in the
+// K-major core-matrix layout (8 rows x 16 bytes per core matrix).  One thread
+// then issues the tile's 4 x NMAT tcgen05.mma (M = 128, N = tokens rounded up
+// to 16, at most 64, K = 16, BF16 x BF16 -> FP32 in TMEM) and commits them to the tile's
+// mbarrier; two tiles alternate, so the dequantisation of one overlaps the
+// products of the other.  The epilogue reads the accumulators from TMEM
+// (tcgen05.ld: warp w reads rows 32 (w % 4) .. + 31, the (w / 4)-th quarter
+// of the token columns) and applies the same
+// rounding points as the other paths: h = BF16(BF16(silu(BF16(g))) BF16(u))
+// for gate / up, o = BF16(acc) for down.  Products are exact in FP32; only
+// the FP32 summation order differs from the oracle.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "gemv.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kTcM = 128;          // matrix rows per CTA (MMA M)
+constexpr int kTcK = 64;           // K per shared-memory tile (4 MMAs of K = 16)
+constexpr int kTcMaxN = 64;        // tokens per pass (MMA N <= 64, a multiple of 16)
+constexpr int kTcThreads = 512;    // 4 threads per weight row, 16 warps
+constexpr uint32_t kTcTileA = kTcM * kTcK * 2;    // 16 KB of BF16 per matrix
+constexpr uint32_t kTcTileB = kTcMaxN * kTcK * 2; // 8 KB of BF16
+constexpr int kTcBSlots = 4;                      // B tiles in flight (ring)
+
+__host__ __device__ constexpr uint32_t tc_stage_bytes(int nmat) {
+    return (uint32_t)nmat * kTcTileA;  // an MMA stage holds the A tiles
+}
+
+// Byte offset of element (row, k) of a K-major tile with 64 K per row: core
+// matrices of 8 rows x 8 elements (16 bytes per row, 128 bytes each); the 8
+// K-chunks of a group of 8 rows lie 128 bytes apart (leading byte offset),
+// groups of 8 rows 1024 bytes apart (stride byte offset).
+__device__ __forceinline__ uint32_t tc_off(int row, int kchunk) {
+    return (uint32_t)(row >> 3) * 1024u + (uint32_t)kchunk * 128u + (uint32_t)(row & 7) * 16u;
+}
+
+// Shared-memory matrix descriptor: no swizzle, K-major; start address,
+// leading byte offset 128 (next K-chunk), stride byte offset 1024 (next 8
+// rows), all in 16-byte units; version 1 (bits 46..47).
+__device__ __forceinline__ uint64_t tc_desc(uint32_t smem_addr) {
+    return (uint64_t)((smem_addr >> 4) & 0x3FFFu) | ((uint64_t)(128u >> 4) << 16) |
+           ((uint64_t)(1024u >> 4) << 32) | (1ull << 46);
+}
+
+// Instruction descriptor of kind::f16: FP32 accumulator (bits 4..5 = 1),
+// A and B BF16 (bits 7..9 and 10..12 = 1), both K-major, N / 8 at bit 17,
+// M / 16 at bit 24.
+__device__ __forceinline__ uint32_t tc_idesc(int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+           ((uint32_t)(kTcM >> 4) << 24);
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, bool accumulate) {
+    asm volatile(
+        "{\n\t"
+        ".reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate ? 1u : 0u)
+        : "memory");
+}
+
+// Arrive on *bar once every tcgen05 operation issued so far by this thread
+// has completed.
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Generic-proxy shared-memory writes -> visible to the tensor core.
+__device__ __forceinline__ void fence_async_shared() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 32 lanes x 32 bits x 8 columns of TMEM: lane l of the warp gets row
+// (taddr lane field + l), columns taddr .. taddr + 7.
+__device__ __forceinline__ void tc_ld8(uint32_t taddr, float (&v)[8]) {
+    uint32_t r[8];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void cp_async16_tc(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// 8 E2M1 codes (one 4-byte word) times the scale sf -> 8 BF16 (exact: the
+// products have at most 2 significant bits).
+__device__ __forceinline__ uint4 dequant8_bf16(uint32_t w, float sf) {
+    uint32_t h[4];
+    e2m1x8_to_f16x8(w, h);
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        o[i] = pack_bf16x2(f16_bits_to_f32(h[i] & 0xFFFFu) * sf, f16_bits_to_f32(h[i] >> 16) * sf);
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ const uint8_t *tc_scales(const GroupedParams &p, int e, int m) {
+    return p.codes_base ? p.scales_base + (size_t)(3 * e + m) * p.scales_stride
+                        : p.table[e].scales[m];
+}
+
+}  // namespace
+
+namespace {
+
+constexpr int kTcRaw = 4;  // packed K tiles in flight (TMA ring slots)
+constexpr int kTcTma = 32; // the thread issuing the TMA loads (thread 0 issues the MMAs)
+constexpr uint32_t kTcRawSlot = kTcM * 32;  // bytes of one matrix's packed tile
+
+// Shared-memory plan of one CTA (dynamic part): 2 MMA stages of A tiles
+// (NMAT x 16 KB BF16); the B ring [kTcBSlots][8 KB BF16]; the packed codes
+// ring [kTcRaw][NMAT][128 rows][32 bytes]; the CTA's scale rows
+// [NMAT][128][K/32].
+__host__ __device__ constexpr uint32_t tc_b_off(int nmat) { return 2 * tc_stage_bytes(nmat); }
+__host__ __device__ constexpr uint32_t tc_raw_off(int nmat) {
+    return tc_b_off(nmat) + (uint32_t)kTcBSlots * kTcTileB;
+}
+__host__ __device__ constexpr uint32_t tc_sc_off(int nmat) {
+    return tc_raw_off(nmat) + (uint32_t)kTcRaw * nmat * kTcRawSlot;
+}
+__host__ __device__ inline uint32_t tc_smem_bytes(int nmat, int K) {
+    return tc_sc_off(nmat) + (uint32_t)nmat * kTcM * (uint32_t)(K / 32);
+}
+
+// One TMA tile load of the 3-D code tensor (x: byte in the row, y: row,
+// z: matrix 3 e + m) into shared memory, completing on *bar.  Loads only
+// this GPU's memory; no multicast.
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int x, int y, int z,
+                                            uint64_t *bar, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
+}
+
+template <int NMAT>
+__global__ void __launch_bounds__(kTcThreads, 1)
+grouped_tc_kernel(const GroupedParams p, const __grid_constant__ CUtensorMap codes_map) {
+    extern __shared__ __align__(1024) uint8_t sm[];
+    __shared__ __align__(8) uint64_t s_mma[2];        // tile products of stage s done
+    __shared__ __align__(8) uint64_t s_raw[kTcRaw];  // packed tile of ring slot j landed
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_src[2][kTcMaxN];  // B row of each token of pass P (parity P & 1)
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int e = blockIdx.y;
+    pdl_wait();
+    pdl_launch_dependents();
+    const int seg0 = p.offs[e], n_e = p.offs[e + 1] - seg0;
+    if (n_e <= 0) return;  // uniform: no token chose this expert (no TMEM taken)
+
+    const int K = NMAT == 2 ? p.H : p.I;  // reduction length
+    const int M = NMAT == 2 ? p.I : p.H;  // matrix rows (a multiple of 128)
+    const int row0 = blockIdx.x * kTcM;
+    const int nkt = K / kTcK;
+    const int npass = (n_e + kTcMaxN - 1) / kTcMaxN;
+    const int total = npass * nkt;  // (pass, K tile) iterations
+    const uint32_t rs = (uint32_t)K >> 5;
+    uint8_t *raw = sm + tc_raw_off(NMAT);
+    uint8_t *scl = sm + tc_sc_off(NMAT);
+
+    if (warp == 0) {  // TMEM: NMAT x 256 FP32 columns x 128 lanes
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(&s_tmem)), "r"(NMAT * kTcMaxN)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        mbar_init(&s_mma[0], 1);
+        mbar_init(&s_mma[1], 1);
+#pragma unroll
+        for (int j = 0; j < kTcRaw; ++j) mbar_init(&s_raw[j], 1);
+        mbar_fence_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    const uint64_t pol = l2_evict_first_policy();  // packed rows are read once
+
+    // packed tile of iteration it (K tile it % nkt) into ring slot it % kTcRaw,
+    // by thread kTcTma (raw_next: loads issued so far, in iteration order)
+    int raw_next = 0;
+    auto issue_raw = [&](int it) {
+        raw_next = it + 1;
+        const int j = it % kTcRaw, kt = it % nkt;
+        mbar_arrive_expect_tx(&s_raw[j], (unsigned)(NMAT * kTcRawSlot));
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m)
+            tma_load_3d(raw + ((uint32_t)j * NMAT + m) * kTcRawSlot, &codes_map, kt * 32, row0,
+                        3 * e + (NMAT == 2 ? m : 2), &s_raw[j], pol);
+    };
+    // B rows of iteration it (its pass's tokens, K tile kt) into ring slot it % kTcBSlots
+    auto issue_b = [&](int it) {
+        const int pass = it / nkt, kt = it % nkt;
+        const int tc = pass * kTcMaxN, nt = min(kTcMaxN, n_e - tc);
+        uint8_t *b = sm + tc_b_off(NMAT) + (uint32_t)(it % kTcBSlots) * kTcTileB;
+        const uint16_t *base = NMAT == 2 ? p.x : p.h;
+        for (int i = tid; i < nt * 8; i += kTcThreads) {
+            const int n = i >> 3, c = i & 7;
+            cp_async16_tc(b + tc_off(n, c), base + (size_t)s_src[pass & 1][n] * K + kt * kTcK + c * 8);
+        }
+    };
+    // the B rows (x row of the pair's token, or h row of the pair) of pass P's
+    // tokens into s_src[P & 1]
+    auto fill_src = [&](int P) {
+        const int tc = P * kTcMaxN;
+        if (tid < kTcMaxN && tc + tid < n_e) {
+            const int pr = p.perm[seg0 + tc + tid];
+            s_src[P & 1][tid] = NMAT == 2 ? pr / p.k : pr;
+        }
+    };
+
+    // prologue: the CTA's scale rows and B of iteration 0 (one copy group), B
+    // of iteration 1 (another), packed tiles 0 .. kTcRaw - 2
+    // this thread's row and K quarter (a warp covers 8 consecutive rows: its
+    // reads of the packed ring are contiguous)
+    const int rrow = tid >> 2, quarter = tid & 3;
+    fill_src(0);
+    if (npass > 1) fill_src(1);
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < NMAT; ++m) {
+        const int mat = NMAT == 2 ? m : 2;
+        const uint8_t *gsc = tc_scales(p, e, mat) + (size_t)(row0 + rrow) * rs;
+        // K / 32 is a multiple of 4 (K % 128 == 0): the row's scales in 4-byte
+        // pieces, spread over its four threads
+        for (uint32_t c = 4 * quarter; c < rs; c += 16)
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
+                             smem_u32(scl + ((uint32_t)m * kTcM + rrow) * rs + c)),
+                         "l"(gsc + c)
+                         : "memory");
+    }
+    issue_b(0);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    if (total > 1) issue_b(1);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    if (tid == kTcTma) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&codes_map))
+                     : "memory");
+#pragma unroll 1
+        for (int j = 0; j < kTcRaw - 1 && j < total; ++j) issue_raw(j);
+    }
+
+    bool ok = true;
+    int issued = 0;  // iterations whose products were issued (uniform)
+    #pragma unroll 1
+    for (int it = 0; it < total; ++it) {
+        const int s = it & 1, pass = it / nkt, kt = it % nkt;
+        const int tc = pass * kTcMaxN, nt = min(kTcMaxN, n_e - tc);
+        // ring slot of iteration it - 1 was read by every thread before the
+        // barrier that ended it: refill it with tile it + kTcRaw - 1
+        if (tid == kTcTma && it + kTcRaw - 1 < total) issue_raw(it + kTcRaw - 1);
+        // the next pass's B rows, read from iteration (pass + 2) nkt - 2 on
+        if (kt == 0 && pass >= 1 && pass + 1 < npass) fill_src(pass + 1);
+        // A stage s and B slot (it + 2) % kTcBSlots were last read by the
+        // products of iteration it - 2
+        if (it >= 2 && !mbar_wait(&s_mma[s], (unsigned)((it - 2) >> 1) & 1u)) ok = false;
+        if (it + 2 < total) issue_b(it + 2);
+        // one group per iteration: all but the 2 newest = B of this iteration
+        // (and, at it = 0, the scale rows)
+        asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 2;" ::: "memory");
+        if (!mbar_wait(&s_raw[it % kTcRaw], (unsigned)(it / kTcRaw) & 1u)) ok = false;
+        // ---- dequantise this thread's part of tile kt into stage s ----
+        uint8_t *st = sm + (uint32_t)s * tc_stage_bytes(NMAT);
+        const uint8_t *slot = raw + (uint32_t)(it % kTcRaw) * NMAT * kTcRawSlot;
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m) {
+            // K-chunks 2 q, 2 q + 1 of the row (8 code bytes; one scale group)
+            const uint2 cw = *reinterpret_cast<const uint2 *>(
+                slot + (uint32_t)m * kTcRawSlot + (uint32_t)rrow * 32 + 8 * quarter);
+            const float sf = e8m0_to_f32(scl[((uint32_t)m * kTcM + rrow) * rs + 2 * kt + (quarter >> 1)]);
+            uint8_t *a = st + (uint32_t)m * kTcTileA;
+            *reinterpret_cast<uint4 *>(a + tc_off(rrow, 2 * quarter)) = dequant8_bf16(cw.x, sf);
+            *reinterpret_cast<uint4 *>(a + tc_off(rrow, 2 * quarter + 1)) = dequant8_bf16(cw.y, sf);
+        }
+        fence_async_shared();
+        ok = __syncthreads_and(ok) != 0;  // every thread's A and B writes
+        if (!ok) break;  // uniform; every copy and product is drained below
+        if (tid == 0) {
+            tc_fence_after();
+            const int N = (nt + 15) & ~15;
+            const uint32_t idesc = tc_idesc(N);
+            const uint32_t b_addr =
+                smem_u32(sm + tc_b_off(NMAT) + (uint32_t)(it % kTcBSlots) * kTcTileB);
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m) {
+                const uint32_t a_addr = smem_u32(st + (uint32_t)m * kTcTileA);
+#pragma unroll
+                for (int kk = 0; kk < kTcK / 16; ++kk)
+                    tc_mma(tmem + (uint32_t)(m * kTcMaxN), tc_desc(a_addr + kk * 256),
+                           tc_desc(b_addr + kk * 256), idesc, kt > 0 || kk > 0);
+            }
+            tc_commit(&s_mma[s]);
+        }
+        issued = it + 1;
+        if (kt == nkt - 1) {
+            // ---- epilogue of this pass: accumulators -> outputs ----
+            if (!mbar_wait(&s_mma[s], (unsigned)(it >> 1) & 1u)) ok = false;
+            tc_fence_after();
+            const int lq = warp & 3;                // TMEM lane quarter of this warp
+            const int r = row0 + lq * 32 + lane;    // this thread's matrix row
+            const uint32_t lane_base = tmem + ((uint32_t)(lq * 32) << 16);
+            const int N = (nt + 15) & ~15;
+            #pragma unroll 1
+            for (int c0 = 8 * (warp >> 2); c0 < N; c0 += 32) {
+                float g[8], u[8];
+                tc_ld8(lane_base + (uint32_t)c0, g);
+                if (NMAT == 2) tc_ld8(lane_base + (uint32_t)(kTcMaxN + c0), u);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int idx = tc + c0 + j;
+                    if (!ok || idx >= tc + nt) continue;
+                    const int pr = p.perm[seg0 + idx];
+                    if (NMAT == 2) {
+                        const float gv = round_bf16(g[j]);
+                        const float uv = round_bf16(u[j]);
+                        const float sl = round_bf16(gv / (1.0f + expf(-gv)));
+                        p.h[(size_t)pr * M + r] = f32_to_bf16(sl * uv);
+                    } else {
+                        p.o[(size_t)pr * M + r] = f32_to_bf16(g[j]);
+                    }
+                }
+            }
+            tc_fence_before();
+            ok = __syncthreads_and(ok) != 0;  // TMEM read before the next pass overwrites it
+            if (!ok) break;
+        }
+    }
+    if (!ok && tid == 0) atomicOr(p.status, kTimeoutStatus);
+    // nothing in flight at exit (bounded waits): this thread's copies, the
+    // products issued, the packed tiles issued
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    if (issued > 0) mbar_wait(&s_mma[(issued - 1) & 1], (unsigned)((issued - 1) >> 1) & 1u);
+    if (tid == kTcTma)  // the last loads issued, one per ring slot (earlier ones were consumed)
+        for (int j = max(0, raw_next - kTcRaw); j < raw_next; ++j)
+            mbar_wait(&s_raw[j % kTcRaw], (unsigned)(j / kTcRaw) & 1u);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(NMAT * kTcMaxN)
+                     : "memory");
+    }
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ host --
+
+namespace {
+
+// The 3-D tensor map of the packed codes of one matrix kind: x = byte in a
+// row (K / 2), y = row (M), z = matrix index 3 e + m over every expert;
+// boxes of 32 bytes x 128 rows x 1 matrix.  Encoded once per (base, shape).
+struct CodesMap {
+    const void *base = nullptr;
+    int E = 0, rows = 0, K = 0;
+    CUtensorMap map;
+};
+
+PFN_cuTensorMapEncodeTiled encode_fn() {
+    static PFN_cuTensorMapEncodeTiled fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(p);
+    }
+    return fn;
+}
+
+cudaError_t codes_map(CodesMap &c, const uint8_t *base, size_t matrix_stride, int E, int rows,
+                      int K) {
+    if (c.base == base && c.E == E && c.rows == rows && c.K == K) return cudaSuccess;
+    PFN_cuTensorMapEncodeTiled fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[3] = {(cuuint64_t)K / 2, (cuuint64_t)rows, (cuuint64_t)3 * E};
+    const cuuint64_t strides[2] = {(cuuint64_t)K / 2, (cuuint64_t)matrix_stride};
+    const cuuint32_t box[3] = {32, (cuuint32_t)kTcM, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(&c.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    c.base = base;
+    c.E = E;
+    c.rows = rows;
+    c.K = K;
+    return cudaSuccess;
+}
+
+template <int NMAT>
+cudaError_t launch_tc(const GroupedParams &p, const CUtensorMap &map, cudaStream_t s, bool pdl) {
+    const int K = NMAT == 2 ? p.H : p.I, M = NMAT == 2 ? p.I : p.H;
+    const size_t smem = tc_smem_bytes(NMAT, K);
+    static size_t attr_smem = 0;  // largest dynamic shared memory enabled so far
+    if (smem > attr_smem) {
+        cudaError_t e = cudaFuncSetAttribute(grouped_tc_kernel<NMAT>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_smem = smem;
+    }
+    return launch_ex(grouped_tc_kernel<NMAT>, dim3(M / kTcM, p.E), dim3(kTcThreads), smem, s, pdl,
+                     p, map);
+}
+
+}  // namespace
+
+// The tensor-core products need the contiguous weight layout (one tensor map
+// per matrix kind), H and I multiples of 128 and the shared-memory plan
+// within the budget.
+bool grouped_tc_supported(int H, int I) {
+    return H % 128 == 0 && I % 128 == 0 && tc_smem_bytes(2, H) <= 220 * 1024 &&
+           tc_smem_bytes(1, I) <= 220 * 1024;
+}
+
+cudaError_t launch_grouped_tc_gateup(const GroupedParams &p, cudaStream_t s, bool pdl) {
+    static CodesMap gu;
+    if (!p.codes_base) return cudaErrorInvalidValue;
+    cudaError_t e = codes_map(gu, p.codes_base, p.codes_stride, p.E, p.I, p.H);
+    if (e != cudaSuccess) return e;
+    return launch_tc<2>(p, gu.map, s, pdl);
+}
+
+cudaError_t launch_grouped_tc_down(const GroupedParams &p, cudaStream_t s, bool pdl) {
+    static CodesMap dn;
+    if (!p.codes_base) return cudaErrorInvalidValue;
+    cudaError_t e = codes_map(dn, p.codes_base, p.codes_stride, p.E, p.H, p.I);
+    if (e != cudaSuccess) return e;
+    return launch_tc<1>(p, dn.map, s, pdl);
+}
+
+}  // namespace moe

@@ -117,7 +117,7 @@ struct DownParams {
 };
 
 // The (token, expert)-sorted grouped path (grouped.cu), for batches of tokens.
-constexpr int kGroupedMaxT = 256;  // tokens per grouped launch sequence (more: chunks)
+constexpr int kGroupedMaxT = 2048;  // tokens per grouped launch sequence (more: chunks)
 struct GroupedParams {
     const ExpertPtrs *table;
     const uint8_t *codes_base, *scales_base;  // contiguous layout fast path (or null)
@@ -139,9 +139,15 @@ struct GroupedParams {
     uint16_t *o;               // [T k][H] BF16 expert outputs
     unsigned *status;
     int T, k, E, H, I;
+    int tcgen05;               // products on tcgen05 (else mma.sync tiles)
 };
 bool grouped_supported(int E, int H, int I);
 cudaError_t launch_grouped(const GroupedParams &p, cudaStream_t s, bool pdl);
+// Products on tcgen05 (grouped_tc.cu), on request: measured slower than the
+// mma.sync tiles at every batch tried (T <= 1024, 24B shape).
+bool grouped_tc_supported(int H, int I);
+cudaError_t launch_grouped_tc_gateup(const GroupedParams &p, cudaStream_t s, bool pdl);
+cudaError_t launch_grouped_tc_down(const GroupedParams &p, cudaStream_t s, bool pdl);
 
 // Host-side launchers (decode.cu).  `pdl` sets programmatic stream
 // serialization so the kernel may start while the previous one drains.
