@@ -492,14 +492,17 @@ def kernel_breakdown(torch, moe, st, reps):
 
 
 BATCHED_CASES = ((32, "uniform"), (32, "zipf"), (64, "uniform"), (256, "uniform"),
-                 (256, "zipf"))
+                 (256, "zipf"), (1024, "uniform"), (2048, "uniform"), (2048, "zipf"))
+TC_AUTO_GROUP = 40  # the library's tcgen05 products from T k >= 40 E on
 
 
 def batched_cases(torch, moe, st, seed, reps=20):
     """The grouped (token, expert)-sorted path on one 24B layer of the stack at
     batch sizes beyond decode: synthetic routing (k distinct experts per token,
     uniform or Zipf(1.1) popularity), moe_forward timed in a CUDA graph of
-    `reps` calls.  Bytes: the touched experts' packed weights + activations."""
+    `reps` calls.  Bytes: the touched experts' packed weights + activations.
+    Where the library picks the tcgen05 products, the mma.sync tiles are timed
+    beside them (FWD_FORCE_MMA)."""
     L = st.layers[0]
     out = []
     expert = 3 * SHAPE.I * SHAPE.H // 2 + 3 * SHAPE.I * SHAPE.H // 32
@@ -514,28 +517,37 @@ def batched_cases(torch, moe, st, seed, reps=20):
                                         synth.rng_for(seed, 91, T))
         ids, w = torch.from_numpy(ids_h).cuda(), torch.from_numpy(w_h).cuda()
         y = torch.empty_like(x)
-        s.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(s):
-            lay.forward(x, ids, w, y=y, stream=s)
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=s):
-            for _ in range(reps):
-                lay.forward(x, ids, w, y=y, stream=s)
-        g.replay()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        g.replay()
-        e1.record()
-        torch.cuda.synchronize()
-        us = e0.elapsed_time(e1) * 1e3 / reps
+        tc = T * SHAPE.top_k >= TC_AUTO_GROUP * SHAPE.E
+
+        def timed(flags):
+            s.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(s):
+                lay.forward(x, ids, w, y=y, flags=flags, stream=s)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                for _ in range(reps):
+                    lay.forward(x, ids, w, y=y, flags=flags, stream=s)
+            g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            del g
+            return e0.elapsed_time(e1) * 1e3 / reps
+
+        us = timed(0)
         touched = len(set(ids_h.ravel().tolist()))
         nbytes = touched * expert + T * SHAPE.H * 2 * 2
-        out.append({"T": T, "routing": dist, "experts_touched": touched,
-                    "us_per_call": us, "tokens_per_s": T / (us * 1e-6),
-                    "hbm_gbs": nbytes / (us * 1e-6) / 1e9})
-        del g
+        row = {"T": T, "routing": dist, "experts_touched": touched,
+               "products": "tcgen05" if tc else "mma.sync",
+               "us_per_call": us, "tokens_per_s": T / (us * 1e-6),
+               "hbm_gbs": nbytes / (us * 1e-6) / 1e9}
+        if tc:
+            row["us_per_call_mma_sync"] = timed(moe.FWD_FORCE_MMA)
+        out.append(row)
     lay.close()
     return out
 

@@ -123,6 +123,8 @@ typedef enum moe_status {
                                       loads of the packed codes); needs the
                                       contiguous weights of moe_load_packed
                                       and H, I multiples of 128, else ARG  */
+#define MOE_FWD_FORCE_MMA 0x40u    /* grouped path with its products on
+                                      mma.sync tiles (never tcgen05)        */
 
 /* Create a layer of E experts with hidden size H, intermediate size I and
  * top_k experts per token.  Requires H % 32 == 0, I % 32 == 0,
@@ -214,9 +216,12 @@ MOE_API int moe_route_ex(moe_handle_t h, const uint16_t *x, int T,
  * makes that slot contribute 0 and sets MOE_DEVICE_BAD_EXPERT_ID in the
  * device status word.  T = 1..4 runs the per-(token, slot) GEMV path;
  * larger T the (token, expert)-sorted grouped path, in chunks of up to 2048
- * tokens: its products run on mma.sync tiles, or with MOE_FWD_FORCE_TCGEN05
- * on tcgen05 (BF16 weight tiles dequantised once per CTA, FP32 accumulators
- * in tensor memory, packed codes brought in by TMA tensor loads).  Errors: ARG,
+ * tokens: its products run on mma.sync tiles, or on tcgen05 (BF16 weight tiles
+ * dequantised once per CTA, FP32 accumulators in tensor memory, packed codes
+ * brought in by TMA tensor loads) when a chunk's groups average at least 40
+ * (token, slot) pairs per expert (T k >= 40 E) and the weights allow it
+ * (contiguous MXFP4 from moe_load_packed, H and I multiples of 128);
+ * MOE_FWD_FORCE_TCGEN05 / MOE_FWD_FORCE_MMA pin the choice.  Errors: ARG,
  * NOT_LOADED, NOT_DEVICE, ALIGN, WORKSPACE, CUDA. */
 MOE_API int moe_forward(moe_handle_t h, const uint16_t *x, int T,
                 const int32_t *topk_ids, const float *topk_w, uint16_t *y,

@@ -29,7 +29,7 @@ __all__ = [
     "moe_bytes_per_expert", "moe_set_tuning", "moe_device_check", "moe_debug_dequant",
     "moe_forward_noalloc",
     "ROUTE_RMSNORM", "ROUTE_SIGMOID", "FWD_KEEP_INTERMEDIATES", "FWD_FORCE_DECODE", "FWD_FORCE_GROUPED",
-    "FWD_PHASE_GATEUP", "FWD_PHASE_DOWN", "FWD_FORCE_TCGEN05",
+    "FWD_PHASE_GATEUP", "FWD_PHASE_DOWN", "FWD_FORCE_TCGEN05", "FWD_FORCE_MMA",
     "FUSION_NONE", "FUSION_ROUTER", "FUSION_LAYER", "moe_set_fusion",
     "DEVICE_BAD_EXPERT_ID",
 ]
@@ -42,6 +42,7 @@ FWD_FORCE_GROUPED = 0x4
 FWD_PHASE_GATEUP = 0x8
 FWD_PHASE_DOWN = 0x10
 FWD_FORCE_TCGEN05 = 0x20
+FWD_FORCE_MMA = 0x40
 FUSION_NONE, FUSION_ROUTER, FUSION_LAYER = 0, 1, 2
 DEVICE_BAD_EXPERT_ID = 0x1
 DEVICE_TIMEOUT = 0x2

@@ -332,11 +332,18 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
     if (!h || T < 1) return MOE_ERR_ARG;
     const unsigned known = MOE_FWD_KEEP_INTERMEDIATES | MOE_FWD_FORCE_DECODE |
                            MOE_FWD_FORCE_GROUPED | MOE_FWD_PHASE_GATEUP | MOE_FWD_PHASE_DOWN |
-                           MOE_FWD_FORCE_TCGEN05;
+                           MOE_FWD_FORCE_TCGEN05 | MOE_FWD_FORCE_MMA;
     if (flags & ~known) return MOE_ERR_ARG;
+    if ((flags & MOE_FWD_FORCE_TCGEN05) && (flags & MOE_FWD_FORCE_MMA)) return MOE_ERR_ARG;
+    if (flags & MOE_FWD_FORCE_MMA) {
+        if (flags & MOE_FWD_FORCE_DECODE) return MOE_ERR_ARG;
+        flags |= MOE_FWD_FORCE_GROUPED;
+    }
     if (flags & MOE_FWD_FORCE_TCGEN05) {
         if (flags & MOE_FWD_FORCE_DECODE) return MOE_ERR_ARG;
-        if (h->nv || !h->codes_base || !moe::grouped_tc_supported(h->H, h->I)) return MOE_ERR_ARG;
+        const int Tc = T < moe::kGroupedMaxT ? T : moe::kGroupedMaxT;
+        if (h->nv || !h->codes_base || !moe::grouped_tc_supported(h->H, h->I, Tc * h->k))
+            return MOE_ERR_ARG;
         flags |= MOE_FWD_FORCE_GROUPED;
     }
     if ((flags & MOE_FWD_FORCE_DECODE) && (flags & MOE_FWD_FORCE_GROUPED)) return MOE_ERR_ARG;
@@ -396,7 +403,13 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
             gp.E = h->E;
             gp.H = h->H;
             gp.I = h->I;
-            gp.tcgen05 = (flags & MOE_FWD_FORCE_TCGEN05) ? 1 : 0;
+            // tcgen05 when the groups are large enough to amortise a CTA's
+            // dequantised tiles over its token passes
+            const bool tc_ok = !h->nv && h->codes_base &&
+                               moe::grouped_tc_supported(h->H, h->I, Tc * h->k);
+            gp.tcgen05 = (flags & MOE_FWD_FORCE_TCGEN05) ||
+                         (!(flags & MOE_FWD_FORCE_MMA) && tc_ok &&
+                          (long long)Tc * h->k >= (long long)moe::kTcAutoGroup * h->E);
             if ((rc = cuda_rc(moe::launch_grouped(gp, s, h->use_pdl))) != MOE_OK) return rc;
         }
         h->kept = keep;

@@ -434,6 +434,8 @@ bool grouped_supported(int E, int H, int I) {
 cudaError_t launch_grouped(const GroupedParams &p, cudaStream_t s, bool pdl) {
     if (p.T < 1 || p.T > kGroupedMaxT || !grouped_supported(p.E, p.H, p.I))
         return cudaErrorInvalidValue;
+    if (p.tcgen05 && (!p.codes_base || !grouped_tc_supported(p.H, p.I, p.T * p.k)))
+        return cudaErrorInvalidValue;
     cudaError_t e;
     if ((e = launch_ex(grouped_prep_kernel, dim3(p.T + 1), dim3(kGpThreads), 0, s, pdl, p)) !=
         cudaSuccess)
@@ -441,7 +443,6 @@ cudaError_t launch_grouped(const GroupedParams &p, cudaStream_t s, bool pdl) {
     if (p.tcgen05) {
         // the products on tcgen05 (BF16 tiles, TMEM accumulators; they read
         // x and h in BF16, so h needs no FP16 staging)
-        if (!p.codes_base || !grouped_tc_supported(p.H, p.I)) return cudaErrorInvalidValue;
         if ((e = launch_grouped_tc_gateup(p, s, pdl)) != cudaSuccess) return e;
         if ((e = launch_grouped_tc_down(p, s, pdl)) != cudaSuccess) return e;
     } else {

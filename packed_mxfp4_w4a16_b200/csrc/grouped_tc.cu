@@ -9,19 +9,19 @@
 // (.aimodel)", section "Provenance" (the batched path sorts the (token,
 // expert) pairs so that each expert's tokens form one group).
 //
-// One CTA per (128 rows of a matrix, expert), 16 warps.  The CTA walks K in
-// tiles of 64.  The packed codes of each tile (128 rows x 32 bytes per
-// matrix) arrive by one TMA tensor load into a ring of shared-memory slots,
-// several tiles ahead (mbarrier completion); per tile, the threads (four per
-// row, a quarter of the tile's K each) dequantise the 128 x 64 packed weights
-// of each matrix into BF16 (value = E2M1 code x 2^(e-127), exact in BF16: the
-// E8M0 scale is folded into A, so the tensor core accumulates the whole K
-// range in FP32 without a per-group step) and copy the BF16 activation rows
-// of up to 64 tokens of the expert (B, in a ring of its own, two tiles
-// ahead), both into shared memory in the
+// One CTA per (128 rows of a matrix, expert), 16 conversion warps and one
+// MMA / TMA warp.  The CTA walks K in tiles of 64.  The packed codes of each
+// tile (128 rows x 32 bytes per matrix) arrive by one TMA tensor load into a
+// ring of shared-memory slots, several tiles ahead (mbarrier completion); per
+// tile, the threads (four per row, a quarter of the tile's K each) dequantise
+// the 128 x 64 packed weights of each matrix into BF16 (code x 2^(e-127),
+// exact in BF16: the E8M0 scale is folded into A, so the tensor core
+// accumulates the whole K range in FP32 without a per-group step) and copy
+// the BF16 activation rows of up to 128 tokens of the expert (B, in a ring of
+// its own, two tiles ahead), both into shared memory in the
 // K-major core-matrix layout (8 rows x 16 bytes per core matrix).  One thread
 // then issues the tile's 4 x NMAT tcgen05.mma (M = 128, N = tokens rounded up
-// to 16, at most 64, K = 16, BF16 x BF16 -> FP32 in TMEM) and commits them to the tile's
+// to 16, at most 128, K = 16, BF16 x BF16 -> FP32 in TMEM) and commits them to the tile's
 // mbarrier; two tiles alternate, so the dequantisation of one overlaps the
 // products of the other.  The epilogue reads the accumulators from TMEM
 // (tcgen05.ld: warp w reads rows 32 (w % 4) .. + 31, the (w / 4)-th quarter
@@ -43,10 +43,11 @@ namespace {
 
 constexpr int kTcM = 128;          // matrix rows per CTA (MMA M)
 constexpr int kTcK = 64;           // K per shared-memory tile (4 MMAs of K = 16)
-constexpr int kTcMaxN = 64;        // tokens per pass (MMA N <= 64, a multiple of 16)
-constexpr int kTcThreads = 512;    // 4 threads per weight row, 16 warps
+constexpr int kTcMaxN = 128;       // tokens per pass (MMA N <= 128, a multiple of 16)
+constexpr int kTcWork = 512;       // conversion threads: 4 per weight row, 16 warps
+constexpr int kTcThreads = kTcWork + 32;  // + the MMA / TMA warp
 constexpr uint32_t kTcTileA = kTcM * kTcK * 2;    // 16 KB of BF16 per matrix
-constexpr uint32_t kTcTileB = kTcMaxN * kTcK * 2; // 8 KB of BF16
+constexpr uint32_t kTcTileB = kTcMaxN * kTcK * 2; // 16 KB of BF16
 constexpr int kTcBSlots = 4;                      // B tiles in flight (ring)
 
 __host__ __device__ constexpr uint32_t tc_stage_bytes(int nmat) {
@@ -145,6 +146,12 @@ __device__ __forceinline__ uint4 dequant8_bf16(uint32_t w, float sf) {
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// Barrier of the conversion threads alone (named barrier 1; every
+// conversion warp executes it, the MMA warp does not).
+__device__ __forceinline__ void conv_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kTcWork) : "memory");
+}
+
 __device__ __forceinline__ const uint8_t *tc_scales(const GroupedParams &p, int e, int m) {
     return p.codes_base ? p.scales_base + (size_t)(3 * e + m) * p.scales_stride
                         : p.table[e].scales[m];
@@ -155,11 +162,10 @@ __device__ __forceinline__ const uint8_t *tc_scales(const GroupedParams &p, int 
 namespace {
 
 constexpr int kTcRaw = 4;  // packed K tiles in flight (TMA ring slots)
-constexpr int kTcTma = 32; // the thread issuing the TMA loads (thread 0 issues the MMAs)
 constexpr uint32_t kTcRawSlot = kTcM * 32;  // bytes of one matrix's packed tile
 
 // Shared-memory plan of one CTA (dynamic part): 2 MMA stages of A tiles
-// (NMAT x 16 KB BF16); the B ring [kTcBSlots][8 KB BF16]; the packed codes
+// (NMAT x 16 KB BF16); the B ring [kTcBSlots][16 KB BF16]; the packed codes
 // ring [kTcRaw][NMAT][128 rows][32 bytes]; the CTA's scale rows
 // [NMAT][128][K/32].
 __host__ __device__ constexpr uint32_t tc_b_off(int nmat) { return 2 * tc_stage_bytes(nmat); }
@@ -169,8 +175,13 @@ __host__ __device__ constexpr uint32_t tc_raw_off(int nmat) {
 __host__ __device__ constexpr uint32_t tc_sc_off(int nmat) {
     return tc_raw_off(nmat) + (uint32_t)kTcRaw * nmat * kTcRawSlot;
 }
-__host__ __device__ inline uint32_t tc_smem_bytes(int nmat, int K) {
+// then the B row of every token of the group ([pairs] ints; a group holds at
+// most all the launch's T k pairs)
+__host__ __device__ inline uint32_t tc_src_off(int nmat, int K) {
     return tc_sc_off(nmat) + (uint32_t)nmat * kTcM * (uint32_t)(K / 32);
+}
+__host__ __device__ inline uint32_t tc_smem_bytes(int nmat, int K, int pairs) {
+    return tc_src_off(nmat, K) + (uint32_t)pairs * sizeof(int);
 }
 
 // One TMA tile load of the 3-D code tensor (x: byte in the row, y: row,
@@ -185,14 +196,34 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
+// Bounded wait on phase `parity` of *bar that also gives up once *abort is
+// set; a timeout sets *abort, so every other wait of the CTA ends too.
+__device__ __forceinline__ bool tc_wait(uint64_t *bar, unsigned parity, volatile int *abort) {
+    #pragma unroll 1
+    for (int i = 0; i < kMaxSpin; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+    }
+    *abort = 1;
+    return false;
+}
+
+// Warp-specialised: warps 0..15 convert (A tiles, B copies, epilogue), warp
+// 16 (lane 0) issues the TMA loads of the packed codes and the MMAs.  Stage
+// hand-offs: s_full[s] (16 conversion-warp arrivals: A and B of the tile are
+// in shared memory), s_mma[s] (tcgen05.commit: the tile's products are done,
+// the stage may be rewritten), s_raw[j] (TMA bytes of ring slot j), s_tfree
+// (16 arrivals: the pass's accumulators were read).
 template <int NMAT>
 __global__ void __launch_bounds__(kTcThreads, 1)
 grouped_tc_kernel(const GroupedParams p, const __grid_constant__ CUtensorMap codes_map) {
     extern __shared__ __align__(1024) uint8_t sm[];
-    __shared__ __align__(8) uint64_t s_mma[2];        // tile products of stage s done
-    __shared__ __align__(8) uint64_t s_raw[kTcRaw];  // packed tile of ring slot j landed
+    __shared__ __align__(8) uint64_t s_full[2];
+    __shared__ __align__(8) uint64_t s_mma[2];
+    __shared__ __align__(8) uint64_t s_raw[kTcRaw];
+    __shared__ __align__(8) uint64_t s_tfree;
     __shared__ uint32_t s_tmem;
-    __shared__ int s_src[2][kTcMaxN];  // B row of each token of pass P (parity P & 1)
+    __shared__ int s_abort;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int e = blockIdx.y;
     pdl_wait();
@@ -209,185 +240,195 @@ grouped_tc_kernel(const GroupedParams p, const __grid_constant__ CUtensorMap cod
     const uint32_t rs = (uint32_t)K >> 5;
     uint8_t *raw = sm + tc_raw_off(NMAT);
     uint8_t *scl = sm + tc_sc_off(NMAT);
+    // per token of the group: its B row (x row of the pair's token, or h row
+    // of the pair)
+    int *s_src = reinterpret_cast<int *>(sm + tc_src_off(NMAT, K));
 
-    if (warp == 0) {  // TMEM: NMAT x 256 FP32 columns x 128 lanes
+    if (warp == 0) {  // TMEM: NMAT x 128 FP32 columns x 128 lanes
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      ::"r"(smem_u32(&s_tmem)), "r"(NMAT * kTcMaxN)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid == 0) {
+        mbar_init(&s_full[0], kTcWork / 32);
+        mbar_init(&s_full[1], kTcWork / 32);
         mbar_init(&s_mma[0], 1);
         mbar_init(&s_mma[1], 1);
 #pragma unroll
         for (int j = 0; j < kTcRaw; ++j) mbar_init(&s_raw[j], 1);
+        mbar_init(&s_tfree, kTcWork / 32);
+        s_abort = 0;
         mbar_fence_init();
+    }
+    for (int i = tid; i < n_e; i += kTcThreads) {
+        const int pr = p.perm[seg0 + i];
+        s_src[i] = NMAT == 2 ? pr / p.k : pr;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s_tmem;
-    const uint64_t pol = l2_evict_first_policy();  // packed rows are read once
+    volatile int *abort = &s_abort;
 
-    // packed tile of iteration it (K tile it % nkt) into ring slot it % kTcRaw,
-    // by thread kTcTma (raw_next: loads issued so far, in iteration order)
-    int raw_next = 0;
-    auto issue_raw = [&](int it) {
-        raw_next = it + 1;
-        const int j = it % kTcRaw, kt = it % nkt;
-        mbar_arrive_expect_tx(&s_raw[j], (unsigned)(NMAT * kTcRawSlot));
-#pragma unroll
-        for (int m = 0; m < NMAT; ++m)
-            tma_load_3d(raw + ((uint32_t)j * NMAT + m) * kTcRawSlot, &codes_map, kt * 32, row0,
-                        3 * e + (NMAT == 2 ? m : 2), &s_raw[j], pol);
-    };
-    // B rows of iteration it (its pass's tokens, K tile kt) into ring slot it % kTcBSlots
-    auto issue_b = [&](int it) {
-        const int pass = it / nkt, kt = it % nkt;
-        const int tc = pass * kTcMaxN, nt = min(kTcMaxN, n_e - tc);
-        uint8_t *b = sm + tc_b_off(NMAT) + (uint32_t)(it % kTcBSlots) * kTcTileB;
-        const uint16_t *base = NMAT == 2 ? p.x : p.h;
-        for (int i = tid; i < nt * 8; i += kTcThreads) {
-            const int n = i >> 3, c = i & 7;
-            cp_async16_tc(b + tc_off(n, c), base + (size_t)s_src[pass & 1][n] * K + kt * kTcK + c * 8);
-        }
-    };
-    // the B rows (x row of the pair's token, or h row of the pair) of pass P's
-    // tokens into s_src[P & 1]
-    auto fill_src = [&](int P) {
-        const int tc = P * kTcMaxN;
-        if (tid < kTcMaxN && tc + tid < n_e) {
-            const int pr = p.perm[seg0 + tc + tid];
-            s_src[P & 1][tid] = NMAT == 2 ? pr / p.k : pr;
-        }
-    };
-
-    // prologue: the CTA's scale rows and B of iteration 0 (one copy group), B
-    // of iteration 1 (another), packed tiles 0 .. kTcRaw - 2
-    // this thread's row and K quarter (a warp covers 8 consecutive rows: its
-    // reads of the packed ring are contiguous)
-    const int rrow = tid >> 2, quarter = tid & 3;
-    fill_src(0);
-    if (npass > 1) fill_src(1);
-    __syncthreads();
-#pragma unroll
-    for (int m = 0; m < NMAT; ++m) {
-        const int mat = NMAT == 2 ? m : 2;
-        const uint8_t *gsc = tc_scales(p, e, mat) + (size_t)(row0 + rrow) * rs;
-        // K / 32 is a multiple of 4 (K % 128 == 0): the row's scales in 4-byte
-        // pieces, spread over its four threads
-        for (uint32_t c = 4 * quarter; c < rs; c += 16)
-            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
-                             smem_u32(scl + ((uint32_t)m * kTcM + rrow) * rs + c)),
-                         "l"(gsc + c)
+    if (warp == kTcWork / 32) {
+        // ---- MMA + TMA warp: lane 0 issues, the other lanes wait at the end ----
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&codes_map))
                          : "memory");
-    }
-    issue_b(0);
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    if (total > 1) issue_b(1);
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    if (tid == kTcTma) {
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&codes_map))
-                     : "memory");
-#pragma unroll 1
-        for (int j = 0; j < kTcRaw - 1 && j < total; ++j) issue_raw(j);
-    }
-
-    bool ok = true;
-    int issued = 0;  // iterations whose products were issued (uniform)
-    #pragma unroll 1
-    for (int it = 0; it < total; ++it) {
-        const int s = it & 1, pass = it / nkt, kt = it % nkt;
-        const int tc = pass * kTcMaxN, nt = min(kTcMaxN, n_e - tc);
-        // ring slot of iteration it - 1 was read by every thread before the
-        // barrier that ended it: refill it with tile it + kTcRaw - 1
-        if (tid == kTcTma && it + kTcRaw - 1 < total) issue_raw(it + kTcRaw - 1);
-        // the next pass's B rows, read from iteration (pass + 2) nkt - 2 on
-        if (kt == 0 && pass >= 1 && pass + 1 < npass) fill_src(pass + 1);
-        // A stage s and B slot (it + 2) % kTcBSlots were last read by the
-        // products of iteration it - 2
-        if (it >= 2 && !mbar_wait(&s_mma[s], (unsigned)((it - 2) >> 1) & 1u)) ok = false;
-        if (it + 2 < total) issue_b(it + 2);
-        // one group per iteration: all but the 2 newest = B of this iteration
-        // (and, at it = 0, the scale rows)
-        asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 2;" ::: "memory");
-        if (!mbar_wait(&s_raw[it % kTcRaw], (unsigned)(it / kTcRaw) & 1u)) ok = false;
-        // ---- dequantise this thread's part of tile kt into stage s ----
-        uint8_t *st = sm + (uint32_t)s * tc_stage_bytes(NMAT);
-        const uint8_t *slot = raw + (uint32_t)(it % kTcRaw) * NMAT * kTcRawSlot;
+            const uint64_t pol = l2_evict_first_policy();  // packed rows are read once
+            int raw_next = 0;
+            auto issue_raw = [&](int it) {
+                raw_next = it + 1;
+                const int j = it % kTcRaw, kt = it % nkt;
+                mbar_arrive_expect_tx(&s_raw[j], (unsigned)(NMAT * kTcRawSlot));
+#pragma unroll
+                for (int m = 0; m < NMAT; ++m)
+                    tma_load_3d(raw + ((uint32_t)j * NMAT + m) * kTcRawSlot, &codes_map, kt * 32,
+                                row0, 3 * e + (NMAT == 2 ? m : 2), &s_raw[j], pol);
+            };
+            for (int j = 0; j < kTcRaw && j < total; ++j) issue_raw(j);
+            int issued = 0;
+            #pragma unroll 1
+            for (int it = 0; it < total; ++it) {
+                const int s = it & 1, pass = it / nkt, kt = it % nkt;
+                const int nt = min(kTcMaxN, n_e - pass * kTcMaxN);
+                if (!tc_wait(&s_full[s], (unsigned)(it >> 1) & 1u, abort)) break;
+                // the first tile of a pass overwrites the accumulators: the
+                // previous pass's epilogue must have read them
+                if (kt == 0 && pass > 0 && !tc_wait(&s_tfree, (unsigned)(pass - 1) & 1u, abort))
+                    break;
+                tc_fence_after();
+                const uint32_t idesc = tc_idesc((nt + 15) & ~15);
+                const uint32_t b_addr =
+                    smem_u32(sm + tc_b_off(NMAT) + (uint32_t)(it % kTcBSlots) * kTcTileB);
+#pragma unroll
+                for (int m = 0; m < NMAT; ++m) {
+                    const uint32_t a_addr =
+                        smem_u32(sm + (uint32_t)s * tc_stage_bytes(NMAT) + (uint32_t)m * kTcTileA);
+#pragma unroll
+                    for (int kk = 0; kk < kTcK / 16; ++kk)
+                        tc_mma(tmem + (uint32_t)(m * kTcMaxN), tc_desc(a_addr + kk * 256),
+                               tc_desc(b_addr + kk * 256), idesc, kt > 0 || kk > 0);
+                }
+                tc_commit(&s_mma[s]);
+                issued = it + 1;
+                // ring slot it % kTcRaw was read by every conversion thread
+                // before its s_full arrival: refill it
+                if (it + kTcRaw < total) issue_raw(it + kTcRaw);
+            }
+            // nothing in flight at exit (bounded): the products issued, the
+            // last packed loads (one per ring slot; earlier ones were consumed)
+            if (issued > 0) mbar_wait(&s_mma[(issued - 1) & 1], (unsigned)((issued - 1) >> 1) & 1u);
+            for (int j = max(0, raw_next - kTcRaw); j < raw_next; ++j)
+                mbar_wait(&s_raw[j % kTcRaw], (unsigned)(j / kTcRaw) & 1u);
+        }
+        __syncwarp();
+    } else {
+        // ---- conversion warps ----
+        // this thread's row and K quarter (a warp covers 8 consecutive rows:
+        // its reads of the packed ring are contiguous)
+        const int rrow = tid >> 2, quarter = tid & 3;
 #pragma unroll
         for (int m = 0; m < NMAT; ++m) {
-            // K-chunks 2 q, 2 q + 1 of the row (8 code bytes; one scale group)
-            const uint2 cw = *reinterpret_cast<const uint2 *>(
-                slot + (uint32_t)m * kTcRawSlot + (uint32_t)rrow * 32 + 8 * quarter);
-            const float sf = e8m0_to_f32(scl[((uint32_t)m * kTcM + rrow) * rs + 2 * kt + (quarter >> 1)]);
-            uint8_t *a = st + (uint32_t)m * kTcTileA;
-            *reinterpret_cast<uint4 *>(a + tc_off(rrow, 2 * quarter)) = dequant8_bf16(cw.x, sf);
-            *reinterpret_cast<uint4 *>(a + tc_off(rrow, 2 * quarter + 1)) = dequant8_bf16(cw.y, sf);
+            const int mat = NMAT == 2 ? m : 2;
+            const uint8_t *gsc = tc_scales(p, e, mat) + (size_t)(row0 + rrow) * rs;
+            // K / 32 is a multiple of 4 (K % 128 == 0): the row's scales in
+            // 4-byte pieces, spread over its four threads
+            for (uint32_t c = 4 * quarter; c < rs; c += 16)
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
+                                 smem_u32(scl + ((uint32_t)m * kTcM + rrow) * rs + c)),
+                             "l"(gsc + c)
+                             : "memory");
         }
-        fence_async_shared();
-        ok = __syncthreads_and(ok) != 0;  // every thread's A and B writes
-        if (!ok) break;  // uniform; every copy and product is drained below
-        if (tid == 0) {
-            tc_fence_after();
-            const int N = (nt + 15) & ~15;
-            const uint32_t idesc = tc_idesc(N);
-            const uint32_t b_addr =
-                smem_u32(sm + tc_b_off(NMAT) + (uint32_t)(it % kTcBSlots) * kTcTileB);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        // B rows of iteration it (its pass's tokens, K tile kt) into ring
+        // slot it % kTcBSlots
+        const uint16_t *bbase = NMAT == 2 ? p.x : p.h;
+        auto issue_b = [&](int it) {
+            const int pass = it / nkt, kt = it % nkt;
+            const int tc = pass * kTcMaxN, nt = min(kTcMaxN, n_e - tc);
+            uint8_t *b = sm + tc_b_off(NMAT) + (uint32_t)(it % kTcBSlots) * kTcTileB;
+            for (int i = tid; i < nt * 8; i += kTcWork) {
+                const int n = i >> 3, c = i & 7;
+                cp_async16_tc(b + tc_off(n, c), bbase + (size_t)s_src[tc + n] * K + kt * kTcK + c * 8);
+            }
+        };
+        // copy groups: {scales}, {B(0)}, {B(1)}, then one per iteration
+        issue_b(0);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        if (total > 1) issue_b(1);
+        asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 2;" ::: "memory");
+        // every row's scale bytes (copied by its four threads) visible to all
+        conv_sync();
+        #pragma unroll 1
+        for (int it = 0; it < total; ++it) {
+            const int s = it & 1, pass = it / nkt, kt = it % nkt;
+            const int tc = pass * kTcMaxN, nt = min(kTcMaxN, n_e - tc);
+            // A stage s and B slot (it + 2) % kTcBSlots were last read by the
+            // products of iteration it - 2
+            bool ok = it < 2 || tc_wait(&s_mma[s], (unsigned)((it - 2) >> 1) & 1u, abort);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            if (it + 2 < total) issue_b(it + 2);
+            // all but the 2 newest groups: B of this iteration
+            asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 2;" ::: "memory");
+            ok = tc_wait(&s_raw[it % kTcRaw], (unsigned)(it / kTcRaw) & 1u, abort);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            // ---- dequantise this thread's part of tile kt into stage s ----
+            uint8_t *st = sm + (uint32_t)s * tc_stage_bytes(NMAT);
+            const uint8_t *slot = raw + (uint32_t)(it % kTcRaw) * NMAT * kTcRawSlot;
 #pragma unroll
             for (int m = 0; m < NMAT; ++m) {
-                const uint32_t a_addr = smem_u32(st + (uint32_t)m * kTcTileA);
-#pragma unroll
-                for (int kk = 0; kk < kTcK / 16; ++kk)
-                    tc_mma(tmem + (uint32_t)(m * kTcMaxN), tc_desc(a_addr + kk * 256),
-                           tc_desc(b_addr + kk * 256), idesc, kt > 0 || kk > 0);
+                // K-chunks 2 q, 2 q + 1 of the row (8 code bytes; one scale group)
+                const uint2 cw = *reinterpret_cast<const uint2 *>(
+                    slot + (uint32_t)m * kTcRawSlot + (uint32_t)rrow * 32 + 8 * quarter);
+                const float sf = e8m0_to_f32(scl[((uint32_t)m * kTcM + rrow) * rs + 2 * kt + (quarter >> 1)]);
+                uint8_t *a = st + (uint32_t)m * kTcTileA;
+                *reinterpret_cast<uint4 *>(a + tc_off(rrow, 2 * quarter)) = dequant8_bf16(cw.x, sf);
+                *reinterpret_cast<uint4 *>(a + tc_off(rrow, 2 * quarter + 1)) = dequant8_bf16(cw.y, sf);
             }
-            tc_commit(&s_mma[s]);
-        }
-        issued = it + 1;
-        if (kt == nkt - 1) {
-            // ---- epilogue of this pass: accumulators -> outputs ----
-            if (!mbar_wait(&s_mma[s], (unsigned)(it >> 1) & 1u)) ok = false;
-            tc_fence_after();
-            const int lq = warp & 3;                // TMEM lane quarter of this warp
-            const int r = row0 + lq * 32 + lane;    // this thread's matrix row
-            const uint32_t lane_base = tmem + ((uint32_t)(lq * 32) << 16);
-            const int N = (nt + 15) & ~15;
-            #pragma unroll 1
-            for (int c0 = 8 * (warp >> 2); c0 < N; c0 += 32) {
-                float g[8], u[8];
-                tc_ld8(lane_base + (uint32_t)c0, g);
-                if (NMAT == 2) tc_ld8(lane_base + (uint32_t)(kTcMaxN + c0), u);
+            fence_async_shared();  // this thread's A and B writes -> the tensor core
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_full[s]);
+            if (kt == nkt - 1) {
+                // ---- epilogue of this pass: accumulators -> outputs ----
+                ok = tc_wait(&s_mma[s], (unsigned)(it >> 1) & 1u, abort);
+                if (!__all_sync(0xffffffffu, ok)) break;
+                tc_fence_after();
+                const int lq = warp & 3;           // TMEM lane quarter of this warp
+                const int r = row0 + lq * 32 + lane;  // this thread's matrix row
+                const uint32_t lane_base = tmem + ((uint32_t)(lq * 32) << 16);
+                const int N = (nt + 15) & ~15;
+                #pragma unroll 1
+                for (int c0 = 8 * (warp >> 2); c0 < N; c0 += 32) {
+                    float g[8], u[8];
+                    tc_ld8(lane_base + (uint32_t)c0, g);
+                    if (NMAT == 2) tc_ld8(lane_base + (uint32_t)(kTcMaxN + c0), u);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int idx = tc + c0 + j;
-                    if (!ok || idx >= tc + nt) continue;
-                    const int pr = p.perm[seg0 + idx];
-                    if (NMAT == 2) {
-                        const float gv = round_bf16(g[j]);
-                        const float uv = round_bf16(u[j]);
-                        const float sl = round_bf16(gv / (1.0f + expf(-gv)));
-                        p.h[(size_t)pr * M + r] = f32_to_bf16(sl * uv);
-                    } else {
-                        p.o[(size_t)pr * M + r] = f32_to_bf16(g[j]);
+                    for (int j = 0; j < 8; ++j) {
+                        const int idx = tc + c0 + j;
+                        if (idx >= tc + nt) continue;
+                        const int pr = p.perm[seg0 + idx];
+                        if (NMAT == 2) {
+                            const float gv = round_bf16(g[j]);
+                            const float uv = round_bf16(u[j]);
+                            const float sl = round_bf16(gv / (1.0f + expf(-gv)));
+                            p.h[(size_t)pr * M + r] = f32_to_bf16(sl * uv);
+                        } else {
+                            p.o[(size_t)pr * M + r] = f32_to_bf16(g[j]);
+                        }
                     }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_tfree);
             }
-            tc_fence_before();
-            ok = __syncthreads_and(ok) != 0;  // TMEM read before the next pass overwrites it
-            if (!ok) break;
         }
+        asm volatile("cp.async.wait_all;" ::: "memory");  // no copy in flight at exit
     }
-    if (!ok && tid == 0) atomicOr(p.status, kTimeoutStatus);
-    // nothing in flight at exit (bounded waits): this thread's copies, the
-    // products issued, the packed tiles issued
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    if (issued > 0) mbar_wait(&s_mma[(issued - 1) & 1], (unsigned)((issued - 1) >> 1) & 1u);
-    if (tid == kTcTma)  // the last loads issued, one per ring slot (earlier ones were consumed)
-        for (int j = max(0, raw_next - kTcRaw); j < raw_next; ++j)
-            mbar_wait(&s_raw[j % kTcRaw], (unsigned)(j / kTcRaw) & 1u);
     tc_fence_before();
     __syncthreads();
+    if (tid == 0 && s_abort) atomicOr(p.status, kTimeoutStatus);
     if (warp == 0) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
@@ -447,7 +488,7 @@ cudaError_t codes_map(CodesMap &c, const uint8_t *base, size_t matrix_stride, in
 template <int NMAT>
 cudaError_t launch_tc(const GroupedParams &p, const CUtensorMap &map, cudaStream_t s, bool pdl) {
     const int K = NMAT == 2 ? p.H : p.I, M = NMAT == 2 ? p.I : p.H;
-    const size_t smem = tc_smem_bytes(NMAT, K);
+    const size_t smem = tc_smem_bytes(NMAT, K, p.T * p.k);
     static size_t attr_smem = 0;  // largest dynamic shared memory enabled so far
     if (smem > attr_smem) {
         cudaError_t e = cudaFuncSetAttribute(grouped_tc_kernel<NMAT>,
@@ -463,11 +504,11 @@ cudaError_t launch_tc(const GroupedParams &p, const CUtensorMap &map, cudaStream
 }  // namespace
 
 // The tensor-core products need the contiguous weight layout (one tensor map
-// per matrix kind), H and I multiples of 128 and the shared-memory plan
-// within the budget.
-bool grouped_tc_supported(int H, int I) {
-    return H % 128 == 0 && I % 128 == 0 && tc_smem_bytes(2, H) <= 220 * 1024 &&
-           tc_smem_bytes(1, I) <= 220 * 1024;
+// per matrix kind), H and I multiples of 128 and the shared-memory plan of a
+// launch of `pairs` (token, slot) pairs within the budget.
+bool grouped_tc_supported(int H, int I, int pairs) {
+    return H % 128 == 0 && I % 128 == 0 && tc_smem_bytes(2, H, pairs) <= 220 * 1024 &&
+           tc_smem_bytes(1, I, pairs) <= 220 * 1024;
 }
 
 cudaError_t launch_grouped_tc_gateup(const GroupedParams &p, cudaStream_t s, bool pdl) {

@@ -143,9 +143,11 @@ struct GroupedParams {
 };
 bool grouped_supported(int E, int H, int I);
 cudaError_t launch_grouped(const GroupedParams &p, cudaStream_t s, bool pdl);
-// Products on tcgen05 (grouped_tc.cu), on request: measured slower than the
-// mma.sync tiles at every batch tried (T <= 1024, 24B shape).
-bool grouped_tc_supported(int H, int I);
+// Products on tcgen05 (grouped_tc.cu): chosen by the forward when the groups
+// average at least kTcAutoGroup pairs (the mma.sync tiles convert the codes
+// again for every 8 tokens, the tcgen05 CTAs once per 128), or on request.
+constexpr int kTcAutoGroup = 40;
+bool grouped_tc_supported(int H, int I, int pairs);
 cudaError_t launch_grouped_tc_gateup(const GroupedParams &p, cudaStream_t s, bool pdl);
 cudaError_t launch_grouped_tc_down(const GroupedParams &p, cudaStream_t s, bool pdl);
 

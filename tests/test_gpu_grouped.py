@@ -120,6 +120,41 @@ def test_grouped_tcgen05_is_deterministic_and_needs_contiguous_weights():
         moe.moe_destroy(h)
 
 
+def test_grouped_tcgen05_wide_scale_span_rows():
+    """Rows whose E8M0 exponents span 23, 24 and 30 binades (a group far
+    below the row's largest): the BF16 weight tiles hold every code x scale
+    exactly, so h, o, y still meet the oracle."""
+    shape = synth.TINY
+    T = 200
+    L = synth.make_layer(shape, seed=82)
+    H, I = shape.H, shape.I
+    mat = I * H // 32  # scales of one matrix
+
+    def put(e, m, r, g, v):
+        K = H if m < 2 else I
+        L.scales[e, m * mat + r * (K // 32) + g] = v
+
+    hi = synth.E8M0_HI
+    put(3, 0, 5, 0, hi)
+    put(3, 0, 5, 1, hi - 30)        # gate row 5 of expert 3: span 30
+    put(7, 2, 200, 0, hi)
+    put(7, 2, 200, 2, hi - 24)      # down row 200 of expert 7: span 24
+    put(5, 1, 70, 3, hi)
+    put(5, 1, 70, 4, hi - 23)       # up row 70 of expert 5: span 23
+    put(11, 2, 3, 0, hi)
+    put(11, 2, 3, 1, hi - 23)       # down row 3 of expert 11: span 23
+    codes, scales, rw, rb = dev_layer(L)
+    layer = moe.MoELayer(shape.E, shape.H, shape.I, shape.top_k, codes, scales, rw, rb,
+                         max_tokens=T)
+    x = synth.make_tokens(T, shape.H, seed=82)
+    ids, w = synth.make_routing(T, shape.E, shape.top_k, "uniform", synth.rng_for(82, 13, T))
+    for e in (3, 5, 7, 11):
+        assert (ids == e).any()
+    _check(L, layer, x, ids, w, shape, flags=moe.FWD_FORCE_TCGEN05)
+    assert layer.status() == 0
+    layer.close()
+
+
 def test_grouped_residual_and_determinism():
     shape = synth.L24B
     L, layer, x, ids, w = _setup(shape, 72, 24, "zipf")
@@ -142,16 +177,39 @@ def test_grouped_one_expert_takes_every_token():
 
 @pytest.mark.parametrize("T", [150])
 def test_grouped_one_expert_group_beyond_one_pass(T):
-    """Groups of T = 150 tokens: three 64-token passes of the tcgen05 products
-    (and 19 chunks of the mma.sync tiles)."""
+    """Groups of T = 150 tokens: two token passes (128 + 22) of the tcgen05
+    products (and 19 chunks of the mma.sync tiles)."""
     shape = synth.TINY
     L, layer, x, _, w = _setup(shape, 78, T, "uniform")
     ids = np.tile(np.array([[5, 2, 9, 14]], dtype=np.int32), (T, 1))
-    y_mma = _check(L, layer, x, ids, w, shape)
+    y_mma = _check(L, layer, x, ids, w, shape, flags=moe.FWD_FORCE_MMA)
     y_tc = _check(L, layer, x, ids, w, shape, flags=moe.FWD_FORCE_TCGEN05)
     assert_close_rms(y_tc, y_mma, what="tcgen05 vs mma.sync", max_ulps=4)
     assert layer.status() == 0
     layer.close()
+
+
+@pytest.mark.parametrize("shape", [synth.TINY, synth.L24B])
+def test_grouped_product_choice_follows_group_size(shape):
+    """Without a forcing flag the products run on tcgen05 exactly when the
+    groups average at least 40 (token, slot) pairs (T k >= 40 E), else on the
+    mma.sync tiles: the default call gives the bits of the forced one on each
+    side of the threshold.  The two forcing flags exclude each other and the
+    per-(token, slot) path."""
+    t_min = 40 * shape.E // shape.top_k
+    for T, forced in ((t_min, moe.FWD_FORCE_TCGEN05), (t_min - 1, moe.FWD_FORCE_MMA)):
+        L, layer, x, ids, w = _setup(shape, 81, T, "zipf")
+        args = (dev_bf16(x), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda())
+        y0 = host_bf16(layer.forward(*args, flags=0)).copy()
+        y1 = host_bf16(layer.forward(*args, flags=forced)).copy()
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(y0, y1)
+        assert layer.status() == 0
+        for bad in (moe.FWD_FORCE_MMA | moe.FWD_FORCE_TCGEN05,
+                    moe.FWD_FORCE_MMA | moe.FWD_FORCE_DECODE):
+            with pytest.raises(moe.MoEError):
+                layer.forward(*args, flags=bad)
+        layer.close()
 
 
 def test_grouped_more_tokens_than_one_launch_sequence():
