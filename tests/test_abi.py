@@ -98,6 +98,30 @@ def test_calls_fail_cleanly_without_weights_or_device(lib):
     lib.moe_destroy(h)
 
 
+def test_forward_flags_are_validated_on_the_host(lib):
+    """Flag combinations that exclude each other, unknown bits and a forced
+    tcgen05 path without contiguous weights are refused (MOE_ERR_ARG) before
+    any device work; a valid combination gets as far as the missing weights
+    (MOE_ERR_NOT_LOADED)."""
+    from packed_mxfp4_w4a16_b200 import (FWD_FORCE_DECODE, FWD_FORCE_GROUPED, FWD_FORCE_MMA,
+                                         FWD_FORCE_TCGEN05, FWD_PHASE_DOWN, FWD_PHASE_GATEUP)
+    h = C.c_void_p()
+    assert lib.moe_create(64, 2048, 1536, 4, C.byref(h)) == 0
+    try:
+        def fwd(flags, T=64):
+            return lib.moe_forward_ex(h, None, T, None, None, None, None, flags, None)
+        for bad in (0x80, 1 << 31, FWD_FORCE_MMA | FWD_FORCE_TCGEN05,
+                    FWD_FORCE_MMA | FWD_FORCE_DECODE, FWD_FORCE_TCGEN05 | FWD_FORCE_DECODE,
+                    FWD_FORCE_DECODE | FWD_FORCE_GROUPED, FWD_PHASE_GATEUP | FWD_PHASE_DOWN,
+                    FWD_FORCE_TCGEN05):  # no contiguous weights bound
+            assert fwd(bad) == -1, hex(bad)
+        assert fwd(0, T=0) == -1
+        for good in (0, FWD_FORCE_MMA, FWD_FORCE_GROUPED, FWD_FORCE_DECODE, FWD_PHASE_GATEUP):
+            assert fwd(good) == -2, hex(good)
+    finally:
+        lib.moe_destroy(h)
+
+
 def test_status_strings(lib):
     for code in range(-8, 1):
         s = lib.moe_status_string(code).decode()
