@@ -349,9 +349,15 @@ grouped_tc_kernel(const GroupedParams p, const __grid_constant__ CUtensorMap cod
             const int pass = it / nkt, kt = it % nkt;
             const int tc = pass * kTcMaxN, nt = min(kTcMaxN, n_e - tc);
             uint8_t *b = sm + tc_b_off(NMAT) + (uint32_t)(it % kTcBSlots) * kTcTileB;
-            for (int i = tid; i < nt * 8; i += kTcWork) {
-                const int n = i >> 3, c = i & 7;
-                cp_async16_tc(b + tc_off(n, c), bbase + (size_t)s_src[tc + n] * K + kt * kTcK + c * 8);
+            // 64 consecutive i cover 8 rows x 8 chunks, row fastest: the 8
+            // lanes of each shared-memory phase write 8 different rows of a
+            // core matrix (distinct banks); each row gets 64 contiguous bytes
+            // per warp from global memory
+            for (int i = tid; i < ((nt + 7) & ~7) * 8; i += kTcWork) {
+                const int n = ((i >> 6) << 3) | (i & 7), c = (i >> 3) & 7;
+                if (n < nt)
+                    cp_async16_tc(b + tc_off(n, c),
+                                  bbase + (size_t)s_src[tc + n] * K + kt * kTcK + c * 8);
             }
         };
         // copy groups: {scales}, {B(0)}, {B(1)}, then one per iteration
