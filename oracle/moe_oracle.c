@@ -26,6 +26,9 @@
  *         weight-only build): sections "What's quantized to what" (routed
  *         experts in NVFP4, compute in 16-bit; format nvfp4-pack-quantized;
  *         w1 and w3 of each expert share one global scale).
+ *   [CA]  "LFM2.5-8B-A1B — Core AI (.aimodel)": table "Provenance", row
+ *         "Weight format" (sym8: symmetric-linear int8 with one scale per
+ *         block of 32 along K, read through a gather matvec kernel).
  *   [BW]  "LFM2.5-24B-A2B on Your Own Hardware: The RAM, KV Cache and
  *         Bandwidth Budget": section "Where do the 2.45B active parameters
  *         actually go?" (SwiGLU expert = gate, up, down; H=2048, I=1536).
@@ -56,6 +59,10 @@
  *     subnormal, S.1111.111 NaN, no infinity); one FP32 multiplier per
  *     expert shared by gate and up and one for down (gscales [E][2]);
  *     w = e2m1(c) * e4m3(s) * g.
+ *   - sym8 ([CA] names the format only): one two's-complement int8 q per
+ *     weight (codes [E][3][rows][K], one byte each), one IEEE binary16
+ *     scale per 32 consecutive K elements (scales [E][3][rows][K/32] as
+ *     little-endian 16-bit words); symmetric, so no zero point: w = q * s.
  */
 #include <math.h>
 #include <stddef.h>
@@ -151,6 +158,39 @@ static double weight_at_nv(const uint8_t *row_codes, const uint8_t *row_scales,
     uint8_t byte = row_codes[j >> 1];
     unsigned nib = (j & 1) ? (unsigned)(byte >> 4) : (unsigned)(byte & 0x0F);
     return oracle_e2m1_value(nib) * oracle_e4m3_value(row_scales[j >> 4]) * gscale;
+}
+
+/* IEEE 754 binary16 value of the 16-bit pattern b (the sym8 block scale):
+ * sign, 5 exponent bits with bias 15, 10 mantissa bits, exponent 0
+ * subnormal, exponent 31 infinity or NaN. */
+double oracle_f16_value(unsigned b)
+{
+    unsigned sign = (b >> 15) & 1u, ex = (b >> 10) & 31u, man = b & 1023u;
+    double m;
+    if (ex == 31u)
+        m = man ? NAN : INFINITY;
+    else if (ex == 0u)
+        m = ldexp((double)man, -24);               /* subnormal */
+    else
+        m = ldexp(1.0 + (double)man / 1024.0, (int)ex - 15);
+    return sign ? -m : m;
+}
+
+/* [CA] sym8 weight element j of a row: the signed byte q_j times the
+ * binary16 scale of its 32-element block (no zero point). */
+static double weight_at_s8(const uint8_t *row_q, const uint8_t *row_scales, int64_t j)
+{
+    int q = (int)(int8_t)row_q[j];
+    const uint8_t *s = row_scales + 2 * (j >> 5);
+    return (double)q * oracle_f16_value((unsigned)s[0] | ((unsigned)s[1] << 8));
+}
+
+/* sym8 dequantisation of n consecutive elements (n a multiple of 32);
+ * scales: the little-endian binary16 words as bytes. */
+void oracle_dequant_sym8(const uint8_t *q, const uint8_t *scales, int64_t n, double *out)
+{
+    for (int64_t j = 0; j < n; ++j)
+        out[j] = weight_at_s8(q, scales, j);
 }
 
 /* NVFP4 dequantisation of n consecutive elements (n a multiple of 16). */
@@ -300,22 +340,46 @@ void oracle_route_sigmoid(const uint16_t *x, int T, int H, const uint16_t *Wr,
 
 static double silu(double g) { return g / (1.0 + exp(-g)); }
 
-/* One SwiGLU expert on one BF16 activation vector, for either weight format.
+/* Weight formats of the expert matrices. */
+enum { FMT_MXFP4 = 0, FMT_NVFP4 = 1, FMT_SYM8 = 2 };
+
+/* Bytes of one row of K weights: codes, and block scales. */
+static size_t row_code_bytes(int fmt, int K) { return fmt == FMT_SYM8 ? (size_t)K : (size_t)K / 2; }
+static size_t row_scale_bytes(int fmt, int K)
+{
+    return fmt == FMT_NVFP4 ? (size_t)K / 16 : fmt == FMT_SYM8 ? (size_t)K / 16 : (size_t)K / 32;
+}
+
+/* Weight element j of a row in format fmt (g: the NVFP4 multiplier). */
+static double weight_fmt(int fmt, const uint8_t *rc, const uint8_t *rs, double g, int64_t j)
+{
+    if (fmt == FMT_NVFP4)
+        return weight_at_nv(rc, rs, g, j);
+    if (fmt == FMT_SYM8)
+        return weight_at_s8(rc, rs, j);
+    return weight_at(rc, rs, j);
+}
+
+/* One SwiGLU expert on one BF16 activation vector, for any weight format.
  * [MC] "Grouped top-4 expert execution": gate projection, up projection,
  * activation and multiplication, down projection; "Model and quantization":
  * accumulation wider than BF16, BF16 outputs.  [BW]: the expert is the three
  * matrices gate, up (I x H) and down (H x I).
- *   nv = 0 (MXFP4): codes_e / scales_e: this expert's [3][rows][K/2] /
+ *   FMT_MXFP4: codes_e / scales_e: this expert's [3][rows][K/2] /
  *     [3][rows][K/32], gs ignored.
- *   nv = 1 (NVFP4): scales_e [3][rows][K/16] E4M3, gs[0] multiplies gate and
- *     up, gs[1] down.
+ *   FMT_NVFP4: scales_e [3][rows][K/16] E4M3, gs[0] multiplies gate and up,
+ *     gs[1] down.
+ *   FMT_SYM8: codes_e [3][rows][K] int8, scales_e [3][rows][K/32] binary16
+ *     (2 bytes each), gs ignored.
  *   h_out (nullable): the BF16 SwiGLU output [I].  o_out: BF16 [H]. */
 static void expert_any(const uint16_t *x, const uint8_t *codes_e,
-                       const uint8_t *scales_e, const float *gs, int nv,
+                       const uint8_t *scales_e, const float *gs, int fmt,
                        int H, int I, uint16_t *h_out, uint16_t *o_out)
 {
-    const int sdiv = nv ? 16 : 32;  /* K elements per scale */
-    const size_t mc = (size_t)I * H / 2, ms = (size_t)I * H / (size_t)sdiv;
+    const int nv = fmt == FMT_NVFP4;
+    const size_t rcH = row_code_bytes(fmt, H), rsH = row_scale_bytes(fmt, H);
+    const size_t rcI = row_code_bytes(fmt, I), rsI = row_scale_bytes(fmt, I);
+    const size_t mc = (size_t)I * rcH, ms = (size_t)I * rsH;  /* one matrix */
     const uint8_t *gate_c = codes_e, *up_c = codes_e + mc, *down_c = codes_e + 2 * mc;
     const uint8_t *gate_s = scales_e, *up_s = scales_e + ms, *down_s = scales_e + 2 * ms;
     const double g_gu = nv ? (double)gs[0] : 1.0, g_dn = nv ? (double)gs[1] : 1.0;
@@ -323,18 +387,13 @@ static void expert_any(const uint16_t *x, const uint8_t *codes_e,
 
 #pragma omp parallel for schedule(static)
     for (int i = 0; i < I; ++i) {
-        const uint8_t *gc = gate_c + (size_t)i * (H / 2), *gsc = gate_s + (size_t)i * (H / sdiv);
-        const uint8_t *uc = up_c + (size_t)i * (H / 2), *usc = up_s + (size_t)i * (H / sdiv);
+        const uint8_t *gc = gate_c + (size_t)i * rcH, *gsc = gate_s + (size_t)i * rsH;
+        const uint8_t *uc = up_c + (size_t)i * rcH, *usc = up_s + (size_t)i * rsH;
         double g = 0.0, u = 0.0;
         for (int j = 0; j < H; ++j) {
             double xv = oracle_bf16_to_double(x[j]);
-            if (nv) {
-                g += weight_at_nv(gc, gsc, g_gu, j) * xv;
-                u += weight_at_nv(uc, usc, g_gu, j) * xv;
-            } else {
-                g += weight_at(gc, gsc, j) * xv;
-                u += weight_at(uc, usc, j) * xv;
-            }
+            g += weight_fmt(fmt, gc, gsc, g_gu, j) * xv;
+            u += weight_fmt(fmt, uc, usc, g_gu, j) * xv;
         }
         double gb = oracle_bf16_to_double(oracle_bf16_from_double(g));
         double ub = oracle_bf16_to_double(oracle_bf16_from_double(u));
@@ -344,10 +403,10 @@ static void expert_any(const uint16_t *x, const uint8_t *codes_e,
 
 #pragma omp parallel for schedule(static)
     for (int n = 0; n < H; ++n) {
-        const uint8_t *dc = down_c + (size_t)n * (I / 2), *ds = down_s + (size_t)n * (I / sdiv);
+        const uint8_t *dc = down_c + (size_t)n * rcI, *ds = down_s + (size_t)n * rsI;
         double o = 0.0;
         for (int j = 0; j < I; ++j) {
-            double wv = nv ? weight_at_nv(dc, ds, g_dn, j) : weight_at(dc, ds, j);
+            double wv = weight_fmt(fmt, dc, ds, g_dn, j);
             o += wv * oracle_bf16_to_double(hb[j]);
         }
         o_out[n] = oracle_bf16_from_double(o);
@@ -362,7 +421,7 @@ void oracle_expert(const uint16_t *x, const uint8_t *codes_e,
                    const uint8_t *scales_e, int H, int I, uint16_t *h_out,
                    uint16_t *o_out)
 {
-    expert_any(x, codes_e, scales_e, NULL, 0, H, I, h_out, o_out);
+    expert_any(x, codes_e, scales_e, NULL, FMT_MXFP4, H, I, h_out, o_out);
 }
 
 /* One NVFP4 expert: gs = {gate/up multiplier, down multiplier}. */
@@ -370,7 +429,16 @@ void oracle_expert_nvfp4(const uint16_t *x, const uint8_t *codes_e,
                          const uint8_t *scales_e, const float *gs, int H, int I,
                          uint16_t *h_out, uint16_t *o_out)
 {
-    expert_any(x, codes_e, scales_e, gs, 1, H, I, h_out, o_out);
+    expert_any(x, codes_e, scales_e, gs, FMT_NVFP4, H, I, h_out, o_out);
+}
+
+/* One sym8 expert: codes_e [3][rows][K] int8, scales_e [3][rows][K/32]
+ * binary16 words (as bytes). */
+void oracle_expert_sym8(const uint16_t *x, const uint8_t *codes_e,
+                        const uint8_t *scales_e, int H, int I, uint16_t *h_out,
+                        uint16_t *o_out)
+{
+    expert_any(x, codes_e, scales_e, NULL, FMT_SYM8, H, I, h_out, o_out);
 }
 
 /* ------------------------------------------------------------- combine -- */
@@ -400,20 +468,24 @@ void oracle_combine(const uint16_t *o, const double *w, int k, int H,
 
 /* ---------------------------------------------------------- MoE layer -- */
 
-/* Experts + combine for T tokens with given routing, either weight format.
- *   x [T][H], ids [T][k], w [T][k] (double), codes [E][3*I*H/2],
+/* Experts + combine for T tokens with given routing, any weight format.
+ *   x [T][H], ids [T][k], w [T][k] (double); codes [E][3*I*H/2] with
  *   scales [E][3*I*H/32] (MXFP4) or [E][3*I*H/16] (NVFP4, with gscales
- *   [E][2]), residual [T][H] or NULL, y [T][H], o_out (nullable)
+ *   [E][2]), or codes [E][3*I*H] int8 with scales [E][3*I*H/32] binary16
+ *   words (sym8); residual [T][H] or NULL, y [T][H], o_out (nullable)
  *   [T][k][H], h_out (nullable) [T][k][I].
  * An id outside [0, E) gives a zero expert output for that slot. */
 static void moe_forward_any(const uint16_t *x, int T, int E, int H, int I, int k,
                             const int32_t *ids, const double *w,
                             const uint8_t *codes, const uint8_t *scales,
-                            const float *gscales, int nv,
+                            const float *gscales, int fmt,
                             const uint16_t *residual, uint16_t *y,
                             uint16_t *o_out, uint16_t *h_out)
 {
-    const size_t ce = (size_t)3 * I * H / 2, se = (size_t)3 * I * H / (nv ? 16 : 32);
+    /* bytes of one expert: three matrices of I x H weights */
+    const size_t ce = (size_t)3 * I * row_code_bytes(fmt, H);
+    const size_t se = (size_t)3 * I * row_scale_bytes(fmt, H);
+    const int nv = fmt == FMT_NVFP4;
     uint16_t *o = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)k * H);
     for (int t = 0; t < T; ++t) {
         for (int j = 0; j < k; ++j) {
@@ -426,7 +498,7 @@ static void moe_forward_any(const uint16_t *x, int T, int E, int H, int I, int k
                 continue;
             }
             expert_any(x + (size_t)t * H, codes + (size_t)e * ce, scales + (size_t)e * se,
-                       nv ? gscales + (size_t)e * 2 : NULL, nv, H, I, hj,
+                       nv ? gscales + (size_t)e * 2 : NULL, fmt, H, I, hj,
                        o + (size_t)j * H);
         }
         if (o_out)
@@ -444,7 +516,7 @@ void oracle_moe_forward(const uint16_t *x, int T, int E, int H, int I, int k,
                         const uint16_t *residual, uint16_t *y,
                         uint16_t *o_out, uint16_t *h_out)
 {
-    moe_forward_any(x, T, E, H, I, k, ids, w, codes, scales, NULL, 0, residual, y,
+    moe_forward_any(x, T, E, H, I, k, ids, w, codes, scales, NULL, FMT_MXFP4, residual, y,
                     o_out, h_out);
 }
 
@@ -454,7 +526,17 @@ void oracle_moe_forward_nvfp4(const uint16_t *x, int T, int E, int H, int I, int
                               const float *gscales, const uint16_t *residual,
                               uint16_t *y, uint16_t *o_out, uint16_t *h_out)
 {
-    moe_forward_any(x, T, E, H, I, k, ids, w, codes, scales, gscales, 1, residual, y,
+    moe_forward_any(x, T, E, H, I, k, ids, w, codes, scales, gscales, FMT_NVFP4, residual, y,
+                    o_out, h_out);
+}
+
+void oracle_moe_forward_sym8(const uint16_t *x, int T, int E, int H, int I, int k,
+                             const int32_t *ids, const double *w,
+                             const uint8_t *codes, const uint8_t *scales,
+                             const uint16_t *residual, uint16_t *y, uint16_t *o_out,
+                             uint16_t *h_out)
+{
+    moe_forward_any(x, T, E, H, I, k, ids, w, codes, scales, NULL, FMT_SYM8, residual, y,
                     o_out, h_out);
 }
 

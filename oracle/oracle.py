@@ -43,6 +43,12 @@ def _declare(L):
     L.oracle_expert_nvfp4.argtypes = [vp, vp, vp, vp, i32, i32, vp, vp]
     L.oracle_moe_forward_nvfp4.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp, vp,
                                            vp, vp, vp, vp, vp, vp]
+    L.oracle_f16_value.argtypes = [C.c_uint]
+    L.oracle_f16_value.restype = dbl
+    L.oracle_dequant_sym8.argtypes = [vp, vp, i64, vp]
+    L.oracle_expert_sym8.argtypes = [vp, vp, vp, i32, i32, vp, vp]
+    L.oracle_moe_forward_sym8.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp, vp,
+                                          vp, vp, vp, vp, vp]
     L.oracle_dequant.argtypes = [vp, vp, i64, vp]
     L.oracle_dequant_f32.argtypes = [vp, vp, i64, vp]
     L.oracle_select_topk.argtypes = [vp, i32, i32, vp, vp]
@@ -62,6 +68,7 @@ def _declare(L):
                  "oracle_select_topk_sigmoid", "oracle_route", "oracle_route_sigmoid",
                  "oracle_expert", "oracle_combine", "oracle_moe_forward", "oracle_moe_layer",
                  "oracle_dequant_nvfp4", "oracle_expert_nvfp4", "oracle_moe_forward_nvfp4",
+                 "oracle_dequant_sym8", "oracle_expert_sym8", "oracle_moe_forward_sym8",
                  "oracle_rmsnorm",
                  "oracle_stack_step"):
         getattr(L, name).restype = None
@@ -110,6 +117,11 @@ def e4m3_value(b: int) -> float:
     return lib().oracle_e4m3_value(int(b))
 
 
+def f16_value(b: int) -> float:
+    """IEEE binary16 bit pattern -> value (sym8 block scales)."""
+    return lib().oracle_f16_value(int(b))
+
+
 def bf16_from_f64_array(v: np.ndarray) -> np.ndarray:
     f = lib().oracle_bf16_from_double
     flat = np.asarray(v, dtype=np.float64).ravel()
@@ -145,6 +157,16 @@ def dequant_nvfp4(codes: np.ndarray, scales: np.ndarray, gscale: float, n: int) 
     assert n % 16 == 0 and codes.size >= n // 2 and scales.size >= n // 16
     out = np.empty(n, dtype=np.float64)
     lib().oracle_dequant_nvfp4(_p(codes), _p(scales), float(gscale), n, _p(out))
+    return out
+
+
+def dequant_sym8(q: np.ndarray, scales: np.ndarray, n: int) -> np.ndarray:
+    """sym8: int8 q x binary16 scale per 32 (scales as uint16 words)."""
+    q = _c(np.asarray(q).view(np.uint8), np.uint8)
+    scales = _c(scales, np.uint16)
+    assert n % 32 == 0 and q.size >= n and scales.size >= n // 32
+    out = np.empty(n, dtype=np.float64)
+    lib().oracle_dequant_sym8(_p(q), _p(scales), n, _p(out))
     return out
 
 
@@ -215,6 +237,18 @@ def expert_nvfp4(x, codes_e, scales_e, gs, H, I):
     return h, o
 
 
+def expert_sym8(x, q_e, scales_e, H, I):
+    """One sym8 expert on one token -> (h bf16 [I], o bf16 [H]); q_e int8
+    [3*I*H], scales_e binary16 words [3*I*H/32]."""
+    x = _c(x, np.uint16).ravel()
+    q_e = _c(np.asarray(q_e).view(np.uint8), np.uint8)
+    scales_e = _c(scales_e, np.uint16)
+    h = np.empty(I, dtype=np.uint16)
+    o = np.empty(H, dtype=np.uint16)
+    lib().oracle_expert_sym8(_p(x), _p(q_e), _p(scales_e), H, I, _p(h), _p(o))
+    return h, o
+
+
 def combine(o, w, residual=None):
     """o bf16 [k,H], w [k] -> y bf16 [H] (sequential BF16 combine)."""
     o = _c(o, np.uint16)
@@ -243,6 +277,31 @@ def moe_forward_nvfp4(x, ids, w, codes, scales, gscales, E, H, I, residual=None,
     h = np.empty((T, k, I), dtype=np.uint16) if want_h else None
     lib().oracle_moe_forward_nvfp4(_p(x), T, E, H, I, k, _p(ids), _p(w), _p(codes),
                                    _p(scales), _p(gscales), _p(r), _p(y), _p(o), _p(h))
+    out = [y]
+    if want_o:
+        out.append(o)
+    if want_h:
+        out.append(h)
+    return out[0] if len(out) == 1 else tuple(out)
+
+
+def moe_forward_sym8(x, ids, w, q, scales, E, H, I, residual=None,
+                     want_o=False, want_h=False):
+    """moe_forward for sym8 experts: q [E, 3*I*H] int8, scales [E, 3*I*H/32]
+    binary16 words."""
+    x = _c(x, np.uint16)
+    T = x.shape[0]
+    ids = _c(ids, np.int32)
+    k = ids.shape[1]
+    w = _c(w, np.float64)
+    q = _c(np.asarray(q).view(np.uint8), np.uint8)
+    scales = _c(scales, np.uint16)
+    r = _c(residual, np.uint16) if residual is not None else None
+    y = np.empty((T, H), dtype=np.uint16)
+    o = np.empty((T, k, H), dtype=np.uint16) if want_o else None
+    h = np.empty((T, k, I), dtype=np.uint16) if want_h else None
+    lib().oracle_moe_forward_sym8(_p(x), T, E, H, I, k, _p(ids), _p(w), _p(q), _p(scales),
+                                  _p(r), _p(y), _p(o), _p(h))
     out = [y]
     if want_o:
         out.append(o)

@@ -540,3 +540,115 @@ def test_nvfp4_reduces_to_mxfp4_when_scales_coincide():
     y_nv = oracle.moe_forward_nvfp4(x, ids, w, L.codes, nv_scales, gs, shape.E, shape.H,
                                     shape.I)
     np.testing.assert_array_equal(y_nv, y_mx)
+
+
+# ---------------------------------------------------------------- sym8
+
+def unpack_dense_sym8(q_m, scales_m, rows, K):
+    """Independent unpacker: int8 [rows][K] times the binary16 scale of each
+    32-element block, decoded by numpy's own float16 -> f64."""
+    q = np.asarray(q_m).view(np.int8).reshape(rows, K).astype(np.float64)
+    s = np.asarray(scales_m, dtype=np.uint16).view(np.float16).astype(np.float64)
+    return q * np.repeat(s.reshape(rows, K // 32), 32, axis=1)
+
+
+def test_f16_matches_numpy_binary16_all_patterns():
+    b = np.arange(65536, dtype=np.uint32)
+    want = b.astype(np.uint16).view(np.float16).astype(np.float64)
+    got = np.array([oracle.f16_value(int(v)) for v in b])
+    nan = np.isnan(want)
+    assert nan.sum() == 2 * 1023 and np.array_equal(np.isnan(got), nan)
+    np.testing.assert_array_equal(got[~nan], want[~nan])
+    # closed forms: 1.0, the largest finite 65504, the least subnormal 2^-24,
+    # the least normal 2^-14, infinities, a signed zero
+    assert (got[0x3C00], got[0x7BFF], got[0x0001], got[0x0400]) == (1.0, 65504.0, 2.0 ** -24,
+                                                                    2.0 ** -14)
+    assert got[0x7C00] == np.inf and got[0xFC00] == -np.inf
+    assert np.signbit(got[0x8000]) and got[0x8000] == 0.0
+
+
+def test_dequant_sym8_block_indexing_and_sign():
+    """q = j - 64 over 128 elements (every sign, -128 included), a different
+    binary16 scale per 32-element block: element j is (j - 64) times
+    scale[j // 32]."""
+    n = 128
+    q = (np.arange(n) - 64).astype(np.int8)
+    scales = np.array([0x3C00, 0x4000, 0x3800, 0xBC00], dtype=np.uint16)  # 1, 2, 0.5, -1
+    out = oracle.dequant_sym8(q, scales, n)
+    want = (np.arange(n) - 64) * np.repeat([1.0, 2.0, 0.5, -1.0], 32)
+    np.testing.assert_array_equal(out, want)
+    assert out[0] == -64.0 and out[127] == -63.0
+
+
+def _rand_expert_sym8(H, I, seed):
+    rng = synth.rng_for(seed, 98)
+    shape = synth.LayerShape(E=1, H=H, I=I)
+    q, scales = synth.make_expert_weights_sym8(shape, rng)
+    x = synth.f32_to_bf16_bits(rng.standard_normal(H, dtype=np.float32))
+    return q[0], scales[0], x
+
+
+@pytest.mark.parametrize("H,I,seed", [(64, 32, 0), (128, 96, 1), (512, 384, 2)])
+def test_expert_sym8_matches_dense_bruteforce(H, I, seed):
+    q, scales, x = _rand_expert_sym8(H, I, seed)
+    h, o = oracle.expert_sym8(x, q, scales, H, I)
+    mc, ms = I * H, I * H // 32
+    Wg = unpack_dense_sym8(q[:mc], scales[:ms], I, H)
+    Wu = unpack_dense_sym8(q[mc:2 * mc], scales[ms:2 * ms], I, H)
+    Wd = unpack_dense_sym8(q[2 * mc:], scales[2 * ms:], H, I)
+    xf = bf16_f64(x)
+    g = bf16_f64(bf16_via_f32(Wg @ xf))
+    u = bf16_f64(bf16_via_f32(Wu @ xf))
+    s = bf16_f64(bf16_via_f32(g / (1.0 + np.exp(-g))))
+    hb = bf16_via_f32(s * u)
+    ob = bf16_via_f32(Wd @ bf16_f64(hb))
+    dh, do = ulp_diff(h, hb), ulp_diff(o, ob)
+    assert dh.max() <= 1 and (dh > 0).sum() <= max(1, I // 500)
+    assert do.max() <= 1 and (do > 0).sum() <= max(1, H // 500)
+    # the structure matters: gate/up swapped gives a different answer
+    q_sw = np.concatenate([q[mc:2 * mc], q[:mc], q[2 * mc:]])
+    s_sw = np.concatenate([scales[ms:2 * ms], scales[:ms], scales[2 * ms:]])
+    h2, _ = oracle.expert_sym8(x, q_sw, s_sw, H, I)
+    assert (ulp_diff(h, h2) > 1).mean() > 0.5
+
+
+def test_expert_sym8_negated_down_weights_negate_output():
+    """q of the down matrix negated (the grid is symmetric): o changes sign
+    exactly, h does not change."""
+    H, I = 128, 64
+    q, scales, x = _rand_expert_sym8(H, I, 5)
+    h, o = oracle.expert_sym8(x, q, scales, H, I)
+    q2 = q.copy()
+    q2[2 * I * H:] = -q2[2 * I * H:]
+    h2, o2 = oracle.expert_sym8(x, q2, scales, H, I)
+    np.testing.assert_array_equal(h2, h)
+    np.testing.assert_array_equal(bf16_f64(o2), -bf16_f64(o))
+
+
+def test_sym8_reduces_to_mxfp4_when_values_coincide():
+    """Each E2M1 code c with E8M0 group exponent e is the int8 value 2 e2m1(c)
+    with the binary16 scale 2^(e - 128): the sym8 layer then equals the MXFP4
+    layer bit for bit (same weights, same summation order)."""
+    shape = synth.LayerShape(E=4, H=128, I=96)
+    L = synth.make_layer(shape, seed=6)
+    n = 3 * shape.I * shape.H
+    nib = np.empty((shape.E, n), dtype=np.int64)
+    nib[:, 0::2] = L.codes & 0x0F
+    nib[:, 1::2] = L.codes >> 4
+    twice = np.array([2 * e2m1_bitfield(c) for c in range(16)])
+    q = twice[nib].astype(np.int8)
+    # 2^(e - 128) for e = 118 .. 124 is a normal binary16 (exponent field e - 113)
+    f16 = ((L.scales.astype(np.uint16) - 113) << 10).astype(np.uint16)
+    assert np.array_equal(f16.view(np.float16).astype(np.float64),
+                          2.0 ** (L.scales.astype(np.float64) - 128))
+    x = synth.make_tokens(3, shape.H, seed=6)
+    ids = np.array([[0, 1, 2, 3], [3, 1, 0, 2], [2, 9, 1, 0]], dtype=np.int32)  # 9: invalid
+    w = np.array([[0.4, 0.3, 0.2, 0.1]] * 3)
+    r = synth.make_tokens(3, shape.H, seed=7)
+    y_mx, o_mx, h_mx = oracle.moe_forward(x, ids, w, L.codes, L.scales, shape.E, shape.H,
+                                          shape.I, residual=r, want_o=True, want_h=True)
+    y_s8, o_s8, h_s8 = oracle.moe_forward_sym8(x, ids, w, q, f16, shape.E, shape.H, shape.I,
+                                               residual=r, want_o=True, want_h=True)
+    np.testing.assert_array_equal(h_s8, h_mx)
+    np.testing.assert_array_equal(o_s8, o_mx)
+    np.testing.assert_array_equal(y_s8, y_mx)

@@ -147,6 +147,22 @@ def make_expert_weights_nvfp4(shape: LayerShape, rng: np.random.Generator):
     return codes, scales, gscales
 
 
+def make_expert_weights_sym8(shape: LayerShape, rng: np.random.Generator):
+    """sym8 experts of one layer: one int8 weight per element, uniform over
+    the symmetric grid -127 .. 127, and one IEEE binary16 block scale per 32
+    K elements, positive normal values 2^-13 .. 2^-9 (exponent fields 2..5,
+    uniform 10-bit mantissas), so |w| <= 127 * 2^-9.
+
+    Returns (q int8 [E, 3*I*H], scales uint16 [E, 3*I*H/32] binary16 bits).
+    """
+    n = 3 * shape.I * shape.H
+    q = rng.integers(-127, 128, size=(shape.E, n), dtype=np.int16).astype(np.int8)
+    ex = rng.integers(2, 6, size=(shape.E, n // 32), dtype=np.uint16)
+    man = rng.integers(0, 1024, size=(shape.E, n // 32), dtype=np.uint16)
+    scales = ((ex << 10) | man).astype(np.uint16)
+    return q, scales
+
+
 def make_activations(T: int, H: int, rng: np.random.Generator) -> np.ndarray:
     """x ~ N(0, 1) in BF16 bits, [T, H]."""
     return f32_to_bf16_bits(rng.standard_normal((T, H), dtype=np.float32))
@@ -206,6 +222,7 @@ class LayerInputs:
     router_w: np.ndarray   # uint16 (bf16) [E, H]
     router_b: np.ndarray | None  # float32 [E] or None
     gscales: np.ndarray | None = None  # NVFP4: float32 [E, 2]; scales are E4M3 [E, 3*I*H/16]
+    fmt: str = "mxfp4"  # "mxfp4", "nvfp4" or "sym8" (codes int8 [E, 3*I*H], scales binary16 [E, 3*I*H/32])
 
 
 def make_layer(shape: LayerShape, seed: int, layer: int = 0,
@@ -223,7 +240,16 @@ def make_layer_nvfp4(shape: LayerShape, seed: int, layer: int = 0,
     codes, scales, gscales = make_expert_weights_nvfp4(shape, rng)
     router_w = make_router(shape, rng)
     router_b = make_router_bias(shape, rng) if bias else None
-    return LayerInputs(shape, codes, scales, router_w, router_b, gscales)
+    return LayerInputs(shape, codes, scales, router_w, router_b, gscales, fmt="nvfp4")
+
+
+def make_layer_sym8(shape: LayerShape, seed: int, layer: int = 0,
+                    bias: bool = False) -> LayerInputs:
+    rng = rng_for(seed, 6, layer)
+    q, scales = make_expert_weights_sym8(shape, rng)
+    router_w = make_router(shape, rng)
+    router_b = make_router_bias(shape, rng) if bias else None
+    return LayerInputs(shape, q, scales, router_w, router_b, fmt="sym8")
 
 
 def make_tokens(T: int, H: int, seed: int, stream: int = 0) -> np.ndarray:
