@@ -498,14 +498,11 @@ cudaError_t launch_gu(const GateUpParams &p, int grid, cudaStream_t s, bool pdl)
 
 template <int TL, int KCH, bool SR, bool NV>
 cudaError_t launch_dn_v(const DownParams &p, int grid, size_t smem, cudaStream_t s, bool pdl) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(down_decode_kernel<TL, KCH, SR, NV>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kDownSmemMax);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    // once per process (thread-safe static initialisation)
+    static const cudaError_t attr = cudaFuncSetAttribute(
+        down_decode_kernel<TL, KCH, SR, NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)kDownSmemMax);
+    if (attr != cudaSuccess) return attr;
     return launch_ex(down_decode_kernel<TL, KCH, SR, NV>, dim3(grid), dim3(kDownThreads), smem, s,
                      pdl, p);
 }
@@ -568,16 +565,13 @@ int gateup_tma_slots(int H, int nv) {
 
 template <int KCH, bool NV>
 cudaError_t launch_gu_tma(const GateUpParams &p, int grid, cudaStream_t s, bool pdl) {
-    static bool attr_set = false;
     const size_t smem = (size_t)p.nslots * tma_slot_bytes(p.H, NV ? 1 : 0);
     if (smem > kTmaSmemBudget) return cudaErrorInvalidValue;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gateup_tma_kernel<KCH, NV>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kTmaSmemBudget);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    // once per process (thread-safe static initialisation)
+    static const cudaError_t attr = cudaFuncSetAttribute(
+        gateup_tma_kernel<KCH, NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)kTmaSmemBudget);
+    if (attr != cudaSuccess) return attr;
     return launch_ex(gateup_tma_kernel<KCH, NV>, dim3(grid), dim3(kTmaThreads), smem, s, pdl, p);
 }
 

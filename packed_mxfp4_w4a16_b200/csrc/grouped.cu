@@ -411,14 +411,12 @@ template <int NMAT>
 cudaError_t launch_mma(const GroupedParams &p, cudaStream_t s, bool pdl) {
     const int K = NMAT == 2 ? p.H : p.I, M = NMAT == 2 ? p.I : p.H;
     const size_t smem = mma_smem(NMAT, K);
-    static size_t attr_smem = 0;  // largest dynamic shared memory enabled so far
-    if (smem > attr_smem) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_mma_kernel<NMAT, kRowTiles>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
-        if (e != cudaSuccess) return e;
-        attr_smem = smem;
-    }
+    if (smem > kMmaSmemBudget) return cudaErrorInvalidValue;
+    // the budget, once per process (thread-safe static initialisation)
+    static const cudaError_t attr = cudaFuncSetAttribute(
+        grouped_mma_kernel<NMAT, kRowTiles>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)kMmaSmemBudget);
+    if (attr != cudaSuccess) return attr;
     return launch_ex(grouped_mma_kernel<NMAT, kRowTiles>, dim3(M / (kGpRows * kRowTiles), p.E),
                      dim3(128 * kRowTiles), smem, s, pdl, p);
 }

@@ -35,6 +35,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "gemv.cuh"
 
 namespace moe {
@@ -49,6 +51,7 @@ constexpr int kTcThreads = kTcWork + 32;  // + the MMA / TMA warp
 constexpr uint32_t kTcTileA = kTcM * kTcK * 2;    // 16 KB of BF16 per matrix
 constexpr uint32_t kTcTileB = kTcMaxN * kTcK * 2; // 16 KB of BF16
 constexpr int kTcBSlots = 4;                      // B tiles in flight (ring)
+constexpr size_t kTcSmemBudget = 220 * 1024;      // dynamic shared memory of a CTA
 
 __host__ __device__ constexpr uint32_t tc_stage_bytes(int nmat) {
     return (uint32_t)nmat * kTcTileA;  // an MMA stage holds the A tiles
@@ -459,15 +462,16 @@ struct CodesMap {
 };
 
 PFN_cuTensorMapEncodeTiled encode_fn() {
-    static PFN_cuTensorMapEncodeTiled fn = nullptr;
-    if (!fn) {
+    // looked up once (thread-safe static initialisation)
+    static const PFN_cuTensorMapEncodeTiled fn = [] {
         void *p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(p);
-    }
+            return reinterpret_cast<PFN_cuTensorMapEncodeTiled>(p);
+        return PFN_cuTensorMapEncodeTiled(nullptr);
+    }();
     return fn;
 }
 
@@ -491,18 +495,27 @@ cudaError_t codes_map(CodesMap &c, const uint8_t *base, size_t matrix_stride, in
     return cudaSuccess;
 }
 
+// The map of the weights bound last, re-encoded when they change; the lock
+// makes check, encode and copy one step for callers on several host threads
+// (a launch never sees a map another thread is rewriting).
+cudaError_t codes_map_copy(CodesMap &c, std::mutex &mu, const GroupedParams &p, int rows, int K,
+                           CUtensorMap *out) {
+    std::lock_guard<std::mutex> lock(mu);
+    cudaError_t e = codes_map(c, p.codes_base, p.codes_stride, p.E, rows, K);
+    if (e == cudaSuccess) *out = c.map;
+    return e;
+}
+
 template <int NMAT>
 cudaError_t launch_tc(const GroupedParams &p, const CUtensorMap &map, cudaStream_t s, bool pdl) {
     const int K = NMAT == 2 ? p.H : p.I, M = NMAT == 2 ? p.I : p.H;
     const size_t smem = tc_smem_bytes(NMAT, K, p.T * p.k);
-    static size_t attr_smem = 0;  // largest dynamic shared memory enabled so far
-    if (smem > attr_smem) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_tc_kernel<NMAT>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)smem);
-        if (e != cudaSuccess) return e;
-        attr_smem = smem;
-    }
+    if (smem > kTcSmemBudget) return cudaErrorInvalidValue;
+    // the budget, once per process (thread-safe static initialisation)
+    static const cudaError_t attr = cudaFuncSetAttribute(
+        grouped_tc_kernel<NMAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)kTcSmemBudget);
+    if (attr != cudaSuccess) return attr;
     return launch_ex(grouped_tc_kernel<NMAT>, dim3(M / kTcM, p.E), dim3(kTcThreads), smem, s, pdl,
                      p, map);
 }
@@ -513,24 +526,28 @@ cudaError_t launch_tc(const GroupedParams &p, const CUtensorMap &map, cudaStream
 // per matrix kind), H and I multiples of 128 and the shared-memory plan of a
 // launch of `pairs` (token, slot) pairs within the budget.
 bool grouped_tc_supported(int H, int I, int pairs) {
-    return H % 128 == 0 && I % 128 == 0 && tc_smem_bytes(2, H, pairs) <= 220 * 1024 &&
-           tc_smem_bytes(1, I, pairs) <= 220 * 1024;
+    return H % 128 == 0 && I % 128 == 0 && tc_smem_bytes(2, H, pairs) <= kTcSmemBudget &&
+           tc_smem_bytes(1, I, pairs) <= kTcSmemBudget;
 }
 
 cudaError_t launch_grouped_tc_gateup(const GroupedParams &p, cudaStream_t s, bool pdl) {
     static CodesMap gu;
+    static std::mutex mu;
     if (!p.codes_base) return cudaErrorInvalidValue;
-    cudaError_t e = codes_map(gu, p.codes_base, p.codes_stride, p.E, p.I, p.H);
+    CUtensorMap map;
+    cudaError_t e = codes_map_copy(gu, mu, p, p.I, p.H, &map);
     if (e != cudaSuccess) return e;
-    return launch_tc<2>(p, gu.map, s, pdl);
+    return launch_tc<2>(p, map, s, pdl);
 }
 
 cudaError_t launch_grouped_tc_down(const GroupedParams &p, cudaStream_t s, bool pdl) {
     static CodesMap dn;
+    static std::mutex mu;
     if (!p.codes_base) return cudaErrorInvalidValue;
-    cudaError_t e = codes_map(dn, p.codes_base, p.codes_stride, p.E, p.H, p.I);
+    CUtensorMap map;
+    cudaError_t e = codes_map_copy(dn, mu, p, p.H, p.I, &map);
     if (e != cudaSuccess) return e;
-    return launch_tc<1>(p, dn.map, s, pdl);
+    return launch_tc<1>(p, map, s, pdl);
 }
 
 }  // namespace moe

@@ -427,14 +427,11 @@ namespace {
 template <int KCH, int TLD, int KCHD>
 cudaError_t launch_lk(const GateUpParams &p, const FusedRouteParams &r, const LayerDownParams &d,
                       int grid, size_t smem, cudaStream_t s, bool pdl) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(layer_kernel<KCH, TLD, KCHD>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kFusedSmemBudget);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    // once per process (thread-safe static initialisation)
+    static const cudaError_t smem_attr = cudaFuncSetAttribute(
+        layer_kernel<KCH, TLD, KCHD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)kFusedSmemBudget);
+    if (smem_attr != cudaSuccess) return smem_attr;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kTmaThreads);
