@@ -20,6 +20,9 @@
 //   grouped_stage_h_kernel   per pair: FP16 staging of h.
 //   grouped_mma_kernel<1>    per (expert, 16 down rows): o = BF16(W_down h).
 //   grouped_combine_kernel   per token: sequential BF16 combine (+ residual).
+// When the groups average at least kTcAutoGroup pairs (or on request) the
+// two products and the h staging between them are replaced by the tcgen05
+// kernels of grouped_tc.cu (BF16 tiles, TMEM accumulators).
 //
 // Tensor-core tile.  A CTA holds 16 packed rows of one expert matrix (codes
 // and E8M0 scales; gate and up together) in shared memory and passes the
