@@ -33,7 +33,7 @@
  *         Bandwidth Budget": section "Where do the 2.45B active parameters
  *         actually go?" (SwiGLU expert = gate, up, down; H=2048, I=1536).
  *
- * Readings of points the pages leave open (each also listed in the design doc):
+ * Readings of points the pages leave open:
  *   - E2M1 code c: sign = bit 3, magnitude = {0,0.5,1,1.5,2,3,4,6}[c & 7].
  *   - Nibble order: element 2i is the low nibble of byte i.
  *   - E8M0 e: 2^(e-127); e = 255 is NaN.
