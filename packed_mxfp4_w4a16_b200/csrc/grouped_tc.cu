@@ -189,7 +189,7 @@ __host__ __device__ inline uint32_t tc_smem_bytes(int nmat, int K, int pairs) {
 
 // One TMA tile load of the 3-D code tensor (x: byte in the row, y: row,
 // z: matrix 3 e + m) into shared memory, completing on *bar.  Loads only
-// this GPU's memory; no multicast.
+// this GPU's memory, into this CTA alone.
 __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int x, int y, int z,
                                             uint64_t *bar, uint64_t pol) {
     asm volatile(
