@@ -59,6 +59,13 @@ def parse_args():
     ap.add_argument("--layers", type=int, default=N_LAYERS,
                     help="layers in the stack (fewer: a smaller case for profiling; "
                          "the bench workload is the full stack)")
+    ap.add_argument("--layered", action="store_true",
+                    help="run the step one layer at a time (three launches per layer) instead "
+                         "of the one-launch stack kernel")
+    ap.add_argument("--skip-configs", action="store_true",
+                    help="skip the tiny-layer, single-layer and 8B-stack measurements")
+    ap.add_argument("--only-main", action="store_true",
+                    help="time the main line only (for profiler runs)")
     return ap.parse_args()
 
 
@@ -103,40 +110,33 @@ def bytes_per_layer(shape, distinct_experts, T):
     return distinct_experts * expert + router + act
 
 
-def gateup_bytes(shape, pairs, prefetch_down):
-    """Algorithmic DRAM bytes of one gate/up launch: gate + up rows of every
-    selected expert, plus the down matrices it stages into L2 when
-    prefetching (they are then read from L2 by the down launch)."""
-    gu = 2 * (shape.I * shape.H // 2 + shape.I * shape.H // 32)
-    dn = shape.I * shape.H // 2 + shape.I * shape.H // 32
-    return pairs * (gu + (dn if prefetch_down else 0))
-
-
-# the translation unit of the decode kernels (gateup_tma_kernel among them)
-# and every header it includes: a change to any of them may change the kernel
-DECODE_TU = ("decode.cu", "down.cuh", "gemv.cuh", "kernels.cuh", "common.cuh")
+# the translation unit of the stack kernel and every header it includes: a
+# change to any of them may change the kernel
+STACK_TU = ("stack.cu", "down.cuh", "gemv.cuh", "kernels.cuh", "common.cuh")
 
 
 def csrc_digest():
     h = hashlib.sha256()
     d = os.path.join(ROOT, "packed_mxfp4_w4a16_b200", "csrc")
-    for name in DECODE_TU:
+    for name in STACK_TU:
         with open(os.path.join(d, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
-def stored_traffic():
-    """DRAM bytes per gate/up launch from the committed ncu summary, if it was
-    taken from the current kernel sources; else None."""
-    p = os.path.join(ROOT, "profiles", "gateup_tma_traffic.json")
+def stored_traffic(n_layers):
+    """DRAM bytes of one stack-kernel launch of n_layers from the committed
+    ncu summary (taken on a smaller stack and scaled by layers: the traffic
+    of a layer does not depend on the layer count), if it was taken from the
+    current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "stack_decode_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     if d.get("csrc_digest") != csrc_digest():
         return None
-    return d.get("dram_bytes_per_launch")
+    return d["dram_bytes_per_layer"] * n_layers
 
 
 # ------------------------------------------------------------------ clocks
@@ -264,9 +264,9 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ ours
 
-def build_stack(torch, moe, seed, n_layers):
+def stack_weights(torch, shape, seed, n_layers, bias=False):
     def gen(l):
-        return synth.make_layer(SHAPE, seed=seed, layer=l)
+        return synth.make_layer(shape, seed=seed, layer=l, bias=bias)
 
     weights = []
     with ThreadPoolExecutor(4) as ex:
@@ -274,8 +274,31 @@ def build_stack(torch, moe, seed, n_layers):
             codes = torch.from_numpy(L.codes).cuda()
             scales = torch.from_numpy(L.scales).cuda()
             rw = torch.from_numpy(L.router_w.view(np.int16)).cuda().view(torch.bfloat16)
-            weights.append((codes, scales, rw, None))
-    return moe.MoEStack(weights, SHAPE.E, SHAPE.H, SHAPE.I, SHAPE.top_k, T=1)
+            rb = None if L.router_b is None else torch.from_numpy(L.router_b).cuda()
+            weights.append((codes, scales, rw, rb))
+    return weights
+
+
+def build_stack(torch, moe, seed, n_layers, persistent=None):
+    weights = stack_weights(torch, SHAPE, seed, n_layers)
+    return moe.MoEStack(weights, SHAPE.E, SHAPE.H, SHAPE.I, SHAPE.top_k, T=1,
+                        persistent=persistent)
+
+
+def replay_rate(torch, graph, n, stream):
+    """Seconds per replay of `graph` over n back-to-back replays (CUDA events
+    on `stream`, after two warm replays)."""
+    with torch.cuda.stream(stream):
+        graph.replay()
+        graph.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / 1e3 / n
 
 
 def nvfp4_stack(torch, moe, st, args, max_steps=8):
@@ -344,7 +367,10 @@ def run_ours(args):
             dist.barrier()
 
     n_layers = args.layers
-    st = build_stack(torch, moe, seed=args.seed + rank, n_layers=n_layers)
+    st = build_stack(torch, moe, seed=args.seed + rank, n_layers=n_layers,
+                     persistent=False if args.layered else None)
+    if not args.layered:
+        assert st.stack is not None, "the stack kernel does not take this shape"
     st.set_tuning(use_pdl=not args.no_pdl, prefetch_down=not args.no_prefetch)
     x0 = torch.from_numpy(synth.make_tokens(1, SHAPE.H, seed=args.seed + rank, stream=3)
                           .view(np.int16)).cuda().view(torch.bfloat16)
@@ -374,28 +400,17 @@ def run_ours(args):
     t_ms = e0.elapsed_time(e1)
     t_ms = max_over_ranks(t_ms, world, "cuda")
     tok_s = job_throughput(TOKENS_PER_STEP * args.steps, world, t_ms)
+    status = st.status()
+    assert status == 0, f"device status {status:#x}"
 
     # bytes per token from the routing of the last replay (distinct experts)
     ids = st.ids.cpu().numpy()
     step_bytes = sum(bytes_per_layer(SHAPE, len(set(ids[l].ravel().tolist())), 1)
                      for l in range(n_layers))
-    gbs = step_bytes * TOKENS_PER_STEP * args.steps / (t_ms / 1e3) / 1e9
+    n_tok = TOKENS_PER_STEP * args.steps
+    us_tok = t_ms * 1e3 / n_tok
+    gbs = step_bytes * n_tok / (t_ms / 1e3) / 1e9
     peak, peak_kind = load_peaks()
-
-    # ---- per-kernel breakdown: graph with external timing events ----
-    kern = kernel_breakdown(torch, moe, st, reps=max(8, min(64, args.steps)))
-    pf = not args.no_prefetch
-    gu_bytes = gateup_bytes(SHAPE, SHAPE.top_k, pf) + SHAPE.H * 2
-    gu_gbs = gu_bytes / (kern["gateup_us"] * 1e-6) / 1e9
-
-    # ---- end to end through the public API with host buffers ----
-    e2e = run_e2e(torch, st, args)
-
-    # ---- the grouped path at batch sizes beyond decode (one layer) ----
-    batched = batched_cases(torch, moe, st, args.seed) if not args.skip_batched else None
-
-    # ---- the same stack with NVFP4 experts ----
-    nvfp4 = nvfp4_stack(torch, moe, st, args) if not args.skip_nvfp4 else None
 
     out = {
         "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world,
@@ -408,24 +423,49 @@ def run_ours(args):
                    "H": SHAPE.H, "I": SHAPE.I, "top_k": SHAPE.top_k,
                    "tokens_per_step": TOKENS_PER_STEP, "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (12.19 GB resident, 0.77 GB streamed per token "
-                         "vs 126 MB L2); no flush", "pdl": not args.no_pdl,
-                   "prefetch_down": pf},
+                         "vs 126 MB L2); no flush",
+                   "launch": "layered" if args.layered else "one stack launch per token"},
         "hbm_gbs": gbs, "hbm_frac": gbs / peak, "hbm_peak_gbs": peak,
-        "hbm_peak_kind": peak_kind, "bytes_per_token": step_bytes,
-        "us_per_token": t_ms * 1e3 / (TOKENS_PER_STEP * args.steps),
-        "roofline": {"bound": "hbm", "kernel": "gateup_tma_kernel",
-                     "achieved": gu_gbs, "peak": peak, "unit": "GB/s",
-                     "frac": gu_gbs / peak, "traffic": stored_traffic(),
-                     "bytes_per_launch": gu_bytes, "peak_kind": peak_kind},
-        "kernels": kern,
-        "e2e": e2e,
-        "batched": batched,
-        "nvfp4": nvfp4,
-        "gpu_launches": 3 * n_layers * TOKENS_PER_STEP * args.steps,
+        "hbm_peak_kind": peak_kind, "bytes_per_token": step_bytes, "us_per_token": us_tok,
         "clocks": clk.summary(),
     }
+    if args.layered:
+        out["roofline"] = {"bound": "hbm", "kernel": "whole step (3 launches per layer)",
+                           "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                           "traffic": None, "bytes_per_launch": None, "peak_kind": peak_kind}
+        out["gpu_launches"] = 3 * n_layers * n_tok
+    else:
+        # the step is one launch of the stack kernel: its duration is the time
+        # of one replay (graph launch gaps included, so a lower bound on the
+        # kernel's own rate)
+        out["roofline"] = {"bound": "hbm", "kernel": "stack_decode_kernel",
+                           "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                           "traffic": stored_traffic(n_layers), "bytes_per_launch": step_bytes,
+                           "launch_us": us_tok, "peak_kind": peak_kind,
+                           "peak_note": "burst copy bandwidth; the kernel is timed in a loop "
+                                        "of back-to-back launches"}
+        out["gpu_launches"] = n_tok
+
+    if not args.only_main:
+        # ---- end to end through the public API with host buffers ----
+        out["e2e"] = run_e2e(torch, st, args)
+        # ---- the same step one layer at a time (context: the launch structure
+        # this kernel replaces) ----
+        if not args.layered:
+            out["layered"] = layered_rate(torch, moe, st, x0, n_layers, step_bytes)
+        if not args.skip_configs:
+            out["configs"] = {
+                "tiny_layer": config_tiny(torch, moe, args.seed),
+                "layer24b": config_layer24b(torch, moe, st, args.seed),
+                "stack8b": config_stack8b(torch, moe, args.seed),
+            }
+        # ---- the grouped path at batch sizes beyond decode (one layer) ----
+        out["batched"] = (batched_cases(torch, moe, st, args.seed)
+                          if not args.skip_batched else None)
+        # ---- the same stack with NVFP4 experts ----
+        out["nvfp4"] = nvfp4_stack(torch, moe, st, args) if not args.skip_nvfp4 else None
+
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
-        import oracle
         rate, evals, threads, sample = oracle_layer_rate(12.0)
         out["cpu_baseline"] = {"value": rate / N_LAYERS, "unit": "tokens/s", "cores": threads,
                                "kind": "oracle", "sample": sample}
@@ -438,60 +478,161 @@ def run_ours(args):
     return 0
 
 
-def kernel_breakdown(torch, moe, st, reps):
-    """Average launch duration of each decode kernel kind, measured live: for
-    each kind a CUDA graph holds that kind's launch of every layer, back to
-    back on the stack's stream (programmatic serialization between them, as
-    in the decode graph), timed with CUDA events around whole replays.  The
-    routing of the last decoded token stays in place, so every launch does
-    the work of a real token.  The down-only graph reads its matrices from
-    HBM (no gate/up launch before it stages them into L2)."""
+def layered_rate(torch, moe, st, x0, n_layers, step_bytes):
+    """The same decode step with one moe_layer_ex per layer (router, gate/up
+    and down launches, programmatic serialization), one CUDA graph per token:
+    tokens/s, for comparison with the one-launch stack."""
+    lay = moe.MoEStack([(L.codes, L.scales, L.router_w, L.router_b) for L in st.layers],
+                       SHAPE.E, SHAPE.H, SHAPE.I, SHAPE.top_k, T=1, persistent=False)
+    lay.r.copy_(x0)
+    lay.capture()
+    sec = replay_rate(torch, lay.graph, 4 * TOKENS_PER_STEP, lay.stream)
+    lay.close()
+    return {"tokens_per_s": 1.0 / sec, "us_per_token": sec * 1e6,
+            "hbm_gbs": step_bytes / sec / 1e9, "launches_per_token": 3 * n_layers}
+
+
+def config_tiny(torch, moe, seed, reps=200):
+    """Tiny single MoE layer (H 512, I 384, E 16, top-4, 4 tokens): route +
+    expert FFN + combine (moe_layer_ex, three launches), CUDA graph of `reps`
+    calls."""
+    shape = synth.TINY
+    L = synth.make_layer(shape, seed=seed)
+    codes = torch.from_numpy(L.codes).cuda()
+    scales = torch.from_numpy(L.scales).cuda()
+    rw = torch.from_numpy(L.router_w.view(np.int16)).cuda().view(torch.bfloat16)
+    lay = moe.MoELayer(shape.E, shape.H, shape.I, shape.top_k, codes, scales, rw, None,
+                       max_tokens=4)
+    x = torch.from_numpy(synth.make_tokens(4, shape.H, seed=seed).view(np.int16)).cuda() \
+        .view(torch.bfloat16)
+    ids = torch.empty(4, shape.top_k, dtype=torch.int32, device="cuda")
+    w = torch.empty(4, shape.top_k, dtype=torch.float32, device="cuda")
+    y = torch.empty_like(x)
+    s = torch.cuda.Stream()
+
+    def call():
+        moe.moe_layer_ex(lay.handle, x, rw, None, 0, None, None, ids, w, None, y, 0, s)
+
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        call()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for _ in range(reps):
+            call()
+    sec = replay_rate(torch, g, 5, s) / reps
+    touched = len(set(ids.cpu().numpy().ravel().tolist()))
+    nbytes = bytes_per_layer(shape, touched, 4)
+    del g
+    lay.close()
+    return {"workload": "tiny: one layer H=512, I=384, E=16, top-4, T=4 (route + experts + "
+                        "combine, moe_layer_ex)", "us_per_call": sec * 1e6,
+            "tokens_per_s": 4 / sec, "hbm_gbs": nbytes / sec / 1e9, "experts_touched": touched}
+
+
+def config_layer24b(torch, moe, st, seed, calls=1000):
+    """One 24B layer at batch-1 decode with fresh routing on every call: the
+    stack's 38 layers as 38 one-layer stacks, cycled (1000 calls in a CUDA
+    graph, each on its own N(0,1) input token, so every call routes anew and
+    the weights read by consecutive calls are different layers' -- 38 x 320
+    MB of experts, no L2 reuse).  Each call = one stack-kernel launch of one
+    layer (RMSNorm, route, experts, combine, residual).  Also the API path
+    moe_route + moe_forward (the four-call boundary), same inputs."""
     n = len(st.layers)
-    s = st.stream
-    saved = st.r.clone()
+    stacks = []
+    for L in st.layers:
+        h = moe.moe_stack_create([L.handle], [L.router_w], [L.router_b])
+        ws = torch.empty(moe.moe_stack_workspace_bytes(h), dtype=torch.uint8, device="cuda")
+        moe.moe_stack_set_workspace(h, ws)
+        stacks.append((h, ws))
+    xs = torch.from_numpy(synth.make_tokens(calls, SHAPE.H, seed=seed, stream=99)
+                          .view(np.int16)).cuda().view(torch.bfloat16)
+    ids = torch.zeros(calls, SHAPE.top_k, dtype=torch.int32, device="cuda")
+    w = torch.zeros(calls, SHAPE.top_k, dtype=torch.float32, device="cuda")
+    s = torch.cuda.Stream()
+    r = xs.clone()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for i in range(calls):
+            h = stacks[i % n][0]
+            moe.moe_stack_decode(h, r[i], topk_ids=ids[i], topk_w=w[i], stream=s)
+    with torch.cuda.stream(s):
+        r.copy_(xs)
+    sec = replay_rate(torch, g, 1, s) / calls
+    del g
+    ids_h = ids.cpu().numpy()
+    touched = float(np.mean([len(set(row.tolist())) for row in ids_h]))
+    nbytes = bytes_per_layer(SHAPE, touched, 1)
+    for h, _ in stacks:
+        moe.moe_stack_destroy(h)
+    # the four-call API path: moe_route + moe_forward per call
+    y = torch.empty_like(xs)
+    g2 = torch.cuda.CUDAGraph()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g2, stream=s):
+        for i in range(calls):
+            L = st.layers[i % n]
+            moe.moe_route(L.handle, xs[i:i + 1], L.router_w, L.router_b, ids[i:i + 1],
+                          w[i:i + 1], stream=s)
+            moe.moe_forward(L.handle, xs[i:i + 1], ids[i:i + 1], w[i:i + 1], y[i:i + 1],
+                            stream=s)
+    sec2 = replay_rate(torch, g2, 1, s) / calls
+    del g2
+    return {"workload": "layer24b: one H=2048, I=1536, E=64, top-4 layer, T=1, fresh input "
+                        "and routing per call, 38 distinct layers cycled (no L2 reuse), "
+                        f"{calls} calls", "us_per_layer": sec * 1e6,
+            "hbm_gbs": nbytes / sec / 1e9, "bytes_per_call": nbytes,
+            "launch": "one stack-kernel launch per call (RMSNorm + layer + residual)",
+            "api_route_forward_us": sec2 * 1e6, "api_route_forward_gbs": nbytes / sec2 / 1e9}
 
-    def route(l, L):
-        moe.moe_route_ex(L.handle, st.r, L.router_w, L.router_b, moe.ROUTE_RMSNORM, st.xn, None,
-                         st.ids[l], st.w[l], s)
 
-    def gateup(l, L):
-        moe.moe_forward_ex(L.handle, st.xn, st.ids[l], st.w[l], st.r, st.r,
-                           moe.FWD_PHASE_GATEUP, s)
+def config_stack8b(torch, moe, seed, steps=4):
+    """8B-A1B-like stack: 22 layers of E=32, H=2048, I=1536, top-4, with a
+    per-expert router bias ~N(0,1) skewing popularity; batch-1 decode, one
+    stack launch per token, 64 tokens per step.  Bytes per token from the
+    actual routing of every timed token (distinct experts per layer)."""
+    shape = synth.L8B
+    n_layers = 22
+    w8 = stack_weights(torch, shape, seed + 8, n_layers, bias=True)
+    st = moe.MoEStack(w8, shape.E, shape.H, shape.I, shape.top_k, T=1)
+    assert st.stack is not None
+    x0 = torch.from_numpy(synth.make_tokens(1, shape.H, seed=seed, stream=8)
+                          .view(np.int16)).cuda().view(torch.bfloat16)
+    st.r.copy_(x0)
+    st.capture()
+    n_tok = steps * TOKENS_PER_STEP
+    sec = replay_rate(torch, st.graph, n_tok, st.stream)
+    # the routing of n_tok consecutive tokens (untimed pass from the same state)
+    ids_all = torch.zeros(n_tok, n_layers, shape.top_k, dtype=torch.int32, device="cuda")
+    with torch.cuda.stream(st.stream):
+        for t in range(n_tok):
+            moe.moe_stack_decode(st.stack, st.r, topk_ids=ids_all[t], stream=st.stream)
+    torch.cuda.synchronize()
+    assert st.status() == 0
+    ids_h = ids_all.cpu().numpy()
+    per_tok = [sum(bytes_per_layer(shape, len(set(ids_h[t, l].tolist())), 1)
+                   for l in range(n_layers)) for t in range(n_tok)]
+    tok_bytes = float(np.mean(per_tok))
+    # reuse between consecutive tokens: experts a layer already read for the
+    # previous token (their bytes may still be in L2)
+    same = np.mean([len(set(ids_h[t, l].tolist()) & set(ids_h[t - 1, l].tolist())) / shape.top_k
+                    for t in range(1, n_tok) for l in range(n_layers)])
+    counts = np.bincount(ids_h.ravel(), minlength=shape.E) / ids_h.size
+    st.close()
+    return {"workload": "stack8b: 22 layers x (H=2048, I=1536, E=32, top-4), router bias "
+                        "N(0,1), batch-1 decode, one stack launch per token",
+            "tokens_per_s": 1.0 / sec, "us_per_token": sec * 1e6, "bytes_per_token": tok_bytes,
+            "hbm_gbs": tok_bytes / sec / 1e9, "tokens": n_tok,
+            "expert_repeat_frac_vs_previous_token": float(same),
+            "top_expert_share": float(np.sort(counts)[::-1][:4].sum()),
+            "l2_note": "444 MB of experts per token against a 126 MB L2: repeats between "
+                       "consecutive tokens can hit L2; GB/s counts every touched expert once "
+                       "per token"}
 
-    def down(l, L):
-        moe.moe_forward_ex(L.handle, st.xn, st.ids[l], st.w[l], st.r, st.r,
-                           moe.FWD_PHASE_DOWN, s)
 
-    per = {}
-    for name, fn in (("route", route), ("gateup", gateup), ("down", down)):
-        g = torch.cuda.CUDAGraph()
-        s.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.graph(g, stream=s):
-            for l, L in enumerate(st.layers):
-                fn(l, L)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(s):  # replays and events on the stack's stream
-            for _ in range(3):
-                g.replay()
-            torch.cuda.synchronize()
-            e0.record(s)
-            for _ in range(reps):
-                g.replay()
-            e1.record(s)
-        torch.cuda.synchronize()
-        per[name] = e0.elapsed_time(e1) * 1e3 / (reps * n)
-        del g
-    st.r.copy_(saved)
-    total = sum(per.values())
-    return {"route_us": per["route"], "gateup_us": per["gateup"], "down_us": per["down"],
-            "share": {k: v / total for k, v in per.items()},
-            "launches_timed_per_kind": reps * n,
-            "method": "per kind: a graph of that kind's launch for every layer, back to back "
-                      "with programmatic serialization, CUDA events around the replays"}
-
-
-BATCHED_CASES = ((32, "uniform"), (32, "zipf"), (64, "uniform"), (256, "uniform"),
+BATCHED_CASES = ((32, "uniform"), (32, "zipf"), (64, "uniform"), (64, "zipf"), (256, "uniform"),
                  (256, "zipf"), (1024, "uniform"), (2048, "uniform"), (2048, "zipf"))
 TC_AUTO_GROUP = 40  # the library's tcgen05 products from T k >= 40 E on
 
@@ -542,6 +683,8 @@ def batched_cases(torch, moe, st, seed, reps=20):
         touched = len(set(ids_h.ravel().tolist()))
         nbytes = touched * expert + T * SHAPE.H * 2 * 2
         row = {"T": T, "routing": dist, "experts_touched": touched,
+               "case": "S=64 prefill chunk" if T == 64 else ("decode batch" if T <= 256 else
+                                                             "prefill"),
                "products": "tcgen05" if tc else "mma.sync",
                "us_per_call": us, "tokens_per_s": T / (us * 1e-6),
                "hbm_gbs": nbytes / (us * 1e-6) / 1e9}

@@ -304,6 +304,83 @@ MOE_API int moe_set_tuning(moe_handle_t h, int use_pdl, int prefetch_down);
 MOE_API int moe_set_fusion(moe_handle_t h, int mode);
 
 /* ---------------------------------------------------------------------
+ * A decode stack: the batch-1 decode step of n_layers MoE layers on a
+ * residual stream r, in ONE kernel launch (model card sections "Grouped
+ * top-4 expert execution", "GPU routing inside resident-layer graphs",
+ * "Direct reads from GPU-resident weights"; the RMS cells of "CUDA Graph
+ * lifetime and state management").  For each layer l in order:
+ *   xn = BF16(r / sqrt(mean(r^2) + 1e-6))            (weightless RMSNorm)
+ *   routing of xn as moe_route (softmax over the top-k biased logits)
+ *   r  = BF16(r + combine(experts(xn)))              (as moe_forward_ex
+ *                                                     with residual r)
+ * i.e. exactly moe_layer_ex(MOE_ROUTE_RMSNORM, residual = y = r) per layer,
+ * bit for bit.  One CTA per SM stays resident for the whole step
+ * (cooperative launch) and the CTAs hand each layer's grid-wide steps to one
+ * another through tagged words in the stack's workspace; every wait is
+ * bounded and a wait that gives up sets MOE_DEVICE_TIMEOUT. */
+typedef struct moe_stack_ctx *moe_stack_t;
+
+/* Create a stack over n_layers (1..64) layer handles that are already bound
+ * to MXFP4 weights (moe_load_packed or moe_load_expert_table) on the current
+ * device and share E, H, I, top_k.  router_w: HOST array of n_layers device
+ * pointers, BF16 [E][H] each (16-byte aligned); router_bias: NULL or a HOST
+ * array of n_layers device pointers, FP32 [E] or NULL each.  The layers'
+ * weight bindings and these pointers are read now: rebinding a layer later
+ * needs a new stack; the memory must stay valid until moe_stack_destroy.
+ * Shapes the stack kernel holds: H a multiple of 512 up to 2048, I a multiple
+ * of 128 up to 4096 with I/32 in {12, 16, 32, 48, 64} (I = 384, 512, 1024,
+ * 1536, 2048), top_k <= E <= 256 and E <= the SM count; NVFP4 layers are not
+ * taken.  Errors: ARG (including a shape or format outside that set: run the
+ * layers with moe_layer_ex instead), NOT_LOADED, NOT_DEVICE, ALIGN,
+ * UNSUPPORTED, CUDA. */
+MOE_API int moe_stack_create(const moe_handle_t *layers, int n_layers,
+                             const uint16_t *const *router_w,
+                             const float *const *router_bias, moe_stack_t *out);
+
+/* Release the stack (host memory only; no device synchronisation).  Work
+ * already enqueued keeps the pointers it was given.  NULL is a no-op. */
+MOE_API int moe_stack_destroy(moe_stack_t s);
+
+/* Bytes of device workspace the stack needs (tagged exchange words, launch
+ * counters, status; about 35 KB for H 2048, I 1536, E 64, top-4).
+ * Errors: ARG. */
+MOE_API int moe_stack_workspace_bytes(moe_stack_t s, size_t *bytes);
+
+/* Give the stack its device workspace (caller-owned, 256-byte aligned, at
+ * least moe_stack_workspace_bytes).  Zeroes it synchronously.  One
+ * workspace serves one stack, and its decode calls must be ordered on the
+ * GPU (one stream, or explicit dependencies): calls that overlap race on
+ * the exchange words.  Errors: ARG, NOT_DEVICE, ALIGN, WORKSPACE, CUDA. */
+MOE_API int moe_stack_set_workspace(moe_stack_t s, void *workspace, size_t bytes);
+
+/* One decode step of one token.  r: device BF16 [H], the residual stream,
+ * read as the first layer's input and overwritten with the last layer's
+ * output.  Optional outputs (device, or NULL): r_hist BF16 [n_layers][H]
+ * (each layer's input r), xn_hist BF16 [n_layers][H] (each layer's routed
+ * vector), logits FP32 [n_layers][E], topk_ids int32 [n_layers][top_k],
+ * topk_w FP32 [n_layers][top_k].  Enqueues one kernel on `stream`: no
+ * allocation, no synchronisation, capturable in a CUDA graph.  Needs every
+ * SM of the device free for the kernel (the launch fails with CUDA
+ * otherwise).  Errors: ARG, NOT_LOADED (no workspace), NOT_DEVICE, ALIGN,
+ * CUDA. */
+MOE_API int moe_stack_decode(moe_stack_t s, uint16_t *r, uint16_t *r_hist,
+                             uint16_t *xn_hist, float *logits,
+                             int32_t *topk_ids, float *topk_w, void *stream);
+
+/* Synchronise `stream`, return the stack's device status word
+ * (MOE_DEVICE_* bits) in *device_status and clear it.  After
+ * MOE_DEVICE_TIMEOUT the outputs of that step are invalid (r may hold the
+ * step's input or a partial result); later steps run normally.
+ * Errors: ARG, NOT_LOADED, CUDA. */
+MOE_API int moe_stack_get_status(moe_stack_t s, void *stream, unsigned *device_status);
+
+/* Test hook: the number of polls after which a wait on another CTA's tagged
+ * words gives up (default 2^20; 0 makes every such wait give up at once).
+ * Waits on the CTA's own copies in flight keep their full bound, so no copy
+ * outlives a launch that gave up.  Errors: ARG. */
+MOE_API int moe_stack_set_spin_limit(moe_stack_t s, int polls);
+
+/* ---------------------------------------------------------------------
  * Forward without any device allocation.  No counterpart in the paper: this
  * entry point exists for callers that may not call cudaMalloc -- code that
  * runs inside another framework's memory pool or allocator callback, hosts
@@ -311,34 +388,42 @@ MOE_API int moe_set_fusion(moe_handle_t h, int mode);
  * must not allocate while other streams are being captured.  It computes
  * exactly what moe_create + moe_load_packed + moe_set_workspace +
  * moe_forward_ex(residual) compute, with the same kernels, but without a
- * handle: its scratch (expert table, status word, SwiGLU activations h)
- * lives in one file-scope device array of MOE_NOALLOC_SCRATCH_BYTES bytes
- * that every GPU loading this library holds until the process exits.
+ * handle: its scratch (status word, SwiGLU activations h) lives in one
+ * file-scope device array of MOE_NOALLOC_SCRATCH_BYTES bytes that every GPU
+ * loading this library holds until the process exits.
  *
- * Limits (beyond them the call returns MOE_ERR_WORKSPACE and enqueues
- * nothing): E <= MOE_NOALLOC_MAX_EXPERTS and T * top_k * I * 2 <=
- * MOE_NOALLOC_MAX_H_BYTES.  Shapes as for moe_create.
+ * Limit (beyond it the call returns MOE_ERR_WORKSPACE and enqueues
+ * nothing): T * top_k * I * 2 <= MOE_NOALLOC_MAX_H_BYTES.  Shapes as for
+ * moe_create.
  * Arguments: codes_u8 / scales_e8m0 as for moe_load_packed (device,
  * contiguous [E][3][...], 16-byte aligned, read in place); x, topk_ids,
  * topk_w, residual (or NULL; may alias y), y as for moe_forward_ex.  These
  * pointers are not checked to be device memory (that check would itself be
- * a runtime call per pointer); they must be.
+ * a runtime call per pointer); they must be, and must hold the sizes the
+ * shape implies.
  * The first call on a device (with that device current) looks up the
  * scratch's device address with cudaGetSymbolAddress; make that first call
- * before any stream capture.  Every call rewrites the shared scratch (the
- * expert table by a cudaMemcpyAsync from the host stack, the status word by
- * a cudaMemsetAsync) on `stream`: calls that overlap on the GPU (different
- * streams, or different threads without ordering) race on it.
+ * before any stream capture.  Every call enqueues its kernels on `stream`
+ * and shares the one scratch array: calls that overlap on the GPU
+ * (different streams, or different threads without ordering) race on it.
+ * The kernels report an id outside [0, E) (that slot contributes 0) or a
+ * bounded wait that gave up in the scratch's status word; it accumulates
+ * over calls until moe_forward_noalloc_status reads and clears it.
  * Errors: ARG, ALIGN, WORKSPACE, UNSUPPORTED, CUDA. */
-#define MOE_NOALLOC_MAX_EXPERTS 256
 #define MOE_NOALLOC_MAX_H_BYTES (512u * 1024u)
-#define MOE_NOALLOC_SCRATCH_BYTES (12288u + 256u + MOE_NOALLOC_MAX_H_BYTES)
+#define MOE_NOALLOC_SCRATCH_BYTES (256u + MOE_NOALLOC_MAX_H_BYTES)
 MOE_API int moe_forward_noalloc(int E, int H, int I, int top_k,
                                 const uint8_t *codes_u8,
                                 const uint8_t *scales_e8m0, const uint16_t *x,
                                 int T, const int32_t *topk_ids,
                                 const float *topk_w, const uint16_t *residual,
                                 uint16_t *y, void *stream);
+
+/* Device status word of moe_forward_noalloc on the current device
+ * (MOE_DEVICE_* bits, accumulated since the last read): synchronises
+ * `stream`, copies the word to *device_status and clears it (no
+ * allocation).  Errors: ARG, UNSUPPORTED, CUDA. */
+MOE_API int moe_forward_noalloc_status(void *stream, unsigned *device_status);
 
 /* Human-readable name of a status code (static string, never NULL). */
 MOE_API const char *moe_status_string(int status);

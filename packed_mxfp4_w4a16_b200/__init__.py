@@ -27,7 +27,9 @@ __all__ = [
     "moe_workspace_bytes", "moe_set_workspace", "moe_route", "moe_route_ex",
     "moe_forward", "moe_forward_ex", "moe_layer_ex", "moe_get_intermediates", "moe_get_status",
     "moe_bytes_per_expert", "moe_set_tuning", "moe_device_check", "moe_debug_dequant",
-    "moe_forward_noalloc",
+    "moe_forward_noalloc", "moe_forward_noalloc_status", "moe_stack_create", "moe_stack_destroy", "moe_stack_workspace_bytes",
+    "moe_stack_set_workspace", "moe_stack_decode", "moe_stack_get_status",
+    "moe_stack_set_spin_limit",
     "ROUTE_RMSNORM", "ROUTE_SIGMOID", "FWD_KEEP_INTERMEDIATES", "FWD_FORCE_DECODE", "FWD_FORCE_GROUPED",
     "FWD_PHASE_GATEUP", "FWD_PHASE_DOWN", "FWD_FORCE_TCGEN05", "FWD_FORCE_MMA",
     "FUSION_NONE", "FUSION_ROUTER", "FUSION_LAYER", "moe_set_fusion",
@@ -205,21 +207,111 @@ def moe_debug_dequant(codes, scales, n, out, stream=None) -> None:
     check("moe_debug_dequant", load().moe_debug_dequant(_p(codes), _p(scales), n, _p(out), _s(stream)))
 
 
+def _noalloc_args_ok(E, H, I, top_k, codes, scales, x, topk_ids, topk_w, residual, y,
+                     device=None):
+    """Shape, dtype, layout and device checks of moe_forward_noalloc's tensors
+    (the C call takes bare pointers and cannot check sizes).  Raises MoEError
+    (MOE_ERR_ARG) on a mismatch.  `device`: the device every tensor must be on
+    (default: the current CUDA device)."""
+    if device is None:
+        device = torch.device("cuda", torch.cuda.current_device())
+    device = torch.device(device)
+
+    def need(t, dtype, numel, what):
+        ok = (t is not None and t.dtype == dtype and t.is_contiguous() and t.numel() == numel
+              and t.device == device)
+        if not ok:
+            raise MoEError(f"moe_forward_noalloc ({what})", -1)
+
+    if x is None or x.dim() != 2 or x.shape[1] != H:
+        raise MoEError("moe_forward_noalloc (x shape)", -1)
+    T = x.shape[0]
+    need(codes, torch.uint8, E * 3 * I * H // 2, "codes")
+    need(scales, torch.uint8, E * 3 * I * H // 32, "scales")
+    need(x, torch.bfloat16, T * H, "x")
+    need(topk_ids, torch.int32, T * top_k, "topk_ids")
+    need(topk_w, torch.float32, T * top_k, "topk_w")
+    need(y, torch.bfloat16, T * H, "y")
+    if residual is not None:
+        need(residual, torch.bfloat16, T * H, "residual")
+    return T
+
+
 def moe_forward_noalloc(E, H, I, top_k, codes, scales, x, topk_ids, topk_w, residual, y,
                         stream=None) -> None:
     """Expert FFN + combine for callers that may not allocate device memory:
     no handle, no workspace; scratch lives in a fixed device array inside the
-    library (see include/moe_mxfp4.h for its limits and its sharing rules)."""
-    _need(codes, torch.uint8, "moe_forward_noalloc")
-    _need(scales, torch.uint8, "moe_forward_noalloc")
-    _need(x, torch.bfloat16, "moe_forward_noalloc", 2)
-    _need(topk_ids, torch.int32, "moe_forward_noalloc")
-    _need(topk_w, torch.float32, "moe_forward_noalloc")
-    _need(residual, torch.bfloat16, "moe_forward_noalloc")
-    _need(y, torch.bfloat16, "moe_forward_noalloc")
+    library (see include/moe_mxfp4.h for its limits and its sharing rules).
+    Every tensor is checked against E, H, I, top_k and T = x.shape[0] and must
+    be on the current device."""
+    T = _noalloc_args_ok(E, H, I, top_k, codes, scales, x, topk_ids, topk_w, residual, y)
     check("moe_forward_noalloc", load().moe_forward_noalloc(
-        E, H, I, top_k, _p(codes), _p(scales), _p(x), x.shape[0], _p(topk_ids), _p(topk_w),
+        E, H, I, top_k, _p(codes), _p(scales), _p(x), T, _p(topk_ids), _p(topk_w),
         _p(residual), _p(y), _s(stream)))
+
+
+def moe_forward_noalloc_status(stream=None) -> int:
+    """Status bits of moe_forward_noalloc on the current device since the
+    last read (synchronises `stream`), cleared."""
+    v = C.c_uint()
+    check("moe_forward_noalloc_status", load().moe_forward_noalloc_status(_s(stream), C.byref(v)))
+    return v.value
+
+
+def moe_stack_create(handles, router_ws, router_bs=None) -> int:
+    """A decode stack over layer handles (ints); router_ws / router_bs:
+    sequences of device tensors (BF16 [E, H]; FP32 [E] or None)."""
+    n = len(handles)
+    for t in router_ws:
+        _need(t, torch.bfloat16, "moe_stack_create", 2)
+    ha = (C.c_void_p * n)(*handles)
+    wa = (C.c_void_p * n)(*[t.data_ptr() for t in router_ws])
+    ba = None
+    if router_bs is not None and any(b is not None for b in router_bs):
+        for t in router_bs:
+            _need(t, torch.float32, "moe_stack_create")
+        ba = (C.c_void_p * n)(*[None if b is None else b.data_ptr() for b in router_bs])
+    out = C.c_void_p()
+    check("moe_stack_create", load().moe_stack_create(ha, n, wa, ba, C.byref(out)))
+    return out.value
+
+
+def moe_stack_destroy(s: int) -> None:
+    check("moe_stack_destroy", load().moe_stack_destroy(C.c_void_p(s)))
+
+
+def moe_stack_workspace_bytes(s: int) -> int:
+    n = C.c_size_t()
+    check("moe_stack_workspace_bytes", load().moe_stack_workspace_bytes(C.c_void_p(s), C.byref(n)))
+    return n.value
+
+
+def moe_stack_set_workspace(s: int, ws: torch.Tensor) -> None:
+    _need(ws, torch.uint8, "moe_stack_set_workspace")
+    check("moe_stack_set_workspace", load().moe_stack_set_workspace(C.c_void_p(s), _p(ws), ws.numel()))
+
+
+def moe_stack_decode(s, r, r_hist=None, xn_hist=None, logits=None, topk_ids=None, topk_w=None,
+                     stream=None) -> None:
+    _need(r, torch.bfloat16, "moe_stack_decode")
+    _need(r_hist, torch.bfloat16, "moe_stack_decode")
+    _need(xn_hist, torch.bfloat16, "moe_stack_decode")
+    _need(logits, torch.float32, "moe_stack_decode")
+    _need(topk_ids, torch.int32, "moe_stack_decode")
+    _need(topk_w, torch.float32, "moe_stack_decode")
+    check("moe_stack_decode", load().moe_stack_decode(
+        C.c_void_p(s), _p(r), _p(r_hist), _p(xn_hist), _p(logits), _p(topk_ids), _p(topk_w),
+        _s(stream)))
+
+
+def moe_stack_get_status(s: int, stream=None) -> int:
+    v = C.c_uint()
+    check("moe_stack_get_status", load().moe_stack_get_status(C.c_void_p(s), _s(stream), C.byref(v)))
+    return v.value
+
+
+def moe_stack_set_spin_limit(s: int, polls: int) -> None:
+    check("moe_stack_set_spin_limit", load().moe_stack_set_spin_limit(C.c_void_p(s), int(polls)))
 
 
 # ------------------------------------------------------------- bundles
@@ -310,9 +402,14 @@ class MoEStack:
     r = BF16(r + combine).  ``step()`` replays one CUDA graph of all layers.
     Layers share one workspace (they run in order on one stream).
     ``layers_weights``: per layer (codes, scales, router_w, router_b), or
-    with a fifth item, the NVFP4 multipliers [E, 2] (see MoELayer)."""
+    with a fifth item, the NVFP4 multipliers [E, 2] (see MoELayer).
 
-    def __init__(self, layers_weights, E, H, I, top_k, T=1, device="cuda"):
+    ``persistent``: run the whole step as one launch (moe_stack_decode);
+    None = when the shape allows it (T = 1, MXFP4 layers, shapes of
+    moe_stack_create), False = one layer at a time (moe_layer_ex), True =
+    required."""
+
+    def __init__(self, layers_weights, E, H, I, top_k, T=1, device="cuda", persistent=None):
         moe_device_check()
         self.E, self.H, self.I, self.k, self.T = E, H, I, top_k, T
         self.layers = []
@@ -332,6 +429,25 @@ class MoEStack:
         self.w = torch.zeros(n, T, top_k, dtype=torch.float32, device=dev)
         self.graph = None
         self.stream = torch.cuda.Stream(device=dev)
+        # one launch for the whole step (moe_stack_*) when the shape allows it
+        self.stack = None
+        self.stack_ws = None
+        if persistent is not False and T == 1:
+            try:
+                self.stack = moe_stack_create([L.handle for L in self.layers],
+                                              [L.router_w for L in self.layers],
+                                              [L.router_b for L in self.layers])
+                self.stack_ws = torch.empty(moe_stack_workspace_bytes(self.stack),
+                                            dtype=torch.uint8, device=dev)
+                moe_stack_set_workspace(self.stack, self.stack_ws)
+            except MoEError:
+                if self.stack is not None:
+                    moe_stack_destroy(self.stack)
+                self.stack = None
+                if persistent:
+                    raise
+        elif persistent:
+            raise MoEError("moe_stack_create", -1)
 
     def set_tuning(self, use_pdl=True, prefetch_down=True):
         for L in self.layers:
@@ -344,9 +460,26 @@ class MoEStack:
 
     def enqueue(self, stream=None):
         """Enqueue one decode step (all layers) on `stream`."""
+        if self.stack is not None:
+            moe_stack_decode(self.stack, self.r, topk_ids=self.ids, topk_w=self.w, stream=stream)
+        else:
+            self.enqueue_layers(stream)
+
+    def enqueue_layers(self, stream=None):
+        """The same step as one moe_layer_ex call per layer."""
         for l, L in enumerate(self.layers):
             moe_layer_ex(L.handle, self.r, L.router_w, L.router_b, ROUTE_RMSNORM, self.xn, None,
                          self.ids[l], self.w[l], self.r, self.r, 0, stream)
+
+    def status(self, stream=None) -> int:
+        """Device status bits of the stack kernel and of every layer handle
+        (synchronises), cleared."""
+        st = 0
+        if self.stack is not None:
+            st |= moe_stack_get_status(self.stack, stream)
+        for L in self.layers:
+            st |= L.status()
+        return st
 
     def capture(self):
         """Capture one decode step into a CUDA graph (warm-up run first)."""
@@ -388,5 +521,8 @@ class MoEStack:
 
     def close(self):
         self.graph = None
+        if getattr(self, "stack", None) is not None:
+            moe_stack_destroy(self.stack)
+            self.stack = None
         for L in self.layers:
             L.close()

@@ -43,6 +43,14 @@ SIGNATURES = [
     ("moe_device_check", _i, []),
     ("moe_debug_dequant", _i, [_vp, _vp, _i64, _vp, _vp]),
     ("moe_forward_noalloc", _i, [_i, _i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp]),
+    ("moe_forward_noalloc_status", _i, [_vp, C.POINTER(_u)]),
+    ("moe_stack_create", _i, [C.POINTER(_vp), _i, C.POINTER(_vp), C.POINTER(_vp), C.POINTER(_vp)]),
+    ("moe_stack_destroy", _i, [_vp]),
+    ("moe_stack_workspace_bytes", _i, [_vp, C.POINTER(_sz)]),
+    ("moe_stack_set_workspace", _i, [_vp, _vp, _sz]),
+    ("moe_stack_decode", _i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    ("moe_stack_get_status", _i, [_vp, _vp, C.POINTER(_u)]),
+    ("moe_stack_set_spin_limit", _i, [_vp, _i]),
 ]
 
 

@@ -765,6 +765,191 @@ int moe_set_fusion(moe_handle_t h, int mode) {
     return MOE_OK;
 }
 
+// ------------------------------------------------------------ stacks --
+
+}  // extern "C"
+
+struct moe_stack_ctx {
+    int L = 0, E = 0, H = 0, I = 0, k = 0;
+    int device = -1;
+    int num_sms = 0;
+    uint8_t *ws = nullptr;
+    size_t ws_bytes = 0;
+    int spin_limit = moe::kMaxSpin;
+    moe::StackPlan plan = {};
+    moe::StackLayer layer[moe::kStackMaxLayers] = {};
+};
+
+namespace {
+
+struct StackWs {
+    size_t x_tag, lg_tag, h_tag, seq, abort, status, total;
+};
+
+StackWs stack_ws_layout(const moe_stack_ctx *s) {
+    StackWs W;
+    size_t off = 0;
+    auto take = [&](size_t n) {
+        size_t o = off;
+        off = align_up(off + n, 256);
+        return o;
+    };
+    W.x_tag = take((size_t)s->H / 2 * sizeof(uint2));
+    W.lg_tag = take((size_t)s->E * sizeof(uint2));
+    W.h_tag = take((size_t)s->k * s->I / 2 * sizeof(uint2));
+    W.seq = take((size_t)s->num_sms * sizeof(unsigned));
+    W.abort = take(sizeof(unsigned));
+    W.status = take(sizeof(unsigned));
+    W.total = off;
+    return W;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_stack_create(const moe_handle_t *layers, int n_layers, const uint16_t *const *router_w,
+                     const float *const *router_bias, moe_stack_t *out) {
+    if (!out) return MOE_ERR_ARG;
+    *out = nullptr;
+    if (!layers || !router_w || n_layers < 1 || n_layers > moe::kStackMaxLayers) return MOE_ERR_ARG;
+    const moe_ctx *l0 = layers[0];
+    if (!l0) return MOE_ERR_ARG;
+    for (int l = 0; l < n_layers; ++l) {
+        const moe_ctx *h = layers[l];
+        if (!h || h->E != l0->E || h->H != l0->H || h->I != l0->I || h->k != l0->k) return MOE_ERR_ARG;
+        if (!h->loaded) return MOE_ERR_NOT_LOADED;
+        if (h->nv) return MOE_ERR_ARG;  // the stack kernel reads MXFP4 experts
+        if (h->device != l0->device) return MOE_ERR_NOT_DEVICE;
+    }
+    int dev = -1, sms = 0;
+    int rc = current_device_ok(&dev, &sms);
+    if (rc != MOE_OK) return rc;
+    if (dev != l0->device) return MOE_ERR_NOT_DEVICE;
+    moe::StackPlan plan;
+    if (!moe::stack_plan(l0->E, l0->H, l0->I, l0->k, sms, &plan)) return MOE_ERR_ARG;
+    for (int l = 0; l < n_layers; ++l) {
+        if ((rc = check_device_ptr(l0, router_w[l], 16)) != MOE_OK) return rc;
+        if (router_bias && router_bias[l] && (rc = check_device_ptr(l0, router_bias[l], 4)) != MOE_OK)
+            return rc;
+    }
+    moe_stack_ctx *s = new (std::nothrow) moe_stack_ctx;
+    if (!s) return MOE_ERR_ARG;
+    s->L = n_layers;
+    s->E = l0->E;
+    s->H = l0->H;
+    s->I = l0->I;
+    s->k = l0->k;
+    s->device = dev;
+    s->num_sms = sms;
+    s->plan = plan;
+    for (int l = 0; l < n_layers; ++l) {
+        const moe_ctx *h = layers[l];
+        moe::StackLayer &ly = s->layer[l];
+        ly.codes_base = h->codes_base;
+        ly.scales_base = h->scales_base;
+        ly.table = h->d_table;
+        ly.router_w = router_w[l];
+        ly.bias = router_bias ? router_bias[l] : nullptr;
+    }
+    *out = s;
+    return MOE_OK;
+}
+
+int moe_stack_destroy(moe_stack_t s) {
+    delete s;
+    return MOE_OK;
+}
+
+int moe_stack_workspace_bytes(moe_stack_t s, size_t *bytes) {
+    if (!s || !bytes) return MOE_ERR_ARG;
+    *bytes = stack_ws_layout(s).total;
+    return MOE_OK;
+}
+
+int moe_stack_set_workspace(moe_stack_t s, void *workspace, size_t bytes) {
+    if (!s || !workspace) return MOE_ERR_ARG;
+    int rc;
+    moe_ctx probe;
+    probe.device = s->device;
+    if ((rc = check_device_ptr(&probe, workspace, 256)) != MOE_OK) return rc;
+    if (bytes < stack_ws_layout(s).total) return MOE_ERR_WORKSPACE;
+    if ((rc = cuda_rc(cudaMemset(workspace, 0, bytes))) != MOE_OK) return rc;
+    s->ws = static_cast<uint8_t *>(workspace);
+    s->ws_bytes = bytes;
+    return MOE_OK;
+}
+
+int moe_stack_set_spin_limit(moe_stack_t s, int polls) {
+    if (!s || polls < 0) return MOE_ERR_ARG;
+    s->spin_limit = polls;
+    return MOE_OK;
+}
+
+int moe_stack_decode(moe_stack_t s, uint16_t *r, uint16_t *r_hist, uint16_t *xn_hist,
+                     float *logits, int32_t *topk_ids, float *topk_w, void *stream) {
+    if (!s) return MOE_ERR_ARG;
+    if (!s->ws) return MOE_ERR_NOT_LOADED;
+    moe_ctx probe;
+    probe.device = s->device;
+    int rc;
+    if ((rc = check_device_ptr(&probe, r, 16)) != MOE_OK) return rc;
+    if (r_hist && (rc = check_device_ptr(&probe, r_hist, 16)) != MOE_OK) return rc;
+    if (xn_hist && (rc = check_device_ptr(&probe, xn_hist, 16)) != MOE_OK) return rc;
+    if (logits && (rc = check_device_ptr(&probe, logits, 4)) != MOE_OK) return rc;
+    if (topk_ids && (rc = check_device_ptr(&probe, topk_ids, 4)) != MOE_OK) return rc;
+    if (topk_w && (rc = check_device_ptr(&probe, topk_w, 4)) != MOE_OK) return rc;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    if (dev != s->device) return MOE_ERR_NOT_DEVICE;
+    const StackWs W = stack_ws_layout(s);
+    moe::StackParams p;
+    memset(&p, 0, sizeof p);
+    p.L = s->L;
+    p.E = s->E;
+    p.H = s->H;
+    p.I = s->I;
+    p.k = s->k;
+    p.codes_stride = (size_t)s->I * s->H / 2;
+    p.scales_stride = (size_t)s->I * s->H / 32;
+    p.r = r;
+    p.r_hist = r_hist;
+    p.xn_hist = xn_hist;
+    p.logits_hist = logits;
+    p.ids_hist = topk_ids;
+    p.w_hist = topk_w;
+    p.x_tag = reinterpret_cast<uint2 *>(s->ws + W.x_tag);
+    p.lg_tag = reinterpret_cast<uint2 *>(s->ws + W.lg_tag);
+    p.h_tag = reinterpret_cast<uint2 *>(s->ws + W.h_tag);
+    p.seq = reinterpret_cast<unsigned *>(s->ws + W.seq);
+    p.abort = reinterpret_cast<unsigned *>(s->ws + W.abort);
+    p.status = reinterpret_cast<unsigned *>(s->ws + W.status);
+    p.spin_limit = s->spin_limit;
+    p.plan = s->plan;
+    for (int l = 0; l < s->L; ++l) p.layer[l] = s->layer[l];
+    return cuda_rc(moe::launch_stack(p, s->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_stack_get_status(moe_stack_t s, void *stream, unsigned *device_status) {
+    if (!s || !device_status) return MOE_ERR_ARG;
+    if (!s->ws) return MOE_ERR_NOT_LOADED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const StackWs W = stack_ws_layout(s);
+    unsigned *d = reinterpret_cast<unsigned *>(s->ws + W.status);
+    int rc;
+    if ((rc = cuda_rc(cudaStreamSynchronize(st))) != MOE_OK) return rc;
+    unsigned v = 0;
+    if ((rc = cuda_rc(cudaMemcpyAsync(&v, d, sizeof v, cudaMemcpyDeviceToHost, st))) != MOE_OK)
+        return rc;
+    if ((rc = cuda_rc(cudaMemsetAsync(d, 0, sizeof v, st))) != MOE_OK) return rc;
+    if ((rc = cuda_rc(cudaStreamSynchronize(st))) != MOE_OK) return rc;
+    *device_status = v;
+    return MOE_OK;
+}
+
 const char *moe_status_string(int status) {
     switch (status) {
     case MOE_OK: return "MOE_OK";

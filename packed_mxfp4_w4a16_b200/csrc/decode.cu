@@ -233,7 +233,12 @@ gateup_decode_kernel(const GateUpParams p) {
         if (q != cur_q) {
             const int e = s_ids[q];
             bad = (e < 0 || e >= p.E);
-            if (!bad) {
+            if (!bad && p.codes_base) {
+                gc = p.codes_base + (size_t)(3 * e) * p.codes_stride;
+                uc = p.codes_base + (size_t)(3 * e + 1) * p.codes_stride;
+                gs = p.scales_base + (size_t)(3 * e) * p.scales_stride;
+                us = p.scales_base + (size_t)(3 * e + 1) * p.scales_stride;
+            } else if (!bad) {
                 const ExpertPtrs *ep = p.table + e;
                 gc = ep->codes[0];
                 gs = ep->scales[0];
@@ -498,10 +503,12 @@ cudaError_t launch_gu(const GateUpParams &p, int grid, cudaStream_t s, bool pdl)
 
 template <int TL, int KCH, bool SR, bool NV>
 cudaError_t launch_dn_v(const DownParams &p, int grid, size_t smem, cudaStream_t s, bool pdl) {
-    // once per process (thread-safe static initialisation)
-    static const cudaError_t attr = cudaFuncSetAttribute(
-        down_decode_kernel<TL, KCH, SR, NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-        (int)kDownSmemMax);
+    // once per device (the attribute belongs to the current device's context)
+    static PerDeviceOnce once;
+    const cudaError_t attr = per_device_once(once, [] {
+        return cudaFuncSetAttribute(down_decode_kernel<TL, KCH, SR, NV>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDownSmemMax);
+    });
     if (attr != cudaSuccess) return attr;
     return launch_ex(down_decode_kernel<TL, KCH, SR, NV>, dim3(grid), dim3(kDownThreads), smem, s,
                      pdl, p);
@@ -567,10 +574,13 @@ template <int KCH, bool NV>
 cudaError_t launch_gu_tma(const GateUpParams &p, int grid, cudaStream_t s, bool pdl) {
     const size_t smem = (size_t)p.nslots * tma_slot_bytes(p.H, NV ? 1 : 0);
     if (smem > kTmaSmemBudget) return cudaErrorInvalidValue;
-    // once per process (thread-safe static initialisation)
-    static const cudaError_t attr = cudaFuncSetAttribute(
-        gateup_tma_kernel<KCH, NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-        (int)kTmaSmemBudget);
+    // once per device (the attribute belongs to the current device's context)
+    static PerDeviceOnce once;
+    const cudaError_t attr = per_device_once(once, [] {
+        return cudaFuncSetAttribute(gateup_tma_kernel<KCH, NV>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kTmaSmemBudget);
+    });
     if (attr != cudaSuccess) return attr;
     return launch_ex(gateup_tma_kernel<KCH, NV>, dim3(grid), dim3(kTmaThreads), smem, s, pdl, p);
 }

@@ -415,10 +415,14 @@ cudaError_t launch_mma(const GroupedParams &p, cudaStream_t s, bool pdl) {
     const int K = NMAT == 2 ? p.H : p.I, M = NMAT == 2 ? p.I : p.H;
     const size_t smem = mma_smem(NMAT, K);
     if (smem > kMmaSmemBudget) return cudaErrorInvalidValue;
-    // the budget, once per process (thread-safe static initialisation)
-    static const cudaError_t attr = cudaFuncSetAttribute(
-        grouped_mma_kernel<NMAT, kRowTiles>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-        (int)kMmaSmemBudget);
+    // the budget, once per device (the attribute belongs to the current
+    // device's context)
+    static PerDeviceOnce once;
+    const cudaError_t attr = per_device_once(once, [] {
+        return cudaFuncSetAttribute(grouped_mma_kernel<NMAT, kRowTiles>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kMmaSmemBudget);
+    });
     if (attr != cudaSuccess) return attr;
     return launch_ex(grouped_mma_kernel<NMAT, kRowTiles>, dim3(M / (kGpRows * kRowTiles), p.E),
                      dim3(128 * kRowTiles), smem, s, pdl, p);

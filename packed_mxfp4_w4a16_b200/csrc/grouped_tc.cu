@@ -511,10 +511,14 @@ cudaError_t launch_tc(const GroupedParams &p, const CUtensorMap &map, cudaStream
     const int K = NMAT == 2 ? p.H : p.I, M = NMAT == 2 ? p.I : p.H;
     const size_t smem = tc_smem_bytes(NMAT, K, p.T * p.k);
     if (smem > kTcSmemBudget) return cudaErrorInvalidValue;
-    // the budget, once per process (thread-safe static initialisation)
-    static const cudaError_t attr = cudaFuncSetAttribute(
-        grouped_tc_kernel<NMAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-        (int)kTcSmemBudget);
+    // the budget, once per device (the attribute belongs to the current
+    // device's context)
+    static PerDeviceOnce once;
+    const cudaError_t attr = per_device_once(once, [] {
+        return cudaFuncSetAttribute(grouped_tc_kernel<NMAT>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kTcSmemBudget);
+    });
     if (attr != cudaSuccess) return attr;
     return launch_ex(grouped_tc_kernel<NMAT>, dim3(M / kTcM, p.E), dim3(kTcThreads), smem, s, pdl,
                      p, map);

@@ -4,9 +4,36 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "common.cuh"
 
 namespace moe {
+
+// One-time host set-up per (call site, device): a kernel's dynamic
+// shared-memory limit is a property of the function in the context of the
+// device that is current when it is set, so a process that drives several
+// GPUs must set it on each.  Thread-safe; `set` runs with the device current.
+struct PerDeviceOnce {
+    static constexpr int kMaxDevices = 64;
+    std::atomic<unsigned long long> done{0};
+    std::mutex m;
+};
+template <class F>
+inline cudaError_t per_device_once(PerDeviceOnce &o, F &&set) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= PerDeviceOnce::kMaxDevices) return cudaErrorInvalidDevice;
+    const unsigned long long bit = 1ull << dev;
+    if (o.done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+    std::lock_guard<std::mutex> g(o.m);
+    if (o.done.load(std::memory_order_relaxed) & bit) return cudaSuccess;
+    e = set();
+    if (e == cudaSuccess) o.done.fetch_or(bit, std::memory_order_release);
+    return e;
+}
 
 constexpr int kDecodeMaxT = 4;      // tokens handled by the per-(token,slot) GEMV path
 constexpr int kMaxTopK = 8;
@@ -175,6 +202,59 @@ bool layer_plan(int T, int E, int H, int I, int k, int grid, size_t *smem, int *
 cudaError_t launch_layer(const GateUpParams &p, const FusedRouteParams &r,
                          const LayerDownParams &d, int grid, size_t smem, cudaStream_t s,
                          bool pdl);
+// ------------------------------------------------------------------------
+// The whole batch-1 decode step of a stack of layers in one persistent,
+// cooperative launch (stack.cu): one CTA per SM, every layer's RMSNorm,
+// router, top-k, gate/up + SwiGLU, down, combine and residual add, with the
+// three grid-wide hand-offs of a layer (layer input, router logits, h) done
+// through tagged 8-byte words {tag, value} in the workspace.
+constexpr int kStackMaxLayers = 64;
+constexpr int kStackThreads = 768;  // 24 warps: 23 gate/up consumers + a producer
+constexpr int kStackChunks = 4;     // gate/up copy groups per CTA, each with an mbarrier
+
+struct StackLayer {
+    const uint8_t *codes_base, *scales_base;  // contiguous [E][3][...], or null
+    const ExpertPtrs *table;                  // device expert table (codes_base null)
+    const uint16_t *router_w;                 // [E][H] BF16
+    const float *bias;                        // [E] or null
+};
+
+// Shared-memory plan of the stack kernel (host-computed, passed by value).
+struct StackPlan {
+    size_t smem;                         // dynamic shared memory bytes
+    unsigned off_gu, off_dn, off_rt, off_sx, off_x16, off_sh, off_so;
+    int np_max;   // gate/up row pairs of the largest CTA share
+    int ppc;      // row pairs per copy group
+    int R;        // down rows of the largest CTA share (a multiple of U)
+    int U;        // down rows per unit of the CTA split (2 or 4: 16-byte scale copies)
+};
+
+struct StackParams {
+    int L, E, H, I, k;
+    size_t codes_stride, scales_stride;   // bytes per matrix (contiguous layers)
+    uint16_t *r;                          // [H] residual stream, in and out
+    uint16_t *r_hist;                     // [L][H] each layer's input, or null
+    uint16_t *xn_hist;                    // [L][H] each layer's routed vector, or null
+    float *logits_hist;                   // [L][E] or null
+    int32_t *ids_hist;                    // [L][k] or null
+    float *w_hist;                        // [L][k] or null
+    // workspace
+    uint2 *x_tag;                         // [H/2] {tag, 2 x BF16} layer outputs
+    uint2 *lg_tag;                        // [E] {tag, FP32} router logits
+    uint2 *h_tag;                         // [k][I/2] {tag, 2 x BF16} SwiGLU outputs
+    unsigned *seq;                        // [grid] launches made by CTA b
+    unsigned *abort;                      // launch tag of a launch that gave up
+    unsigned *status;                     // device status bits
+    int spin_limit;                       // polls of a tagged-word wait before it gives up
+    StackPlan plan;
+    StackLayer layer[kStackMaxLayers];
+};
+
+// False when the shape is outside what the stack kernel holds (then the
+// layers run one by one).
+bool stack_plan(int E, int H, int I, int k, int grid, StackPlan *plan);
+cudaError_t launch_stack(const StackParams &p, int grid, cudaStream_t s);
+
 cudaError_t launch_debug_dequant(const uint8_t *codes, const uint8_t *scales, int64_t n,
                                  float *out, cudaStream_t s);
 size_t gateup_decode_smem(int T, int H);

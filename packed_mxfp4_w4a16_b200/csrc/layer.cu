@@ -427,10 +427,13 @@ namespace {
 template <int KCH, int TLD, int KCHD>
 cudaError_t launch_lk(const GateUpParams &p, const FusedRouteParams &r, const LayerDownParams &d,
                       int grid, size_t smem, cudaStream_t s, bool pdl) {
-    // once per process (thread-safe static initialisation)
-    static const cudaError_t smem_attr = cudaFuncSetAttribute(
-        layer_kernel<KCH, TLD, KCHD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-        (int)kFusedSmemBudget);
+    // once per device (the attribute belongs to the current device's context)
+    static PerDeviceOnce once;
+    const cudaError_t smem_attr = per_device_once(once, [] {
+        return cudaFuncSetAttribute(layer_kernel<KCH, TLD, KCHD>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kFusedSmemBudget);
+    });
     if (smem_attr != cudaSuccess) return smem_attr;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);

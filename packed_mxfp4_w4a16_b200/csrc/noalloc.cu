@@ -5,24 +5,24 @@
 // framework's memory pool or allocator callback, embedders whose device
 // memory is budgeted and accounted by someone else, or code paths that must
 // not allocate while other streams are being captured.  For them this entry
-// point keeps its scratch (the device expert table, the status word and the
-// SwiGLU activations h) in one file-scope device array of fixed size instead
-// of a caller-supplied workspace.  The kernels are the same ones moe_forward
-// runs.
+// point keeps its scratch (the device status word and the SwiGLU activations
+// h) in one file-scope device array of fixed size instead of a
+// caller-supplied workspace.  The kernels are the same ones moe_forward runs,
+// reading the experts from the contiguous weights' base address (no expert
+// table is needed).
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <string.h>
+
+#include <mutex>
 
 #include "../../include/moe_mxfp4.h"
 #include "kernels.cuh"
 
 namespace {
 
-constexpr size_t kTableBytes = (size_t)MOE_NOALLOC_MAX_EXPERTS * sizeof(moe::ExpertPtrs);
-static_assert(kTableBytes <= 12288, "expert table must fit its slot");
-constexpr size_t kTableOff = 0;
-constexpr size_t kStatusOff = 12288;
-constexpr size_t kHOff = kStatusOff + 256;
+constexpr size_t kStatusOff = 0;
+constexpr size_t kHOff = 256;
 constexpr size_t kScratchBytes = kHOff + (size_t)MOE_NOALLOC_MAX_H_BYTES;
 static_assert(kScratchBytes == MOE_NOALLOC_SCRATCH_BYTES, "scratch size as declared");
 
@@ -30,34 +30,48 @@ static_assert(kScratchBytes == MOE_NOALLOC_SCRATCH_BYTES, "scratch size as decla
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-uint8_t *g_scratch_addr[kMaxDevices];  // device address of g_noalloc_scratch per device
-int g_sms[kMaxDevices];
+struct DeviceScratch {
+    std::once_flag once;
+    int rc = MOE_ERR_CUDA;
+    uint8_t *addr = nullptr;  // device address of g_noalloc_scratch on this device
+    int sms = 0;
+};
+DeviceScratch g_dev[kMaxDevices];
 
-// Per device, once, with that device current: the symbol's device address.
+// Per device, once (thread-safe), with that device current: the symbol's
+// device address and the SM count.
 int scratch_for_current_device(uint8_t **base, int *sms) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
         cudaGetLastError();
         return MOE_ERR_CUDA;
     }
-    if (!g_scratch_addr[dev]) {
+    DeviceScratch &d = g_dev[dev];
+    std::call_once(d.once, [&d, dev] {
         int major = 0, n = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
             cudaGetLastError();
-            return MOE_ERR_CUDA;
+            d.rc = MOE_ERR_CUDA;
+            return;
         }
-        if (major != 10) return MOE_ERR_UNSUPPORTED;
+        if (major != 10) {
+            d.rc = MOE_ERR_UNSUPPORTED;
+            return;
+        }
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
             cudaGetLastError();
-            return MOE_ERR_CUDA;
+            d.rc = MOE_ERR_CUDA;
+            return;
         }
-        g_sms[dev] = n;
-        g_scratch_addr[dev] = static_cast<uint8_t *>(p);
-    }
-    *base = g_scratch_addr[dev];
-    *sms = g_sms[dev];
+        d.sms = n;
+        d.addr = static_cast<uint8_t *>(p);
+        d.rc = MOE_OK;
+    });
+    if (d.rc != MOE_OK) return d.rc;
+    *base = d.addr;
+    *sms = d.sms;
     return MOE_OK;
 }
 
@@ -71,7 +85,6 @@ extern "C" int moe_forward_noalloc(int E, int H, int I, int top_k, const uint8_t
                                    const uint16_t *residual, uint16_t *y, void *stream) {
     if (E < 1 || H < 32 || I < 32 || H % 32 || I % 32 || H > 4096 || I > 4096) return MOE_ERR_ARG;
     if (top_k < 1 || top_k > moe::kMaxTopK || top_k > E || T < 1) return MOE_ERR_ARG;
-    if (E > MOE_NOALLOC_MAX_EXPERTS) return MOE_ERR_WORKSPACE;
     if ((size_t)T * top_k * I * 2 > (size_t)MOE_NOALLOC_MAX_H_BYTES) return MOE_ERR_WORKSPACE;
     if (!codes_u8 || !scales_e8m0 || !x || !topk_ids || !topk_w || !y || y == x) return MOE_ERR_ARG;
     if (!aligned16(codes_u8) || !aligned16(scales_e8m0) || !aligned16(x) || !aligned16(y) ||
@@ -88,22 +101,8 @@ extern "C" int moe_forward_noalloc(int E, int H, int I, int top_k, const uint8_t
     const size_t mc = (size_t)I * H / 2, ms = (size_t)I * H / 32;
     if (ms % 16) return MOE_ERR_ALIGN;
 
-    // expert table for this call's weights, built on the host stack
-    moe::ExpertPtrs table[MOE_NOALLOC_MAX_EXPERTS];
-    for (int e = 0; e < E; ++e)
-        for (int m = 0; m < 3; ++m) {
-            table[e].codes[m] = codes_u8 + ((size_t)e * 3 + m) * mc;
-            table[e].scales[m] = scales_e8m0 + ((size_t)e * 3 + m) * ms;
-        }
-    moe::ExpertPtrs *d_table = reinterpret_cast<moe::ExpertPtrs *>(base + kTableOff);
     unsigned *d_status = reinterpret_cast<unsigned *>(base + kStatusOff);
     uint16_t *d_h = reinterpret_cast<uint16_t *>(base + kHOff);
-    if (cudaMemcpyAsync(d_table, table, sizeof(moe::ExpertPtrs) * (size_t)E, cudaMemcpyHostToDevice,
-                        s) != cudaSuccess ||
-        cudaMemsetAsync(d_status, 0, sizeof(unsigned), s) != cudaSuccess) {
-        cudaGetLastError();
-        return MOE_ERR_CUDA;
-    }
 
     // same per-(token, slot) GEMV path as moe_forward, in token chunks sized so
     // that the down kernel's staged activations fit in shared memory
@@ -116,7 +115,7 @@ extern "C" int moe_forward_noalloc(int E, int H, int I, int top_k, const uint8_t
     for (int t0 = 0; t0 < T; t0 += chunk) {
         const int Tc = (T - t0 < chunk) ? T - t0 : chunk;
         moe::GateUpParams g = {};
-        g.table = d_table;
+        g.table = nullptr;  // experts addressed from the contiguous base
         g.codes_base = codes_u8;
         g.scales_base = scales_e8m0;
         g.codes_stride = mc;
@@ -144,7 +143,7 @@ extern "C" int moe_forward_noalloc(int E, int H, int I, int top_k, const uint8_t
             return MOE_ERR_CUDA;
         }
         moe::DownParams d = {};
-        d.table = d_table;
+        d.table = nullptr;
         d.codes_base = codes_u8;
         d.scales_base = scales_e8m0;
         d.codes_stride = mc;
@@ -170,5 +169,25 @@ extern "C" int moe_forward_noalloc(int E, int H, int I, int top_k, const uint8_t
             return MOE_ERR_CUDA;
         }
     }
+    return MOE_OK;
+}
+
+extern "C" int moe_forward_noalloc_status(void *stream, unsigned *device_status) {
+    if (!device_status) return MOE_ERR_ARG;
+    uint8_t *base = nullptr;
+    int sms = 0;
+    int rc = scratch_for_current_device(&base, &sms);
+    if (rc != MOE_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned *d_status = reinterpret_cast<unsigned *>(base + kStatusOff);
+    unsigned v = 0;
+    if (cudaStreamSynchronize(s) != cudaSuccess ||
+        cudaMemcpyAsync(&v, d_status, sizeof v, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemsetAsync(d_status, 0, sizeof v, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess) {
+        cudaGetLastError();
+        return MOE_ERR_CUDA;
+    }
+    *device_status = v;
     return MOE_OK;
 }

@@ -57,6 +57,12 @@ def assert_close_rms(gpu_u16, ref_u16, tol=TOL, what="", max_ulps=1, max_flip_fr
     ulps = ulp_distance(gpu_u16, ref_u16)
     flip = (~within) & (ulps <= max_ulps)
     bad = (~within) & ~flip
+    worst = int(ulps.max()) if ulps.size else 0
+    if what:
+        # observed distances, so that any loosening of a rule shows in the log
+        print(f"[parity] {what}: {gpu_u16.size} elements, {int(np.count_nonzero(g != r))} "
+              f"differ, {int(flip.sum())} rounding flips beyond tol, worst {worst} ulp, "
+              f"max err {float((err / rms).max()):.2e} x rms")
     assert not np.any(bad), (f"{what}: {bad.sum()} elements beyond tolerance, worst "
                              f"{(err / rms)[bad].max():.3e} x rms, {ulps[bad].max()} ulps")
     assert flip.mean() <= max_flip_frac, f"{what}: flip fraction {flip.mean():.4f}"

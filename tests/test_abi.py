@@ -127,3 +127,68 @@ def test_status_strings(lib):
         s = lib.moe_status_string(code).decode()
         assert s.startswith("MOE_")
     assert lib.moe_status_string(-99).decode() == "unknown moe status"
+
+
+def test_stack_calls_validate_on_the_host(lib):
+    """moe_stack_* refuse bad arguments before any device work."""
+    out = C.c_void_p(123)
+    assert lib.moe_stack_create(None, 1, None, None, C.byref(out)) == -1 and out.value is None
+    h = C.c_void_p()
+    assert lib.moe_create(64, 2048, 1536, 4, C.byref(h)) == 0
+    try:
+        arr = (C.c_void_p * 1)(h.value)
+        rws = (C.c_void_p * 1)(None)
+        assert lib.moe_stack_create(arr, 0, rws, None, C.byref(out)) == -1
+        assert lib.moe_stack_create(arr, 65, rws, None, C.byref(out)) == -1
+        # weights not bound yet
+        assert lib.moe_stack_create(arr, 1, rws, None, C.byref(out)) == -2
+        assert lib.moe_stack_create(arr, 1, rws, None, None) == -1
+    finally:
+        lib.moe_destroy(h)
+    assert lib.moe_stack_destroy(None) == 0
+    assert lib.moe_stack_decode(None, None, None, None, None, None, None, None) == -1
+    assert lib.moe_stack_set_spin_limit(None, 0) == -1
+    n = C.c_size_t()
+    assert lib.moe_stack_workspace_bytes(None, C.byref(n)) == -1
+    st = C.c_uint()
+    assert lib.moe_stack_get_status(None, None, C.byref(st)) == -1
+    assert lib.moe_forward_noalloc_status(None, None) == -1
+
+
+def test_noalloc_wrapper_checks_every_tensor_against_the_shape():
+    """The Python wrapper of moe_forward_noalloc checks sizes, dtypes,
+    contiguity and device of every tensor before the C call (which takes bare
+    pointers): here on CPU tensors against device 'cpu'."""
+    import torch
+
+    import packed_mxfp4_w4a16_b200 as moe
+    E, H, I, k, T = 4, 64, 32, 2, 3
+    t = dict(codes=torch.zeros(E * 3 * I * H // 2, dtype=torch.uint8),
+             scales=torch.zeros(E * 3 * I * H // 32, dtype=torch.uint8),
+             x=torch.zeros(T, H, dtype=torch.bfloat16),
+             topk_ids=torch.zeros(T, k, dtype=torch.int32),
+             topk_w=torch.zeros(T, k, dtype=torch.float32),
+             residual=None, y=torch.zeros(T, H, dtype=torch.bfloat16))
+
+    def run(**over):
+        a = dict(t, **over)
+        return moe._noalloc_args_ok(E, H, I, k, a["codes"], a["scales"], a["x"], a["topk_ids"],
+                                    a["topk_w"], a["residual"], a["y"], device="cpu")
+
+    assert run() == T
+    assert run(residual=torch.zeros(T, H, dtype=torch.bfloat16)) == T
+    bad = [dict(codes=t["codes"][:-1]), dict(scales=torch.zeros(7, dtype=torch.uint8)),
+           dict(x=torch.zeros(T, H + 32, dtype=torch.bfloat16)),
+           dict(x=torch.zeros(T, H, dtype=torch.float32)),
+           dict(topk_ids=torch.zeros(T, k + 1, dtype=torch.int32)),
+           dict(topk_ids=torch.zeros(T, k, dtype=torch.int64)),
+           dict(topk_w=torch.zeros(T - 1, k, dtype=torch.float32)),
+           dict(y=torch.zeros(T + 1, H, dtype=torch.bfloat16)),
+           dict(y=torch.zeros(H, T, dtype=torch.bfloat16).t()),
+           dict(residual=torch.zeros(T, H - 32, dtype=torch.bfloat16))]
+    for over in bad:
+        with pytest.raises(moe.MoEError):
+            run(**over)
+    with pytest.raises(moe.MoEError):  # tensors on another device than asked
+        moe._noalloc_args_ok(E, H, I, k, t["codes"], t["scales"], t["x"], t["topk_ids"],
+                             t["topk_w"], None, t["y"], device="meta")

@@ -125,12 +125,21 @@ def test_layer_end_to_end(shape, T):
         y = layer.forward(xd, ids, w)
         torch.cuda.synchronize()
         rids, rw, rlg = oracle.route(x, L.router_w, L.router_b, shape.top_k)
-        ties = check_routing(ids.cpu().numpy(), w.cpu().numpy(), logits.cpu().numpy(), rids,
-                             rw, rlg, shape.top_k)
-        if ties == 0:
-            _, _, y_r = oracle.moe_layer(x, L.router_w, L.router_b, L.codes, L.scales, shape.E,
-                                         shape.H, shape.I, shape.top_k)
-            assert_close_rms(host_bf16(y), y_r, what="layer y", max_ulps=2)
+        ids_g, w_g = ids.cpu().numpy(), w.cpu().numpy()
+        ties = check_routing(ids_g, w_g, logits.cpu().numpy(), rids, rw, rlg, shape.top_k)
+        if ties:
+            # a near-tie token may legitimately pick other experts (the GPU's
+            # own selection was checked above): its y is compared with the
+            # oracle's forward under the GPU's routing, the others' with the
+            # oracle's whole layer
+            print(f"[parity] layer y seed {seed}: {ties} near-tie token(s) of {T}")
+        _, _, y_r = oracle.moe_layer(x, L.router_w, L.router_b, L.codes, L.scales, shape.E,
+                                     shape.H, shape.I, shape.top_k)
+        y_own = oracle.moe_forward(x, ids_g, w_g.astype(np.float64), L.codes, L.scales, shape.E,
+                                   shape.H, shape.I)
+        same = np.all(ids_g == rids, axis=1)
+        y_ref = np.where(same[:, None], y_r, y_own)
+        assert_close_rms(host_bf16(y), y_ref, what="layer y", max_ulps=2)
         layer.close()
 
 

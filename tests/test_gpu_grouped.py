@@ -42,10 +42,11 @@ def _check(L, layer, x, ids, w, shape, flags=0, residual=None):
     # h = BF16(BF16(silu(BF16(g))) * BF16(u)): a one-ulp flip of g or u near a
     # rounding midpoint (different FP32 summation order on the tensor cores)
     # carries through silu and the product; when g and u both flip, s can move
-    # two ulps and h (and o after it) land three BF16 values away; such flips
-    # stay rare (at most 1 % of the elements)
+    # two ulps and h land three BF16 values away; such flips stay rare (at most
+    # 1 % of the elements).  o sums I such h terms, so one rare h flip moves it
+    # far less than an ulp: o keeps the decode path's rule (one-ulp flips).
     assert_close_rms(h_g[valid], h_r[valid], what="grouped h", max_ulps=3)
-    assert_close_rms(o_g[valid], o_r[valid], what="grouped o", max_ulps=3)
+    assert_close_rms(o_g[valid], o_r[valid], what="grouped o", max_ulps=1)
     # y is a function of o alone (the bit-exact combine check below), so its
     # distance to the oracle's y is bounded by the o differences through the
     # routing weights plus the two combines' own roundings (the kernel's and
@@ -62,6 +63,8 @@ def _check(L, layer, x, ids, w, shape, flags=0, residual=None):
     bound = 1.01 * (wa * np.abs(og - orr)).sum(axis=1) + 2 * (2 * k + 1) * scale * 2.0 ** -8
     dy = np.abs(f64(y_g) - f64(y_r))
     assert np.all(dy <= bound), f"grouped y: {(dy > bound).sum()} elements beyond the o-derived bound"
+    # and the decode path's rule for y: 1e-2 rms, rare flips of at most two ulps
+    assert_close_rms(y_g, y_r, what="grouped y", max_ulps=2)
     # combine in slot order, bit-exact given the kernel's own expert outputs
     for t in range(T):
         o_t = np.where(valid[t][:, None], o_g[t], 0).astype(np.uint16)

@@ -59,6 +59,32 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     w = torch.zeros(T, 4, dtype=torch.float32, device="cuda")
     y = torch.empty_like(x)
     assert _call_raw(shape, codes, scales, x, ids, w, None, y) == -5  # MOE_ERR_WORKSPACE
-    big = synth.LayerShape(E=300, H=64, I=64, top_k=4)
-    assert _call_raw(big, codes, scales, x[:1, :64].contiguous(), ids[:1], w[:1], None,
-                     y[:1, :64].contiguous()) == -5
+
+
+def test_noalloc_reports_a_bad_expert_id_through_its_status_word():
+    """An id outside [0, E) zeroes that slot and sets MOE_DEVICE_BAD_EXPERT_ID
+    in the scratch's status word, read (and cleared) by
+    moe_forward_noalloc_status; the other slots still match the workspace
+    forward given the same ids."""
+    shape = synth.TINY
+    T = 2
+    L = synth.make_layer(shape, seed=43)
+    codes, scales, rw, _ = dev_layer(L)
+    layer = moe.MoELayer(shape.E, shape.H, shape.I, shape.top_k, codes, scales, rw, None,
+                         max_tokens=T)
+    x = dev_bf16(synth.make_tokens(T, shape.H, seed=43))
+    ids_h, w_h = synth.make_routing(T, shape.E, shape.top_k, "uniform", synth.rng_for(43, 1))
+    assert moe.moe_forward_noalloc_status() == 0
+    ids_h = ids_h.copy()
+    ids_h[1, 2] = shape.E + 3
+    ids, w = torch.from_numpy(ids_h).cuda(), torch.from_numpy(w_h).cuda()
+    y = torch.empty_like(x)
+    moe.moe_forward_noalloc(shape.E, shape.H, shape.I, shape.top_k, codes, scales, x, ids, w,
+                            None, y)
+    assert moe.moe_forward_noalloc_status() & moe.DEVICE_BAD_EXPERT_ID
+    assert moe.moe_forward_noalloc_status() == 0  # cleared by the read
+    ref = layer.forward(x, ids, w)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host_bf16(y), host_bf16(ref))
+    assert layer.status() & moe.DEVICE_BAD_EXPERT_ID
+    layer.close()
