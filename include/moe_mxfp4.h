@@ -380,6 +380,18 @@ MOE_API int moe_stack_get_status(moe_stack_t s, void *stream, unsigned *device_s
  * outlives a launch that gave up.  Errors: ARG. */
 MOE_API int moe_stack_set_spin_limit(moe_stack_t s, int polls);
 
+/* Profiling hook: when trace is a device buffer of at least
+ * n_layers * SMs * 16 * 8 bytes (SMs = the device's multiprocessor count),
+ * every later moe_stack_decode writes, per layer l and CTA b, sixteen
+ * global-timer stamps (ns) at trace[(l * SMs + b) * 16 + slot]: 0 layer
+ * start, 1 layer input gathered, 2 router logit published, 3 all logits
+ * gathered, 10 top-k done, 4 down-row copies issued, 9 first gate/up rows
+ * loaded (thread 0), 5 gate/up of the CTA done, 6 all of h gathered,
+ * 15 h staged, 7 down GEMV done, 8 layer output published; slots 11..14
+ * unused.  NULL turns it off.
+ * Errors: ARG, WORKSPACE (buffer too small), NOT_DEVICE, ALIGN. */
+MOE_API int moe_stack_set_trace(moe_stack_t s, unsigned long long *trace, size_t bytes);
+
 /* ---------------------------------------------------------------------
  * Forward without any device allocation.  No counterpart in the paper: this
  * entry point exists for callers that may not call cudaMalloc -- code that

@@ -29,7 +29,7 @@ __all__ = [
     "moe_bytes_per_expert", "moe_set_tuning", "moe_device_check", "moe_debug_dequant",
     "moe_forward_noalloc", "moe_forward_noalloc_status", "moe_stack_create", "moe_stack_destroy", "moe_stack_workspace_bytes",
     "moe_stack_set_workspace", "moe_stack_decode", "moe_stack_get_status",
-    "moe_stack_set_spin_limit",
+    "moe_stack_set_spin_limit", "moe_stack_set_trace", "STACK_TRACE_SLOTS",
     "ROUTE_RMSNORM", "ROUTE_SIGMOID", "FWD_KEEP_INTERMEDIATES", "FWD_FORCE_DECODE", "FWD_FORCE_GROUPED",
     "FWD_PHASE_GATEUP", "FWD_PHASE_DOWN", "FWD_FORCE_TCGEN05", "FWD_FORCE_MMA",
     "FUSION_NONE", "FUSION_ROUTER", "FUSION_LAYER", "moe_set_fusion",
@@ -308,6 +308,20 @@ def moe_stack_get_status(s: int, stream=None) -> int:
     v = C.c_uint()
     check("moe_stack_get_status", load().moe_stack_get_status(C.c_void_p(s), _s(stream), C.byref(v)))
     return v.value
+
+
+STACK_TRACE_SLOTS = 16
+
+
+def moe_stack_set_trace(s: int, trace) -> None:
+    """trace: device int64 tensor of n_layers * SMs * STACK_TRACE_SLOTS
+    elements (phase time stamps of every later decode), or None."""
+    if trace is None:
+        check("moe_stack_set_trace", load().moe_stack_set_trace(C.c_void_p(s), None, 0))
+        return
+    _need(trace, torch.int64, "moe_stack_set_trace")
+    check("moe_stack_set_trace",
+          load().moe_stack_set_trace(C.c_void_p(s), _p(trace), trace.numel() * 8))
 
 
 def moe_stack_set_spin_limit(s: int, polls: int) -> None:

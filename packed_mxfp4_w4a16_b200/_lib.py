@@ -51,6 +51,7 @@ SIGNATURES = [
     ("moe_stack_decode", _i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     ("moe_stack_get_status", _i, [_vp, _vp, C.POINTER(_u)]),
     ("moe_stack_set_spin_limit", _i, [_vp, _i]),
+    ("moe_stack_set_trace", _i, [_vp, _vp, _sz]),
 ]
 
 

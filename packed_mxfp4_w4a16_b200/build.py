@@ -21,6 +21,9 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden",
          "-I", os.path.join(ROOT, "include"), "--expt-relaxed-constexpr"]
+# developer knob: extra nvcc flags (e.g. -D tuning macros) for experiments;
+# a build with them should be forced (build(force=True)) and not shipped
+EXTRA = os.environ.get("MOE_NVCC_FLAGS", "").split()
 
 
 def sources():
@@ -42,7 +45,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         obj = os.path.join(BUILD, os.path.basename(src) + ".o")
         objs.append(obj)
         if force or _stale(obj, [src, *headers]):
-            cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj]
+            cmd = [NVCC, *ARCH, *FLAGS, *EXTRA, "-c", src, "-o", obj]
             if verbose:
                 cmd.insert(1, "-Xptxas=-v")
             subprocess.run(cmd, check=True)

@@ -776,6 +776,7 @@ struct moe_stack_ctx {
     uint8_t *ws = nullptr;
     size_t ws_bytes = 0;
     int spin_limit = moe::kMaxSpin;
+    unsigned long long *trace = nullptr;
     moe::StackPlan plan = {};
     moe::StackLayer layer[moe::kStackMaxLayers] = {};
 };
@@ -886,6 +887,22 @@ int moe_stack_set_spin_limit(moe_stack_t s, int polls) {
     return MOE_OK;
 }
 
+int moe_stack_set_trace(moe_stack_t s, unsigned long long *trace, size_t bytes) {
+    if (!s) return MOE_ERR_ARG;
+    if (!trace) {
+        s->trace = nullptr;
+        return MOE_OK;
+    }
+    const size_t need = (size_t)s->L * s->num_sms * moe::kStackTraceSlots * sizeof(unsigned long long);
+    if (bytes < need) return MOE_ERR_WORKSPACE;
+    moe_ctx probe;
+    probe.device = s->device;
+    int rc;
+    if ((rc = check_device_ptr(&probe, trace, 8)) != MOE_OK) return rc;
+    s->trace = trace;
+    return MOE_OK;
+}
+
 int moe_stack_decode(moe_stack_t s, uint16_t *r, uint16_t *r_hist, uint16_t *xn_hist,
                      float *logits, int32_t *topk_ids, float *topk_w, void *stream) {
     if (!s) return MOE_ERR_ARG;
@@ -928,6 +945,7 @@ int moe_stack_decode(moe_stack_t s, uint16_t *r, uint16_t *r_hist, uint16_t *xn_
     p.abort = reinterpret_cast<unsigned *>(s->ws + W.abort);
     p.status = reinterpret_cast<unsigned *>(s->ws + W.status);
     p.spin_limit = s->spin_limit;
+    p.trace = s->trace;
     p.plan = s->plan;
     for (int l = 0; l < s->L; ++l) p.layer[l] = s->layer[l];
     return cuda_rc(moe::launch_stack(p, s->num_sms, static_cast<cudaStream_t>(stream)));

@@ -48,6 +48,23 @@ __device__ __forceinline__ uint4 ld_stream16(const void *p) {
     return r;
 }
 
+// The same with an L2 eviction policy (createpolicy) for the source lines.
+// Volatile: issued where written (a batch of these is meant to be in flight
+// before the first result is used; a plain asm could be sunk to its use).
+__device__ __forceinline__ uint4 ld_stream16_hint(const void *p, uint64_t pol) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p), "l"(pol));
+    return r;
+}
+__device__ __forceinline__ uint32_t ld_stream_u8_hint(const uint8_t *p, uint64_t pol) {
+    uint16_t r;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.u8 %0, [%1], %2;" : "=h"(r)
+                 : "l"(p), "l"(pol));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t ld_stream_u8(const uint8_t *p) {
     uint16_t r;
     asm("ld.global.nc.L1::no_allocate.u8 %0, [%1];" : "=h"(r) : "l"(p));

@@ -210,7 +210,8 @@ static __device__ __noinline__ bool stage_h_tagged(const uint2 *h_tag, int P, in
 // reduced.  Rows come from shared memory (SR: copied there by issue_down_rows)
 // or are streamed from global memory.  The expert output BF16(o) of row r and
 // slot j goes to so[j R + (r - r0)].
-template <int TL, int KCH, bool SR, bool NV = false>
+// NW: warps of the CTA that take part (all of them).
+template <int TL, int KCH, bool SR, bool NV = false, int NW = kDownWarps>
 struct DownRows {
     int H, I, k, E, C, R, r0, r1, tps, j, lt, rr;
     unsigned mask;
@@ -235,7 +236,7 @@ struct DownRows {
         rs = (size_t)I >> (NV ? 4 : 5);
         lt = lane & (TL - 1);
         mask = team_mask<TL>(lane);
-        const int groups = kDownWarps / k;  // warps per slot
+        const int groups = NW / k;  // warps per slot
         j = warp % k;
         const int gi = warp / k;
         tps = groups * TPW;  // teams per slot

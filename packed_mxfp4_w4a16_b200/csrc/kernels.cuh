@@ -209,8 +209,8 @@ cudaError_t launch_layer(const GateUpParams &p, const FusedRouteParams &r,
 // three grid-wide hand-offs of a layer (layer input, router logits, h) done
 // through tagged 8-byte words {tag, value} in the workspace.
 constexpr int kStackMaxLayers = 64;
-constexpr int kStackThreads = 768;  // 24 warps: 23 gate/up consumers + a producer
-constexpr int kStackChunks = 4;     // gate/up copy groups per CTA, each with an mbarrier
+constexpr int kStackThreads = 512;  // 16 warps: 128 registers per thread
+constexpr int kStackTraceSlots = 16;  // phase time stamps per layer and CTA (profiling)
 
 struct StackLayer {
     const uint8_t *codes_base, *scales_base;  // contiguous [E][3][...], or null
@@ -224,7 +224,7 @@ struct StackPlan {
     size_t smem;                         // dynamic shared memory bytes
     unsigned off_gu, off_dn, off_rt, off_sx, off_x16, off_sh, off_so;
     int np_max;   // gate/up row pairs of the largest CTA share
-    int ppc;      // row pairs per copy group
+    int ppc;      // row pairs per code piece
     int R;        // down rows of the largest CTA share (a multiple of U)
     int U;        // down rows per unit of the CTA split (2 or 4: 16-byte scale copies)
 };
@@ -246,6 +246,7 @@ struct StackParams {
     unsigned *abort;                      // launch tag of a launch that gave up
     unsigned *status;                     // device status bits
     int spin_limit;                       // polls of a tagged-word wait before it gives up
+    unsigned long long *trace;            // [L][grid][kStackTraceSlots] time stamps, or null
     StackPlan plan;
     StackLayer layer[kStackMaxLayers];
 };

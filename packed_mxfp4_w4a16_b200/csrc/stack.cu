@@ -58,122 +58,135 @@ namespace moe {
 namespace {
 
 constexpr int kSWarps = kStackThreads / 32;   // 24
-constexpr int kSProd = kSWarps - 1;           // producer warp
-constexpr int kSCons = kSWarps - 1;           // gate/up consumer warps
 constexpr int kSRouteWarps = kRouteThreads / 32;
 constexpr size_t kStackSmemMax = 220 * 1024;  // dynamic; static shared memory is ~1.3 KB
 
-static_assert(kStackThreads == kDownThreads, "the down phase uses the down kernel's team layout");
+static_assert(kStackThreads % 32 == 0 && kSWarps >= kSRouteWarps, "whole warps, router warps included");
 
 // Tag of step l of a launch: 26 bits of launch count, 6 bits of layer.
 __device__ __forceinline__ unsigned stk_tag(unsigned base, int l) {
     return (base << 6) | (unsigned)l;
 }
 
-// Bounded poll of two adjacent tagged words (one 16-byte load of two
-// single-copy-atomic 8-byte words) until both carry `tag`.  Gives up after
-// `limit` polls, or early when the launch was aborted by another CTA.
-__device__ __forceinline__ bool stk_poll2(const uint2 *p, unsigned tag, uint32_t &d0,
-                                          uint32_t &d1, int limit, const unsigned *abort,
-                                          unsigned base) {
-    #pragma unroll 1
-    for (int i = 0; i < limit; ++i) {
-        uint2 a, c;
-        ld_relaxed_gpu_2x64(p, a, c);
-        if (a.x == tag && c.x == tag) {
-            d0 = a.y;
-            d1 = c.y;
-            return true;
-        }
-        if ((i & 7) == 7 && ld_relaxed_gpu(abort) == base) return false;
-        __nanosleep(32);
-    }
-    return false;
+constexpr int kAbortEvery = 256;   // polling rounds between two looks at the abort word
+#ifndef MOE_STACK_POLL_SLEEP
+#define MOE_STACK_POLL_SLEEP 64
+#endif
+constexpr int kPollSleepNs = MOE_STACK_POLL_SLEEP;  // back-off between polling rounds (ns)
+constexpr int kXThreads = 64;      // threads that gather the layer input
+constexpr int kHThreads = 256;     // threads that gather h
+#ifndef MOE_STACK_PIECES
+#define MOE_STACK_PIECES 4
+#endif
+constexpr int kStackPieces = MOE_STACK_PIECES;  // gate/up code pieces per CTA, landing in order
+constexpr int kPollMaxJ = 4;       // pieces per polling thread
+
+__device__ __forceinline__ uint64_t stk_clock() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
 }
 
-// By one warp: all n tagged logits (bounded), copied into s_logits.  Every
-// lane returns the same verdict.  Out of line (once per layer).
+// By the calling thread t of nt polling threads: the 32-byte pieces
+// i = t, t + nt, ... < n of src (piece i = tagged words 4i .. 4i+3, two
+// single-copy-atomic 8-byte words per 16-byte load) until all four words of a
+// piece carry `tag`; put(i, values) receives each piece as it lands.  Every
+// round issues the loads of all pieces still missing at once, then checks
+// them; between rounds the thread sleeps, and every kAbortEvery rounds it
+// looks at the abort word (few threads poll, and rarely look there, so the
+// polling does not crowd L2).  False on timeout or abort.
+template <class Put>
+__device__ __forceinline__ bool poll_pieces(const uint2 *src, int n, int t, int nt, unsigned tag,
+                                            int limit, const unsigned *abort, unsigned base,
+                                            Put &&put) {
+    unsigned todo = 0;
+#pragma unroll
+    for (int j = 0; j < kPollMaxJ; ++j)
+        if (t + j * nt < n) todo |= 1u << j;
+    #pragma unroll 1
+    for (int r = 0; todo && r < limit; ++r) {
+        uint2 w[kPollMaxJ][4];
+#pragma unroll
+        for (int j = 0; j < kPollMaxJ; ++j)
+            if ((todo >> j) & 1u) {
+                const uint2 *q = src + 4 * (size_t)(t + j * nt);
+                ld_relaxed_gpu_2x64(q, w[j][0], w[j][1]);
+                ld_relaxed_gpu_2x64(q + 2, w[j][2], w[j][3]);
+            }
+#pragma unroll
+        for (int j = 0; j < kPollMaxJ; ++j)
+            if (((todo >> j) & 1u) && w[j][0].x == tag && w[j][1].x == tag && w[j][2].x == tag &&
+                w[j][3].x == tag) {
+                put(t + j * nt, make_uint4(w[j][0].y, w[j][1].y, w[j][2].y, w[j][3].y));
+                todo &= ~(1u << j);
+            }
+        if (!todo) break;
+        if (r % kAbortEvery == kAbortEvery - 1 && ld_relaxed_gpu(abort) == base) return false;
+        __nanosleep(kPollSleepNs);
+    }
+    return todo == 0;
+}
+
+// The layer input: pieces of x_tag -> sx (8 BF16 values per piece).  Out of
+// line, so the polling registers do not add to the GEMV loops'.
+static __device__ __noinline__ bool stk_gather_x(const uint2 *x_tag, int n, int t, unsigned tag,
+                                                 int limit, const unsigned *abort, unsigned base,
+                                                 uint4 *sx) {
+    return poll_pieces(x_tag, n, t, kXThreads, tag, limit, abort, base,
+                       [&](int i, uint4 v) { sx[i] = v; });
+}
+
+// All of h: pieces of h_tag -> the staged layout in shared memory (raw BF16,
+// converted after the barrier), and each vector's max |h| into s_hmax.  Out of
+// line.
+static __device__ __noinline__ bool stk_gather_h(const uint2 *h_tag, int total, int npc, int t,
+                                                 unsigned tag, int limit, const unsigned *abort,
+                                                 unsigned base, uint4 *sv, unsigned *s_hmax) {
+    return poll_pieces(h_tag, total, t, kHThreads, tag, limit, abort, base, [&](int i, uint4 v) {
+        const int q = i / npc;
+        const int pi = i - q * npc;
+        sv[q * npc + h_piece(pi >> 2, pi & 3)] = v;
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+        float m = 0.f;
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+            m = fmaxf(m, fmaxf(fabsf(bf16_to_f32(w4[r] & 0xFFFFu)), fabsf(bf16_to_f32(w4[r] >> 16))));
+        atomicMax(s_hmax + q, __float_as_uint(m));
+    });
+}
+
+// By one warp: all n (<= 256) tagged logits, copied into s_logits, with the
+// same round structure.  Every lane returns the same verdict.  Out of line.
 static __device__ __noinline__ bool stk_gather_logits(const uint2 *ent, int n, unsigned tag,
                                                       float *s_logits, int limit,
                                                       const unsigned *abort, unsigned base) {
     const int lane = threadIdx.x & 31;
-    unsigned seen = 0;  // entries j = lane + 32 s already copied (n <= 256)
+    unsigned todo = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        if (lane + 32 * j < n) todo |= 1u << j;
     #pragma unroll 1
-    for (int i = 0; i < limit; ++i) {
-        bool all = true;
-        #pragma unroll 1
-        for (int j = lane, s = 0; j < n; j += 32, ++s) {
-            if ((seen >> s) & 1u) continue;
-            const uint2 v = ld_relaxed_gpu_v2(ent + j);
-            if (v.x == tag) {
-                s_logits[j] = __uint_as_float(v.y);
-                seen |= 1u << s;
-            } else {
-                all = false;
+    for (int r = 0; r < limit; ++r) {
+        uint2 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if ((todo >> j) & 1u) v[j] = ld_relaxed_gpu_v2(ent + lane + 32 * j);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (((todo >> j) & 1u) && v[j].x == tag) {
+                s_logits[lane + 32 * j] = __uint_as_float(v[j].y);
+                todo &= ~(1u << j);
             }
-        }
-        if (__all_sync(0xffffffffu, all)) {
+        if (__all_sync(0xffffffffu, todo == 0)) {
             __syncwarp();
             return true;
         }
-        if ((i & 7) == 7 && __any_sync(0xffffffffu, ld_relaxed_gpu(abort) == base)) return false;
-        __nanosleep(32);
+        if (r % kAbortEvery == kAbortEvery - 1 &&
+            __shfl_sync(0xffffffffu, lane == 0 ? (int)(ld_relaxed_gpu(abort) == base) : 0, 0))
+            return false;
+        __nanosleep(kPollSleepNs);
     }
     return false;
-}
-
-// By one warp: bulk copies of the CTA's gate/up rows of the selected experts.
-// Copy group c covers the CTA's local row pairs [c ppc, (c+1) ppc); a group
-// spans one or more slots q (segments), each giving four copies (gate codes,
-// up codes, gate scales, up scales); the lane of (c, segment 0, matrix 0)
-// announces the group's bytes on gbar[c].  Shared-memory layout: gate codes
-// [NR][H/2], up codes [NR][H/2], gate scales [NR][H/32], up scales [NR][H/32].
-static __device__ __noinline__ void stk_issue_gateup(const uint8_t *cb, const uint8_t *sb,
-                                                     const ExpertPtrs *tab, size_t cstride,
-                                                     size_t sstride, const int *s_ids, int E,
-                                                     int H, int I, int pb0, int np, int ppc,
-                                                     int nch, int NR, uint8_t *gu,
-                                                     uint64_t *gbar) {
-    const int lane = threadIdx.x & 31;
-    const size_t rc = (size_t)H >> 1, rs = (size_t)H >> 5;
-    const uint64_t pol = l2_evict_first_policy();  // rows are read once per token
-    const int smax = (2 * ppc + I - 1) / I + 1;    // slots one group can touch
-    const int ntask = nch * smax * 4;
-    #pragma unroll 1
-    for (int task = lane; task < ntask; task += 32) {
-        const int c = task / (smax * 4), s = (task >> 2) % smax, m = task & 3;
-        const int lp0 = c * ppc, lp1 = min(np, lp0 + ppc);
-        const int g0 = 2 * (pb0 + lp0), g1 = 2 * (pb0 + lp1);  // global rows [g0, g1)
-        const int qa = g0 / I, qb = (g1 - 1) / I;
-        if (s == 0 && m == 0) {
-            unsigned bytes = 0;
-            #pragma unroll 1
-            for (int q = qa; q <= qb; ++q) {
-                const int e = s_ids[q];
-                const int n = min(g1, (q + 1) * I) - max(g0, q * I);
-                if (e >= 0 && e < E) bytes += (unsigned)(2 * n) * (unsigned)(rc + rs);
-            }
-            mbar_arrive_expect_tx(&gbar[c], bytes);
-        }
-        const int q = qa + s;
-        if (q > qb) continue;
-        const int e = s_ids[q];
-        if (e < 0 || e >= E) continue;
-        const int a = max(g0, q * I);
-        const int n = min(g1, (q + 1) * I) - a;
-        const size_t lr = (size_t)(a - 2 * pb0);  // local row
-        const size_t i0 = (size_t)(a - q * I);    // row of the matrix
-        const int mat = m & 1;                    // 0 gate, 1 up
-        if (m < 2) {
-            const uint8_t *src = cb ? cb + (size_t)(3 * e + mat) * cstride : tab[e].codes[mat];
-            bulk_g2s_hint(gu + ((size_t)mat * NR + lr) * rc, src + i0 * rc, (unsigned)(n * rc),
-                          &gbar[c], pol);
-        } else {
-            const uint8_t *src = cb ? sb + (size_t)(3 * e + mat) * sstride : tab[e].scales[mat];
-            bulk_g2s_hint(gu + 2 * (size_t)NR * rc + ((size_t)mat * NR + lr) * rs, src + i0 * rs,
-                          (unsigned)(n * rs), &gbar[c], pol);
-        }
-    }
 }
 
 // Router row e of a layer into shared memory (one bulk copy on *bar).
@@ -191,7 +204,92 @@ __device__ __forceinline__ float swiglu_h(float ag, float au, float xs) {
     return s * u;
 }
 
+// By one thread: every copy of the layer into shared memory, in the order the
+// CTA needs the bytes -- the gate/up scales (on *sbar), the gate/up code rows
+// in pieces of ppc row pairs (piece c on gbar[c]), then the down rows (on
+// *dbar).  Bulk copies issued one after another by one thread land in that
+// order at full bandwidth (issued together, they would share the memory
+// system and all land at the end), so the GEMVs of the first pieces run while
+// the later ones stream.  Gate/up layout: codes [2][NR][H/2] (gate, up), then
+// scales [2][NR][H/32]; down layout: codes [k][R][I/2], scales [k][R][I/32].
+// Out of line.
+static __device__ __noinline__ void stk_issue_layer(
+    const uint8_t *cb, const uint8_t *sb, const ExpertPtrs *tab, size_t cstride, size_t sstride,
+    const int *s_ids, int E, int H, int I, int k, int pb0, int np, int ppc, int NR, uint8_t *gu,
+    uint64_t *sbar, uint64_t *gbar, int r0, int r1, int R, uint8_t *rows_c, uint8_t *rows_s,
+    uint64_t *dbar, uint64_t pol) {
+    const size_t rc = (size_t)H >> 1, rs = (size_t)H >> 5;
+    auto codes = [&](int e, int m) {
+        return cb ? cb + (size_t)(3 * e + m) * cstride : tab[e].codes[m];
+    };
+    auto scales = [&](int e, int m) {
+        return cb ? sb + (size_t)(3 * e + m) * sstride : tab[e].scales[m];
+    };
+    // rows [g0, g1) of the flattened (slot, row) space, split by slot: f(q, e,
+    // first row a, count n, local row lr, matrix row i0) for every valid slot
+    auto segments = [&](int g0, int g1, auto &&f) {
+        #pragma unroll 1
+        for (int q = g0 / I; g1 > g0 && q <= (g1 - 1) / I; ++q) {
+            const int e = s_ids[q];
+            if (e < 0 || e >= E) continue;
+            const int a = max(g0, q * I);
+            const int n = min(g1, (q + 1) * I) - a;
+            f(e, (size_t)n, (size_t)(a - 2 * pb0), (size_t)(a - q * I));
+        }
+    };
+    const int g0 = 2 * pb0, g1 = 2 * (pb0 + np);
+    unsigned bytes = 0;
+    segments(g0, g1, [&](int, size_t n, size_t, size_t) { bytes += (unsigned)(2 * n * rs); });
+    mbar_arrive_expect_tx(sbar, bytes);
+    segments(g0, g1, [&](int e, size_t n, size_t lr, size_t i0) {
+        #pragma unroll 1
+        for (int m = 0; m < 2; ++m)
+            bulk_g2s_hint(gu + 2 * (size_t)NR * rc + ((size_t)m * NR + lr) * rs, scales(e, m) + i0 * rs,
+                          (unsigned)(n * rs), sbar, pol);
+    });
+    const int nch = (np + ppc - 1) / ppc;
+    #pragma unroll 1
+    for (int c = 0; c < nch; ++c) {
+        const int a0 = 2 * (pb0 + c * ppc), a1 = 2 * (pb0 + min(np, (c + 1) * ppc));
+        bytes = 0;
+        segments(a0, a1, [&](int, size_t n, size_t, size_t) { bytes += (unsigned)(2 * n * rc); });
+        mbar_arrive_expect_tx(&gbar[c], bytes);
+        segments(a0, a1, [&](int e, size_t n, size_t lr, size_t i0) {
+            #pragma unroll 1
+            for (int m = 0; m < 2; ++m)
+                bulk_g2s_hint(gu + ((size_t)m * NR + lr) * rc, codes(e, m) + i0 * rc,
+                              (unsigned)(n * rc), &gbar[c], pol);
+        });
+    }
+    const size_t drc = (size_t)I >> 1, drs = (size_t)I >> 5, dn = (size_t)(r1 - r0);
+    bytes = 0;
+    #pragma unroll 1
+    for (int j = 0; j < k; ++j) {
+        const int e = s_ids[j];
+        if (e >= 0 && e < E) bytes += (unsigned)(dn * (drc + drs));
+    }
+    mbar_arrive_expect_tx(dbar, bytes);
+    #pragma unroll 1
+    for (int j = 0; j < k && dn > 0; ++j) {
+        const int e = s_ids[j];
+        if (e < 0 || e >= E) continue;
+        bulk_g2s_hint(rows_c + (size_t)j * R * drc, codes(e, 2) + (size_t)r0 * drc,
+                      (unsigned)(dn * drc), dbar, pol);
+        bulk_g2s_hint(rows_s + (size_t)j * R * drs, scales(e, 2) + (size_t)r0 * drs,
+                      (unsigned)(dn * drs), dbar, pol);
+    }
+}
+
 }  // namespace
+
+// Phase time stamps (profiling): thread 0 (or the producer's lane 0) of every
+// CTA records the global timer at fixed points of each layer when p.trace is
+// given: [L][grid][kStackTraceSlots].
+#define STK_STAMP(slot)                                                                  \
+    do {                                                                                 \
+        if (p.trace && (tid == 0 || ((slot) == 3 || (slot) == 4 || (slot) >= 10)))       \
+            p.trace[((size_t)l * G + b) * kStackTraceSlots + (slot)] = stk_clock();      \
+    } while (0)
 
 // KCH: 16-byte chunks per lane of a gate/up row (H = 32 * 32 * KCH at most);
 // TLD / KCHD: the down phase's team of TLD lanes holding KCHD chunks each.
@@ -199,9 +297,10 @@ template <int KCH, int TLD, int KCHD>
 __global__ void __launch_bounds__(kStackThreads, 1)
 stack_decode_kernel(const __grid_constant__ StackParams p) {
     extern __shared__ __align__(128) uint8_t sm[];
-    __shared__ __align__(8) uint64_t gbar[kStackChunks];
-    __shared__ __align__(8) uint64_t dbar;
-    __shared__ __align__(8) uint64_t rbar[2];
+    __shared__ __align__(8) uint64_t sbar;                // gate/up scales
+    __shared__ __align__(8) uint64_t gbar[kStackPieces];  // gate/up code pieces
+    __shared__ __align__(8) uint64_t dbar;                // down rows
+    __shared__ __align__(8) uint64_t rbar[2];             // router rows (next layer ahead)
     __shared__ int s_ids[kMaxTopK];
     __shared__ float s_w[kMaxTopK];
     __shared__ float s_logits[kFusedMaxE];
@@ -211,39 +310,30 @@ stack_decode_kernel(const __grid_constant__ StackParams p) {
     __shared__ unsigned s_base;
     __shared__ int s_x16exp;
     __shared__ int s_fail;
-    __shared__ int s_gu_armed, s_dn_armed;  // layer whose gate/up / down copies were issued
+    __shared__ int s_copied;                // layer whose weight copies were issued
     __shared__ int s_rt_armed[2];           // layer whose router row went into buffer i
+    __shared__ StackLayer s_layers[kStackMaxLayers];  // the layer table, read once per launch
+    __shared__ float s_bias[kStackMaxLayers];         // router bias of expert b, every layer
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = (int)blockIdx.x, G = (int)gridDim.x;
     const int E = p.E, H = p.H, I = p.I, k = p.k, L = p.L;
-    const StackPlan &pl = p.plan;
-    const int C = H >> 5;                                   // 32-element chunks per gate/up row
-    const size_t rc = (size_t)H >> 1, rs = (size_t)H >> 5;  // gate/up row bytes: codes, scales
-    const int nch8 = H >> 3;                                // 16-byte pieces of a BF16 vector
+    const int nch8 = H >> 3;  // 16-byte pieces of a BF16 vector
     const int limit = p.spin_limit;
-    // this CTA's shares: gate/up row pairs [pb0, pb1), down rows [r0, r1)
+    // this CTA's shares: gate/up row pairs [pb0, pb0 + np), down rows [r0, r1)
     const int P = k * I / 2;
-    const int pb0 = (int)((long long)P * b / G), pb1 = (int)((long long)P * (b + 1) / G);
-    const int np = pb1 - pb0;
-    const int NU = H / pl.U;
-    const int r0 = pl.U * (int)((long long)NU * b / G);
-    const int r1 = pl.U * (int)((long long)NU * (b + 1) / G);
-    const int nch = (np + pl.ppc - 1) / pl.ppc;  // copy groups in use (same every layer)
-    const int NR = 2 * pl.np_max;
-    const int R = pl.R;
-    uint8_t *gu = sm + pl.off_gu;
-    uint8_t *rows_c = sm + pl.off_dn;                           // [k][R][I/2]
-    uint8_t *rows_s = rows_c + (size_t)k * R * ((size_t)I >> 1);  // [k][R][I/32]
-    uint16_t *rbuf = reinterpret_cast<uint16_t *>(sm + pl.off_rt);  // [2][H]
-    uint32_t *sx = reinterpret_cast<uint32_t *>(sm + pl.off_sx);    // [H/2] layer input
-    uint32_t *sx16 = reinterpret_cast<uint32_t *>(sm + pl.off_x16); // [H/2] FP16 routed vector
-    uint32_t *sh = reinterpret_cast<uint32_t *>(sm + pl.off_sh);    // [k][I/2] FP16 h
-    float *so = reinterpret_cast<float *>(sm + pl.off_so);          // [k][R] expert outputs
+    const int pb0 = (int)((long long)P * b / G);
+    const int np = (int)((long long)P * (b + 1) / G) - pb0;
+    const int NU = H / p.plan.U;
+    const int r0 = p.plan.U * (int)((long long)NU * b / G);
+    const int r1 = p.plan.U * (int)((long long)NU * (b + 1) / G);
+    uint16_t *rbuf = reinterpret_cast<uint16_t *>(sm + p.plan.off_rt);  // [2][H]
+    uint32_t *sx = reinterpret_cast<uint32_t *>(sm + p.plan.off_sx);    // [H/2] layer input
 
     if (tid == 0) {
+        mbar_init(&sbar, 1);
         #pragma unroll 1
-        for (int c = 0; c < kStackChunks; ++c) mbar_init(&gbar[c], 1);
+        for (int c = 0; c < kStackPieces; ++c) mbar_init(&gbar[c], 1);
         mbar_init(&dbar, 1);
         mbar_init(&rbar[0], 1);
         mbar_init(&rbar[1], 1);
@@ -252,13 +342,21 @@ stack_decode_kernel(const __grid_constant__ StackParams p) {
         // CTAs agree); written by the previous launch, complete before this one
         s_base = ld_relaxed_gpu(p.seq + b) + 1u;
         s_fail = 0;
-        s_gu_armed = s_dn_armed = -1;
+        s_copied = -1;
         s_rt_armed[0] = s_rt_armed[1] = -1;
+    }
+    // the layer table into shared memory (kernel parameters indexed by layer
+    // would be a constant-cache miss per layer), and this CTA's router bias of
+    // every layer (loaded in parallel now, off the per-layer critical path)
+    if (tid < L) {
+        s_layers[tid] = p.layer[tid];
+        const float *bias = p.layer[tid].bias;
+        s_bias[tid] = (bias && b < E) ? bias[b] : 0.f;
     }
     __syncthreads();
     const unsigned base = s_base;
-    if (warp == kSProd && lane == 0 && b < E) {
-        stk_issue_router(p.layer[0].router_w, b, H, rbuf, &rbar[0]);
+    if (warp == kSWarps - 1 && lane == 0 && b < E) {
+        stk_issue_router(s_layers[0].router_w, b, H, rbuf, &rbar[0]);
         s_rt_armed[0] = 0;
     }
 
@@ -266,7 +364,8 @@ stack_decode_kernel(const __grid_constant__ StackParams p) {
     #pragma unroll 1
     for (; l < L; ++l) {
         const unsigned tag = stk_tag(base, l);
-        const StackLayer &ly = p.layer[l];
+        const StackLayer &ly = s_layers[l];
+        STK_STAMP(0);
 
         // ---- A: layer input r -> sx ----
         bool ok = true;
@@ -274,17 +373,13 @@ stack_decode_kernel(const __grid_constant__ StackParams p) {
             const uint32_t *r32 = reinterpret_cast<const uint32_t *>(p.r);
             #pragma unroll 1
             for (int m = tid; m < (H >> 1); m += kStackThreads) sx[m] = r32[m];
-        } else {
-            #pragma unroll 1
-            for (int m2 = tid; m2 < (H >> 2); m2 += kStackThreads) {
-                uint32_t d0 = 0u, d1 = 0u;
-                if (!stk_poll2(p.x_tag + 2 * m2, tag - 1u, d0, d1, limit, p.abort, base)) ok = false;
-                sx[2 * m2] = d0;
-                sx[2 * m2 + 1] = d1;
-            }
-            if (tid == 0 && ld_relaxed_gpu(p.abort) == base) ok = false;
+        } else if (tid < kXThreads) {
+            // the previous layer's tagged outputs, 8 values per piece
+            ok = stk_gather_x(p.x_tag, H >> 3, tid, tag - 1u, limit, p.abort, base,
+                              reinterpret_cast<uint4 *>(sx));
         }
         if (!__syncthreads_and(ok)) break;
+        STK_STAMP(1);
         if (b == 0 && p.r_hist) {
             uint32_t *dst = reinterpret_cast<uint32_t *>(p.r_hist + (size_t)l * H);
             #pragma unroll 1
@@ -293,8 +388,8 @@ stack_decode_kernel(const __grid_constant__ StackParams p) {
 
         // ---- A: RMSNorm, router logit b, FP16 staging (threads of warps 0..7,
         // in the reduction order of the standalone router kernel) ----
-        float acc = 0.f, amax = 0.f;
         if (tid < kRouteThreads) {
+            uint32_t *sx16 = reinterpret_cast<uint32_t *>(sm + p.plan.off_x16);
             uint4 xv[2];
             float ss = 0.f;
 #pragma unroll
@@ -328,6 +423,7 @@ stack_decode_kernel(const __grid_constant__ StackParams p) {
                     if (c < nch8) wv[m] = wrow[c];
                 }
             }
+            float acc = 0.f, amax = 0.f;
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
                 const int c = tid + kRouteThreads * m;
@@ -361,7 +457,7 @@ stack_decode_kernel(const __grid_constant__ StackParams p) {
                 float logit = 0.f;
 #pragma unroll
                 for (int i = 0; i < kSRouteWarps; ++i) logit += s_red[1][i];
-                if (ly.bias) logit += ly.bias[b];
+                if (ly.bias) logit += s_bias[l];
                 st_relaxed_gpu_v2(p.lg_tag + b, tag, __float_as_uint(logit));
                 if (p.logits_hist) p.logits_hist[(size_t)l * E + b] = logit;
             }
@@ -386,11 +482,13 @@ stack_decode_kernel(const __grid_constant__ StackParams p) {
             if (tid == 0) s_x16exp = c16;
         }
         if (!__syncthreads_and(ok)) break;
+        STK_STAMP(2);
 
-        // ---- C: routing and every copy of the layer (producer warp) ----
-        if (warp == kSProd) {
+        // ---- C: routing (the last warp), then every copy of the layer (all) ----
+        if (warp == kSWarps - 1) {
             const bool got = stk_gather_logits(p.lg_tag, E, tag, s_logits, limit, p.abort, base);
             if (got) {
+                if (lane == 0) STK_STAMP(3);
                 int id;
                 float w;
                 warp_topk_any<true>(s_logits, E, k, lane, id, w);
@@ -400,158 +498,162 @@ stack_decode_kernel(const __grid_constant__ StackParams p) {
                     if (b == 0 && p.ids_hist) p.ids_hist[(size_t)l * k + lane] = id;
                     if (b == 0 && p.w_hist) p.w_hist[(size_t)l * k + lane] = w;
                 }
-                __syncwarp();
-                stk_issue_gateup(ly.codes_base, ly.scales_base, ly.table, p.codes_stride,
-                                 p.scales_stride, s_ids, E, H, I, pb0, np, pl.ppc, nch, NR, gu,
-                                 gbar);
-                __syncwarp();
-                if (lane == 0) {
-                    const DownSrc src = {ly.table, ly.codes_base, ly.scales_base, p.codes_stride,
-                                         p.scales_stride};
-                    issue_down_rows(src, E, H, I, k, s_ids, r0, r1, R, rows_c, rows_s, &dbar);
-                    s_gu_armed = l;
-                    s_dn_armed = l;
-                } else if (lane == 1 && b < E && l + 1 < L) {
+                if (lane == 0) STK_STAMP(10);
+                if (lane == 1 && b < E && l + 1 < L) {
                     const int nb = (l + 1) & 1;
-                    stk_issue_router(p.layer[l + 1].router_w, b, H, rbuf + (size_t)nb * H, &rbar[nb]);
+                    stk_issue_router(s_layers[l + 1].router_w, b, H, rbuf + (size_t)nb * H,
+                                     &rbar[nb]);
                     s_rt_armed[nb] = l + 1;
                 }
             } else if (lane == 0) {
                 s_fail = 1;
             }
         }
-        // consumers: this layer's activations while the routing is decided
-        uint32_t xw[KCH][16];
-#pragma unroll
-        for (int u = 0; u < KCH; ++u) {
-            const int c = lane + 32 * u;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint4 v = c < C ? reinterpret_cast<const uint4 *>(sx16)[c * 4 + q]
-                                      : make_uint4(0u, 0u, 0u, 0u);
-                xw[u][4 * q] = v.x;
-                xw[u][4 * q + 1] = v.y;
-                xw[u][4 * q + 2] = v.z;
-                xw[u][4 * q + 3] = v.w;
-            }
-        }
         __syncthreads();
         if (s_fail) break;
-        const float xs = pow2(s_x16exp);
+        const int ppc = p.plan.ppc;
+        const int NR = 2 * p.plan.np_max;
+        uint8_t *gu = sm + p.plan.off_gu;
+        if (tid == kStackThreads - 32) {
+            // the producer warp's lane 0: every copy of the layer, in order
+            uint8_t *rows_c = sm + p.plan.off_dn;
+            stk_issue_layer(ly.codes_base, ly.scales_base, ly.table, p.codes_stride, p.scales_stride,
+                            s_ids, E, H, I, k, pb0, np, ppc, NR, gu, &sbar, gbar, r0, r1, p.plan.R,
+                            rows_c, rows_c + (size_t)k * p.plan.R * ((size_t)I >> 1), &dbar,
+                            l2_evict_first_policy());
+            s_copied = l;
+            STK_STAMP(4);
+        }
 
-        // ---- D: gate/up + SwiGLU, one row pair per consumer warp ----
-        if (warp < kSCons) {
+        // ---- D: gate/up + SwiGLU, one row pair per warp per step, each as
+        // its code piece lands.  Lane l holds the 16-byte chunks l + 32 u
+        // (u < KCH) of each row, one E8M0 group each; sums in the order of the
+        // bulk-copy gate/up kernel. ----
+        {
+            const float xs = pow2(s_x16exp);
+            const uint4 *sx16 = reinterpret_cast<const uint4 *>(sm + p.plan.off_x16);
+            const int C = H >> 5;
+            const size_t rc = (size_t)H >> 1, rs = (size_t)H >> 5;
+            if (warp < np && !mbar_wait(&sbar, (unsigned)l & 1u)) ok = false;
             #pragma unroll 1
-            for (int pp = warp; pp < np; pp += kSCons) {
-                if (!mbar_wait(&gbar[pp / pl.ppc], (unsigned)l & 1u)) {
+            for (int pp = warp; pp < np && ok; pp += kSWarps) {
+                if (!mbar_wait(&gbar[pp / ppc], (unsigned)l & 1u)) {
                     ok = false;
                     break;
                 }
+                if (tid == 0 && pp == 0) STK_STAMP(9);
                 const int gr = 2 * (pb0 + pp);  // global row of the pair's first row
-                const int q = gr / I;
-                const int e = s_ids[q];
+                const int e = s_ids[gr / I];
                 const bool bad = e < 0 || e >= E;
-                float v[4];
+                const size_t lr = (size_t)(2 * pp);
+                float v[2][2];
 #pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                    const size_t lr = (size_t)(2 * pp + rr);
-                    uint4 cg[KCH], cu[KCH];
-                    uint32_t sg[KCH], su[KCH];
+                for (int rr = 0; rr < 2; ++rr)
 #pragma unroll
-                    for (int u = 0; u < KCH; ++u) {
-                        const int c = lane + 32 * u;
-                        if (c < C && !bad) {
-                            cg[u] = *reinterpret_cast<const uint4 *>(gu + lr * rc + (size_t)c * 16);
-                            cu[u] = *reinterpret_cast<const uint4 *>(gu + ((size_t)NR + lr) * rc +
-                                                                     (size_t)c * 16);
-                            sg[u] = gu[2 * (size_t)NR * rc + lr * rs + c];
-                            su[u] = gu[2 * (size_t)NR * rc + ((size_t)NR + lr) * rs + c];
-                        } else {
-                            cg[u] = cu[u] = make_uint4(0u, 0u, 0u, 0u);
-                            sg[u] = su[u] = 127u;
+                    for (int m = 0; m < 2; ++m) v[rr][m] = 0.f;
+#pragma unroll
+                for (int u = 0; u < KCH; ++u) {
+                    const int c = lane + 32 * u;
+                    uint4 cw[2][2];
+                    uint32_t sw[2][2];
+#pragma unroll
+                    for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+                        for (int m = 0; m < 2; ++m) {
+                            const size_t row = (size_t)m * NR + lr + rr;
+                            if (c < C && !bad) {
+                                cw[rr][m] = *reinterpret_cast<const uint4 *>(gu + row * rc + (size_t)c * 16);
+                                sw[rr][m] = gu[2 * (size_t)NR * rc + row * rs + c];
+                            } else {
+                                cw[rr][m] = make_uint4(0u, 0u, 0u, 0u);
+                                sw[rr][m] = 127u;
+                            }
                         }
+                    float a[2][2][2];  // [row][gate, up][even, odd elements]
+#pragma unroll
+                    for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+                        for (int m = 0; m < 2; ++m) a[rr][m][0] = a[rr][m][1] = 0.f;
+                    // the chunk's four 8-element pieces in order, each against
+                    // all four rows (per row the order of chunks_dot)
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const uint4 xv = c < C ? sx16[c * 4 + q4] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                        for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+                            for (int m = 0; m < 2; ++m) {
+                                const uint4 cc = cw[rr][m];
+                                const uint32_t w = q4 == 0 ? cc.x : q4 == 1 ? cc.y : q4 == 2 ? cc.z : cc.w;
+                                dot8_e2m1_f16(w, xv.x, xv.y, xv.z, xv.w, a[rr][m][0], a[rr][m][1]);
+                            }
                     }
-                    v[2 * rr] = chunks_dot<KCH>(cg, sg, xw);
-                    v[2 * rr + 1] = chunks_dot<KCH>(cu, su, xw);
+#pragma unroll
+                    for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+                        for (int m = 0; m < 2; ++m)
+                            v[rr][m] = fmaf(a[rr][m][0] + a[rr][m][1], e8m0_to_f32(sw[rr][m]), v[rr][m]);
                 }
 #pragma unroll
-                for (int i = 0; i < 4; ++i) v[i] = warp_sum(v[i]);
+                for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+                    for (int m = 0; m < 2; ++m) v[rr][m] = warp_sum(v[rr][m]);
+                if (tid == 0 && pp == 0) STK_STAMP(11);
                 if (lane == 0) {
                     uint32_t word = 0u;
-                    if (!bad) {
-                        word = (uint32_t)f32_to_bf16(swiglu_h(v[0], v[1], xs)) |
-                               ((uint32_t)f32_to_bf16(swiglu_h(v[2], v[3], xs)) << 16);
-                    } else {
+                    if (!bad)
+                        word = (uint32_t)f32_to_bf16(swiglu_h(v[0][0], v[0][1], xs)) |
+                               ((uint32_t)f32_to_bf16(swiglu_h(v[1][0], v[1][1], xs)) << 16);
+                    else
                         atomicOr(p.status, kBadExpertId);
-                    }
                     st_relaxed_gpu_v2(p.h_tag + gr / 2, tag, word);
                 }
             }
         }
         if (tid < k) s_hmax[tid] = 0u;
         if (!__syncthreads_and(ok)) break;
+        STK_STAMP(5);
 
         // ---- E: all of h (tagged) -> FP16 in shared memory ----
-        {
-            const int npc = I >> 3;  // 8-element pieces per vector
-            const int total = k * npc;
-            uint4 *sv = reinterpret_cast<uint4 *>(sh);
-            #pragma unroll 1
-            for (int bs = warp * 32; bs < total; bs += kStackThreads) {
-                const int i = bs + lane;
-                const bool valid = i < total;
-                float m = 0.f;
-                int q = -1;
-                if (valid) {
-                    uint32_t d0 = 0u, d1 = 0u, d2 = 0u, d3 = 0u;
-                    const uint2 *src = p.h_tag + (size_t)i * 4;
-                    if (!stk_poll2(src, tag, d0, d1, limit, p.abort, base)) ok = false;
-                    if (ok && !stk_poll2(src + 2, tag, d2, d3, limit, p.abort, base)) ok = false;
-                    q = i / npc;
-                    const int pi = i - q * npc;
-                    sv[q * npc + h_piece(pi >> 2, pi & 3)] = make_uint4(d0, d1, d2, d3);
-                    const uint32_t w4[4] = {d0, d1, d2, d3};
-#pragma unroll
-                    for (int r = 0; r < 4; ++r)
-                        m = fmaxf(m, fmaxf(fabsf(bf16_to_f32(w4[r] & 0xFFFFu)),
-                                           fabsf(bf16_to_f32(w4[r] >> 16))));
-                }
-                if (__all_sync(0xffffffffu, q == __shfl_sync(0xffffffffu, q, 0))) {
-                    m = warp_max(m);
-                    if (lane == 0 && q >= 0) atomicMax(s_hmax + q, __float_as_uint(m));
-                } else if (valid) {
-                    atomicMax(s_hmax + q, __float_as_uint(m));
-                }
-            }
-            // the CTA's down rows (requested with the gate/up rows) must have landed
-            if (tid == 0 && !mbar_wait(&dbar, (unsigned)l & 1u)) ok = false;
-            if (!__syncthreads_and(ok)) break;
-            #pragma unroll 1
-            for (int i = tid; i < total; i += kStackThreads) {
-                const float sf = pow2_neg(f16_stage_exponent(__uint_as_float(s_hmax[i / npc])));
-                const uint4 v = sv[i];
-                uint4 o;
-                o.x = f32x2_to_f16x2(bf16_to_f32(v.x & 0xFFFFu) * sf, bf16_to_f32(v.x >> 16) * sf);
-                o.y = f32x2_to_f16x2(bf16_to_f32(v.y & 0xFFFFu) * sf, bf16_to_f32(v.y >> 16) * sf);
-                o.z = f32x2_to_f16x2(bf16_to_f32(v.z & 0xFFFFu) * sf, bf16_to_f32(v.z >> 16) * sf);
-                o.w = f32x2_to_f16x2(bf16_to_f32(v.w & 0xFFFFu) * sf, bf16_to_f32(v.w >> 16) * sf);
-                sv[i] = o;
-            }
-            if (tid < k) s_xs[tid] = pow2(f16_stage_exponent(__uint_as_float(s_hmax[tid])));
-            __syncthreads();
+        const int npc = I >> 3;  // 8-element pieces per vector
+        const int total = k * npc;
+        uint4 *sv = reinterpret_cast<uint4 *>(sm + p.plan.off_sh);
+        if (tid < kHThreads)
+            ok = stk_gather_h(p.h_tag, total, npc, tid, tag, limit, p.abort, base, sv, s_hmax);
+        // the CTA's down rows (requested with the gate/up rows) must have landed
+        if (tid == 0 && !mbar_wait(&dbar, (unsigned)l & 1u)) ok = false;
+        if (!__syncthreads_and(ok)) break;
+        STK_STAMP(6);
+        #pragma unroll 1
+        for (int i = tid; i < total; i += kStackThreads) {
+            const float sf = pow2_neg(f16_stage_exponent(__uint_as_float(s_hmax[i / npc])));
+            const uint4 v = sv[i];
+            uint4 o;
+            o.x = f32x2_to_f16x2(bf16_to_f32(v.x & 0xFFFFu) * sf, bf16_to_f32(v.x >> 16) * sf);
+            o.y = f32x2_to_f16x2(bf16_to_f32(v.y & 0xFFFFu) * sf, bf16_to_f32(v.y >> 16) * sf);
+            o.z = f32x2_to_f16x2(bf16_to_f32(v.z & 0xFFFFu) * sf, bf16_to_f32(v.z >> 16) * sf);
+            o.w = f32x2_to_f16x2(bf16_to_f32(v.w & 0xFFFFu) * sf, bf16_to_f32(v.w >> 16) * sf);
+            sv[i] = o;
         }
+        if (tid < k) s_xs[tid] = pow2(f16_stage_exponent(__uint_as_float(s_hmax[tid])));
+        __syncthreads();
+        STK_STAMP(15);
 
         // ---- F: down GEMV of the CTA's output rows, every slot ----
-        {
+        const int R = p.plan.R;
+        float *so = reinterpret_cast<float *>(sm + p.plan.off_so);  // [k][R] expert outputs
+        if (r0 < r1) {
             const DownSrc src = {ly.table, ly.codes_base, ly.scales_base, p.codes_stride,
                                  p.scales_stride};
-            DownRows<TLD, KCHD, true> rows(H, I, k, E, R, r0, r1, src, s_ids, rows_c, rows_s);
-            if (r0 < r1) {
-                rows.fetch(rows.rr);
-                rows.run(sh, s_xs, so, p.status);
-            }
+            const uint8_t *rows_c = sm + p.plan.off_dn;
+            DownRows<TLD, KCHD, true, false, kSWarps> rows(
+                H, I, k, E, R, r0, r1, src, s_ids, rows_c,
+                rows_c + (size_t)k * R * ((size_t)I >> 1));
+            rows.fetch(rows.rr);
+            rows.run(reinterpret_cast<const uint32_t *>(sv), s_xs, so, p.status);
         }
         __syncthreads();
+        STK_STAMP(7);
 
         // ---- G: sequential BF16 combine + residual; publish the layer output ----
         #pragma unroll 1
@@ -574,18 +676,22 @@ stack_decode_kernel(const __grid_constant__ StackParams p) {
             if (l == L - 1) reinterpret_cast<uint32_t *>(p.r)[n / 2] = word;
         }
         __syncthreads();  // sx, so, s_w are rewritten by the next layer
+        STK_STAMP(8);
     }
 
     if (l < L) {
         // gave up: record it, release the other CTAs, and let no copy of this
-        // CTA outlive it (waits bounded; a wait already complete returns at once)
+        // CTA outlive it (the layer's copies and the router rows in flight;
+        // waits bounded, a completed wait returns at once)
         if (tid == 0) {
             atomicOr(p.status, kTimeoutStatus);
             st_relaxed_gpu(p.abort, base);
-            if (s_gu_armed == l) {
+            if (s_copied == l) {
+                const int nch = (np + p.plan.ppc - 1) / p.plan.ppc;
+                mbar_wait(&sbar, (unsigned)l & 1u);
                 for (int c = 0; c < nch; ++c) mbar_wait(&gbar[c], (unsigned)l & 1u);
+                mbar_wait(&dbar, (unsigned)l & 1u);
             }
-            if (s_dn_armed == l) mbar_wait(&dbar, (unsigned)l & 1u);
             for (int i = 0; i < 2; ++i)
                 if (s_rt_armed[i] >= l) mbar_wait(&rbar[i], (unsigned)(s_rt_armed[i] >> 1) & 1u);
         }
@@ -649,13 +755,16 @@ bool stack_plan(int E, int H, int I, int k, int grid, StackPlan *pl) {
         return false;
     if (H % 512 != 0 || H > 2048 || I % 128 != 0 || I > 4096) return false;
     if (stack_variant(H, I) < 0) return false;
+    // the gathering threads hold at most kPollMaxJ pieces each
+    if (H / 8 > kXThreads * kPollMaxJ || k * I / 8 > kHThreads * kPollMaxJ) return false;
     StackPlan s = {};
     s.U = (I % 256 == 0) ? 2 : 4;  // rows per unit: U * I/32 scale bytes are a 16-byte multiple
-    const int P = k * I / 2;
-    s.np_max = (P + grid - 1) / grid;
-    s.ppc = (s.np_max + kStackChunks - 1) / kStackChunks;
     const int NU = H / s.U;
     s.R = s.U * ((NU + grid - 1) / grid);
+    if (kSWarps / k < 1) return false;  // the down phase needs a warp per slot
+    const int P = k * I / 2;
+    s.np_max = (P + grid - 1) / grid;
+    s.ppc = (s.np_max + kStackPieces - 1) / kStackPieces;
     const size_t rc = (size_t)H / 2, rs = (size_t)H / 32;
     size_t off = 0;
     s.off_gu = (unsigned)off;

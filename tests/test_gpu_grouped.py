@@ -43,10 +43,13 @@ def _check(L, layer, x, ids, w, shape, flags=0, residual=None):
     # rounding midpoint (different FP32 summation order on the tensor cores)
     # carries through silu and the product; when g and u both flip, s can move
     # two ulps and h land three BF16 values away; such flips stay rare (at most
-    # 1 % of the elements).  o sums I such h terms, so one rare h flip moves it
-    # far less than an ulp: o keeps the decode path's rule (one-ulp flips).
+    # 1 % of the elements).  o sums I products of h with weights whose E8M0
+    # scales span 2^6: a flipped h under one of the largest weights of a row
+    # moves o by up to ~0.4 % of rms(o), so o lands at most two BF16 values
+    # away, rarely (observed: 2 of 67,584 elements at 1.37e-2 rms, 2 ulps, in
+    # the 150-token single-group case).
     assert_close_rms(h_g[valid], h_r[valid], what="grouped h", max_ulps=3)
-    assert_close_rms(o_g[valid], o_r[valid], what="grouped o", max_ulps=1)
+    assert_close_rms(o_g[valid], o_r[valid], what="grouped o", max_ulps=2)
     # y is a function of o alone (the bit-exact combine check below), so its
     # distance to the oracle's y is bounded by the o differences through the
     # routing weights plus the two combines' own roundings (the kernel's and
@@ -63,8 +66,12 @@ def _check(L, layer, x, ids, w, shape, flags=0, residual=None):
     bound = 1.01 * (wa * np.abs(og - orr)).sum(axis=1) + 2 * (2 * k + 1) * scale * 2.0 ** -8
     dy = np.abs(f64(y_g) - f64(y_r))
     assert np.all(dy <= bound), f"grouped y: {(dy > bound).sum()} elements beyond the o-derived bound"
-    # and the decode path's rule for y: 1e-2 rms, rare flips of at most two ulps
-    assert_close_rms(y_g, y_r, what="grouped y", max_ulps=2)
+    # and a count limit on the elements beyond 1e-2 rms: an o flip under a
+    # combine that cancels (|y| << |w o|) is many ulps of y, so the ulp
+    # distance of those few elements is capped loosely but their number is
+    # held to 0.05 % (observed worst: 7 of 65,536 at 2.8e-2 rms, 8 ulps, T=260
+    # Zipf on tcgen05; all inside the o-derived bound above)
+    assert_close_rms(y_g, y_r, what="grouped y", max_ulps=16, max_flip_frac=5e-4)
     # combine in slot order, bit-exact given the kernel's own expert outputs
     for t in range(T):
         o_t = np.where(valid[t][:, None], o_g[t], 0).astype(np.uint16)
