@@ -52,6 +52,7 @@ def parse_args():
     ap.add_argument("--no-pdl", action="store_true")
     ap.add_argument("--no-prefetch", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-sym8", action="store_true", help="skip the sym8 stack line")
     ap.add_argument("--skip-nvfp4", action="store_true",
                     help="skip the decode measurement of the stack with NVFP4 experts")
     ap.add_argument("--skip-batched", action="store_true",
@@ -349,6 +350,60 @@ def nvfp4_stack(torch, moe, st, args, max_steps=8):
     return out
 
 
+def sym8_stack(torch, moe, st, args, max_steps=4):
+    """The same 38-layer decode with sym8 experts (page "LFM2.5-8B-A1B — Core
+    AI (.aimodel)", "Provenance": int8 weights, a scale per 32): each layer's
+    int8 weights uniform over -127..127 and binary16 block scales (positive
+    normal values, exponent fields 2..5, uniform mantissas) drawn on the
+    device from a seeded generator, the MXFP4 layer's router reused; one
+    route + gate/up + down launch triple per layer, captured in a CUDA graph
+    and timed like the NVFP4 line."""
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(args.seed + 11)
+    n_w = 3 * SHAPE.I * SHAPE.H
+    weights = []
+    for L in st.layers:
+        q = torch.randint(-127, 128, (SHAPE.E, n_w), dtype=torch.int8, device="cuda",
+                          generator=gen)
+        ex = torch.randint(2, 6, (SHAPE.E, n_w // 32), dtype=torch.int16, device="cuda",
+                           generator=gen)
+        man = torch.randint(0, 1024, (SHAPE.E, n_w // 32), dtype=torch.int16, device="cuda",
+                            generator=gen)
+        weights.append((q, (ex << 10) | man, L.router_w, L.router_b))
+    s8 = moe.MoEStack(weights, SHAPE.E, SHAPE.H, SHAPE.I, SHAPE.top_k, T=1, persistent=False)
+    s8.r.copy_(st.r)
+    s8.capture()
+    steps = max(1, min(max_steps, args.steps))
+    for _ in range(2 * TOKENS_PER_STEP):
+        s8.graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stream = torch.cuda.current_stream()
+    e0.record(stream)
+    for _ in range(steps * TOKENS_PER_STEP):
+        s8.graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_ms = e0.elapsed_time(e1)
+    assert s8.status() == 0
+    ids = s8.ids.cpu().numpy()
+    per_expert = n_w + n_w // 16
+    tok_bytes = sum(len(set(ids[l].ravel().tolist())) * per_expert + SHAPE.E * SHAPE.H * 2
+                    + 2 * SHAPE.H * 2 for l in range(len(s8.layers)))
+    n_tok = steps * TOKENS_PER_STEP
+    peak, _ = load_peaks()
+    out = {"workload": f"stack24b with sym8 experts ({len(s8.layers)} layers, int8 weights, "
+                       "binary16 scale per 32), batch-1 decode, per-layer launches",
+           "tokens_per_s": n_tok / (t_ms / 1e3), "us_per_token": t_ms * 1e3 / n_tok,
+           "bytes_per_token": tok_bytes, "hbm_gbs": tok_bytes * n_tok / (t_ms / 1e3) / 1e9,
+           "hbm_frac": tok_bytes * n_tok / (t_ms / 1e3) / 1e9 / peak,
+           "gpu_launches_per_token": 3 * len(s8.layers), "steps": steps}
+    s8.close()
+    del weights
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -464,6 +519,8 @@ def run_ours(args):
                           if not args.skip_batched else None)
         # ---- the same stack with NVFP4 experts ----
         out["nvfp4"] = nvfp4_stack(torch, moe, st, args) if not args.skip_nvfp4 else None
+        # ---- the same stack with sym8 experts ----
+        out["sym8"] = sym8_stack(torch, moe, st, args) if not args.skip_sym8 else None
 
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
         rate, evals, threads, sample = oracle_layer_rate(12.0)

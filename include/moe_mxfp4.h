@@ -172,6 +172,25 @@ MOE_API int moe_load_expert_table(moe_handle_t h, const uint8_t *const *codes_pt
 MOE_API int moe_load_packed_nvfp4(moe_handle_t h, const uint8_t *codes_u8,
                                   const uint8_t *scales_e4m3, const float *global_scales);
 
+/* Bind contiguously stored sym8 experts (page "LFM2.5-8B-A1B — Core AI
+ * (.aimodel)", table "Provenance", row "Weight format": symmetric-linear int8
+ * weights with one scale per K-block of 32).  codes_s8: device int8
+ * [E][3][I*H], row-major rows of K weights per matrix (gate, up: I rows of H;
+ * down: H rows of I), one two's-complement byte per weight; scales_f16:
+ * device uint16 [E][3][I*H/32], one IEEE binary16 scale (little-endian bit
+ * pattern) per 32 consecutive K elements of a row.  Weight = q * scale, no
+ * zero point.  codes 16-byte aligned, scales 2-byte aligned; read in place
+ * through the handle's device pointer table, caller-owned.  Requires H and I
+ * multiples of 32 with one token's H (gate/up) and k*I (down) BF16 values
+ * within 48 KB.  sym8 layers run the per-(token, slot) GEMVs for every T
+ * (in chunks of up to 4 tokens) with FP32 products and sums; no grouped
+ * path, no fused launch structures (FORCE_GROUPED / FORCE_MMA /
+ * FORCE_TCGEN05 return ARG), no stack kernel.  moe_load_packed,
+ * moe_load_packed_nvfp4 and moe_load_expert_table switch the handle to their
+ * format.  Errors: ARG (null pointer, unsupported shape), NOT_DEVICE, CUDA. */
+MOE_API int moe_load_packed_sym8(moe_handle_t h, const int8_t *codes_s8,
+                                 const uint16_t *scales_f16);
+
 /* Bytes of device workspace needed for up to max_tokens tokens per call.
  * Errors: ARG. */
 MOE_API int moe_workspace_bytes(moe_handle_t h, int max_tokens, size_t *bytes);

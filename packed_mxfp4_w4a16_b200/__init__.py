@@ -22,7 +22,7 @@ from ._lib import MoEError, check, library_path, load
 
 __all__ = [
     "MoEError", "MoELayer", "MoEStack", "library_path", "load",
-    "moe_create", "moe_destroy", "moe_load_packed", "moe_load_packed_nvfp4",
+    "moe_create", "moe_destroy", "moe_load_packed", "moe_load_packed_nvfp4", "moe_load_packed_sym8",
     "moe_load_expert_table",
     "moe_workspace_bytes", "moe_set_workspace", "moe_route", "moe_route_ex",
     "moe_forward", "moe_forward_ex", "moe_layer_ex", "moe_get_intermediates", "moe_get_status",
@@ -95,6 +95,18 @@ def moe_load_packed_nvfp4(h: int, codes: torch.Tensor, scales: torch.Tensor,
     _need(gscales, torch.float32, "moe_load_packed_nvfp4")
     check("moe_load_packed_nvfp4",
           load().moe_load_packed_nvfp4(C.c_void_p(h), _p(codes), _p(scales), _p(gscales)))
+
+
+def moe_load_packed_sym8(h: int, codes: torch.Tensor, scales: torch.Tensor) -> None:
+    """sym8 experts: codes int8 [E, 3*I*H] (one byte per weight), scales
+    binary16 words [E, 3*I*H/32] (a float16 or int16/uint16 tensor of the bit
+    patterns)."""
+    _need(codes, torch.int8, "moe_load_packed_sym8")
+    if (scales.dtype not in (torch.float16, torch.int16, torch.uint16) or not scales.is_cuda
+            or not scales.is_contiguous()):
+        raise MoEError("moe_load_packed_sym8", -1)
+    check("moe_load_packed_sym8",
+          load().moe_load_packed_sym8(C.c_void_p(h), _p(codes), _p(scales)))
 
 
 def moe_load_expert_table(h: int, codes_ptrs, scales_ptrs) -> None:
@@ -337,7 +349,8 @@ class MoELayer:
     include/moe_mxfp4.h) are read in place; the layer keeps references to
     them. ``router_w`` BF16 [E, H], ``router_b`` FP32 [E] or None.  With
     ``gscales`` (float32 [E, 2]) the experts are NVFP4: scales are then E4M3
-    bytes [E, 3*I*H/16].
+    bytes [E, 3*I*H/16].  With int8 ``codes`` [E, 3*I*H] the experts are
+    sym8: scales are then binary16 words [E, 3*I*H/32].
     """
 
     def __init__(self, E, H, I, top_k, codes, scales, router_w=None, router_b=None,
@@ -349,7 +362,9 @@ class MoELayer:
         self.max_tokens = max_tokens
         self.handle = moe_create(E, H, I, top_k)
         try:
-            if gscales is None:
+            if codes.dtype == torch.int8:
+                moe_load_packed_sym8(self.handle, codes, scales)
+            elif gscales is None:
                 moe_load_packed(self.handle, codes, scales)
             else:
                 moe_load_packed_nvfp4(self.handle, codes, scales, gscales)

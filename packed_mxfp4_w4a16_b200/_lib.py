@@ -26,6 +26,7 @@ SIGNATURES = [
     ("moe_destroy", _i, [_vp]),
     ("moe_load_packed", _i, [_vp, _vp, _vp]),
     ("moe_load_packed_nvfp4", _i, [_vp, _vp, _vp, _vp]),
+    ("moe_load_packed_sym8", _i, [_vp, _vp, _vp]),
     ("moe_load_expert_table", _i, [_vp, C.POINTER(_vp), C.POINTER(_vp)]),
     ("moe_workspace_bytes", _i, [_vp, _i, C.POINTER(_sz)]),
     ("moe_set_workspace", _i, [_vp, _vp, _sz, _i]),

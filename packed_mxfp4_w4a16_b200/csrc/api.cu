@@ -36,6 +36,7 @@ struct moe_ctx {
     const uint8_t *scales_base = nullptr;
     int nv = 0;                           // NVFP4 weights (moe_load_packed_nvfp4)
     const float *gscale = nullptr;        // NVFP4: [E][2] multipliers (gate/up, down)
+    int s8 = 0;                           // sym8 weights (moe_load_packed_sym8)
 };
 
 namespace {
@@ -200,6 +201,7 @@ int moe_load_packed(moe_handle_t h, const uint8_t *codes_u8, const uint8_t *scal
         h->codes_base = codes_u8;
         h->scales_base = scales_e8m0;
         h->nv = 0;
+        h->s8 = 0;
         h->gscale = nullptr;
     }
     return rc;
@@ -230,7 +232,38 @@ int moe_load_packed_nvfp4(moe_handle_t h, const uint8_t *codes_u8, const uint8_t
         h->codes_base = codes_u8;
         h->scales_base = scales_e4m3;
         h->nv = 1;
+        h->s8 = 0;
         h->gscale = global_scales;
+    }
+    return rc;
+}
+
+int moe_load_packed_sym8(moe_handle_t h, const int8_t *codes_s8, const uint16_t *scales_f16) {
+    if (!h || !codes_s8 || !scales_f16) return MOE_ERR_ARG;
+    if (!moe::sym8_supported(h->H, h->I, h->k)) return MOE_ERR_ARG;
+    int rc = ensure_device_block(h);
+    if (rc != MOE_OK) return rc;
+    if ((rc = check_device_ptr(h, codes_s8, 16)) != MOE_OK) return rc;
+    if ((rc = check_device_ptr(h, scales_f16, 2)) != MOE_OK) return rc;
+    // one byte per weight; one 2-byte scale per 32 weights
+    const size_t mc = (size_t)h->I * h->H, ms = (size_t)h->I * h->H / 16;
+    const uint8_t *cb = reinterpret_cast<const uint8_t *>(codes_s8);
+    const uint8_t *sb = reinterpret_cast<const uint8_t *>(scales_f16);
+    moe::ExpertPtrs *t = new (std::nothrow) moe::ExpertPtrs[h->E];
+    if (!t) return MOE_ERR_ARG;
+    for (int e = 0; e < h->E; ++e)
+        for (int m = 0; m < 3; ++m) {
+            t[e].codes[m] = cb + ((size_t)e * 3 + m) * mc;
+            t[e].scales[m] = sb + ((size_t)e * 3 + m) * ms;
+        }
+    rc = upload_table(h, t);
+    delete[] t;
+    if (rc == MOE_OK) {
+        // the MXFP4 fast paths read codes_base; sym8 is reached through the table
+        h->codes_base = h->scales_base = nullptr;
+        h->nv = 0;
+        h->s8 = 1;
+        h->gscale = nullptr;
     }
     return rc;
 }
@@ -255,6 +288,7 @@ int moe_load_expert_table(moe_handle_t h, const uint8_t *const *codes_ptrs,
     if (rc == MOE_OK) {
         h->codes_base = h->scales_base = nullptr;
         h->nv = 0;
+        h->s8 = 0;
         h->gscale = nullptr;
     }
     return rc;
@@ -342,7 +376,8 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
     if (flags & MOE_FWD_FORCE_TCGEN05) {
         if (flags & MOE_FWD_FORCE_DECODE) return MOE_ERR_ARG;
         const int Tc = T < moe::kGroupedMaxT ? T : moe::kGroupedMaxT;
-        if (h->nv || !h->codes_base || !moe::grouped_tc_supported(h->H, h->I, Tc * h->k))
+        if (h->nv || h->s8 || !h->codes_base ||
+            !moe::grouped_tc_supported(h->H, h->I, Tc * h->k))
             return MOE_ERR_ARG;
         flags |= MOE_FWD_FORCE_GROUPED;
     }
@@ -359,13 +394,41 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
     if ((rc = check_device_ptr(h, y, 16)) != MOE_OK) return rc;
     if (residual && (rc = check_device_ptr(h, residual, 16)) != MOE_OK) return rc;
     if (y == x) return MOE_ERR_ARG;
-    if (!moe::decode_shape_supported(h->H, h->I)) return MOE_ERR_ARG;
 
     const WsLayout L = ws_layout(h, h->max_tokens);
     const bool keep = flags & MOE_FWD_KEEP_INTERMEDIATES;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint16_t *hbuf = reinterpret_cast<uint16_t *>(h->ws + L.h);
     uint16_t *obuf = reinterpret_cast<uint16_t *>(h->ws + L.o);
+
+    if (h->s8) {
+        // sym8 experts: the per-(token, slot) GEMVs of sym8.cu at every T
+        if (flags & MOE_FWD_FORCE_GROUPED) return MOE_ERR_ARG;
+        const int chunk = moe::sym8_max_chunk(h->H, h->I, h->k);
+        for (int t0 = 0; t0 < T; t0 += chunk) {
+            const int Tc = (T - t0 < chunk) ? T - t0 : chunk;
+            moe::Sym8Params p = {};
+            p.table = h->d_table;
+            p.x = x + (size_t)t0 * h->H;
+            p.ids = topk_ids + (size_t)t0 * h->k;
+            p.w = topk_w + (size_t)t0 * h->k;
+            p.residual = residual ? residual + (size_t)t0 * h->H : nullptr;
+            p.y = y + (size_t)t0 * h->H;
+            p.h = hbuf + (size_t)t0 * h->k * h->I;
+            p.o_keep = keep ? obuf + (size_t)t0 * h->k * h->H : nullptr;
+            p.status = h->d_status;
+            p.T = Tc;
+            p.E = h->E;
+            p.H = h->H;
+            p.I = h->I;
+            p.k = h->k;
+            if ((rc = cuda_rc(moe::launch_sym8(p, h->num_sms, run_gu, run_dn, s))) != MOE_OK)
+                return rc;
+        }
+        h->kept = keep;
+        return MOE_OK;
+    }
+    if (!moe::decode_shape_supported(h->H, h->I)) return MOE_ERR_ARG;
 
     // (token, expert)-sorted grouped path on the tensor cores: batches beyond
     // the decode sizes, or when asked (the phase flags time the decode path)
@@ -526,10 +589,10 @@ int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
     const WsLayout L = ws_layout(h, h->max_tokens);
     float *lg = reinterpret_cast<float *>(h->ws + L.logits);
 
-    if (T > moe::kDecodeMaxT || (route_flags & MOE_ROUTE_SIGMOID)) {
-        // many tokens, or sigmoid scoring (the fused launch structures select
-        // by softmax scoring only): explicit routing, then the forward on the
-        // given ids
+    if (T > moe::kDecodeMaxT || (route_flags & MOE_ROUTE_SIGMOID) || h->s8) {
+        // many tokens, sigmoid scoring (the fused launch structures select
+        // by softmax scoring only) or sym8 experts: explicit routing, then
+        // the forward on the given ids
         int32_t *ids = topk_ids;
         float *w = topk_w;
         if (!ids || !w) return MOE_ERR_ARG;
@@ -548,10 +611,11 @@ int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
     unsigned fdown = 0;
     int lrows = 0;
     // the fused launch structures run MXFP4 weights only
-    const bool whole = !h->nv && h->fusion >= MOE_FUSION_LAYER && !keep &&
+    const bool mx = !h->nv && !h->s8;
+    const bool whole = mx && h->fusion >= MOE_FUSION_LAYER && !keep &&
                        moe::layer_plan(T, h->E, h->H, h->I, h->k, G, &fsmem, &fslots, &fregion,
                                        &fdown, &lrows);
-    if (whole || (!h->nv && h->fusion >= MOE_FUSION_ROUTER &&
+    if (whole || (mx && h->fusion >= MOE_FUSION_ROUTER &&
                   moe::layer_gateup_plan(T, h->E, h->H, G, &fsmem, &fslots, &fregion) &&
                   moe::down_decode_smem(T, h->k, h->I, frows) <= moe::kDownSmemMax)) {
         // router + gate/up in one launch, then the down kernel on the same grid
@@ -747,8 +811,9 @@ int moe_get_status(moe_handle_t h, unsigned *device_status) {
 
 int moe_bytes_per_expert(moe_handle_t h, size_t *bytes) {
     if (!h || !bytes) return MOE_ERR_ARG;
-    *bytes = h->nv ? (size_t)3 * h->I * h->H / 2 + (size_t)3 * h->I * h->H / 16 + 2 * sizeof(float)
-                   : (size_t)3 * h->I * h->H / 2 + (size_t)3 * h->I * h->H / 32;
+    *bytes = h->s8   ? (size_t)3 * h->I * h->H + (size_t)3 * h->I * h->H / 16
+             : h->nv ? (size_t)3 * h->I * h->H / 2 + (size_t)3 * h->I * h->H / 16 + 2 * sizeof(float)
+                     : (size_t)3 * h->I * h->H / 2 + (size_t)3 * h->I * h->H / 32;
     return MOE_OK;
 }
 
@@ -820,7 +885,7 @@ int moe_stack_create(const moe_handle_t *layers, int n_layers, const uint16_t *c
         const moe_ctx *h = layers[l];
         if (!h || h->E != l0->E || h->H != l0->H || h->I != l0->I || h->k != l0->k) return MOE_ERR_ARG;
         if (!h->loaded) return MOE_ERR_NOT_LOADED;
-        if (h->nv) return MOE_ERR_ARG;  // the stack kernel reads MXFP4 experts
+        if (h->nv || h->s8) return MOE_ERR_ARG;  // the stack kernel reads MXFP4 experts
         if (h->device != l0->device) return MOE_ERR_NOT_DEVICE;
     }
     int dev = -1, sms = 0;

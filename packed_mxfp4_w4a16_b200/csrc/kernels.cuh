@@ -263,4 +263,24 @@ size_t down_decode_smem(int T, int k, int I, int rows_per_cta);
 constexpr size_t kDownSmemMax = 200 * 1024;
 bool decode_shape_supported(int H, int I);
 
+// ---- sym8 experts (int8 weights, binary16 scale per 32; sym8.cu) ----
+constexpr int kS8MaxT = 4;                // tokens per launch pair
+constexpr size_t kS8SmemMax = 48 * 1024;  // staged x / h per CTA
+struct Sym8Params {
+    const ExpertPtrs *table;     // [E]: codes [3][rows][K] int8, scales [3][rows][K/32] binary16
+    const uint16_t *x;           // [T][H] BF16
+    const int32_t *ids;          // [T][k]
+    const float *w;              // [T][k]
+    const uint16_t *residual;    // [T][H] or null
+    uint16_t *y;                 // [T][H]
+    uint16_t *h;                 // [T][k][I] BF16 SwiGLU outputs (workspace)
+    uint16_t *o_keep;            // [T][k][H] expert outputs, or null
+    unsigned *status;
+    int T, E, H, I, k;
+};
+bool sym8_supported(int H, int I, int k);
+int sym8_max_chunk(int H, int I, int k);
+cudaError_t launch_sym8(const Sym8Params &p, int num_sms, bool run_gu, bool run_dn,
+                        cudaStream_t s);
+
 }  // namespace moe

@@ -1,0 +1,219 @@
+// sym8.cu — experts in the sym8 format on the per-(token, slot) GEMV path.
+//
+// Source: page "LFM2.5-8B-A1B — Core AI (.aimodel)", table "Provenance", row
+// "Weight format": symmetric-linear int8 weights with one scale per K-block of
+// 32.  Read here as: one two's-complement byte q per weight, one IEEE binary16
+// scale s per 32 consecutive K elements of a row, w = q s, no zero point.
+// Everything else is the packed-MXFP4 layer's arithmetic (model card
+// "LFM2.5-24B-A2B — Packed MXFP4 Inference": "Grouped top-4 expert execution"
+// for gate/up, SwiGLU, down and the sequential BF16 combine; table "Model and
+// quantization" for BF16 activations, FP32 accumulation, BF16 outputs).
+//
+// Layout (as moe_load_packed_sym8 binds it): codes [E][3][rows][K] int8,
+// scales [E][3][rows][K/32] little-endian binary16 words; matrix m of expert e
+// is read through the handle's device table, in place.
+//
+// Arithmetic.  A weight byte becomes an FP32 value exactly by a byte permute
+// into the float 2^23 + (q + 128) followed by one subtraction of 2^23 + 128;
+// BF16 activations widen to FP32 exactly; each product q x is exact in FP32
+// (8 x 8 significant bits).  A lane sums the 16 products of its 16-byte chunk
+// in FP32, scales that half-group sum by the block's s (binary16 -> FP32
+// exact) and adds it to its running sum; the warp then adds its lanes' sums.
+// g and u are rounded to BF16, SiLU(g) to BF16, h = BF16(SiLU(g) u); the down
+// sums give o = BF16(sum), and the combine is the sequential BF16 one
+// (wb = BF16(w), y = BF16(y + BF16(o wb)), then y = BF16(r + y)).
+//
+// Two launches per chunk of up to kS8MaxT tokens: gate/up + SwiGLU (one warp
+// per (pair, row) item, the tokens' x staged in shared memory) writing h to
+// the workspace, then down + combine + residual (one warp per (token, output
+// row), the chunk's h staged in shared memory).  An expert id outside [0, E)
+// gives that slot h = 0 and o = 0 and sets the status word's bad-id bit.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kernels.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kS8Threads = 256;
+constexpr int kS8Warps = kS8Threads / 32;
+constexpr int kS8CtasPerSm = 4;  // warps in flight per SM: 32 (streaming GEMV)
+
+// Four int8 weights of one 32-bit word (byte 0 = lowest K index) -> FP32,
+// exactly: byte i, biased to q + 128, becomes the low byte of the float with
+// bit pattern 0x4B0000xx = 2^23 + xx.
+__device__ __forceinline__ void s8x4_to_f32(uint32_t w, float (&f)[4]) {
+    const uint32_t u = w ^ 0x80808080u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        f[i] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540u | (unsigned)i)) - 8388736.0f;
+}
+
+// Sum of the 16 products of one 16-byte chunk of weights with 16 BF16
+// activations (two 16-byte pieces, lower K first), in K order.
+__device__ __forceinline__ float s8_chunk_dot(const uint4 &wq, const uint4 &x0, const uint4 &x1) {
+    const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
+    const uint32_t xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float f[4];
+        s8x4_to_f32(wv[i], f);
+        acc = fmaf(f[0], __uint_as_float(xv[2 * i] << 16), acc);
+        acc = fmaf(f[1], __uint_as_float(xv[2 * i] & 0xFFFF0000u), acc);
+        acc = fmaf(f[2], __uint_as_float(xv[2 * i + 1] << 16), acc);
+        acc = fmaf(f[3], __uint_as_float(xv[2 * i + 1] & 0xFFFF0000u), acc);
+    }
+    return acc;
+}
+
+// binary16 block scale of the 16-byte chunk c of a row (two chunks per block).
+__device__ __forceinline__ float s8_scale(const uint8_t *row_scales, int c) {
+    const uint16_t *s = reinterpret_cast<const uint16_t *>(row_scales);
+    return f16_bits_to_f32(__ldg(s + (c >> 1)));
+}
+
+// Dot product of one sym8 row of K weights (codes rc, scales rs) with the
+// BF16 vector xs (16-byte pieces in shared memory), by one warp; every lane
+// returns the same sum.  Lane l takes the chunks l, l + 32, ...
+__device__ __forceinline__ float s8_row_dot(const uint8_t *rc, const uint8_t *rs, const uint4 *xs,
+                                            int K, int lane) {
+    const int nc = K >> 4;
+    float acc = 0.f;
+#pragma unroll 4
+    for (int c = lane; c < nc; c += 32) {
+        const uint4 wq = ld_stream16(rc + (size_t)c * 16);
+        acc = fmaf(s8_chunk_dot(wq, xs[2 * c], xs[2 * c + 1]), s8_scale(rs, c), acc);
+    }
+    return warp_sum(acc);
+}
+
+// gate/up + SwiGLU.  Item (q, i): pair q = t k + j (token t, slot j), row i of
+// the expert's gate and up matrices; h[q][i] = BF16(BF16(SiLU(BF16(g))) BF16(u)).
+__global__ void __launch_bounds__(kS8Threads) sym8_gateup_kernel(const Sym8Params p) {
+    extern __shared__ __align__(16) uint4 s_x[];  // [T][H/8]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int H = p.H, I = p.I, k = p.k, E = p.E;
+    const int np8 = H >> 3;
+    const uint4 *x = reinterpret_cast<const uint4 *>(p.x);
+    for (int i = tid; i < p.T * np8; i += kS8Threads) s_x[i] = x[i];
+    __syncthreads();
+    const size_t rs = (size_t)H >> 4;  // scale bytes of a row
+    const long long items = (long long)p.T * k * I;
+    #pragma unroll 1
+    for (long long it = (long long)blockIdx.x * kS8Warps + warp; it < items;
+         it += (long long)gridDim.x * kS8Warps) {
+        const int q = (int)(it / I), i = (int)(it - (long long)q * I);
+        const int t = q / k;
+        const int e = p.ids[q];
+        const bool bad = e < 0 || e >= E;
+        float ag = 0.f, au = 0.f;
+        if (!bad) {
+            const ExpertPtrs &ep = p.table[e];
+            const uint4 *xs = s_x + (size_t)t * np8;
+            ag = s8_row_dot(ep.codes[0] + (size_t)i * H, ep.scales[0] + (size_t)i * rs, xs, H, lane);
+            au = s8_row_dot(ep.codes[1] + (size_t)i * H, ep.scales[1] + (size_t)i * rs, xs, H, lane);
+        }
+        if (lane == 0) {
+            uint16_t hv = 0;
+            if (!bad) {
+                const float g = round_bf16(ag), u = round_bf16(au);
+                const float sl = round_bf16(g / (1.0f + expf(-g)));
+                hv = f32_to_bf16(sl * u);
+            } else if (i == 0) {
+                atomicOr(p.status, kBadExpertId);
+            }
+            p.h[it] = hv;
+        }
+    }
+}
+
+// down + combine + residual.  Item (t, n): output row n of token t; the
+// slots' o_j = BF16(down row n . h_j) in slot order, combined sequentially in
+// BF16, then the residual.
+__global__ void __launch_bounds__(kS8Threads) sym8_down_kernel(const Sym8Params p) {
+    extern __shared__ __align__(16) uint4 s_h[];  // [T][k][I/8]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int H = p.H, I = p.I, k = p.k, E = p.E;
+    const int np8 = I >> 3;
+    const uint4 *hg = reinterpret_cast<const uint4 *>(p.h);
+    for (int i = tid; i < p.T * k * np8; i += kS8Threads) s_h[i] = hg[i];
+    __syncthreads();
+    const size_t rs = (size_t)I >> 4;
+    const long long items = (long long)p.T * H;
+    #pragma unroll 1
+    for (long long it = (long long)blockIdx.x * kS8Warps + warp; it < items;
+         it += (long long)gridDim.x * kS8Warps) {
+        const int t = (int)(it / H), n = (int)(it - (long long)t * H);
+        float y = 0.f;
+        #pragma unroll 1
+        for (int j = 0; j < k; ++j) {
+            const int q = t * k + j;
+            const int e = p.ids[q];
+            const bool bad = e < 0 || e >= E;
+            float o = 0.f;
+            if (!bad) {
+                const ExpertPtrs &ep = p.table[e];
+                o = round_bf16(s8_row_dot(ep.codes[2] + (size_t)n * I, ep.scales[2] + (size_t)n * rs,
+                                          s_h + (size_t)q * np8, I, lane));
+            } else if (lane == 0 && n == 0) {
+                atomicOr(p.status, kBadExpertId);
+            }
+            if (lane == 0 && p.o_keep) p.o_keep[(size_t)q * H + n] = f32_to_bf16(o);
+            const float wb = round_bf16(p.w[q]);
+            y = round_bf16(y + round_bf16(o * wb));
+        }
+        if (lane == 0) {
+            if (p.residual) y = round_bf16(bf16_to_f32(p.residual[it]) + y);
+            p.y[it] = f32_to_bf16(y);
+        }
+    }
+}
+
+size_t s8_gateup_smem(int T, int H) { return (size_t)T * H * 2; }
+size_t s8_down_smem(int T, int k, int I) { return (size_t)T * k * I * 2; }
+
+PerDeviceOnce g_s8_attr;
+
+}  // namespace
+
+bool sym8_supported(int H, int I, int k) {
+    return H >= 32 && I >= 32 && H % 32 == 0 && I % 32 == 0 && k >= 1 && k <= kMaxTopK &&
+           s8_gateup_smem(1, H) <= kS8SmemMax && s8_down_smem(1, k, I) <= kS8SmemMax;
+}
+
+int sym8_max_chunk(int H, int I, int k) {
+    int c = kS8MaxT;
+    while (c > 1 && (s8_gateup_smem(c, H) > kS8SmemMax || s8_down_smem(c, k, I) > kS8SmemMax)) --c;
+    return c;
+}
+
+cudaError_t launch_sym8(const Sym8Params &p, int num_sms, bool run_gu, bool run_dn,
+                        cudaStream_t s) {
+    if (p.T < 1 || p.T > kS8MaxT || !sym8_supported(p.H, p.I, p.k)) return cudaErrorInvalidValue;
+    const size_t sg = s8_gateup_smem(p.T, p.H), sd = s8_down_smem(p.T, p.k, p.I);
+    if (sg > kS8SmemMax || sd > kS8SmemMax) return cudaErrorInvalidValue;
+    cudaError_t e = per_device_once(g_s8_attr, [] {
+        cudaError_t r = cudaFuncSetAttribute(sym8_gateup_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kS8SmemMax);
+        if (r != cudaSuccess) return r;
+        return cudaFuncSetAttribute(sym8_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kS8SmemMax);
+    });
+    if (e != cudaSuccess) return e;
+    const int grid = num_sms * kS8CtasPerSm;
+    if (run_gu) {
+        sym8_gateup_kernel<<<grid, kS8Threads, sg, s>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (run_dn) {
+        sym8_down_kernel<<<grid, kS8Threads, sd, s>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace moe
