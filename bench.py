@@ -65,6 +65,9 @@ def parse_args():
                          "of the one-launch stack kernel")
     ap.add_argument("--skip-configs", action="store_true",
                     help="skip the tiny-layer, single-layer and 8B-stack measurements")
+    ap.add_argument("--only-batched", default=None, metavar="T:ROUTING",
+                    help="time one grouped-path case of one 24B layer only, e.g. 256:uniform "
+                         "(a small command for profiler captures)")
     ap.add_argument("--only-main", action="store_true",
                     help="time the main line only (for profiler runs)")
     return ap.parse_args()
@@ -421,6 +424,15 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
+    if args.only_batched:
+        T, dist = args.only_batched.split(":")
+        st = build_stack(torch, moe, seed=args.seed + rank, n_layers=1, persistent=False)
+        rows = batched_cases(torch, moe, st, args.seed, cases=((int(T), dist),))
+        if rank == 0:
+            print(json.dumps({"batched": rows}), flush=True)
+        st.close()
+        return 0
+
     n_layers = args.layers
     st = build_stack(torch, moe, seed=args.seed + rank, n_layers=n_layers,
                      persistent=False if args.layered else None)
@@ -694,7 +706,7 @@ BATCHED_CASES = ((32, "uniform"), (32, "zipf"), (64, "uniform"), (64, "zipf"), (
 TC_AUTO_GROUP = 40  # the library's tcgen05 products from T k >= 40 E on
 
 
-def batched_cases(torch, moe, st, seed, reps=20):
+def batched_cases(torch, moe, st, seed, reps=20, cases=BATCHED_CASES):
     """The grouped (token, expert)-sorted path on one 24B layer of the stack at
     batch sizes beyond decode: synthetic routing (k distinct experts per token,
     uniform or Zipf(1.1) popularity), moe_forward timed in a CUDA graph of
@@ -704,11 +716,11 @@ def batched_cases(torch, moe, st, seed, reps=20):
     L = st.layers[0]
     out = []
     expert = 3 * SHAPE.I * SHAPE.H // 2 + 3 * SHAPE.I * SHAPE.H // 32
-    tmax = max(t for t, _ in BATCHED_CASES)
+    tmax = max(t for t, _ in cases)
     lay = moe.MoELayer(SHAPE.E, SHAPE.H, SHAPE.I, SHAPE.top_k, L.codes, L.scales, L.router_w,
                        L.router_b, max_tokens=tmax)
     s = torch.cuda.Stream()
-    for T, dist in BATCHED_CASES:
+    for T, dist in cases:
         x = torch.from_numpy(synth.make_tokens(T, SHAPE.H, seed=seed, stream=T)
                              .view(np.int16)).cuda().view(torch.bfloat16)
         ids_h, w_h = synth.make_routing(T, SHAPE.E, SHAPE.top_k, dist,
