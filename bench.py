@@ -349,6 +349,38 @@ def nvfp4_stack(torch, moe, st, args, max_steps=8):
            "tokens_per_s": n_tok / (t_ms / 1e3), "us_per_token": t_ms * 1e3 / n_tok,
            "bytes_per_token": tok_bytes, "hbm_gbs": tok_bytes * n_tok / (t_ms / 1e3) / 1e9,
            "steps": steps}
+    # the grouped path (mma.sync products) with NVFP4 experts, one layer
+    codes, sc, rw, rb, gs = weights[0]
+    lay = moe.MoELayer(SHAPE.E, SHAPE.H, SHAPE.I, SHAPE.top_k, codes, sc, rw, rb,
+                       max_tokens=256, gscales=gs)
+    grouped = []
+    for T in (64, 256):
+        x = torch.from_numpy(synth.make_tokens(T, SHAPE.H, seed=args.seed, stream=T)
+                             .view(np.int16)).cuda().view(torch.bfloat16)
+        ids_h, w_h = synth.make_routing(T, SHAPE.E, SHAPE.top_k, "uniform",
+                                        synth.rng_for(args.seed, 93, T))
+        ids, w = torch.from_numpy(ids_h).cuda(), torch.from_numpy(w_h).cuda()
+        y = torch.empty_like(x)
+        lay.forward(x, ids, w, y=y)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(20):
+                lay.forward(x, ids, w, y=y)
+        g.replay()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / 20
+        del g
+        touched = len(set(ids_h.ravel().tolist()))
+        grouped.append({"T": T, "routing": "uniform", "experts_touched": touched,
+                        "products": "mma.sync", "us_per_call": us,
+                        "hbm_gbs": (touched * per_expert + 2 * T * SHAPE.H * 2) / (us * 1e-6) / 1e9})
+    assert lay.status() == 0
+    lay.close()
+    out["grouped"] = grouped
     nv.close()
     return out
 

@@ -435,7 +435,7 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
     const bool phase = flags & (MOE_FWD_PHASE_GATEUP | MOE_FWD_PHASE_DOWN);
     const bool grouped = !phase && !(flags & MOE_FWD_FORCE_DECODE) &&
                          (T > moe::kDecodeMaxT || (flags & MOE_FWD_FORCE_GROUPED)) &&
-                         !h->nv && moe::grouped_supported(h->E, h->H, h->I);
+                         moe::grouped_supported(h->E, h->H, h->I, h->nv);
     if ((flags & MOE_FWD_FORCE_GROUPED) && !grouped) return MOE_ERR_ARG;
     if (grouped) {
         for (int t0 = 0; t0 < T; t0 += moe::kGroupedMaxT) {
@@ -445,7 +445,9 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
             gp.codes_base = h->codes_base;
             gp.scales_base = h->scales_base;
             gp.codes_stride = (size_t)h->I * h->H / 2;
-            gp.scales_stride = (size_t)h->I * h->H / 32;
+            gp.scales_stride = (size_t)h->I * h->H / (h->nv ? 16 : 32);
+            gp.nv = h->nv;
+            gp.gscale = h->gscale;
             gp.x = x + (size_t)t0 * h->H;
             gp.ids = topk_ids + (size_t)t0 * h->k;
             gp.w = topk_w + (size_t)t0 * h->k;

@@ -139,6 +139,18 @@ __device__ __forceinline__ void mma_group_e2m1(float (&acc)[4], uint32_t w_lo, u
     acc[3] = fmaf(dd[3], sh, acc[3]);
 }
 
+// NVFP4 form of the same: a 32-element group is two 16-element blocks with
+// their own E4M3 scales (sc_lo: the two scale bytes of row g, block 0 in the
+// low byte; sc_hi: those of row g + 8).  Thread (g, q) supplies codes
+// 4q..4q+3 of block 0 in the low half of its word and codes 4q..4q+3 of block
+// 1 in the high half (w_lo: row g, w_hi: row g + 8), and the activations of
+// column g in the same order (b.x, b.y: block 0 elements 4q..4q+3; b.z, b.w:
+// block 1).  The first MMA then sums block 0 and the second block 1, each
+// from a fresh accumulator; each block's partial product times its row's
+// E4M3 scale is added to acc in FP32, block 0 first: exactly per-block scaling.
+__device__ __forceinline__ void mma_group_nvfp4(float (&acc)[4], uint32_t w_lo, uint32_t w_hi,
+                                                uint32_t sc_lo, uint32_t sc_hi, const uint4 &b);
+
 __device__ __forceinline__ float f16_bits_to_f32(uint32_t h) {
     float f;
     asm("{ .reg .f16 t; mov.b16 t, %1; cvt.f32.f16 %0, t; }" : "=f"(f) : "h"((uint16_t)h));
@@ -224,6 +236,24 @@ __device__ __forceinline__ void e4m3x2_to_f32(uint32_t s, float &lo, float &hi) 
         : "r"(s));
     lo = f16_bits_to_f32(h2 & 0xFFFFu);
     hi = f16_bits_to_f32(h2 >> 16);
+}
+
+__device__ __forceinline__ void mma_group_nvfp4(float (&acc)[4], uint32_t w_lo, uint32_t w_hi,
+                                                uint32_t sc_lo, uint32_t sc_hi, const uint4 &b) {
+    uint32_t fa[2][4];
+    e2m1x8_to_f16x8(w_lo, fa[0]);
+    e2m1x8_to_f16x8(w_hi, fa[1]);
+    const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+    float d0[4], d1[4];
+    mma_f16(d0, fa[0][0], fa[1][0], fa[0][1], fa[1][1], b.x, b.y, zero);
+    mma_f16(d1, fa[0][2], fa[1][2], fa[0][3], fa[1][3], b.z, b.w, zero);
+    float l0, l1, h0, h1;
+    e4m3x2_to_f32(sc_lo, l0, l1);
+    e4m3x2_to_f32(sc_hi, h0, h1);
+    acc[0] = fmaf(d1[0], l1, fmaf(d0[0], l0, acc[0]));
+    acc[1] = fmaf(d1[1], l1, fmaf(d0[1], l0, acc[1]));
+    acc[2] = fmaf(d1[2], h1, fmaf(d0[2], h0, acc[2]));
+    acc[3] = fmaf(d1[3], h1, fmaf(d0[3], h0, acc[3]));
 }
 
 // ------------------------------------------------ FP16 staging of BF16 ----

@@ -191,7 +191,10 @@ __device__ __forceinline__ void cp_async_commit_wait() {
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-template <int NMAT, int RT>
+// NV: NVFP4 weights (two E4M3 scales per 32-element group, mma_group_nvfp4's
+// K order; the expert's multiplier joins the power-of-two staging scale in the
+// epilogue, an exact product).
+template <int NMAT, int RT, bool NV>
 __global__ void __launch_bounds__(128 * RT) grouped_mma_kernel(const GroupedParams p) {
     constexpr int kWarps = 4 * RT;
     extern __shared__ __align__(16) uint8_t sm[];
@@ -206,7 +209,7 @@ __global__ void __launch_bounds__(128 * RT) grouped_mma_kernel(const GroupedPara
     const int M = NMAT == 2 ? p.I : p.H;  // rows of the matrix (a multiple of 16 RT)
     const int row0 = blockIdx.x * (kGpRows * RT);
     const int ng = K >> 5;                // 32-element groups
-    const uint32_t rc = (uint32_t)K >> 1, rs = (uint32_t)K >> 5;
+    const uint32_t rc = (uint32_t)K >> 1, rs = (uint32_t)K >> (NV ? 4 : 5);
     const uint32_t rcp = rc + 16, rsp = rs + 16;  // padded row pitches (bank spread)
     const uint32_t bp = (uint32_t)K * 2 + 64;     // padded pitch of a staged B row
     constexpr int R = kGpRows * RT;               // rows held by the CTA
@@ -254,11 +257,12 @@ __global__ void __launch_bounds__(128 * RT) grouped_mma_kernel(const GroupedPara
     const int gq = (ng + 3) >> 2;
     const int gb = min(ng, kq * gq), ge = min(ng, gb + gq);
     // this thread's A words (rows g / g + 8 of its tile) and scales
-    const uint8_t *a_lo = s_codes + (rt * kGpRows + g) * rcp + 4 * q;
+    const uint8_t *a_lo = s_codes + (rt * kGpRows + g) * rcp + (NV ? 2 * q : 4 * q);
     const uint8_t *s_lo = s_scales + (rt * kGpRows + g) * rsp;
     const uint32_t a_hi = 8 * rcp, sc_hi = 8 * rsp;
     const uint32_t a_m = R * rcp, sc_m = R * rsp;
-    const uint8_t *bcol = s_b + g * bp + 16 * q;  // column g = token tc + g of the group
+    // column g = token tc + g of the group
+    const uint8_t *bcol = s_b + g * bp + (NV ? 8 * q : 16 * q);
 
     #pragma unroll 1
     for (int tc = 0; tc < n_e; tc += 8) {
@@ -275,13 +279,33 @@ __global__ void __launch_bounds__(128 * RT) grouped_mma_kernel(const GroupedPara
 
         #pragma unroll 4
         for (int G = gb; G < ge; ++G) {
-            const uint4 b = *reinterpret_cast<const uint4 *>(bcol + G * 64);
+            if (NV) {
+                // block 0 elements 4q..4q+3, then block 1's
+                const uint2 b0 = *reinterpret_cast<const uint2 *>(bcol + G * 64);
+                const uint2 b1 = *reinterpret_cast<const uint2 *>(bcol + G * 64 + 32);
+                const uint4 b = make_uint4(b0.x, b0.y, b1.x, b1.y);
 #pragma unroll
-            for (int m = 0; m < NMAT; ++m) {
-                const uint8_t *cb = a_lo + m * a_m + G * 16;
-                const uint8_t *sb = s_lo + m * sc_m + G;
-                mma_group_e2m1(acc[m], *reinterpret_cast<const uint32_t *>(cb),
-                               *reinterpret_cast<const uint32_t *>(cb + a_hi), sb[0], sb[sc_hi], b);
+                for (int m = 0; m < NMAT; ++m) {
+                    const uint8_t *cb = a_lo + m * a_m + G * 16;
+                    const uint16_t *sb = reinterpret_cast<const uint16_t *>(s_lo + m * sc_m + 2 * G);
+                    const uint32_t wl = *reinterpret_cast<const uint16_t *>(cb) |
+                                        ((uint32_t)*reinterpret_cast<const uint16_t *>(cb + 8) << 16);
+                    const uint32_t wh = *reinterpret_cast<const uint16_t *>(cb + a_hi) |
+                                        ((uint32_t)*reinterpret_cast<const uint16_t *>(cb + a_hi + 8) << 16);
+                    mma_group_nvfp4(acc[m], wl, wh, sb[0],
+                                    *reinterpret_cast<const uint16_t *>(
+                                        reinterpret_cast<const uint8_t *>(sb) + sc_hi),
+                                    b);
+                }
+            } else {
+                const uint4 b = *reinterpret_cast<const uint4 *>(bcol + G * 64);
+#pragma unroll
+                for (int m = 0; m < NMAT; ++m) {
+                    const uint8_t *cb = a_lo + m * a_m + G * 16;
+                    const uint8_t *sb = s_lo + m * sc_m + G;
+                    mma_group_e2m1(acc[m], *reinterpret_cast<const uint32_t *>(cb),
+                                   *reinterpret_cast<const uint32_t *>(cb + a_hi), sb[0], sb[sc_hi], b);
+                }
             }
         }
         // ---- the 4 K quarters of each row tile, added in order 0, 1, 2, 3 ----
@@ -313,13 +337,15 @@ __global__ void __launch_bounds__(128 * RT) grouped_mma_kernel(const GroupedPara
                 for (int hr = 0; hr < 2; ++hr) {
                     const int r = row0 + rt * kGpRows + g + 8 * hr;
                     if (NMAT == 2) {
-                        const float xs = pow2(p.x_exp[pr / p.k]);
+                        const float xs = NV ? pow2(p.x_exp[pr / p.k]) * __ldg(p.gscale + 2 * e)
+                                            : pow2(p.x_exp[pr / p.k]);
                         const float gv = round_bf16(acc[0][hr * 2 + cc] * xs);
                         const float uv = round_bf16(acc[NMAT - 1][hr * 2 + cc] * xs);
                         const float sl = round_bf16(gv / (1.0f + expf(-gv)));
                         p.h[(size_t)pr * M + r] = f32_to_bf16(sl * uv);
                     } else {
-                        const float hs = pow2(p.h_exp[pr]);
+                        const float hs = NV ? pow2(p.h_exp[pr]) * __ldg(p.gscale + 2 * e + 1)
+                                            : pow2(p.h_exp[pr]);
                         p.o[(size_t)pr * M + r] = f32_to_bf16(acc[0][hr * 2 + cc] * hs);
                     }
                 }
@@ -403,44 +429,45 @@ namespace {
 
 constexpr size_t kMmaSmemBudget = 220 * 1024;
 
-size_t mma_smem(int nmat, int K) {
+size_t mma_smem(int nmat, int K, int nv) {
     const size_t R = (size_t)kGpRows * kRowTiles;
-    const size_t rcp = (size_t)K / 2 + 16, rsp = (size_t)K / 32 + 16;
+    const size_t rcp = (size_t)K / 2 + 16, rsp = (size_t)K / (nv ? 16 : 32) + 16;
     return (size_t)nmat * R * (rcp + rsp) + (size_t)kRowTiles * 3 * 32 * nmat * 4 * sizeof(float) +
            (size_t)8 * ((size_t)K * 2 + 64);
 }
 
-template <int NMAT>
+template <int NMAT, bool NV>
 cudaError_t launch_mma(const GroupedParams &p, cudaStream_t s, bool pdl) {
     const int K = NMAT == 2 ? p.H : p.I, M = NMAT == 2 ? p.I : p.H;
-    const size_t smem = mma_smem(NMAT, K);
+    const size_t smem = mma_smem(NMAT, K, NV ? 1 : 0);
     if (smem > kMmaSmemBudget) return cudaErrorInvalidValue;
     // the budget, once per device (the attribute belongs to the current
     // device's context)
     static PerDeviceOnce once;
     const cudaError_t attr = per_device_once(once, [] {
-        return cudaFuncSetAttribute(grouped_mma_kernel<NMAT, kRowTiles>,
+        return cudaFuncSetAttribute(grouped_mma_kernel<NMAT, kRowTiles, NV>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)kMmaSmemBudget);
     });
     if (attr != cudaSuccess) return attr;
-    return launch_ex(grouped_mma_kernel<NMAT, kRowTiles>, dim3(M / (kGpRows * kRowTiles), p.E),
+    return launch_ex(grouped_mma_kernel<NMAT, kRowTiles, NV>, dim3(M / (kGpRows * kRowTiles), p.E),
                      dim3(128 * kRowTiles), smem, s, pdl, p);
 }
 
 }  // namespace
 
-bool grouped_supported(int E, int H, int I) {
+bool grouped_supported(int E, int H, int I, int nv) {
     // the pipeline stages of both products must fit the shared memory budget
     return E <= kGpMaxE && H % 128 == 0 && I % 128 == 0 && H <= 4096 && I <= 4096 &&
-           mma_smem(2, H) <= kMmaSmemBudget && mma_smem(1, I) <= kMmaSmemBudget;
+           mma_smem(2, H, nv) <= kMmaSmemBudget && mma_smem(1, I, nv) <= kMmaSmemBudget;
 }
 
 cudaError_t launch_grouped(const GroupedParams &p, cudaStream_t s, bool pdl) {
-    if (p.T < 1 || p.T > kGroupedMaxT || !grouped_supported(p.E, p.H, p.I))
+    if (p.T < 1 || p.T > kGroupedMaxT || !grouped_supported(p.E, p.H, p.I, p.nv))
         return cudaErrorInvalidValue;
-    if (p.tcgen05 && (!p.codes_base || !grouped_tc_supported(p.H, p.I, p.T * p.k)))
+    if (p.tcgen05 && (p.nv || !p.codes_base || !grouped_tc_supported(p.H, p.I, p.T * p.k)))
         return cudaErrorInvalidValue;
+    if (p.nv && !p.gscale) return cudaErrorInvalidValue;
     cudaError_t e;
     if ((e = launch_ex(grouped_prep_kernel, dim3(p.T + 1), dim3(kGpThreads), 0, s, pdl, p)) !=
         cudaSuccess)
@@ -451,11 +478,15 @@ cudaError_t launch_grouped(const GroupedParams &p, cudaStream_t s, bool pdl) {
         if ((e = launch_grouped_tc_gateup(p, s, pdl)) != cudaSuccess) return e;
         if ((e = launch_grouped_tc_down(p, s, pdl)) != cudaSuccess) return e;
     } else {
-        if ((e = launch_mma<2>(p, s, pdl)) != cudaSuccess) return e;
+        if ((e = p.nv ? launch_mma<2, true>(p, s, pdl) : launch_mma<2, false>(p, s, pdl)) !=
+            cudaSuccess)
+            return e;
         if ((e = launch_ex(grouped_stage_h_kernel, dim3(p.T * p.k), dim3(kGpThreads), 0, s, pdl,
                            p)) != cudaSuccess)
             return e;
-        if ((e = launch_mma<1>(p, s, pdl)) != cudaSuccess) return e;
+        if ((e = p.nv ? launch_mma<1, true>(p, s, pdl) : launch_mma<1, false>(p, s, pdl)) !=
+            cudaSuccess)
+            return e;
     }
     return launch_ex(grouped_combine_kernel, dim3(p.T), dim3(kGpThreads), 0, s, pdl, p);
 }

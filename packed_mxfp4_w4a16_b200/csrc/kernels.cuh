@@ -167,8 +167,10 @@ struct GroupedParams {
     unsigned *status;
     int T, k, E, H, I;
     int tcgen05;               // products on tcgen05 (else mma.sync tiles)
+    int nv;                    // NVFP4 weights: E4M3 scale per 16 (mma.sync tiles only)
+    const float *gscale;       // NVFP4: [E][2] FP32 multipliers (gate/up, down)
 };
-bool grouped_supported(int E, int H, int I);
+bool grouped_supported(int E, int H, int I, int nv = 0);
 cudaError_t launch_grouped(const GroupedParams &p, cudaStream_t s, bool pdl);
 // Products on tcgen05 (grouped_tc.cu): chosen by the forward when the groups
 // average at least kTcAutoGroup pairs (the mma.sync tiles convert the codes

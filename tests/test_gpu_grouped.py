@@ -10,7 +10,7 @@ import torch
 
 import oracle
 import packed_mxfp4_w4a16_b200 as moe
-from gpu_util import assert_close_rms, dev_bf16, dev_layer, f64, host_bf16
+from gpu_util import check_grouped_y, assert_close_rms, dev_bf16, dev_layer, f64, host_bf16
 from workloads import synth
 
 pytestmark = pytest.mark.gpu
@@ -50,28 +50,7 @@ def _check(L, layer, x, ids, w, shape, flags=0, residual=None):
     # the 150-token single-group case).
     assert_close_rms(h_g[valid], h_r[valid], what="grouped h", max_ulps=3)
     assert_close_rms(o_g[valid], o_r[valid], what="grouped o", max_ulps=2)
-    # y is a function of o alone (the bit-exact combine check below), so its
-    # distance to the oracle's y is bounded by the o differences through the
-    # routing weights plus the two combines' own roundings (the kernel's and
-    # the oracle's): k products, k sums and the residual add each, every one
-    # off by at most half a BF16 ulp (<= 2^-8 of the value) of a value no
-    # larger than the largest term, the result or the residual
-    og, orr = f64(o_g), f64(o_r)
-    og[~valid], orr[~valid] = 0.0, 0.0
-    wa = np.abs(w64)[:, :, None]
-    scale = np.maximum(np.abs(f64(y_r)), (wa * np.abs(orr)).max(axis=1))
-    if residual is not None:
-        scale = np.maximum(scale, np.abs(f64(residual)))
-    k = ids.shape[1]
-    bound = 1.01 * (wa * np.abs(og - orr)).sum(axis=1) + 2 * (2 * k + 1) * scale * 2.0 ** -8
-    dy = np.abs(f64(y_g) - f64(y_r))
-    assert np.all(dy <= bound), f"grouped y: {(dy > bound).sum()} elements beyond the o-derived bound"
-    # and a count limit on the elements beyond 1e-2 rms: an o flip under a
-    # combine that cancels (|y| << |w o|) is many ulps of y, so the ulp
-    # distance of those few elements is capped loosely but their number is
-    # held to 0.05 % (observed worst: 7 of 65,536 at 2.8e-2 rms, 8 ulps, T=260
-    # Zipf on tcgen05; all inside the o-derived bound above)
-    assert_close_rms(y_g, y_r, what="grouped y", max_ulps=16, max_flip_frac=5e-4)
+    check_grouped_y(y_g, y_r, o_g, o_r, w64, valid, residual, what="grouped y")
     # combine in slot order, bit-exact given the kernel's own expert outputs
     for t in range(T):
         o_t = np.where(valid[t][:, None], o_g[t], 0).astype(np.uint16)

@@ -1,16 +1,16 @@
 """NVFP4 experts (E2M1 codes, an FP8 E4M3 scale per 16 elements, an FP32
-multiplier per expert for gate/up and one for down) on the per-(token, slot)
-path against the oracle: SwiGLU vectors h, expert outputs o and combined y
-at the tolerance of the MXFP4 decode path; the combine bit-exact given the
-kernel's own o; every T (the path chunks beyond 4 tokens); invalid ids; the
-whole layer; argument errors."""
+multiplier per expert for gate/up and one for down) against the oracle: the
+per-(token, slot) path (T <= 4) and the grouped mma.sync products (larger
+T, or forced) — SwiGLU vectors h, expert outputs o and combined y at the
+tolerance of the MXFP4 paths; the combine bit-exact given the kernel's own o;
+uniform and Zipf routing; invalid ids; the whole layer; argument errors."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import packed_mxfp4_w4a16_b200 as moe
-from gpu_util import assert_close_rms, dev_bf16, dev_u8, host_bf16
+from gpu_util import assert_close_rms, check_grouped_y, dev_bf16, dev_u8, host_bf16
 from workloads import synth
 
 pytestmark = pytest.mark.gpu
@@ -25,10 +25,10 @@ def _layer(shape, seed, max_tokens=4, bias=False):
     return L, layer
 
 
-def _check(L, layer, x, ids, w, shape, residual=None):
+def _check(L, layer, x, ids, w, shape, residual=None, flags=0, ulps=1):
     T = x.shape[0]
     y = layer.forward(dev_bf16(x), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(),
-                      flags=moe.FWD_KEEP_INTERMEDIATES,
+                      flags=moe.FWD_KEEP_INTERMEDIATES | flags,
                       residual=None if residual is None else dev_bf16(residual))
     torch.cuda.synchronize()
     h_g, o_g = layer.intermediates(T)
@@ -38,9 +38,13 @@ def _check(L, layer, x, ids, w, shape, residual=None):
                                              shape.H, shape.I, residual=residual, want_o=True,
                                              want_h=True)
     valid = (ids >= 0) & (ids < shape.E)
-    assert_close_rms(h_g[valid], h_r[valid], what="nvfp4 h")
-    assert_close_rms(o_g[valid], o_r[valid], what="nvfp4 o")
-    assert_close_rms(y_g, y_r, what="nvfp4 y", max_ulps=2)
+    assert_close_rms(h_g[valid], h_r[valid], what="nvfp4 h", max_ulps=ulps)
+    assert_close_rms(o_g[valid], o_r[valid], what="nvfp4 o", max_ulps=ulps)
+    if ulps > 1:
+        # grouped products: the grouped paths' y rule (o-derived bound)
+        check_grouped_y(y_g, y_r, o_g, o_r, w64, valid, residual, what="nvfp4 grouped y")
+    else:
+        assert_close_rms(y_g, y_r, what="nvfp4 y", max_ulps=2)
     for t in range(T):
         o_t = np.where(valid[t][:, None], o_g[t], 0).astype(np.uint16)
         want = oracle.combine(o_t, w64[t], None if residual is None else residual[t])
@@ -60,17 +64,46 @@ def test_nvfp4_forward_matches_oracle(shape, T):
     layer.close()
 
 
-def test_nvfp4_many_tokens_run_in_decode_chunks():
-    """Beyond 4 tokens NVFP4 stays on the per-(token, slot) path, in chunks."""
-    shape = synth.TINY
-    T = 11
+# The grouped mma.sync products sum the exact products in another FP32
+# order than the decode GEMVs; the tolerance is the MXFP4 grouped path's
+# (reading R14: h and o within 2 BF16 values of the oracle).
+@pytest.mark.parametrize("shape,T,dist,flags", [
+    (synth.TINY, 11, "zipf", 0), (synth.TINY, 3, "uniform", moe.FWD_FORCE_MMA),
+    (synth.L24B, 64, "uniform", 0), (synth.L24B, 64, "zipf", 0),
+    (synth.L8B, 40, "uniform", moe.FWD_FORCE_GROUPED)])
+def test_nvfp4_grouped_matches_oracle(shape, T, dist, flags):
+    """Beyond 4 tokens (or forced) NVFP4 runs the grouped mma.sync products;
+    the tcgen05 products refuse NVFP4."""
     L, layer = _layer(shape, 43, max_tokens=T)
-    x = synth.make_tokens(T, shape.H, seed=43)
-    ids, w = synth.make_routing(T, shape.E, shape.top_k, "zipf", synth.rng_for(43, 13, T))
-    _check(L, layer, x, ids, w, shape)
+    x = synth.make_tokens(T, shape.H, seed=43, stream=T)
+    ids, w = synth.make_routing(T, shape.E, shape.top_k, dist, synth.rng_for(43, 13, T))
+    r = synth.make_tokens(T, shape.H, seed=44, stream=T)
+    _check(L, layer, x, ids, w, shape, residual=r, flags=flags, ulps=2)
+    assert layer.status() == 0
     with pytest.raises(moe.MoEError):
         layer.forward(dev_bf16(x), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(),
-                      flags=moe.FWD_FORCE_GROUPED)
+                      flags=moe.FWD_FORCE_TCGEN05)
+    layer.close()
+
+
+def test_nvfp4_grouped_invalid_ids_and_decode_agreement():
+    """Invalid ids on the grouped path zero the slot and flag; the forced
+    per-(token, slot) path at the same T agrees with the grouped one within
+    the tolerance and is deterministic."""
+    shape = synth.L24B
+    T = 9
+    L, layer = _layer(shape, 48, max_tokens=T)
+    x = synth.make_tokens(T, shape.H, seed=48)
+    ids, w = synth.make_routing(T, shape.E, shape.top_k, "uniform", synth.rng_for(48, 13, T))
+    ids[2, 1] = 99
+    ids[7, 3] = -1
+    y_g = _check(L, layer, x, ids, w, shape, ulps=2)
+    assert layer.status() & moe.DEVICE_BAD_EXPERT_ID
+    y_d = _check(L, layer, x, ids, w, shape, flags=moe.FWD_FORCE_DECODE)
+    y_d2 = _check(L, layer, x, ids, w, shape, flags=moe.FWD_FORCE_DECODE)
+    np.testing.assert_array_equal(y_d, y_d2)
+    assert_close_rms(y_g, y_d, what="nvfp4 grouped vs decode y", max_ulps=2)
+    layer.status()
     layer.close()
 
 
