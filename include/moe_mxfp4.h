@@ -293,6 +293,14 @@ MOE_API int moe_get_intermediates(moe_handle_t h, const uint16_t **h_out,
  */
 MOE_API int moe_get_status(moe_handle_t h, unsigned *device_status);
 
+/* Device status of the handle's work queued on `stream` (the handle's
+ * kernels must have been enqueued on that stream), then cleared: waits for
+ * that stream only (moe_get_status waits for the whole device).  stream: a
+ * cudaStream_t, or NULL for the legacy default stream.  The read goes to
+ * pageable host memory, so it completes before the call returns.  Errors:
+ * ARG, NOT_LOADED, CUDA. */
+MOE_API int moe_get_status_stream(moe_handle_t h, void *stream, unsigned *device_status);
+
 /* Packed bytes of one expert: 3*I*H/2 code bytes + 3*I*H/32 scale bytes
  * (5,013,504 for H=2048, I=1536).  Errors: ARG. */
 MOE_API int moe_bytes_per_expert(moe_handle_t h, size_t *bytes);

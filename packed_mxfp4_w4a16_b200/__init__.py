@@ -25,7 +25,7 @@ __all__ = [
     "moe_create", "moe_destroy", "moe_load_packed", "moe_load_packed_nvfp4", "moe_load_packed_sym8",
     "moe_load_expert_table",
     "moe_workspace_bytes", "moe_set_workspace", "moe_route", "moe_route_ex",
-    "moe_forward", "moe_forward_ex", "moe_layer_ex", "moe_get_intermediates", "moe_get_status",
+    "moe_forward", "moe_forward_ex", "moe_layer_ex", "moe_get_intermediates", "moe_get_status", "moe_get_status_stream",
     "moe_bytes_per_expert", "moe_set_tuning", "moe_device_check", "moe_debug_dequant",
     "moe_forward_noalloc", "moe_forward_noalloc_status", "moe_stack_create", "moe_stack_destroy", "moe_stack_workspace_bytes",
     "moe_stack_set_workspace", "moe_stack_decode", "moe_stack_get_status",
@@ -191,6 +191,17 @@ def moe_get_intermediates(h: int):
 def moe_get_status(h: int) -> int:
     v = C.c_uint()
     check("moe_get_status", load().moe_get_status(C.c_void_p(h), C.byref(v)))
+    return v.value
+
+
+def moe_get_status_stream(h: int, stream=None) -> int:
+    """Device status of the handle's work on `stream` (torch stream or None:
+    the current stream), cleared; waits for that stream only."""
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    v = C.c_uint()
+    check("moe_get_status_stream",
+          load().moe_get_status_stream(C.c_void_p(h), C.c_void_p(s.cuda_stream), C.byref(v)))
     return v.value
 
 
@@ -421,7 +432,11 @@ class MoELayer:
         return (hv.view(torch.bfloat16).view(T, self.k, self.I),
                 ov.view(torch.bfloat16).view(T, self.k, self.H))
 
-    def status(self) -> int:
+    def status(self, stream=None) -> int:
+        """Device status bits (cleared).  With a stream: waits for that stream
+        only; without: for the whole device."""
+        if stream is not None:
+            return moe_get_status_stream(self.handle, stream)
         return moe_get_status(self.handle)
 
 

@@ -37,6 +37,7 @@ SIGNATURES = [
     ("moe_layer_ex", _i, [_vp, _vp, _i, _vp, _vp, _u, _vp, _vp, _vp, _vp, _vp, _vp, _u, _vp]),
     ("moe_get_intermediates", _i, [_vp, C.POINTER(_vp), C.POINTER(_vp)]),
     ("moe_get_status", _i, [_vp, C.POINTER(_u)]),
+    ("moe_get_status_stream", _i, [_vp, _vp, C.POINTER(_u)]),
     ("moe_bytes_per_expert", _i, [_vp, C.POINTER(_sz)]),
     ("moe_set_tuning", _i, [_vp, _i, _i]),
     ("moe_set_fusion", _i, [_vp, _i]),

@@ -37,6 +37,7 @@ struct moe_ctx {
     int nv = 0;                           // NVFP4 weights (moe_load_packed_nvfp4)
     const float *gscale = nullptr;        // NVFP4: [E][2] multipliers (gate/up, down)
     int s8 = 0;                           // sym8 weights (moe_load_packed_sym8)
+    moe::TcMapCache tc_maps;              // tensor maps of the bound codes (tcgen05 products)
 };
 
 namespace {
@@ -448,6 +449,7 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
             gp.scales_stride = (size_t)h->I * h->H / (h->nv ? 16 : 32);
             gp.nv = h->nv;
             gp.gscale = h->gscale;
+            gp.tc_maps = &h->tc_maps;
             gp.x = x + (size_t)t0 * h->H;
             gp.ids = topk_ids + (size_t)t0 * h->k;
             gp.w = topk_w + (size_t)t0 * h->k;
@@ -807,6 +809,22 @@ int moe_get_status(moe_handle_t h, unsigned *device_status) {
     if ((rc = cuda_rc(cudaMemcpy(&v, h->d_status, sizeof v, cudaMemcpyDeviceToHost))) != MOE_OK)
         return rc;
     if ((rc = cuda_rc(cudaMemset(h->d_status, 0, sizeof v))) != MOE_OK) return rc;
+    *device_status = v;
+    return MOE_OK;
+}
+
+int moe_get_status_stream(moe_handle_t h, void *stream, unsigned *device_status) {
+    if (!h || !device_status) return MOE_ERR_ARG;
+    if (!h->dblock) return MOE_ERR_NOT_LOADED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int rc;
+    unsigned v = 0;
+    // read and clear on the caller's stream, after the work queued on it
+    if ((rc = cuda_rc(cudaMemcpyAsync(&v, h->d_status, sizeof v, cudaMemcpyDeviceToHost, s))) !=
+        MOE_OK)
+        return rc;
+    if ((rc = cuda_rc(cudaMemsetAsync(h->d_status, 0, sizeof v, s))) != MOE_OK) return rc;
+    if ((rc = cuda_rc(cudaStreamSynchronize(s))) != MOE_OK) return rc;
     *device_status = v;
     return MOE_OK;
 }

@@ -534,12 +534,41 @@ bool grouped_tc_supported(int H, int I, int pairs) {
            tc_smem_bytes(1, I, pairs) <= kTcSmemBudget;
 }
 
+namespace {
+
+static_assert(sizeof(CUtensorMap) == sizeof(TcMapCache::map[0]), "opaque tensor-map bytes");
+
+// The map of matrix kind `kind` from the handle's cache (encoded when the
+// bound weights differ from the cached ones), else from the process-wide
+// cache of the weights bound last.
+cudaError_t kind_map(const GroupedParams &p, int kind, int rows, int K, CodesMap &shared,
+                     std::mutex &mu, CUtensorMap *out) {
+    if (!p.tc_maps) return codes_map_copy(shared, mu, p, rows, K, out);
+    TcMapCache &c = *p.tc_maps;
+    CUtensorMap *m = reinterpret_cast<CUtensorMap *>(c.map[kind]);
+    if (c.base[kind] != p.codes_base || c.E[kind] != p.E || c.rows[kind] != rows ||
+        c.K[kind] != K) {
+        CodesMap fresh;
+        const cudaError_t e = codes_map(fresh, p.codes_base, p.codes_stride, p.E, rows, K);
+        if (e != cudaSuccess) return e;
+        *m = fresh.map;
+        c.base[kind] = p.codes_base;
+        c.E[kind] = p.E;
+        c.rows[kind] = rows;
+        c.K[kind] = K;
+    }
+    *out = *m;
+    return cudaSuccess;
+}
+
+}  // namespace
+
 cudaError_t launch_grouped_tc_gateup(const GroupedParams &p, cudaStream_t s, bool pdl) {
     static CodesMap gu;
     static std::mutex mu;
     if (!p.codes_base) return cudaErrorInvalidValue;
     CUtensorMap map;
-    cudaError_t e = codes_map_copy(gu, mu, p, p.I, p.H, &map);
+    cudaError_t e = kind_map(p, 0, p.I, p.H, gu, mu, &map);
     if (e != cudaSuccess) return e;
     return launch_tc<2>(p, map, s, pdl);
 }
@@ -549,7 +578,7 @@ cudaError_t launch_grouped_tc_down(const GroupedParams &p, cudaStream_t s, bool 
     static std::mutex mu;
     if (!p.codes_base) return cudaErrorInvalidValue;
     CUtensorMap map;
-    cudaError_t e = codes_map_copy(dn, mu, p, p.H, p.I, &map);
+    cudaError_t e = kind_map(p, 1, p.H, p.I, dn, mu, &map);
     if (e != cudaSuccess) return e;
     return launch_tc<1>(p, map, s, pdl);
 }

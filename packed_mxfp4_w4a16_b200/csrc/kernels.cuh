@@ -145,6 +145,16 @@ struct DownParams {
 
 // The (token, expert)-sorted grouped path (grouped.cu), for batches of tokens.
 constexpr int kGroupedMaxT = 2048;  // tokens per grouped launch sequence (more: chunks)
+// Tensor maps of a handle's packed codes for the tcgen05 products (one per
+// matrix kind: 0 gate/up, 1 down), encoded when first needed and again only
+// when the bound weights change; opaque CUtensorMap bytes.  Owned by the
+// handle (calls on one handle are serialised by its owner).
+struct TcMapCache {
+    alignas(64) unsigned char map[2][128];
+    const uint8_t *base[2] = {nullptr, nullptr};
+    int E[2] = {0, 0}, rows[2] = {0, 0}, K[2] = {0, 0};
+};
+
 struct GroupedParams {
     const ExpertPtrs *table;
     const uint8_t *codes_base, *scales_base;  // contiguous layout fast path (or null)
@@ -169,6 +179,7 @@ struct GroupedParams {
     int tcgen05;               // products on tcgen05 (else mma.sync tiles)
     int nv;                    // NVFP4 weights: E4M3 scale per 16 (mma.sync tiles only)
     const float *gscale;       // NVFP4: [E][2] FP32 multipliers (gate/up, down)
+    TcMapCache *tc_maps;       // the handle's tensor-map cache (host), or null
 };
 bool grouped_supported(int E, int H, int I, int nv = 0);
 cudaError_t launch_grouped(const GroupedParams &p, cudaStream_t s, bool pdl);

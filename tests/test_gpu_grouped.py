@@ -232,3 +232,46 @@ def test_forced_grouped_small_batch_matches_decode(T):
     y_d = _check(L, layer, x, ids, w, shape, flags=moe.FWD_FORCE_DECODE)
     assert_close_rms(y_g, y_d, what="grouped vs decode", max_ulps=2)
     layer.close()
+
+
+def test_tcgen05_two_layers_alternating_keep_their_tensor_maps():
+    """Two handles bound to different weights, their tcgen05 forwards
+    interleaved: each handle encodes its own tensor maps, so every call gives
+    the bits of the same handle's first call."""
+    shape = synth.TINY
+    T = 100
+    a = _setup(shape, 81, T, "uniform")
+    b = _setup(shape, 82, T, "uniform")
+    flags = moe.FWD_FORCE_TCGEN05
+    firsts = []
+    for L, layer, x, ids, w in (a, b):
+        y = layer.forward(dev_bf16(x), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(),
+                          flags=flags)
+        torch.cuda.synchronize()
+        firsts.append(host_bf16(y).copy())
+    for _ in range(3):
+        for i, (L, layer, x, ids, w) in enumerate((a, b)):
+            y = layer.forward(dev_bf16(x), torch.from_numpy(ids).cuda(),
+                              torch.from_numpy(w).cuda(), flags=flags)
+            torch.cuda.synchronize()
+            np.testing.assert_array_equal(host_bf16(y), firsts[i])
+    _check(*a[:5], shape, flags=flags)
+    for t in (a, b):
+        t[1].close()
+
+
+def test_status_read_on_one_stream():
+    """moe_get_status_stream reads (and clears) the status of the work queued
+    on the given stream."""
+    shape = synth.TINY
+    L, layer, x, ids, w = _setup(shape, 83, 9, "uniform")
+    ids = ids.copy()
+    ids[4, 0] = 200
+    s = torch.cuda.Stream()
+    xd, idd, wd = dev_bf16(x), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        layer.forward(xd, idd, wd, stream=s)
+    assert layer.status(stream=s) & moe.DEVICE_BAD_EXPERT_ID
+    assert layer.status(stream=s) == 0  # cleared
+    layer.close()
