@@ -426,9 +426,8 @@ MOE_API int moe_stack_set_trace(moe_stack_t s, unsigned long long *trace, size_t
 /* ---------------------------------------------------------------------
  * Forward without any device allocation.  No counterpart in the paper: this
  * entry point exists for callers that may not call cudaMalloc -- code that
- * runs inside another framework's memory pool or allocator callback, hosts
- * whose device memory is budgeted and accounted elsewhere, or paths that
- * must not allocate while other streams are being captured.  It computes
+ * runs inside another framework's memory pool or allocator callback, or
+ * hosts whose device memory is budgeted and accounted elsewhere.  It computes
  * exactly what moe_create + moe_load_packed + moe_set_workspace +
  * moe_forward_ex(residual) compute, with the same kernels, but without a
  * handle: its scratch (status word, SwiGLU activations h) lives in one
@@ -445,8 +444,8 @@ MOE_API int moe_stack_set_trace(moe_stack_t s, unsigned long long *trace, size_t
  * a runtime call per pointer); they must be, and must hold the sizes the
  * shape implies.
  * The first call on a device (with that device current) looks up the
- * scratch's device address with cudaGetSymbolAddress; make that first call
- * before any stream capture.  Every call enqueues its kernels on `stream`
+ * scratch's device address with cudaGetSymbolAddress (a runtime call, made
+ * once per device).  Every call enqueues its kernels on `stream`
  * and shares the one scratch array: calls that overlap on the GPU
  * (different streams, or different threads without ordering) race on it.
  * The kernels report an id outside [0, E) (that slot contributes 0) or a
