@@ -29,18 +29,20 @@
 //      xn = BF16(r / sqrt(mean(r^2) + 1e-6)); FP16 staging of xn for the GEMVs;
 //      CTA b < E also computes router logit b (its router row was copied into
 //      shared memory one layer ahead) and publishes it.
-//   C  (producer warp) gathers all E logits, top-k + softmax, then requests
-//      with bulk copies ALL of the CTA's weight bytes of the layer at once: its
-//      share of the selected experts' gate/up rows (kStackChunks groups, one
-//      mbarrier each, so the GEMVs start when the first group lands) and its
-//      output rows of the down matrices (one mbarrier); and the router row of
-//      the next layer.  The whole layer's ~20 MB is in flight from here on.
-//   D  (23 consumer warps) one pair of gate/up rows per warp: E2M1 codes
-//      decoded in registers against the FP16 activations, FP32 sums, SwiGLU,
-//      the two h values published as one tagged word.
-//   E  every CTA gathers all of h and stages it in shared memory as FP16.
+//   C  (producer warp) gathers all E logits, top-k + softmax; then ONE lane
+//      requests with bulk copies all of the CTA's weight bytes of the layer,
+//      in the order they are needed: the gate/up scales, the gate/up code
+//      rows in a few pieces (one mbarrier each, so the GEMVs start when the
+//      first piece lands), the CTA's output rows of the down matrices (one
+//      mbarrier); another lane requests the next layer's router row.  The
+//      whole layer's ~20 MB is in flight from here on.
+//   D  (all warps) pairs of gate/up rows per warp from shared memory: E2M1
+//      codes decoded in registers against the FP16 activations, FP32 sums,
+//      SwiGLU, the two h values published as one tagged word.
+//   E  kHThreads threads gather all of h (tagged) and stage it in shared
+//      memory as FP16 (per-vector power of two).
 //   F  the down GEMV of the CTA's output rows for every slot (rows already in
-//      shared memory).
+//      shared memory), by lane teams two rows at a time.
 //   G  sequential BF16 combine in slot order and the residual add; the layer
 //      output rows are published as tagged words (the next layer's input).
 //
