@@ -97,7 +97,8 @@ def test_fused_layer_in_graph_with_shared_workspace(fusion):
     eager bits, replay after replay (the per-call tags keep advancing)."""
     shape = synth.L24B
     layers = [synth.make_layer(shape, seed=61, layer=l) for l in range(3)]
-    st = moe.MoEStack([dev_layer(L) for L in layers], shape.E, shape.H, shape.I, shape.top_k)
+    st = moe.MoEStack([dev_layer(L) for L in layers], shape.E, shape.H, shape.I, shape.top_k,
+                      persistent=False)
     r0 = dev_bf16(synth.make_tokens(1, shape.H, seed=61, stream=1))
     want = {}
     for mode in (moe.FUSION_NONE, fusion):  # the fused stack matches the unfused one
