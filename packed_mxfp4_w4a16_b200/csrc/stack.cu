@@ -42,7 +42,8 @@
 //   E  kHThreads threads gather all of h (tagged) and stage it in shared
 //      memory as FP16 (per-vector power of two).
 //   F  the down GEMV of the CTA's output rows for every slot (rows already in
-//      shared memory), by lane teams two rows at a time.
+//      shared memory), by lane teams two rows at a time, each chunk of h
+//      loaded once for both rows.
 //   G  sequential BF16 combine in slot order and the residual add; the layer
 //      output rows are published as tagged words (the next layer's input).
 //
@@ -279,6 +280,70 @@ static __device__ __noinline__ void stk_issue_layer(
                       (unsigned)(dn * drc), dbar, pol);
         bulk_g2s_hint(rows_s + (size_t)j * R * drs, scales(e, 2) + (size_t)r0 * drs,
                       (unsigned)(dn * drs), dbar, pol);
+    }
+}
+
+// Phase F: the down GEMV of the CTA's nr output rows for every slot, rows
+// (codes [k][R][I/2], scales [k][R][I/32]) and the FP16-staged h ([k][I/2]
+// words, h_piece order) in shared memory.  Warp w serves slot j = w % k; its
+// teams of TLD lanes take local rows ti, ti + tps, ... two at a time (the
+// h chunk loaded once for both rows), lane lt the 16-byte chunks lt + TLD u
+// of each row, one E8M0 group each.  Per row the sums and their order are
+// those of the per-layer down kernel (same bits).  so[j R + row] = BF16(o).
+template <int TLD, int KCHD>
+__device__ __forceinline__ void stk_down_rows(int I, int k, int E, int R, int nr, const int *s_ids,
+                                              const uint8_t *rows_c, const uint8_t *rows_s,
+                                              const uint32_t *sh, const float *s_xs, float *so,
+                                              unsigned *status) {
+    constexpr int TPW = 32 / TLD;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int groups = kSWarps / k;  // warps per slot
+    const int j = warp % k, gi = warp / k;
+    if (gi >= groups) return;
+    const int tps = groups * TPW;  // teams per slot
+    const int lt = lane & (TLD - 1);
+    const unsigned mask = team_mask<TLD>(lane);
+    const int C = I >> 5;
+    const size_t rc = (size_t)I >> 1, rs = (size_t)I >> 5;
+    const int e = s_ids[j];
+    const bool bad = e < 0 || e >= E;
+    const uint32_t *xv = sh + (size_t)j * (I >> 1);
+    const float xs = s_xs[j];
+    #pragma unroll 1
+    for (int ra = gi * TPW + lane / TLD; ra < nr; ra += 2 * tps) {
+        const int rb = ra + tps;
+        const bool has_b = rb < nr;
+        const uint8_t *ca = rows_c + (size_t)(j * R + ra) * rc, *sa = rows_s + (size_t)(j * R + ra) * rs;
+        const uint8_t *cb = rows_c + (size_t)(j * R + rb) * rc, *sb = rows_s + (size_t)(j * R + rb) * rs;
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int u = 0; u < KCHD; ++u) {
+            const int c = lt + TLD * u;
+            if (c < C && !bad) {
+                const uint4 *xq = reinterpret_cast<const uint4 *>(xv + (size_t)c * 16);
+                uint32_t x[16];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 v = xq[q ^ ((c >> 1) & 3)];  // h_piece order
+                    x[4 * q] = v.x;
+                    x[4 * q + 1] = v.y;
+                    x[4 * q + 2] = v.z;
+                    x[4 * q + 3] = v.w;
+                }
+                a0 = fmaf(dot32_e2m1_f16(*reinterpret_cast<const uint4 *>(ca + (size_t)c * 16), x),
+                          e8m0_to_f32(sa[c]), a0);
+                if (has_b)
+                    a1 = fmaf(dot32_e2m1_f16(*reinterpret_cast<const uint4 *>(cb + (size_t)c * 16), x),
+                              e8m0_to_f32(sb[c]), a1);
+            }
+        }
+        a0 = team_add<TLD>(a0, mask);
+        a1 = team_add<TLD>(a1, mask);
+        if (lt == 0) {
+            so[j * R + ra] = bad ? 0.f : round_bf16(a0 * xs);
+            if (has_b) so[j * R + rb] = bad ? 0.f : round_bf16(a1 * xs);
+            if (bad) atomicOr(status, kBadExpertId);
+        }
     }
 }
 
@@ -645,14 +710,10 @@ stack_decode_kernel(const __grid_constant__ StackParams p) {
         const int R = p.plan.R;
         float *so = reinterpret_cast<float *>(sm + p.plan.off_so);  // [k][R] expert outputs
         if (r0 < r1) {
-            const DownSrc src = {ly.table, ly.codes_base, ly.scales_base, p.codes_stride,
-                                 p.scales_stride};
             const uint8_t *rows_c = sm + p.plan.off_dn;
-            DownRows<TLD, KCHD, true, false, kSWarps> rows(
-                H, I, k, E, R, r0, r1, src, s_ids, rows_c,
-                rows_c + (size_t)k * R * ((size_t)I >> 1));
-            rows.fetch(rows.rr);
-            rows.run(reinterpret_cast<const uint32_t *>(sv), s_xs, so, p.status);
+            stk_down_rows<TLD, KCHD>(I, k, E, R, r1 - r0, s_ids, rows_c,
+                                     rows_c + (size_t)k * R * ((size_t)I >> 1),
+                                     reinterpret_cast<const uint32_t *>(sv), s_xs, so, p.status);
         }
         __syncthreads();
         STK_STAMP(7);
