@@ -460,7 +460,6 @@ down_decode_kernel(const DownParams p) {
     if (SR) {
         rows_ok = __syncthreads_and(mbar_wait(&s_rbar, 0u)) != 0;  // uniform over the CTA
         if (!rows_ok && threadIdx.x == 0) atomicOr(p.status, kTimeoutStatus);
-        if (rows_ok) rows.fetch(rows.rr);
     }
     if (rows_ok) rows.run(sh, s_xs, so, p.status, s_gs);
     __syncthreads();

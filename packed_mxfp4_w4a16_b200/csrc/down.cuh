@@ -280,11 +280,78 @@ struct DownRows {
         }
     }
 
-    // The loop, from the rows fetched by fetch(rr); h staged in sh / s_xs.
-    // NV: s_gs[q] is pair q's down multiplier (folded into the exact
+    // Rows in shared memory (SR): the same steps, each chunk's codes and scale
+    // read at use (no fetch ahead: fewer live registers, same bits).
+    __device__ __forceinline__ void run_smem(const uint32_t *sh, const float *s_xs, float *so,
+                                             unsigned *status, const float *s_gs) {
+        #pragma unroll 1
+        while (worker && rr < r1) {
+            const int t = rr / H;
+            const uint32_t *xv = sh + (size_t)(t * k + j) * (I >> 1);
+            const float xs = NV ? s_xs[t * k + j] * s_gs[t * k + j] : s_xs[t * k + j];
+            const int rb = rr + tps;
+            const bool second = rb < r1 && rb / H == t;
+            const int e = s_ids[t * k + j];
+            const bool bad = e < 0 || e >= E;
+            const size_t l0 = (size_t)j * R + (size_t)(rr - r0), l1 = (size_t)j * R + (size_t)(rb - r0);
+            const uint8_t *dc0 = rows_c + l0 * rc, *ds0 = rows_s + l0 * rs;
+            const uint8_t *dc1 = rows_c + l1 * rc, *ds1 = rows_s + l1 * rs;
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int u = 0; u < KCH; ++u) {
+                const int c = lt + TL * u;
+                if (c < C && !bad) {
+                    const uint4 *xq = reinterpret_cast<const uint4 *>(xv + (size_t)c * 16);
+                    uint32_t x[16];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 v = xq[q ^ ((c >> 1) & 3)];  // h_piece order
+                        x[4 * q] = v.x;
+                        x[4 * q + 1] = v.y;
+                        x[4 * q + 2] = v.z;
+                        x[4 * q + 3] = v.w;
+                    }
+                    const uint4 w0 = *reinterpret_cast<const uint4 *>(dc0 + (size_t)c * 16);
+                    if (NV) {
+                        float lo, hi, slo, shi;
+                        dot32_e2m1_f16_halves(w0, x, lo, hi);
+                        e4m3x2_to_f32(*reinterpret_cast<const uint16_t *>(ds0 + 2 * c), slo, shi);
+                        a0 = fmaf(hi, shi, fmaf(lo, slo, a0));
+                        if (second) {
+                            const uint4 w1 = *reinterpret_cast<const uint4 *>(dc1 + (size_t)c * 16);
+                            dot32_e2m1_f16_halves(w1, x, lo, hi);
+                            e4m3x2_to_f32(*reinterpret_cast<const uint16_t *>(ds1 + 2 * c), slo, shi);
+                            a1 = fmaf(hi, shi, fmaf(lo, slo, a1));
+                        }
+                    } else {
+                        a0 = fmaf(dot32_e2m1_f16(w0, x), e8m0_to_f32(ds0[c]), a0);
+                        if (second)
+                            a1 = fmaf(dot32_e2m1_f16(*reinterpret_cast<const uint4 *>(dc1 + (size_t)c * 16), x),
+                                      e8m0_to_f32(ds1[c]), a1);
+                    }
+                }
+            }
+            a0 = team_add<TL>(a0, mask);
+            a1 = team_add<TL>(a1, mask);
+            if (lt == 0) {
+                so[j * R + (rr - r0)] = bad ? 0.f : round_bf16(a0 * xs);
+                if (second) so[j * R + (rb - r0)] = bad ? 0.f : round_bf16(a1 * xs);
+                if (bad) atomicOr(status, kBadExpertId);
+            }
+            rr = second ? rr + 2 * tps : rr + tps;
+        }
+    }
+
+    // The loop, from the rows fetched by fetch(rr) (streamed rows; rows in
+    // shared memory go through run_smem, no fetch needed); h staged in sh /
+    // s_xs.  NV: s_gs[q] is pair q's down multiplier (folded into the exact
     // power-of-two staging scale).
     __device__ __forceinline__ void run(const uint32_t *sh, const float *s_xs, float *so,
                                         unsigned *status, const float *s_gs = nullptr) {
+        if constexpr (SR) {
+            run_smem(sh, s_xs, so, status, s_gs);
+            return;
+        }
         #pragma unroll 1
         while (worker && rr < r1) {
             const int t = rr / H;

@@ -366,10 +366,7 @@ layer_kernel(const GateUpParams p, const FusedRouteParams r, const LayerDownPara
         if (!ok && threadIdx.x == 0) atomicOr(p.status, kTimeoutStatus);
         ok = __syncthreads_and(ok && mbar_wait(&s_dbar, 0u)) != 0;  // uniform over the CTA
         DownRows<TLD, KCHD, true> rows(H, I, k, E, R, dr0, dr1, src, s_ids, rows_c, rows_s);
-        if (ok) {
-            rows.fetch(rows.rr);
-            rows.run(sh, s_xs, so, p.status);
-        }
+        if (ok) rows.run(sh, s_xs, so, p.status);
         __syncthreads();
         if (ok) down_combine(dr0, dr1, H, k, R, so, s_w, dp.residual, dp.y, nullptr);
         // no row copy may outlive the CTA (complete unless its wait timed out)
