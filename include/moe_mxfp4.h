@@ -372,9 +372,9 @@ MOE_API int moe_stack_create(const moe_handle_t *layers, int n_layers,
  * already enqueued keeps the pointers it was given.  NULL is a no-op. */
 MOE_API int moe_stack_destroy(moe_stack_t s);
 
-/* Bytes of device workspace the stack needs (tagged exchange words, launch
- * counters, status; about 35 KB for H 2048, I 1536, E 64, top-4).
- * Errors: ARG. */
+/* Bytes of device workspace the stack needs (tagged exchange words, one
+ * 4-word piece or one router logit per 128-byte line, launch counters,
+ * status; 140,544 bytes for H 2048, I 1536, E 64, top-4).  Errors: ARG. */
 MOE_API int moe_stack_workspace_bytes(moe_stack_t s, size_t *bytes);
 
 /* Give the stack its device workspace (caller-owned, 256-byte aligned, at

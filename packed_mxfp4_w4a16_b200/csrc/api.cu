@@ -880,9 +880,11 @@ StackWs stack_ws_layout(const moe_stack_ctx *s) {
         off = align_up(off + n, 256);
         return o;
     };
-    W.x_tag = take((size_t)s->H / 2 * sizeof(uint2));
-    W.lg_tag = take((size_t)s->E * sizeof(uint2));
-    W.h_tag = take((size_t)s->k * s->I / 2 * sizeof(uint2));
+    // tagged words spread one 4-word piece (or one logit) per 128-byte line
+    // (moe::kStkLine): see the stack kernel's exchange layout
+    W.x_tag = take((size_t)s->H / 8 * moe::kStkLine);
+    W.lg_tag = take((size_t)s->E * moe::kStkLine);
+    W.h_tag = take((size_t)s->k * s->I / 8 * moe::kStkLine);
     W.seq = take((size_t)s->num_sms * sizeof(unsigned));
     W.abort = take(sizeof(unsigned));
     W.status = take(sizeof(unsigned));

@@ -224,6 +224,15 @@ cudaError_t launch_layer(const GateUpParams &p, const FusedRouteParams &r,
 constexpr int kStackMaxLayers = 64;
 constexpr int kStackThreads = 512;  // 16 warps: 128 registers per thread
 constexpr int kStackTraceSlots = 16;  // phase time stamps per layer and CTA (profiling)
+// Exchange layout of the stack kernel's tagged words: word w of an exchange
+// buffer sits at uint2 index (w / 4) * kStkLineWords + w % 4, i.e. each
+// 4-word piece (and each router logit, at index e * kStkLineWords) on a
+// 128-byte line of its own.  Every CTA polls every line of an exchange, so
+// packed words would put ~150 readers' polls on a few L2 lines; spread, the
+// polls of one round go to as many lines as there are pieces (measured: a
+// grid-wide exchange of 1,036 words took 2.5 us packed, 1.5 us spread).
+constexpr size_t kStkLine = 128;
+constexpr int kStkLineWords = (int)(kStkLine / 8);
 
 struct StackLayer {
     const uint8_t *codes_base, *scales_base;  // contiguous [E][3][...], or null
@@ -252,6 +261,7 @@ struct StackParams {
     int32_t *ids_hist;                    // [L][k] or null
     float *w_hist;                        // [L][k] or null
     // workspace
+    // exchange buffers, words spread one piece per line (kStkLineWords)
     uint2 *x_tag;                         // [H/2] {tag, 2 x BF16} layer outputs
     uint2 *lg_tag;                        // [E] {tag, FP32} router logits
     uint2 *h_tag;                         // [k][I/2] {tag, 2 x BF16} SwiGLU outputs

@@ -66,6 +66,11 @@ constexpr size_t kStackSmemMax = 220 * 1024;  // dynamic; static shared memory i
 
 static_assert(kStackThreads % 32 == 0 && kSWarps >= kSRouteWarps, "whole warps, router warps included");
 
+// Word w of a spread exchange buffer (one 4-word piece per 128-byte line).
+__device__ __forceinline__ uint2 *stk_word(uint2 *base, int w) {
+    return base + (size_t)(w >> 2) * kStkLineWords + (w & 3);
+}
+
 // Tag of step l of a launch: 26 bits of launch count, 6 bits of layer.
 __device__ __forceinline__ unsigned stk_tag(unsigned base, int l) {
     return (base << 6) | (unsigned)l;
@@ -91,8 +96,9 @@ __device__ __forceinline__ uint64_t stk_clock() {
 }
 
 // By the calling thread t of nt polling threads: the 32-byte pieces
-// i = t, t + nt, ... < n of src (piece i = tagged words 4i .. 4i+3, two
-// single-copy-atomic 8-byte words per 16-byte load) until all four words of a
+// i = t, t + nt, ... < n of src (piece i = tagged words 4i .. 4i+3, at the
+// start of line i of the spread layout; two single-copy-atomic 8-byte words
+// per 16-byte load) until all four words of a
 // piece carry `tag`; put(i, values) receives each piece as it lands.  Every
 // round issues the loads of all pieces still missing at once, then checks
 // them; between rounds the thread sleeps, and every kAbortEvery rounds it
@@ -112,7 +118,7 @@ __device__ __forceinline__ bool poll_pieces(const uint2 *src, int n, int t, int 
 #pragma unroll
         for (int j = 0; j < kPollMaxJ; ++j)
             if ((todo >> j) & 1u) {
-                const uint2 *q = src + 4 * (size_t)(t + j * nt);
+                const uint2 *q = src + (size_t)(t + j * nt) * kStkLineWords;
                 ld_relaxed_gpu_2x64(q, w[j][0], w[j][1]);
                 ld_relaxed_gpu_2x64(q + 2, w[j][2], w[j][3]);
             }
@@ -158,8 +164,9 @@ static __device__ __noinline__ bool stk_gather_h(const uint2 *h_tag, int total, 
     });
 }
 
-// By one warp: all n (<= 256) tagged logits, copied into s_logits, with the
-// same round structure.  Every lane returns the same verdict.  Out of line.
+// By one warp: all n (<= 256) tagged logits (logit e on line e), copied into
+// s_logits, with the same round structure.  Every lane returns the same
+// verdict.  Out of line.
 static __device__ __noinline__ bool stk_gather_logits(const uint2 *ent, int n, unsigned tag,
                                                       float *s_logits, int limit,
                                                       const unsigned *abort, unsigned base) {
@@ -173,7 +180,8 @@ static __device__ __noinline__ bool stk_gather_logits(const uint2 *ent, int n, u
         uint2 v[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-            if ((todo >> j) & 1u) v[j] = ld_relaxed_gpu_v2(ent + lane + 32 * j);
+            if ((todo >> j) & 1u)
+                v[j] = ld_relaxed_gpu_v2(ent + (size_t)(lane + 32 * j) * kStkLineWords);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
             if (((todo >> j) & 1u) && v[j].x == tag) {
@@ -525,7 +533,8 @@ stack_decode_kernel(const __grid_constant__ StackParams p) {
 #pragma unroll
                 for (int i = 0; i < kSRouteWarps; ++i) logit += s_red[1][i];
                 if (ly.bias) logit += s_bias[l];
-                st_relaxed_gpu_v2(p.lg_tag + b, tag, __float_as_uint(logit));
+                st_relaxed_gpu_v2(p.lg_tag + (size_t)b * kStkLineWords, tag,
+                                  __float_as_uint(logit));
                 if (p.logits_hist) p.logits_hist[(size_t)l * E + b] = logit;
             }
             float mx = 0.f;
@@ -673,7 +682,7 @@ stack_decode_kernel(const __grid_constant__ StackParams p) {
                                ((uint32_t)f32_to_bf16(swiglu_h(v[1][0], v[1][1], xs)) << 16);
                     else
                         atomicOr(p.status, kBadExpertId);
-                    st_relaxed_gpu_v2(p.h_tag + gr / 2, tag, word);
+                    st_relaxed_gpu_v2(stk_word(p.h_tag, gr / 2), tag, word);
                 }
             }
         }
@@ -735,7 +744,7 @@ stack_decode_kernel(const __grid_constant__ StackParams p) {
                 y = round_bf16(bf16_to_f32(rb) + y);
                 word |= (uint32_t)f32_to_bf16(y) << (16 * d);
             }
-            st_relaxed_gpu_v2(p.x_tag + n / 2, tag, word);
+            st_relaxed_gpu_v2(stk_word(p.x_tag, n / 2), tag, word);
             if (l == L - 1) reinterpret_cast<uint32_t *>(p.r)[n / 2] = word;
         }
         __syncthreads();  // sx, so, s_w are rewritten by the next layer
