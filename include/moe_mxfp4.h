@@ -352,16 +352,18 @@ MOE_API int moe_set_fusion(moe_handle_t h, int mode);
 typedef struct moe_stack_ctx *moe_stack_t;
 
 /* Create a stack over n_layers (1..64) layer handles that are already bound
- * to MXFP4 weights (moe_load_packed or moe_load_expert_table) on the current
- * device and share E, H, I, top_k.  router_w: HOST array of n_layers device
+ * to MXFP4 weights (moe_load_packed or moe_load_expert_table), or all to
+ * NVFP4 weights (moe_load_packed_nvfp4), on the current device and share E,
+ * H, I, top_k.  router_w: HOST array of n_layers device
  * pointers, BF16 [E][H] each (16-byte aligned); router_bias: NULL or a HOST
  * array of n_layers device pointers, FP32 [E] or NULL each.  The layers'
  * weight bindings and these pointers are read now: rebinding a layer later
  * needs a new stack; the memory must stay valid until moe_stack_destroy.
  * Shapes the stack kernel holds: H a multiple of 512 up to 2048, I a multiple
  * of 128 up to 4096 with I/32 in {12, 16, 32, 48, 64} (I = 384, 512, 1024,
- * 1536, 2048), top_k <= E <= 256 and E <= the SM count; NVFP4 layers are not
- * taken.  Errors: ARG (including a shape or format outside that set: run the
+ * 1536, 2048), top_k <= E <= 256 and E <= the SM count; sym8 layers and
+ * stacks that mix formats are not taken.  Errors: ARG (including a shape or
+ * format outside that set: run the
  * layers with moe_layer_ex instead), NOT_LOADED, NOT_DEVICE, ALIGN,
  * UNSUPPORTED, CUDA. */
 MOE_API int moe_stack_create(const moe_handle_t *layers, int n_layers,

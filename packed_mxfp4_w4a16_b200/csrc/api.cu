@@ -856,6 +856,7 @@ int moe_set_fusion(moe_handle_t h, int mode) {
 
 struct moe_stack_ctx {
     int L = 0, E = 0, H = 0, I = 0, k = 0;
+    int nv = 0;  // NVFP4 layers
     int device = -1;
     int num_sms = 0;
     uint8_t *ws = nullptr;
@@ -907,7 +908,8 @@ int moe_stack_create(const moe_handle_t *layers, int n_layers, const uint16_t *c
         const moe_ctx *h = layers[l];
         if (!h || h->E != l0->E || h->H != l0->H || h->I != l0->I || h->k != l0->k) return MOE_ERR_ARG;
         if (!h->loaded) return MOE_ERR_NOT_LOADED;
-        if (h->nv || h->s8) return MOE_ERR_ARG;  // the stack kernel reads MXFP4 experts
+        // the stack kernel reads MXFP4 or NVFP4 experts, one format per stack
+        if (h->s8 || h->nv != l0->nv) return MOE_ERR_ARG;
         if (h->device != l0->device) return MOE_ERR_NOT_DEVICE;
     }
     int dev = -1, sms = 0;
@@ -915,7 +917,7 @@ int moe_stack_create(const moe_handle_t *layers, int n_layers, const uint16_t *c
     if (rc != MOE_OK) return rc;
     if (dev != l0->device) return MOE_ERR_NOT_DEVICE;
     moe::StackPlan plan;
-    if (!moe::stack_plan(l0->E, l0->H, l0->I, l0->k, sms, &plan)) return MOE_ERR_ARG;
+    if (!moe::stack_plan(l0->E, l0->H, l0->I, l0->k, sms, &plan, l0->nv)) return MOE_ERR_ARG;
     for (int l = 0; l < n_layers; ++l) {
         if ((rc = check_device_ptr(l0, router_w[l], 16)) != MOE_OK) return rc;
         if (router_bias && router_bias[l] && (rc = check_device_ptr(l0, router_bias[l], 4)) != MOE_OK)
@@ -928,6 +930,7 @@ int moe_stack_create(const moe_handle_t *layers, int n_layers, const uint16_t *c
     s->H = l0->H;
     s->I = l0->I;
     s->k = l0->k;
+    s->nv = l0->nv;
     s->device = dev;
     s->num_sms = sms;
     s->plan = plan;
@@ -939,6 +942,7 @@ int moe_stack_create(const moe_handle_t *layers, int n_layers, const uint16_t *c
         ly.table = h->d_table;
         ly.router_w = router_w[l];
         ly.bias = router_bias ? router_bias[l] : nullptr;
+        ly.gscale = h->gscale;
     }
     *out = s;
     return MOE_OK;
@@ -1017,8 +1021,9 @@ int moe_stack_decode(moe_stack_t s, uint16_t *r, uint16_t *r_hist, uint16_t *xn_
     p.H = s->H;
     p.I = s->I;
     p.k = s->k;
+    p.nv = s->nv;
     p.codes_stride = (size_t)s->I * s->H / 2;
-    p.scales_stride = (size_t)s->I * s->H / 32;
+    p.scales_stride = (size_t)s->I * s->H / (s->nv ? 16 : 32);
     p.r = r;
     p.r_hist = r_hist;
     p.xn_hist = xn_hist;

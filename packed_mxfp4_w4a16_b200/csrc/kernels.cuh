@@ -239,6 +239,7 @@ struct StackLayer {
     const ExpertPtrs *table;                  // device expert table (codes_base null)
     const uint16_t *router_w;                 // [E][H] BF16
     const float *bias;                        // [E] or null
+    const float *gscale;                      // NVFP4: [E][2] FP32 multipliers (gate/up, down)
 };
 
 // Shared-memory plan of the stack kernel (host-computed, passed by value).
@@ -253,6 +254,7 @@ struct StackPlan {
 
 struct StackParams {
     int L, E, H, I, k;
+    int nv;                               // NVFP4 layers (E4M3 scale per 16) else MXFP4
     size_t codes_stride, scales_stride;   // bytes per matrix (contiguous layers)
     uint16_t *r;                          // [H] residual stream, in and out
     uint16_t *r_hist;                     // [L][H] each layer's input, or null
@@ -275,8 +277,8 @@ struct StackParams {
 };
 
 // False when the shape is outside what the stack kernel holds (then the
-// layers run one by one).
-bool stack_plan(int E, int H, int I, int k, int grid, StackPlan *plan);
+// layers run one by one).  nv: NVFP4 layers (twice the scale bytes).
+bool stack_plan(int E, int H, int I, int k, int grid, StackPlan *plan, int nv = 0);
 cudaError_t launch_stack(const StackParams &p, int grid, cudaStream_t s);
 
 cudaError_t launch_debug_dequant(const uint8_t *codes, const uint8_t *scales, int64_t n,

@@ -222,14 +222,15 @@ __device__ __forceinline__ float swiglu_h(float ag, float au, float xs) {
 // order at full bandwidth (issued together, they would share the memory
 // system and all land at the end), so the GEMVs of the first pieces run while
 // the later ones stream.  Gate/up layout: codes [2][NR][H/2] (gate, up), then
-// scales [2][NR][H/32]; down layout: codes [k][R][I/2], scales [k][R][I/32].
+// scales [2][NR][H/32] (NVFP4: [2][NR][H/16]); down layout: codes [k][R][I/2],
+// scales [k][R][I/32] (NVFP4: I/16).
 // Out of line.
 static __device__ __noinline__ void stk_issue_layer(
     const uint8_t *cb, const uint8_t *sb, const ExpertPtrs *tab, size_t cstride, size_t sstride,
     const int *s_ids, int E, int H, int I, int k, int pb0, int np, int ppc, int NR, uint8_t *gu,
     uint64_t *sbar, uint64_t *gbar, int r0, int r1, int R, uint8_t *rows_c, uint8_t *rows_s,
-    uint64_t *dbar, uint64_t pol) {
-    const size_t rc = (size_t)H >> 1, rs = (size_t)H >> 5;
+    uint64_t *dbar, uint64_t pol, int nv) {
+    const size_t rc = (size_t)H >> 1, rs = (size_t)H >> (nv ? 4 : 5);
     auto codes = [&](int e, int m) {
         return cb ? cb + (size_t)(3 * e + m) * cstride : tab[e].codes[m];
     };
@@ -272,7 +273,7 @@ static __device__ __noinline__ void stk_issue_layer(
                               (unsigned)(n * rc), &gbar[c], pol);
         });
     }
-    const size_t drc = (size_t)I >> 1, drs = (size_t)I >> 5, dn = (size_t)(r1 - r0);
+    const size_t drc = (size_t)I >> 1, drs = (size_t)I >> (nv ? 4 : 5), dn = (size_t)(r1 - r0);
     bytes = 0;
     #pragma unroll 1
     for (int j = 0; j < k; ++j) {
@@ -296,9 +297,12 @@ static __device__ __noinline__ void stk_issue_layer(
 // words, h_piece order) in shared memory.  Warp w serves slot j = w % k; its
 // teams of TLD lanes take local rows ti, ti + tps, ... two at a time (the
 // h chunk loaded once for both rows), lane lt the 16-byte chunks lt + TLD u
-// of each row, one E8M0 group each.  Per row the sums and their order are
-// those of the per-layer down kernel (same bits).  so[j R + row] = BF16(o).
-template <int TLD, int KCHD>
+// of each row, one E8M0 group each (NV: two E4M3 scales per chunk, each
+// 16-element half sum scaled in FP32).  Per row the sums and their order are
+// those of the per-layer down kernel (same bits).  so[j R + row] = BF16(o),
+// o = sum * s_xs[j] (NV: s_xs holds the staging scale times the expert's down
+// multiplier).
+template <int TLD, int KCHD, bool NV>
 __device__ __forceinline__ void stk_down_rows(int I, int k, int E, int R, int nr, const int *s_ids,
                                               const uint8_t *rows_c, const uint8_t *rows_s,
                                               const uint32_t *sh, const float *s_xs, float *so,
@@ -312,7 +316,7 @@ __device__ __forceinline__ void stk_down_rows(int I, int k, int E, int R, int nr
     const int lt = lane & (TLD - 1);
     const unsigned mask = team_mask<TLD>(lane);
     const int C = I >> 5;
-    const size_t rc = (size_t)I >> 1, rs = (size_t)I >> 5;
+    const size_t rc = (size_t)I >> 1, rs = (size_t)I >> (NV ? 4 : 5);
     const int e = s_ids[j];
     const bool bad = e < 0 || e >= E;
     const uint32_t *xv = sh + (size_t)j * (I >> 1);
@@ -338,11 +342,26 @@ __device__ __forceinline__ void stk_down_rows(int I, int k, int E, int R, int nr
                     x[4 * q + 2] = v.z;
                     x[4 * q + 3] = v.w;
                 }
-                a0 = fmaf(dot32_e2m1_f16(*reinterpret_cast<const uint4 *>(ca + (size_t)c * 16), x),
-                          e8m0_to_f32(sa[c]), a0);
-                if (has_b)
-                    a1 = fmaf(dot32_e2m1_f16(*reinterpret_cast<const uint4 *>(cb + (size_t)c * 16), x),
-                              e8m0_to_f32(sb[c]), a1);
+                if (NV) {
+                    float lo, hi, slo, shi;
+                    dot32_e2m1_f16_halves(*reinterpret_cast<const uint4 *>(ca + (size_t)c * 16), x, lo,
+                                          hi);
+                    e4m3x2_to_f32(*reinterpret_cast<const uint16_t *>(sa + 2 * c), slo, shi);
+                    a0 = fmaf(hi, shi, fmaf(lo, slo, a0));
+                    if (has_b) {
+                        dot32_e2m1_f16_halves(*reinterpret_cast<const uint4 *>(cb + (size_t)c * 16), x,
+                                              lo, hi);
+                        e4m3x2_to_f32(*reinterpret_cast<const uint16_t *>(sb + 2 * c), slo, shi);
+                        a1 = fmaf(hi, shi, fmaf(lo, slo, a1));
+                    }
+                } else {
+                    a0 = fmaf(dot32_e2m1_f16(*reinterpret_cast<const uint4 *>(ca + (size_t)c * 16), x),
+                              e8m0_to_f32(sa[c]), a0);
+                    if (has_b)
+                        a1 = fmaf(
+                            dot32_e2m1_f16(*reinterpret_cast<const uint4 *>(cb + (size_t)c * 16), x),
+                            e8m0_to_f32(sb[c]), a1);
+                }
             }
         }
         a0 = team_add<TLD>(a0, mask);
@@ -368,7 +387,8 @@ __device__ __forceinline__ void stk_down_rows(int I, int k, int E, int R, int nr
 
 // KCH: 16-byte chunks per lane of a gate/up row (H = 32 * 32 * KCH at most);
 // TLD / KCHD: the down phase's team of TLD lanes holding KCHD chunks each.
-template <int KCH, int TLD, int KCHD>
+// NV: NVFP4 layers (E4M3 scale per 16 elements, FP32 multipliers per expert).
+template <int KCH, int TLD, int KCHD, bool NV>
 __global__ void __launch_bounds__(kStackThreads, 1)
 stack_decode_kernel(const __grid_constant__ StackParams p) {
     extern __shared__ __align__(128) uint8_t sm[];
@@ -596,7 +616,7 @@ stack_decode_kernel(const __grid_constant__ StackParams p) {
             stk_issue_layer(ly.codes_base, ly.scales_base, ly.table, p.codes_stride, p.scales_stride,
                             s_ids, E, H, I, k, pb0, np, ppc, NR, gu, &sbar, gbar, r0, r1, p.plan.R,
                             rows_c, rows_c + (size_t)k * p.plan.R * ((size_t)I >> 1), &dbar,
-                            l2_evict_first_policy());
+                            l2_evict_first_policy(), NV ? 1 : 0);
             s_copied = l;
             STK_STAMP(4);
         }
@@ -609,7 +629,7 @@ stack_decode_kernel(const __grid_constant__ StackParams p) {
             const float xs = pow2(s_x16exp);
             const uint4 *sx16 = reinterpret_cast<const uint4 *>(sm + p.plan.off_x16);
             const int C = H >> 5;
-            const size_t rc = (size_t)H >> 1, rs = (size_t)H >> 5;
+            const size_t rc = (size_t)H >> 1, rs = (size_t)H >> (NV ? 4 : 5);
             if (warp < np && !mbar_wait(&sbar, (unsigned)l & 1u)) ok = false;
             #pragma unroll 1
             for (int pp = warp; pp < np && ok; pp += kSWarps) {
@@ -639,36 +659,77 @@ stack_decode_kernel(const __grid_constant__ StackParams p) {
                             const size_t row = (size_t)m * NR + lr + rr;
                             if (c < C && !bad) {
                                 cw[rr][m] = *reinterpret_cast<const uint4 *>(gu + row * rc + (size_t)c * 16);
-                                sw[rr][m] = gu[2 * (size_t)NR * rc + row * rs + c];
+                                sw[rr][m] = NV ? *reinterpret_cast<const uint16_t *>(
+                                                     gu + 2 * (size_t)NR * rc + row * rs + 2 * c)
+                                               : gu[2 * (size_t)NR * rc + row * rs + c];
                             } else {
                                 cw[rr][m] = make_uint4(0u, 0u, 0u, 0u);
-                                sw[rr][m] = 127u;
+                                sw[rr][m] = NV ? 0x3838u : 127u;
                             }
                         }
-                    float a[2][2][2];  // [row][gate, up][even, odd elements]
-#pragma unroll
-                    for (int rr = 0; rr < 2; ++rr)
-#pragma unroll
-                        for (int m = 0; m < 2; ++m) a[rr][m][0] = a[rr][m][1] = 0.f;
-                    // the chunk's four 8-element pieces in order, each against
-                    // all four rows (per row the order of chunks_dot)
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const uint4 xv = c < C ? sx16[c * 4 + q4] : make_uint4(0u, 0u, 0u, 0u);
+                    if (NV) {
+                        // each chunk's two 16-element halves (words 0-1, 2-3),
+                        // each half sum scaled by its E4M3 scale in FP32 (the
+                        // order of chunks_dot_nv)
+                        float a[2][2][4];
 #pragma unroll
                         for (int rr = 0; rr < 2; ++rr)
 #pragma unroll
-                            for (int m = 0; m < 2; ++m) {
-                                const uint4 cc = cw[rr][m];
-                                const uint32_t w = q4 == 0 ? cc.x : q4 == 1 ? cc.y : q4 == 2 ? cc.z : cc.w;
-                                dot8_e2m1_f16(w, xv.x, xv.y, xv.z, xv.w, a[rr][m][0], a[rr][m][1]);
+                            for (int m = 0; m < 2; ++m)
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) a[rr][m][i] = 0.f;
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const uint4 xv = c < C ? sx16[c * 4 + q4] : make_uint4(0u, 0u, 0u, 0u);
+                            const int i0 = (q4 & 1) * 2;
+#pragma unroll
+                            for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+                                for (int m = 0; m < 2; ++m) {
+                                    const uint4 cc = cw[rr][m];
+                                    const uint32_t w = q4 == 0 ? cc.x : q4 == 1 ? cc.y : q4 == 2 ? cc.z : cc.w;
+                                    dot8_e2m1_f16(w, xv.x, xv.y, xv.z, xv.w, a[rr][m][i0], a[rr][m][i0 + 1]);
+                                }
+                            if (q4 & 1) {
+#pragma unroll
+                                for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+                                    for (int m = 0; m < 2; ++m) {
+                                        float slo, shi;
+                                        e4m3x2_to_f32(sw[rr][m], slo, shi);
+                                        const float half = (a[rr][m][0] + a[rr][m][1]) + (a[rr][m][2] + a[rr][m][3]);
+                                        v[rr][m] = fmaf(half, q4 == 1 ? slo : shi, v[rr][m]);
+#pragma unroll
+                                        for (int i = 0; i < 4; ++i) a[rr][m][i] = 0.f;
+                                    }
                             }
+                        }
+                    } else {
+                        float a[2][2][2];  // [row][gate, up][even, odd elements]
+#pragma unroll
+                        for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+                            for (int m = 0; m < 2; ++m) a[rr][m][0] = a[rr][m][1] = 0.f;
+                        // the chunk's four 8-element pieces in order, each against
+                        // all four rows (per row the order of chunks_dot)
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const uint4 xv = c < C ? sx16[c * 4 + q4] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                            for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+                                for (int m = 0; m < 2; ++m) {
+                                    const uint4 cc = cw[rr][m];
+                                    const uint32_t w = q4 == 0 ? cc.x : q4 == 1 ? cc.y : q4 == 2 ? cc.z : cc.w;
+                                    dot8_e2m1_f16(w, xv.x, xv.y, xv.z, xv.w, a[rr][m][0], a[rr][m][1]);
+                                }
+                        }
+#pragma unroll
+                        for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+                            for (int m = 0; m < 2; ++m)
+                                v[rr][m] = fmaf(a[rr][m][0] + a[rr][m][1], e8m0_to_f32(sw[rr][m]), v[rr][m]);
                     }
-#pragma unroll
-                    for (int rr = 0; rr < 2; ++rr)
-#pragma unroll
-                        for (int m = 0; m < 2; ++m)
-                            v[rr][m] = fmaf(a[rr][m][0] + a[rr][m][1], e8m0_to_f32(sw[rr][m]), v[rr][m]);
                 }
 #pragma unroll
                 for (int rr = 0; rr < 2; ++rr)
@@ -677,9 +738,12 @@ stack_decode_kernel(const __grid_constant__ StackParams p) {
                 if (tid == 0 && pp == 0) STK_STAMP(11);
                 if (lane == 0) {
                     uint32_t word = 0u;
+                    // NVFP4: the expert's gate/up multiplier joins the exact
+                    // power-of-two staging scale (as in the per-layer kernel)
+                    const float sx = NV && !bad ? xs * __ldg(ly.gscale + 2 * e) : xs;
                     if (!bad)
-                        word = (uint32_t)f32_to_bf16(swiglu_h(v[0][0], v[0][1], xs)) |
-                               ((uint32_t)f32_to_bf16(swiglu_h(v[1][0], v[1][1], xs)) << 16);
+                        word = (uint32_t)f32_to_bf16(swiglu_h(v[0][0], v[0][1], sx)) |
+                               ((uint32_t)f32_to_bf16(swiglu_h(v[1][0], v[1][1], sx)) << 16);
                     else
                         atomicOr(p.status, kBadExpertId);
                     st_relaxed_gpu_v2(stk_word(p.h_tag, gr / 2), tag, word);
@@ -711,7 +775,12 @@ stack_decode_kernel(const __grid_constant__ StackParams p) {
             o.w = f32x2_to_f16x2(bf16_to_f32(v.w & 0xFFFFu) * sf, bf16_to_f32(v.w >> 16) * sf);
             sv[i] = o;
         }
-        if (tid < k) s_xs[tid] = pow2(f16_stage_exponent(__uint_as_float(s_hmax[tid])));
+        if (tid < k) {
+            const float xs = pow2(f16_stage_exponent(__uint_as_float(s_hmax[tid])));
+            const int e = s_ids[tid];
+            // NVFP4: times the expert's down multiplier (an exact product)
+            s_xs[tid] = NV && e >= 0 && e < E ? xs * __ldg(ly.gscale + 2 * e + 1) : xs;
+        }
         __syncthreads();
         STK_STAMP(15);
 
@@ -720,7 +789,7 @@ stack_decode_kernel(const __grid_constant__ StackParams p) {
         float *so = reinterpret_cast<float *>(sm + p.plan.off_so);  // [k][R] expert outputs
         if (r0 < r1) {
             const uint8_t *rows_c = sm + p.plan.off_dn;
-            stk_down_rows<TLD, KCHD>(I, k, E, R, r1 - r0, s_ids, rows_c,
+            stk_down_rows<TLD, KCHD, NV>(I, k, E, R, r1 - r0, s_ids, rows_c,
                                      rows_c + (size_t)k * R * ((size_t)I >> 1),
                                      reinterpret_cast<const uint32_t *>(sv), s_xs, so, p.status);
         }
@@ -794,11 +863,11 @@ int stack_variant(int H, int I) {
     }
 }
 
-template <int KCH, int TLD, int KCHD>
+template <int KCH, int TLD, int KCHD, bool NV>
 cudaError_t launch_stk(const StackParams &p, int grid, cudaStream_t s) {
     static PerDeviceOnce once;
     cudaError_t e = per_device_once(once, [] {
-        return cudaFuncSetAttribute(stack_decode_kernel<KCH, TLD, KCHD>,
+        return cudaFuncSetAttribute(stack_decode_kernel<KCH, TLD, KCHD, NV>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)kStackSmemMax);
     });
@@ -815,14 +884,14 @@ cudaError_t launch_stk(const StackParams &p, int grid, cudaStream_t s) {
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, stack_decode_kernel<KCH, TLD, KCHD>, p);
+    return cudaLaunchKernelEx(&cfg, stack_decode_kernel<KCH, TLD, KCHD, NV>, p);
 }
 
 size_t al128(size_t v) { return (v + 127) & ~(size_t)127; }
 
 }  // namespace
 
-bool stack_plan(int E, int H, int I, int k, int grid, StackPlan *pl) {
+bool stack_plan(int E, int H, int I, int k, int grid, StackPlan *pl, int nv) {
     if (grid < 1 || E < 1 || E > grid || E > kFusedMaxE || k < 1 || k > kMaxTopK || k > E)
         return false;
     if (H % 512 != 0 || H > 2048 || I % 128 != 0 || I > 4096) return false;
@@ -830,19 +899,21 @@ bool stack_plan(int E, int H, int I, int k, int grid, StackPlan *pl) {
     // the gathering threads hold at most kPollMaxJ pieces each
     if (H / 8 > kXThreads * kPollMaxJ || k * I / 8 > kHThreads * kPollMaxJ) return false;
     StackPlan s = {};
-    s.U = (I % 256 == 0) ? 2 : 4;  // rows per unit: U * I/32 scale bytes are a 16-byte multiple
+    // rows per unit (even: the combine writes row pairs): U * (I/32 or I/16)
+    // scale bytes are a 16-byte multiple
+    s.U = nv ? 2 : ((I % 256 == 0) ? 2 : 4);
     const int NU = H / s.U;
     s.R = s.U * ((NU + grid - 1) / grid);
     if (kSWarps / k < 1) return false;  // the down phase needs a warp per slot
     const int P = k * I / 2;
     s.np_max = (P + grid - 1) / grid;
     s.ppc = (s.np_max + kStackPieces - 1) / kStackPieces;
-    const size_t rc = (size_t)H / 2, rs = (size_t)H / 32;
+    const size_t rc = (size_t)H / 2, rs = (size_t)H / (nv ? 16 : 32);
     size_t off = 0;
     s.off_gu = (unsigned)off;
     off = al128(off + (size_t)2 * s.np_max * 2 * (rc + rs));
     s.off_dn = (unsigned)off;
-    off = al128(off + (size_t)k * s.R * ((size_t)I / 2 + (size_t)I / 32));
+    off = al128(off + (size_t)k * s.R * ((size_t)I / 2 + (size_t)I / (nv ? 16 : 32)));
     s.off_rt = (unsigned)off;
     off = al128(off + (size_t)2 * H * 2);
     s.off_sx = (unsigned)off;
@@ -860,14 +931,15 @@ bool stack_plan(int E, int H, int I, int k, int grid, StackPlan *pl) {
 }
 
 cudaError_t launch_stack(const StackParams &p, int grid, cudaStream_t s) {
+    const bool nv = p.nv != 0;
     switch (stack_variant(p.H, p.I)) {
-    case 0: return launch_stk<1, 4, 3>(p, grid, s);
-    case 1: return launch_stk<1, 16, 1>(p, grid, s);
-    case 2: return launch_stk<1, 32, 1>(p, grid, s);
-    case 3: return launch_stk<2, 16, 3>(p, grid, s);
-    case 4: return launch_stk<2, 32, 2>(p, grid, s);
-    case 5: return launch_stk<2, 16, 1>(p, grid, s);
-    case 6: return launch_stk<2, 32, 1>(p, grid, s);
+    case 0: return nv ? launch_stk<1, 4, 3, true>(p, grid, s) : launch_stk<1, 4, 3, false>(p, grid, s);
+    case 1: return nv ? launch_stk<1, 16, 1, true>(p, grid, s) : launch_stk<1, 16, 1, false>(p, grid, s);
+    case 2: return nv ? launch_stk<1, 32, 1, true>(p, grid, s) : launch_stk<1, 32, 1, false>(p, grid, s);
+    case 3: return nv ? launch_stk<2, 16, 3, true>(p, grid, s) : launch_stk<2, 16, 3, false>(p, grid, s);
+    case 4: return nv ? launch_stk<2, 32, 2, true>(p, grid, s) : launch_stk<2, 32, 2, false>(p, grid, s);
+    case 5: return nv ? launch_stk<2, 16, 1, true>(p, grid, s) : launch_stk<2, 16, 1, false>(p, grid, s);
+    case 6: return nv ? launch_stk<2, 32, 1, true>(p, grid, s) : launch_stk<2, 32, 1, false>(p, grid, s);
     default: return cudaErrorInvalidValue;
     }
 }

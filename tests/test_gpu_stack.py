@@ -30,10 +30,11 @@ def _hist(shape, n):
                 topk_w=torch.zeros(n, shape.top_k, dtype=torch.float32, device=dev))
 
 
-def _check_layers_against_oracle(shape, layers, hist, r_out):
+def _check_layers_against_oracle(shape, layers, hist, r_out, nvfp4=False):
     """Layer l: xn = RMSNorm(r_in) and the routing of xn against the oracle;
     the layer output (next layer's input, or the final r) against the
-    oracle's expert FFN + combine + residual fed the GPU's xn and routing."""
+    oracle's expert FFN + combine + residual fed the GPU's xn and routing
+    (nvfp4: the oracle's NVFP4 experts)."""
     n = len(layers)
     r_hist = host_bf16(hist["r_hist"])
     xn_hist = host_bf16(hist["xn_hist"])
@@ -46,9 +47,14 @@ def _check_layers_against_oracle(shape, layers, hist, r_out):
         assert_close_rms(xn_hist[l:l + 1], xn_r, what=f"rmsnorm layer {l}")
         rids, rw, rlg = oracle.route(xn_hist[l:l + 1], L.router_w, L.router_b, shape.top_k)
         ties += check_routing(ids[l:l + 1], w[l:l + 1], logits[l:l + 1], rids, rw, rlg, shape.top_k)
-        out_ref = oracle.moe_forward(xn_hist[l:l + 1], ids[l:l + 1], w[l:l + 1].astype(np.float64),
-                                     L.codes, L.scales, shape.E, shape.H, shape.I,
-                                     residual=r_hist[l:l + 1])
+        w64 = w[l:l + 1].astype(np.float64)
+        if nvfp4:
+            out_ref = oracle.moe_forward_nvfp4(xn_hist[l:l + 1], ids[l:l + 1], w64, L.codes,
+                                               L.scales, L.gscales, shape.E, shape.H, shape.I,
+                                               residual=r_hist[l:l + 1])
+        else:
+            out_ref = oracle.moe_forward(xn_hist[l:l + 1], ids[l:l + 1], w64, L.codes, L.scales,
+                                         shape.E, shape.H, shape.I, residual=r_hist[l:l + 1])
         out_gpu = r_hist[l + 1:l + 2] if l + 1 < n else r_out
         assert_close_rms(out_gpu, out_ref, what=f"layer {l} output", max_ulps=2)
     return ties
@@ -97,6 +103,42 @@ def test_stack_kernel_matches_oracle_and_layer_path(shape, n_layers, bias):
     st.enqueue_layers()
     torch.cuda.synchronize()
     np.testing.assert_array_equal(host_bf16(st.r), r2)
+    assert st.status() == 0
+    st.close()
+
+
+@pytest.mark.parametrize("shape,n_layers", [(synth.L24B, 4), (synth.TINY, 5)])
+def test_stack_kernel_nvfp4_matches_oracle_and_layer_path(shape, n_layers):
+    """NVFP4 experts (an E4M3 scale per 16 elements, FP32 multipliers per
+    expert) in the one-launch stack: bit-for-bit the same step run one layer
+    at a time (route + NVFP4 gate/up + down kernels), every layer within the
+    oracle's tolerance (NVFP4 expert FFN fed the GPU's routed vector and
+    routing), and a graph replay gives the eager bits."""
+    layers = [synth.make_layer_nvfp4(shape, seed=63, layer=l) for l in range(n_layers)]
+    w = [dev_layer(L) + (torch.from_numpy(L.gscales).cuda(),) for L in layers]
+    st = moe.MoEStack(w, shape.E, shape.H, shape.I, shape.top_k)
+    assert st.stack is not None
+    r0 = dev_bf16(synth.make_tokens(1, shape.H, seed=63, stream=3))
+    st.r.copy_(r0)
+    st.enqueue_layers()
+    torch.cuda.synchronize()
+    r_layers = host_bf16(st.r).copy()
+    ids_layers = st.ids.cpu().numpy().copy()
+    hist = _hist(shape, n_layers)
+    st.r.copy_(r0)
+    moe.moe_stack_decode(st.stack, st.r, **hist)
+    torch.cuda.synchronize()
+    assert st.status() == 0
+    r_stack = host_bf16(st.r).copy()
+    np.testing.assert_array_equal(r_stack, r_layers)
+    np.testing.assert_array_equal(hist["topk_ids"].cpu().numpy(), ids_layers.reshape(n_layers, -1))
+    _check_layers_against_oracle(shape, layers, hist, r_stack, nvfp4=True)
+    st.r.copy_(r0)
+    st.capture()
+    st.r.copy_(r0)
+    st.step()
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host_bf16(st.r), r_stack)
     assert st.status() == 0
     st.close()
 
@@ -199,18 +241,20 @@ def test_stack_wait_that_gives_up_is_reported_and_the_next_step_runs():
 
 
 def test_stack_refuses_what_it_does_not_hold():
-    """NVFP4 layers and several tokens per step run one layer at a time."""
+    """A stack mixing MXFP4 and NVFP4 layers, and several tokens per step,
+    run one layer at a time (moe_stack_create refuses the mixed stack)."""
     shape = synth.L24B
     L = synth.make_layer_nvfp4(shape, seed=65)
+    Lm = synth.make_layer(shape, seed=65)
     codes, scales = torch.from_numpy(L.codes).cuda(), torch.from_numpy(L.scales).cuda()
     gs = torch.from_numpy(L.gscales).cuda()
     rw = dev_bf16(L.router_w)
-    st = moe.MoEStack([(codes, scales, rw, None, gs)], shape.E, shape.H, shape.I, shape.top_k)
+    st = moe.MoEStack([dev_layer(Lm), (codes, scales, rw, None, gs)], shape.E, shape.H, shape.I,
+                      shape.top_k)
     assert st.stack is None
     with pytest.raises(moe.MoEError):
-        moe.moe_stack_create([st.layers[0].handle], [rw])
+        moe.moe_stack_create([x.handle for x in st.layers], [x.router_w for x in st.layers])
     st.close()
-    Lm = synth.make_layer(shape, seed=65)
     st2 = moe.MoEStack([dev_layer(Lm)], shape.E, shape.H, shape.I, shape.top_k, T=2)
     assert st2.stack is None
     st2.close()
