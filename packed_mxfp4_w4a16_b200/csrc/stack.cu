@@ -20,8 +20,15 @@
 // grid drain and a launch; here the CTAs (one per SM, co-resident by a
 // cooperative launch) stay in the kernel for all layers and hand each step over
 // through 8-byte words {tag, value} in global memory, single-copy atomic, so a
-// reader that sees this step's tag also sees the value written with it.  Every
+// reader that sees this step's tag also sees the value written with it.  The
+// words sit one 4-word piece (or one router logit) per 128-byte line, so the
+// polls of ~150 CTAs spread over as many L2 lines as there are pieces.  Every
 // wait is bounded.
+//
+// Weight formats: MXFP4 (E8M0 scale per 32) or, with NV, NVFP4 (two E4M3
+// scales per 32-element chunk, each 16-element half sum scaled in FP32; the
+// expert's FP32 gate/up and down multipliers folded into the power-of-two
+// staging scales), one format per stack.
 //
 // One layer, CTA b of G:
 //   A  the layer input r (the previous layer's tagged outputs, or the input
@@ -48,8 +55,8 @@
 //      output rows are published as tagged words (the next layer's input).
 //
 // The reduction orders are those of the one-launch-per-step kernels (router
-// kernel, bulk-copy gate/up kernel, down kernel), so the results are
-// bit-identical to running the layers one by one.
+// kernel, bulk-copy gate/up kernel, down kernel, in either format), so the
+// results are bit-identical to running the layers one by one.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
