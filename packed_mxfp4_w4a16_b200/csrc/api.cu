@@ -423,7 +423,8 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
             p.H = h->H;
             p.I = h->I;
             p.k = h->k;
-            if ((rc = cuda_rc(moe::launch_sym8(p, h->num_sms, run_gu, run_dn, s))) != MOE_OK)
+            if ((rc = cuda_rc(moe::launch_sym8(p, h->num_sms, run_gu, run_dn, s, h->use_pdl))) !=
+                MOE_OK)
                 return rc;
         }
         h->kept = keep;

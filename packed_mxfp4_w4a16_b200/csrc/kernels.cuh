@@ -306,6 +306,6 @@ struct Sym8Params {
 bool sym8_supported(int H, int I, int k);
 int sym8_max_chunk(int H, int I, int k);
 cudaError_t launch_sym8(const Sym8Params &p, int num_sms, bool run_gu, bool run_dn,
-                        cudaStream_t s);
+                        cudaStream_t s, bool pdl);
 
 }  // namespace moe

@@ -31,7 +31,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "kernels.cuh"
+#include "gemv.cuh"  // kernels.cuh, launch_ex
 
 namespace moe {
 
@@ -40,6 +40,7 @@ namespace {
 constexpr int kS8Threads = 256;
 constexpr int kS8Warps = kS8Threads / 32;
 constexpr int kS8CtasPerSm = 4;  // warps in flight per SM: 32 (streaming GEMV)
+constexpr int kS8DownSlots = 4;  // slots whose down rows one warp streams together
 
 // Four int8 weights of one 32-bit word (byte 0 = lowest K index) -> FP32,
 // exactly: byte i, biased to q + 128, becomes the low byte of the float with
@@ -90,11 +91,32 @@ __device__ __forceinline__ float s8_row_dot(const uint8_t *rc, const uint8_t *rs
     return warp_sum(acc);
 }
 
+// Two rows' dot products against the same vector, their loads interleaved
+// (twice the bytes in flight per lane); per row the chunks, their order and
+// the sums are those of s8_row_dot (same bits).
+__device__ __forceinline__ void s8_row_dot2(const uint8_t *ra, const uint8_t *sa, const uint8_t *rb,
+                                            const uint8_t *sb, const uint4 *xs, int K, int lane,
+                                            float &da, float &db) {
+    const int nc = K >> 4;
+    float aa = 0.f, ab = 0.f;
+#pragma unroll 4
+    for (int c = lane; c < nc; c += 32) {
+        const uint4 wa = ld_stream16(ra + (size_t)c * 16);
+        const uint4 wb = ld_stream16(rb + (size_t)c * 16);
+        aa = fmaf(s8_chunk_dot(wa, xs[2 * c], xs[2 * c + 1]), s8_scale(sa, c), aa);
+        ab = fmaf(s8_chunk_dot(wb, xs[2 * c], xs[2 * c + 1]), s8_scale(sb, c), ab);
+    }
+    da = warp_sum(aa);
+    db = warp_sum(ab);
+}
+
 // gate/up + SwiGLU.  Item (q, i): pair q = t k + j (token t, slot j), row i of
 // the expert's gate and up matrices; h[q][i] = BF16(BF16(SiLU(BF16(g))) BF16(u)).
 __global__ void __launch_bounds__(kS8Threads) sym8_gateup_kernel(const Sym8Params p) {
     extern __shared__ __align__(16) uint4 s_x[];  // [T][H/8]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_wait();  // x and the routing come from earlier kernels
+    pdl_launch_dependents();
     const int H = p.H, I = p.I, k = p.k, E = p.E;
     const int np8 = H >> 3;
     const uint4 *x = reinterpret_cast<const uint4 *>(p.x);
@@ -113,8 +135,9 @@ __global__ void __launch_bounds__(kS8Threads) sym8_gateup_kernel(const Sym8Param
         if (!bad) {
             const ExpertPtrs &ep = p.table[e];
             const uint4 *xs = s_x + (size_t)t * np8;
-            ag = s8_row_dot(ep.codes[0] + (size_t)i * H, ep.scales[0] + (size_t)i * rs, xs, H, lane);
-            au = s8_row_dot(ep.codes[1] + (size_t)i * H, ep.scales[1] + (size_t)i * rs, xs, H, lane);
+            s8_row_dot2(ep.codes[0] + (size_t)i * H, ep.scales[0] + (size_t)i * rs,
+                        ep.codes[1] + (size_t)i * H, ep.scales[1] + (size_t)i * rs, xs, H, lane, ag,
+                        au);
         }
         if (lane == 0) {
             uint16_t hv = 0;
@@ -132,10 +155,14 @@ __global__ void __launch_bounds__(kS8Threads) sym8_gateup_kernel(const Sym8Param
 
 // down + combine + residual.  Item (t, n): output row n of token t; the
 // slots' o_j = BF16(down row n . h_j) in slot order, combined sequentially in
-// BF16, then the residual.
+// BF16, then the residual.  The slots' rows are streamed together (every
+// slot's chunk c loaded before any of them is used); per row the chunks, their
+// order and the sums are those of s8_row_dot (same bits).
 __global__ void __launch_bounds__(kS8Threads) sym8_down_kernel(const Sym8Params p) {
     extern __shared__ __align__(16) uint4 s_h[];  // [T][k][I/8]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_wait();  // h comes from the gate/up kernel
+    pdl_launch_dependents();
     const int H = p.H, I = p.I, k = p.k, E = p.E;
     const int np8 = I >> 3;
     const uint4 *hg = reinterpret_cast<const uint4 *>(p.h);
@@ -148,22 +175,50 @@ __global__ void __launch_bounds__(kS8Threads) sym8_down_kernel(const Sym8Params 
          it += (long long)gridDim.x * kS8Warps) {
         const int t = (int)(it / H), n = (int)(it - (long long)t * H);
         float y = 0.f;
+        // slots in groups of kS8DownSlots, each group's rows streamed together
         #pragma unroll 1
-        for (int j = 0; j < k; ++j) {
-            const int q = t * k + j;
-            const int e = p.ids[q];
-            const bool bad = e < 0 || e >= E;
-            float o = 0.f;
-            if (!bad) {
-                const ExpertPtrs &ep = p.table[e];
-                o = round_bf16(s8_row_dot(ep.codes[2] + (size_t)n * I, ep.scales[2] + (size_t)n * rs,
-                                          s_h + (size_t)q * np8, I, lane));
-            } else if (lane == 0 && n == 0) {
-                atomicOr(p.status, kBadExpertId);
+        for (int j0 = 0; j0 < k; j0 += kS8DownSlots) {
+            const uint8_t *rc[kS8DownSlots];
+            const uint8_t *rsc[kS8DownSlots];
+            bool ok[kS8DownSlots];
+#pragma unroll
+            for (int d = 0; d < kS8DownSlots; ++d) {
+                const int j = j0 + d;
+                const int e = j < k ? p.ids[t * k + j] : -1;
+                ok[d] = e >= 0 && e < E;
+                if (j < k && !ok[d] && lane == 0 && n == 0) atomicOr(p.status, kBadExpertId);
+                rc[d] = ok[d] ? p.table[e].codes[2] + (size_t)n * I : nullptr;
+                rsc[d] = ok[d] ? p.table[e].scales[2] + (size_t)n * rs : nullptr;
             }
-            if (lane == 0 && p.o_keep) p.o_keep[(size_t)q * H + n] = f32_to_bf16(o);
-            const float wb = round_bf16(p.w[q]);
-            y = round_bf16(y + round_bf16(o * wb));
+            float acc[kS8DownSlots];
+#pragma unroll
+            for (int d = 0; d < kS8DownSlots; ++d) acc[d] = 0.f;
+            const int nc = I >> 4;
+            #pragma unroll 1
+            for (int c = lane; c < nc; c += 32) {
+                uint4 wq[kS8DownSlots];
+#pragma unroll
+                for (int d = 0; d < kS8DownSlots; ++d)
+                    if (ok[d]) wq[d] = ld_stream16(rc[d] + (size_t)c * 16);
+#pragma unroll
+                for (int d = 0; d < kS8DownSlots; ++d)
+                    if (ok[d]) {
+                        const uint4 *hs = s_h + (size_t)(t * k + j0 + d) * np8;
+                        acc[d] = fmaf(s8_chunk_dot(wq[d], hs[2 * c], hs[2 * c + 1]),
+                                      s8_scale(rsc[d], c), acc[d]);
+                    }
+            }
+#pragma unroll
+            for (int d = 0; d < kS8DownSlots; ++d) {
+                const int j = j0 + d;
+                if (j >= k) break;
+                const int q = t * k + j;
+                const float a = warp_sum(acc[d]);
+                const float o = ok[d] ? round_bf16(a) : 0.f;
+                if (lane == 0 && p.o_keep) p.o_keep[(size_t)q * H + n] = f32_to_bf16(o);
+                const float wb = round_bf16(p.w[q]);
+                y = round_bf16(y + round_bf16(o * wb));
+            }
         }
         if (lane == 0) {
             if (p.residual) y = round_bf16(bf16_to_f32(p.residual[it]) + y);
@@ -191,7 +246,7 @@ int sym8_max_chunk(int H, int I, int k) {
 }
 
 cudaError_t launch_sym8(const Sym8Params &p, int num_sms, bool run_gu, bool run_dn,
-                        cudaStream_t s) {
+                        cudaStream_t s, bool pdl) {
     if (p.T < 1 || p.T > kS8MaxT || !sym8_supported(p.H, p.I, p.k)) return cudaErrorInvalidValue;
     const size_t sg = s8_gateup_smem(p.T, p.H), sd = s8_down_smem(p.T, p.k, p.I);
     if (sg > kS8SmemMax || sd > kS8SmemMax) return cudaErrorInvalidValue;
@@ -205,14 +260,12 @@ cudaError_t launch_sym8(const Sym8Params &p, int num_sms, bool run_gu, bool run_
     });
     if (e != cudaSuccess) return e;
     const int grid = num_sms * kS8CtasPerSm;
-    if (run_gu) {
-        sym8_gateup_kernel<<<grid, kS8Threads, sg, s>>>(p);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
-    if (run_dn) {
-        sym8_down_kernel<<<grid, kS8Threads, sd, s>>>(p);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
+    if (run_gu && (e = launch_ex(sym8_gateup_kernel, dim3(grid), dim3(kS8Threads), sg, s, pdl, p)) !=
+                      cudaSuccess)
+        return e;
+    if (run_dn && (e = launch_ex(sym8_down_kernel, dim3(grid), dim3(kS8Threads), sd, s, pdl, p)) !=
+                      cudaSuccess)
+        return e;
     return cudaSuccess;
 }
 
