@@ -23,11 +23,16 @@
 // sums give o = BF16(sum), and the combine is the sequential BF16 one
 // (wb = BF16(w), y = BF16(y + BF16(o wb)), then y = BF16(r + y)).
 //
-// Two launches per chunk of up to kS8MaxT tokens: gate/up + SwiGLU (one warp
-// per (pair, row) item, the tokens' x staged in shared memory) writing h to
-// the workspace, then down + combine + residual (one warp per (token, output
-// row), the chunk's h staged in shared memory).  An expert id outside [0, E)
-// gives that slot h = 0 and o = 0 and sets the status word's bad-id bit.
+// Two launches per chunk of up to kS8MaxT tokens, in the layer's programmatic
+// launch chain: gate/up + SwiGLU (a warp takes kS8GuItems consecutive
+// (pair, row) items per step and streams their gate and up rows together,
+// the tokens' x staged in shared memory) writing h to the workspace, then
+// down + combine + residual (one warp per (token, output row), the down rows
+// of up to kS8DownSlots slots streamed together, the chunk's h staged in
+// shared memory).  Lane l takes the 16-byte chunks l, l + 32, ... of a row:
+// per row the sums and their order do not depend on how many rows stream
+// together.  An expert id outside [0, E) gives that slot h = 0 and o = 0 and
+// sets the status word's bad-id bit.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -41,6 +46,10 @@ constexpr int kS8Threads = 256;
 constexpr int kS8Warps = kS8Threads / 32;
 constexpr int kS8CtasPerSm = 4;  // warps in flight per SM: 32 (streaming GEMV)
 constexpr int kS8DownSlots = 4;  // slots whose down rows one warp streams together
+#ifndef MOE_S8_GU_ITEMS
+#define MOE_S8_GU_ITEMS 2
+#endif
+constexpr int kS8GuItems = MOE_S8_GU_ITEMS;  // gate/up items one warp streams together
 
 // Four int8 weights of one 32-bit word (byte 0 = lowest K index) -> FP32,
 // exactly: byte i, biased to q + 128, becomes the low byte of the float with
@@ -76,40 +85,6 @@ __device__ __forceinline__ float s8_scale(const uint8_t *row_scales, int c) {
     return f16_bits_to_f32(__ldg(s + (c >> 1)));
 }
 
-// Dot product of one sym8 row of K weights (codes rc, scales rs) with the
-// BF16 vector xs (16-byte pieces in shared memory), by one warp; every lane
-// returns the same sum.  Lane l takes the chunks l, l + 32, ...
-__device__ __forceinline__ float s8_row_dot(const uint8_t *rc, const uint8_t *rs, const uint4 *xs,
-                                            int K, int lane) {
-    const int nc = K >> 4;
-    float acc = 0.f;
-#pragma unroll 4
-    for (int c = lane; c < nc; c += 32) {
-        const uint4 wq = ld_stream16(rc + (size_t)c * 16);
-        acc = fmaf(s8_chunk_dot(wq, xs[2 * c], xs[2 * c + 1]), s8_scale(rs, c), acc);
-    }
-    return warp_sum(acc);
-}
-
-// Two rows' dot products against the same vector, their loads interleaved
-// (twice the bytes in flight per lane); per row the chunks, their order and
-// the sums are those of s8_row_dot (same bits).
-__device__ __forceinline__ void s8_row_dot2(const uint8_t *ra, const uint8_t *sa, const uint8_t *rb,
-                                            const uint8_t *sb, const uint4 *xs, int K, int lane,
-                                            float &da, float &db) {
-    const int nc = K >> 4;
-    float aa = 0.f, ab = 0.f;
-#pragma unroll 4
-    for (int c = lane; c < nc; c += 32) {
-        const uint4 wa = ld_stream16(ra + (size_t)c * 16);
-        const uint4 wb = ld_stream16(rb + (size_t)c * 16);
-        aa = fmaf(s8_chunk_dot(wa, xs[2 * c], xs[2 * c + 1]), s8_scale(sa, c), aa);
-        ab = fmaf(s8_chunk_dot(wb, xs[2 * c], xs[2 * c + 1]), s8_scale(sb, c), ab);
-    }
-    da = warp_sum(aa);
-    db = warp_sum(ab);
-}
-
 // gate/up + SwiGLU.  Item (q, i): pair q = t k + j (token t, slot j), row i of
 // the expert's gate and up matrices; h[q][i] = BF16(BF16(SiLU(BF16(g))) BF16(u)).
 __global__ void __launch_bounds__(kS8Threads) sym8_gateup_kernel(const Sym8Params p) {
@@ -124,31 +99,63 @@ __global__ void __launch_bounds__(kS8Threads) sym8_gateup_kernel(const Sym8Param
     __syncthreads();
     const size_t rs = (size_t)H >> 4;  // scale bytes of a row
     const long long items = (long long)p.T * k * I;
+    // kS8GuItems consecutive items per warp per step: their gate and up rows
+    // stream together (per row the same chunks, order and sums)
     #pragma unroll 1
-    for (long long it = (long long)blockIdx.x * kS8Warps + warp; it < items;
-         it += (long long)gridDim.x * kS8Warps) {
-        const int q = (int)(it / I), i = (int)(it - (long long)q * I);
-        const int t = q / k;
-        const int e = p.ids[q];
-        const bool bad = e < 0 || e >= E;
-        float ag = 0.f, au = 0.f;
-        if (!bad) {
-            const ExpertPtrs &ep = p.table[e];
-            const uint4 *xs = s_x + (size_t)t * np8;
-            s8_row_dot2(ep.codes[0] + (size_t)i * H, ep.scales[0] + (size_t)i * rs,
-                        ep.codes[1] + (size_t)i * H, ep.scales[1] + (size_t)i * rs, xs, H, lane, ag,
-                        au);
+    for (long long it0 = ((long long)blockIdx.x * kS8Warps + warp) * kS8GuItems; it0 < items;
+         it0 += (long long)gridDim.x * kS8Warps * kS8GuItems) {
+        const uint8_t *rg[kS8GuItems], *sg[kS8GuItems], *ru[kS8GuItems], *su[kS8GuItems];
+        const uint4 *xs[kS8GuItems];
+        bool ok[kS8GuItems];
+#pragma unroll
+        for (int d = 0; d < kS8GuItems; ++d) {
+            const long long it = it0 + d;
+            const int q = it < items ? (int)(it / I) : 0, i = it < items ? (int)(it - (long long)q * I) : 0;
+            const int e = it < items ? p.ids[q] : -1;
+            ok[d] = e >= 0 && e < E;
+            if (it < items && !ok[d] && i == 0 && lane == 0) atomicOr(p.status, kBadExpertId);
+            const ExpertPtrs *ep = ok[d] ? p.table + e : nullptr;
+            rg[d] = ok[d] ? ep->codes[0] + (size_t)i * H : nullptr;
+            sg[d] = ok[d] ? ep->scales[0] + (size_t)i * rs : nullptr;
+            ru[d] = ok[d] ? ep->codes[1] + (size_t)i * H : nullptr;
+            su[d] = ok[d] ? ep->scales[1] + (size_t)i * rs : nullptr;
+            xs[d] = s_x + (size_t)(q / k) * np8;
         }
-        if (lane == 0) {
-            uint16_t hv = 0;
-            if (!bad) {
-                const float g = round_bf16(ag), u = round_bf16(au);
-                const float sl = round_bf16(g / (1.0f + expf(-g)));
-                hv = f32_to_bf16(sl * u);
-            } else if (i == 0) {
-                atomicOr(p.status, kBadExpertId);
+        float ag[kS8GuItems], au[kS8GuItems];
+#pragma unroll
+        for (int d = 0; d < kS8GuItems; ++d) ag[d] = au[d] = 0.f;
+        const int nc = H >> 4;
+        #pragma unroll 1
+        for (int c = lane; c < nc; c += 32) {
+            uint4 wg[kS8GuItems], wu[kS8GuItems];
+#pragma unroll
+            for (int d = 0; d < kS8GuItems; ++d)
+                if (ok[d]) {
+                    wg[d] = ld_stream16(rg[d] + (size_t)c * 16);
+                    wu[d] = ld_stream16(ru[d] + (size_t)c * 16);
+                }
+#pragma unroll
+            for (int d = 0; d < kS8GuItems; ++d)
+                if (ok[d]) {
+                    ag[d] = fmaf(s8_chunk_dot(wg[d], xs[d][2 * c], xs[d][2 * c + 1]), s8_scale(sg[d], c),
+                                 ag[d]);
+                    au[d] = fmaf(s8_chunk_dot(wu[d], xs[d][2 * c], xs[d][2 * c + 1]), s8_scale(su[d], c),
+                                 au[d]);
+                }
+        }
+#pragma unroll
+        for (int d = 0; d < kS8GuItems; ++d) {
+            const long long it = it0 + d;
+            const float g0 = warp_sum(ag[d]), u0 = warp_sum(au[d]);
+            if (lane == 0 && it < items) {
+                uint16_t hv = 0;
+                if (ok[d]) {
+                    const float g = round_bf16(g0), u = round_bf16(u0);
+                    const float sl = round_bf16(g / (1.0f + expf(-g)));
+                    hv = f32_to_bf16(sl * u);
+                }
+                p.h[it] = hv;
             }
-            p.h[it] = hv;
         }
     }
 }
@@ -157,7 +164,7 @@ __global__ void __launch_bounds__(kS8Threads) sym8_gateup_kernel(const Sym8Param
 // slots' o_j = BF16(down row n . h_j) in slot order, combined sequentially in
 // BF16, then the residual.  The slots' rows are streamed together (every
 // slot's chunk c loaded before any of them is used); per row the chunks, their
-// order and the sums are those of s8_row_dot (same bits).
+// order and the sums are those of the one-row form (same bits).
 __global__ void __launch_bounds__(kS8Threads) sym8_down_kernel(const Sym8Params p) {
     extern __shared__ __align__(16) uint4 s_h[];  // [T][k][I/8]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
