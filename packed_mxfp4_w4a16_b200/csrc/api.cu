@@ -594,6 +594,49 @@ int moe_layer_ex(moe_handle_t h, const uint16_t *x, int T, const uint16_t *route
     const WsLayout L = ws_layout(h, h->max_tokens);
     float *lg = reinterpret_cast<float *>(h->ws + L.logits);
 
+    if (h->s8 && !(route_flags & MOE_ROUTE_SIGMOID) && T <= moe::sym8_max_chunk(h->H, h->I, h->k)) {
+        // sym8 experts, one chunk of tokens, softmax scoring: the router
+        // kernel writes the logits, and each sym8 kernel takes the top-k of
+        // them itself (gate/up CTA 0 writes the routing out): three launches
+        if (!topk_ids || !topk_w) return MOE_ERR_ARG;
+        moe::RouteParams rp = {};
+        rp.x = x;
+        rp.wr = router_w;
+        rp.bias = router_bias;
+        rp.x_norm = x_norm;
+        rp.logits_ws = lg;
+        rp.logits_out = logits;
+        rp.T = T;
+        rp.E = h->E;
+        rp.H = h->H;
+        rp.k = h->k;
+        rp.rmsnorm = norm ? 1 : 0;
+        rp.eps = 1e-6f;
+        rp.x16 = reinterpret_cast<uint32_t *>(h->ws + L.x16);
+        rp.x16_exp = reinterpret_cast<int *>(h->ws + L.x16_exp);
+        if ((rc = cuda_rc(moe::launch_route_logits(rp, s, h->use_pdl))) != MOE_OK) return rc;
+        const bool keep = fwd_flags & MOE_FWD_KEEP_INTERMEDIATES;
+        moe::Sym8Params p = {};
+        p.table = h->d_table;
+        p.x = norm ? x_norm : x;
+        p.logits = lg;
+        p.ids_out = topk_ids;
+        p.w_out = topk_w;
+        p.residual = residual;
+        p.y = y;
+        p.h = reinterpret_cast<uint16_t *>(h->ws + L.h);
+        p.o_keep = keep ? reinterpret_cast<uint16_t *>(h->ws + L.o) : nullptr;
+        p.status = h->d_status;
+        p.T = T;
+        p.E = h->E;
+        p.H = h->H;
+        p.I = h->I;
+        p.k = h->k;
+        if ((rc = cuda_rc(moe::launch_sym8(p, h->num_sms, true, true, s, h->use_pdl))) != MOE_OK)
+            return rc;
+        h->kept = keep;
+        return MOE_OK;
+    }
     if (T > moe::kDecodeMaxT || (route_flags & MOE_ROUTE_SIGMOID) || h->s8) {
         // many tokens, sigmoid scoring (the fused launch structures select
         // by softmax scoring only) or sym8 experts: explicit routing, then

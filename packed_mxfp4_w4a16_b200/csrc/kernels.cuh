@@ -294,8 +294,11 @@ constexpr size_t kS8SmemMax = 48 * 1024;  // staged x / h per CTA
 struct Sym8Params {
     const ExpertPtrs *table;     // [E]: codes [3][rows][K] int8, scales [3][rows][K/32] binary16
     const uint16_t *x;           // [T][H] BF16
-    const int32_t *ids;          // [T][k]
+    const int32_t *ids;          // [T][k] given routing, or null: route from logits
     const float *w;              // [T][k]
+    const float *logits;         // [T][E] router logits when ids is null (softmax top-k)
+    int32_t *ids_out;            // [T][k] or null: written by gate/up CTA 0 when routing
+    float *w_out;                // [T][k] or null
     const uint16_t *residual;    // [T][H] or null
     uint16_t *y;                 // [T][H]
     uint16_t *h;                 // [T][k][I] BF16 SwiGLU outputs (workspace)

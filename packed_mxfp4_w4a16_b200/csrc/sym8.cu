@@ -79,6 +79,41 @@ __device__ __forceinline__ float s8_chunk_dot(const uint4 &wq, const uint4 &x0, 
     return acc;
 }
 
+// The routing of the launch's tokens into shared memory: the given ids and
+// weights, or (logits given) the softmax top-k of each token's logits by
+// warp 0, the warp_topk that the standalone top-k kernel runs (same ids and
+// weights); gate/up CTA 0 also writes them out when asked.  All threads; ends
+// with a CTA barrier.
+__device__ __forceinline__ void s8_routing(const Sym8Params &p, int *s_ids, float *s_w,
+                                           bool write_out) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int k = p.k;
+    if (p.logits) {
+        if (warp == 0) {
+            #pragma unroll 1
+            for (int t = 0; t < p.T; ++t) {
+                int id;
+                float w;
+                warp_topk_any(p.logits + (size_t)t * p.E, p.E, k, lane, id, w);
+                if (lane < k) {
+                    s_ids[t * k + lane] = id;
+                    s_w[t * k + lane] = w;
+                    if (write_out && p.ids_out) {
+                        p.ids_out[t * k + lane] = id;
+                        p.w_out[t * k + lane] = w;
+                    }
+                }
+            }
+        }
+    } else {
+        for (int i = tid; i < p.T * k; i += kS8Threads) {
+            s_ids[i] = p.ids[i];
+            s_w[i] = p.w[i];
+        }
+    }
+    __syncthreads();
+}
+
 // binary16 block scale of the 16-byte chunk c of a row (two chunks per block).
 __device__ __forceinline__ float s8_scale(const uint8_t *row_scales, int c) {
     const uint16_t *s = reinterpret_cast<const uint16_t *>(row_scales);
@@ -90,13 +125,15 @@ __device__ __forceinline__ float s8_scale(const uint8_t *row_scales, int c) {
 __global__ void __launch_bounds__(kS8Threads) sym8_gateup_kernel(const Sym8Params p) {
     extern __shared__ __align__(16) uint4 s_x[];  // [T][H/8]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ int s_ids[kS8MaxT * kMaxTopK];
+    __shared__ float s_w[kS8MaxT * kMaxTopK];
     pdl_wait();  // x and the routing come from earlier kernels
     pdl_launch_dependents();
     const int H = p.H, I = p.I, k = p.k, E = p.E;
     const int np8 = H >> 3;
     const uint4 *x = reinterpret_cast<const uint4 *>(p.x);
     for (int i = tid; i < p.T * np8; i += kS8Threads) s_x[i] = x[i];
-    __syncthreads();
+    s8_routing(p, s_ids, s_w, blockIdx.x == 0);
     const size_t rs = (size_t)H >> 4;  // scale bytes of a row
     const long long items = (long long)p.T * k * I;
     // kS8GuItems consecutive items per warp per step: their gate and up rows
@@ -111,7 +148,7 @@ __global__ void __launch_bounds__(kS8Threads) sym8_gateup_kernel(const Sym8Param
         for (int d = 0; d < kS8GuItems; ++d) {
             const long long it = it0 + d;
             const int q = it < items ? (int)(it / I) : 0, i = it < items ? (int)(it - (long long)q * I) : 0;
-            const int e = it < items ? p.ids[q] : -1;
+            const int e = it < items ? s_ids[q] : -1;
             ok[d] = e >= 0 && e < E;
             if (it < items && !ok[d] && i == 0 && lane == 0) atomicOr(p.status, kBadExpertId);
             const ExpertPtrs *ep = ok[d] ? p.table + e : nullptr;
@@ -168,13 +205,15 @@ __global__ void __launch_bounds__(kS8Threads) sym8_gateup_kernel(const Sym8Param
 __global__ void __launch_bounds__(kS8Threads) sym8_down_kernel(const Sym8Params p) {
     extern __shared__ __align__(16) uint4 s_h[];  // [T][k][I/8]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ int s_ids[kS8MaxT * kMaxTopK];
+    __shared__ float s_w[kS8MaxT * kMaxTopK];
     pdl_wait();  // h comes from the gate/up kernel
     pdl_launch_dependents();
     const int H = p.H, I = p.I, k = p.k, E = p.E;
     const int np8 = I >> 3;
     const uint4 *hg = reinterpret_cast<const uint4 *>(p.h);
     for (int i = tid; i < p.T * k * np8; i += kS8Threads) s_h[i] = hg[i];
-    __syncthreads();
+    s8_routing(p, s_ids, s_w, false);
     const size_t rs = (size_t)I >> 4;
     const long long items = (long long)p.T * H;
     #pragma unroll 1
@@ -191,7 +230,7 @@ __global__ void __launch_bounds__(kS8Threads) sym8_down_kernel(const Sym8Params 
 #pragma unroll
             for (int d = 0; d < kS8DownSlots; ++d) {
                 const int j = j0 + d;
-                const int e = j < k ? p.ids[t * k + j] : -1;
+                const int e = j < k ? s_ids[t * k + j] : -1;
                 ok[d] = e >= 0 && e < E;
                 if (j < k && !ok[d] && lane == 0 && n == 0) atomicOr(p.status, kBadExpertId);
                 rc[d] = ok[d] ? p.table[e].codes[2] + (size_t)n * I : nullptr;
@@ -223,7 +262,7 @@ __global__ void __launch_bounds__(kS8Threads) sym8_down_kernel(const Sym8Params 
                 const float a = warp_sum(acc[d]);
                 const float o = ok[d] ? round_bf16(a) : 0.f;
                 if (lane == 0 && p.o_keep) p.o_keep[(size_t)q * H + n] = f32_to_bf16(o);
-                const float wb = round_bf16(p.w[q]);
+                const float wb = round_bf16(s_w[q]);
                 y = round_bf16(y + round_bf16(o * wb));
             }
         }
