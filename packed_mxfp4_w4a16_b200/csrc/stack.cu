@@ -85,7 +85,7 @@ __device__ __forceinline__ unsigned stk_tag(unsigned base, int l) {
 
 constexpr int kAbortEvery = 256;   // polling rounds between two looks at the abort word
 #ifndef MOE_STACK_POLL_SLEEP
-#define MOE_STACK_POLL_SLEEP 32
+#define MOE_STACK_POLL_SLEEP 16
 #endif
 constexpr int kPollSleepNs = MOE_STACK_POLL_SLEEP;  // back-off between polling rounds (ns)
 constexpr int kXThreads = 256;     // threads that gather the layer input (one piece each at H = 2048)

@@ -107,14 +107,15 @@ def test_stack_kernel_matches_oracle_and_layer_path(shape, n_layers, bias):
     st.close()
 
 
-@pytest.mark.parametrize("shape,n_layers", [(synth.L24B, 4), (synth.TINY, 5)])
-def test_stack_kernel_nvfp4_matches_oracle_and_layer_path(shape, n_layers):
+@pytest.mark.parametrize("shape,n_layers,bias", [(synth.L24B, 4, False), (synth.TINY, 5, False),
+                                                 (synth.L8B, 3, True)])
+def test_stack_kernel_nvfp4_matches_oracle_and_layer_path(shape, n_layers, bias):
     """NVFP4 experts (an E4M3 scale per 16 elements, FP32 multipliers per
     expert) in the one-launch stack: bit-for-bit the same step run one layer
     at a time (route + NVFP4 gate/up + down kernels), every layer within the
     oracle's tolerance (NVFP4 expert FFN fed the GPU's routed vector and
     routing), and a graph replay gives the eager bits."""
-    layers = [synth.make_layer_nvfp4(shape, seed=63, layer=l) for l in range(n_layers)]
+    layers = [synth.make_layer_nvfp4(shape, seed=63, layer=l, bias=bias) for l in range(n_layers)]
     w = [dev_layer(L) + (torch.from_numpy(L.gscales).cuda(),) for L in layers]
     st = moe.MoEStack(w, shape.E, shape.H, shape.I, shape.top_k)
     assert st.stack is not None
