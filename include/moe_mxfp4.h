@@ -185,10 +185,16 @@ MOE_API int moe_load_packed_nvfp4(moe_handle_t h, const uint8_t *codes_u8,
  * zero point.  codes 16-byte aligned, scales 2-byte aligned; read in place
  * through the handle's device pointer table, caller-owned.  Requires H and I
  * multiples of 32 with one token's H (gate/up) and k*I (down) BF16 values
- * within 48 KB.  sym8 layers run the per-(token, slot) GEMVs for every T
- * (in chunks of up to 4 tokens) with FP32 products and sums; no grouped
- * path, no fused launch structures (FORCE_GROUPED / FORCE_MMA /
- * FORCE_TCGEN05 return ARG), no stack kernel.  moe_load_packed,
+ * within 48 KB.  sym8 layers run the per-(token, slot) GEMVs (FP32 products
+ * and sums) up to 4 tokens, and beyond that (or with FORCE_GROUPED /
+ * FORCE_MMA) the grouped mma.sync products: int8 rows converted to FP16
+ * exactly, the binary16 scale applied per 32-element group in FP32.  The
+ * grouped products need the scales 4-byte aligned and H, I multiples of 128
+ * within the tiles' shared memory (H, I <= 4096 and both products' tiles
+ * within 220 KB); otherwise every T runs the GEMVs in chunks of up to 4
+ * tokens (FORCE_GROUPED / FORCE_MMA then return ARG).  No tcgen05 products
+ * (FORCE_TCGEN05 returns ARG), no fused launch structures, no stack kernel.
+ * moe_load_packed,
  * moe_load_packed_nvfp4 and moe_load_expert_table switch the handle to their
  * format.  Errors: ARG (null pointer, unsupported shape), NOT_DEVICE, CUDA. */
 MOE_API int moe_load_packed_sym8(moe_handle_t h, const int8_t *codes_s8,
@@ -243,7 +249,7 @@ MOE_API int moe_route_ex(moe_handle_t h, const uint16_t *x, int T,
  * brought in by TMA tensor loads) when a chunk's groups average at least 40
  * (token, slot) pairs per expert (T k >= 40 E) and the weights allow it
  * (contiguous MXFP4 from moe_load_packed, H and I multiples of 128; NVFP4
- * weights always take the mma.sync tiles, sym8 weights their own GEMVs);
+ * and sym8 weights always take the mma.sync tiles);
  * MOE_FWD_FORCE_TCGEN05 / MOE_FWD_FORCE_MMA pin the choice.  Errors: ARG,
  * NOT_LOADED, NOT_DEVICE, ALIGN, WORKSPACE, CUDA. */
 MOE_API int moe_forward(moe_handle_t h, const uint16_t *x, int T,

@@ -37,6 +37,7 @@ struct moe_ctx {
     int nv = 0;                           // NVFP4 weights (moe_load_packed_nvfp4)
     const float *gscale = nullptr;        // NVFP4: [E][2] multipliers (gate/up, down)
     int s8 = 0;                           // sym8 weights (moe_load_packed_sym8)
+    bool s8_scales4 = false;              // sym8 scales 4-byte aligned (grouped products)
     moe::TcMapCache tc_maps;              // tensor maps of the bound codes (tcgen05 products)
 };
 
@@ -264,6 +265,7 @@ int moe_load_packed_sym8(moe_handle_t h, const int8_t *codes_s8, const uint16_t 
         h->codes_base = h->scales_base = nullptr;
         h->nv = 0;
         h->s8 = 1;
+        h->s8_scales4 = (reinterpret_cast<uintptr_t>(sb) & 3) == 0;
         h->gscale = nullptr;
     }
     return rc;
@@ -402,9 +404,19 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
     uint16_t *hbuf = reinterpret_cast<uint16_t *>(h->ws + L.h);
     uint16_t *obuf = reinterpret_cast<uint16_t *>(h->ws + L.o);
 
-    if (h->s8) {
-        // sym8 experts: the per-(token, slot) GEMVs of sym8.cu at every T
-        if (flags & MOE_FWD_FORCE_GROUPED) return MOE_ERR_ARG;
+    // (token, expert)-sorted grouped path on the tensor cores: batches beyond
+    // the decode sizes, or when asked (the phase flags time the decode path);
+    // sym8 weights need their scales 4-byte aligned there
+    const bool phase = flags & (MOE_FWD_PHASE_GATEUP | MOE_FWD_PHASE_DOWN);
+    const bool grouped = !phase && !(flags & MOE_FWD_FORCE_DECODE) &&
+                         (T > moe::kDecodeMaxT || (flags & MOE_FWD_FORCE_GROUPED)) &&
+                         (!h->s8 || h->s8_scales4) &&
+                         moe::grouped_supported(h->E, h->H, h->I, h->nv, h->s8);
+    if ((flags & MOE_FWD_FORCE_GROUPED) && !grouped) return MOE_ERR_ARG;
+
+    if (h->s8 && !grouped) {
+        // sym8 experts off the grouped path: the per-(token, slot) GEMVs of
+        // sym8.cu
         const int chunk = moe::sym8_max_chunk(h->H, h->I, h->k);
         for (int t0 = 0; t0 < T; t0 += chunk) {
             const int Tc = (T - t0 < chunk) ? T - t0 : chunk;
@@ -430,15 +442,8 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
         h->kept = keep;
         return MOE_OK;
     }
-    if (!moe::decode_shape_supported(h->H, h->I)) return MOE_ERR_ARG;
+    if (!h->s8 && !moe::decode_shape_supported(h->H, h->I)) return MOE_ERR_ARG;
 
-    // (token, expert)-sorted grouped path on the tensor cores: batches beyond
-    // the decode sizes, or when asked (the phase flags time the decode path)
-    const bool phase = flags & (MOE_FWD_PHASE_GATEUP | MOE_FWD_PHASE_DOWN);
-    const bool grouped = !phase && !(flags & MOE_FWD_FORCE_DECODE) &&
-                         (T > moe::kDecodeMaxT || (flags & MOE_FWD_FORCE_GROUPED)) &&
-                         moe::grouped_supported(h->E, h->H, h->I, h->nv);
-    if ((flags & MOE_FWD_FORCE_GROUPED) && !grouped) return MOE_ERR_ARG;
     if (grouped) {
         for (int t0 = 0; t0 < T; t0 += moe::kGroupedMaxT) {
             const int Tc = (T - t0 < moe::kGroupedMaxT) ? T - t0 : moe::kGroupedMaxT;
@@ -449,6 +454,7 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
             gp.codes_stride = (size_t)h->I * h->H / 2;
             gp.scales_stride = (size_t)h->I * h->H / (h->nv ? 16 : 32);
             gp.nv = h->nv;
+            gp.s8 = h->s8;
             gp.gscale = h->gscale;
             gp.tc_maps = &h->tc_maps;
             gp.x = x + (size_t)t0 * h->H;
@@ -473,7 +479,7 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
             gp.I = h->I;
             // tcgen05 when the groups are large enough to amortise a CTA's
             // dequantised tiles over its token passes
-            const bool tc_ok = !h->nv && h->codes_base &&
+            const bool tc_ok = !h->nv && !h->s8 && h->codes_base &&
                                moe::grouped_tc_supported(h->H, h->I, Tc * h->k);
             gp.tcgen05 = (flags & MOE_FWD_FORCE_TCGEN05) ||
                          (!(flags & MOE_FWD_FORCE_MMA) && tc_ok &&

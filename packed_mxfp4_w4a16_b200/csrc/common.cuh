@@ -256,6 +256,40 @@ __device__ __forceinline__ void mma_group_nvfp4(float (&acc)[4], uint32_t w_lo, 
     acc[3] = fmaf(d1[3], h1, fmaf(d0[3], h0, acc[3]));
 }
 
+// sym8 form (int8 weights, one binary16 scale per 32 K elements): thread
+// (g, q) supplies weights 8q..8q+7 of rows g and g + 8 (8 bytes each, w_lo /
+// w_hi) and elements 8q..8q+7 of column g (b), in the K order of
+// mma_group_e2m1.  A weight byte q becomes FP16 exactly: its biased value
+// q + 128 is the low mantissa byte of the FP16 1024 + (q + 128), and one
+// subtraction of 1152 leaves q (an integer below 2^11).  The group's partial
+// product (fresh accumulator, exact products) times the row's scale (s_lo /
+// s_hi: binary16 bits, FP32 exactly) is added to acc in FP32.
+__device__ __forceinline__ void s8x8_to_f16x8(uint2 w, uint32_t (&out)[4]) {
+    const uint32_t u0 = w.x ^ 0x80808080u, u1 = w.y ^ 0x80808080u;
+    const uint32_t hi = 0x64646464u;  // high byte of 1024 + b in FP16
+    const uint32_t bias = 0x64806480u;  // 1152 in both halves
+    const uint32_t p[4] = {__byte_perm(u0, hi, 0x5150u), __byte_perm(u0, hi, 0x5352u),
+                           __byte_perm(u1, hi, 0x5150u), __byte_perm(u1, hi, 0x5352u)};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(out[i]) : "r"(p[i]), "r"(bias));
+}
+
+__device__ __forceinline__ void mma_group_s8(float (&acc)[4], uint2 w_lo, uint2 w_hi,
+                                             uint32_t s_lo, uint32_t s_hi, const uint4 &b) {
+    uint32_t fa[2][4];
+    s8x8_to_f16x8(w_lo, fa[0]);
+    s8x8_to_f16x8(w_hi, fa[1]);
+    const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+    float dd[4];
+    mma_f16(dd, fa[0][0], fa[1][0], fa[0][1], fa[1][1], b.x, b.y, zero);
+    mma_f16(dd, fa[0][2], fa[1][2], fa[0][3], fa[1][3], b.z, b.w, dd);
+    const float sl = f16_bits_to_f32(s_lo), sh = f16_bits_to_f32(s_hi);
+    acc[0] = fmaf(dd[0], sl, acc[0]);
+    acc[1] = fmaf(dd[1], sl, acc[1]);
+    acc[2] = fmaf(dd[2], sh, acc[2]);
+    acc[3] = fmaf(dd[3], sh, acc[3]);
+}
+
 // ------------------------------------------------ FP16 staging of BF16 ----
 // The GEMVs multiply FP16 weights (exact E2M1 values) with activations held
 // in FP16.  A BF16 vector v is staged as v * 2^-c with c chosen from max|v|

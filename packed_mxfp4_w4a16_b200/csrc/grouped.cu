@@ -193,8 +193,9 @@ __device__ __forceinline__ void cp_async_commit_wait() {
 
 // NV: NVFP4 weights (two E4M3 scales per 32-element group, mma_group_nvfp4's
 // K order; the expert's multiplier joins the power-of-two staging scale in the
-// epilogue, an exact product).
-template <int NMAT, int RT, bool NV>
+// epilogue, an exact product).  S8: sym8 weights (one byte per weight, a
+// binary16 scale per 32-element group, mma_group_s8).
+template <int NMAT, int RT, bool NV, bool S8>
 __global__ void __launch_bounds__(128 * RT) grouped_mma_kernel(const GroupedParams p) {
     constexpr int kWarps = 4 * RT;
     extern __shared__ __align__(16) uint8_t sm[];
@@ -209,7 +210,10 @@ __global__ void __launch_bounds__(128 * RT) grouped_mma_kernel(const GroupedPara
     const int M = NMAT == 2 ? p.I : p.H;  // rows of the matrix (a multiple of 16 RT)
     const int row0 = blockIdx.x * (kGpRows * RT);
     const int ng = K >> 5;                // 32-element groups
-    const uint32_t rc = (uint32_t)K >> 1, rs = (uint32_t)K >> (NV ? 4 : 5);
+    // row bytes: codes (K/2 packed, K for sym8), scales (K/32 E8M0, K/16 for
+    // E4M3 per 16 or binary16 per 32)
+    const uint32_t rc = S8 ? (uint32_t)K : (uint32_t)K >> 1,
+                   rs = (uint32_t)K >> (NV || S8 ? 4 : 5);
     const uint32_t rcp = rc + 16, rsp = rs + 16;  // padded row pitches (bank spread)
     const uint32_t bp = (uint32_t)K * 2 + 64;     // padded pitch of a staged B row
     constexpr int R = kGpRows * RT;               // rows held by the CTA
@@ -257,7 +261,7 @@ __global__ void __launch_bounds__(128 * RT) grouped_mma_kernel(const GroupedPara
     const int gq = (ng + 3) >> 2;
     const int gb = min(ng, kq * gq), ge = min(ng, gb + gq);
     // this thread's A words (rows g / g + 8 of its tile) and scales
-    const uint8_t *a_lo = s_codes + (rt * kGpRows + g) * rcp + (NV ? 2 * q : 4 * q);
+    const uint8_t *a_lo = s_codes + (rt * kGpRows + g) * rcp + (NV ? 2 * q : S8 ? 8 * q : 4 * q);
     const uint8_t *s_lo = s_scales + (rt * kGpRows + g) * rsp;
     const uint32_t a_hi = 8 * rcp, sc_hi = 8 * rsp;
     const uint32_t a_m = R * rcp, sc_m = R * rsp;
@@ -296,6 +300,17 @@ __global__ void __launch_bounds__(128 * RT) grouped_mma_kernel(const GroupedPara
                                     *reinterpret_cast<const uint16_t *>(
                                         reinterpret_cast<const uint8_t *>(sb) + sc_hi),
                                     b);
+                }
+            } else if (S8) {
+                const uint4 b = *reinterpret_cast<const uint4 *>(bcol + G * 64);
+#pragma unroll
+                for (int m = 0; m < NMAT; ++m) {
+                    const uint8_t *cb = a_lo + m * a_m + G * 32;
+                    const uint8_t *sb = s_lo + m * sc_m + 2 * G;
+                    mma_group_s8(acc[m], *reinterpret_cast<const uint2 *>(cb),
+                                 *reinterpret_cast<const uint2 *>(cb + a_hi),
+                                 *reinterpret_cast<const uint16_t *>(sb),
+                                 *reinterpret_cast<const uint16_t *>(sb + sc_hi), b);
                 }
             } else {
                 const uint4 b = *reinterpret_cast<const uint4 *>(bcol + G * 64);
@@ -429,43 +444,54 @@ namespace {
 
 constexpr size_t kMmaSmemBudget = 220 * 1024;
 
-size_t mma_smem(int nmat, int K, int nv) {
-    const size_t R = (size_t)kGpRows * kRowTiles;
-    const size_t rcp = (size_t)K / 2 + 16, rsp = (size_t)K / (nv ? 16 : 32) + 16;
-    return (size_t)nmat * R * (rcp + rsp) + (size_t)kRowTiles * 3 * 32 * nmat * 4 * sizeof(float) +
+// row tiles per CTA of the sym8 products (their rows take twice the bytes)
+#ifndef MOE_S8_GROUPED_RT
+#define MOE_S8_GROUPED_RT 1
+#endif
+constexpr int kS8RowTiles = MOE_S8_GROUPED_RT;
+
+size_t mma_smem(int nmat, int K, int nv, int s8) {
+    const int rt = s8 ? kS8RowTiles : kRowTiles;
+    const size_t R = (size_t)kGpRows * rt;
+    const size_t rcp = (size_t)K / (s8 ? 1 : 2) + 16,
+                 rsp = (size_t)K / (nv || s8 ? 16 : 32) + 16;
+    return (size_t)nmat * R * (rcp + rsp) + (size_t)rt * 3 * 32 * nmat * 4 * sizeof(float) +
            (size_t)8 * ((size_t)K * 2 + 64);
 }
 
-template <int NMAT, bool NV>
+template <int NMAT, bool NV, bool S8>
 cudaError_t launch_mma(const GroupedParams &p, cudaStream_t s, bool pdl) {
+    constexpr int RT = S8 ? kS8RowTiles : kRowTiles;
     const int K = NMAT == 2 ? p.H : p.I, M = NMAT == 2 ? p.I : p.H;
-    const size_t smem = mma_smem(NMAT, K, NV ? 1 : 0);
+    const size_t smem = mma_smem(NMAT, K, NV ? 1 : 0, S8 ? 1 : 0);
     if (smem > kMmaSmemBudget) return cudaErrorInvalidValue;
     // the budget, once per device (the attribute belongs to the current
     // device's context)
     static PerDeviceOnce once;
     const cudaError_t attr = per_device_once(once, [] {
-        return cudaFuncSetAttribute(grouped_mma_kernel<NMAT, kRowTiles, NV>,
+        return cudaFuncSetAttribute(grouped_mma_kernel<NMAT, RT, NV, S8>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)kMmaSmemBudget);
     });
     if (attr != cudaSuccess) return attr;
-    return launch_ex(grouped_mma_kernel<NMAT, kRowTiles, NV>, dim3(M / (kGpRows * kRowTiles), p.E),
-                     dim3(128 * kRowTiles), smem, s, pdl, p);
+    return launch_ex(grouped_mma_kernel<NMAT, RT, NV, S8>, dim3(M / (kGpRows * RT), p.E),
+                     dim3(128 * RT), smem, s, pdl, p);
 }
 
 }  // namespace
 
-bool grouped_supported(int E, int H, int I, int nv) {
+bool grouped_supported(int E, int H, int I, int nv, int s8) {
     // the pipeline stages of both products must fit the shared memory budget
     return E <= kGpMaxE && H % 128 == 0 && I % 128 == 0 && H <= 4096 && I <= 4096 &&
-           mma_smem(2, H, nv) <= kMmaSmemBudget && mma_smem(1, I, nv) <= kMmaSmemBudget;
+           !(nv && s8) && mma_smem(2, H, nv, s8) <= kMmaSmemBudget &&
+           mma_smem(1, I, nv, s8) <= kMmaSmemBudget;
 }
 
 cudaError_t launch_grouped(const GroupedParams &p, cudaStream_t s, bool pdl) {
-    if (p.T < 1 || p.T > kGroupedMaxT || !grouped_supported(p.E, p.H, p.I, p.nv))
+    if (p.T < 1 || p.T > kGroupedMaxT || !grouped_supported(p.E, p.H, p.I, p.nv, p.s8))
         return cudaErrorInvalidValue;
-    if (p.tcgen05 && (p.nv || !p.codes_base || !grouped_tc_supported(p.H, p.I, p.T * p.k)))
+    if (p.tcgen05 &&
+        (p.nv || p.s8 || !p.codes_base || !grouped_tc_supported(p.H, p.I, p.T * p.k)))
         return cudaErrorInvalidValue;
     if (p.nv && !p.gscale) return cudaErrorInvalidValue;
     cudaError_t e;
@@ -478,14 +504,16 @@ cudaError_t launch_grouped(const GroupedParams &p, cudaStream_t s, bool pdl) {
         if ((e = launch_grouped_tc_gateup(p, s, pdl)) != cudaSuccess) return e;
         if ((e = launch_grouped_tc_down(p, s, pdl)) != cudaSuccess) return e;
     } else {
-        if ((e = p.nv ? launch_mma<2, true>(p, s, pdl) : launch_mma<2, false>(p, s, pdl)) !=
-            cudaSuccess)
+        if ((e = p.s8   ? launch_mma<2, false, true>(p, s, pdl)
+                 : p.nv ? launch_mma<2, true, false>(p, s, pdl)
+                        : launch_mma<2, false, false>(p, s, pdl)) != cudaSuccess)
             return e;
         if ((e = launch_ex(grouped_stage_h_kernel, dim3(p.T * p.k), dim3(kGpThreads), 0, s, pdl,
                            p)) != cudaSuccess)
             return e;
-        if ((e = p.nv ? launch_mma<1, true>(p, s, pdl) : launch_mma<1, false>(p, s, pdl)) !=
-            cudaSuccess)
+        if ((e = p.s8   ? launch_mma<1, false, true>(p, s, pdl)
+                 : p.nv ? launch_mma<1, true, false>(p, s, pdl)
+                        : launch_mma<1, false, false>(p, s, pdl)) != cudaSuccess)
             return e;
     }
     return launch_ex(grouped_combine_kernel, dim3(p.T), dim3(kGpThreads), 0, s, pdl, p);

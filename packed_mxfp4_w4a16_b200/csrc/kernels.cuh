@@ -178,10 +178,11 @@ struct GroupedParams {
     int T, k, E, H, I;
     int tcgen05;               // products on tcgen05 (else mma.sync tiles)
     int nv;                    // NVFP4 weights: E4M3 scale per 16 (mma.sync tiles only)
+    int s8;                    // sym8 weights: int8, binary16 scale per 32 (mma.sync tiles only)
     const float *gscale;       // NVFP4: [E][2] FP32 multipliers (gate/up, down)
     TcMapCache *tc_maps;       // the handle's tensor-map cache (host), or null
 };
-bool grouped_supported(int E, int H, int I, int nv = 0);
+bool grouped_supported(int E, int H, int I, int nv = 0, int s8 = 0);
 cudaError_t launch_grouped(const GroupedParams &p, cudaStream_t s, bool pdl);
 // Products on tcgen05 (grouped_tc.cu): chosen by the forward when the groups
 // average at least kTcAutoGroup pairs (the mma.sync tiles convert the codes

@@ -1,17 +1,18 @@
 """sym8 experts (one int8 weight per element, one binary16 scale per 32 K
 elements; page "LFM2.5-8B-A1B — Core AI (.aimodel)", table "Provenance", row
-"Weight format") on the per-(token, slot) GEMV path against the oracle:
-SwiGLU vectors h, expert outputs o and combined y at the tolerance of the
-MXFP4 decode path; the combine bit-exact given the kernel's own o; every T
-(chunks of up to 4 tokens); invalid ids; the whole layer (route, then the
-forward); argument errors."""
+"Weight format") against the oracle: on the per-(token, slot) GEMV path
+(up to 4 tokens, or in chunks when asked) the SwiGLU vectors h, expert
+outputs o and combined y at the tolerance of the MXFP4 decode path; on the
+grouped mma.sync products (beyond 4 tokens) at the grouped path's tolerance;
+the combine bit-exact given the kernel's own o; invalid ids; the whole layer
+(route, then the forward); argument errors."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import packed_mxfp4_w4a16_b200 as moe
-from gpu_util import assert_close_rms, dev_bf16, host_bf16
+from gpu_util import assert_close_rms, check_grouped_y, dev_bf16, host_bf16
 from workloads import synth
 
 pytestmark = pytest.mark.gpu
@@ -67,20 +68,94 @@ def test_sym8_forward_matches_oracle(shape, T):
     layer.close()
 
 
-def test_sym8_many_tokens_run_in_chunks():
-    """Beyond 4 tokens the sym8 path runs in chunks; the grouped path is
-    refused."""
+def _check_grouped(L, layer, x, ids, w, shape, flags=0, residual=None):
+    """The grouped products against the oracle at the grouped path's
+    tolerance (the tensor-core tiles sum the exact products in another FP32
+    order: h within three BF16 values, o within two, both rarely; y by the
+    bound the combine's arithmetic gives), and the combine bit-exact given
+    the kernel's own o."""
+    T = x.shape[0]
+    y = layer.forward(dev_bf16(x), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(),
+                      flags=flags | moe.FWD_KEEP_INTERMEDIATES,
+                      residual=None if residual is None else dev_bf16(residual))
+    torch.cuda.synchronize()
+    h_g, o_g = layer.intermediates(T)
+    h_g, o_g, y_g = host_bf16(h_g), host_bf16(o_g), host_bf16(y)
+    w64 = w.astype(np.float64)
+    y_r, o_r, h_r = oracle.moe_forward_sym8(x, ids, w64, L.codes, L.scales, shape.E, shape.H,
+                                            shape.I, residual=residual, want_o=True, want_h=True)
+    valid = (ids >= 0) & (ids < shape.E)
+    assert_close_rms(h_g[valid], h_r[valid], what="sym8 grouped h", max_ulps=3)
+    assert_close_rms(o_g[valid], o_r[valid], what="sym8 grouped o", max_ulps=2)
+    check_grouped_y(y_g, y_r, o_g, o_r, w64, valid, residual, what="sym8 grouped y")
+    for t in range(T):
+        o_t = np.where(valid[t][:, None], o_g[t], 0).astype(np.uint16)
+        want = oracle.combine(o_t, w64[t], None if residual is None else residual[t])
+        np.testing.assert_array_equal(y_g[t], want)
+    return y_g
+
+
+@pytest.mark.parametrize("shape,T,dist", [
+    (synth.TINY, 5, "uniform"), (synth.TINY, 33, "zipf"), (synth.TINY, 60, "uniform"),
+    (synth.L24B, 5, "uniform"), (synth.L24B, 64, "uniform"), (synth.L24B, 64, "zipf"),
+    (synth.L24B, 200, "uniform"), (synth.L8B, 17, "zipf")])
+def test_sym8_grouped_matches_oracle(shape, T, dist):
+    """Beyond the decode sizes sym8 experts run the (token, expert)-sorted
+    grouped products (int8 rows converted to FP16 exactly on the tensor
+    cores, the binary16 block scale applied per 32-element group in FP32):
+    h, o and y against the oracle."""
+    L, layer = _layer(shape, 79, max_tokens=T)
+    x = synth.make_tokens(T, shape.H, seed=79, stream=T)
+    ids, w = synth.make_routing(T, shape.E, shape.top_k, dist, synth.rng_for(79, 13, T))
+    r = synth.make_tokens(T, shape.H, seed=80, stream=T) if T % 2 else None
+    _check_grouped(L, layer, x, ids, w, shape, residual=r)
+    assert layer.status() == 0
+    layer.close()
+
+
+def test_sym8_grouped_and_per_pair_paths_both_hold():
+    """The same batch on the grouped products (default beyond 4 tokens,
+    FWD_FORCE_MMA, and FWD_FORCE_GROUPED at 3 tokens) and on the per-(token,
+    slot) GEMVs in chunks (FWD_FORCE_DECODE), each against the oracle;
+    invalid ids on the grouped path zero the slot and flag; the tcgen05
+    products are refused; scales that are only 2-byte aligned keep the batch
+    on the per-pair GEMVs (the grouped products are refused)."""
     shape = synth.TINY
     T = 11
     L, layer = _layer(shape, 73, max_tokens=T)
     x = synth.make_tokens(T, shape.H, seed=73)
     ids, w = synth.make_routing(T, shape.E, shape.top_k, "zipf", synth.rng_for(73, 13, T))
-    _check(L, layer, x, ids, w, shape)
-    for flags in (moe.FWD_FORCE_GROUPED, moe.FWD_FORCE_MMA):
-        with pytest.raises(moe.MoEError):
-            layer.forward(dev_bf16(x), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(),
-                          flags=flags)
+    y_g = _check_grouped(L, layer, x, ids, w, shape)
+    np.testing.assert_array_equal(_check_grouped(L, layer, x, ids, w, shape,
+                                                 flags=moe.FWD_FORCE_MMA), y_g)
+    y_d = layer.forward(dev_bf16(x), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(),
+                        flags=moe.FWD_FORCE_DECODE | moe.FWD_KEEP_INTERMEDIATES)
+    torch.cuda.synchronize()
+    y_r = oracle.moe_forward_sym8(x, ids, w.astype(np.float64), L.codes, L.scales, shape.E,
+                                  shape.H, shape.I)
+    assert_close_rms(host_bf16(y_d), y_r, what="sym8 per-pair y", max_ulps=2)
+    _check_grouped(L, layer, x[:3], ids[:3], w[:3], shape, flags=moe.FWD_FORCE_GROUPED)
+    with pytest.raises(moe.MoEError):
+        layer.forward(dev_bf16(x), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(),
+                      flags=moe.FWD_FORCE_TCGEN05)
+    bad = ids.copy()
+    bad[2, 1] = 99
+    bad[7, 0] = -3
+    _check_grouped(L, layer, x, bad, w, shape)
+    assert layer.status() & moe.DEVICE_BAD_EXPERT_ID
     layer.close()
+
+    q, s = _dev_sym8(L)
+    pool = torch.zeros(s.numel() + 8, dtype=torch.int16, device="cuda")
+    s2 = pool[1:1 + s.numel()].view(s.shape)  # 2-byte aligned only
+    s2.copy_(s)
+    rw = dev_bf16(L.router_w)
+    layer2 = moe.MoELayer(shape.E, shape.H, shape.I, shape.top_k, q, s2, rw, None, max_tokens=T)
+    _check(L, layer2, x, ids, w, shape)
+    with pytest.raises(moe.MoEError):
+        layer2.forward(dev_bf16(x), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(),
+                       flags=moe.FWD_FORCE_GROUPED)
+    layer2.close()
 
 
 def test_sym8_invalid_ids_zero_the_slot_and_flag():
