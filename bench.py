@@ -434,6 +434,7 @@ def sym8_stack(torch, moe, st, args, max_steps=4):
            "hbm_frac": tok_bytes * n_tok / (t_ms / 1e3) / 1e9 / peak,
            "gpu_launches_per_token": 3 * len(s8.layers), "steps": steps}
     s8.close()
+    out["prefill_s64"] = sym8_prefill_chunk(torch, moe, weights[0], args.seed, peak)
     del weights
     torch.cuda.empty_cache()
     return out
@@ -736,6 +737,48 @@ def config_stack8b(torch, moe, seed, steps=4):
 BATCHED_CASES = ((32, "uniform"), (32, "zipf"), (64, "uniform"), (64, "zipf"), (256, "uniform"),
                  (256, "zipf"), (1024, "uniform"), (2048, "uniform"), (2048, "zipf"))
 TC_AUTO_GROUP = 40  # the library's tcgen05 products from T k >= 40 E on
+
+
+def sym8_prefill_chunk(torch, moe, lw, seed, peak, T=64, reps=10):
+    """One sym8 layer (the first layer's weights of the sym8 stack) at the
+    S = 64 prefill chunk with uniform routing: the grouped mma.sync products,
+    moe_forward timed in a CUDA graph of `reps` calls.  Bytes: the touched
+    experts' int8 codes and binary16 scales + activations."""
+    q, sc, rw, rb = lw
+    lay = moe.MoELayer(SHAPE.E, SHAPE.H, SHAPE.I, SHAPE.top_k, q, sc, rw, rb, max_tokens=T)
+    x = torch.from_numpy(synth.make_tokens(T, SHAPE.H, seed=seed, stream=T)
+                         .view(np.int16)).cuda().view(torch.bfloat16)
+    ids_h, w_h = synth.make_routing(T, SHAPE.E, SHAPE.top_k, "uniform",
+                                    synth.rng_for(seed, 91, T))
+    ids, w = torch.from_numpy(ids_h).cuda(), torch.from_numpy(w_h).cuda()
+    y = torch.empty_like(x)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        lay.forward(x, ids, w, y=y, stream=s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for _ in range(reps):
+            lay.forward(x, ids, w, y=y, stream=s)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    assert lay.status() == 0
+    del g
+    lay.close()
+    n_w = 3 * SHAPE.I * SHAPE.H
+    touched = len(set(ids_h.ravel().tolist()))
+    nbytes = touched * (n_w + n_w // 16) + T * SHAPE.H * 2 * 2
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"T": T, "routing": "uniform", "products": "mma.sync (grouped)",
+            "experts_touched": touched, "us_per_call": us, "hbm_gbs": gbs,
+            "hbm_frac": gbs / peak}
 
 
 def batched_cases(torch, moe, st, seed, reps=20, cases=BATCHED_CASES):

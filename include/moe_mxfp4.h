@@ -166,12 +166,16 @@ MOE_API int moe_load_expert_table(moe_handle_t h, const uint8_t *const *codes_pt
  * multiplier.  codes / scales 16-byte aligned, global_scales 4-byte aligned;
  * read in place, caller-owned.  Requires H a multiple of 512 up to 4096 (the
  * bulk-copy gate/up kernel).  NVFP4 layers run the per-(token, slot) path
- * for T = 1..4 and the grouped path's mma.sync products beyond (each 16-
+ * for T = 1..4 and the grouped path beyond: mma.sync products (each 16-
  * element block's partial product scaled by its E4M3 scale in FP32, the
- * multiplier applied with the activation staging scale); no tcgen05
- * products (FORCE_TCGEN05 returns ARG), no fused launch structures, no stack
- * kernel.  moe_load_packed / moe_load_expert_table switch the handle back to
- * MXFP4.  Errors: as moe_load_packed. */
+ * multiplier applied with the activation staging scale), or, for large
+ * groups, tcgen05 products (A = code x its block's E4M3 scale in BF16,
+ * exact; the multiplier applied to the FP32 accumulator).  The grouped path
+ * takes NVFP4 batches in chunks of up to 1024 tokens at the 24B shape (a
+ * chunk's tcgen05 plan must fit the shared memory).  The one-launch stack
+ * takes NVFP4 layers; no fused launch structures.  moe_load_packed /
+ * moe_load_expert_table switch the handle back to MXFP4.  Errors: as
+ * moe_load_packed. */
 MOE_API int moe_load_packed_nvfp4(moe_handle_t h, const uint8_t *codes_u8,
                                   const uint8_t *scales_e4m3, const float *global_scales);
 
@@ -244,12 +248,13 @@ MOE_API int moe_route_ex(moe_handle_t h, const uint16_t *x, int T,
  * makes that slot contribute 0 and sets MOE_DEVICE_BAD_EXPERT_ID in the
  * device status word.  T = 1..4 runs the per-(token, slot) GEMV path;
  * larger T the (token, expert)-sorted grouped path, in chunks of up to 2048
- * tokens: its products run on mma.sync tiles, or on tcgen05 (BF16 weight tiles
- * dequantised once per CTA, FP32 accumulators in tensor memory, packed codes
- * brought in by TMA tensor loads) when a chunk's groups average at least 40
- * (token, slot) pairs per expert (T k >= 40 E) and the weights allow it
- * (contiguous MXFP4 from moe_load_packed, H and I multiples of 128; NVFP4
- * and sym8 weights always take the mma.sync tiles);
+ * tokens (NVFP4: halved until a chunk's tcgen05 plan fits): its products run
+ * on mma.sync tiles, or on tcgen05 (BF16 weight tiles dequantised once per
+ * CTA, FP32 accumulators in tensor memory, packed codes brought in by TMA
+ * tensor loads) when a chunk's groups average at least 40 (token, slot)
+ * pairs per expert (T k >= 40 E) and the weights allow it (contiguous MXFP4
+ * or NVFP4 from moe_load_packed / moe_load_packed_nvfp4, H and I multiples
+ * of 128; sym8 weights always take the mma.sync tiles);
  * MOE_FWD_FORCE_TCGEN05 / MOE_FWD_FORCE_MMA pin the choice.  Errors: ARG,
  * NOT_LOADED, NOT_DEVICE, ALIGN, WORKSPACE, CUDA. */
 MOE_API int moe_forward(moe_handle_t h, const uint16_t *x, int T,

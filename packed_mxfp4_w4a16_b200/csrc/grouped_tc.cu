@@ -179,12 +179,13 @@ __host__ __device__ constexpr uint32_t tc_sc_off(int nmat) {
     return tc_raw_off(nmat) + (uint32_t)kTcRaw * nmat * kTcRawSlot;
 }
 // then the B row of every token of the group ([pairs] ints; a group holds at
-// most all the launch's T k pairs)
-__host__ __device__ inline uint32_t tc_src_off(int nmat, int K) {
-    return tc_sc_off(nmat) + (uint32_t)nmat * kTcM * (uint32_t)(K / 32);
+// most all the launch's T k pairs).  Scale rows: K/32 E8M0 bytes, or K/16
+// E4M3 bytes (nv).
+__host__ __device__ inline uint32_t tc_src_off(int nmat, int K, int nv) {
+    return tc_sc_off(nmat) + (uint32_t)nmat * kTcM * (uint32_t)(K / (nv ? 16 : 32));
 }
-__host__ __device__ inline uint32_t tc_smem_bytes(int nmat, int K, int pairs) {
-    return tc_src_off(nmat, K) + (uint32_t)pairs * sizeof(int);
+__host__ __device__ inline uint32_t tc_smem_bytes(int nmat, int K, int pairs, int nv) {
+    return tc_src_off(nmat, K, nv) + (uint32_t)pairs * sizeof(int);
 }
 
 // One TMA tile load of the 3-D code tensor (x: byte in the row, y: row,
@@ -217,7 +218,10 @@ __device__ __forceinline__ bool tc_wait(uint64_t *bar, unsigned parity, volatile
 // in shared memory), s_mma[s] (tcgen05.commit: the tile's products are done,
 // the stage may be rewritten), s_raw[j] (TMA bytes of ring slot j), s_tfree
 // (16 arrivals: the pass's accumulators were read).
-template <int NMAT>
+// NV: NVFP4 weights: A = code x its 16-element block's E4M3 scale (exact in
+// BF16: at most 6 significant bits), the expert's FP32 multiplier applied to
+// the accumulator in the epilogue (one FP32 rounding before the BF16 one).
+template <int NMAT, bool NV>
 __global__ void __launch_bounds__(kTcThreads, 1)
 grouped_tc_kernel(const GroupedParams p, const __grid_constant__ CUtensorMap codes_map) {
     extern __shared__ __align__(1024) uint8_t sm[];
@@ -240,12 +244,12 @@ grouped_tc_kernel(const GroupedParams p, const __grid_constant__ CUtensorMap cod
     const int nkt = K / kTcK;
     const int npass = (n_e + kTcMaxN - 1) / kTcMaxN;
     const int total = npass * nkt;  // (pass, K tile) iterations
-    const uint32_t rs = (uint32_t)K >> 5;
+    const uint32_t rs = (uint32_t)K >> (NV ? 4 : 5);  // scale bytes per row
     uint8_t *raw = sm + tc_raw_off(NMAT);
     uint8_t *scl = sm + tc_sc_off(NMAT);
     // per token of the group: its B row (x row of the pair's token, or h row
     // of the pair)
-    int *s_src = reinterpret_cast<int *>(sm + tc_src_off(NMAT, K));
+    int *s_src = reinterpret_cast<int *>(sm + tc_src_off(NMAT, K, NV ? 1 : 0));
 
     if (warp == 0) {  // TMEM: NMAT x 128 FP32 columns x 128 lanes
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -336,8 +340,8 @@ grouped_tc_kernel(const GroupedParams p, const __grid_constant__ CUtensorMap cod
         for (int m = 0; m < NMAT; ++m) {
             const int mat = NMAT == 2 ? m : 2;
             const uint8_t *gsc = tc_scales(p, e, mat) + (size_t)(row0 + rrow) * rs;
-            // K / 32 is a multiple of 4 (K % 128 == 0): the row's scales in
-            // 4-byte pieces, spread over its four threads
+            // K / 32 and K / 16 are multiples of 4 (K % 128 == 0): the row's
+            // scales in 4-byte pieces, spread over its four threads
             for (uint32_t c = 4 * quarter; c < rs; c += 16)
                 asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
                                  smem_u32(scl + ((uint32_t)m * kTcM + rrow) * rs + c)),
@@ -388,10 +392,18 @@ grouped_tc_kernel(const GroupedParams p, const __grid_constant__ CUtensorMap cod
             const uint8_t *slot = raw + (uint32_t)(it % kTcRaw) * NMAT * kTcRawSlot;
 #pragma unroll
             for (int m = 0; m < NMAT; ++m) {
-                // K-chunks 2 q, 2 q + 1 of the row (8 code bytes; one scale group)
+                // K-chunks 2 q, 2 q + 1 of the row (8 code bytes: one E8M0
+                // group, or exactly one 16-element E4M3 block)
                 const uint2 cw = *reinterpret_cast<const uint2 *>(
                     slot + (uint32_t)m * kTcRawSlot + (uint32_t)rrow * 32 + 8 * quarter);
-                const float sf = e8m0_to_f32(scl[((uint32_t)m * kTcM + rrow) * rs + 2 * kt + (quarter >> 1)]);
+                const uint8_t *srow = scl + ((uint32_t)m * kTcM + rrow) * rs;
+                float sf;
+                if (NV) {
+                    float hi_unused;
+                    e4m3x2_to_f32(srow[4 * kt + quarter], sf, hi_unused);
+                } else {
+                    sf = e8m0_to_f32(srow[2 * kt + (quarter >> 1)]);
+                }
                 uint8_t *a = st + (uint32_t)m * kTcTileA;
                 *reinterpret_cast<uint4 *>(a + tc_off(rrow, 2 * quarter)) = dequant8_bf16(cw.x, sf);
                 *reinterpret_cast<uint4 *>(a + tc_off(rrow, 2 * quarter + 1)) = dequant8_bf16(cw.y, sf);
@@ -408,6 +420,8 @@ grouped_tc_kernel(const GroupedParams p, const __grid_constant__ CUtensorMap cod
                 const int r = row0 + lq * 32 + lane;  // this thread's matrix row
                 const uint32_t lane_base = tmem + ((uint32_t)(lq * 32) << 16);
                 const int N = (nt + 15) & ~15;
+                // NVFP4: the expert's multiplier (gate/up or down)
+                const float gm = NV ? __ldg(p.gscale + 2 * e + (NMAT == 2 ? 0 : 1)) : 1.0f;
                 #pragma unroll 1
                 for (int c0 = 8 * (warp >> 2); c0 < N; c0 += 32) {
                     float g[8], u[8];
@@ -419,12 +433,12 @@ grouped_tc_kernel(const GroupedParams p, const __grid_constant__ CUtensorMap cod
                         if (idx >= tc + nt) continue;
                         const int pr = p.perm[seg0 + idx];
                         if (NMAT == 2) {
-                            const float gv = round_bf16(g[j]);
-                            const float uv = round_bf16(u[j]);
+                            const float gv = round_bf16(NV ? g[j] * gm : g[j]);
+                            const float uv = round_bf16(NV ? u[j] * gm : u[j]);
                             const float sl = round_bf16(gv / (1.0f + expf(-gv)));
                             p.h[(size_t)pr * M + r] = f32_to_bf16(sl * uv);
                         } else {
-                            p.o[(size_t)pr * M + r] = f32_to_bf16(g[j]);
+                            p.o[(size_t)pr * M + r] = f32_to_bf16(NV ? g[j] * gm : g[j]);
                         }
                     }
                 }
@@ -506,22 +520,22 @@ cudaError_t codes_map_copy(CodesMap &c, std::mutex &mu, const GroupedParams &p, 
     return e;
 }
 
-template <int NMAT>
+template <int NMAT, bool NV>
 cudaError_t launch_tc(const GroupedParams &p, const CUtensorMap &map, cudaStream_t s, bool pdl) {
     const int K = NMAT == 2 ? p.H : p.I, M = NMAT == 2 ? p.I : p.H;
-    const size_t smem = tc_smem_bytes(NMAT, K, p.T * p.k);
+    const size_t smem = tc_smem_bytes(NMAT, K, p.T * p.k, NV ? 1 : 0);
     if (smem > kTcSmemBudget) return cudaErrorInvalidValue;
     // the budget, once per device (the attribute belongs to the current
     // device's context)
     static PerDeviceOnce once;
     const cudaError_t attr = per_device_once(once, [] {
-        return cudaFuncSetAttribute(grouped_tc_kernel<NMAT>,
+        return cudaFuncSetAttribute(grouped_tc_kernel<NMAT, NV>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)kTcSmemBudget);
     });
     if (attr != cudaSuccess) return attr;
-    return launch_ex(grouped_tc_kernel<NMAT>, dim3(M / kTcM, p.E), dim3(kTcThreads), smem, s, pdl,
-                     p, map);
+    return launch_ex(grouped_tc_kernel<NMAT, NV>, dim3(M / kTcM, p.E), dim3(kTcThreads), smem, s,
+                     pdl, p, map);
 }
 
 }  // namespace
@@ -529,9 +543,9 @@ cudaError_t launch_tc(const GroupedParams &p, const CUtensorMap &map, cudaStream
 // The tensor-core products need the contiguous weight layout (one tensor map
 // per matrix kind), H and I multiples of 128 and the shared-memory plan of a
 // launch of `pairs` (token, slot) pairs within the budget.
-bool grouped_tc_supported(int H, int I, int pairs) {
-    return H % 128 == 0 && I % 128 == 0 && tc_smem_bytes(2, H, pairs) <= kTcSmemBudget &&
-           tc_smem_bytes(1, I, pairs) <= kTcSmemBudget;
+bool grouped_tc_supported(int H, int I, int pairs, int nv) {
+    return H % 128 == 0 && I % 128 == 0 && tc_smem_bytes(2, H, pairs, nv) <= kTcSmemBudget &&
+           tc_smem_bytes(1, I, pairs, nv) <= kTcSmemBudget;
 }
 
 namespace {
@@ -570,7 +584,7 @@ cudaError_t launch_grouped_tc_gateup(const GroupedParams &p, cudaStream_t s, boo
     CUtensorMap map;
     cudaError_t e = kind_map(p, 0, p.I, p.H, gu, mu, &map);
     if (e != cudaSuccess) return e;
-    return launch_tc<2>(p, map, s, pdl);
+    return p.nv ? launch_tc<2, true>(p, map, s, pdl) : launch_tc<2, false>(p, map, s, pdl);
 }
 
 cudaError_t launch_grouped_tc_down(const GroupedParams &p, cudaStream_t s, bool pdl) {
@@ -580,7 +594,7 @@ cudaError_t launch_grouped_tc_down(const GroupedParams &p, cudaStream_t s, bool 
     CUtensorMap map;
     cudaError_t e = kind_map(p, 1, p.H, p.I, dn, mu, &map);
     if (e != cudaSuccess) return e;
-    return launch_tc<1>(p, map, s, pdl);
+    return p.nv ? launch_tc<1, true>(p, map, s, pdl) : launch_tc<1, false>(p, map, s, pdl);
 }
 
 }  // namespace moe

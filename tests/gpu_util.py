@@ -98,7 +98,7 @@ def check_routing(gpu_ids, gpu_w, gpu_logits, ref_ids, ref_w, ref_logits, k):
     return int(ties.sum())
 
 
-def check_grouped_y(y_g, y_r, o_g, o_r, w64, valid, residual=None, what="grouped y"):
+def check_grouped_y(y_g, y_r, o_g, o_r, w64, valid, residual=None, what="grouped y", cap=True):
     """The grouped paths' rule for the combined output y (reading R14)."""
     # y is a function of o alone (the bit-exact combine check below), so its
     # distance to the oracle's y is bounded by the o differences through the
@@ -120,5 +120,8 @@ def check_grouped_y(y_g, y_r, o_g, o_r, w64, valid, residual=None, what="grouped
     # combine that cancels (|y| << |w o|) is many ulps of y, so the ulp
     # distance of those few elements is capped loosely but their number is
     # held to 0.05 % (observed worst: 7 of 65,536 at 2.8e-2 rms, 8 ulps, T=260
-    # Zipf on tcgen05; all inside the o-derived bound above)
-    assert_close_rms(y_g, y_r, what=what, max_ulps=16, max_flip_frac=5e-4)
+    # Zipf on tcgen05; all inside the o-derived bound above).  cap=False: the
+    # caller verified o stage by stage (against the oracle's down product of
+    # the kernel's own h), so only the derived bound applies here.
+    if cap:
+        assert_close_rms(y_g, y_r, what=what, max_ulps=16, max_flip_frac=5e-4)

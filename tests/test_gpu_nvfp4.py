@@ -1,16 +1,17 @@
 """NVFP4 experts (E2M1 codes, an FP8 E4M3 scale per 16 elements, an FP32
 multiplier per expert for gate/up and one for down) against the oracle: the
-per-(token, slot) path (T <= 4) and the grouped mma.sync products (larger
-T, or forced) — SwiGLU vectors h, expert outputs o and combined y at the
-tolerance of the MXFP4 paths; the combine bit-exact given the kernel's own o;
-uniform and Zipf routing; invalid ids; the whole layer; argument errors."""
+per-(token, slot) path (T <= 4), the grouped mma.sync products (larger T,
+or forced) and the grouped tcgen05 products (large groups, or forced) —
+SwiGLU vectors h, expert outputs o and combined y at the tolerance of the
+MXFP4 paths; the combine bit-exact given the kernel's own o; uniform and
+Zipf routing; invalid ids; the whole layer; argument errors."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import packed_mxfp4_w4a16_b200 as moe
-from gpu_util import assert_close_rms, check_grouped_y, dev_bf16, dev_u8, host_bf16
+from gpu_util import assert_close_rms, check_grouped_y, dev_bf16, dev_u8, f64, host_bf16
 from workloads import synth
 
 pytestmark = pytest.mark.gpu
@@ -25,7 +26,7 @@ def _layer(shape, seed, max_tokens=4, bias=False):
     return L, layer
 
 
-def _check(L, layer, x, ids, w, shape, residual=None, flags=0, ulps=1):
+def _check(L, layer, x, ids, w, shape, residual=None, flags=0, ulps=1, h_ulps=None):
     T = x.shape[0]
     y = layer.forward(dev_bf16(x), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(),
                       flags=moe.FWD_KEEP_INTERMEDIATES | flags,
@@ -38,7 +39,7 @@ def _check(L, layer, x, ids, w, shape, residual=None, flags=0, ulps=1):
                                              shape.H, shape.I, residual=residual, want_o=True,
                                              want_h=True)
     valid = (ids >= 0) & (ids < shape.E)
-    assert_close_rms(h_g[valid], h_r[valid], what="nvfp4 h", max_ulps=ulps)
+    assert_close_rms(h_g[valid], h_r[valid], what="nvfp4 h", max_ulps=h_ulps or ulps)
     assert_close_rms(o_g[valid], o_r[valid], what="nvfp4 o", max_ulps=ulps)
     if ulps > 1:
         # grouped products: the grouped paths' y rule (o-derived bound)
@@ -72,17 +73,147 @@ def test_nvfp4_forward_matches_oracle(shape, T):
     (synth.L24B, 64, "uniform", 0), (synth.L24B, 64, "zipf", 0),
     (synth.L8B, 40, "uniform", moe.FWD_FORCE_GROUPED)])
 def test_nvfp4_grouped_matches_oracle(shape, T, dist, flags):
-    """Beyond 4 tokens (or forced) NVFP4 runs the grouped mma.sync products;
-    the tcgen05 products refuse NVFP4."""
+    """Beyond 4 tokens (or forced) NVFP4 runs the grouped mma.sync products
+    while the groups are small."""
     L, layer = _layer(shape, 43, max_tokens=T)
     x = synth.make_tokens(T, shape.H, seed=43, stream=T)
     ids, w = synth.make_routing(T, shape.E, shape.top_k, dist, synth.rng_for(43, 13, T))
     r = synth.make_tokens(T, shape.H, seed=44, stream=T)
     _check(L, layer, x, ids, w, shape, residual=r, flags=flags, ulps=2)
     assert layer.status() == 0
-    with pytest.raises(moe.MoEError):
-        layer.forward(dev_bf16(x), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(),
-                      flags=moe.FWD_FORCE_TCGEN05)
+    layer.close()
+
+
+def _nv_matrix(L, shape, e, m):
+    """The oracle's dequantised matrix m (0 gate, 1 up, 2 down) of expert e:
+    code x E4M3 block scale x the expert's multiplier, FP64 [rows, K]."""
+    n = shape.I * shape.H
+    c = np.ascontiguousarray(L.codes.reshape(shape.E, 3, n // 2)[e, m])
+    s = np.ascontiguousarray(L.scales.reshape(shape.E, 3, n // 16)[e, m])
+    rows, K = (shape.I, shape.H) if m < 2 else (shape.H, shape.I)
+    return oracle.dequant_nvfp4(c, s, float(L.gscales[e, 0 if m < 2 else 1]), n).reshape(rows, K)
+
+
+def _near_midpoint(v, mag, rel=2.0 ** -16):
+    """v lies within rel * mag of a BF16 rounding midpoint (mag: the sum of
+    the magnitudes the FP32 accumulation added, or |v| for one operation)."""
+    b = oracle.bf16_from_f64(v)
+    lo = oracle.bf16_to_f64(b)
+    nb = oracle.bf16_to_f64(b + 1 if (v >= lo) == (v >= 0) else b - 1)
+    return abs(v - (lo + nb) / 2) <= rel * mag
+
+
+def _neighbours(v, movable):
+    b = oracle.bf16_from_f64(v)
+    vals = [oracle.bf16_to_f64(b)]
+    if movable and b & 0x7FFF:
+        vals += [oracle.bf16_to_f64(b + 1), oracle.bf16_to_f64(b - 1)]
+    return vals
+
+
+def _check_tcgen05_stages(L, layer, x, ids, w, shape, residual=None, flags=moe.FWD_FORCE_TCGEN05):
+    """Stage by stage against the oracle (reading R14).  h: within 1e-2 rms of
+    the oracle's h, except elements that the oracle's own rounding chain
+    reproduces, h = BF16(BF16(silu(g')) u') , with g', u' and silu(g') each
+    allowed one BF16 ulp away only where the exact value (FP64 from the
+    oracle's dequantised rows) lies within 2^-16 of its accumulated magnitude
+    of a rounding midpoint; such elements stay rare.  o: the oracle's down
+    product of the kernel's own h (FP64, rounded once), within the decode
+    tolerance.  y: bit-exact given the kernel's o, and within the o-derived
+    bound of the oracle's y."""
+    T = x.shape[0]
+    y = layer.forward(dev_bf16(x), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(),
+                      flags=moe.FWD_KEEP_INTERMEDIATES | flags,
+                      residual=None if residual is None else dev_bf16(residual))
+    torch.cuda.synchronize()
+    h_g, o_g = layer.intermediates(T)
+    h_g, o_g, y_g = host_bf16(h_g), host_bf16(o_g), host_bf16(y)
+    _verify_stages(L, shape, x, ids, w, h_g, o_g, y_g, residual)
+    return y_g
+
+
+def _verify_stages(L, shape, x, ids, w, h_g, o_g, y_g, residual=None):
+    """The checks of _check_tcgen05_stages on given kernel outputs (rows of
+    a batch: x, ids, w, h, o, y of the same tokens)."""
+    T = x.shape[0]
+    w64 = w.astype(np.float64)
+    y_r, o_r, h_r = oracle.moe_forward_nvfp4(x, ids, w64, L.codes, L.scales, L.gscales, shape.E,
+                                             shape.H, shape.I, residual=residual, want_o=True,
+                                             want_h=True)
+    valid = (ids >= 0) & (ids < shape.E)
+    hg64, hr64 = f64(h_g), f64(h_r)
+    rms = np.sqrt(np.mean(hr64 ** 2, axis=2, keepdims=True))
+    far = valid[:, :, None] & (np.abs(hg64 - hr64) > 1e-2 * rms)
+    cache = {}
+    for t, j, i in np.argwhere(far):
+        e = int(ids[t, j])
+        if e not in cache:
+            cache = {e: (_nv_matrix(L, shape, e, 0), _nv_matrix(L, shape, e, 1))}
+        wg, wu = cache[e][0][i], cache[e][1][i]
+        xt = f64(x[t])
+        g, u = float(wg @ xt), float(wu @ xt)
+        g_ok = _near_midpoint(g, float(np.abs(wg * xt).sum()))
+        u_ok = _near_midpoint(u, float(np.abs(wu * xt).sum()))
+        want = float(hg64[t, j, i])
+        hits = False
+        for gg in _neighbours(g, g_ok):
+            sl = gg / (1.0 + np.exp(-gg))
+            for ss in _neighbours(sl, _near_midpoint(sl, abs(sl))):
+                for uu in _neighbours(u, u_ok):
+                    hits |= oracle.bf16_to_f64(oracle.bf16_from_f64(ss * uu)) == want
+        assert hits, f"h[{t},{j},{i}] = {want} is no one-ulp rounding move of g={g}, u={u}"
+    assert far.sum() <= 1e-3 * valid.sum() * shape.I, f"h: {far.sum()} elements beyond 1e-2 rms"
+    # o against the oracle's down product of the kernel's own h
+    o_ref = np.zeros_like(o_g)
+    for e in np.unique(ids[valid]):
+        wd = _nv_matrix(L, shape, int(e), 2)
+        sel = valid & (ids == e)
+        o_ref[sel] = oracle.bf16_from_f64_array(hg64[sel] @ wd.T)
+    assert_close_rms(o_g[valid], o_ref[valid], what="nvfp4 tcgen05 o (given h)", max_ulps=2)
+    check_grouped_y(y_g, y_r, o_g, o_r, w64, valid, residual, what="nvfp4 tcgen05 y", cap=False)
+    for t in range(T):
+        o_t = np.where(valid[t][:, None], o_g[t], 0).astype(np.uint16)
+        want = oracle.combine(o_t, w64[t], None if residual is None else residual[t])
+        np.testing.assert_array_equal(y_g[t], want)
+
+
+@pytest.mark.parametrize("shape,T,dist", [
+    (synth.L24B, 320, "uniform"), (synth.L24B, 260, "zipf"), (synth.L24B, 9, "uniform"),
+    (synth.TINY, 100, "zipf"), (synth.TINY, 33, "uniform"), (synth.L8B, 40, "zipf")])
+def test_nvfp4_tcgen05_matches_oracle(shape, T, dist):
+    """NVFP4 on the tcgen05 products (A = E2M1 code x its block's E4M3 scale
+    in BF16, exact; the expert's multiplier on the FP32 accumulator), stage
+    by stage against the oracle; two runs give the same bits."""
+    L, layer = _layer(shape, 49, max_tokens=T)
+    x = synth.make_tokens(T, shape.H, seed=49, stream=T)
+    ids, w = synth.make_routing(T, shape.E, shape.top_k, dist, synth.rng_for(49, 13, T))
+    r = synth.make_tokens(T, shape.H, seed=50, stream=T) if T % 2 else None
+    y1 = _check_tcgen05_stages(L, layer, x, ids, w, shape, residual=r)
+    y2 = _check_tcgen05_stages(L, layer, x, ids, w, shape, residual=r)
+    np.testing.assert_array_equal(y1, y2)
+    assert layer.status() == 0
+    layer.close()
+
+
+def test_nvfp4_tcgen05_chunks_and_automatic_choice():
+    """1100 tokens of the 24B shape: the NVFP4 batch runs in chunks of 1024
+    tokens (a chunk's tcgen05 plan must fit the shared memory with E4M3 scale
+    rows), the first on tcgen05 (its groups average 64 pairs per expert) and
+    the ragged rest on mma.sync.  Sampled tokens from both chunks (h, o, y)
+    against the oracle."""
+    shape = synth.L24B
+    T = 1100
+    L, layer = _layer(shape, 51, max_tokens=T)
+    x = synth.make_tokens(T, shape.H, seed=51, stream=T)
+    ids, w = synth.make_routing(T, shape.E, shape.top_k, "uniform", synth.rng_for(51, 13, T))
+    y = layer.forward(dev_bf16(x), torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(),
+                      flags=moe.FWD_KEEP_INTERMEDIATES)
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    h_g, o_g = layer.intermediates(T)
+    h_g, o_g, y_g = host_bf16(h_g), host_bf16(o_g), host_bf16(y)
+    rows = np.r_[0:6, 1018:1030, 1094:1100]
+    _verify_stages(L, shape, x[rows], ids[rows], w[rows], h_g[rows], o_g[rows], y_g[rows])
     layer.close()
 
 
