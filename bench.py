@@ -349,12 +349,13 @@ def nvfp4_stack(torch, moe, st, args, max_steps=8):
            "tokens_per_s": n_tok / (t_ms / 1e3), "us_per_token": t_ms * 1e3 / n_tok,
            "bytes_per_token": tok_bytes, "hbm_gbs": tok_bytes * n_tok / (t_ms / 1e3) / 1e9,
            "steps": steps}
-    # the grouped path (mma.sync products) with NVFP4 experts, one layer
+    # the grouped path with NVFP4 experts, one layer (mma.sync products at
+    # T = 64 and 256, tcgen05 at T = 1024)
     codes, sc, rw, rb, gs = weights[0]
     lay = moe.MoELayer(SHAPE.E, SHAPE.H, SHAPE.I, SHAPE.top_k, codes, sc, rw, rb,
-                       max_tokens=256, gscales=gs)
+                       max_tokens=1024, gscales=gs)
     grouped = []
-    for T in (64, 256):
+    for T in (64, 256, 1024):
         x = torch.from_numpy(synth.make_tokens(T, SHAPE.H, seed=args.seed, stream=T)
                              .view(np.int16)).cuda().view(torch.bfloat16)
         ids_h, w_h = synth.make_routing(T, SHAPE.E, SHAPE.top_k, "uniform",
@@ -375,8 +376,9 @@ def nvfp4_stack(torch, moe, st, args, max_steps=8):
         us = e0.elapsed_time(e1) * 1e3 / 20
         del g
         touched = len(set(ids_h.ravel().tolist()))
+        tc = T * SHAPE.top_k >= TC_AUTO_GROUP * SHAPE.E
         grouped.append({"T": T, "routing": "uniform", "experts_touched": touched,
-                        "products": "mma.sync", "us_per_call": us,
+                        "products": "tcgen05" if tc else "mma.sync", "us_per_call": us,
                         "hbm_gbs": (touched * per_expert + 2 * T * SHAPE.H * 2) / (us * 1e-6) / 1e9})
     assert lay.status() == 0
     lay.close()

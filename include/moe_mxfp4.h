@@ -170,9 +170,7 @@ MOE_API int moe_load_expert_table(moe_handle_t h, const uint8_t *const *codes_pt
  * element block's partial product scaled by its E4M3 scale in FP32, the
  * multiplier applied with the activation staging scale), or, for large
  * groups, tcgen05 products (A = code x its block's E4M3 scale in BF16,
- * exact; the multiplier applied to the FP32 accumulator).  The grouped path
- * takes NVFP4 batches in chunks of up to 1024 tokens at the 24B shape (a
- * chunk's tcgen05 plan must fit the shared memory).  The one-launch stack
+ * exact; the multiplier applied to the FP32 accumulator).  The one-launch stack
  * takes NVFP4 layers; no fused launch structures.  moe_load_packed /
  * moe_load_expert_table switch the handle back to MXFP4.  Errors: as
  * moe_load_packed. */
@@ -248,7 +246,7 @@ MOE_API int moe_route_ex(moe_handle_t h, const uint16_t *x, int T,
  * makes that slot contribute 0 and sets MOE_DEVICE_BAD_EXPERT_ID in the
  * device status word.  T = 1..4 runs the per-(token, slot) GEMV path;
  * larger T the (token, expert)-sorted grouped path, in chunks of up to 2048
- * tokens (NVFP4: halved until a chunk's tcgen05 plan fits): its products run
+ * tokens: its products run
  * on mma.sync tiles, or on tcgen05 (BF16 weight tiles dequantised once per
  * CTA, FP32 accumulators in tensor memory, packed codes brought in by TMA
  * tensor loads) when a chunk's groups average at least 40 (token, slot)

@@ -45,17 +45,6 @@ namespace {
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Tokens per launch sequence of the grouped path: kGroupedMaxT, halved for
-// NVFP4 weights until a chunk's tcgen05 plan fits the shared memory (their
-// E4M3 scale rows take twice the bytes of E8M0 ones).  Ends: the plan of one
-// token fits whenever the first test passes.
-int grouped_chunk(const moe_ctx *h) {
-    int c = moe::kGroupedMaxT;
-    if (h->nv && h->codes_base && moe::grouped_tc_supported(h->H, h->I, h->k, 1))
-        while (!moe::grouped_tc_supported(h->H, h->I, c * h->k, 1)) c /= 2;
-    return c;
-}
-
 struct WsLayout {
     size_t counters, logits, h, o, x16, x16_exp;
     size_t hand_seq, hand_ack, hand_ent;  // fused-layer routing handoff
@@ -389,9 +378,7 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
     }
     if (flags & MOE_FWD_FORCE_TCGEN05) {
         if (flags & MOE_FWD_FORCE_DECODE) return MOE_ERR_ARG;
-        const int chunk = grouped_chunk(h);
-        const int Tc = T < chunk ? T : chunk;
-        if (h->s8 || !h->codes_base || !moe::grouped_tc_supported(h->H, h->I, Tc * h->k, h->nv))
+        if (h->s8 || !h->codes_base || !moe::grouped_tc_supported(h->H, h->I, h->nv))
             return MOE_ERR_ARG;
         flags |= MOE_FWD_FORCE_GROUPED;
     }
@@ -456,9 +443,8 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
     if (!h->s8 && !moe::decode_shape_supported(h->H, h->I)) return MOE_ERR_ARG;
 
     if (grouped) {
-        const int chunk = grouped_chunk(h);
-        for (int t0 = 0; t0 < T; t0 += chunk) {
-            const int Tc = (T - t0 < chunk) ? T - t0 : chunk;
+        for (int t0 = 0; t0 < T; t0 += moe::kGroupedMaxT) {
+            const int Tc = (T - t0 < moe::kGroupedMaxT) ? T - t0 : moe::kGroupedMaxT;
             moe::GroupedParams gp = {};
             gp.table = h->d_table;
             gp.codes_base = h->codes_base;
@@ -492,7 +478,7 @@ int moe_forward_ex(moe_handle_t h, const uint16_t *x, int T, const int32_t *topk
             // tcgen05 when the groups are large enough to amortise a CTA's
             // dequantised tiles over its token passes
             const bool tc_ok = !h->s8 && h->codes_base &&
-                               moe::grouped_tc_supported(h->H, h->I, Tc * h->k, h->nv);
+                               moe::grouped_tc_supported(h->H, h->I, h->nv);
             gp.tcgen05 = (flags & MOE_FWD_FORCE_TCGEN05) ||
                          (!(flags & MOE_FWD_FORCE_MMA) && tc_ok &&
                           (long long)Tc * h->k >= (long long)moe::kTcAutoGroup * h->E);

@@ -491,7 +491,7 @@ cudaError_t launch_grouped(const GroupedParams &p, cudaStream_t s, bool pdl) {
     if (p.T < 1 || p.T > kGroupedMaxT || !grouped_supported(p.E, p.H, p.I, p.nv, p.s8))
         return cudaErrorInvalidValue;
     if (p.tcgen05 &&
-        (p.s8 || !p.codes_base || !grouped_tc_supported(p.H, p.I, p.T * p.k, p.nv)))
+        (p.s8 || !p.codes_base || !grouped_tc_supported(p.H, p.I, p.nv)))
         return cudaErrorInvalidValue;
     if (p.nv && !p.gscale) return cudaErrorInvalidValue;
     cudaError_t e;

@@ -178,9 +178,10 @@ __host__ __device__ constexpr uint32_t tc_raw_off(int nmat) {
 __host__ __device__ constexpr uint32_t tc_sc_off(int nmat) {
     return tc_raw_off(nmat) + (uint32_t)kTcRaw * nmat * kTcRawSlot;
 }
-// then the B row of every token of the group ([pairs] ints; a group holds at
-// most all the launch's T k pairs).  Scale rows: K/32 E8M0 bytes, or K/16
-// E4M3 bytes (nv).
+// Scale rows: K/32 E8M0 bytes, or K/16 E4M3 bytes (nv).  Then, when the plan
+// has room for it ([pairs] ints: a group holds at most all the launch's T k
+// pairs), the B row of every token of the group; else the kernel reads the
+// rows from the sorted pair list in global memory.
 __host__ __device__ inline uint32_t tc_src_off(int nmat, int K, int nv) {
     return tc_sc_off(nmat) + (uint32_t)nmat * kTcM * (uint32_t)(K / (nv ? 16 : 32));
 }
@@ -221,7 +222,9 @@ __device__ __forceinline__ bool tc_wait(uint64_t *bar, unsigned parity, volatile
 // NV: NVFP4 weights: A = code x its 16-element block's E4M3 scale (exact in
 // BF16: at most 6 significant bits), the expert's FP32 multiplier applied to
 // the accumulator in the epilogue (one FP32 rounding before the BF16 one).
-template <int NMAT, bool NV>
+// TAB: the token-row table in shared memory (else read from the sorted pair
+// list in global memory).
+template <int NMAT, bool NV, bool TAB>
 __global__ void __launch_bounds__(kTcThreads, 1)
 grouped_tc_kernel(const GroupedParams p, const __grid_constant__ CUtensorMap codes_map) {
     extern __shared__ __align__(1024) uint8_t sm[];
@@ -248,7 +251,7 @@ grouped_tc_kernel(const GroupedParams p, const __grid_constant__ CUtensorMap cod
     uint8_t *raw = sm + tc_raw_off(NMAT);
     uint8_t *scl = sm + tc_sc_off(NMAT);
     // per token of the group: its B row (x row of the pair's token, or h row
-    // of the pair)
+    // of the pair), in shared memory when the launch's plan holds the table
     int *s_src = reinterpret_cast<int *>(sm + tc_src_off(NMAT, K, NV ? 1 : 0));
 
     if (warp == 0) {  // TMEM: NMAT x 128 FP32 columns x 128 lanes
@@ -268,7 +271,7 @@ grouped_tc_kernel(const GroupedParams p, const __grid_constant__ CUtensorMap cod
         s_abort = 0;
         mbar_fence_init();
     }
-    for (int i = tid; i < n_e; i += kTcThreads) {
+    for (int i = tid; TAB && i < n_e; i += kTcThreads) {
         const int pr = p.perm[seg0 + i];
         s_src[i] = NMAT == 2 ? pr / p.k : pr;
     }
@@ -362,9 +365,16 @@ grouped_tc_kernel(const GroupedParams p, const __grid_constant__ CUtensorMap cod
             // per warp from global memory
             for (int i = tid; i < ((nt + 7) & ~7) * 8; i += kTcWork) {
                 const int n = ((i >> 6) << 3) | (i & 7), c = (i >> 3) & 7;
-                if (n < nt)
-                    cp_async16_tc(b + tc_off(n, c),
-                                  bbase + (size_t)s_src[tc + n] * K + kt * kTcK + c * 8);
+                if (n < nt) {
+                    int src;
+                    if (TAB) {
+                        src = s_src[tc + n];
+                    } else {
+                        const int pr = p.perm[seg0 + tc + n];
+                        src = NMAT == 2 ? pr / p.k : pr;
+                    }
+                    cp_async16_tc(b + tc_off(n, c), bbase + (size_t)src * K + kt * kTcK + c * 8);
+                }
             }
         };
         // copy groups: {scales}, {B(0)}, {B(1)}, then one per iteration
@@ -520,32 +530,43 @@ cudaError_t codes_map_copy(CodesMap &c, std::mutex &mu, const GroupedParams &p, 
     return e;
 }
 
-template <int NMAT, bool NV>
-cudaError_t launch_tc(const GroupedParams &p, const CUtensorMap &map, cudaStream_t s, bool pdl) {
-    const int K = NMAT == 2 ? p.H : p.I, M = NMAT == 2 ? p.I : p.H;
-    const size_t smem = tc_smem_bytes(NMAT, K, p.T * p.k, NV ? 1 : 0);
-    if (smem > kTcSmemBudget) return cudaErrorInvalidValue;
+template <int NMAT, bool NV, bool TAB>
+cudaError_t launch_tc_v(const GroupedParams &p, const CUtensorMap &map, size_t smem,
+                        cudaStream_t s, bool pdl) {
     // the budget, once per device (the attribute belongs to the current
     // device's context)
     static PerDeviceOnce once;
     const cudaError_t attr = per_device_once(once, [] {
-        return cudaFuncSetAttribute(grouped_tc_kernel<NMAT, NV>,
+        return cudaFuncSetAttribute(grouped_tc_kernel<NMAT, NV, TAB>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)kTcSmemBudget);
     });
     if (attr != cudaSuccess) return attr;
-    return launch_ex(grouped_tc_kernel<NMAT, NV>, dim3(M / kTcM, p.E), dim3(kTcThreads), smem, s,
-                     pdl, p, map);
+    const int M = NMAT == 2 ? p.I : p.H;
+    return launch_ex(grouped_tc_kernel<NMAT, NV, TAB>, dim3(M / kTcM, p.E), dim3(kTcThreads), smem,
+                     s, pdl, p, map);
+}
+
+template <int NMAT, bool NV>
+cudaError_t launch_tc(const GroupedParams &p, const CUtensorMap &map, cudaStream_t s, bool pdl) {
+    const int K = NMAT == 2 ? p.H : p.I;
+    // the token-row table in shared memory when it fits beside the tiles
+    const size_t with_table = tc_smem_bytes(NMAT, K, p.T * p.k, NV ? 1 : 0);
+    if (with_table <= kTcSmemBudget)
+        return launch_tc_v<NMAT, NV, true>(p, map, with_table, s, pdl);
+    const size_t smem = tc_smem_bytes(NMAT, K, 0, NV ? 1 : 0);
+    if (smem > kTcSmemBudget) return cudaErrorInvalidValue;
+    return launch_tc_v<NMAT, NV, false>(p, map, smem, s, pdl);
 }
 
 }  // namespace
 
 // The tensor-core products need the contiguous weight layout (one tensor map
-// per matrix kind), H and I multiples of 128 and the shared-memory plan of a
-// launch of `pairs` (token, slot) pairs within the budget.
-bool grouped_tc_supported(int H, int I, int pairs, int nv) {
-    return H % 128 == 0 && I % 128 == 0 && tc_smem_bytes(2, H, pairs, nv) <= kTcSmemBudget &&
-           tc_smem_bytes(1, I, pairs, nv) <= kTcSmemBudget;
+// per matrix kind), H and I multiples of 128 and the shared-memory plan of
+// both products within the budget.
+bool grouped_tc_supported(int H, int I, int nv) {
+    return H % 128 == 0 && I % 128 == 0 && tc_smem_bytes(2, H, 0, nv) <= kTcSmemBudget &&
+           tc_smem_bytes(1, I, 0, nv) <= kTcSmemBudget;
 }
 
 namespace {

@@ -188,7 +188,7 @@ cudaError_t launch_grouped(const GroupedParams &p, cudaStream_t s, bool pdl);
 // average at least kTcAutoGroup pairs (the mma.sync tiles convert the codes
 // again for every 8 tokens, the tcgen05 CTAs once per 128), or on request.
 constexpr int kTcAutoGroup = 40;
-bool grouped_tc_supported(int H, int I, int pairs, int nv = 0);
+bool grouped_tc_supported(int H, int I, int nv = 0);
 cudaError_t launch_grouped_tc_gateup(const GroupedParams &p, cudaStream_t s, bool pdl);
 cudaError_t launch_grouped_tc_down(const GroupedParams &p, cudaStream_t s, bool pdl);
 

@@ -196,13 +196,12 @@ def test_nvfp4_tcgen05_matches_oracle(shape, T, dist):
 
 
 def test_nvfp4_tcgen05_chunks_and_automatic_choice():
-    """1100 tokens of the 24B shape: the NVFP4 batch runs in chunks of 1024
-    tokens (a chunk's tcgen05 plan must fit the shared memory with E4M3 scale
-    rows), the first on tcgen05 (its groups average 64 pairs per expert) and
-    the ragged rest on mma.sync.  Sampled tokens from both chunks (h, o, y)
-    against the oracle."""
+    """2100 tokens of the 24B shape: the NVFP4 batch runs in launch sequences
+    of 2048 tokens, the first on tcgen05 (its groups average 128 pairs per
+    expert) and the ragged rest of 52 tokens on mma.sync.  Sampled tokens from
+    both (h, o, y) against the oracle, stage by stage."""
     shape = synth.L24B
-    T = 1100
+    T = 2100
     L, layer = _layer(shape, 51, max_tokens=T)
     x = synth.make_tokens(T, shape.H, seed=51, stream=T)
     ids, w = synth.make_routing(T, shape.E, shape.top_k, "uniform", synth.rng_for(51, 13, T))
@@ -212,7 +211,7 @@ def test_nvfp4_tcgen05_chunks_and_automatic_choice():
     assert layer.status() == 0
     h_g, o_g = layer.intermediates(T)
     h_g, o_g, y_g = host_bf16(h_g), host_bf16(o_g), host_bf16(y)
-    rows = np.r_[0:6, 1018:1030, 1094:1100]
+    rows = np.r_[0:6, 2040:2056, 2094:2100]
     _verify_stages(L, shape, x[rows], ids[rows], w[rows], h_g[rows], o_g[rows], y_g[rows])
     layer.close()
 
