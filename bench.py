@@ -70,6 +70,9 @@ def parse_args():
                          "(a small command for profiler captures)")
     ap.add_argument("--only-main", action="store_true",
                     help="time the main line only (for profiler runs)")
+    ap.add_argument("--only-sym8-prefill", action="store_true",
+                    help="time the S = 64 chunk of one sym8 layer only (grouped products; a "
+                         "small command for profiler captures)")
     return ap.parse_args()
 
 
@@ -395,18 +398,8 @@ def sym8_stack(torch, moe, st, args, max_steps=4):
     device from a seeded generator, the MXFP4 layer's router reused; one
     route + gate/up + down launch triple per layer, captured in a CUDA graph
     and timed like the NVFP4 line."""
-    gen = torch.Generator(device="cuda")
-    gen.manual_seed(args.seed + 11)
     n_w = 3 * SHAPE.I * SHAPE.H
-    weights = []
-    for L in st.layers:
-        q = torch.randint(-127, 128, (SHAPE.E, n_w), dtype=torch.int8, device="cuda",
-                          generator=gen)
-        ex = torch.randint(2, 6, (SHAPE.E, n_w // 32), dtype=torch.int16, device="cuda",
-                           generator=gen)
-        man = torch.randint(0, 1024, (SHAPE.E, n_w // 32), dtype=torch.int16, device="cuda",
-                            generator=gen)
-        weights.append((q, (ex << 10) | man, L.router_w, L.router_b))
+    weights = draw_sym8_weights(torch, st.layers, args.seed)
     s8 = moe.MoEStack(weights, SHAPE.E, SHAPE.H, SHAPE.I, SHAPE.top_k, T=1, persistent=False)
     s8.r.copy_(st.r)
     s8.capture()
@@ -458,6 +451,17 @@ def run_ours(args):
     def barrier():
         if world > 1:
             dist.barrier()
+
+    if args.only_sym8_prefill:
+        st = build_stack(torch, moe, seed=args.seed + rank, n_layers=1, persistent=False)
+        weights = draw_sym8_weights(torch, st.layers, args.seed)
+        peak, _ = load_peaks()
+        row = sym8_prefill_chunk(torch, moe, weights[0], args.seed, peak)
+        if rank == 0:
+            print(json.dumps({"sym8_prefill_s64": row}), flush=True)
+        del weights
+        st.close()
+        return 0
 
     if args.only_batched:
         T, dist = args.only_batched.split(":")
@@ -739,6 +743,26 @@ def config_stack8b(torch, moe, seed, steps=4):
 BATCHED_CASES = ((32, "uniform"), (32, "zipf"), (64, "uniform"), (64, "zipf"), (256, "uniform"),
                  (256, "zipf"), (1024, "uniform"), (2048, "uniform"), (2048, "zipf"))
 TC_AUTO_GROUP = 40  # the library's tcgen05 products from T k >= 40 E on
+
+
+def draw_sym8_weights(torch, layers, seed):
+    """Per layer of `layers` (their routers are reused): int8 weights uniform
+    over -127..127 and binary16 block scales (positive normal values,
+    exponent fields 2..5, uniform mantissas), drawn on the device from a
+    generator seeded with seed + 11."""
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(seed + 11)
+    n_w = 3 * SHAPE.I * SHAPE.H
+    weights = []
+    for L in layers:
+        q = torch.randint(-127, 128, (SHAPE.E, n_w), dtype=torch.int8, device="cuda",
+                          generator=gen)
+        ex = torch.randint(2, 6, (SHAPE.E, n_w // 32), dtype=torch.int16, device="cuda",
+                           generator=gen)
+        man = torch.randint(0, 1024, (SHAPE.E, n_w // 32), dtype=torch.int16, device="cuda",
+                            generator=gen)
+        weights.append((q, (ex << 10) | man, L.router_w, L.router_b))
+    return weights
 
 
 def sym8_prefill_chunk(torch, moe, lw, seed, peak, T=64, reps=10):
