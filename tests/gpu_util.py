@@ -125,3 +125,89 @@ def check_grouped_y(y_g, y_r, o_g, o_r, w64, valid, residual=None, what="grouped
     # the kernel's own h), so only the derived bound applies here.
     if cap:
         assert_close_rms(y_g, y_r, what=what, max_ulps=16, max_flip_frac=5e-4)
+
+
+# ---- stage-by-stage checks of the grouped products (reading R14) ----
+
+def expert_matrix(L, shape, e, m, fmt="mxfp4"):
+    """The oracle's dequantised matrix m (0 gate, 1 up, 2 down) of expert e,
+    FP64 [rows, K]: MXFP4 (code x 2^(e-127)), NVFP4 (code x E4M3 block scale
+    x the expert's multiplier) or sym8 (int8 x binary16 block scale)."""
+    n = shape.I * shape.H
+    rows, K = (shape.I, shape.H) if m < 2 else (shape.H, shape.I)
+    if fmt == "sym8":
+        q = np.ascontiguousarray(np.asarray(L.codes).reshape(shape.E, 3, n)[e, m])
+        s = np.ascontiguousarray(np.asarray(L.scales).reshape(shape.E, 3, n // 32)[e, m])
+        return oracle.dequant_sym8(q, s, n).reshape(rows, K)
+    c = np.ascontiguousarray(L.codes.reshape(shape.E, 3, n // 2)[e, m])
+    if fmt == "nvfp4":
+        s = np.ascontiguousarray(L.scales.reshape(shape.E, 3, n // 16)[e, m])
+        gs = float(L.gscales[e, 0 if m < 2 else 1])
+        return oracle.dequant_nvfp4(c, s, gs, n).reshape(rows, K)
+    s = np.ascontiguousarray(L.scales.reshape(shape.E, 3, n // 32)[e, m])
+    return oracle.dequant(c, s, n).reshape(rows, K)
+
+
+def _near_midpoint(v, mag, rel=2.0 ** -16):
+    """v lies within rel * mag of a BF16 rounding midpoint (mag: the sum of
+    the magnitudes an FP32 accumulation added, or |v| for one operation)."""
+    b = oracle.bf16_from_f64(v)
+    lo = oracle.bf16_to_f64(b)
+    nb = oracle.bf16_to_f64(b + 1 if (v >= lo) == (v >= 0) else b - 1)
+    return abs(v - (lo + nb) / 2) <= rel * mag
+
+
+def _bf16_and_neighbours(v, movable):
+    b = oracle.bf16_from_f64(v)
+    vals = [oracle.bf16_to_f64(b)]
+    if movable and b & 0x7FFF:
+        vals += [oracle.bf16_to_f64(b + 1), oracle.bf16_to_f64(b - 1)]
+    return vals
+
+
+def verify_h_flips(h_g, h_r, x, ids, valid, matrix, what="h", max_frac=1e-3):
+    """h of the grouped products against the oracle's h: every element beyond
+    1e-2 rms must be the oracle's rounding chain h = BF16(BF16(silu(g')) u')
+    with g', u' and silu(g') each allowed one BF16 ulp away only where that
+    exact value (FP64, from the oracle's dequantised rows: matrix(e, m))
+    lies within 2^-16 of its accumulated magnitude from a rounding midpoint;
+    such elements stay below max_frac.  (With h = s u, two ulps of s can be
+    four or more ulps of h, so an ulp count alone bounds nothing.)"""
+    hg64, hr64 = f64(h_g), f64(h_r)
+    rms = np.sqrt(np.mean(hr64 ** 2, axis=2, keepdims=True))
+    far = valid[:, :, None] & (np.abs(hg64 - hr64) > TOL * rms)
+    cache = {}
+    for t, j, i in np.argwhere(far):
+        e = int(ids[t, j])
+        if e not in cache:
+            cache = {e: (matrix(e, 0), matrix(e, 1))}
+        wg, wu = cache[e][0][i], cache[e][1][i]
+        xt = f64(x[t])
+        g, u = float(wg @ xt), float(wu @ xt)
+        g_ok = _near_midpoint(g, float(np.abs(wg * xt).sum()))
+        u_ok = _near_midpoint(u, float(np.abs(wu * xt).sum()))
+        want = float(hg64[t, j, i])
+        hit = False
+        for gg in _bf16_and_neighbours(g, g_ok):
+            sl = gg / (1.0 + np.exp(-gg))
+            for ss in _bf16_and_neighbours(sl, _near_midpoint(sl, abs(sl))):
+                for uu in _bf16_and_neighbours(u, u_ok):
+                    hit |= oracle.bf16_to_f64(oracle.bf16_from_f64(ss * uu)) == want
+        assert hit, f"{what}[{t},{j},{i}] = {want} is no one-ulp rounding move of g={g}, u={u}"
+    n = int(valid.sum()) * h_g.shape[2]
+    print(f"[parity] {what}: {n} elements, {int(np.count_nonzero(hg64[valid] != hr64[valid]))} "
+          f"differ, {int(far.sum())} beyond tol, each a one-ulp move of g, u or silu(g) at a "
+          f"rounding midpoint")
+    assert far.sum() <= max_frac * n, f"{what}: {far.sum()} elements beyond {TOL} rms"
+
+
+def o_given_h(h_g, ids, valid, matrix, H):
+    """The oracle's down product of the kernel's own h: o = BF16(W_down h) in
+    FP64 per valid (token, slot), [T, k, H] BF16 bits (0 elsewhere)."""
+    hg64 = f64(h_g)
+    o_ref = np.zeros(h_g.shape[:2] + (H,), dtype=np.uint16)
+    for e in np.unique(ids[valid]):
+        wd = matrix(int(e), 2)
+        sel = valid & (ids == e)
+        o_ref[sel] = oracle.bf16_from_f64_array(hg64[sel] @ wd.T)
+    return o_ref

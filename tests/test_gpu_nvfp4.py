@@ -11,7 +11,8 @@ import torch
 
 import oracle
 import packed_mxfp4_w4a16_b200 as moe
-from gpu_util import assert_close_rms, check_grouped_y, dev_bf16, dev_u8, f64, host_bf16
+from gpu_util import (assert_close_rms, check_grouped_y, dev_bf16, dev_u8, expert_matrix,
+                      host_bf16, o_given_h, verify_h_flips)
 from workloads import synth
 
 pytestmark = pytest.mark.gpu
@@ -84,33 +85,6 @@ def test_nvfp4_grouped_matches_oracle(shape, T, dist, flags):
     layer.close()
 
 
-def _nv_matrix(L, shape, e, m):
-    """The oracle's dequantised matrix m (0 gate, 1 up, 2 down) of expert e:
-    code x E4M3 block scale x the expert's multiplier, FP64 [rows, K]."""
-    n = shape.I * shape.H
-    c = np.ascontiguousarray(L.codes.reshape(shape.E, 3, n // 2)[e, m])
-    s = np.ascontiguousarray(L.scales.reshape(shape.E, 3, n // 16)[e, m])
-    rows, K = (shape.I, shape.H) if m < 2 else (shape.H, shape.I)
-    return oracle.dequant_nvfp4(c, s, float(L.gscales[e, 0 if m < 2 else 1]), n).reshape(rows, K)
-
-
-def _near_midpoint(v, mag, rel=2.0 ** -16):
-    """v lies within rel * mag of a BF16 rounding midpoint (mag: the sum of
-    the magnitudes the FP32 accumulation added, or |v| for one operation)."""
-    b = oracle.bf16_from_f64(v)
-    lo = oracle.bf16_to_f64(b)
-    nb = oracle.bf16_to_f64(b + 1 if (v >= lo) == (v >= 0) else b - 1)
-    return abs(v - (lo + nb) / 2) <= rel * mag
-
-
-def _neighbours(v, movable):
-    b = oracle.bf16_from_f64(v)
-    vals = [oracle.bf16_to_f64(b)]
-    if movable and b & 0x7FFF:
-        vals += [oracle.bf16_to_f64(b + 1), oracle.bf16_to_f64(b - 1)]
-    return vals
-
-
 def _check_tcgen05_stages(L, layer, x, ids, w, shape, residual=None, flags=moe.FWD_FORCE_TCGEN05):
     """Stage by stage against the oracle (reading R14).  h: within 1e-2 rms of
     the oracle's h, except elements that the oracle's own rounding chain
@@ -141,34 +115,9 @@ def _verify_stages(L, shape, x, ids, w, h_g, o_g, y_g, residual=None):
                                              shape.H, shape.I, residual=residual, want_o=True,
                                              want_h=True)
     valid = (ids >= 0) & (ids < shape.E)
-    hg64, hr64 = f64(h_g), f64(h_r)
-    rms = np.sqrt(np.mean(hr64 ** 2, axis=2, keepdims=True))
-    far = valid[:, :, None] & (np.abs(hg64 - hr64) > 1e-2 * rms)
-    cache = {}
-    for t, j, i in np.argwhere(far):
-        e = int(ids[t, j])
-        if e not in cache:
-            cache = {e: (_nv_matrix(L, shape, e, 0), _nv_matrix(L, shape, e, 1))}
-        wg, wu = cache[e][0][i], cache[e][1][i]
-        xt = f64(x[t])
-        g, u = float(wg @ xt), float(wu @ xt)
-        g_ok = _near_midpoint(g, float(np.abs(wg * xt).sum()))
-        u_ok = _near_midpoint(u, float(np.abs(wu * xt).sum()))
-        want = float(hg64[t, j, i])
-        hits = False
-        for gg in _neighbours(g, g_ok):
-            sl = gg / (1.0 + np.exp(-gg))
-            for ss in _neighbours(sl, _near_midpoint(sl, abs(sl))):
-                for uu in _neighbours(u, u_ok):
-                    hits |= oracle.bf16_to_f64(oracle.bf16_from_f64(ss * uu)) == want
-        assert hits, f"h[{t},{j},{i}] = {want} is no one-ulp rounding move of g={g}, u={u}"
-    assert far.sum() <= 1e-3 * valid.sum() * shape.I, f"h: {far.sum()} elements beyond 1e-2 rms"
-    # o against the oracle's down product of the kernel's own h
-    o_ref = np.zeros_like(o_g)
-    for e in np.unique(ids[valid]):
-        wd = _nv_matrix(L, shape, int(e), 2)
-        sel = valid & (ids == e)
-        o_ref[sel] = oracle.bf16_from_f64_array(hg64[sel] @ wd.T)
+    matrix = lambda e, m: expert_matrix(L, shape, e, m, fmt="nvfp4")  # noqa: E731
+    verify_h_flips(h_g, h_r, x, ids, valid, matrix, what="nvfp4 tcgen05 h")
+    o_ref = o_given_h(h_g, ids, valid, matrix, shape.H)
     assert_close_rms(o_g[valid], o_ref[valid], what="nvfp4 tcgen05 o (given h)", max_ulps=2)
     check_grouped_y(y_g, y_r, o_g, o_r, w64, valid, residual, what="nvfp4 tcgen05 y", cap=False)
     for t in range(T):
