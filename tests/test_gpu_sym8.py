@@ -233,7 +233,7 @@ def test_sym8_layer_is_route_then_forward():
 
 def test_sym8_argument_errors():
     """Shapes outside the kernels' set, a misaligned code pointer, and the
-    one-launch stack (MXFP4 only) are refused."""
+    one-launch stack (MXFP4 and NVFP4 layers only) are refused."""
     # top_k * I BF16 values of h (8 * 4096 * 2 bytes) beyond the staged 48 KB
     bad = synth.LayerShape(E=8, H=512, I=4096, top_k=8)
     h = moe.moe_create(bad.E, bad.H, bad.I, bad.top_k)
