@@ -36,6 +36,11 @@
 // MMAs, fresh accumulator) is then scaled by the group's E8M0 exponent in
 // FP32 and added to the running FP32 sum, which is exactly per-group scaling.
 // The K quarters (one per warp of a row tile) are added in a fixed order.
+// The same tiles serve NVFP4 weights (page "primitive-ai/LFM2.5-24B-A2B-
+// NVFP4A16": each 16-element block's partial product scaled by its E4M3
+// scale) and sym8 weights (page "LFM2.5-8B-A1B — Core AI (.aimodel)",
+// "Provenance": 8 int8 bytes per thread and row converted to FP16 exactly,
+// the group's partial product scaled by its binary16 scale).
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>

@@ -16,7 +16,10 @@
 // tile, the threads (four per row, a quarter of the tile's K each) dequantise
 // the 128 x 64 packed weights of each matrix into BF16 (code x 2^(e-127),
 // exact in BF16: the E8M0 scale is folded into A, so the tensor core
-// accumulates the whole K range in FP32 without a per-group step) and copy
+// accumulates the whole K range in FP32 without a per-group step; NVFP4
+// weights, page "primitive-ai/LFM2.5-24B-A2B-NVFP4A16": code x its 16-element
+// block's E4M3 scale, also exact, the expert's FP32 multiplier applied to the
+// accumulator in the epilogue) and copy
 // the BF16 activation rows of up to 128 tokens of the expert (B, in a ring of
 // its own, two tiles ahead), both into shared memory in the
 // K-major core-matrix layout (8 rows x 16 bytes per core matrix).  One thread

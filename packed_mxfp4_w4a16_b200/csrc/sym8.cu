@@ -1,4 +1,7 @@
-// sym8.cu — experts in the sym8 format on the per-(token, slot) GEMV path.
+// sym8.cu — experts in the sym8 format on the per-(token, slot) GEMV path
+// (up to 4 tokens; larger batches take the grouped mma.sync tiles of
+// grouped.cu, unless asked for this path or the scales are not 4-byte
+// aligned).
 //
 // Source: page "LFM2.5-8B-A1B — Core AI (.aimodel)", table "Provenance", row
 // "Weight format": symmetric-linear int8 weights with one scale per K-block of
