@@ -122,7 +122,8 @@ typedef enum moe_status {
                                       tcgen05 (TMEM accumulators, TMA tensor
                                       loads of the packed codes); needs the
                                       contiguous weights of moe_load_packed
-                                      and H, I multiples of 128, else ARG  */
+                                      or moe_load_packed_nvfp4 and H, I
+                                      multiples of 128, else ARG           */
 #define MOE_FWD_FORCE_MMA 0x40u    /* grouped path with its products on
                                       mma.sync tiles (never tcgen05)        */
 
